@@ -1,0 +1,139 @@
+"""fp64 CPU oracle for the per-sample kernel-mixture convolution.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module; the product library never does.
+
+The arithmetic lives in ``dynconv_oracle.c`` (plain C, fp64, direct loops,
+threads over samples only). This module compiles it with gcc and marshals
+numpy arrays in and out; it adds no arithmetic of its own.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against closed
+forms, a library convolution (n=1), brute force on tiny inputs and the
+identities that the pages' definition implies.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dynconv_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+SIGMOID = 0
+SOFTMAX = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no GPU, no CUDA) and return the .so path."""
+    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+             "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"],
+            check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def configure(lib):
+    """Declare the C signatures on a loaded oracle library and return it."""
+    dp = ctypes.POINTER(ctypes.c_double)
+    i = ctypes.c_int
+    lib.oracle_route.argtypes = [i, i, i, i, dp, i, dp, dp, i, ctypes.c_double, dp, i]
+    lib.oracle_route.restype = i
+    lib.oracle_forward.argtypes = [i] * 11 + [dp, dp, dp, dp, i, i, dp, i]
+    lib.oracle_forward.restype = i
+    lib.oracle_assemble.argtypes = [i, ctypes.c_long, dp, dp, dp]
+    lib.oracle_assemble.restype = None
+    lib.oracle_threads_used.argtypes = [i, i]
+    lib.oracle_threads_used.restype = i
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = configure(ctypes.CDLL(build()))
+    return _lib
+
+
+def _dp(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _f64(a):
+    if a is None:
+        return None
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def threads_used(nthreads: int, nb: int) -> int:
+    return _load().oracle_threads_used(int(nthreads), int(nb))
+
+
+def route(x, Wr, br, mode: int, tau: float = 1.0, nthreads: int = 0):
+    """alpha[B][n] = act(FC(GAP(x_b))) for NHWC x[B][H][W][C]; Wr[n][C], br[n] (or None)."""
+    x = _f64(x)
+    Wr = _f64(Wr)
+    br = _f64(br)
+    B, H, W, C = x.shape
+    n = Wr.shape[0]
+    assert Wr.shape == (n, C)
+    assert br is None or br.shape == (n,)
+    alpha = np.empty((B, n), dtype=np.float64)
+    rc = _load().oracle_route(B, C, H, W, _dp(x), n, _dp(Wr), _dp(br), int(mode), float(tau),
+                              _dp(alpha), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_route rejected its arguments (rc={rc})")
+    return alpha
+
+
+def forward(x, experts, alpha, bias=None, stride: int = 1, pad: int = 0, groups: int = 1,
+            samples: tuple[int, int] | None = None, nthreads: int = 0):
+    """y = conv2d(x_b, sum_i alpha_bi W_i) + sum_i alpha_bi bias_i, NHWC, fp64.
+
+    x[B][H][W][C_in], experts[n][C_out][KH][KW][C_in/groups], alpha[B][n],
+    bias[n][C_out] or None.  ``samples=(b0, nb)`` computes only samples
+    b0..b0+nb-1 and returns y[nb][H_out][W_out][C_out].
+    """
+    x = _f64(x)
+    experts = _f64(experts)
+    alpha = _f64(alpha)
+    bias = _f64(bias)
+    B, H, W, Cin = x.shape
+    n, Cout, KH, KW, Cg = experts.shape
+    assert Cg * groups == Cin, "experts' last dim must be C_in/groups"
+    assert alpha.shape == (B, n)
+    assert bias is None or bias.shape == (n, Cout)
+    b0, nb = (0, B) if samples is None else samples
+    Ho = (H + 2 * pad - KH) // stride + 1
+    Wo = (W + 2 * pad - KW) // stride + 1
+    y = np.empty((nb, Ho, Wo, Cout), dtype=np.float64)
+    rc = _load().oracle_forward(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n,
+                                _dp(x), _dp(experts), _dp(alpha), _dp(bias), b0, nb, _dp(y),
+                                int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_forward rejected its arguments (rc={rc})")
+    return y
+
+
+def assemble(experts, alpha_b):
+    """W_b = sum_i alpha_b[i] * experts[i] (any expert shape), fp64."""
+    experts = _f64(experts)
+    alpha_b = _f64(alpha_b)
+    n = experts.shape[0]
+    assert alpha_b.shape == (n,)
+    wsize = int(np.prod(experts.shape[1:]))
+    out = np.empty(experts.shape[1:], dtype=np.float64)
+    _load().oracle_assemble(n, wsize, _dp(experts), _dp(alpha_b), _dp(out))
+    return out

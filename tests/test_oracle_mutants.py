@@ -1,0 +1,65 @@
+"""The pins are sensitive: plant plausible mistakes in a COPY of the oracle's C
+source (on the CPU, in a temporary directory), rebuild it, and check that at
+least one pin fails for every mutant. The committed oracle is not touched."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+
+from . import test_oracle_pins as pins
+
+# (name, original text, mutated text) -- each replacement must hit exactly once
+MUTANTS = [
+    ("flipped_orientation", "const int ih = oh * f->stride + kh - f->pad;",
+     "const int ih = oh * f->stride + (f->KH - 1 - kh) - f->pad;"),
+    ("swapped_kh_kw", "(((size_t)co * f->KH + kh) * f->KW + kw) * Cg",
+     "(((size_t)co * f->KH + kw) * f->KW + kh) * Cg"),
+    ("dropped_bias", "double s = bb[co];", "double s = 0.0;"),
+    ("alpha_transposed", "const double *ab = f->alpha + (size_t)b * f->n;",
+     "const double *ab = f->alpha + (size_t)b;"),
+    ("wrong_group_offset", "+ (size_t)g * Cg;", "+ (size_t)0 * Cg;"),
+    ("gap_not_averaged", "g[c] = s / (double)(H * W);", "g[c] = s;"),
+    ("softmax_without_tau", "den += exp(z[j] / tau);", "den += exp(z[j]);"),
+    ("router_bias_dropped", "double s = br ? br[i] : 0.0;", "double s = 0.0;"),
+    ("sign_error_in_sigmoid", "1.0 / (1.0 + exp(-z[i]))", "1.0 / (1.0 + exp(z[i]))"),
+    ("stride_ignored_in_w", "const int iw = ow * f->stride + kw - f->pad;",
+     "const int iw = ow + kw - f->pad;"),
+]
+
+PIN_TESTS = [
+    lambda: [pins.test_n1_alpha1_is_static_conv_torch(s) for s in pins.SHAPES],
+    lambda: [pins.test_mixed_kernel_matches_torch_conv(s) for s in pins.SHAPES],
+    lambda: [pins.test_brute_force_second_formulation(s) for s in range(12)],
+    pins.test_impulse_pins_orientation,
+    pins.test_zero_input_gives_mixed_bias_and_route_of_br,
+    pins.test_constant_input_route_closed_form,
+    lambda: [pins.test_route_against_library_routines(m, t)
+             for m, t in [(0, 1.0), (1, 1.0), (1, 0.3), (1, 30.0)]],
+    pins.test_route_invariants,
+]
+
+
+@pytest.mark.parametrize("name,orig,mut", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, orig, mut):
+    src = open(oracle._SRC).read()
+    assert src.count(orig) == 1, f"mutation anchor for {name} not unique"
+    path_c = tmp_path / "mutant.c"
+    path_c.write_text(src.replace(orig, mut))
+    so = tmp_path / "mutant.so"
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-pthread", str(path_c),
+                    "-o", str(so), "-lm"], check=True)
+    saved = oracle._lib
+    oracle._lib = oracle.configure(ctypes.CDLL(str(so)))
+    failures = 0
+    try:
+        for t in PIN_TESTS:
+            try:
+                t()
+            except (AssertionError, ValueError):
+                failures += 1
+    finally:
+        oracle._lib = saved
+    assert failures > 0, f"no pin caught mutant {name}"
