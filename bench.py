@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the dynamic-convolution hot path on B200.
+
+One step = routing + forward of one dynamic-convolution layer over one batch
+(default: the ResNet-18-style 3x3 layer, B=64, 128->128 channels, 28x28, bf16,
+n=4 experts, softmax routing). Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--variant V]
+  python bench.py --impl reference ...     # the fp64 CPU oracle on the host cores
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of the
+same layer (weak scaling, no collective on the data path); the time is the max
+over ranks.
+
+Timing: inputs are rotated over enough x/alpha/y buffer sets that their total
+footprint exceeds the 126 MB L2, so each step starts cold in L2. The K timed
+steps run as CUDA-graph replays (8 steps per graph: 8 routing launches, then 8
+forward launches) with CUDA events between the graphs, bracketed by a barrier
+and a device synchronisation; the events also give the per-kernel average
+launch durations used for the roofline.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=None)
+    ap.add_argument("--variant", default="auto",
+                    choices=["auto", "fused", "outside", "premix", "direct", "depthwise"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def workload_name(cfg) -> str:
+    return cfg.name
+
+
+def config_dict(cfg, extra=None):
+    d = {"workload": cfg.name, "B": cfg.B, "C_in": cfg.C_in, "C_out": cfg.C_out,
+         "H": cfg.H, "W": cfg.W, "kernel": f"{cfg.KH}x{cfg.KW}", "stride": cfg.stride,
+         "pad": cfg.pad, "groups": cfg.groups, "n_experts": cfg.n,
+         "routing": "softmax" if cfg.mode == 1 else "sigmoid", "tau": cfg.tau}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# --------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- reference arm
+
+def run_reference(args, cfg):
+    """The fp64 CPU oracle, as it stands, on the host cores. Each step is a bounded
+    sample of the workload: routing of one image plus one output row of its forward."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    from dynamic_convolution_b200 import synth
+    inp = synth.make_inputs(cfg)
+    x = inp.x_f64
+    Wr = inp.Wr.astype(np.float64)
+    br = inp.br.astype(np.float64)
+    E = inp.experts_f64
+    bias = inp.bias.astype(np.float64)
+
+    def step(k):
+        b = k % cfg.B
+        a = oracle.route(x[b:b + 1], Wr, br, cfg.mode, cfg.tau, nthreads=1)
+        full_a = np.zeros((cfg.B, cfg.n))
+        full_a[b] = a[0]
+        oracle.forward_rows(x, E, full_a, bias, b, k % cfg.H_out, 1, stride=cfg.stride,
+                            pad=cfg.pad, groups=cfg.groups)
+
+    for k in range(args.warmup):
+        step(k)
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        step(k)
+    dt = time.perf_counter() - t0
+    images = args.steps / cfg.H_out          # one output row of H_out per step
+    value = images / dt
+    flops_per_img = cfg.conv_flops / cfg.B
+    line = {
+        "impl": "reference", "metric": "images/s per dynconv layer (route + forward)",
+        "value": value, "unit": "images/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(cfg, {"sample": "route 1 image + 1 output row of its forward per step"}),
+        "eff_tflops": value * flops_per_img / 1e12,
+        "cpu_baseline": {"value": value, "unit": "images/s", "cores": 1, "kind": "oracle",
+                         "sample": "per step: routing of one image and one output row of its "
+                                   "forward (fp64 C oracle, one thread)"},
+        "e2e": {"value": value, "unit": "images/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------- our arm
+
+def cpu_baseline(cfg, inp):
+    import oracle
+    cores = os.cpu_count() or 1
+    nb = min(cfg.B, max(16, cores))
+    x = inp.x_f64[:nb]
+    t0 = time.perf_counter()
+    a = oracle.route(x, inp.Wr, inp.br, cfg.mode, cfg.tau, nthreads=0)
+    oracle.forward(x, inp.experts_f64, a, inp.bias, stride=cfg.stride, pad=cfg.pad,
+                   groups=cfg.groups, nthreads=0)
+    dt = time.perf_counter() - t0
+    return {"value": nb / dt, "unit": "images/s", "cores": oracle.threads_used(0, nb),
+            "kind": "oracle",
+            "sample": f"route + forward of {nb} of the {cfg.B} images, fp64 C oracle, "
+                      f"threads over images"}
+
+
+def profile_traffic(kernel_tag: str, workload: str, src_hash: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}__{workload}.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("source_hash") != src_hash:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "dynamic_convolution_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import dynamic_convolution_b200 as dc
+    from dynamic_convolution_b200 import build, synth
+
+    world, rank, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.cuda.current_device()
+    build.build()
+    dc.load()
+
+    variant = {"auto": 0, "fused": 1, "outside": 2, "premix": 3, "direct": 4,
+               "depthwise": 5}[args.variant]
+    inp = synth.make_inputs(cfg, seed=rank)
+    desc = dc.desc_from_config(cfg, variant)
+    tdt = torch.bfloat16 if cfg.dtype == synth.BF16 else torch.float32
+
+    def dev_tensor(a):
+        if cfg.dtype == synth.BF16:
+            return torch.from_numpy(a).view(torch.bfloat16).cuda()
+        return torch.from_numpy(a).cuda()
+
+    x0 = dev_tensor(inp.x_store)
+    experts = dev_tensor(inp.experts_store)
+    Wr = torch.from_numpy(inp.Wr).cuda()
+    br = torch.from_numpy(inp.br).cuda()
+    bias = torch.from_numpy(inp.bias).cuda()
+    set_bytes = x0.numel() * x0.element_size() * 2
+    nsets = max(2, math.ceil(2 * L2_BYTES / set_bytes))
+    nsets = min(nsets, 64)
+    xs = [x0] + [x0.clone() for _ in range(nsets - 1)]
+    ys = [torch.empty((cfg.B, cfg.H_out, cfg.W_out, cfg.C_out), dtype=tdt, device="cuda")
+          for _ in range(nsets)]
+    alphas = [torch.empty((cfg.B, cfg.n), dtype=torch.float32, device="cuda") for _ in range(nsets)]
+    ws_bytes = dc.dynconv_workspace_size(desc)
+    workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    chosen = dc.dynconv_select_variant(desc, ws_bytes)
+
+    stream = torch.cuda.Stream()
+
+    def route(s, st):
+        dc.check(dc.dynconv_route(desc, xs[s], Wr, br, cfg.mode, cfg.tau, alphas[s], st), "route")
+
+    def forward(s, st):
+        dc.check(dc.dynconv_forward(desc, xs[s], experts, alphas[s], bias, ys[s], workspace,
+                                    ws_bytes, st), "forward")
+
+    # warm-up outside capture (also sets kernel attributes once)
+    with torch.cuda.stream(stream):
+        for k in range(max(args.warmup, 3)):
+            route(k % nsets, stream)
+            forward(k % nsets, stream)
+    stream.synchronize()
+    st = dc.dynconv_device_status(stream)
+    dc.check(st, "device status after warm-up")
+
+    # graphs: all routes of a group of sets, then all forwards of the same group
+    G = min(8, nsets)
+    groups = [list(range(g, min(g + G, nsets))) for g in range(0, nsets, G)]
+    graphs = []
+    n0 = dc.dynconv_launch_count()
+    for grp in groups:
+        gr, gf = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for s in grp:
+                route(s, stream)
+        with torch.cuda.graph(gf, stream=stream):
+            for s in grp:
+                forward(s, stream)
+        graphs.append((gr, gf, len(grp)))
+    launches_per_step = (dc.dynconv_launch_count() - n0) / nsets
+    tails = {}
+    for s in range(nsets):  # single-step graphs for an exact step count
+        gr, gf = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            route(s, stream)
+        with torch.cuda.graph(gf, stream=stream):
+            forward(s, stream)
+        tails[s] = (gr, gf)
+    for gr, gf, _ in graphs:  # warm the graphs
+        gr.replay()
+        gf.replay()
+    torch.cuda.synchronize()
+
+    # schedule of exactly K steps
+    plan = []
+    k = 0
+    gi = 0
+    while k < args.steps:
+        gr, gf, m = graphs[gi % len(graphs)]
+        if k + m <= args.steps:
+            plan.append((gr, gf, m))
+            k += m
+        else:
+            for s in range(args.steps - k):
+                trg, tfg = tails[s]
+                plan.append((trg, tfg, 1))
+            k = args.steps
+        gi += 1
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(plan) + 1)]
+
+    sampler = ClockSampler(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.2)
+    with torch.cuda.stream(stream):
+        ev[0].record(stream)
+        for i, (gr, gf, m) in enumerate(plan):
+            gr.replay()
+            ev[2 * i + 1].record(stream)
+            gf.replay()
+            ev[2 * i + 2].record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = ev[0].elapsed_time(ev[-1])
+    route_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(len(plan)))
+    fwd_ms = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(len(plan)))
+    st = dc.dynconv_device_status(stream)
+    dc.check(st, "device status after timing")
+
+    t = torch.tensor([total_ms, fwd_ms, route_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_ms, route_ms = t.tolist()
+
+    # ---- end to end through the public API, host buffers, copies inside the timed region
+    xh = torch.from_numpy(inp.x_store).pin_memory()
+    if cfg.dtype == synth.BF16:
+        xh = xh.view(torch.bfloat16)
+    yh = torch.empty(ys[0].shape, dtype=tdt).pin_memory()
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for k in range(e2e_steps):
+            s = k % nsets
+            xs[s].copy_(xh, non_blocking=True)
+            route(s, stream)
+            forward(s, stream)
+            yh.copy_(ys[s], non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_ms = e2e_ms.item()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    del graphs, tails
+    peaks, peak_kind = measured_peaks()
+    K = args.steps
+    images = world * cfg.B * K
+    value = images / (total_ms / 1e3)
+    fwd_launch_ms = fwd_ms / K
+    route_launch_ms = route_ms / K
+    conv_flops = cfg.conv_flops
+    eb = cfg.elem_bytes
+    algo_bytes = (cfg.B * cfg.H * cfg.W * cfg.C_in + cfg.B * cfg.H_out * cfg.W_out * cfg.C_out
+                  + cfg.n * cfg.weight_elems) * eb
+    src_hash = kernel_source_hash()
+    variant_name = dc.VARIANT_NAMES.get(chosen, str(chosen))
+    if cfg.dtype == synth.BF16 and cfg.groups == 1:
+        achieved = conv_flops / (fwd_launch_ms / 1e3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_kind": f"bf16 dense burst, {peak_kind}",
+                "kernel": f"tc_conv_kernel<{variant_name}>",
+                "algorithmic": f"{conv_flops} conv FLOP per launch (2*B*HW*Cout*Cin*KH*KW)"}
+    else:
+        achieved = algo_bytes / (fwd_launch_ms / 1e3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_kind": f"HBM copy, {peak_kind}",
+                "kernel": f"{variant_name}_kernel",
+                "algorithmic": f"{algo_bytes} bytes per launch (x + y + experts)"}
+    roof["traffic"] = profile_traffic(variant_name, cfg.name, src_hash)
+    roof["launch_ms"] = fwd_launch_ms
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, inp)
+
+    line = {
+        "metric": "images/s per dynconv layer (route + forward)",
+        "value": value, "unit": "images/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32",
+        "data": "synthetic (seeded; recipe in DESIGN.md)",
+        "config": config_dict(cfg, {"variant": variant_name,
+                                    "l2": f"inputs rotated over {nsets} x/y sets "
+                                          f"({nsets * set_bytes / 2**20:.0f} MiB > 126 MiB L2)",
+                                    "parallelism": f"dp{world} (independent batches)"}),
+        "eff_tflops": world * conv_flops * K / (total_ms / 1e3) / 1e12,
+        "forward_ms": fwd_launch_ms, "route_ms": route_launch_ms,
+        "forward_images_per_s": cfg.B / (fwd_launch_ms / 1e3),
+        "forward_eff_tflops": conv_flops / (fwd_launch_ms / 1e3) / 1e12,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * cfg.B * e2e_steps / (e2e_ms / 1e3), "unit": "images/s",
+                "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
+                "d2h_bytes_per_step": int(yh.numel() * yh.element_size()),
+                "steps": e2e_steps},
+        "gpu_launches": int(round(launches_per_step * K)),
+        "clocks": clocks,
+        "source_hash": src_hash,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    from dynamic_convolution_b200 import synth
+    name = args.config or synth.HEADLINE
+    cfg = synth.CONFIGS[name]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

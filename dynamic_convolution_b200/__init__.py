@@ -1,0 +1,148 @@
+"""Python binding of the sm_100a dynamic-convolution C ABI (``include/dynconv.h``).
+
+Argument marshalling only: every function forwards to the symbol of the same
+name in ``libdynconv.so``; all arithmetic runs in the library's CUDA kernels.
+Tensors may be passed as torch CUDA tensors (their data pointers are taken) or
+as raw integer device addresses. There is no CPU fallback: if the library is
+missing or no sm_100 device is present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdynconv.so")
+
+# dynconv_dtype / dynconv_mode / dynconv_variant
+F32, BF16 = 0, 1
+SIGMOID, SOFTMAX = 0, 1
+VARIANT_AUTO, VARIANT_FUSED, VARIANT_OUTSIDE, VARIANT_PREMIX, VARIANT_DIRECT, VARIANT_DEPTHWISE = range(6)
+VARIANT_NAMES = {0: "auto", 1: "fused", 2: "outside", 3: "premix", 4: "direct", 5: "depthwise"}
+
+# status codes
+OK = 0
+ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = -1, -2, -3, -4, -5, -6
+
+SYMBOLS = ("dynconv_route", "dynconv_forward", "dynconv_workspace_size", "dynconv_select_variant",
+           "dynconv_status_string", "dynconv_last_error", "dynconv_device_status",
+           "dynconv_launch_count", "dynconv_test_hook")
+
+
+class dynconv_desc(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int) for f in
+                ("B", "C_in", "H", "W", "C_out", "KH", "KW", "stride", "pad", "groups", "n",
+                 "dtype", "variant")]
+
+
+class DynconvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {dynconv_status_string(status)} ({status}) {dynconv_last_error()}")
+
+
+_lib = None
+
+
+def load():
+    """Load libdynconv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m dynamic_convolution_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P = ctypes.c_void_p
+        D = ctypes.POINTER(dynconv_desc)
+        lib.dynconv_route.argtypes = [D, P, P, P, ctypes.c_int, ctypes.c_float, P, P]
+        lib.dynconv_route.restype = ctypes.c_int
+        lib.dynconv_forward.argtypes = [D, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.dynconv_forward.restype = ctypes.c_int
+        lib.dynconv_workspace_size.argtypes = [D]
+        lib.dynconv_workspace_size.restype = ctypes.c_size_t
+        lib.dynconv_select_variant.argtypes = [D, ctypes.c_size_t]
+        lib.dynconv_select_variant.restype = ctypes.c_int
+        lib.dynconv_status_string.argtypes = [ctypes.c_int]
+        lib.dynconv_status_string.restype = ctypes.c_char_p
+        lib.dynconv_last_error.argtypes = []
+        lib.dynconv_last_error.restype = ctypes.c_char_p
+        lib.dynconv_device_status.argtypes = [P]
+        lib.dynconv_device_status.restype = ctypes.c_int
+        lib.dynconv_launch_count.argtypes = []
+        lib.dynconv_launch_count.restype = ctypes.c_ulonglong
+        lib.dynconv_test_hook.argtypes = [ctypes.c_int, ctypes.c_longlong]
+        lib.dynconv_test_hook.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def make_desc(B, C_in, H, W, C_out, KH, KW, stride=1, pad=0, groups=1, n=1, dtype=BF16,
+              variant=VARIANT_AUTO) -> dynconv_desc:
+    return dynconv_desc(B, C_in, H, W, C_out, KH, KW, stride, pad, groups, n, dtype, variant)
+
+
+def desc_from_config(cfg, variant=VARIANT_AUTO, B=None) -> dynconv_desc:
+    """Descriptor for a ``synth.LayerConfig``."""
+    return make_desc(cfg.B if B is None else B, cfg.C_in, cfg.H, cfg.W, cfg.C_out, cfg.KH, cfg.KW,
+                     cfg.stride, cfg.pad, cfg.groups, cfg.n, cfg.dtype, variant)
+
+
+def dynconv_route(desc, x, Wr, br, mode, tau, alpha, stream=None) -> int:
+    return load().dynconv_route(ctypes.byref(desc), _ptr(x), _ptr(Wr), _ptr(br), int(mode),
+                                float(tau), _ptr(alpha), _stream(stream))
+
+
+def dynconv_forward(desc, x, experts, alpha, bias, y, workspace=None, workspace_bytes=0,
+                    stream=None) -> int:
+    return load().dynconv_forward(ctypes.byref(desc), _ptr(x), _ptr(experts), _ptr(alpha),
+                                  _ptr(bias), _ptr(y), _ptr(workspace), int(workspace_bytes),
+                                  _stream(stream))
+
+
+def dynconv_workspace_size(desc) -> int:
+    return int(load().dynconv_workspace_size(ctypes.byref(desc)))
+
+
+def dynconv_select_variant(desc, workspace_bytes=0) -> int:
+    return int(load().dynconv_select_variant(ctypes.byref(desc), int(workspace_bytes)))
+
+
+def dynconv_status_string(status: int) -> str:
+    return load().dynconv_status_string(int(status)).decode()
+
+
+def dynconv_last_error() -> str:
+    return load().dynconv_last_error().decode()
+
+
+def dynconv_device_status(stream=None) -> int:
+    return int(load().dynconv_device_status(_stream(stream)))
+
+
+def dynconv_launch_count() -> int:
+    return int(load().dynconv_launch_count())
+
+
+def dynconv_test_hook(key: int, value: int) -> int:
+    return int(load().dynconv_test_hook(int(key), int(value)))
+
+
+def check(status: int, where: str = "dynconv") -> None:
+    if status != OK:
+        raise DynconvError(status, where)

@@ -1,0 +1,570 @@
+// Host side of the C ABI declared in include/dynconv.h: argument validation,
+// variant selection, tensor-map encoding and kernel launches. Device code lives
+// in the *.cuh files included below (one translation unit, sm_100a only).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "dynconv.h"
+
+#include "common.cuh"
+#include "conv_tc.cuh"
+#include "depthwise.cuh"
+#include "direct.cuh"
+#include "premix.cuh"
+#include "route.cuh"
+
+namespace {
+
+// One error word per device (module globals are instantiated per device).
+__device__ int g_device_err;
+
+constexpr long long kDefaultWaitNs = 500LL * 1000 * 1000;  // 0.5 s
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int* err = nullptr;  // device address of g_device_err on this device
+  int sms = 0;
+  int max_smem_optin = 0;
+  int cc_major = 0, cc_minor = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+std::atomic<unsigned long long> g_launches{0};
+std::atomic<long long> g_wait_ns{kDefaultWaitNs};
+std::atomic<int> g_inject_skip{0};
+thread_local char g_last_err[256] = "";
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int cuda_fail(cudaError_t e, const char* what) {
+  std::snprintf(g_last_err, sizeof(g_last_err), "%s: %s", what, cudaGetErrorString(e));
+  return DYNCONV_ERR_CUDA;
+}
+
+// Current device's state; initialises it on first use (error-word address, limits).
+int device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice, "device index");
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    if (prop.major != 10) {
+      std::snprintf(g_last_err, sizeof(g_last_err),
+                    "device %d is sm_%d%d; this library is built for sm_100a only", dev,
+                    prop.major, prop.minor);
+      return DYNCONV_ERR_CUDA;
+    }
+    st.sms = prop.multiProcessorCount;
+    st.max_smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
+    st.cc_major = prop.major;
+    st.cc_minor = prop.minor;
+    void* addr = nullptr;
+    e = cudaGetSymbolAddress(&addr, g_device_err);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+    st.err = static_cast<int*>(addr);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+      if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+        return cuda_fail(e == cudaSuccess ? cudaErrorSymbolNotFound : e,
+                         "cuTensorMapEncodeTiled entry point");
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    st.ready = true;
+  }
+  *out = &st;
+  return DYNCONV_OK;
+}
+
+// cudaFuncSetAttribute once per (device, kernel, size): keeps launches cheap
+// and keeps the call out of stream captures after the first launch.
+std::mutex g_smem_mu;
+std::map<std::pair<int, const void*>, size_t> g_smem_set;
+
+template <typename K>
+cudaError_t ensure_smem(K kern, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const auto key = std::make_pair(dev, reinterpret_cast<const void*>(kern));
+  std::lock_guard<std::mutex> lk(g_smem_mu);
+  auto it = g_smem_set.find(key);
+  if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes));
+  if (e == cudaSuccess) g_smem_set[key] = bytes;
+  return e;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int out_size(int in, int k, int stride, int pad) { return (in + 2 * pad - k) / stride + 1; }
+
+int validate_desc(const dynconv_desc* d) {
+  if (!d) return DYNCONV_ERR_INVALID_ARG;
+  if (d->B < 0 || d->C_in <= 0 || d->H <= 0 || d->W <= 0 || d->C_out <= 0 || d->KH <= 0 ||
+      d->KW <= 0 || d->stride <= 0 || d->pad < 0 || d->groups <= 0 || d->n <= 0)
+    return DYNCONV_ERR_INVALID_ARG;
+  if (d->dtype != DYNCONV_F32 && d->dtype != DYNCONV_BF16) return DYNCONV_ERR_INVALID_ARG;
+  if (d->variant < DYNCONV_VARIANT_AUTO || d->variant > DYNCONV_VARIANT_DEPTHWISE)
+    return DYNCONV_ERR_INVALID_ARG;
+  if (d->C_in % d->groups != 0 || d->C_out % d->groups != 0) return DYNCONV_ERR_INVALID_ARG;
+  if (out_size(d->H, d->KH, d->stride, d->pad) <= 0 || out_size(d->W, d->KW, d->stride, d->pad) <= 0)
+    return DYNCONV_ERR_INVALID_ARG;
+  // 32-bit index arithmetic inside the kernels
+  const long long xe = 1LL * d->B * d->H * d->W * d->C_in;
+  const long long ye = 1LL * d->B * out_size(d->H, d->KH, d->stride, d->pad) *
+                       out_size(d->W, d->KW, d->stride, d->pad) * d->C_out;
+  if (xe >= (1LL << 40) || ye >= (1LL << 40)) return DYNCONV_ERR_UNSUPPORTED;
+  return DYNCONV_OK;
+}
+
+size_t elem_bytes(const dynconv_desc* d) { return d->dtype == DYNCONV_F32 ? 4 : 2; }
+
+// ------------------------------------------------------------------ planning
+
+struct TcPlan {
+  dc::TcParams p;
+  int grid = 0;
+  size_t smem = 0;
+  double cost = 0;  // estimated SM cycles of the longest SM
+};
+
+bool tc_shape_ok(const dynconv_desc* d) {
+  return d->dtype == DYNCONV_BF16 && d->groups == 1 && d->stride == 1 && d->C_in % 8 == 0 &&
+         d->C_out % 8 == 0 && d->W <= 256 && d->n <= 1024 &&
+         out_size(d->H, d->KH, 1, d->pad) == d->H && out_size(d->W, d->KW, 1, d->pad) == d->W;
+}
+
+// Build the tensor-core plan for one variant, or return false.
+bool tc_plan(const dynconv_desc* d, int variant, int sms, int max_smem, TcPlan* out) {
+  if (!tc_shape_ok(d)) return false;
+  const int taps = d->KH * d->KW;
+  const int kc = (d->C_in + 63) / 64;
+  const int m_tiles = (d->C_out + 127) / 128;
+  const int steps_conv = taps * kc;
+  const int k_steps = variant == DYNCONV_VARIANT_OUTSIDE ? steps_conv * d->n : steps_conv;
+  bool found = false;
+  TcPlan best;
+  for (int R = 1; R <= d->H; ++R) {
+    const int n_valid = R * d->W;
+    const int n_pad = (n_valid + 15) / 16 * 16;
+    if (n_pad > 512) break;
+    if (R > 256) break;
+    int n0 = n_pad, n1 = 0;
+    if (n_pad > 256) { n0 = 256; n1 = n_pad - 256; }
+    const int b_tile = (n_pad * 128 + 1023) / 1024 * 1024;
+    const size_t per_stage = dc::kTcATileBytes + b_tile;
+    const size_t fixed = 1024 /*align slack*/ + 8 * 64 /*barriers*/ + 16 + 4 * d->n + 64;
+    int stages = static_cast<int>((static_cast<size_t>(max_smem) - fixed) / per_stage);
+    stages = std::min(stages, 8);
+    if (stages < 2) continue;
+    const int tiles_h = (d->H + R - 1) / R;
+    const long long units = 1LL * d->B * tiles_h * m_tiles;
+    const long long waves = (units + sms - 1) / sms;
+    // per-step cycle estimates: MMA 2*n_pad; operand A production; B tile from L2
+    const double mma = 2.0 * n_pad;
+    double a_cost;
+    if (variant == DYNCONV_VARIANT_FUSED) a_cost = 256.0 * d->n;     // n x 16 KB of experts
+    else if (variant == DYNCONV_VARIANT_OUTSIDE) a_cost = 256.0;      // one expert tile
+    else a_cost = 256.0;                                              // W_b tile by TMA
+    const double step = std::max(mma, a_cost);
+    const double epilogue = 40.0 * n_pad;
+    const double t_unit = k_steps * step + epilogue + 2000.0;
+    const double cost = waves * t_unit;
+    if (!found || cost < best.cost) {
+      found = true;
+      best.cost = cost;
+      best.grid = static_cast<int>(units);
+      best.smem = fixed + stages * per_stage;
+      dc::TcParams& p = best.p;
+      std::memset(&p, 0, sizeof(p));
+      p.B = d->B; p.H = d->H; p.W = d->W; p.Cin = d->C_in; p.Cout = d->C_out;
+      p.KH = d->KH; p.KW = d->KW; p.pad = d->pad; p.n = d->n;
+      p.R = R; p.tiles_h = tiles_h; p.m_tiles = m_tiles; p.n_valid = n_valid;
+      p.n_mma0 = n0; p.n_mma1 = n1; p.kc = kc; p.k_steps = k_steps; p.stages = stages;
+      p.b_tile_bytes = b_tile;
+      uint32_t cols = 32;
+      while (cols < static_cast<uint32_t>(n_pad)) cols <<= 1;
+      p.tmem_cols = cols;
+    }
+  }
+  if (!found || best.grid <= 0 || best.grid > (1 << 30)) return false;
+  *out = best;
+  return true;
+}
+
+bool depthwise_ok(const dynconv_desc* d) {
+  return d->dtype == DYNCONV_BF16 && d->groups == d->C_in && d->C_in == d->C_out &&
+         d->stride == 1 && d->KH == d->KW && (d->KH == 3 || d->KH == 5 || d->KH == 7) &&
+         d->C_in % 8 == 0 && d->n <= 4096;
+}
+
+size_t premix_workspace(const dynconv_desc* d) {
+  if (!tc_shape_ok(d)) return 0;
+  if (!dc::premix_shape_ok(d->B, d->n, d->C_out, d->KH * d->KW, d->C_in)) return 0;
+  return static_cast<size_t>(d->B) * d->C_out * d->KH * d->KW * d->C_in * 2;
+}
+
+// Cost-model choice among the kernels that can run this descriptor.
+int select_variant(const dynconv_desc* d, size_t ws_bytes, int sms, int max_smem) {
+  if (d->dtype == DYNCONV_F32) return DYNCONV_VARIANT_DIRECT;
+  if (d->groups != 1) return depthwise_ok(d) ? DYNCONV_VARIANT_DEPTHWISE : DYNCONV_VARIANT_DIRECT;
+  if (!tc_shape_ok(d)) return DYNCONV_VARIANT_DIRECT;
+  int best = DYNCONV_VARIANT_DIRECT;
+  double best_cost = 0;
+  for (int v : {DYNCONV_VARIANT_FUSED, DYNCONV_VARIANT_OUTSIDE, DYNCONV_VARIANT_PREMIX}) {
+    TcPlan pl;
+    if (!tc_plan(d, v, sms, max_smem, &pl)) continue;
+    double cost = pl.cost;
+    if (v == DYNCONV_VARIANT_PREMIX) {
+      const size_t need = premix_workspace(d);
+      if (need == 0 || ws_bytes < need) continue;
+      // mixing GEMM: expert read + workspace write, bandwidth-bound (~23 B/clk/SM of HBM)
+      const double bytes = 2.0 * d->n * d->C_out * d->KH * d->KW * d->C_in + static_cast<double>(need);
+      cost += bytes / (23.0 * sms) + 3000.0;
+    }
+    if (best == DYNCONV_VARIANT_DIRECT || cost < best_cost) {
+      best = v;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
+// ------------------------------------------------------------------ launches
+
+int check_launch(const char* what) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return DYNCONV_OK;
+}
+
+int encode_x_map(CUtensorMap* map, const void* x, const dynconv_desc* d, int R) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d->C_in), static_cast<cuuint64_t>(d->W),
+                              static_cast<cuuint64_t>(d->H), static_cast<cuuint64_t>(d->B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d->C_in) * 2,
+                                 static_cast<cuuint64_t>(d->W) * d->C_in * 2,
+                                 static_cast<cuuint64_t>(d->H) * d->W * d->C_in * 2};
+  const cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(d->W), static_cast<cuuint32_t>(R), 1u};
+  const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(x) failed: %d",
+                  static_cast<int>(r));
+    return DYNCONV_ERR_CUDA;
+  }
+  return DYNCONV_OK;
+}
+
+// Mixed kernels in the workspace, viewed as [B*C_out rows][taps][C_in], box {64, 1, 128}.
+int encode_w_map(CUtensorMap* map, const void* w, const dynconv_desc* d) {
+  const int taps = d->KH * d->KW;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d->C_in), static_cast<cuuint64_t>(taps),
+                              static_cast<cuuint64_t>(d->B) * d->C_out};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d->C_in) * 2,
+                                 static_cast<cuuint64_t>(taps) * d->C_in * 2};
+  const cuuint32_t box[3] = {64u, 1u, 128u};
+  const cuuint32_t es[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(w), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(w) failed: %d",
+                  static_cast<int>(r));
+    return DYNCONV_ERR_CUDA;
+  }
+  return DYNCONV_OK;
+}
+
+template <int V>
+int launch_tc(const TcPlan& plan, const CUtensorMap& xmap, const CUtensorMap& wmap,
+              cudaStream_t stream) {
+  cudaError_t e = ensure_smem(dc::tc_conv_kernel<V>, plan.smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc_conv)");
+  dc::tc_conv_kernel<V><<<plan.grid, dc::kTcThreads, plan.smem, stream>>>(xmap, wmap, plan.p);
+  return check_launch("tc_conv_kernel");
+}
+
+int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void* x,
+           const void* experts, const float* alpha, const float* bias, void* y, void* ws,
+           size_t ws_bytes, cudaStream_t stream) {
+  TcPlan plan;
+  if (!tc_plan(d, variant, st->sms, st->max_smem_optin, &plan)) return DYNCONV_ERR_UNSUPPORTED;
+  plan.p.experts = static_cast<const __nv_bfloat16*>(experts);
+  plan.p.alpha = alpha;
+  plan.p.bias = bias;
+  plan.p.y = static_cast<__nv_bfloat16*>(y);
+  plan.p.err = st->err;
+  plan.p.wait_ns = g_wait_ns.load();
+  plan.p.inject_skip = g_inject_skip.exchange(0);
+  CUtensorMap xmap, wmap;
+  std::memset(&wmap, 0, sizeof(wmap));
+  int rc = encode_x_map(&xmap, x, d, plan.p.R);
+  if (rc) return rc;
+  if (variant == DYNCONV_VARIANT_FUSED) return launch_tc<dc::kFused>(plan, xmap, wmap, stream);
+  if (variant == DYNCONV_VARIANT_OUTSIDE) return launch_tc<dc::kOutside>(plan, xmap, wmap, stream);
+  // PREMIX: mix every sample's kernel into the workspace, then convolve from it
+  const size_t need = premix_workspace(d);
+  if (need == 0) return DYNCONV_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < need) return DYNCONV_ERR_WORKSPACE;
+  if (!aligned16(ws)) return DYNCONV_ERR_MISALIGNED;
+  plan.p.inject_skip = 0;
+  rc = dc::launch_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
+                         static_cast<__nv_bfloat16*>(ws), d->B, d->n,
+                         static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in, st->err,
+                         g_wait_ns.load(), st->sms, stream, g_encode,
+                         [](auto k, size_t b) { return ensure_smem(k, b); });
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (rc == -1) return cuda_fail(cudaGetLastError(), "premix launch");
+  if (rc == -2) {
+    std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(premix) failed");
+    return DYNCONV_ERR_CUDA;
+  }
+  if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
+  rc = encode_w_map(&wmap, ws, d);
+  if (rc) return rc;
+  return launch_tc<dc::kPremix>(plan, xmap, wmap, stream);
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+const char* dynconv_status_string(int status) {
+  switch (status) {
+    case DYNCONV_OK: return "ok";
+    case DYNCONV_ERR_INVALID_ARG: return "invalid argument";
+    case DYNCONV_ERR_UNSUPPORTED: return "unsupported shape or variant";
+    case DYNCONV_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case DYNCONV_ERR_CUDA: return "CUDA error";
+    case DYNCONV_ERR_TIMEOUT: return "a kernel's bounded wait expired";
+    case DYNCONV_ERR_WORKSPACE: return "workspace too small for the requested variant";
+    default: return "unknown status";
+  }
+}
+
+const char* dynconv_last_error(void) { return g_last_err; }
+
+unsigned long long dynconv_launch_count(void) { return g_launches.load(); }
+
+int dynconv_test_hook(int key, long long value) {
+  if (key == 1) {
+    if (value < 0) return DYNCONV_ERR_INVALID_ARG;
+    g_wait_ns.store(value == 0 ? kDefaultWaitNs : value * 1000LL);
+    return DYNCONV_OK;
+  }
+  if (key == 2) {
+    g_inject_skip.store(value != 0 ? 1 : 0);
+    return DYNCONV_OK;
+  }
+  return DYNCONV_ERR_INVALID_ARG;
+}
+
+size_t dynconv_workspace_size(const dynconv_desc* desc) {
+  if (validate_desc(desc) != DYNCONV_OK) return 0;
+  return premix_workspace(desc);
+}
+
+int dynconv_select_variant(const dynconv_desc* desc, size_t workspace_bytes) {
+  int rc = validate_desc(desc);
+  if (rc) return rc;
+  if (desc->variant != DYNCONV_VARIANT_AUTO) return desc->variant;
+  // 148 SMs and 227 KB of opt-in shared memory per CTA: the B200 figures, so
+  // that the choice is available without a device.
+  return select_variant(desc, workspace_bytes, 148, 232448);
+}
+
+int dynconv_route(const dynconv_desc* desc, const void* x, const float* Wr, const float* br,
+                  int mode, float tau, float* alpha, void* stream) {
+  int rc = validate_desc(desc);
+  if (rc) return rc;
+  if (!x || !Wr || !alpha) return DYNCONV_ERR_INVALID_ARG;
+  if (mode != DYNCONV_SIGMOID && mode != DYNCONV_SOFTMAX) return DYNCONV_ERR_INVALID_ARG;
+  if (mode == DYNCONV_SOFTMAX && !(tau > 0.f)) return DYNCONV_ERR_INVALID_ARG;
+  if (desc->n > 1024 || desc->C_in > 16384) return DYNCONV_ERR_UNSUPPORTED;
+  if (desc->B == 0) return DYNCONV_OK;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc) return rc;
+
+  const int C = desc->C_in;
+  const size_t eb = elem_bytes(desc);
+  const bool vec = aligned16(x) && (C * eb) % 16 == 0;
+  const int VEC = vec ? static_cast<int>(16 / eb) : 1;
+  const int nv = C / VEC;
+  const int tpp = std::min(nv, dc::kRouteThreads);
+  const int lanes_p = dc::kRouteThreads / tpp;
+  const size_t smem = sizeof(float) * (static_cast<size_t>(lanes_p) * C + 2 * C + desc->n);
+  const int HW = desc->H * desc->W;
+  // enough CTAs per sample to keep ~2 CTAs per SM streaming, at most 8 (portable cluster)
+  int nsplit = (2 * st->sms + desc->B - 1) / std::max(desc->B, 1);
+  nsplit = std::max(1, std::min({nsplit, 8, HW}));
+
+  dc::RouteParams p{desc->B, C, HW, desc->n, mode, tau, x, Wr, br, alpha};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nsplit, desc->B, 1);
+  cfg.blockDim = dim3(dc::kRouteThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nsplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+
+  cudaError_t e;
+  auto launch = [&](auto kern) {
+    if (smem > 48 * 1024) {
+      cudaError_t ea = ensure_smem(kern, smem);
+      if (ea != cudaSuccess) return ea;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, p);
+  };
+  if (desc->dtype == DYNCONV_BF16)
+    e = vec ? launch(dc::route_kernel<__nv_bfloat16, 8>) : launch(dc::route_kernel<__nv_bfloat16, 1>);
+  else
+    e = vec ? launch(dc::route_kernel<float, 4>) : launch(dc::route_kernel<float, 1>);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) return cuda_fail(e, "route_kernel launch");
+  return check_launch("route_kernel");
+}
+
+int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts,
+                    const float* alpha, const float* bias, void* y, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  int rc = validate_desc(desc);
+  if (rc) return rc;
+  if (!x || !experts || !alpha || !y) return DYNCONV_ERR_INVALID_ARG;
+  if (desc->B == 0) return DYNCONV_OK;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  int variant = desc->variant;
+  if (variant == DYNCONV_VARIANT_AUTO)
+    variant = select_variant(desc, workspace ? workspace_bytes : 0, st->sms, st->max_smem_optin);
+
+  switch (variant) {
+    case DYNCONV_VARIANT_FUSED:
+    case DYNCONV_VARIANT_OUTSIDE:
+    case DYNCONV_VARIANT_PREMIX: {
+      if (!tc_shape_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
+      if (!aligned16(x) || !aligned16(experts) || !aligned16(y)) return DYNCONV_ERR_MISALIGNED;
+      return run_tc(desc, variant, st, x, experts, alpha, bias, y, workspace, workspace_bytes, s);
+    }
+    case DYNCONV_VARIANT_DEPTHWISE: {
+      if (!depthwise_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
+      if (!aligned16(x) || !aligned16(y)) return DYNCONV_ERR_MISALIGNED;
+      dc::DwParams p{};
+      p.B = desc->B; p.C = desc->C_in; p.H = desc->H; p.W = desc->W; p.pad = desc->pad;
+      p.n = desc->n;
+      p.Ho = out_size(desc->H, desc->KH, 1, desc->pad);
+      p.Wo = out_size(desc->W, desc->KW, 1, desc->pad);
+      p.tile_cols = std::min(p.Wo, dc::kDwMaxCols);
+      p.x = static_cast<const __nv_bfloat16*>(x);
+      p.experts = static_cast<const __nv_bfloat16*>(experts);
+      p.alpha = alpha;
+      p.bias = bias;
+      p.y = static_cast<__nv_bfloat16*>(y);
+      const int K = desc->KH;
+      const int TC = p.tile_cols + K - 1, TR = dc::kDwRows + K - 1;
+      const size_t smem = sizeof(float) * (dc::kDwChunk * K * K + dc::kDwChunk + ((p.n + 3) & ~3)) +
+                          static_cast<size_t>(TR) * TC * dc::kDwChunk * 2;
+      if (smem > static_cast<size_t>(st->max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
+      const int row_blocks = (p.Ho + dc::kDwRows - 1) / dc::kDwRows;
+      const int col_blocks = (p.Wo + p.tile_cols - 1) / p.tile_cols;
+      dim3 grid(row_blocks * col_blocks, (desc->C_in + dc::kDwChunk - 1) / dc::kDwChunk, desc->B);
+      dim3 block(dc::kDwPairs * p.tile_cols);
+      auto go = [&](auto kern) -> int {
+        cudaError_t e = ensure_smem(kern, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(depthwise)");
+        kern<<<grid, block, smem, s>>>(p);
+        return check_launch("depthwise_kernel");
+      };
+      if (K == 3) return go(dc::depthwise_kernel<3>);
+      if (K == 5) return go(dc::depthwise_kernel<5>);
+      return go(dc::depthwise_kernel<7>);
+    }
+    case DYNCONV_VARIANT_DIRECT: {
+      const int Cg = desc->C_in / desc->groups;
+      const long long wrow = 1LL * desc->KH * desc->KW * Cg;
+      const long long budget = (st->max_smem_optin - 4LL * desc->n - 1024) / 4;
+      long long cob = std::min<long long>(desc->C_out, 64);
+      while (cob > 1 && cob * (wrow + 1) > budget) cob /= 2;
+      if (cob * (wrow + 1) > budget) return DYNCONV_ERR_UNSUPPORTED;
+      dc::DirectParams p{};
+      p.B = desc->B; p.Cin = desc->C_in; p.H = desc->H; p.W = desc->W; p.Cout = desc->C_out;
+      p.KH = desc->KH; p.KW = desc->KW; p.stride = desc->stride; p.pad = desc->pad;
+      p.groups = desc->groups; p.n = desc->n;
+      p.Ho = out_size(desc->H, desc->KH, desc->stride, desc->pad);
+      p.Wo = out_size(desc->W, desc->KW, desc->stride, desc->pad);
+      p.cob = static_cast<int>(cob);
+      p.x = x; p.experts = experts; p.alpha = alpha; p.bias = bias; p.y = y;
+      const size_t smem = sizeof(float) * (desc->n + cob + cob * wrow);
+      dim3 grid((p.Ho * p.Wo + dc::kDirectPix - 1) / dc::kDirectPix,
+                static_cast<unsigned>((desc->C_out + cob - 1) / cob), desc->B);
+      auto go = [&](auto kern) -> int {
+        cudaError_t e = ensure_smem(kern, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(direct)");
+        kern<<<grid, dc::kDirectThreads, smem, s>>>(p);
+        return check_launch("direct_conv_kernel");
+      };
+      if (desc->dtype == DYNCONV_F32) return go(dc::direct_conv_kernel<float>);
+      return go(dc::direct_conv_kernel<__nv_bfloat16>);
+    }
+    default:
+      return DYNCONV_ERR_INVALID_ARG;
+  }
+}
+
+int dynconv_device_status(void* stream) {
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_device_err, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  if (word != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_err, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+    std::snprintf(g_last_err, sizeof(g_last_err), "device error word 0x%x", word);
+    return DYNCONV_ERR_TIMEOUT;
+  }
+  return DYNCONV_OK;
+}
+
+}  // extern "C"

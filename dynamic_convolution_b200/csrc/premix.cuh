@@ -1,0 +1,273 @@
+// Tensor-core kernel mixing: W[b][w] = sum_i alpha[b][i] * E[i][w] for every
+// sample b and every weight element w -- "a linear mixture of n static
+// kernels weighted with their input-dependent attentions" (KernelWarehouse,
+// abstract), done for all samples at once so that every expert byte is read
+// from HBM once per pass instead of once per sample.
+//
+// As a GEMM: M = samples (128 per tile), N = weight elements (256 per tile),
+// K = experts (padded to a multiple of 16).
+//  * A = alpha, converted once per CTA into two bf16 operands, alpha_hi =
+//    bf16(alpha) and alpha_lo = bf16(alpha - alpha_hi), K-major with the
+//    128-byte swizzle; two MMAs per K step (hi and lo) keep ~16 bits of alpha.
+//  * B = the experts exactly as they are stored, E[i][w] with w contiguous:
+//    an MN-major operand. TMA boxes {64 weights, K experts} land as 128-byte
+//    rows per expert with the 128-byte swizzle; 64-weight atoms sit
+//    LBO = K*128 bytes apart, 8-expert groups SBO = 1024 bytes apart.
+//  * D (fp32) lives in TMEM, double-buffered (2 x 256 columns) so the
+//    epilogue of one tile overlaps the MMAs of the next; the epilogue rounds to
+//    bf16 and each thread (one sample) stores 64 contiguous bytes per chunk.
+// Persistent: one CTA per SM walks the (weight-tile, sample-tile) space.
+#pragma once
+
+#include "common.cuh"
+
+namespace dc {
+
+constexpr int kPmThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kPmN = 256;         // weights per tile
+
+__host__ __device__ inline int pm_nk(int n) { return (n + 15) / 16 * 16; }
+__host__ __device__ inline int pm_kcols(int n) { return (pm_nk(n) + 63) / 64; }
+
+inline bool premix_shape_ok(int B, int n, int Cout, int taps, int Cin) {
+  if (n > 256 || B <= 0) return false;
+  const long long wsize = 1LL * Cout * taps * Cin;
+  if (wsize % 8 != 0) return false;
+  const int m_tiles = (B + 127) / 128;
+  const long long a_bytes = 2LL * m_tiles * pm_kcols(n) * 16384;
+  const long long stage = 1LL * pm_nk(n) * 512;
+  return a_bytes <= 98304 && a_bytes + 2 * stage <= 200 * 1024;
+}
+
+struct PmParams {
+  int B, n, nk, m_tiles, stages;
+  long long wsize;       // weight elements per expert
+  long long tiles;       // n_tiles * m_tiles
+  int a_bytes;           // bytes of all A operands
+  int stage_bytes;       // bytes of one expert stage
+  const float* alpha;
+  __nv_bfloat16* out;    // [B][wsize]
+  int* err;
+  long long wait_ns;
+};
+
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;  // between 64-element MN atoms
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;             // between 8-row K groups
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+__global__ void __launch_bounds__(kPmThreads, 1)
+    premix_kernel(const __grid_constant__ CUtensorMap emap, PmParams p) {
+  extern __shared__ __align__(1024) unsigned char pm_smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t raw = smem_u32(pm_smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* base_ptr = pm_smem_raw + (base - raw);
+  const int S = p.stages;
+  const int kcols = (p.nk + 63) / 64;
+  const uint32_t a_base = base;                         // [m_tile][hi/lo][kcol][128 rows x 128 B]
+  const uint32_t e_base = a_base + p.a_bytes;           // [stage][4 atoms][nk rows x 128 B]
+  const uint32_t bar_base = e_base + S * p.stage_bytes;
+  auto full = [&](int s) { return bar_base + 8u * s; };
+  auto empty = [&](int s) { return bar_base + 8u * (S + s); };
+  auto tfull = [&](int a) { return bar_base + 8u * (2 * S + a); };
+  auto tempty = [&](int a) { return bar_base + 8u * (2 * S + 2 + a); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * S + 4);
+  unsigned char* misc = base_ptr + (bar_base - base) + 8u * (2 * S + 5);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&emap);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), 512);
+    tmem_relinquish();
+  }
+  // A operands: alpha split into bf16 hi + lo, zero outside [B) x [n)
+  const int a_elems = p.m_tiles * 128 * kcols * 64;
+  for (int e = threadIdx.x; e < a_elems; e += kPmThreads) {
+    const int k = e % (kcols * 64);
+    const int m = e / (kcols * 64);  // global sample row
+    const int mt = m / 128, r = m % 128;
+    float a = 0.f;
+    if (m < p.B && k < p.n) a = p.alpha[static_cast<size_t>(m) * p.n + k];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(a);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(a - __bfloat162float(hi));
+    const uint32_t off = static_cast<uint32_t>(k / 64) * 16384u + r * 128u +
+                         ((((k % 64) >> 3) ^ (r & 7)) << 4) + (k & 7) * 2;
+    const uint32_t hi_addr = a_base + (mt * 2 + 0) * kcols * 16384u + off;
+    const uint32_t lo_addr = a_base + (mt * 2 + 1) * kcols * 16384u + off;
+    asm volatile("st.shared.b16 [%0], %1;" ::"r"(hi_addr),
+                 "h"(*reinterpret_cast<const unsigned short*>(&hi)) : "memory");
+    asm volatile("st.shared.b16 [%0], %1;" ::"r"(lo_addr),
+                 "h"(*reinterpret_cast<const unsigned short*>(&lo)) : "memory");
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const long long my_tiles =
+      p.tiles > blockIdx.x ? (p.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      long long issued = 0;
+      for (long long j = 0; j < my_tiles; ++j) {
+        const long long t = blockIdx.x + j * gridDim.x;
+        const long long ntile = t / p.m_tiles;
+        const int s = static_cast<int>(j % S);
+        const uint32_t ph = static_cast<uint32_t>((j / S) & 1);
+        if (!wait_bounded(empty(s), ph ^ 1u, ctl, kErrWaitProducer)) break;
+        mbar_arrive_expect_tx(full(s), static_cast<uint32_t>(p.stage_bytes));
+        const uint32_t dst = e_base + s * p.stage_bytes;
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+          tma_load_2d(dst + a * p.nk * 128, &emap, full(s),
+                      static_cast<int>(ntile * kPmN + a * 64), 0);
+        ++issued;
+      }
+      for (long long j = (issued > S ? issued - S : 0); j < issued; ++j)
+        wait_drain(full(static_cast<int>(j % S)), static_cast<uint32_t>((j / S) & 1), p.wait_ns,
+                   p.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, kPmN) | (1u << 16);  // B is MN-major
+      const uint32_t lbo = static_cast<uint32_t>(p.nk) * 128u;
+      bool ok = true;
+      for (long long j = 0; j < my_tiles && ok; ++j) {
+        const long long t = blockIdx.x + j * gridDim.x;
+        const int mt = static_cast<int>(t % p.m_tiles);
+        const int s = static_cast<int>(j % S);
+        const int ab = static_cast<int>(j & 1);
+        if (!wait_bounded(full(s), static_cast<uint32_t>((j / S) & 1), ctl, kErrWaitMma)) { ok = false; break; }
+        if (!wait_bounded(tempty(ab), static_cast<uint32_t>((j >> 1) & 1) ^ 1u, ctl, kErrWaitMma)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t e_s = e_base + s * p.stage_bytes;
+        const uint32_t d = tmem_base + ab * kPmN;
+        for (int kk = 0; kk < p.nk / 16; ++kk) {
+          const uint64_t bd = smem_desc_mn_sw128(e_s + kk * 2048, lbo);
+          const uint32_t aoff = static_cast<uint32_t>(kk / 4) * 16384u + (kk % 4) * 32u;
+          const uint64_t ahi = smem_desc_sw128(a_base + (mt * 2 + 0) * kcols * 16384u + aoff);
+          const uint64_t alo = smem_desc_sw128(a_base + (mt * 2 + 1) * kcols * 16384u + aoff);
+          tc_mma_f16(d, ahi, bd, idesc, kk > 0 ? 1u : 0u);
+          tc_mma_f16(d, alo, bd, idesc, 1u);
+        }
+        tc_commit(empty(s));
+        tc_commit(tfull(ab));
+      }
+      if (!ok) {
+        tc_commit(drain_bar);
+        wait_drain(drain_bar, 0, p.wait_ns, p.err);
+      }
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = samples of the tile
+    const int q = warp & 3;
+    for (long long j = 0; j < my_tiles; ++j) {
+      const long long t = blockIdx.x + j * gridDim.x;
+      const long long ntile = t / p.m_tiles;
+      const int mt = static_cast<int>(t % p.m_tiles);
+      const int ab = static_cast<int>(j & 1);
+      if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j >> 1) & 1), ctl, kErrWaitEpilogue)) break;
+      tc_fence_after();
+      const int b = mt * 128 + 32 * q + lane;
+      const long long w0 = ntile * kPmN;
+#pragma unroll 1
+      for (int ch = 0; ch < kPmN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * kPmN + ch * 32, r);
+        tmem_ld_wait();
+        const long long w = w0 + ch * 32;
+        if (b < p.B && w < p.wsize) {
+          __nv_bfloat16* dst = p.out + static_cast<size_t>(b) * p.wsize + w;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            if (w + v * 8 < p.wsize) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+              o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+              o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+              o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+              *reinterpret_cast<uint4*>(dst + v * 8) = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty(ab));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// Host launcher. Returns 0, -1 (CUDA launch error), -2 (tensor map), -3 (shape).
+template <typename EncodeFn, typename SmemFn>
+inline int launch_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bfloat16* out,
+                         int B, int n, long long wsize, int* err, long long wait_ns, int sms,
+                         cudaStream_t stream, EncodeFn encode, SmemFn ensure_smem_fn) {
+  PmParams p{};
+  p.B = B;
+  p.n = n;
+  p.nk = pm_nk(n);
+  p.m_tiles = (B + 127) / 128;
+  p.wsize = wsize;
+  const long long n_tiles = (wsize + kPmN - 1) / kPmN;
+  p.tiles = n_tiles * p.m_tiles;
+  p.a_bytes = 2 * p.m_tiles * pm_kcols(n) * 16384;
+  p.stage_bytes = p.nk * 512;
+  const int budget = 200 * 1024 - p.a_bytes;
+  p.stages = std::min(4, budget / p.stage_bytes);
+  if (p.stages < 2) return -3;
+  p.alpha = alpha;
+  p.out = out;
+  p.err = err;
+  p.wait_ns = wait_ns;
+
+  CUtensorMap emap;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(wsize), static_cast<cuuint64_t>(n)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(wsize) * 2};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(p.nk)};
+  const cuuint32_t es[2] = {1u, 1u};
+  if (encode(&emap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(experts), dims,
+             strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return -2;
+  // at least 120 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
+  const size_t smem = std::max<size_t>(120 * 1024, 1024 + static_cast<size_t>(p.a_bytes) +
+                                                       static_cast<size_t>(p.stages) * p.stage_bytes +
+                                                       8 * (2 * p.stages + 5) + 16);
+  if (ensure_smem_fn(premix_kernel, smem) != cudaSuccess) return -1;
+  const long long grid = std::min<long long>(p.tiles, sms);
+  premix_kernel<<<static_cast<unsigned>(grid), kPmThreads, smem, stream>>>(emap, p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace dc

@@ -1,0 +1,166 @@
+/*
+ * dynconv.h -- C ABI of the B200 (sm_100a) dynamic-convolution library.
+ *
+ * The library computes the per-sample kernel-mixture convolution:
+ *
+ *   alpha_b = sigmoid(FC(GAP(x_b)))  or  softmax(FC(GAP(x_b)) / tau)
+ *   W_b     = sum_i alpha_{b,i} W_i                 (n static experts W_i)
+ *   y_b     = conv2d(x_b, W_b) + sum_i alpha_{b,i} bias_i
+ *
+ * Sources: the linear mixture of n static kernels weighted with input-dependent
+ * attentions is the definition in "KernelWarehouse: Rethinking the Design of
+ * Dynamic Convolution" (abstract); one specialised kernel per example is
+ * "CondConv: Conditionally Parameterized Convolutions for Efficient Inference"
+ * (abstract); the temperature on the kernel attention is from "FMDConv: Fast
+ * multi-attention dynamic convolution via speed-accuracy trade-off" (abstract).
+ * The router's exact form (global average pool -> one linear layer -> sigmoid
+ * or temperature softmax), the bias mixing, the NHWC layout and the bf16
+ * storage are readings taken where those pages are silent.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees them and keeps no reference after the call's work completes.
+ *  - Calls only enqueue work on `stream` (a cudaStream_t passed as void*;
+ *    NULL is the legacy default stream) and return; results are valid once the
+ *    stream reaches that point.
+ *  - No call allocates device memory. Scratch, where a variant needs it, is a
+ *    caller-provided workspace (see dynconv_workspace_size).
+ *  - Return value: DYNCONV_OK (0) or a negative status below. Argument errors
+ *    are detected on the host before anything is launched. No C++ exception
+ *    crosses this interface. There is no CPU fallback: without a usable
+ *    sm_100 device the calls fail with DYNCONV_ERR_CUDA.
+ *
+ * Layouts (row-major, last index fastest):
+ *   x        [B][H][W][C_in]                    dtype (fp32 or bf16), NHWC
+ *   experts  [n][C_out][KH][KW][C_in/groups]    dtype
+ *   Wr       [n][C_in] fp32,  br [n] fp32       router weights / bias
+ *   bias     [n][C_out] fp32, or NULL for none  per-expert output bias
+ *   alpha    [B][n] fp32                        routing weights
+ *   y        [B][H_out][W_out][C_out]           dtype, NHWC
+ * with H_out = (H + 2*pad - KH)/stride + 1, W_out likewise.
+ */
+#ifndef DYNCONV_H
+#define DYNCONV_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------- */
+#define DYNCONV_OK               0
+#define DYNCONV_ERR_INVALID_ARG (-1)  /* NULL pointer, non-positive size, tau <= 0 with softmax,
+                                         groups not dividing the channels, bad enum value */
+#define DYNCONV_ERR_UNSUPPORTED (-2)  /* a shape or variant that no kernel here handles */
+#define DYNCONV_ERR_MISALIGNED  (-3)  /* a pointer not 16-byte aligned (vector loads / TMA) */
+#define DYNCONV_ERR_CUDA        (-4)  /* a CUDA runtime or driver error (no device, launch failure) */
+#define DYNCONV_ERR_TIMEOUT     (-5)  /* a kernel's bounded wait expired (see dynconv_device_status) */
+#define DYNCONV_ERR_WORKSPACE   (-6)  /* the forced variant needs a larger workspace */
+
+/* ---- enums -------------------------------------------------------------- */
+typedef enum { DYNCONV_F32 = 0, DYNCONV_BF16 = 1 } dynconv_dtype;
+typedef enum { DYNCONV_SIGMOID = 0, DYNCONV_SOFTMAX = 1 } dynconv_mode;
+
+/* Which forward kernel runs.
+ *  AUTO    - chosen by a host cost model from the descriptor (and the workspace
+ *            the caller passed);
+ *  FUSED   - input-side mixing inside the tensor-core convolution: every CTA
+ *            mixes its sample's weight tile from the experts on CUDA cores
+ *            into a bf16 shared-memory operand of tcgen05 MMAs (bf16 only);
+ *  OUTSIDE - output-side mixing: y_b = sum_i alpha_{b,i} (x_b conv W_i) + b_b as
+ *            one K-stacked tensor-core GEMM over (expert, tap, channel) with the
+ *            operand alpha_{b,i} W_i (bf16 only; n times the conv work);
+ *  PREMIX  - W_b for all samples is mixed first by a tensor-core GEMM into the
+ *            workspace (bf16), then a tensor-core convolution reads it
+ *            (bf16 only; needs dynconv_workspace_size bytes);
+ *  DIRECT  - CUDA-core direct convolution, fp32 accumulation, any shape
+ *            (the fp32 path; also bf16 shapes the tensor-core kernels reject);
+ *  DEPTHWISE - CUDA-core depthwise kernel (groups == C_in == C_out). */
+typedef enum {
+  DYNCONV_VARIANT_AUTO = 0,
+  DYNCONV_VARIANT_FUSED = 1,
+  DYNCONV_VARIANT_OUTSIDE = 2,
+  DYNCONV_VARIANT_PREMIX = 3,
+  DYNCONV_VARIANT_DIRECT = 4,
+  DYNCONV_VARIANT_DEPTHWISE = 5
+} dynconv_variant;
+
+/* Layer descriptor. groups must divide C_in and C_out; the depthwise kernel
+ * takes groups == C_in == C_out. `variant` forces a kernel (AUTO: cost model). */
+typedef struct {
+  int B, C_in, H, W, C_out, KH, KW, stride, pad, groups, n;
+  int dtype;    /* dynconv_dtype */
+  int variant;  /* dynconv_variant */
+} dynconv_desc;
+
+/* ---- routing ------------------------------------------------------------
+ * alpha[b][i] for every sample b of x (steps: global average pool over the
+ * H*W unpadded pixels, one linear layer z = Wr g + br, then sigmoid(z), or
+ * softmax(z / tau) over the n experts).
+ *   desc   uses B, C_in, H, W, n, dtype;
+ *   x      device, [B][H][W][C_in] of desc->dtype, 16-byte aligned, and
+ *          C_in * sizeof(dtype) a multiple of 16;
+ *   Wr     device fp32 [n][C_in];  br device fp32 [n] or NULL (zero bias);
+ *   mode   dynconv_mode; tau > 0 required for SOFTMAX, ignored for SIGMOID;
+ *   alpha  device fp32 [B][n], written.
+ * Deterministic: the reduction order is fixed. Errors: INVALID_ARG,
+ * MISALIGNED, UNSUPPORTED (n > 1024 or C_in > 16384), CUDA. */
+int dynconv_route(const dynconv_desc* desc, const void* x, const float* Wr, const float* br,
+                  int mode, float tau, float* alpha, void* stream);
+
+/* ---- forward -------------------------------------------------------------
+ * y_b = conv2d(x_b, sum_i alpha[b][i] W_i) + sum_i alpha[b][i] bias_i for every b.
+ *   x, experts, y  device, layouts above, desc->dtype, 16-byte aligned;
+ *   alpha          device fp32 [B][n] (typically written by dynconv_route on
+ *                  the same stream);
+ *   bias           device fp32 [n][C_out] or NULL;
+ *   workspace      device scratch of workspace_bytes bytes, or NULL/0. Only the
+ *                  PREMIX variant uses it; AUTO never picks PREMIX unless the
+ *                  workspace is large enough.
+ * Precision: bf16 in, fp32 accumulate, the mixed kernel rounded once to bf16
+ * (tensor-core variants), y rounded once to bf16. fp32 layers accumulate and
+ * mix in fp32.
+ * Errors: INVALID_ARG, UNSUPPORTED (forced variant cannot take the shape),
+ * MISALIGNED, WORKSPACE (forced PREMIX with too small a workspace), CUDA. */
+int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts,
+                    const float* alpha, const float* bias, void* y, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace the PREMIX variant needs for this descriptor (0 if it
+ * cannot run this shape). Pure host function. */
+size_t dynconv_workspace_size(const dynconv_desc* desc);
+
+/* The variant AUTO resolves to for this descriptor and workspace size
+ * (a dynconv_variant value), or a negative status. Pure host function. */
+int dynconv_select_variant(const dynconv_desc* desc, size_t workspace_bytes);
+
+/* ---- status and diagnostics ------------------------------------------------ */
+
+/* Static, human-readable text for a status code (never NULL). */
+const char* dynconv_status_string(int status);
+
+/* Text of the last CUDA error this thread saw inside the library (static
+ * storage, overwritten by the next error), or "" if none. */
+const char* dynconv_last_error(void);
+
+/* Synchronise `stream`, then read and clear this device's error word, which
+ * kernels set when a bounded wait on a barrier expires (they then skip the
+ * rest of their work and exit cleanly, leaving y unspecified). Returns
+ * DYNCONV_OK, DYNCONV_ERR_TIMEOUT, or DYNCONV_ERR_CUDA. */
+int dynconv_device_status(void* stream);
+
+/* Number of kernel launches the library has issued in this process. */
+unsigned long long dynconv_launch_count(void);
+
+/* Test hook. key 1: bounded-wait limit in microseconds for subsequent launches
+ * (0 restores the default of 500000). key 2: when nonzero, the next forward
+ * launch of a tensor-core variant withholds one producer arrival, so that its
+ * consumer's bounded wait must expire and report DYNCONV_ERR_TIMEOUT.
+ * Returns DYNCONV_OK or DYNCONV_ERR_INVALID_ARG. */
+int dynconv_test_hook(int key, long long value);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DYNCONV_H */

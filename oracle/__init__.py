@@ -51,6 +51,8 @@ def configure(lib):
     lib.oracle_route.restype = i
     lib.oracle_forward.argtypes = [i] * 11 + [dp, dp, dp, dp, i, i, dp, i]
     lib.oracle_forward.restype = i
+    lib.oracle_forward_rows.argtypes = [i] * 11 + [dp, dp, dp, dp, i, i, i, dp]
+    lib.oracle_forward_rows.restype = i
     lib.oracle_assemble.argtypes = [i, ctypes.c_long, dp, dp, dp]
     lib.oracle_assemble.restype = None
     lib.oracle_threads_used.argtypes = [i, i]
@@ -124,6 +126,26 @@ def forward(x, experts, alpha, bias=None, stride: int = 1, pad: int = 0, groups:
                                 int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_forward rejected its arguments (rc={rc})")
+    return y
+
+
+def forward_rows(x, experts, alpha, bias, b: int, oh0: int, noh: int, stride: int = 1,
+                 pad: int = 0, groups: int = 1):
+    """Output rows oh0..oh0+noh-1 of sample b only: y[noh][W_out][C_out] (one thread)."""
+    x = _f64(x)
+    experts = _f64(experts)
+    alpha = _f64(alpha)
+    bias = _f64(bias)
+    B, H, W, Cin = x.shape
+    n, Cout, KH, KW, Cg = experts.shape
+    assert Cg * groups == Cin
+    Wo = (W + 2 * pad - KW) // stride + 1
+    y = np.empty((noh, Wo, Cout), dtype=np.float64)
+    rc = _load().oracle_forward_rows(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n, _dp(x),
+                                     _dp(experts), _dp(alpha), _dp(bias), int(b), int(oh0),
+                                     int(noh), _dp(y))
+    if rc != 0:
+        raise ValueError(f"oracle_forward_rows rejected its arguments (rc={rc})")
     return y
 
 

@@ -180,8 +180,9 @@ void oracle_mix_bias(int n, int Cout, const double *bias, const double *alpha_b,
 
 typedef struct {
   int Cin, H, W, Cout, KH, KW, stride, pad, groups, n, Ho, Wo, b0;
+  int oh_begin, oh_end;   /* output rows computed, [oh_begin, oh_end) */
   const double *x, *experts, *alpha, *bias;
-  double *y;
+  double *y;              /* rows oh_begin.. of samples b0.. */
 } fwd_ctx;
 
 static void forward_one(void *vctx, int b) {
@@ -197,8 +198,9 @@ static void forward_one(void *vctx, int b) {
 
   /* Step 5: y[oh,ow,co] = b_b[co] + sum_{kh,kw,ci} xpad[oh*s+kh-p, ow*s+kw-p, g*Cg+ci] W_b[co,kh,kw,ci] */
   const double *xb = f->x + (size_t)b * f->H * f->W * f->Cin;
-  double *yb = f->y + (size_t)(b - f->b0) * f->Ho * f->Wo * f->Cout;
-  for (int oh = 0; oh < f->Ho; ++oh)
+  const int nrows = f->oh_end - f->oh_begin;
+  double *yb = f->y + (size_t)(b - f->b0) * nrows * f->Wo * f->Cout;
+  for (int oh = f->oh_begin; oh < f->oh_end; ++oh)
     for (int ow = 0; ow < f->Wo; ++ow)
       for (int co = 0; co < f->Cout; ++co) {
         const int g = co / Coutg;
@@ -214,7 +216,7 @@ static void forward_one(void *vctx, int b) {
             for (int ci = 0; ci < Cg; ++ci) s += xp[ci] * wp[ci];
           }
         }
-        yb[((size_t)oh * f->Wo + ow) * f->Cout + co] = s;
+        yb[((size_t)(oh - f->oh_begin) * f->Wo + ow) * f->Cout + co] = s;
       }
   free(Wb);
   free(bb);
@@ -238,7 +240,26 @@ int oracle_forward(int B, int Cin, int H, int W, int Cout, int KH, int KW, int s
   const int Ho = oracle_out_size(H, KH, stride, pad), Wo = oracle_out_size(W, KW, stride, pad);
   if (Ho <= 0 || Wo <= 0) return -1;
   if (nb == 0) return 0;
-  fwd_ctx f = {Cin, H, W, Cout, KH, KW, stride, pad, groups, n, Ho, Wo, b0,
+  fwd_ctx f = {Cin, H, W, Cout, KH, KW, stride, pad, groups, n, Ho, Wo, b0, 0, Ho,
                x, experts, alpha, bias, y};
   return run_samples(forward_one, &f, b0, nb, nthreads);
+}
+
+/* Output rows oh0 .. oh0+noh-1 of sample b only, written to y[noh][Wo][Cout]
+ * (the same definition restricted to a band of output rows; single thread). */
+int oracle_forward_rows(int B, int Cin, int H, int W, int Cout, int KH, int KW, int stride,
+                        int pad, int groups, int n, const double *x, const double *experts,
+                        const double *alpha, const double *bias, int b, int oh0, int noh,
+                        double *y) {
+  if (B <= 0 || Cin <= 0 || H <= 0 || W <= 0 || Cout <= 0 || KH <= 0 || KW <= 0) return -1;
+  if (stride <= 0 || pad < 0 || groups <= 0 || n <= 0) return -1;
+  if (Cin % groups != 0 || Cout % groups != 0) return -1;
+  if (!x || !experts || !alpha || !y) return -1;
+  const int Ho = oracle_out_size(H, KH, stride, pad), Wo = oracle_out_size(W, KW, stride, pad);
+  if (Ho <= 0 || Wo <= 0 || b < 0 || b >= B || oh0 < 0 || noh < 0 || oh0 + noh > Ho) return -1;
+  if (noh == 0) return 0;
+  fwd_ctx f = {Cin, H, W, Cout, KH, KW, stride, pad, groups, n, Ho, Wo, b, oh0, oh0 + noh,
+               x, experts, alpha, bias, y};
+  forward_one(&f, b);
+  return 0;
 }

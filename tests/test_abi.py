@@ -1,0 +1,121 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports
+every function the header declares, validates arguments before touching CUDA,
+and fails loudly (DYNCONV_ERR_CUDA) rather than falling back to the CPU when no
+device is present."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import dynamic_convolution_b200 as dc
+from dynamic_convolution_b200 import build as dcbuild
+from dynamic_convolution_b200 import synth
+
+HEADER = os.path.join(dcbuild.ROOT, "include", "dynconv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dcbuild.build()
+    return dc.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dynconv_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert declared_functions() == sorted(dc.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert dc.dynconv_status_string(code)
+    assert dc.dynconv_status_string(12345) == "unknown status"
+
+
+def _desc(**kw):
+    base = dict(B=2, C_in=8, H=8, W=8, C_out=8, KH=3, KW=3, stride=1, pad=1, groups=1, n=4,
+                dtype=dc.F32, variant=0)
+    base.update(kw)
+    return dc.make_desc(**base)
+
+
+BAD = [dict(C_in=0), dict(H=-1), dict(KH=0), dict(stride=0), dict(pad=-1), dict(groups=3),
+       dict(n=0), dict(dtype=7), dict(variant=9), dict(H=1, W=1, pad=0),
+       dict(groups=2, C_out=5)]
+
+
+@pytest.mark.parametrize("kw", BAD)
+def test_invalid_descriptors_rejected_on_host(lib, kw):
+    d = _desc(**kw)
+    assert dc.dynconv_forward(d, 16, 16, 16, None, 16) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_route(d, 16, 16, None, dc.SIGMOID, 1.0, 16) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_select_variant(d) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_workspace_size(d) == 0
+
+
+def test_null_pointers_and_bad_route_args_rejected(lib):
+    d = _desc()
+    assert dc.dynconv_forward(d, None, 16, 16, None, 16) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_forward(d, 16, 16, 16, None, None) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_route(d, 16, None, None, dc.SIGMOID, 1.0, 16) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_route(d, 16, 16, None, dc.SOFTMAX, 0.0, 16) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_route(d, 16, 16, None, dc.SOFTMAX, -1.0, 16) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_route(d, 16, 16, None, 5, 1.0, 16) == dc.ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_noop(lib):
+    d = _desc(B=0)
+    assert dc.dynconv_forward(d, 16, 16, 16, None, 16) == dc.OK
+    assert dc.dynconv_route(d, 16, 16, None, dc.SIGMOID, 1.0, 16) == dc.OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_no_device_fails_loudly(lib):
+    d = _desc()
+    assert dc.dynconv_forward(d, 16, 16, 16, None, 16) == dc.ERR_CUDA
+    assert dc.dynconv_route(d, 16, 16, None, dc.SIGMOID, 1.0, 16) == dc.ERR_CUDA
+    assert dc.dynconv_last_error() != ""
+
+
+def test_variant_selection_per_config(lib):
+    sel = {name: dc.dynconv_select_variant(dc.desc_from_config(cfg)) for name, cfg in
+           synth.CONFIGS.items()}
+    assert sel["tiny_fp32"] == dc.VARIANT_DIRECT
+    assert sel["effnet_dw_5x5"] == dc.VARIANT_DEPTHWISE
+    for name in ("resnet18_3x3", "effnet_expand_1x1", "deep_3x3_tau30", "large_n64"):
+        assert sel[name] in (dc.VARIANT_FUSED, dc.VARIANT_OUTSIDE), name
+    # with a large enough workspace the premix variant becomes a candidate
+    for name in ("deep_3x3_tau30", "large_n64"):
+        d = dc.desc_from_config(synth.CONFIGS[name])
+        ws = dc.dynconv_workspace_size(d)
+        assert ws == synth.CONFIGS[name].B * synth.CONFIGS[name].weight_elems * 2
+        assert dc.dynconv_select_variant(d, ws) in (dc.VARIANT_FUSED, dc.VARIANT_OUTSIDE,
+                                                     dc.VARIANT_PREMIX)
+    # a forced variant is reported as is
+    d = dc.desc_from_config(synth.CONFIGS["resnet18_3x3"], variant=dc.VARIANT_OUTSIDE)
+    assert dc.dynconv_select_variant(d) == dc.VARIANT_OUTSIDE
+
+
+def test_shapes_outside_tensor_core_kernels_go_direct(lib):
+    # stride 2, odd channel counts, fp32: the CUDA-core direct kernel
+    assert dc.dynconv_select_variant(_desc(dtype=dc.BF16, stride=2)) == dc.VARIANT_DIRECT
+    assert dc.dynconv_select_variant(_desc(dtype=dc.BF16, C_in=12, C_out=12)) == dc.VARIANT_DIRECT
+    assert dc.dynconv_select_variant(_desc(dtype=dc.BF16, groups=2)) == dc.VARIANT_DIRECT
+
+
+def test_test_hook_arguments(lib):
+    assert dc.dynconv_test_hook(1, 0) == dc.OK
+    assert dc.dynconv_test_hook(1, -5) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(99, 0) == dc.ERR_INVALID_ARG

@@ -1,0 +1,214 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the fp64 oracle
+on the same seeded inputs.
+
+* Full-size layer configurations: routing weights on every sample; outputs on
+  sampled whole samples (first, middle, last and two more), computed by the
+  oracle one sample at a time, in the launch configuration the benchmark uses.
+* Small structured cases (per-sample channel offsets, so routing differs
+  strongly between samples) with ragged tails: image heights that do not
+  divide into row blocks, output channels that do not fill a 128-row tile,
+  input channels that do not fill a 64-wide chunk, odd expert counts.
+* Every forward variant the library offers is compared, not only the one the
+  cost model picks.
+"""
+import numpy as np
+import pytest
+import torch
+
+import dynamic_convolution_b200 as dc
+import oracle
+from dynamic_convolution_b200 import synth
+
+from .gpu_util import ALPHA_ABS, Layer, alpha_f32_rounded, compare, from_device
+
+pytestmark = pytest.mark.gpu
+
+DENSE_TC = ["resnet18_3x3", "effnet_expand_1x1", "deep_3x3_tau30", "large_n64"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from dynamic_convolution_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+_CACHE = {}
+
+
+def layer_inputs(name: str) -> synth.LayerInputs:
+    """Seeded inputs; the depthwise layer's input is the bf16-rounded ORACLE output
+    of the 1x1 expand layer of the same block (never the GPU's)."""
+    if name in _CACHE:
+        return _CACHE[name]
+    cfg = synth.CONFIGS[name]
+    inp = synth.make_inputs(cfg)
+    if name == "effnet_dw_5x5":
+        up = layer_inputs("effnet_expand_1x1")
+        a = oracle.route(up.x_f64, up.Wr, up.br, up.cfg.mode, up.cfg.tau)
+        y = oracle.forward(up.x_f64, up.experts_f64, a, up.bias, stride=1, pad=0)
+        inp = inp.with_x(y)
+    _CACHE[name] = inp
+    return inp
+
+
+def sample_ids(B: int):
+    return sorted({0, 1, B // 2, B - 2, B - 1} & set(range(B)))
+
+
+@pytest.mark.parametrize("name", list(synth.CONFIGS))
+def test_route_matches_oracle(name):
+    inp = layer_inputs(name)
+    cfg = inp.cfg
+    L = Layer(inp)
+    L.route()
+    torch.cuda.synchronize()
+    got = from_device(L.alpha)
+    ref = oracle.route(inp.x_f64, inp.Wr, inp.br, cfg.mode, cfg.tau)
+    assert np.abs(got - ref).max() <= ALPHA_ABS, np.abs(got - ref).max()
+    if cfg.mode == synth.SOFTMAX:
+        assert np.abs(got.sum(axis=1) - 1.0).max() < 1e-6
+    # deterministic: a second call gives identical bits
+    first = L.alpha.clone()
+    L.route()
+    torch.cuda.synchronize()
+    assert torch.equal(first, L.alpha)
+
+
+def _forward_case(name, variant, workspace=False):
+    inp = layer_inputs(name)
+    cfg = inp.cfg
+    L = Layer(inp)
+    a64 = alpha_f32_rounded(oracle.route(inp.x_f64, inp.Wr, inp.br, cfg.mode, cfg.tau))
+    L.alpha.copy_(torch.from_numpy(a64.astype(np.float32)))
+    ws = None
+    if workspace:
+        nbytes = dc.dynconv_workspace_size(L.desc(variant))
+        assert nbytes > 0
+        ws = torch.empty(nbytes // 2, dtype=torch.bfloat16, device="cuda")
+    L.forward(variant, workspace=ws)
+    assert dc.dynconv_device_status(None) == dc.OK
+    y = from_device(L.y)
+    for b in sample_ids(cfg.B):
+        ref = oracle.forward(inp.x_f64, inp.experts_f64, a64, inp.bias, stride=cfg.stride,
+                             pad=cfg.pad, groups=cfg.groups, samples=(b, 1))[0]
+        r = compare(y[b], ref, cfg.dtype)
+        assert r["ok"], (name, variant, b, r)
+    assert np.isfinite(y).all()
+
+
+@pytest.mark.parametrize("name", DENSE_TC)
+@pytest.mark.parametrize("variant", [dc.VARIANT_FUSED, dc.VARIANT_OUTSIDE, dc.VARIANT_PREMIX])
+def test_forward_tensor_core_full_size(name, variant):
+    _forward_case(name, variant, workspace=(variant == dc.VARIANT_PREMIX))
+
+
+def test_forward_tiny_fp32_direct():
+    _forward_case("tiny_fp32", dc.VARIANT_DIRECT)
+
+
+@pytest.mark.parametrize("variant", [dc.VARIANT_DEPTHWISE, dc.VARIANT_DIRECT])
+def test_forward_depthwise_full_size(variant):
+    _forward_case("effnet_dw_5x5", variant)
+
+
+@pytest.mark.parametrize("name", list(synth.CONFIGS))
+def test_end_to_end_route_then_forward(name):
+    """GPU route -> GPU forward (AUTO variant) against oracle route -> oracle forward."""
+    inp = layer_inputs(name)
+    cfg = inp.cfg
+    L = Layer(inp)
+    L.route()
+    L.forward()
+    torch.cuda.synchronize()
+    y = from_device(L.y)
+    a = oracle.route(inp.x_f64, inp.Wr, inp.br, cfg.mode, cfg.tau)
+    for b in sample_ids(cfg.B)[:3]:
+        ref = oracle.forward(inp.x_f64, inp.experts_f64, a, inp.bias, stride=cfg.stride,
+                             pad=cfg.pad, groups=cfg.groups, samples=(b, 1))[0]
+        r = compare(y[b], ref, cfg.dtype)
+        assert r["ok"], (name, b, r)
+
+
+SMALL = [
+    # name, B, C_in, C_out, H, W, K, pad, n, mode, tau
+    ("ragged_rows", 3, 64, 128, 13, 11, 3, 1, 4, synth.SOFTMAX, 1.0),
+    ("two_mtiles_partial", 2, 72, 136, 9, 10, 3, 1, 5, synth.SIGMOID, 1.0),
+    ("pointwise_odd_n", 4, 40, 96, 12, 12, 1, 0, 3, synth.SIGMOID, 1.0),
+    ("dense_5x5", 2, 32, 64, 10, 9, 5, 2, 2, synth.SOFTMAX, 0.5),
+    ("single_expert", 2, 64, 128, 8, 8, 3, 1, 1, synth.SOFTMAX, 1.0),
+    ("wide_image", 1, 16, 32, 3, 200, 3, 1, 3, synth.SOFTMAX, 2.0),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+@pytest.mark.parametrize("variant", [dc.VARIANT_FUSED, dc.VARIANT_OUTSIDE, dc.VARIANT_PREMIX,
+                                     dc.VARIANT_DIRECT])
+def test_small_structured_all_variants(case, variant):
+    name, B, Cin, Cout, H, W, K, pad, n, mode, tau = case
+    cfg = synth.LayerConfig(name, synth.BF16, B, Cin, Cout, H, W, K, K, 1, pad, 1, n, mode, tau)
+    inp = synth.make_inputs(cfg, seed=3, structured=1.5)
+    L = Layer(inp)
+    L.route()
+    torch.cuda.synchronize()
+    a_gpu = from_device(L.alpha)
+    a = oracle.route(inp.x_f64, inp.Wr, inp.br, mode, tau)
+    assert np.abs(a_gpu - a).max() <= ALPHA_ABS
+    if n > 1:  # structured inputs: routing really differs between samples
+        assert B == 1 or np.abs(a - a[0]).max() > 1e-2
+    a32 = alpha_f32_rounded(a)
+    L.alpha.copy_(torch.from_numpy(a32.astype(np.float32)))
+    ws = None
+    if variant == dc.VARIANT_PREMIX:
+        ws = torch.empty(dc.dynconv_workspace_size(L.desc(variant)) // 2 + 8,
+                         dtype=torch.bfloat16, device="cuda")
+    L.forward(variant, workspace=ws)
+    torch.cuda.synchronize()
+    ref = oracle.forward(inp.x_f64, inp.experts_f64, a32, inp.bias, stride=1, pad=pad)
+    r = compare(from_device(L.y), ref, synth.BF16)
+    assert r["ok"], (name, variant, r)
+
+
+@pytest.mark.parametrize("variant", [dc.VARIANT_FUSED, dc.VARIANT_DIRECT])
+def test_no_bias(variant):
+    cfg = synth.LayerConfig("nobias", synth.BF16, 2, 64, 64, 7, 7, 3, 3, 1, 1, 1, 3,
+                            synth.SIGMOID, 1.0)
+    inp = synth.make_inputs(cfg, seed=5, structured=1.0)
+    L = Layer(inp)
+    a = alpha_f32_rounded(oracle.route(inp.x_f64, inp.Wr, inp.br, cfg.mode, cfg.tau))
+    L.alpha.copy_(torch.from_numpy(a.astype(np.float32)))
+    L.forward(variant, bias=None)
+    torch.cuda.synchronize()
+    ref = oracle.forward(inp.x_f64, inp.experts_f64, a, None, stride=1, pad=1)
+    assert compare(from_device(L.y), ref, synth.BF16)["ok"]
+
+
+def test_fp32_general_shapes_direct():
+    """fp32 path with stride 2, groups 2 and an odd kernel size."""
+    cfg = synth.LayerConfig("f32_general", synth.F32, 3, 6, 8, 11, 9, 5, 5, 2, 2, 2, 3,
+                            synth.SOFTMAX, 3.0)
+    inp = synth.make_inputs(cfg, seed=9, structured=1.0)
+    L = Layer(inp)
+    L.route()
+    L.forward()
+    torch.cuda.synchronize()
+    a = oracle.route(inp.x_f64, inp.Wr, inp.br, cfg.mode, cfg.tau)
+    assert np.abs(from_device(L.alpha) - a).max() <= ALPHA_ABS
+    ref = oracle.forward(inp.x_f64, inp.experts_f64, a, inp.bias, stride=2, pad=2, groups=2)
+    r = compare(from_device(L.y), ref, synth.F32)
+    assert r["ok"], r
+
+
+def test_outputs_outside_y_untouched():
+    """Canary: the forward writes exactly y, nothing after it."""
+    inp = layer_inputs("resnet18_3x3")
+    cfg = inp.cfg.scaled(B=4)
+    small = synth.make_inputs(cfg)
+    L = Layer(small)
+    big = torch.full((L.y.numel() + 4096,), 7.0, dtype=torch.bfloat16, device="cuda")
+    L.y = big[: L.y.numel()].view(L.y.shape)
+    L.route()
+    for v in (dc.VARIANT_FUSED, dc.VARIANT_OUTSIDE, dc.VARIANT_DIRECT):
+        L.forward(v)
+    torch.cuda.synchronize()
+    assert torch.all(big[L.y.numel():] == 7.0)

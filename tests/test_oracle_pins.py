@@ -346,3 +346,12 @@ def test_synth_recipe_statistics():
     # bf16 rounding is round-to-nearest-even and exact on representable values
     v = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 0.0])
     assert np.array_equal(synth.bf16_to_f64(synth.bf16_bits(v)), [1.0, 1.0, 1.0 + 2 ** -6, -2.5, 0.0])
+
+
+def test_row_band_matches_full_forward():
+    rng = np.random.default_rng(15)
+    x, E, alpha, bias = _rand_layer(rng, 3, 4, 5, 9, 7, 3, 2, 1, 1, 3)
+    full = oracle.forward(x, E, alpha, bias, stride=2, pad=1)
+    for b, oh0, noh in [(0, 0, 1), (2, 1, 3), (1, 0, full.shape[1])]:
+        band = oracle.forward_rows(x, E, alpha, bias, b, oh0, noh, stride=2, pad=1)
+        assert np.array_equal(band, full[b, oh0:oh0 + noh])
