@@ -1,34 +1,41 @@
 // Tensor-core (tcgen05) implicit-GEMM dynamic convolution, bf16 in / out,
-// fp32 accumulation in tensor memory.
+// fp32 accumulation in tensor memory. Stride 1, "same" padding.
 //
-// Per work unit (sample b, block of R image rows, block of 128 output
+// Per work unit (sample b, block of R output rows, block of 128 output
 // channels) the kernel computes
-//     D[co][pix] = sum_k A[co][k] * Bop[pix][k]
-// with k running over (tap kh,kw ; input-channel chunk of 64). The GEMM is
-// "swapped": M = output channels (128 per tile), N = the R*W pixels of the
-// unit, so the per-sample kernel is the A operand and the pixel count only has
-// to be a multiple of 16 (an image row block maps onto N exactly).
+//     D[co][p] = sum_{tap, c} A_tap[co][c] * X[p + s_tap][c]
+// The GEMM is "swapped": M = output channels (128 per tile), N = pixels, so
+// the per-sample kernel is the A operand and the pixel count only has to be a
+// multiple of 16.
 //
-//  * Bop tiles are the activations of tap (kh,kw): one 4-D TMA box
-//    {64 channels, W, R, 1} of x at (c, kw-pad, h0+kh-pad, b). Zero padding is
-//    the TMA's out-of-bounds fill, so the halo costs nothing.
-//  * A tiles (128 x 64 bf16, K-major, 128-byte swizzle) depend on the variant:
-//      FUSED    A = sum_i alpha_{b,i} E_i[co-tile][tap][c-chunk], mixed by 8
-//               warps on CUDA cores from 16-byte expert loads (L2-resident),
-//               rounded once to bf16: "a linear mixture of n static kernels
-//               weighted with their input-dependent attentions"
-//               (KernelWarehouse, abstract), one kernel per example (CondConv,
-//               abstract);
-//      OUTSIDE  k also runs over the experts and A = alpha_{b,i} E_i: the sum
-//               over experts happens in the accumulator, i.e.
-//               y = sum_i alpha_i (x conv W_i), the same result by linearity;
-//      PREMIX   A = W_b tile, TMA-loaded from a workspace where a separate
-//               tensor-core kernel stored every sample's mixed kernel.
-//  * One thread issues tcgen05.mma (M=128, N<=256 per instruction, K=16) into
-//    TMEM and commits each stage back to its "empty" barrier.
-//  * The epilogue (8 warps) reads TMEM lane = output channel, adds the mixed
-//    bias sum_i alpha_i bias_i, rounds to bf16, transposes through shared
-//    memory and writes 16-byte NHWC segments.
+// Activations: the unit's input rows plus the KH-1 halo rows, at the padded
+// width Wp = W + KW - 1, are loaded ONCE per 64-channel chunk with one 4-D TMA
+// box {64 channels, Wp, R+KH-1, 1} at (c, -pad, h0-pad, b); out-of-bounds
+// reads are the zero padding. Output pixels are computed on the same padded
+// grid (p = r*Wp + c; columns c >= W are discarded), so tap (kh, kw) reads the
+// tile at a constant row shift s_tap = kh*Wp + kw: every tap is the same smem
+// tile at another descriptor start address. The 128-byte swizzle is applied
+// on absolute shared-memory address bits by both the TMA and the tensor core,
+// so a view may start at any 128-byte row with the descriptor's base offset
+// left at 0 (checked on B200 against the oracle). Each activation byte
+// crosses L2 once per unit instead of once per tap.
+//
+// The weight operand A (128 x 64 bf16 per step, K-major, 128-byte swizzle)
+// depends on the variant:
+//   FUSED    A = sum_i alpha_{b,i} E_i[co-tile][tap][c-chunk], mixed by 8 warps
+//            on CUDA cores from 16-byte expert loads and rounded once to bf16:
+//            "a linear mixture of n static kernels weighted with their
+//            input-dependent attentions" (KernelWarehouse, abstract), one
+//            kernel per example (CondConv, abstract);
+//   OUTSIDE  the step also runs over the experts and A = alpha_{b,i} E_i: the
+//            sum over experts happens in the accumulator,
+//            y = sum_i alpha_i (x conv W_i) -- the same result by linearity;
+//   PREMIX   A = W_b tile, TMA-loaded from a workspace where the premix kernel
+//            stored every sample's mixed kernel.
+// One thread issues tcgen05.mma (M=128, N<=256 per instruction, K=16) and
+// commits each stage back to its "empty" barrier. The epilogue (8 warps) reads
+// TMEM lane = output channel, adds the mixed bias sum_i alpha_i bias_i, rounds
+// to bf16, transposes through shared memory and writes 16-byte NHWC segments.
 // Every barrier wait is bounded; on expiry the CTA raises an abort flag,
 // records an error word, drains its in-flight TMA / MMA work, frees TMEM and
 // exits.
@@ -47,24 +54,34 @@ enum TcVariant { kFused = 1, kOutside = 2, kPremix = 3 };
 
 struct TcParams {
   int B, H, W, Cin, Cout, KH, KW, pad, n;
-  int R;              // image rows per unit
+  int R;              // output rows per unit
   int tiles_h;        // ceil(H / R)
   int m_tiles;        // ceil(Cout / 128)
-  int n_valid;        // R * W
+  int Wp;             // padded width W + KW - 1
+  int n_virt;         // R * Wp pixels on the padded grid
   int n_mma0, n_mma1; // MMA N of the two column chunks (n_mma1 may be 0)
-  int kc;             // 64-channel chunks per tap: ceil(Cin / 64)
-  int k_steps;        // pipeline steps per unit
-  int stages;
+  int kc;             // 64-channel chunks: ceil(Cin / 64)
+  int spc;            // A steps per chunk: taps (FUSED, PREMIX) or n * taps (OUTSIDE)
+  int k_steps;        // kc * spc
+  int sa, sb;         // A and B pipeline stages
   int b_tile_bytes;   // bytes of one activation stage (1024-aligned)
+  int b_box_rows;     // R + KH - 1
   uint32_t tmem_cols;
+  int desc_base_mode; // 0 (correct on B200); 1 writes (address >> 7) & 7 as base offset
   const __nv_bfloat16* experts;
   const float* alpha;
   const float* bias;  // may be null
   __nv_bfloat16* y;
   int* err;
   long long wait_ns;
-  int inject_skip;    // test hook: withhold the first mixer arrival
+  int inject_skip;    // test hook: withhold the first mixer arrival of CTA 0
 };
+
+__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, int base_mode) {
+  uint64_t d = smem_desc_sw128(saddr);
+  if (base_mode) d |= static_cast<uint64_t>((saddr >> 7) & 7u) << 49;
+  return d;
+}
 
 template <int VARIANT>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -87,17 +104,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t raw = smem_u32(tc_smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* base_ptr = tc_smem_raw + (base - raw);
-  const int S = p.stages;
+  const int SA = p.sa, SB = p.sb;
   const uint32_t a_base = base;
-  const uint32_t b_base = a_base + S * kTcATileBytes;
-  const uint32_t bar_base = b_base + S * p.b_tile_bytes;
-  // barriers: fullA[S], fullB[S], empty[S], accum, drain
+  const uint32_t b_base = a_base + SA * kTcATileBytes;
+  const uint32_t bar_base = b_base + SB * p.b_tile_bytes;
   auto fullA = [&](int s) { return bar_base + 8u * s; };
-  auto fullB = [&](int s) { return bar_base + 8u * (S + s); };
-  auto empty = [&](int s) { return bar_base + 8u * (2 * S + s); };
-  const uint32_t accum_bar = bar_base + 8u * (3 * S);
+  auto emptyA = [&](int s) { return bar_base + 8u * (SA + s); };
+  auto fullB = [&](int s) { return bar_base + 8u * (2 * SA + s); };
+  auto emptyB = [&](int s) { return bar_base + 8u * (2 * SA + SB + s); };
+  const uint32_t accum_bar = bar_base + 8u * (2 * SA + 2 * SB);
   const uint32_t drain_bar = accum_bar + 8u;
-  unsigned char* misc = base_ptr + (bar_base - base) + 8u * (3 * S + 2);
+  unsigned char* misc = base_ptr + (bar_base - base) + 8u * (2 * SA + 2 * SB + 2);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   float* alpha_s = reinterpret_cast<float*>(misc + 16);
@@ -105,17 +122,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < SA; ++s) {
       mbar_init(fullA(s), VARIANT == kPremix ? 1 : kTcMixThreads / 32);
+      mbar_init(emptyA(s), 1);
+    }
+    for (int s = 0; s < SB; ++s) {
       mbar_init(fullB(s), 1);
-      mbar_init(empty(s), 1);
+      mbar_init(emptyB(s), 1);
     }
     mbar_init(accum_bar, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&xmap);
-    if (VARIANT == kPremix) tma_prefetch_desc(&wmap);
+    // The first loads need nothing but the barriers: issue them now so their
+    // latency overlaps the rest of the set-up.
+    const int pre_b = p.kc < SB ? p.kc : SB;
+    for (int cc = 0; cc < pre_b; ++cc) {
+      mbar_arrive_expect_tx(fullB(cc), 64u * 2u * p.Wp * p.b_box_rows);
+      tma_load_4d(b_base + cc * p.b_tile_bytes, &xmap, fullB(cc), cc * 64, -p.pad, h0 - p.pad, b);
+    }
+    if (VARIANT == kPremix) {
+      const int pre_a = p.k_steps < SA ? p.k_steps : SA;
+      for (int k = 0; k < pre_a; ++k) {
+        mbar_arrive_expect_tx(fullA(k), kTcATileBytes);
+        tma_load_3d(a_base + k * kTcATileBytes, &wmap, fullA(k), (k / p.spc) * 64, k % p.spc,
+                    b * p.Cout + m0);
+      }
+    }
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), p.tmem_cols);
@@ -129,67 +162,94 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int taps = p.KH * p.KW;
-  const int steps_per_expert = taps * p.kc;  // OUTSIDE: k = expert * steps_per_expert + kk
 
   if (warp == 0) {
-    // ======================= TMA producer =======================
+    // ======================= activation producer (TMA) =======================
     if (lane == 0) {
-      int issued = 0;
-      for (int k = 0; k < p.k_steps; ++k) {
-        const int s = k % S;
-        const uint32_t ph = static_cast<uint32_t>(k / S) & 1u;
-        if (!wait_bounded(empty(s), ph ^ 1u, ctl, kErrWaitProducer)) break;
-        const int kk = (VARIANT == kOutside) ? k % steps_per_expert : k;
-        const int tap = kk / p.kc, cc = kk % p.kc;
-        const int kh = tap / p.KW, kw = tap % p.KW;
-        mbar_arrive_expect_tx(fullB(s), 64u * 2u * p.W * p.R);
-        tma_load_4d(b_base + s * p.b_tile_bytes, &xmap, fullB(s), cc * 64, kw - p.pad,
-                    h0 + kh - p.pad, b);
-        if (VARIANT == kPremix) {
-          mbar_arrive_expect_tx(fullA(s), kTcATileBytes);
-          tma_load_3d(a_base + s * kTcATileBytes, &wmap, fullA(s), cc * 64, tap,
-                      b * p.Cout + m0);
-        }
+      const int pre_b = p.kc < SB ? p.kc : SB;  // issued during set-up
+      int issued = pre_b;
+      const uint32_t bytes = 64u * 2u * p.Wp * p.b_box_rows;
+      for (int cc = pre_b; cc < p.kc; ++cc) {
+        const int s = cc % SB;
+        const uint32_t ph = static_cast<uint32_t>(cc / SB) & 1u;
+        if (!wait_bounded(emptyB(s), ph ^ 1u, ctl, kErrWaitProducer)) break;
+        mbar_arrive_expect_tx(fullB(s), bytes);
+        tma_load_4d(b_base + s * p.b_tile_bytes, &xmap, fullB(s), cc * 64, -p.pad, h0 - p.pad, b);
         ++issued;
       }
-      // drain: every load issued must land before the CTA may exit
-      for (int j = (issued > S ? issued - S : 0); j < issued; ++j) {
-        const int s = j % S;
-        const uint32_t ph = static_cast<uint32_t>(j / S) & 1u;
-        wait_drain(fullB(s), ph, p.wait_ns, p.err);
-        if (VARIANT == kPremix) wait_drain(fullA(s), ph, p.wait_ns, p.err);
+      for (int j = (issued > SB ? issued - SB : 0); j < issued; ++j)
+        wait_drain(fullB(j % SB), static_cast<uint32_t>(j / SB) & 1u, p.wait_ns, p.err);
+    }
+  } else if (warp == 2) {
+    // ======================= weight producer (PREMIX only) =======================
+    if (VARIANT == kPremix && lane == 0) {
+      const int pre_a = p.k_steps < SA ? p.k_steps : SA;  // issued during set-up
+      int issued = pre_a;
+      for (int k = pre_a; k < p.k_steps; ++k) {
+        const int s = k % SA;
+        const uint32_t ph = static_cast<uint32_t>(k / SA) & 1u;
+        if (!wait_bounded(emptyA(s), ph ^ 1u, ctl, kErrWaitProducer)) break;
+        const int cc = k / p.spc, tap = k % p.spc;
+        mbar_arrive_expect_tx(fullA(s), kTcATileBytes);
+        tma_load_3d(a_base + s * kTcATileBytes, &wmap, fullA(s), cc * 64, tap, b * p.Cout + m0);
+        ++issued;
       }
+      for (int j = (issued > SA ? issued - SA : 0); j < issued; ++j)
+        wait_drain(fullA(j % SA), static_cast<uint32_t>(j / SA) & 1u, p.wait_ns, p.err);
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
+    // The tensor pipe accepts the next MMA only about when it starts the
+    // previous one, so anything this single thread does between two steps
+    // leaves the pipe idle. The loop therefore carries all indices as counters
+    // and builds descriptors by adding offsets to precomputed ones (no
+    // divisions, no tables): start-address fields count 16-byte units.
     if (lane == 0) {
       const uint32_t idesc0 = idesc_bf16_f32(128, p.n_mma0);
       const uint32_t idesc1 = idesc_bf16_f32(128, p.n_mma1 > 0 ? p.n_mma1 : 16);
+      const uint64_t a_desc0 = tc_desc(a_base, 0);
+      const uint64_t b_desc0 = tc_desc(b_base, p.desc_base_mode);
+      const uint64_t b_n1 = static_cast<uint64_t>(p.n_mma0) * 8u;  // n_mma0 rows of 128 B
+      const uint64_t b_stage = static_cast<uint64_t>(p.b_tile_bytes) >> 4;
+      const uint64_t row_skip = static_cast<uint64_t>(p.Wp - p.KW + 1) * 8u;
+      const bool two = p.n_mma1 > 0;
+      uint32_t s = 0, ph = 0, sbi = 0, phb = 0;
+      int t = 0, tap = 0, kw = 0;
+      uint64_t tap_off = 0;  // s_tap * 128 bytes, in 16-byte units
       bool ok = true;
-      int k = 0;
-      for (; k < p.k_steps; ++k) {
-        const int s = k % S;
-        const uint32_t ph = static_cast<uint32_t>(k / S) & 1u;
+      for (int k = 0; k < p.k_steps; ++k) {
+        if (t == 0 && !wait_bounded(fullB(sbi), phb, ctl, kErrWaitMma)) { ok = false; break; }
         if (!wait_bounded(fullA(s), ph, ctl, kErrWaitMma)) { ok = false; break; }
-        if (!wait_bounded(fullB(s), ph, ctl, kErrWaitMma)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a_s = a_base + s * kTcATileBytes;
-        const uint32_t b_s = b_base + s * p.b_tile_bytes;
+        const uint64_t ad = a_desc0 + s * (kTcATileBytes >> 4);
+        const uint64_t bd = b_desc0 + sbi * b_stage + tap_off;
+        const uint32_t acc0 = k > 0 ? 1u : 0u;
+        tc_mma_f16(tmem_base, ad, bd, idesc0, acc0);
+        if (two) tc_mma_f16(tmem_base + p.n_mma0, ad, bd + b_n1, idesc1, acc0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {  // 4 x K=16 per 64-wide stage
-          const uint64_t ad = smem_desc_sw128(a_s + q * 32);
-          const uint32_t acc = (k > 0 || q > 0) ? 1u : 0u;
-          tc_mma_f16(tmem_base, ad, smem_desc_sw128(b_s + q * 32), idesc0, acc);
-          if (p.n_mma1 > 0)
-            tc_mma_f16(tmem_base + p.n_mma0, ad,
-                       smem_desc_sw128(b_s + p.n_mma0 * 128 + q * 32), idesc1, acc);
+        for (int q = 1; q < 4; ++q) {  // K=16 sub-steps: +32 bytes in both operands
+          tc_mma_f16(tmem_base, ad + 2 * q, bd + 2 * q, idesc0, 1u);
+          if (two) tc_mma_f16(tmem_base + p.n_mma0, ad + 2 * q, bd + b_n1 + 2 * q, idesc1, 1u);
         }
-        tc_commit(empty(s));
+        tc_commit(emptyA(s));
+        // advance the tap (kw fastest), the step within the chunk, the stages
+        if (++tap == taps) {
+          tap = 0; kw = 0; tap_off = 0;
+        } else if (++kw == p.KW) {
+          kw = 0; tap_off += row_skip;
+        } else {
+          tap_off += 8u;
+        }
+        if (++t == p.spc) {
+          t = 0;
+          tc_commit(emptyB(sbi));
+          if (++sbi == static_cast<uint32_t>(SB)) { sbi = 0; phb ^= 1u; }
+        }
+        if (++s == static_cast<uint32_t>(SA)) { s = 0; ph ^= 1u; }
       }
       if (ok) {
         tc_commit(accum_bar);
       } else {
-        // drain whatever MMAs were issued before giving up
         tc_commit(drain_bar);
         wait_drain(drain_bar, 0, p.wait_ns, p.err);
       }
@@ -199,31 +259,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ======================= mixers (FUSED / OUTSIDE) =======================
     if (VARIANT != kPremix) {
       const size_t wsize = static_cast<size_t>(p.Cout) * taps * p.Cin;  // one expert
-      bool ok = true;
-      for (int k = 0; k < p.k_steps && ok; ++k) {
-        const int s = k % S;
-        const uint32_t ph = static_cast<uint32_t>(k / S) & 1u;
-        if (!wait_bounded(empty(s), ph ^ 1u, ctl, kErrWaitMixer)) { ok = false; break; }
-        const int kk = (VARIANT == kOutside) ? k % steps_per_expert : k;
-        const int tap = kk / p.kc, cc = kk % p.kc;
+      // this thread's four 16-byte chunks: rows r0 + 32u (u = 0..3), chunk j
+      const int j = mt_id & 7;
+      const int r0 = mt_id >> 3;
+      for (int k = 0; k < p.k_steps; ++k) {
+        const int s = k % SA;
+        const uint32_t ph = static_cast<uint32_t>(k / SA) & 1u;
+        if (!wait_bounded(emptyA(s), ph ^ 1u, ctl, kErrWaitMixer)) break;
+        const int cc = k / p.spc, t = k % p.spc;
+        const int tap = (VARIANT == kOutside) ? t % taps : t;
         const uint32_t a_s = a_base + s * kTcATileBytes;
-        // this thread's four 16-byte chunks: rows r0 + 32u (u = 0..3), chunk j
-        const int j = mt_id & 7;
-        const int r0 = mt_id >> 3;
         const int ci = cc * 64 + j * 8;
         float acc[4][8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int uu = 0; uu < 4; ++uu)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
+          for (int e = 0; e < 8; ++e) acc[uu][e] = 0.f;
         const __nv_bfloat16* src[4];
         bool live[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int co = m0 + r0 + 32 * u;
-          live[u] = co < p.Cout && ci < p.Cin;
-          src[u] = p.experts + (static_cast<size_t>(live[u] ? co : 0) * taps + tap) * p.Cin +
-                   (live[u] ? ci : 0);
+        for (int uu = 0; uu < 4; ++uu) {
+          const int co = m0 + r0 + 32 * uu;
+          live[uu] = co < p.Cout && ci < p.Cin;
+          src[uu] = p.experts + (static_cast<size_t>(live[uu] ? co : 0) * taps + tap) * p.Cin +
+                    (live[uu] ? ci : 0);
         }
         if (VARIANT == kFused) {
           // two experts x four chunks = eight 16-byte loads in flight per thread
@@ -231,46 +290,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const bool two = i + 1 < p.n;
             uint4 v0[4], v1[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              v0[u] = live[u] ? ld_nc_v4(src[u] + i * wsize) : make_uint4(0u, 0u, 0u, 0u);
-              v1[u] = (live[u] && two) ? ld_nc_v4(src[u] + (i + 1) * wsize)
-                                       : make_uint4(0u, 0u, 0u, 0u);
+            for (int uu = 0; uu < 4; ++uu) {
+              v0[uu] = live[uu] ? ld_nc_v4(src[uu] + i * wsize) : make_uint4(0u, 0u, 0u, 0u);
+              v1[uu] = (live[uu] && two) ? ld_nc_v4(src[uu] + (i + 1) * wsize)
+                                         : make_uint4(0u, 0u, 0u, 0u);
             }
             const float a0 = alpha_s[i];
             const float a1 = two ? alpha_s[i + 1] : 0.f;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const uint32_t w0[4] = {v0[u].x, v0[u].y, v0[u].z, v0[u].w};
-              const uint32_t w1[4] = {v1[u].x, v1[u].y, v1[u].z, v1[u].w};
+            for (int uu = 0; uu < 4; ++uu) {
+              const uint32_t w0[4] = {v0[uu].x, v0[uu].y, v0[uu].z, v0[uu].w};
+              const uint32_t w1[4] = {v1[uu].x, v1[uu].y, v1[uu].z, v1[uu].w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                acc[u][2 * e] = fmaf(a0, bf16lo_to_f32(w0[e]), acc[u][2 * e]);
-                acc[u][2 * e + 1] = fmaf(a0, bf16hi_to_f32(w0[e]), acc[u][2 * e + 1]);
-                acc[u][2 * e] = fmaf(a1, bf16lo_to_f32(w1[e]), acc[u][2 * e]);
-                acc[u][2 * e + 1] = fmaf(a1, bf16hi_to_f32(w1[e]), acc[u][2 * e + 1]);
+                acc[uu][2 * e] = fmaf(a0, bf16lo_to_f32(w0[e]), acc[uu][2 * e]);
+                acc[uu][2 * e + 1] = fmaf(a0, bf16hi_to_f32(w0[e]), acc[uu][2 * e + 1]);
+                acc[uu][2 * e] = fmaf(a1, bf16lo_to_f32(w1[e]), acc[uu][2 * e]);
+                acc[uu][2 * e + 1] = fmaf(a1, bf16hi_to_f32(w1[e]), acc[uu][2 * e + 1]);
               }
             }
           }
         } else {  // OUTSIDE: A = alpha_i * W_i for this step's expert i
-          const int i = k / steps_per_expert;
+          const int i = t / taps;
           const float a = alpha_s[i];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 v = live[u] ? ld_nc_v4(src[u] + i * wsize) : make_uint4(0u, 0u, 0u, 0u);
+          for (int uu = 0; uu < 4; ++uu) {
+            const uint4 v = live[uu] ? ld_nc_v4(src[uu] + i * wsize) : make_uint4(0u, 0u, 0u, 0u);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              acc[u][2 * e] = a * bf16lo_to_f32(w[e]);
-              acc[u][2 * e + 1] = a * bf16hi_to_f32(w[e]);
+              acc[uu][2 * e] = a * bf16lo_to_f32(w[e]);
+              acc[uu][2 * e + 1] = a * bf16hi_to_f32(w[e]);
             }
           }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int r = r0 + 32 * u;
+        for (int uu = 0; uu < 4; ++uu) {
+          const int r = r0 + 32 * uu;
           const uint4 packed =
-              make_uint4(pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]),
-                         pack_bf16x2(acc[u][4], acc[u][5]), pack_bf16x2(acc[u][6], acc[u][7]));
+              make_uint4(pack_bf16x2(acc[uu][0], acc[uu][1]), pack_bf16x2(acc[uu][2], acc[uu][3]),
+                         pack_bf16x2(acc[uu][4], acc[uu][5]), pack_bf16x2(acc[uu][6], acc[uu][7]));
           // K-major, 128-byte swizzle: 16-byte chunk j of row r lands at chunk j ^ (r % 8)
           st_shared_v4(a_s + r * 128 + ((j ^ (r & 7)) << 4), packed);
         }
@@ -299,9 +358,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ch * 32, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(r[j]) + bb);
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + j * 64 + lane * 2),
+        for (int jj = 0; jj < 32; ++jj) {
+          const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(r[jj]) + bb);
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + jj * 64 + lane * 2),
                        "h"(*reinterpret_cast<const unsigned short*>(&h))
                        : "memory");
         }
@@ -311,16 +370,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int jj = it * 8 + (lane >> 2);   // pixel within the chunk
           const int part = lane & 3;             // 16-byte part of the 64-byte row
           const int pix = ch * 32 + jj;
-          const int rr = pix / p.W, ww = pix % p.W;
+          const int rr = pix / p.Wp, cw = pix % p.Wp;
           const int oh = h0 + rr;
           const int c8 = m0 + 32 * q + part * 8;
-          if (pix < p.n_valid && oh < p.H && c8 < p.Cout) {
+          if (pix < p.n_virt && cw < p.W && oh < p.H && c8 < p.Cout) {
             uint4 v;
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                          : "r"(stage + jj * 64 + part * 16));
             __nv_bfloat16* dst =
-                p.y + ((static_cast<size_t>(b) * p.H + oh) * p.W + ww) * p.Cout + c8;
+                p.y + ((static_cast<size_t>(b) * p.H + oh) * p.W + cw) * p.Cout + c8;
             *reinterpret_cast<uint4*>(dst) = v;
           }
         }

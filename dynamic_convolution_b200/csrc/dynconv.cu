@@ -42,6 +42,7 @@ DeviceState g_dev[kMaxDevices];
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<long long> g_wait_ns{kDefaultWaitNs};
 std::atomic<int> g_inject_skip{0};
+std::atomic<int> g_route_split{0};  // 0: automatic
 thread_local char g_last_err[256] = "";
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -152,58 +153,71 @@ struct TcPlan {
 
 bool tc_shape_ok(const dynconv_desc* d) {
   return d->dtype == DYNCONV_BF16 && d->groups == 1 && d->stride == 1 && d->C_in % 8 == 0 &&
-         d->C_out % 8 == 0 && d->W <= 256 && d->n <= 1024 &&
+         d->C_out % 8 == 0 && d->W + d->KW - 1 <= 256 && d->KH <= 32 && d->n <= 1024 &&
          out_size(d->H, d->KH, 1, d->pad) == d->H && out_size(d->W, d->KW, 1, d->pad) == d->W;
 }
 
+// Descriptor base-offset mode for shifted activation views (see conv_tc.cuh).
+// 0 is correct on B200: the swizzle is applied on absolute address bits.
+int g_desc_base_mode = 0;
+
 // Build the tensor-core plan for one variant, or return false.
+//
+// Cost model (SM clock cycles of the busiest SM): per A step the MMA takes
+// 2*N_pad cycles (M=128, K=64 at 4096 MAC/clk); producing A costs its L2
+// bytes at ~20 B/clk per SM (the measured share of L2 bandwidth when every
+// SM streams), n*16 KB for FUSED and 16 KB otherwise; the activation tile costs
+// its bytes once per chunk; units run in waves over the SMs.
 bool tc_plan(const dynconv_desc* d, int variant, int sms, int max_smem, TcPlan* out) {
   if (!tc_shape_ok(d)) return false;
   const int taps = d->KH * d->KW;
   const int kc = (d->C_in + 63) / 64;
   const int m_tiles = (d->C_out + 127) / 128;
-  const int steps_conv = taps * kc;
-  const int k_steps = variant == DYNCONV_VARIANT_OUTSIDE ? steps_conv * d->n : steps_conv;
+  const int spc = variant == DYNCONV_VARIANT_OUTSIDE ? taps * d->n : taps;
+  const int k_steps = kc * spc;
+  const int Wp = d->W + d->KW - 1;
+  if (Wp > 256) return false;
+  const int s_tap_max = (d->KH - 1) * Wp + (d->KW - 1);
   bool found = false;
   TcPlan best;
   for (int R = 1; R <= d->H; ++R) {
-    const int n_valid = R * d->W;
-    const int n_pad = (n_valid + 15) / 16 * 16;
+    const int n_virt = R * Wp;
+    const int n_pad = (n_virt + 15) / 16 * 16;
     if (n_pad > 512) break;
-    if (R > 256) break;
+    const int box_rows = R + d->KH - 1;
+    if (box_rows > 256) break;
     int n0 = n_pad, n1 = 0;
     if (n_pad > 256) { n0 = 256; n1 = n_pad - 256; }
-    const int b_tile = (n_pad * 128 + 1023) / 1024 * 1024;
-    const size_t per_stage = dc::kTcATileBytes + b_tile;
+    const int rows = std::max(box_rows * Wp, s_tap_max + n_pad);
+    const int b_tile = (rows * 128 + 1023) / 1024 * 1024;
     const size_t fixed = 1024 /*align slack*/ + 8 * 64 /*barriers*/ + 16 + 4 * d->n + 64;
-    int stages = static_cast<int>((static_cast<size_t>(max_smem) - fixed) / per_stage);
-    stages = std::min(stages, 8);
-    if (stages < 2) continue;
+    const int sb = kc > 1 ? 2 : 1;
+    if (fixed + sb * static_cast<size_t>(b_tile) + 2 * dc::kTcATileBytes > static_cast<size_t>(max_smem))
+      continue;
+    int sa = static_cast<int>((max_smem - fixed - sb * static_cast<size_t>(b_tile)) / dc::kTcATileBytes);
+    sa = std::min(sa, 8);
     const int tiles_h = (d->H + R - 1) / R;
     const long long units = 1LL * d->B * tiles_h * m_tiles;
     const long long waves = (units + sms - 1) / sms;
-    // per-step cycle estimates: MMA 2*n_pad; operand A production; B tile from L2
     const double mma = 2.0 * n_pad;
-    double a_cost;
-    if (variant == DYNCONV_VARIANT_FUSED) a_cost = 256.0 * d->n;     // n x 16 KB of experts
-    else if (variant == DYNCONV_VARIANT_OUTSIDE) a_cost = 256.0;      // one expert tile
-    else a_cost = 256.0;                                              // W_b tile by TMA
-    const double step = std::max(mma, a_cost);
-    const double epilogue = 40.0 * n_pad;
-    const double t_unit = k_steps * step + epilogue + 2000.0;
+    const double a_bytes = variant == DYNCONV_VARIANT_FUSED ? 16384.0 * d->n : 16384.0;
+    const double a_cost = a_bytes / 20.0;
+    const double b_cost = static_cast<double>(box_rows) * Wp * 128.0 / 20.0;
+    const double t_unit = k_steps * std::max(mma, a_cost) + kc * b_cost / 4.0 + 40.0 * n_pad + 3000.0;
     const double cost = waves * t_unit;
     if (!found || cost < best.cost) {
       found = true;
       best.cost = cost;
       best.grid = static_cast<int>(units);
-      best.smem = fixed + stages * per_stage;
+      best.smem = fixed + sb * static_cast<size_t>(b_tile) + sa * static_cast<size_t>(dc::kTcATileBytes);
       dc::TcParams& p = best.p;
       std::memset(&p, 0, sizeof(p));
       p.B = d->B; p.H = d->H; p.W = d->W; p.Cin = d->C_in; p.Cout = d->C_out;
       p.KH = d->KH; p.KW = d->KW; p.pad = d->pad; p.n = d->n;
-      p.R = R; p.tiles_h = tiles_h; p.m_tiles = m_tiles; p.n_valid = n_valid;
-      p.n_mma0 = n0; p.n_mma1 = n1; p.kc = kc; p.k_steps = k_steps; p.stages = stages;
-      p.b_tile_bytes = b_tile;
+      p.R = R; p.tiles_h = tiles_h; p.m_tiles = m_tiles; p.Wp = Wp; p.n_virt = n_virt;
+      p.n_mma0 = n0; p.n_mma1 = n1; p.kc = kc; p.spc = spc; p.k_steps = k_steps;
+      p.sa = sa; p.sb = sb; p.b_tile_bytes = b_tile; p.b_box_rows = box_rows;
+      p.desc_base_mode = g_desc_base_mode;
       uint32_t cols = 32;
       while (cols < static_cast<uint32_t>(n_pad)) cols <<= 1;
       p.tmem_cols = cols;
@@ -261,13 +275,15 @@ int check_launch(const char* what) {
   return DYNCONV_OK;
 }
 
-int encode_x_map(CUtensorMap* map, const void* x, const dynconv_desc* d, int R) {
+// Activations as a 4-D tensor {C_in, W, H, B}; one box = one 64-channel chunk
+// of box_rows input rows at the padded width Wp (zero fill outside the image).
+int encode_x_map(CUtensorMap* map, const void* x, const dynconv_desc* d, int Wp, int box_rows) {
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d->C_in), static_cast<cuuint64_t>(d->W),
                               static_cast<cuuint64_t>(d->H), static_cast<cuuint64_t>(d->B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d->C_in) * 2,
                                  static_cast<cuuint64_t>(d->W) * d->C_in * 2,
                                  static_cast<cuuint64_t>(d->H) * d->W * d->C_in * 2};
-  const cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(d->W), static_cast<cuuint32_t>(R), 1u};
+  const cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(Wp), static_cast<cuuint32_t>(box_rows), 1u};
   const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims,
                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -325,7 +341,7 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   plan.p.inject_skip = g_inject_skip.exchange(0);
   CUtensorMap xmap, wmap;
   std::memset(&wmap, 0, sizeof(wmap));
-  int rc = encode_x_map(&xmap, x, d, plan.p.R);
+  int rc = encode_x_map(&xmap, x, d, plan.p.Wp, plan.p.b_box_rows);
   if (rc) return rc;
   if (variant == DYNCONV_VARIANT_FUSED) return launch_tc<dc::kFused>(plan, xmap, wmap, stream);
   if (variant == DYNCONV_VARIANT_OUTSIDE) return launch_tc<dc::kOutside>(plan, xmap, wmap, stream);
@@ -385,6 +401,16 @@ int dynconv_test_hook(int key, long long value) {
     g_inject_skip.store(value != 0 ? 1 : 0);
     return DYNCONV_OK;
   }
+  if (key == 4) {
+    if (value < 0 || value > 8) return DYNCONV_ERR_INVALID_ARG;
+    g_route_split.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
+  if (key == 3) {
+    if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
+    g_desc_base_mode = static_cast<int>(value);
+    return DYNCONV_OK;
+  }
   return DYNCONV_ERR_INVALID_ARG;
 }
 
@@ -419,14 +445,12 @@ int dynconv_route(const dynconv_desc* desc, const void* x, const float* Wr, cons
   const size_t eb = elem_bytes(desc);
   const bool vec = aligned16(x) && (C * eb) % 16 == 0;
   const int VEC = vec ? static_cast<int>(16 / eb) : 1;
-  const int nv = C / VEC;
-  const int tpp = std::min(nv, dc::kRouteThreads);
-  const int lanes_p = dc::kRouteThreads / tpp;
-  const size_t smem = sizeof(float) * (static_cast<size_t>(lanes_p) * C + 2 * C + desc->n);
   const int HW = desc->H * desc->W;
-  // enough CTAs per sample to keep ~2 CTAs per SM streaming, at most 8 (portable cluster)
-  int nsplit = (2 * st->sms + desc->B - 1) / std::max(desc->B, 1);
+  // about two CTAs per SM in one wave, at most 8 per sample (portable cluster)
+  int nsplit = (2 * st->sms) / std::max(desc->B, 1);
+  if (g_route_split.load() > 0) nsplit = g_route_split.load();
   nsplit = std::max(1, std::min({nsplit, 8, HW}));
+  const size_t smem = sizeof(float) * dc::route_smem_floats(C, desc->n, VEC, nsplit);
 
   dc::RouteParams p{desc->B, C, HW, desc->n, mode, tau, x, Wr, br, alpha};
   cudaLaunchConfig_t cfg = {};
@@ -454,8 +478,10 @@ int dynconv_route(const dynconv_desc* desc, const void* x, const float* Wr, cons
     e = vec ? launch(dc::route_kernel<__nv_bfloat16, 8>) : launch(dc::route_kernel<__nv_bfloat16, 1>);
   else
     e = vec ? launch(dc::route_kernel<float, 4>) : launch(dc::route_kernel<float, 1>);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  if (e != cudaSuccess) return cuda_fail(e, "route_kernel launch");
+  if (e != cudaSuccess) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_fail(e, "route_kernel launch");
+  }
   return check_launch("route_kernel");
 }
 

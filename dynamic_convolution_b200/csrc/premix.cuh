@@ -25,6 +25,7 @@ namespace dc {
 
 constexpr int kPmThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kPmN = 256;         // weights per tile
+constexpr int kPmStageBytes = 32 * kPmN * 2;  // one warp's 32 samples x 256 bf16
 
 __host__ __device__ inline int pm_nk(int n) { return (n + 15) / 16 * 16; }
 __host__ __device__ inline int pm_kcols(int n) { return (pm_nk(n) + 63) / 64; }
@@ -36,7 +37,9 @@ inline bool premix_shape_ok(int B, int n, int Cout, int taps, int Cin) {
   const int m_tiles = (B + 127) / 128;
   const long long a_bytes = 2LL * m_tiles * pm_kcols(n) * 16384;
   const long long stage = 1LL * pm_nk(n) * 512;
-  return a_bytes <= 98304 && a_bytes + 2 * stage <= 200 * 1024;
+  const long long alpha_bytes = 4LL * B * n;  // alpha staged in shared memory
+  return a_bytes <= 65536 && alpha_bytes <= 16384 &&
+         a_bytes + 2 * stage + 4 * kPmStageBytes + alpha_bytes <= 200 * 1024;
 }
 
 struct PmParams {
@@ -72,7 +75,8 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   const int kcols = (p.nk + 63) / 64;
   const uint32_t a_base = base;                         // [m_tile][hi/lo][kcol][128 rows x 128 B]
   const uint32_t e_base = a_base + p.a_bytes;           // [stage][4 atoms][nk rows x 128 B]
-  const uint32_t bar_base = e_base + S * p.stage_bytes;
+  const uint32_t st_base = e_base + S * p.stage_bytes;  // epilogue staging: 4 warps x 16 KB
+  const uint32_t bar_base = st_base + 4 * kPmStageBytes;
   auto full = [&](int s) { return bar_base + 8u * s; };
   auto empty = [&](int s) { return bar_base + 8u * (S + s); };
   auto tfull = [&](int a) { return bar_base + 8u * (2 * S + a); };
@@ -101,18 +105,24 @@ __global__ void __launch_bounds__(kPmThreads, 1)
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), 512);
     tmem_relinquish();
   }
-  // A operands: alpha split into bf16 hi + lo, zero outside [B) x [n)
-  const int a_elems = p.m_tiles * 128 * kcols * 64;
+  // A operands: alpha split into bf16 hi + lo, zero outside [B) x [n).
+  // Stage alpha in shared memory first (all loads in flight at once), then
+  // build both operands from it.
+  float* alpha_s = reinterpret_cast<float*>(misc + 16);
+  const int na = p.B * p.n;
+  for (int e = threadIdx.x; e < na; e += kPmThreads) alpha_s[e] = p.alpha[e];
+  __syncthreads();
+  const int kw64 = kcols * 64;
+  const int a_elems = p.m_tiles * 128 * kw64;
   for (int e = threadIdx.x; e < a_elems; e += kPmThreads) {
-    const int k = e % (kcols * 64);
-    const int m = e / (kcols * 64);  // global sample row
-    const int mt = m / 128, r = m % 128;
-    float a = 0.f;
-    if (m < p.B && k < p.n) a = p.alpha[static_cast<size_t>(m) * p.n + k];
+    const int k = e % kw64;
+    const int m = e / kw64;  // global sample row
+    const int mt = m >> 7, r = m & 127;
+    const float a = (m < p.B && k < p.n) ? alpha_s[m * p.n + k] : 0.f;
     const __nv_bfloat16 hi = __float2bfloat16_rn(a);
     const __nv_bfloat16 lo = __float2bfloat16_rn(a - __bfloat162float(hi));
-    const uint32_t off = static_cast<uint32_t>(k / 64) * 16384u + r * 128u +
-                         ((((k % 64) >> 3) ^ (r & 7)) << 4) + (k & 7) * 2;
+    const uint32_t off = static_cast<uint32_t>(k >> 6) * 16384u + r * 128u +
+                         ((((k & 63) >> 3) ^ (r & 7)) << 4) + (k & 7) * 2;
     const uint32_t hi_addr = a_base + (mt * 2 + 0) * kcols * 16384u + off;
     const uint32_t lo_addr = a_base + (mt * 2 + 1) * kcols * 16384u + off;
     asm volatile("st.shared.b16 [%0], %1;" ::"r"(hi_addr),
@@ -129,14 +139,22 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   const long long my_tiles =
       p.tiles > blockIdx.x ? (p.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
+  // Tile j of this CTA is t = blockIdx.x + j * gridDim.x, i.e. (weight tile
+  // t / m_tiles, sample tile t % m_tiles); every role walks the same sequence
+  // with incremental counters (no 64-bit divisions on the issue paths).
+  const long long ntile0 = blockIdx.x / p.m_tiles;
+  const int mt0 = blockIdx.x % p.m_tiles;
+  const long long dn = gridDim.x / p.m_tiles;
+  const int dm = gridDim.x % p.m_tiles;
+
   if (warp == 0) {
     if (lane == 0) {
       long long issued = 0;
+      long long ntile = ntile0;
+      int mt = mt0;
+      int s = 0;
+      uint32_t ph = 0;
       for (long long j = 0; j < my_tiles; ++j) {
-        const long long t = blockIdx.x + j * gridDim.x;
-        const long long ntile = t / p.m_tiles;
-        const int s = static_cast<int>(j % S);
-        const uint32_t ph = static_cast<uint32_t>((j / S) & 1);
         if (!wait_bounded(empty(s), ph ^ 1u, ctl, kErrWaitProducer)) break;
         mbar_arrive_expect_tx(full(s), static_cast<uint32_t>(p.stage_bytes));
         const uint32_t dst = e_base + s * p.stage_bytes;
@@ -145,6 +163,10 @@ __global__ void __launch_bounds__(kPmThreads, 1)
           tma_load_2d(dst + a * p.nk * 128, &emap, full(s),
                       static_cast<int>(ntile * kPmN + a * 64), 0);
         ++issued;
+        ntile += dn;
+        mt += dm;
+        if (mt >= p.m_tiles) { mt -= p.m_tiles; ++ntile; }
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
       for (long long j = (issued > S ? issued - S : 0); j < issued; ++j)
         wait_drain(full(static_cast<int>(j % S)), static_cast<uint32_t>((j / S) & 1), p.wait_ns,
@@ -154,27 +176,35 @@ __global__ void __launch_bounds__(kPmThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, kPmN) | (1u << 16);  // B is MN-major
       const uint32_t lbo = static_cast<uint32_t>(p.nk) * 128u;
+      const uint64_t e_desc0 = smem_desc_mn_sw128(e_base, lbo);
+      const uint64_t a_desc0 = smem_desc_sw128(a_base);
+      const uint64_t a_half = static_cast<uint64_t>(kcols) * (16384 >> 4);  // hi -> lo
+      const uint64_t stage = static_cast<uint64_t>(p.stage_bytes) >> 4;
+      const int ksteps = p.nk / 16;
+      int mt = mt0;
+      int s = 0;
+      uint32_t ph = 0;
       bool ok = true;
-      for (long long j = 0; j < my_tiles && ok; ++j) {
-        const long long t = blockIdx.x + j * gridDim.x;
-        const int mt = static_cast<int>(t % p.m_tiles);
-        const int s = static_cast<int>(j % S);
+      for (long long j = 0; j < my_tiles; ++j) {
         const int ab = static_cast<int>(j & 1);
-        if (!wait_bounded(full(s), static_cast<uint32_t>((j / S) & 1), ctl, kErrWaitMma)) { ok = false; break; }
+        if (!wait_bounded(full(s), ph, ctl, kErrWaitMma)) { ok = false; break; }
         if (!wait_bounded(tempty(ab), static_cast<uint32_t>((j >> 1) & 1) ^ 1u, ctl, kErrWaitMma)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t e_s = e_base + s * p.stage_bytes;
+        const uint64_t bd = e_desc0 + s * stage;
+        const uint64_t ad = a_desc0 + static_cast<uint64_t>(mt) * 2 * a_half;
         const uint32_t d = tmem_base + ab * kPmN;
-        for (int kk = 0; kk < p.nk / 16; ++kk) {
-          const uint64_t bd = smem_desc_mn_sw128(e_s + kk * 2048, lbo);
-          const uint32_t aoff = static_cast<uint32_t>(kk / 4) * 16384u + (kk % 4) * 32u;
-          const uint64_t ahi = smem_desc_sw128(a_base + (mt * 2 + 0) * kcols * 16384u + aoff);
-          const uint64_t alo = smem_desc_sw128(a_base + (mt * 2 + 1) * kcols * 16384u + aoff);
-          tc_mma_f16(d, ahi, bd, idesc, kk > 0 ? 1u : 0u);
-          tc_mma_f16(d, alo, bd, idesc, 1u);
+        for (int kk = 0; kk < ksteps; ++kk) {
+          // K step kk: 16 expert rows = +2048 bytes of B; A advances 32 bytes within a
+          // 64-wide column, then jumps to the next 16 KB column
+          const uint64_t aoff = static_cast<uint64_t>(kk >> 2) * (16384 >> 4) + (kk & 3) * 2;
+          tc_mma_f16(d, ad + aoff, bd + kk * (2048 >> 4), idesc, kk > 0 ? 1u : 0u);
+          tc_mma_f16(d, ad + a_half + aoff, bd + kk * (2048 >> 4), idesc, 1u);
         }
         tc_commit(empty(s));
         tc_commit(tfull(ab));
+        mt += dm;
+        if (mt >= p.m_tiles) mt -= p.m_tiles;
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
       if (!ok) {
         tc_commit(drain_bar);
@@ -182,41 +212,55 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       }
     }
   } else {
-    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = samples of the tile
+    // Epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 (= 32 samples of the
+    // tile), rounds to bf16 and stages its 32 x 256 block in shared memory with
+    // the 16-byte chunk index XOR-ed by the row, so that the staging writes and
+    // the read-back are both conflict-free; then each store instruction writes
+    // one sample's 512 contiguous bytes (four full lines).
     const int q = warp & 3;
+    const uint32_t stg = st_base + (warp - 2) * kPmStageBytes;
+    long long ntile = ntile0;
+    int mt = mt0;
     for (long long j = 0; j < my_tiles; ++j) {
-      const long long t = blockIdx.x + j * gridDim.x;
-      const long long ntile = t / p.m_tiles;
-      const int mt = static_cast<int>(t % p.m_tiles);
       const int ab = static_cast<int>(j & 1);
       if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j >> 1) & 1), ctl, kErrWaitEpilogue)) break;
       tc_fence_after();
-      const int b = mt * 128 + 32 * q + lane;
-      const long long w0 = ntile * kPmN;
 #pragma unroll 1
       for (int ch = 0; ch < kPmN / 32; ++ch) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * kPmN + ch * 32, r);
         tmem_ld_wait();
-        const long long w = w0 + ch * 32;
-        if (b < p.B && w < p.wsize) {
-          __nv_bfloat16* dst = p.out + static_cast<size_t>(b) * p.wsize + w;
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            if (w + v * 8 < p.wsize) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-              o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-              o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-              o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-              *reinterpret_cast<uint4*>(dst + v * 8) = o;
-            }
-          }
+        for (int v = 0; v < 4; ++v) {
+          uint4 o;
+          o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+          o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+          o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+          o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+          const int c = ch * 4 + v;  // 16-byte chunk of this sample's 512-byte row
+          st_shared_v4(stg + lane * 512 + ((c ^ lane) << 4), o);
         }
       }
+      // TMEM buffer is free once every lane's loads completed
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty(ab));
+      const long long w = ntile * kPmN + lane * 8;
+      const bool wok = w < p.wsize;
+#pragma unroll 4
+      for (int sr = 0; sr < 32; ++sr) {
+        const int b = mt * 128 + 32 * q + sr;
+        uint4 v;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "r"(stg + sr * 512 + ((lane ^ sr) << 4)));
+        if (b < p.B && wok)
+          *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.wsize + w) = v;
+      }
+      __syncwarp();
+      ntile += dn;
+      mt += dm;
+      if (mt >= p.m_tiles) { mt -= p.m_tiles; ++ntile; }
     }
   }
 
@@ -243,7 +287,7 @@ inline int launch_premix(const __nv_bfloat16* experts, const float* alpha, __nv_
   p.tiles = n_tiles * p.m_tiles;
   p.a_bytes = 2 * p.m_tiles * pm_kcols(n) * 16384;
   p.stage_bytes = p.nk * 512;
-  const int budget = 200 * 1024 - p.a_bytes;
+  const int budget = 200 * 1024 - p.a_bytes - 4 * kPmStageBytes - 4 * B * n;
   p.stages = std::min(4, budget / p.stage_bytes);
   if (p.stages < 2) return -3;
   p.alpha = alpha;
@@ -263,7 +307,8 @@ inline int launch_premix(const __nv_bfloat16* experts, const float* alpha, __nv_
   // at least 120 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
   const size_t smem = std::max<size_t>(120 * 1024, 1024 + static_cast<size_t>(p.a_bytes) +
                                                        static_cast<size_t>(p.stages) * p.stage_bytes +
-                                                       8 * (2 * p.stages + 5) + 16);
+                                                       4 * kPmStageBytes + 8 * (2 * p.stages + 5) + 16 +
+                                                       4 * static_cast<size_t>(B) * n);
   if (ensure_smem_fn(premix_kernel, smem) != cudaSuccess) return -1;
   const long long grid = std::min<long long>(p.tiles, sms);
   premix_kernel<<<static_cast<unsigned>(grid), kPmThreads, smem, stream>>>(emap, p);

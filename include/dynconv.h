@@ -157,6 +157,12 @@ unsigned long long dynconv_launch_count(void);
  * (0 restores the default of 500000). key 2: when nonzero, the next forward
  * launch of a tensor-core variant withholds one producer arrival, so that its
  * consumer's bounded wait must expire and report DYNCONV_ERR_TIMEOUT.
+ * key 3: tensor-core descriptor base-offset mode for shifted activation views
+ * (0, the default and the correct choice on B200: left zero; 1: the swizzle
+ * phase (address >> 7) & 7 is written into the descriptor, which gives wrong
+ * results). Only for re-verifying that choice on a device.
+ * key 4: CTAs per sample of the routing kernel's cluster (1..8; 0 restores
+ * the automatic choice), for tuning measurements.
  * Returns DYNCONV_OK or DYNCONV_ERR_INVALID_ARG. */
 int dynconv_test_hook(int key, long long value);
 
