@@ -55,10 +55,8 @@ def parse():
 
 
 def dist_env():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return world, rank, local
+    from dynamic_convolution_b200 import multi
+    return multi.dist_env()
 
 
 def workload_name(cfg) -> str:
@@ -244,7 +242,7 @@ def run_ours(args, cfg):
     import torch.distributed as dist
 
     import dynamic_convolution_b200 as dc
-    from dynamic_convolution_b200 import build, synth
+    from dynamic_convolution_b200 import build, multi, synth
 
     world, rank, local = dist_env()
     if world > 1:
@@ -371,10 +369,7 @@ def run_ours(args, cfg):
     st = dc.dynconv_device_status(stream)
     dc.check(st, "device status after timing")
 
-    t = torch.tensor([total_ms, fwd_ms, route_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_ms, route_ms = t.tolist()
+    total_ms, fwd_ms, route_ms = multi.max_over_ranks([total_ms, fwd_ms, route_ms], device="cuda")
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
     xh = torch.from_numpy(inp.x_store).pin_memory()
@@ -396,11 +391,9 @@ def run_ours(args, cfg):
             yh.copy_(ys[s], non_blocking=True)
         e1.record(stream)
     stream.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
+    e2e_ms = multi.max_over_ranks([e0.elapsed_time(e1)], device="cuda")[0]
     if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_ms = e2e_ms.item()
 
     if rank != 0:
         if world > 1:
@@ -410,8 +403,7 @@ def run_ours(args, cfg):
     del graphs, tails
     peaks, peak_kind = measured_peaks()
     K = args.steps
-    images = world * cfg.B * K
-    value = images / (total_ms / 1e3)
+    value = multi.weak_scaling_rate(cfg.B * K, world, total_ms / 1e3)
     fwd_launch_ms = fwd_ms / K
     route_launch_ms = route_ms / K
     conv_flops = cfg.conv_flops
@@ -457,7 +449,8 @@ def run_ours(args, cfg):
         "forward_eff_tflops": conv_flops / (fwd_launch_ms / 1e3) / 1e12,
         "roofline": roof,
         "cpu_baseline": cpu,
-        "e2e": {"value": world * cfg.B * e2e_steps / (e2e_ms / 1e3), "unit": "images/s",
+        "e2e": {"value": multi.weak_scaling_rate(cfg.B * e2e_steps, world, e2e_ms / 1e3),
+                "unit": "images/s",
                 "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
                 "d2h_bytes_per_step": int(yh.numel() * yh.element_size()),
                 "steps": e2e_steps},

@@ -5,17 +5,22 @@
 // W_b = sum_i alpha_{b,i} W_i (the linear kernel mixture of KernelWarehouse,
 // abstract; per-example kernels of CondConv, abstract).
 //
-// The layer is memory-bound with an ALU floor close to the HBM floor, so the
-// kernel is built to touch each input byte once from HBM and keep the FMA pipe
-// fed:
-//  * one CTA per (sample, block of kRows output rows, 32-channel chunk, column
-//    block); the zero-padded input window (rows + halo) is staged in shared
-//    memory with 16-byte vector loads, so padding costs no branches later;
-//  * the CTA mixes its 32 channels' K*K weights and biases once (fp32);
-//  * each thread owns one channel pair (bf16x2) and one output column, keeps
-//    its 2*K*K weights in registers, and walks down the kRows output rows with
-//    a K-row register window (K new values per row);
-//  * consecutive threads take consecutive channel pairs, so shared-memory reads
+// The layer is memory-bound with an FMA floor close to the HBM floor, so the
+// kernel touches each input byte once from HBM and keeps the FMA pipe fed:
+//  * one CTA per (sample, 32-channel chunk, block of up to kDwMaxRows output
+//    rows, block of output columns); the zero-padded input window is staged
+//    in shared memory by ONE 4-D TMA box {32 channels, cols+K-1, rows+K-1, 1}
+//    whose out-of-bounds fill is the zero padding;
+//  * while the box is in flight the CTA mixes its 32 channels' K*K weights
+//    and biases (fp32), with every expert load of a thread issued at once;
+//  * each thread owns one channel pair (bf16x2) and two adjacent output
+//    columns, keeps its 2*K*K weights in registers and walks down the output
+//    rows with a circular K-row window over K+1 input columns (K+1 new values
+//    per row for two outputs, four independent accumulation chains);
+//  * the channel pair is computed with the packed fp32 instructions of sm_100
+//    (fma.rn.f32x2: two independent fp32 FMAs, each rounded as a scalar FMA),
+//    which halves the instruction count of this issue-bound loop.
+//  * consecutive threads take consecutive channel pairs: shared-memory reads
 //    are conflict-free and the NHWC stores coalesce.
 #pragma once
 
@@ -25,137 +30,177 @@ namespace dc {
 
 constexpr int kDwChunk = 32;       // channels per CTA
 constexpr int kDwPairs = kDwChunk / 2;
-constexpr int kDwRows = 7;         // output rows per CTA
-constexpr int kDwMaxCols = 32;     // output columns per CTA
+constexpr int kDwMaxRows = 28;     // output rows per CTA (at most)
+constexpr int kDwColsPerThread = 2;
+constexpr int kDwMaxColThreads = 16;  // column threads per CTA -> up to 32 output columns
+constexpr int kDwThreads = kDwPairs * kDwMaxColThreads;
 
 struct DwParams {
   int B, C, H, W, pad, n, Ho, Wo;
-  int tile_cols;                   // output columns per CTA (<= kDwMaxCols)
-  const __nv_bfloat16* x;
+  int rows;                        // output rows per CTA
+  int cols;                        // output columns per CTA (<= kDwColsPerThread * kDwMaxColThreads)
+  int col_threads;                 // ceil(cols / kDwColsPerThread)
   const __nv_bfloat16* experts;    // [n][C][K][K][1]
   const float* alpha;
   const float* bias;               // may be null
   __nv_bfloat16* y;
+  int* err;
+  long long wait_ns;
 };
 
 template <int K>
-__global__ void __launch_bounds__(kDwPairs * kDwMaxCols) depthwise_kernel(DwParams p) {
+__global__ void __launch_bounds__(kDwThreads, K <= 5 ? 2 : 1)
+    depthwise_kernel(const __grid_constant__ CUtensorMap xmap, DwParams p) {
   constexpr int KK = K * K;
-  constexpr int TR = kDwRows + K - 1;             // staged input rows
-  const int TC = p.tile_cols + K - 1;             // staged input columns
+  const int TC = ((p.cols + 1) & ~1) + K - 1;      // staged input columns (even column count + halo)
+  const int TR = p.rows + K - 1;                  // staged input rows
   const int b = blockIdx.z;
   const int c0 = blockIdx.y * kDwChunk;
-  const int nrow_blocks = (p.Ho + kDwRows - 1) / kDwRows;
-  const int oh0 = (blockIdx.x % nrow_blocks) * kDwRows;
-  const int ow0 = (blockIdx.x / nrow_blocks) * p.tile_cols;
+  const int nrow_blocks = (p.Ho + p.rows - 1) / p.rows;
+  const int oh0 = (blockIdx.x % nrow_blocks) * p.rows;
+  const int ow0 = (blockIdx.x / nrow_blocks) * p.cols;
   const int t = threadIdx.x;
-  const int nthreads = blockDim.x;
 
-  extern __shared__ __align__(16) unsigned char dw_smem[];
-  float* w_s = reinterpret_cast<float*>(dw_smem);              // [kDwChunk][KK]
-  float* bias_s = w_s + kDwChunk * KK;                          // [kDwChunk]
-  float* alpha_s = bias_s + kDwChunk;                           // [n]
-  uint32_t* tile = reinterpret_cast<uint32_t*>(alpha_s + ((p.n + 3) & ~3));  // [TR][TC][kDwPairs]
+  extern __shared__ __align__(128) unsigned char dw_smem_raw[];
+  // tile first (TMA destination, 128-byte aligned), then the small arrays
+  unsigned char* dw_smem = dw_smem_raw + ((128u - (smem_u32(dw_smem_raw) & 127u)) & 127u);
+  uint32_t* tile = reinterpret_cast<uint32_t*>(dw_smem);                // [TR][TC][kDwPairs]
+  const size_t tile_bytes = static_cast<size_t>(TR) * TC * kDwChunk * 2;
+  float* w_s = reinterpret_cast<float*>(dw_smem + ((tile_bytes + 127) & ~size_t(127)));  // [32][KK]
+  float* bias_s = w_s + kDwChunk * KK;                                  // [32]
+  float* alpha_s = bias_s + kDwChunk;                                   // [n]
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t bar_a = smem_u32(&bar);
+  const WaitCtl ctl{const_cast<volatile int*>(&abort_flag), p.err, p.wait_ns};
 
-  for (int i = t; i < p.n; i += nthreads) alpha_s[i] = p.alpha[static_cast<size_t>(b) * p.n + i];
-
-  // stage the zero-padded input window: 4 x 16-byte vectors per pixel (32 channels)
-  const __nv_bfloat16* xb = p.x + static_cast<size_t>(b) * p.H * p.W * p.C;
-  const int nvec = TR * TC * (kDwChunk / 8);
-  for (int v = t; v < nvec; v += nthreads) {
-    const int q = v & 3;
-    const int pix = v >> 2;
-    const int r = pix / TC, cc = pix % TC;
-    const int ih = oh0 + r - p.pad, iw = ow0 + cc - p.pad;
-    const int ch = c0 + q * 8;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (ih >= 0 && ih < p.H && iw >= 0 && iw < p.W && ch < p.C)
-      val = ld_nc_v4(xb + (static_cast<size_t>(ih) * p.W + iw) * p.C + ch);
-    *reinterpret_cast<uint4*>(tile + (static_cast<size_t>(r) * TC + cc) * kDwPairs + q * 4) = val;
+  if (t == 0) {
+    abort_flag = 0;
+    mbar_init(bar_a, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar_a, static_cast<uint32_t>(tile_bytes));
+    tma_load_4d(smem_u32(tile), &xmap, bar_a, c0, ow0 - p.pad, oh0 - p.pad, b);
   }
+  for (int i = t; i < p.n; i += kDwThreads) alpha_s[i] = p.alpha[static_cast<size_t>(b) * p.n + i];
   __syncthreads();
 
-  // mix this chunk's kernels and biases (fp32)
-  for (int e = t; e < kDwChunk * KK; e += nthreads) {
-    const int cl = e / KK, k = e % KK;
-    const int c = c0 + cl;
-    float s = 0.f;
-    if (c < p.C)
-      for (int i = 0; i < p.n; ++i)
-        s = fmaf(alpha_s[i],
-                 __bfloat162float(p.experts[(static_cast<size_t>(i) * p.C + c) * KK + k]), s);
-    w_s[e] = s;
+  // mix this chunk's kernels and biases (fp32). The loads are the latency
+  // chain of the prologue, so each thread issues the expert values of up to
+  // four weight elements (x 8 experts) before it adds any of them.
+  {
+    constexpr int kE = 4;
+    const size_t es = static_cast<size_t>(p.C) * KK;
+    for (int e0 = t; e0 < kDwChunk * KK; e0 += kE * kDwThreads) {
+      float s[kE];
+      const __nv_bfloat16* src[kE];
+      bool live[kE];
+#pragma unroll
+      for (int u = 0; u < kE; ++u) {
+        const int e = e0 + u * kDwThreads;
+        const int cl = e / KK, k = e - cl * KK;
+        live[u] = e < kDwChunk * KK && c0 + cl < p.C;
+        src[u] = p.experts + static_cast<size_t>(live[u] ? c0 + cl : 0) * KK + (live[u] ? k : 0);
+        s[u] = 0.f;
+      }
+      for (int i = 0; i < p.n; i += 8) {
+        __nv_bfloat16 v[kE][8];
+#pragma unroll
+        for (int u = 0; u < kE; ++u)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            v[u][q] = (live[u] && i + q < p.n) ? src[u][(i + q) * es] : __float2bfloat16_rn(0.f);
+#pragma unroll
+        for (int u = 0; u < kE; ++u)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (i + q < p.n) s[u] = fmaf(alpha_s[i + q], __bfloat162float(v[u][q]), s[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < kE; ++u)
+        if (e0 + u * kDwThreads < kDwChunk * KK) w_s[e0 + u * kDwThreads] = s[u];
+    }
   }
-  for (int cl = t; cl < kDwChunk; cl += nthreads) {
+  if (t < kDwChunk) {
+    const int c = c0 + t;
     float s = 0.f;
-    const int c = c0 + cl;
-    if (p.bias && c < p.C)
-      for (int i = 0; i < p.n; ++i) s = fmaf(alpha_s[i], p.bias[static_cast<size_t>(i) * p.C + c], s);
-    bias_s[cl] = s;
+    if (p.bias && c < p.C) {
+      for (int i = 0; i < p.n; i += 8) {
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = i + q < p.n ? p.bias[static_cast<size_t>(i + q) * p.C + c] : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) if (i + q < p.n) s = fmaf(alpha_s[i + q], v[q], s);
+      }
+    }
+    bias_s[t] = s;
   }
   __syncthreads();
+  const bool tile_ok = wait_bounded(bar_a, 0, ctl, kErrWaitEpilogue);
 
   const int cp = t % kDwPairs;     // channel pair within the chunk
-  const int col = t / kDwPairs;    // output column within the tile
+  const int ct = t / kDwPairs;     // column-pair thread
   const int c = c0 + 2 * cp;
-  const int ow = ow0 + col;
-  if (col >= p.tile_cols || ow >= p.Wo || c >= p.C) return;
+  if (!tile_ok || ct >= p.col_threads || c >= p.C) return;
 
-  float w0[KK], w1[KK];
+  // weights of the channel pair, packed (lo = channel c, hi = channel c+1)
+  uint64_t w2[KK];
 #pragma unroll
-  for (int k = 0; k < KK; ++k) {
-    w0[k] = w_s[(2 * cp) * KK + k];
-    w1[k] = w_s[(2 * cp + 1) * KK + k];
-  }
-  const float bias0 = bias_s[2 * cp], bias1 = bias_s[2 * cp + 1];
+  for (int k = 0; k < KK; ++k) w2[k] = pack_f32x2(w_s[(2 * cp) * KK + k], w_s[(2 * cp + 1) * KK + k]);
+  const uint64_t bias2 = pack_f32x2(bias_s[2 * cp], bias_s[2 * cp + 1]);
+  __nv_bfloat16* yb = p.y + static_cast<size_t>(b) * p.Ho * p.Wo * p.C;
 
-  // K-row register window of the input columns col .. col+K-1
-  float win0[K][K], win1[K][K];
+  // this thread's two adjacent output columns
+  const int col = 2 * ct;
+  const int ow = ow0 + col;
+  const uint32_t* tcol = tile + static_cast<size_t>(col) * kDwPairs + cp;
+  const size_t row_stride = static_cast<size_t>(TC) * kDwPairs;
+  // circular K-row window over the K+1 input columns col .. col+K: input row r
+  // lives in slot r % K. Rows are walked in groups of K with the group body
+  // unrolled, so every slot index is a compile-time constant and the window
+  // never moves between registers.
+  uint64_t win[K][K + 1];
 #pragma unroll
   for (int r = 0; r < K - 1; ++r)
 #pragma unroll
-    for (int kw = 0; kw < K; ++kw) {
-      const uint32_t v = tile[(static_cast<size_t>(r) * TC + col + kw) * kDwPairs + cp];
-      win0[r + 1][kw] = bf16lo_to_f32(v);
-      win1[r + 1][kw] = bf16hi_to_f32(v);
-    }
-
-  __nv_bfloat16* yb = p.y + static_cast<size_t>(b) * p.Ho * p.Wo * p.C;
+    for (int kw = 0; kw <= K; ++kw) win[r][kw] = bf16x2_to_f32x2(tcol[r * row_stride + kw * kDwPairs]);
+#pragma unroll 1
+  for (int g = 0; g < p.rows; g += K) {
 #pragma unroll
-  for (int orow = 0; orow < kDwRows; ++orow) {
-    // slide: drop the top row, load input row orow+K-1
+    for (int j = 0; j < K; ++j) {
+      const int orow = g + j;
+      if (orow >= p.rows) break;
+      const int in_row = orow + K - 1;
 #pragma unroll
-    for (int r = 0; r < K - 1; ++r)
+      for (int kw = 0; kw <= K; ++kw)
+        win[(j + K - 1) % K][kw] = bf16x2_to_f32x2(tcol[in_row * row_stride + kw * kDwPairs]);
+      // four independent chains: two columns x (even, odd kernel rows)
+      uint64_t e0 = bias2, o0 = 0ull, e1 = bias2, o1 = 0ull;
 #pragma unroll
-      for (int kw = 0; kw < K; ++kw) {
-        win0[r][kw] = win0[r + 1][kw];
-        win1[r][kw] = win1[r + 1][kw];
-      }
+      for (int kh = 0; kh < K; ++kh)
 #pragma unroll
-    for (int kw = 0; kw < K; ++kw) {
-      const uint32_t v =
-          tile[(static_cast<size_t>(orow + K - 1) * TC + col + kw) * kDwPairs + cp];
-      win0[K - 1][kw] = bf16lo_to_f32(v);
-      win1[K - 1][kw] = bf16hi_to_f32(v);
-    }
-    // two partial sums per channel for more independent FMA chains
-    float a0 = bias0, a1 = bias1, e0 = 0.f, e1 = 0.f;
-#pragma unroll
-    for (int kh = 0; kh < K; ++kh)
-#pragma unroll
-      for (int kw = 0; kw < K; ++kw) {
-        if (kh & 1) {
-          e0 = fmaf(win0[kh][kw], w0[kh * K + kw], e0);
-          e1 = fmaf(win1[kh][kw], w1[kh * K + kw], e1);
-        } else {
-          a0 = fmaf(win0[kh][kw], w0[kh * K + kw], a0);
-          a1 = fmaf(win1[kh][kw], w1[kh * K + kw], a1);
+        for (int kw = 0; kw < K; ++kw) {
+          const uint64_t w = w2[kh * K + kw];
+          if (kh & 1) {
+            o0 = ffma2(win[(j + kh) % K][kw], w, o0);
+            o1 = ffma2(win[(j + kh) % K][kw + 1], w, o1);
+          } else {
+            e0 = ffma2(win[(j + kh) % K][kw], w, e0);
+            e1 = ffma2(win[(j + kh) % K][kw + 1], w, e1);
+          }
         }
+      const uint64_t s0 = fadd2(e0, o0), s1 = fadd2(e1, o1);
+      const int oh = oh0 + orow;
+      if (oh < p.Ho) {
+        __nv_bfloat16* dst = yb + (static_cast<size_t>(oh) * p.Wo + ow) * p.C + c;
+        if (col < p.cols && ow < p.Wo)
+          *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(__uint_as_float(static_cast<uint32_t>(s0)),
+                                                          __uint_as_float(static_cast<uint32_t>(s0 >> 32)));
+        if (col + 1 < p.cols && ow + 1 < p.Wo)
+          *reinterpret_cast<uint32_t*>(dst + p.C) =
+              pack_bf16x2(__uint_as_float(static_cast<uint32_t>(s1)),
+                          __uint_as_float(static_cast<uint32_t>(s1 >> 32)));
       }
-    const int oh = oh0 + orow;
-    if (oh < p.Ho)
-      *reinterpret_cast<uint32_t*>(yb + (static_cast<size_t>(oh) * p.Wo + ow) * p.C + c) =
-          pack_bf16x2(a0 + e0, a1 + e1);
+    }
   }
 }
 

@@ -231,7 +231,8 @@ bool tc_plan(const dynconv_desc* d, int variant, int sms, int max_smem, TcPlan* 
 bool depthwise_ok(const dynconv_desc* d) {
   return d->dtype == DYNCONV_BF16 && d->groups == d->C_in && d->C_in == d->C_out &&
          d->stride == 1 && d->KH == d->KW && (d->KH == 3 || d->KH == 5 || d->KH == 7) &&
-         d->C_in % 8 == 0 && d->n <= 4096;
+         d->C_in % 8 == 0 && d->n <= 4096 && out_size(d->H, d->KH, 1, d->pad) >= 1 &&
+         out_size(d->W, d->KW, 1, d->pad) >= 1;
 }
 
 size_t premix_workspace(const dynconv_desc* d) {
@@ -513,29 +514,48 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
       if (!depthwise_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
       if (!aligned16(x) || !aligned16(y)) return DYNCONV_ERR_MISALIGNED;
       dc::DwParams p{};
+      const int K = desc->KH;
       p.B = desc->B; p.C = desc->C_in; p.H = desc->H; p.W = desc->W; p.pad = desc->pad;
       p.n = desc->n;
-      p.Ho = out_size(desc->H, desc->KH, 1, desc->pad);
-      p.Wo = out_size(desc->W, desc->KW, 1, desc->pad);
-      p.tile_cols = std::min(p.Wo, dc::kDwMaxCols);
-      p.x = static_cast<const __nv_bfloat16*>(x);
+      p.Ho = out_size(desc->H, K, 1, desc->pad);
+      p.Wo = out_size(desc->W, K, 1, desc->pad);
+      p.rows = std::min(p.Ho, dc::kDwMaxRows);
+      p.cols = std::min(p.Wo, dc::kDwColsPerThread * dc::kDwMaxColThreads);
+      p.col_threads = (p.cols + dc::kDwColsPerThread - 1) / dc::kDwColsPerThread;
       p.experts = static_cast<const __nv_bfloat16*>(experts);
       p.alpha = alpha;
       p.bias = bias;
       p.y = static_cast<__nv_bfloat16*>(y);
-      const int K = desc->KH;
-      const int TC = p.tile_cols + K - 1, TR = dc::kDwRows + K - 1;
-      const size_t smem = sizeof(float) * (dc::kDwChunk * K * K + dc::kDwChunk + ((p.n + 3) & ~3)) +
-                          static_cast<size_t>(TR) * TC * dc::kDwChunk * 2;
+      p.err = st->err;
+      p.wait_ns = g_wait_ns.load();
+      const int TC = ((p.cols + 1) & ~1) + K - 1, TR = p.rows + K - 1;
+      const size_t tile_bytes = static_cast<size_t>(TR) * TC * dc::kDwChunk * 2;
+      const size_t smem = 128 + ((tile_bytes + 127) & ~size_t(127)) +
+                          sizeof(float) * (dc::kDwChunk * K * K + dc::kDwChunk + p.n);
       if (smem > static_cast<size_t>(st->max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
-      const int row_blocks = (p.Ho + dc::kDwRows - 1) / dc::kDwRows;
-      const int col_blocks = (p.Wo + p.tile_cols - 1) / p.tile_cols;
+      // activations {C, W, H, B}; one box = 32 channels of the zero-padded window
+      CUtensorMap xmap;
+      const cuuint64_t dims[4] = {static_cast<cuuint64_t>(desc->C_in), static_cast<cuuint64_t>(desc->W),
+                                  static_cast<cuuint64_t>(desc->H), static_cast<cuuint64_t>(desc->B)};
+      const cuuint64_t strides[3] = {static_cast<cuuint64_t>(desc->C_in) * 2,
+                                     static_cast<cuuint64_t>(desc->W) * desc->C_in * 2,
+                                     static_cast<cuuint64_t>(desc->H) * desc->W * desc->C_in * 2};
+      const cuuint32_t box[4] = {static_cast<cuuint32_t>(dc::kDwChunk), static_cast<cuuint32_t>(TC),
+                                 static_cast<cuuint32_t>(TR), 1u};
+      const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+      if (g_encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(depthwise) failed");
+        return DYNCONV_ERR_CUDA;
+      }
+      const int row_blocks = (p.Ho + p.rows - 1) / p.rows;
+      const int col_blocks = (p.Wo + p.cols - 1) / p.cols;
       dim3 grid(row_blocks * col_blocks, (desc->C_in + dc::kDwChunk - 1) / dc::kDwChunk, desc->B);
-      dim3 block(dc::kDwPairs * p.tile_cols);
       auto go = [&](auto kern) -> int {
         cudaError_t e = ensure_smem(kern, smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(depthwise)");
-        kern<<<grid, block, smem, s>>>(p);
+        kern<<<grid, dc::kDwThreads, smem, s>>>(xmap, p);
         return check_launch("depthwise_kernel");
       };
       if (K == 3) return go(dc::depthwise_kernel<3>);

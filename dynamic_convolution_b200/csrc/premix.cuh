@@ -112,13 +112,14 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   const int na = p.B * p.n;
   for (int e = threadIdx.x; e < na; e += kPmThreads) alpha_s[e] = p.alpha[e];
   __syncthreads();
-  const int kw64 = kcols * 64;
-  const int a_elems = p.m_tiles * 128 * kw64;
-  for (int e = threadIdx.x; e < a_elems; e += kPmThreads) {
-    const int k = e % kw64;
-    const int m = e / kw64;  // global sample row
+  // zero both operands with 16-byte stores, then place the B*n live values
+  for (int e = threadIdx.x; e < p.a_bytes / 16; e += kPmThreads)
+    st_shared_v4(a_base + e * 16, make_uint4(0u, 0u, 0u, 0u));
+  __syncthreads();
+  for (int e = threadIdx.x; e < na; e += kPmThreads) {
+    const int m = e / p.n, k = e - m * p.n;  // sample row, expert
     const int mt = m >> 7, r = m & 127;
-    const float a = (m < p.B && k < p.n) ? alpha_s[m * p.n + k] : 0.f;
+    const float a = alpha_s[e];
     const __nv_bfloat16 hi = __float2bfloat16_rn(a);
     const __nv_bfloat16 lo = __float2bfloat16_rn(a - __bfloat162float(hi));
     const uint32_t off = static_cast<uint32_t>(k >> 6) * 16384u + r * 128u +
