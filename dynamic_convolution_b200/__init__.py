@@ -24,7 +24,8 @@ VARIANT_NAMES = {0: "auto", 1: "fused", 2: "outside", 3: "premix", 4: "direct", 
 OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = -1, -2, -3, -4, -5, -6
 
-SYMBOLS = ("dynconv_route", "dynconv_forward", "dynconv_workspace_size", "dynconv_select_variant",
+SYMBOLS = ("dynconv_route", "dynconv_forward", "dynconv_forward_noalloc",
+           "dynconv_workspace_size", "dynconv_select_variant",
            "dynconv_status_string", "dynconv_last_error", "dynconv_device_status",
            "dynconv_launch_count", "dynconv_test_hook")
 
@@ -58,6 +59,8 @@ def load():
         lib.dynconv_route.restype = ctypes.c_int
         lib.dynconv_forward.argtypes = [D, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.dynconv_forward.restype = ctypes.c_int
+        lib.dynconv_forward_noalloc.argtypes = [D, P, P, P, P, P, P]
+        lib.dynconv_forward_noalloc.restype = ctypes.c_int
         lib.dynconv_workspace_size.argtypes = [D]
         lib.dynconv_workspace_size.restype = ctypes.c_size_t
         lib.dynconv_select_variant.argtypes = [D, ctypes.c_size_t]
@@ -113,6 +116,17 @@ def dynconv_forward(desc, x, experts, alpha, bias, y, workspace=None, workspace_
     return load().dynconv_forward(ctypes.byref(desc), _ptr(x), _ptr(experts), _ptr(alpha),
                                   _ptr(bias), _ptr(y), _ptr(workspace), int(workspace_bytes),
                                   _stream(stream))
+
+
+# Bytes of the library's built-in scratch array (DYNCONV_NOALLOC_MAX_BYTES).
+NOALLOC_MAX_BYTES = 32 * 1024 * 1024
+
+
+def dynconv_forward_noalloc(desc, x, experts, alpha, bias, y, stream=None) -> int:
+    """dynconv_forward (PREMIX variant) with the library's built-in scratch array
+    instead of a caller workspace; for callers that cannot allocate device memory."""
+    return load().dynconv_forward_noalloc(ctypes.byref(desc), _ptr(x), _ptr(experts), _ptr(alpha),
+                                          _ptr(bias), _ptr(y), _stream(stream))
 
 
 def dynconv_workspace_size(desc) -> int:

@@ -26,6 +26,12 @@ namespace {
 // One error word per device (module globals are instantiated per device).
 __device__ int g_device_err;
 
+// Scratch of dynconv_forward_noalloc: a fixed array in device memory, one per
+// device that loads this module. In host code its name is only a stand-in, not
+// a device address: dynconv_forward_noalloc looks the address up on its first
+// call on each device and keeps it in g_noalloc_ptr.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DYNCONV_NOALLOC_MAX_BYTES];
+
 constexpr long long kDefaultWaitNs = 500LL * 1000 * 1000;  // 0.5 s
 constexpr int kMaxDevices = 64;
 
@@ -39,6 +45,8 @@ struct DeviceState {
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<long long> g_wait_ns{kDefaultWaitNs};
 std::atomic<int> g_inject_skip{0};
@@ -592,6 +600,47 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
     default:
       return DYNCONV_ERR_INVALID_ARG;
   }
+}
+
+int dynconv_forward_noalloc(const dynconv_desc* desc, const void* x, const void* experts,
+                            const float* alpha, const float* bias, void* y, void* stream) {
+  int rc = validate_desc(desc);
+  if (rc) return rc;
+  if (!x || !experts || !alpha || !y) return DYNCONV_ERR_INVALID_ARG;
+  if (desc->B == 0) return DYNCONV_OK;
+  dynconv_desc d = *desc;
+  d.variant = DYNCONV_VARIANT_PREMIX;
+  if (!tc_shape_ok(&d)) return DYNCONV_ERR_UNSUPPORTED;
+  const size_t need = premix_workspace(&d);
+  if (need == 0) return DYNCONV_ERR_UNSUPPORTED;
+  if (need > DYNCONV_NOALLOC_MAX_BYTES) {
+    std::snprintf(g_last_err, sizeof(g_last_err),
+                  "shape needs %zu bytes of scratch; the built-in array holds %u", need,
+                  DYNCONV_NOALLOC_MAX_BYTES);
+    return DYNCONV_ERR_WORKSPACE;
+  }
+  if (!aligned16(x) || !aligned16(experts) || !aligned16(y)) return DYNCONV_ERR_MISALIGNED;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc) return rc;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  void* scratch = nullptr;
+  {
+    // first call on this device (which is current): look the array's address up
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      e = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+      if (e != cudaSuccess) {
+        g_noalloc_ptr[dev] = nullptr;
+        return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+      }
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return run_tc(&d, DYNCONV_VARIANT_PREMIX, st, x, experts, alpha, bias, y, scratch,
+                DYNCONV_NOALLOC_MAX_BYTES, static_cast<cudaStream_t>(stream));
 }
 
 int dynconv_device_status(void* stream) {

@@ -127,6 +127,40 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
                     const float* alpha, const float* bias, void* y, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* ---- forward without caller-provided scratch ----------------------------
+ * The pages describe no such entry point; it has no counterpart in the method.
+ *
+ * For callers that cannot allocate device memory where they call the layer:
+ * for example a plugin or callback run by a host framework that owns all
+ * device memory and hands out no workspace, or code that must not call
+ * cudaMalloc after start-up (cudaMalloc synchronises the device and can fail
+ * once memory is committed). It computes exactly what dynconv_forward with the
+ * PREMIX variant computes (tensor-core kernel mixing, then the tensor-core
+ * convolution), but its scratch is a fixed array that the library itself
+ * defines in device memory: DYNCONV_NOALLOC_MAX_BYTES bytes, reserved on every
+ * GPU on which the library's kernels are loaded, for the life of the process.
+ *
+ *   desc, x, experts, alpha, bias, y, stream: as for dynconv_forward (bf16,
+ *   dense, stride 1, "same" padding; desc->variant is ignored).
+ * Limit: the shape must fit, dynconv_workspace_size(desc) <= DYNCONV_NOALLOC_MAX_BYTES;
+ * larger shapes are rejected with DYNCONV_ERR_WORKSPACE before anything runs
+ * (for example B=64, 128->128 channels, 3x3 needs 18.9 MB and fits; B=256,
+ * 256->256, 3x3 needs 302 MB and does not).
+ * Set-up: this entry point's first call on a device, made with that device
+ * current, looks up the array's device address (and, like every entry point's
+ * first call, queries the device); make that first call before any stream
+ * capture.
+ * Shared state: every call uses the same array, which keeps the last call's
+ * contents. Nothing has to start at zero (the mixing kernel writes every
+ * element the convolution reads), but two calls whose kernels overlap on the
+ * GPU (different streams or host threads without ordering) race on the array:
+ * order them (same stream, or events).
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, MISALIGNED, CUDA. */
+#define DYNCONV_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
+int dynconv_forward_noalloc(const dynconv_desc* desc, const void* x, const void* experts,
+                            const float* alpha, const float* bias, void* y, void* stream);
+
 /* Bytes of workspace the PREMIX variant needs for this descriptor (0 if it
  * cannot run this shape). Pure host function. */
 size_t dynconv_workspace_size(const dynconv_desc* desc);
