@@ -51,6 +51,9 @@ def parse():
                     choices=["auto", "fused", "outside", "premix", "direct", "depthwise"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--hooks", default="",
+                    help="implementation knobs for comparisons, e.g. '6=0,5=0' "
+                         "(see dynconv_test_hook in include/dynconv.h)")
     return ap.parse_args()
 
 
@@ -257,6 +260,11 @@ def run_ours(args, cfg):
 
     variant = {"auto": 0, "fused": 1, "outside": 2, "premix": 3, "direct": 4,
                "depthwise": 5}[args.variant]
+    hooks = {}
+    for kv in filter(None, args.hooks.split(",")):
+        k, v = kv.split("=")
+        hooks[int(k)] = int(v)
+        dc.check(dc.dynconv_test_hook(int(k), int(v)), f"test hook {kv}")
     inp = synth.make_inputs(cfg, seed=rank)
     desc = dc.desc_from_config(cfg, variant)
     tdt = torch.bfloat16 if cfg.dtype == synth.BF16 else torch.float32
@@ -457,6 +465,7 @@ def run_ours(args, cfg):
         "gpu_launches": int(round(launches_per_step * K)),
         "clocks": clocks,
         "source_hash": src_hash,
+        "hooks": hooks or None,
     }
     print(json.dumps(line), flush=True)
     if world > 1:

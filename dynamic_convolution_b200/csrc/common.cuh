@@ -17,6 +17,7 @@ enum : int {
   kErrWaitMixer = 0x103,
   kErrWaitEpilogue = 0x104,
   kErrWaitDrain = 0x105,
+  kErrWaitGrid = 0x106,
 };
 
 struct WaitCtl {

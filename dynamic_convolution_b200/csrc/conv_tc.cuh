@@ -121,6 +121,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
 
+  // Everything above this line is set-up that reads no global memory; with a
+  // programmatic launch edge it overlaps the tail of the previous kernel.
+  if (warp == 0) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), p.tmem_cols);
+    tmem_relinquish();
+  }
+  grid_dependency_wait();
   if (threadIdx.x == 0) {
     for (int s = 0; s < SA; ++s) {
       mbar_init(fullA(s), VARIANT == kPremix ? 1 : kTcMixThreads / 32);
@@ -150,12 +157,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), p.tmem_cols);
-    tmem_relinquish();
-  }
-  for (int i = threadIdx.x; i < p.n; i += kTcThreads)
-    alpha_s[i] = p.alpha[static_cast<size_t>(b) * p.n + i];
+  if (VARIANT != kPremix)  // PREMIX needs alpha only for the bias, in the epilogue
+    for (int i = threadIdx.x; i < p.n; i += kTcThreads)
+      alpha_s[i] = p.alpha[static_cast<size_t>(b) * p.n + i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -216,23 +220,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t s = 0, ph = 0, sbi = 0, phb = 0;
       int t = 0, tap = 0, kw = 0;
       uint64_t tap_off = 0;  // s_tap * 128 bytes, in 16-byte units
-      bool ok = true;
-      for (int k = 0; k < p.k_steps; ++k) {
-        if (t == 0 && !wait_bounded(fullB(sbi), phb, ctl, kErrWaitMma)) { ok = false; break; }
-        if (!wait_bounded(fullA(s), ph, ctl, kErrWaitMma)) { ok = false; break; }
-        tc_fence_after();
+      // The operands of step k+1 are waited for before the last two MMAs of
+      // step k are issued, so that the barrier probes and the fence overlap
+      // MMAs already queued in the tensor pipe.
+      bool ok = p.k_steps > 0 && wait_bounded(fullB(0), 0, ctl, kErrWaitMma) &&
+                wait_bounded(fullA(0), 0, ctl, kErrWaitMma);
+      if (ok) tc_fence_after();
+      for (int k = 0; k < p.k_steps && ok; ++k) {
         const uint64_t ad = a_desc0 + s * (kTcATileBytes >> 4);
         const uint64_t bd = b_desc0 + sbi * b_stage + tap_off;
         const uint32_t acc0 = k > 0 ? 1u : 0u;
         tc_mma_f16(tmem_base, ad, bd, idesc0, acc0);
         if (two) tc_mma_f16(tmem_base + p.n_mma0, ad, bd + b_n1, idesc1, acc0);
 #pragma unroll
-        for (int q = 1; q < 4; ++q) {  // K=16 sub-steps: +32 bytes in both operands
+        for (int q = 1; q < 3; ++q) {  // K=16 sub-steps: +32 bytes in both operands
           tc_mma_f16(tmem_base, ad + 2 * q, bd + 2 * q, idesc0, 1u);
           if (two) tc_mma_f16(tmem_base + p.n_mma0, ad + 2 * q, bd + b_n1 + 2 * q, idesc1, 1u);
         }
-        tc_commit(emptyA(s));
         // advance the tap (kw fastest), the step within the chunk, the stages
+        const uint32_t s_cur = s, sbi_cur = sbi;
+        bool chunk_end = false;
         if (++tap == taps) {
           tap = 0; kw = 0; tap_off = 0;
         } else if (++kw == p.KW) {
@@ -242,10 +249,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (++t == p.spc) {
           t = 0;
-          tc_commit(emptyB(sbi));
+          chunk_end = true;
           if (++sbi == static_cast<uint32_t>(SB)) { sbi = 0; phb ^= 1u; }
         }
         if (++s == static_cast<uint32_t>(SA)) { s = 0; ph ^= 1u; }
+        // operands of the next step
+        if (k + 1 < p.k_steps) {
+          if (chunk_end && !wait_bounded(fullB(sbi), phb, ctl, kErrWaitMma)) ok = false;
+          if (ok && !wait_bounded(fullA(s), ph, ctl, kErrWaitMma)) ok = false;
+          if (ok) tc_fence_after();
+        }
+        tc_mma_f16(tmem_base, ad + 6, bd + 6, idesc0, 1u);
+        if (two) tc_mma_f16(tmem_base + p.n_mma0, ad + 6, bd + b_n1 + 6, idesc1, 1u);
+        tc_commit(emptyA(s_cur));
+        if (chunk_end) tc_commit(emptyB(sbi_cur));
       }
       if (ok) {
         tc_commit(accum_bar);
@@ -345,8 +362,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int half = (warp - kTcMixWarp0) >> 2;  // column half
     const int co = m0 + 32 * q + lane;
     float bb = 0.f;
-    if (p.bias != nullptr && co < p.Cout)
-      for (int i = 0; i < p.n; ++i) bb = fmaf(alpha_s[i], p.bias[static_cast<size_t>(i) * p.Cout + co], bb);
+    if (p.bias != nullptr && co < p.Cout) {
+      const float* ab = VARIANT == kPremix ? p.alpha + static_cast<size_t>(b) * p.n : alpha_s;
+      for (int i = 0; i < p.n; ++i) bb = fmaf(ab[i], p.bias[static_cast<size_t>(i) * p.Cout + co], bb);
+    }
     if (wait_bounded(accum_bar, 0, ctl, kErrWaitEpilogue)) {
       tc_fence_after();
       // per-warp 32 px x 32 co bf16 staging tile in the (now idle) A stage buffers

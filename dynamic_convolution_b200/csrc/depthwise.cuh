@@ -16,7 +16,8 @@
 //  * each thread owns one channel pair (bf16x2) and two adjacent output
 //    columns, keeps its 2*K*K weights in registers and walks down the output
 //    rows with a circular K-row window over K+1 input columns (K+1 new values
-//    per row for two outputs, four independent accumulation chains);
+//    per row for two outputs, six independent accumulation chains visited
+//    in rotation, so the packed-FMA latency never stalls a warp);
 //  * the channel pair is computed with the packed fp32 instructions of sm_100
 //    (fma.rn.f32x2: two independent fp32 FMAs, each rounded as a scalar FMA),
 //    which halves the instruction count of this issue-bound loop.
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(kDwThreads, K <= 5 ? 2 : 1)
   const uint32_t bar_a = smem_u32(&bar);
   const WaitCtl ctl{const_cast<volatile int*>(&abort_flag), p.err, p.wait_ns};
 
+  grid_dependency_wait();  // alpha (and possibly x) come from earlier kernels
   if (t == 0) {
     abort_flag = 0;
     mbar_init(bar_a, 1);
@@ -173,22 +175,19 @@ __global__ void __launch_bounds__(kDwThreads, K <= 5 ? 2 : 1)
 #pragma unroll
       for (int kw = 0; kw <= K; ++kw)
         win[(j + K - 1) % K][kw] = bf16x2_to_f32x2(tcol[in_row * row_stride + kw * kDwPairs]);
-      // four independent chains: two columns x (even, odd kernel rows)
-      uint64_t e0 = bias2, o0 = 0ull, e1 = bias2, o1 = 0ull;
+      // six independent chains (kernel row mod 3, two columns), visited in
+      // rotation so that consecutive FMAs never depend on each other
+      uint64_t acc[3][2] = {{bias2, bias2}, {0ull, 0ull}, {0ull, 0ull}};
 #pragma unroll
-      for (int kh = 0; kh < K; ++kh)
+      for (int kw = 0; kw < K; ++kw)
 #pragma unroll
-        for (int kw = 0; kw < K; ++kw) {
+        for (int kh = 0; kh < K; ++kh) {
           const uint64_t w = w2[kh * K + kw];
-          if (kh & 1) {
-            o0 = ffma2(win[(j + kh) % K][kw], w, o0);
-            o1 = ffma2(win[(j + kh) % K][kw + 1], w, o1);
-          } else {
-            e0 = ffma2(win[(j + kh) % K][kw], w, e0);
-            e1 = ffma2(win[(j + kh) % K][kw + 1], w, e1);
-          }
+          acc[kh % 3][0] = ffma2(win[(j + kh) % K][kw], w, acc[kh % 3][0]);
+          acc[kh % 3][1] = ffma2(win[(j + kh) % K][kw + 1], w, acc[kh % 3][1]);
         }
-      const uint64_t s0 = fadd2(e0, o0), s1 = fadd2(e1, o1);
+      const uint64_t s0 = fadd2(fadd2(acc[0][0], acc[1][0]), acc[2][0]);
+      const uint64_t s1 = fadd2(fadd2(acc[0][1], acc[1][1]), acc[2][1]);
       const int oh = oh0 + orow;
       if (oh < p.Ho) {
         __nv_bfloat16* dst = yb + (static_cast<size_t>(oh) * p.Wo + ow) * p.C + c;

@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(kDirectThreads) direct_conv_kernel(DirectParam
   const int taps = p.KH * p.KW;
   const int wrow = taps * Cg;  // weights per output channel
 
+  grid_dependency_wait();  // alpha (and possibly x) come from earlier kernels
   float* alpha_s = dsm;                     // [n]
   float* bias_s = alpha_s + p.n;            // [cob]
   float* w_s = bias_s + p.cob;              // [cob][KH][KW][Cg]

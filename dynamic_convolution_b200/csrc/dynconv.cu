@@ -19,6 +19,7 @@
 #include "depthwise.cuh"
 #include "direct.cuh"
 #include "premix.cuh"
+#include "layer_tc.cuh"
 #include "route.cuh"
 
 namespace {
@@ -51,6 +52,8 @@ std::atomic<unsigned long long> g_launches{0};
 std::atomic<long long> g_wait_ns{kDefaultWaitNs};
 std::atomic<int> g_inject_skip{0};
 std::atomic<int> g_route_split{0};  // 0: automatic
+std::atomic<int> g_use_pdl{1};      // programmatic launch edges on forward kernels
+std::atomic<int> g_fused_premix{0}; // PREMIX as one persistent kernel (else two kernels)
 thread_local char g_last_err[256] = "";
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -123,6 +126,25 @@ cudaError_t ensure_smem(K kern, size_t bytes) {
                            static_cast<int>(bytes));
   if (e == cudaSuccess) g_smem_set[key] = bytes;
   return e;
+}
+
+// Launch with a programmatic stream-serialization edge: the kernel may start
+// while the previous kernel on the stream finishes; it calls
+// griddepcontrol.wait before reading any global memory.
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_use_pdl.load() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -243,10 +265,15 @@ bool depthwise_ok(const dynconv_desc* d) {
          out_size(d->W, d->KW, 1, d->pad) >= 1;
 }
 
+// Workspace of PREMIX: the mixed kernels of every sample, then (256-byte
+// aligned) one word for the fused kernel's grid barrier.
+size_t premix_wb_bytes(const dynconv_desc* d) {
+  return (static_cast<size_t>(d->B) * d->C_out * d->KH * d->KW * d->C_in * 2 + 255) & ~size_t(255);
+}
 size_t premix_workspace(const dynconv_desc* d) {
   if (!tc_shape_ok(d)) return 0;
   if (!dc::premix_shape_ok(d->B, d->n, d->C_out, d->KH * d->KW, d->C_in)) return 0;
-  return static_cast<size_t>(d->B) * d->C_out * d->KH * d->KW * d->C_in * 2;
+  return premix_wb_bytes(d) + 256;
 }
 
 // Cost-model choice among the kernels that can run this descriptor.
@@ -332,8 +359,112 @@ int launch_tc(const TcPlan& plan, const CUtensorMap& xmap, const CUtensorMap& wm
               cudaStream_t stream) {
   cudaError_t e = ensure_smem(dc::tc_conv_kernel<V>, plan.smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc_conv)");
-  dc::tc_conv_kernel<V><<<plan.grid, dc::kTcThreads, plan.smem, stream>>>(xmap, wmap, plan.p);
+  e = launch_pdl(dc::tc_conv_kernel<V>, dim3(plan.grid), dim3(dc::kTcThreads), plan.smem, stream,
+                 xmap, wmap, plan.p);
+  if (e != cudaSuccess) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_fail(e, "tc_conv_kernel launch");
+  }
   return check_launch("tc_conv_kernel");
+}
+
+// Grid-barrier words already zeroed on some stream (per device and address).
+// Cleared when a bounded wait expires, because an aborted launch can leave
+// the words mid-barrier.
+std::mutex g_bar_mu;
+std::map<std::pair<int, const void*>, bool> g_bar_ready;
+
+bool barrier_words_need_reset(const void* words) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return true;
+  std::lock_guard<std::mutex> lk(g_bar_mu);
+  auto key = std::make_pair(dev, words);
+  if (g_bar_ready.count(key)) return false;
+  g_bar_ready[key] = true;
+  return true;
+}
+
+void barrier_words_forget_all() {
+  std::lock_guard<std::mutex> lk(g_bar_mu);
+  g_bar_ready.clear();
+}
+
+// PREMIX as one persistent cooperative kernel: returns DYNCONV_ERR_UNSUPPORTED
+// (and launches nothing) when the two phases cannot share one CTA per SM.
+int run_fused_premix(const dynconv_desc* d, const TcPlan& plan_in, const DeviceState* st,
+                     const void* x, const void* experts, const float* alpha, const float* bias,
+                     void* y, void* ws, const CUtensorMap& xmap, const CUtensorMap& wmap,
+                     cudaStream_t stream) {
+  dc::FusedParams fp{};
+  fp.cv = plan_in.p;
+  dc::PremixLaunch pl;
+  int rc = dc::plan_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
+                           static_cast<__nv_bfloat16*>(ws), d->B, d->n,
+                           static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in, st->err,
+                           g_wait_ns.load(), st->sms, g_encode, &pl);
+  if (rc == -2) {
+    std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(premix) failed");
+    return DYNCONV_ERR_CUDA;
+  }
+  if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
+  fp.pm = pl.p;
+  // shared memory: activation stages (own region) | region used by the mixing
+  // phase, then by the convolution's weight stages + epilogue staging | barriers
+  const size_t b_region = static_cast<size_t>(fp.cv.sb) * fp.cv.b_tile_bytes;
+  const size_t fixed = 1024 + 16 + 64;
+  const size_t budget = static_cast<size_t>(st->max_smem_optin) - fixed - b_region;
+  size_t pm_region = 0;
+  for (;; --fp.pm.stages) {  // as many mixing stages as fit (at least 2)
+    pm_region = (static_cast<size_t>(fp.pm.a_bytes) +
+                 static_cast<size_t>(fp.pm.stages) * fp.pm.stage_bytes + 4 * dc::kFusedPmStage +
+                 4 * static_cast<size_t>(d->B) * d->n + 1023) & ~size_t(1023);
+    if (fp.pm.stages <= 2 || pm_region + 8 * 64 <= budget) break;
+  }
+  int sa = fp.cv.sa;
+  size_t cv_region = 0, total = 0;
+  for (; sa >= 2; --sa) {
+    cv_region = static_cast<size_t>(sa) * dc::kTcATileBytes + dc::kFusedEpiStage;
+    const size_t region = std::max(pm_region, cv_region);
+    const size_t bars = 8 * (2 * fp.pm.stages + 4 + 2 * sa + 2 * fp.cv.sb + 3);
+    total = fixed + b_region + region + bars;
+    if (total <= static_cast<size_t>(st->max_smem_optin)) break;
+  }
+  if (sa < 2) return DYNCONV_ERR_UNSUPPORTED;
+  fp.cv.sa = sa;
+  fp.region_bytes = static_cast<int>(std::max(pm_region, cv_region));
+  fp.cv.experts = static_cast<const __nv_bfloat16*>(experts);
+  fp.cv.alpha = alpha;
+  fp.cv.bias = bias;
+  fp.cv.y = static_cast<__nv_bfloat16*>(y);
+  fp.cv.err = st->err;
+  fp.cv.wait_ns = g_wait_ns.load();
+  fp.units = plan_in.grid;
+  fp.grid_bar = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + premix_wb_bytes(d));
+  cudaError_t e = cudaSuccess;
+  if (barrier_words_need_reset(fp.grid_bar)) {
+    // the barrier resets itself after every use; only a workspace seen for the
+    // first time (or after a timeout) needs its two words zeroed
+    e = cudaMemsetAsync(fp.grid_bar, 0, 2 * sizeof(unsigned int), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(grid barrier words)");
+  }
+  e = ensure_smem(dc::premix_conv_kernel, total);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix_conv)");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(st->sms);
+  cfg.blockDim = dim3(dc::kFusedThreads);
+  cfg.dynamicSmemBytes = total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, dc::premix_conv_kernel, pl.emap, xmap, wmap, fp);
+  if (e != cudaSuccess) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_fail(e, "premix_conv_kernel launch");
+  }
+  return check_launch("premix_conv_kernel");
 }
 
 int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void* x,
@@ -360,18 +491,34 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   if (!ws || ws_bytes < need) return DYNCONV_ERR_WORKSPACE;
   if (!aligned16(ws)) return DYNCONV_ERR_MISALIGNED;
   plan.p.inject_skip = 0;
-  rc = dc::launch_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
-                         static_cast<__nv_bfloat16*>(ws), d->B, d->n,
-                         static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in, st->err,
-                         g_wait_ns.load(), st->sms, stream, g_encode,
-                         [](auto k, size_t b) { return ensure_smem(k, b); });
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  if (rc == -1) return cuda_fail(cudaGetLastError(), "premix launch");
+  if (g_fused_premix.load()) {
+    rc = encode_w_map(&wmap, ws, d);
+    if (rc) return rc;
+    rc = run_fused_premix(d, plan, st, x, experts, alpha, bias, y, ws, xmap, wmap, stream);
+    if (rc != DYNCONV_ERR_UNSUPPORTED) return rc;
+  }
+  dc::PremixLaunch pl;
+  rc = dc::plan_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
+                       static_cast<__nv_bfloat16*>(ws), d->B, d->n,
+                       static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in, st->err,
+                       g_wait_ns.load(), st->sms, g_encode, &pl);
   if (rc == -2) {
     std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(premix) failed");
     return DYNCONV_ERR_CUDA;
   }
   if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
+  {
+    cudaError_t e = ensure_smem(dc::premix_kernel, pl.smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
+    e = launch_pdl(dc::premix_kernel, dim3(pl.grid), dim3(dc::kPmThreads), pl.smem, stream,
+                   pl.emap, pl.p);
+    if (e != cudaSuccess) {
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      return cuda_fail(e, "premix_kernel launch");
+    }
+    rc = check_launch("premix_kernel");
+    if (rc) return rc;
+  }
   rc = encode_w_map(&wmap, ws, d);
   if (rc) return rc;
   return launch_tc<dc::kPremix>(plan, xmap, wmap, stream);
@@ -413,6 +560,16 @@ int dynconv_test_hook(int key, long long value) {
   if (key == 4) {
     if (value < 0 || value > 8) return DYNCONV_ERR_INVALID_ARG;
     g_route_split.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
+  if (key == 5) {
+    if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
+    g_use_pdl.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
+  if (key == 6) {
+    if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
+    g_fused_premix.store(static_cast<int>(value));
     return DYNCONV_OK;
   }
   if (key == 3) {
@@ -563,7 +720,11 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
       auto go = [&](auto kern) -> int {
         cudaError_t e = ensure_smem(kern, smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(depthwise)");
-        kern<<<grid, dc::kDwThreads, smem, s>>>(xmap, p);
+        e = launch_pdl(kern, grid, dim3(dc::kDwThreads), smem, s, xmap, p);
+        if (e != cudaSuccess) {
+          g_launches.fetch_add(1, std::memory_order_relaxed);
+          return cuda_fail(e, "depthwise_kernel launch");
+        }
         return check_launch("depthwise_kernel");
       };
       if (K == 3) return go(dc::depthwise_kernel<3>);
@@ -591,7 +752,11 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
       auto go = [&](auto kern) -> int {
         cudaError_t e = ensure_smem(kern, smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(direct)");
-        kern<<<grid, dc::kDirectThreads, smem, s>>>(p);
+        e = launch_pdl(kern, grid, dim3(dc::kDirectThreads), smem, s, p);
+        if (e != cudaSuccess) {
+          g_launches.fetch_add(1, std::memory_order_relaxed);
+          return cuda_fail(e, "direct_conv_kernel launch");
+        }
         return check_launch("direct_conv_kernel");
       };
       if (desc->dtype == DYNCONV_F32) return go(dc::direct_conv_kernel<float>);
@@ -653,6 +818,7 @@ int dynconv_device_status(void* stream) {
   e = cudaMemcpyFromSymbol(&word, g_device_err, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e, "read error word");
   if (word != 0) {
+    barrier_words_forget_all();
     const int zero = 0;
     e = cudaMemcpyToSymbol(g_device_err, &zero, sizeof(int));
     if (e != cudaSuccess) return cuda_fail(e, "clear error word");

@@ -87,6 +87,13 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
 
+  // the convolution may be scheduled as soon as every CTA of this grid runs
+  grid_launch_dependents();
+  if (warp == 0) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), 512);
+    tmem_relinquish();
+  }
+  grid_dependency_wait();  // alpha comes from the routing kernel
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full(s), 1);
@@ -100,10 +107,6 @@ __global__ void __launch_bounds__(kPmThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&emap);
-  }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), 512);
-    tmem_relinquish();
   }
   // A operands: alpha split into bf16 hi + lo, zero outside [B) x [n).
   // Stage alpha in shared memory first (all loads in flight at once), then
@@ -226,8 +229,10 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       const int ab = static_cast<int>(j & 1);
       if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j >> 1) & 1), ctl, kErrWaitEpilogue)) break;
       tc_fence_after();
+      // a warp whose 32 samples are all past the batch only releases the buffer
+      const bool live = mt * 128 + 32 * q < p.B;
 #pragma unroll 1
-      for (int ch = 0; ch < kPmN / 32; ++ch) {
+      for (int ch = 0; ch < (live ? kPmN / 32 : 0); ++ch) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * kPmN + ch * 32, r);
         tmem_ld_wait();
@@ -248,14 +253,15 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       if (lane == 0) mbar_arrive(tempty(ab));
       const long long w = ntile * kPmN + lane * 8;
       const bool wok = w < p.wsize;
+      const int nrows = live ? min(32, p.B - (mt * 128 + 32 * q)) : 0;
 #pragma unroll 4
-      for (int sr = 0; sr < 32; ++sr) {
+      for (int sr = 0; sr < nrows; ++sr) {
         const int b = mt * 128 + 32 * q + sr;
         uint4 v;
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                      : "r"(stg + sr * 512 + ((lane ^ sr) << 4)));
-        if (b < p.B && wok)
+        if (wok)
           *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.wsize + w) = v;
       }
       __syncwarp();
@@ -273,12 +279,21 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   }
 }
 
-// Host launcher. Returns 0, -1 (CUDA launch error), -2 (tensor map), -3 (shape).
-template <typename EncodeFn, typename SmemFn>
-inline int launch_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bfloat16* out,
-                         int B, int n, long long wsize, int* err, long long wait_ns, int sms,
-                         cudaStream_t stream, EncodeFn encode, SmemFn ensure_smem_fn) {
-  PmParams p{};
+// Host-side plan of one premix launch.
+struct PremixLaunch {
+  PmParams p;
+  CUtensorMap emap;
+  unsigned grid = 0;
+  size_t smem = 0;
+};
+
+// Fills `out`. Returns 0, -2 (tensor map), -3 (shape).
+template <typename EncodeFn>
+inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bfloat16* out_ws,
+                       int B, int n, long long wsize, int* err, long long wait_ns, int sms,
+                       EncodeFn encode, PremixLaunch* out) {
+  PmParams& p = out->p;
+  p = PmParams{};
   p.B = B;
   p.n = n;
   p.nk = pm_nk(n);
@@ -292,28 +307,24 @@ inline int launch_premix(const __nv_bfloat16* experts, const float* alpha, __nv_
   p.stages = std::min(4, budget / p.stage_bytes);
   if (p.stages < 2) return -3;
   p.alpha = alpha;
-  p.out = out;
+  p.out = out_ws;
   p.err = err;
   p.wait_ns = wait_ns;
-
-  CUtensorMap emap;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(wsize), static_cast<cuuint64_t>(n)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(wsize) * 2};
   const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(p.nk)};
   const cuuint32_t es[2] = {1u, 1u};
-  if (encode(&emap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(experts), dims,
-             strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  if (encode(&out->emap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(experts),
+             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return -2;
   // at least 120 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
-  const size_t smem = std::max<size_t>(120 * 1024, 1024 + static_cast<size_t>(p.a_bytes) +
-                                                       static_cast<size_t>(p.stages) * p.stage_bytes +
-                                                       4 * kPmStageBytes + 8 * (2 * p.stages + 5) + 16 +
-                                                       4 * static_cast<size_t>(B) * n);
-  if (ensure_smem_fn(premix_kernel, smem) != cudaSuccess) return -1;
-  const long long grid = std::min<long long>(p.tiles, sms);
-  premix_kernel<<<static_cast<unsigned>(grid), kPmThreads, smem, stream>>>(emap, p);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  out->smem = std::max<size_t>(120 * 1024, 1024 + static_cast<size_t>(p.a_bytes) +
+                                               static_cast<size_t>(p.stages) * p.stage_bytes +
+                                               4 * kPmStageBytes + 8 * (2 * p.stages + 5) + 16 +
+                                               4 * static_cast<size_t>(B) * n);
+  out->grid = static_cast<unsigned>(std::min<long long>(p.tiles, sms));
+  return 0;
 }
 
 }  // namespace dc

@@ -180,6 +180,20 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// ------------------------------------------------- programmatic dependent launch
+
+// Wait until the grids this one depends on have completed and their memory is
+// visible (no-op when the kernel was launched without a programmatic edge).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Allow the dependent grid to be scheduled once every CTA of this grid has
+// executed this (or exited); its CTAs still wait for this grid's completion
+// before they read its results.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+}
+
 // ------------------------------------------------------------------- misc
 
 // Read-only 16-byte load that bypasses L1. Not volatile: the compiler may

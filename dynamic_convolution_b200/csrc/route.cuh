@@ -95,6 +95,9 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
   const int nsplit = static_cast<int>(cluster.num_blocks());
   const int b = blockIdx.y;
   const int t = threadIdx.x;
+  // the forward kernel may be scheduled as soon as every routing CTA runs; it
+  // waits for this grid's completion before it reads alpha
+  grid_launch_dependents();
 
   extern __shared__ float route_smem[];
   const int C = p.C;

@@ -117,7 +117,13 @@ int dynconv_route(const dynconv_desc* desc, const void* x, const float* Wr, cons
  *   bias           device fp32 [n][C_out] or NULL;
  *   workspace      device scratch of workspace_bytes bytes, or NULL/0. Only the
  *                  PREMIX variant uses it; AUTO never picks PREMIX unless the
- *                  workspace is large enough.
+ *                  workspace is large enough. It holds every sample's mixed
+ *                  kernel, then (last 256 bytes) the state of a grid barrier:
+ *                  the library zeroes that state the first time it sees a
+ *                  workspace address on a device (and again after a bounded
+ *                  wait expired) and leaves it valid after each call. A caller
+ *                  that writes those bytes between calls (reusing the memory for
+ *                  other data) zeroes the first 8 of them before the next call.
  * Precision: bf16 in, fp32 accumulate, the mixed kernel rounded once to bf16
  * (tensor-core variants), y rounded once to bf16. fp32 layers accumulate and
  * mix in fp32.
@@ -197,6 +203,12 @@ unsigned long long dynconv_launch_count(void);
  * results). Only for re-verifying that choice on a device.
  * key 4: CTAs per sample of the routing kernel's cluster (1..8; 0 restores
  * the automatic choice), for tuning measurements.
+ * key 5: 1 (default) launches the forward kernels with a programmatic
+ * stream-serialization edge (they may start while the previous kernel on the
+ * stream finishes, and wait for it before reading memory); 0 launches them
+ * plainly. For measurements.
+ * key 6: 1 runs PREMIX as one persistent cooperative kernel (kernel mixing,
+ * grid barrier, convolution); 0 (default) runs it as two kernels.
  * Returns DYNCONV_OK or DYNCONV_ERR_INVALID_ARG. */
 int dynconv_test_hook(int key, long long value);
 

@@ -212,3 +212,27 @@ def test_outputs_outside_y_untouched():
         L.forward(v)
     torch.cuda.synchronize()
     assert torch.all(big[L.y.numel():] == 7.0)
+
+
+@pytest.mark.parametrize("name", ["resnet18_3x3", "effnet_expand_1x1", "large_n64"])
+def test_premix_fused_kernel_equals_two_kernels(name):
+    """PREMIX as one persistent kernel (mixing, grid barrier, convolution; several
+    units per CTA when there are more units than SMs) gives the same bits as the
+    two-kernel form."""
+    inp = layer_inputs(name)
+    L = Layer(inp)
+    L.route()
+    d = L.desc(dc.VARIANT_PREMIX)
+    ws = torch.zeros(dc.dynconv_workspace_size(d), dtype=torch.uint8, device="cuda")
+    outs = []
+    try:
+        for fused in (1, 0):
+            assert dc.dynconv_test_hook(6, fused) == dc.OK
+            L.y.fill_(float("nan"))
+            dc.check(dc.dynconv_forward(d, L.x, L.experts, L.alpha, L.bias, L.y, ws, ws.numel()))
+            assert dc.dynconv_device_status(None) == dc.OK
+            outs.append(L.y.clone())
+    finally:
+        dc.dynconv_test_hook(6, 1)
+    assert torch.equal(outs[0], outs[1])
+    assert torch.isfinite(outs[0].float()).all()
