@@ -425,7 +425,8 @@ def run_ours(args, cfg):
         peak = float(peaks["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "peak_kind": f"bf16 dense burst, {peak_kind}",
-                "kernel": f"tc_conv_kernel<{variant_name}>",
+                "kernel": ("forward call: premix_kernel + tc_conv_kernel<premix>"
+                           if variant_name == "premix" else f"tc_conv_kernel<{variant_name}>"),
                 "algorithmic": f"{conv_flops} conv FLOP per launch (2*B*HW*Cout*Cin*KH*KW)"}
     else:
         achieved = algo_bytes / (fwd_launch_ms / 1e3) / 1e9
