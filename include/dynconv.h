@@ -209,6 +209,10 @@ unsigned long long dynconv_launch_count(void);
  * plainly. For measurements.
  * key 6: 1 runs PREMIX as one persistent cooperative kernel (kernel mixing,
  * grid barrier, convolution); 0 (default) runs it as two kernels.
+ * key 7: which kernel mixes the per-sample kernels of the two-kernel PREMIX
+ * form: 0 (default) the CUDA-core mixer when n <= 8, else the tensor-core
+ * mixing GEMM; 1 always the tensor-core GEMM; 2 the CUDA-core mixer only
+ * (forward returns DYNCONV_ERR_UNSUPPORTED when n > 8).
  * Returns DYNCONV_OK or DYNCONV_ERR_INVALID_ARG. */
 int dynconv_test_hook(int key, long long value);
 

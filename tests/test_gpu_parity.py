@@ -226,6 +226,7 @@ def test_premix_fused_kernel_equals_two_kernels(name):
     ws = torch.zeros(dc.dynconv_workspace_size(d), dtype=torch.uint8, device="cuda")
     outs = []
     try:
+        assert dc.dynconv_test_hook(7, 1) == dc.OK  # both forms mix on tensor cores
         for fused in (1, 0):
             assert dc.dynconv_test_hook(6, fused) == dc.OK
             L.y.fill_(float("nan"))
@@ -233,6 +234,33 @@ def test_premix_fused_kernel_equals_two_kernels(name):
             assert dc.dynconv_device_status(None) == dc.OK
             outs.append(L.y.clone())
     finally:
-        dc.dynconv_test_hook(6, 1)
+        dc.dynconv_test_hook(6, 0)
+        dc.dynconv_test_hook(7, 0)
     assert torch.equal(outs[0], outs[1])
     assert torch.isfinite(outs[0].float()).all()
+
+
+@pytest.mark.parametrize("name", ["resnet18_3x3", "effnet_expand_1x1"])
+@pytest.mark.parametrize("mixer", [1, 2])
+def test_premix_mixers_full_size(name, mixer):
+    """PREMIX with each mixing kernel (1: tensor-core GEMM with a hi/lo split
+    of alpha, 2: CUDA-core fp32 mixer) against the oracle on sampled whole
+    samples."""
+    try:
+        assert dc.dynconv_test_hook(7, mixer) == dc.OK
+        _forward_case(name, dc.VARIANT_PREMIX, workspace=True)
+    finally:
+        dc.dynconv_test_hook(7, 0)
+
+
+def test_premix_cuda_core_mixer_refuses_many_experts():
+    inp = layer_inputs("deep_3x3_tau30")
+    L = Layer(inp)
+    d = L.desc(dc.VARIANT_PREMIX)
+    ws = torch.zeros(dc.dynconv_workspace_size(d), dtype=torch.uint8, device="cuda")
+    try:
+        assert dc.dynconv_test_hook(7, 2) == dc.OK
+        rc = dc.dynconv_forward(d, L.x, L.experts, L.alpha, L.bias, L.y, ws, ws.numel())
+        assert rc == dc.ERR_UNSUPPORTED
+    finally:
+        dc.dynconv_test_hook(7, 0)
