@@ -127,8 +127,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), p.tmem_cols);
     tmem_relinquish();
   }
-  grid_dependency_wait();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 32) {
     for (int s = 0; s < SA; ++s) {
       mbar_init(fullA(s), VARIANT == kPremix ? 1 : kTcMixThreads / 32);
       mbar_init(emptyA(s), 1);
@@ -141,6 +140,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    tma_prefetch_desc(&xmap);
+    if (VARIANT == kPremix) tma_prefetch_desc(&wmap);
+  }
+  __syncwarp();
+  grid_dependency_wait();
+  if (threadIdx.x == 32) {
     // The first loads need nothing but the barriers: issue them now so their
     // latency overlaps the rest of the set-up.
     const int pre_b = p.kc < SB ? p.kc : SB;

@@ -19,6 +19,7 @@
 #include "depthwise.cuh"
 #include "direct.cuh"
 #include "premix.cuh"
+#include "premix_small.cuh"
 #include "layer_tc.cuh"
 #include "route.cuh"
 
@@ -54,6 +55,7 @@ std::atomic<int> g_inject_skip{0};
 std::atomic<int> g_route_split{0};  // 0: automatic
 std::atomic<int> g_use_pdl{1};      // programmatic launch edges on forward kernels
 std::atomic<int> g_fused_premix{0}; // PREMIX as one persistent kernel (else two kernels)
+std::atomic<int> g_premix_mixer{0};  // 0 automatic, 1 tensor-core GEMM, 2 CUDA cores (n <= 8)
 thread_local char g_last_err[256] = "";
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -497,6 +499,33 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
     rc = run_fused_premix(d, plan, st, x, experts, alpha, bias, y, ws, xmap, wmap, stream);
     if (rc != DYNCONV_ERR_UNSUPPORTED) return rc;
   }
+  // few experts: the store-bound CUDA-core mixer (no set-up chain)
+  if (g_premix_mixer.load() != 1) {
+    dc::PsParams ps;
+    unsigned grid = 0;
+    if (dc::plan_premix_small(d->B, d->n,
+                              static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in, st->sms,
+                              &ps, &grid) &&
+        aligned16(experts)) {
+      ps.experts = static_cast<const __nv_bfloat16*>(experts);
+      ps.alpha = alpha;
+      ps.out = static_cast<__nv_bfloat16*>(ws);
+      const size_t smem = sizeof(float) * static_cast<size_t>(d->B) * d->n;
+      auto kern = d->n <= 2 ? dc::premix_small_kernel<2>
+                  : d->n <= 4 ? dc::premix_small_kernel<4> : dc::premix_small_kernel<8>;
+      cudaError_t e = launch_pdl(kern, dim3(grid), dim3(dc::kPsThreads), smem, stream, ps);
+      if (e != cudaSuccess) {
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return cuda_fail(e, "premix_small_kernel launch");
+      }
+      rc = check_launch("premix_small_kernel");
+      if (rc) return rc;
+      rc = encode_w_map(&wmap, ws, d);
+      if (rc) return rc;
+      return launch_tc<dc::kPremix>(plan, xmap, wmap, stream);
+    }
+    if (g_premix_mixer.load() == 2) return DYNCONV_ERR_UNSUPPORTED;
+  }
   dc::PremixLaunch pl;
   rc = dc::plan_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
                        static_cast<__nv_bfloat16*>(ws), d->B, d->n,
@@ -572,6 +601,11 @@ int dynconv_test_hook(int key, long long value) {
     g_fused_premix.store(static_cast<int>(value));
     return DYNCONV_OK;
   }
+  if (key == 7) {
+    if (value < 0 || value > 2) return DYNCONV_ERR_INVALID_ARG;
+    g_premix_mixer.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
   if (key == 3) {
     if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
     g_desc_base_mode = static_cast<int>(value);
@@ -616,9 +650,32 @@ int dynconv_route(const dynconv_desc* desc, const void* x, const float* Wr, cons
   int nsplit = (2 * st->sms) / std::max(desc->B, 1);
   if (g_route_split.load() > 0) nsplit = g_route_split.load();
   nsplit = std::max(1, std::min({nsplit, 8, HW}));
-  const size_t smem = sizeof(float) * dc::route_smem_floats(C, desc->n, VEC, nsplit);
+  // bulk staging of each CTA's contiguous pixel slice when a pixel row is a
+  // 16-byte multiple and one channel vector per thread covers it; pieces of at
+  // most 48 KB, balanced
+  const size_t row_bytes = static_cast<size_t>(C) * eb;
+  int piece_px = 0;
+  if (vec && C / VEC <= dc::kRouteThreads) {
+    const int slice_px = (HW + nsplit - 1) / nsplit;
+    int per = static_cast<int>(std::max<size_t>(1, dc::kRoutePieceBytes / row_bytes));
+    per = std::min(per, slice_px);
+    const int pieces = (slice_px + per - 1) / per;
+    piece_px = (slice_px + pieces - 1) / pieces;
+  }
+  const size_t wr_bytes = static_cast<size_t>(desc->n) * C * 4;
+  const int wr_smem = (wr_bytes <= dc::kRouteWrSmemBytes && wr_bytes % 16 == 0 && aligned16(Wr)) ? 1 : 0;
+  size_t smem = dc::route_smem(C, desc->n, VEC, static_cast<int>(eb), nsplit, piece_px, wr_smem,
+                               piece_px > 0).total;
+  // very wide rows without staged Wr: fewer ranks (rank 0 receives nsplit x C sums)
+  while (smem > static_cast<size_t>(st->max_smem_optin) && nsplit > 1) {
+    --nsplit;
+    smem = dc::route_smem(C, desc->n, VEC, static_cast<int>(eb), nsplit, piece_px, wr_smem,
+                          piece_px > 0).total;
+  }
+  if (smem > static_cast<size_t>(st->max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
 
-  dc::RouteParams p{desc->B, C, HW, desc->n, mode, tau, x, Wr, br, alpha};
+  dc::RouteParams p{desc->B, C, HW, desc->n, mode, tau, x, Wr, br, alpha,
+                    nsplit, piece_px, wr_smem, st->err, g_wait_ns.load()};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nsplit, desc->B, 1);
   cfg.blockDim = dim3(dc::kRouteThreads, 1, 1);

@@ -35,6 +35,8 @@ struct PsParams {
   __nv_bfloat16* out;            // [B][wsize]
 };
 
+// NMAX: the expert count rounded up to 2, 4 or 8 (fewer registers for fewer experts)
+template <int NMAX>
 __global__ void __launch_bounds__(kPsThreads) premix_small_kernel(PsParams p) {
   extern __shared__ float ps_alpha[];  // [B][n]
   // the convolution may be scheduled as soon as every CTA of this grid runs
@@ -50,13 +52,13 @@ __global__ void __launch_bounds__(kPsThreads) premix_small_kernel(PsParams p) {
     const long long sb = it / p.chunks;
     const long long ch = it - sb * p.chunks;
     // the 8 weights of every expert, widened to packed fp32 pairs
-    uint4 raw[kPsMaxExperts];
+    uint4 raw[NMAX];
 #pragma unroll
-    for (int i = 0; i < kPsMaxExperts; ++i)
+    for (int i = 0; i < NMAX; ++i)
       if (i < p.n) raw[i] = ld_nc_v4(p.experts + static_cast<size_t>(i) * p.wsize + ch * 8);
-    uint64_t ef[kPsMaxExperts][4];
+    uint64_t ef[NMAX][4];
 #pragma unroll
-    for (int i = 0; i < kPsMaxExperts; ++i) {
+    for (int i = 0; i < NMAX; ++i) {
       if (i < p.n) {
         ef[i][0] = bf16x2_to_f32x2(raw[i].x);
         ef[i][1] = bf16x2_to_f32x2(raw[i].y);
@@ -71,7 +73,7 @@ __global__ void __launch_bounds__(kPsThreads) premix_small_kernel(PsParams p) {
       const float* ab = ps_alpha + b * p.n;
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int i = 0; i < kPsMaxExperts; ++i) {
+      for (int i = 0; i < NMAX; ++i) {
         if (i < p.n) {
           const float a = ab[i];
           const uint64_t a2 = pack_f32x2(a, a);

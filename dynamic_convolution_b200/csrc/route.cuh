@@ -7,19 +7,23 @@
 // global-average-pool -> single linear layer -> sigmoid / softmax(z/tau) form
 // is the reading taken where the pages give no formula.
 //
-// Design: one thread-block cluster per sample, built around the latency
-// chain rather than bandwidth (the whole input is ~10 MB):
-//  * every thread issues its 16-byte NHWC loads in batches of 16 before it
-//    adds any of them, so the cluster has the sample's bytes in flight at once;
-//  * the rank-0 CTA prefetches the router weights Wr and br into shared
-//    memory while those loads are in flight;
-//  * each CTA reduces its per-thread partial sums in a fixed order, then PUSHES
-//    its per-channel sums into rank 0's shared memory with remote stores
-//    (distributed shared memory) -- one cluster barrier, no remote loads;
-//  * rank 0 adds the slices in rank order, runs the FC from shared memory
-//    (warp-shuffle dot products) and the activation (warp-shuffle max / sum
-//    for the softmax).
-// No global scratch, no atomics, deterministic.
+// Design: one thread-block cluster per sample, each CTA a contiguous slice of
+// the sample's pixels, built around the latency chain (the whole input is a
+// few MB):
+//  * the slice is contiguous in NHWC, so one thread moves it into shared
+//    memory with a few bulk copies (cp.async.bulk, at most two in flight),
+//    together with the router weights Wr when they fit: the bytes in flight
+//    are not limited by per-thread load queues;
+//  * the threads add the staged pixels in a fixed order;
+//  * the linear layer is split over the ranks: each CTA multiplies its own
+//    channel sums by Wr and PUSHES its n partial logits into rank 0's shared
+//    memory (distributed shared memory); after the one cluster barrier rank 0
+//    adds nsplit x n numbers, scales by 1/HW, adds br and applies the
+//    activation.
+// When Wr does not fit in shared memory the CTAs push per-channel sums and
+// rank 0 runs the linear layer reading Wr from global memory. When a pixel's
+// channels are not a multiple of 16 bytes the threads load the pixels
+// themselves (no bulk copy). No global scratch, no atomics, deterministic.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -29,6 +33,9 @@
 namespace dc {
 
 constexpr int kRouteThreads = 256;
+constexpr int kRoutePieceBytes = 48 * 1024;  // largest bulk piece
+constexpr int kRouteWrSmemBytes = 32 * 1024;  // largest Wr staged in shared memory
+constexpr int kErrWaitRoute = 0x107;
 
 struct RouteParams {
   int B, C, HW, n;
@@ -38,31 +45,50 @@ struct RouteParams {
   const float* Wr;
   const float* br;  // may be null
   float* alpha;
+  int nsplit;       // CTAs per sample (the cluster size)
+  int piece_px;     // pixels per bulk piece (bulk path)
+  int wr_smem;      // 1: Wr staged in shared memory, partial logits per rank
+  int* err;
+  long long wait_ns;
 };
 
-// VEC channels per load: 16 bytes when the channel count allows it, else 1.
-// Raw loads and the conversion to fp32 are separate so that a batch of loads
-// is issued before the first one is used.
-template <typename T, int VEC>
-union RawVec {
-  uint4 u;   // 16-byte path
-  T s[VEC];  // scalar path
+// Shared-memory carve-up, in bytes; the host sizes the launch with `total`.
+struct RouteSmem {
+  size_t ring, wr, partial, g, recv, brs, z, bars, flag, total;
 };
 
-template <typename T, int VEC>
-__device__ __forceinline__ void load_raw(const T* p, RawVec<T, VEC>& r) {
-  if constexpr (VEC * sizeof(T) == 16) {
-    r.u = ld_nc_v4(p);
-  } else {
-#pragma unroll
-    for (int j = 0; j < VEC; ++j) r.s[j] = p[j];
-  }
+__host__ __device__ inline RouteSmem route_smem(int C, int n, int VEC, int elem_bytes,
+                                                int nsplit, int piece_px, int wr_smem,
+                                                bool bulk) {
+  const int nv = C / VEC;
+  const int tpp = nv < kRouteThreads ? nv : kRouteThreads;
+  const int lanes_p = kRouteThreads / tpp;
+  RouteSmem s{};
+  size_t off = 0;
+  auto take = [&](size_t bytes, size_t align) {
+    off = (off + align - 1) / align * align;
+    const size_t at = off;
+    off += bytes;
+    return at;
+  };
+  const size_t piece = static_cast<size_t>(piece_px) * C * elem_bytes;
+  s.ring = take(bulk ? 2 * piece : 0, 128);
+  s.wr = take(wr_smem ? static_cast<size_t>(n) * C * 4 : 0, 128);
+  s.partial = take(static_cast<size_t>(lanes_p) * C * 4, 16);
+  s.g = take(static_cast<size_t>(C) * 4, 16);
+  s.recv = take(static_cast<size_t>(nsplit) * (wr_smem ? n : C) * 4, 16);
+  s.brs = take(static_cast<size_t>(n) * 4, 16);
+  s.z = take(static_cast<size_t>(n) * 4, 16);
+  s.bars = take(3 * 8, 8);
+  s.flag = take(4, 4);
+  s.total = off;
+  return s;
 }
 
 template <typename T, int VEC>
-__device__ __forceinline__ void add_raw(const RawVec<T, VEC>& r, float (&acc)[VEC]) {
+__device__ __forceinline__ void add_vec(const void* src, float (&acc)[VEC]) {
   if constexpr (VEC * sizeof(T) == 16) {
-    const uint4 u = r.u;
+    const uint4 u = *reinterpret_cast<const uint4*>(src);
     if constexpr (sizeof(T) == 2) {
       acc[0] += bf16lo_to_f32(u.x); acc[1] += bf16hi_to_f32(u.x);
       acc[2] += bf16lo_to_f32(u.y); acc[3] += bf16hi_to_f32(u.y);
@@ -73,103 +99,176 @@ __device__ __forceinline__ void add_raw(const RawVec<T, VEC>& r, float (&acc)[VE
       acc[2] += __uint_as_float(u.z); acc[3] += __uint_as_float(u.w);
     }
   } else {
+    const T* v = static_cast<const T*>(src);
 #pragma unroll
-    for (int j = 0; j < VEC; ++j) acc[j] += to_f32<T>(r.s[j]);
+    for (int j = 0; j < VEC; ++j) acc[j] += to_f32<T>(v[j]);
   }
-}
-
-// Shared-memory floats the kernel needs (the host sizes the launch with it).
-__host__ __device__ inline size_t route_smem_floats(int C, int n, int VEC, int nsplit) {
-  const int nv = C / VEC;
-  const int tpp = nv < kRouteThreads ? nv : kRouteThreads;
-  const int lanes_p = kRouteThreads / tpp;
-  const size_t wr = static_cast<size_t>(n) * C <= 8192 ? static_cast<size_t>(n) * C : 0;
-  return static_cast<size_t>(lanes_p) * C + static_cast<size_t>(nsplit) * C + C + wr + 2 * n;
 }
 
 template <typename T, int VEC>
 __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) {
   namespace cg = cooperative_groups;
+  constexpr bool kBulk = VEC * sizeof(T) == 16;
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int nsplit = static_cast<int>(cluster.num_blocks());
+  const int nsplit = p.nsplit;
   const int b = blockIdx.y;
   const int t = threadIdx.x;
   // the forward kernel may be scheduled as soon as every routing CTA runs; it
   // waits for this grid's completion before it reads alpha
   grid_launch_dependents();
 
-  extern __shared__ float route_smem[];
+  extern __shared__ __align__(128) unsigned char route_raw[];
   const int C = p.C;
+  const RouteSmem L = route_smem(C, p.n, VEC, static_cast<int>(sizeof(T)), nsplit, p.piece_px,
+                                 p.wr_smem, kBulk && p.piece_px > 0);
+  float* wr_s = reinterpret_cast<float*>(route_raw + L.wr);
+  float* partial = reinterpret_cast<float*>(route_raw + L.partial);  // [lanes_p][C]
+  float* g = reinterpret_cast<float*>(route_raw + L.g);              // [C]
+  float* recv = reinterpret_cast<float*>(route_raw + L.recv);        // rank 0: [nsplit][n or C]
+  float* brs = reinterpret_cast<float*>(route_raw + L.brs);          // [n]
+  float* z = reinterpret_cast<float*>(route_raw + L.z);              // [n]
+  const uint32_t ring = smem_u32(route_raw + L.ring);
+  const uint32_t bar0 = smem_u32(route_raw + L.bars);
+  const uint32_t wrbar = bar0 + 16;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(route_raw + L.flag);
+  const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
+
   const int nv = C / VEC;                                  // vectors per pixel
   const int tpp = nv < kRouteThreads ? nv : kRouteThreads;  // threads per pixel
   const int lanes_p = kRouteThreads / tpp;                  // pixels in flight per step
-  const bool wr_in_smem = static_cast<size_t>(p.n) * C <= 8192;
-  float* partial = route_smem;                                  // [lanes_p][C]
-  float* sums = partial + static_cast<size_t>(lanes_p) * C;     // [nsplit][C], rank 0 only
-  float* g = sums + static_cast<size_t>(nsplit) * C;            // [C]
-  float* wr_s = g + C;                                          // [n][C] if it fits
-  float* br_s = wr_s + (wr_in_smem ? static_cast<size_t>(p.n) * C : 0);  // [n]
-  float* z = br_s + p.n;                                        // [n]
+  const int pl = t / tpp;
+  const size_t row_bytes = static_cast<size_t>(C) * sizeof(T);
 
-  // ---- this CTA's pixel slice: all loads first, then the adds
+  // ---- this CTA's pixel slice
   const int p_begin = static_cast<int>((static_cast<long long>(p.HW) * rank) / nsplit);
   const int p_end = static_cast<int>((static_cast<long long>(p.HW) * (rank + 1)) / nsplit);
-  const T* xb = static_cast<const T*>(p.x) + static_cast<size_t>(b) * p.HW * C;
-  const int pl = t / tpp;
-  if (pl < lanes_p) {
-    for (int v = t % tpp; v < nv; v += tpp) {
+  const int npx = p_end - p_begin;
+  const unsigned char* src =
+      static_cast<const unsigned char*>(p.x) + (static_cast<size_t>(b) * p.HW + p_begin) * row_bytes;
+  const int piece_px = p.piece_px;
+  const int npieces = (kBulk && piece_px > 0) ? (npx + piece_px - 1) / piece_px : 0;
+  const size_t piece_bytes = static_cast<size_t>(piece_px) * row_bytes;
+  int issued = 0;  // pieces issued (thread 0 only)
+  auto issue = [&](int k) {
+    ++issued;
+    const int px = min(piece_px, npx - k * piece_px);
+    const uint32_t bytes = static_cast<uint32_t>(px * row_bytes);
+    mbar_arrive_expect_tx(bar0 + 8u * (k & 1), bytes);
+    bulk_load(ring + static_cast<uint32_t>((k & 1) * piece_bytes), src + k * piece_bytes, bytes,
+              bar0 + 8u * (k & 1));
+  };
+
+  if (t == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+    mbar_init(wrbar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    if (p.wr_smem) {
+      const uint32_t wb = static_cast<uint32_t>(p.n) * C * 4u;
+      mbar_arrive_expect_tx(wrbar, wb);
+      bulk_load(smem_u32(wr_s), p.Wr, wb, wrbar);
+    }
+    for (int k = 0; k < npieces && k < 2; ++k) issue(k);
+  }
+  if (rank == 0)
+    for (int i = t; i < p.n; i += kRouteThreads) brs[i] = p.br ? p.br[i] : 0.f;
+  __syncthreads();
+
+  // ---- per-thread channel sums over the slice, fixed order
+  if (npieces > 0) {
+    // bulk path: one channel vector per thread (nv <= 256), pieces consumed in order
+    const int v = t % tpp;
+    const bool active = pl < lanes_p;
+    float acc[VEC];
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
+    for (int k = 0; k < npieces; ++k) {
+      const bool ok = wait_bounded(bar0 + 8u * (k & 1), static_cast<uint32_t>(k >> 1) & 1u, ctl,
+                                   kErrWaitRoute);
+      if (ok && active) {
+        const int pk = min(piece_px, npx - k * piece_px);
+        const unsigned char* base = route_raw + L.ring + (k & 1) * piece_bytes;
+        for (int px = pl; px < pk; px += lanes_p)
+          add_vec<T, VEC>(base + px * row_bytes + v * (VEC * sizeof(T)), acc);
+      }
+      __syncthreads();  // every reader is done with this slot
+      if (t == 0 && k + 2 < npieces && ok) issue(k + 2);
+    }
+    if (active) {
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) partial[static_cast<size_t>(pl) * C + v * VEC + j] = acc[j];
+    }
+  } else {
+    // register path: rows that are not 16-byte multiples, or very wide rows
+    const T* xb = reinterpret_cast<const T*>(src);
+    for (int v = t % tpp; v < nv && pl < lanes_p; v += tpp) {
       float acc[VEC];
 #pragma unroll
       for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
-      // batches of 16 loads issued back to back, then added in a fixed order
-      for (int px = p_begin + pl; px < p_end; px += 16 * lanes_p) {
-        RawVec<T, VEC> raw[16];
-#pragma unroll
-        for (int uu = 0; uu < 16; ++uu) {
-          const int pp = px + uu * lanes_p;
-          if (pp < p_end) load_raw<T, VEC>(xb + static_cast<size_t>(pp) * C + v * VEC, raw[uu]);
-        }
-#pragma unroll
-        for (int uu = 0; uu < 16; ++uu)
-          if (px + uu * lanes_p < p_end) add_raw<T, VEC>(raw[uu], acc);
-      }
+      for (int px = pl; px < npx; px += lanes_p)
+        add_vec<T, VEC>(xb + static_cast<size_t>(px) * C + v * VEC, acc);
 #pragma unroll
       for (int j = 0; j < VEC; ++j) partial[static_cast<size_t>(pl) * C + v * VEC + j] = acc[j];
     }
   }
-  // rank 0: router weights into shared memory while the loads are in flight
-  if (rank == 0) {
-    if (wr_in_smem)
-      for (int e = t; e < p.n * C; e += kRouteThreads) wr_s[e] = p.Wr[e];
-    for (int i = t; i < p.n; i += kRouteThreads) br_s[i] = p.br ? p.br[i] : 0.f;
-  }
   __syncthreads();
-  // fixed-order reduction over the pixel lanes, pushed into rank 0's slot for this rank
-  float* dst = cluster.map_shared_rank(sums, 0) + static_cast<size_t>(rank) * C;
   for (int c = t; c < C; c += kRouteThreads) {
     float s = 0.f;
     for (int l = 0; l < lanes_p; ++l) s += partial[static_cast<size_t>(l) * C + c];
-    dst[c] = s;
+    g[c] = s;
+  }
+  __syncthreads();
+
+  const int warp = t >> 5, lane = t & 31;
+  if (p.wr_smem) {
+    // partial logits of this slice, pushed into rank 0's slot for this rank
+    const bool ok = wait_bounded(wrbar, 0, ctl, kErrWaitRoute);
+    float* dst = cluster.map_shared_rank(recv, 0) + static_cast<size_t>(rank) * p.n;
+    for (int i = warp; i < p.n; i += kRouteThreads / 32) {
+      float s = 0.f;
+      if (ok)
+        for (int c = lane; c < C; c += 32) s = fmaf(wr_s[static_cast<size_t>(i) * C + c], g[c], s);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) dst[i] = s;
+    }
+  } else {
+    float* dst = cluster.map_shared_rank(recv, 0) + static_cast<size_t>(rank) * C;
+    for (int c = t; c < C; c += kRouteThreads) dst[c] = g[c];
   }
   cluster.sync();  // remote stores visible to rank 0; peers may exit after this
+  if (*abort_flag && t == 0) {
+    // a bounded wait gave up: let the copies still in flight land before exit
+    for (int k = (issued > 2 ? issued - 2 : 0); k < issued; ++k)
+      wait_drain(bar0 + 8u * (k & 1), static_cast<uint32_t>(k >> 1) & 1u, p.wait_ns, p.err);
+    if (p.wr_smem) wait_drain(wrbar, 0, p.wait_ns, p.err);
+  }
   if (rank != 0) return;
 
   const float inv_hw = 1.0f / static_cast<float>(p.HW);
-  for (int c = t; c < C; c += kRouteThreads) {
-    float s = 0.f;
-    for (int r = 0; r < nsplit; ++r) s += sums[static_cast<size_t>(r) * C + c];
-    g[c] = s * inv_hw;
-  }
-  __syncthreads();
-  const int warp = t >> 5, lane = t & 31;
-  for (int i = warp; i < p.n; i += kRouteThreads / 32) {
-    const float* wr = wr_in_smem ? wr_s + static_cast<size_t>(i) * C : p.Wr + static_cast<size_t>(i) * C;
-    float s = 0.f;
-    for (int c = lane; c < C; c += 32) s = fmaf(wr[c], g[c], s);
+  if (p.wr_smem) {
+    for (int i = t; i < p.n; i += kRouteThreads) {
+      float s = 0.f;
+      for (int r = 0; r < nsplit; ++r) s += recv[static_cast<size_t>(r) * p.n + i];
+      z[i] = s * inv_hw + brs[i];
+    }
+  } else {
+    for (int c = t; c < C; c += kRouteThreads) {
+      float s = 0.f;
+      for (int r = 0; r < nsplit; ++r) s += recv[static_cast<size_t>(r) * C + c];
+      g[c] = s * inv_hw;
+    }
+    __syncthreads();
+    for (int i = warp; i < p.n; i += kRouteThreads / 32) {
+      const float* wr = p.Wr + static_cast<size_t>(i) * C;
+      float s = 0.f;
+      for (int c = lane; c < C; c += 32) s = fmaf(wr[c], g[c], s);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) z[i] = s + br_s[i];
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) z[i] = s + brs[i];
+    }
   }
   __syncthreads();
 
