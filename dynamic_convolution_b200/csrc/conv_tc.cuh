@@ -373,41 +373,63 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     if (wait_bounded(accum_bar, 0, ctl, kErrWaitEpilogue)) {
       tc_fence_after();
-      // per-warp 32 px x 32 co bf16 staging tile in the (now idle) A stage buffers
+      // Per warp: chunks of 32 pixels x 32 output channels. The next chunk's
+      // TMEM load is in flight while this one is rounded, transposed through a
+      // 2 KB staging tile in the (now idle) A stage buffers, and written as
+      // 16-byte NHWC segments. Pixel coordinates on the padded grid advance
+      // incrementally (one division per chunk).
       const uint32_t stage = a_base + (warp - kTcMixWarp0) * 2048;
       const int n_pad = p.n_mma0 + p.n_mma1;
       const int nchunks = (n_pad + 31) / 32;
-      for (int ch = half; ch < nchunks; ch += 2) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ch * 32, r);
-        tmem_ld_wait();
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+      const int part = lane & 3;  // 16-byte part of a pixel's 64-byte row
+      const int c8 = m0 + 32 * q + part * 8;
+      const bool c_ok = c8 < p.Cout;
+      __nv_bfloat16* ybase = p.y + static_cast<size_t>(b) * p.H * p.W * p.Cout + c8;
+      auto process = [&](const uint32_t (&r)[32], int ch) {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(r[jj]) + bb);
+        for (int jj = 0; jj < 32; jj += 2) {
+          const uint32_t w = pack_bf16x2(__uint_as_float(r[jj]) + bb, __uint_as_float(r[jj + 1]) + bb);
           asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + jj * 64 + lane * 2),
-                       "h"(*reinterpret_cast<const unsigned short*>(&h))
+                       "h"(static_cast<unsigned short>(w & 0xFFFFu))
+                       : "memory");
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + (jj + 1) * 64 + lane * 2),
+                       "h"(static_cast<unsigned short>(w >> 16))
                        : "memory");
         }
         __syncwarp();
+        int pix = ch * 32 + (lane >> 2);
+        int rr = pix / p.Wp;
+        int cw = pix - rr * p.Wp;
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
-          const int jj = it * 8 + (lane >> 2);   // pixel within the chunk
-          const int part = lane & 3;             // 16-byte part of the 64-byte row
-          const int pix = ch * 32 + jj;
-          const int rr = pix / p.Wp, cw = pix % p.Wp;
           const int oh = h0 + rr;
-          const int c8 = m0 + 32 * q + part * 8;
-          if (pix < p.n_virt && cw < p.W && oh < p.H && c8 < p.Cout) {
+          if (c_ok && pix < p.n_virt && cw < p.W && oh < p.H) {
             uint4 v;
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                         : "r"(stage + jj * 64 + part * 16));
-            __nv_bfloat16* dst =
-                p.y + ((static_cast<size_t>(b) * p.H + oh) * p.W + cw) * p.Cout + c8;
-            *reinterpret_cast<uint4*>(dst) = v;
+                         : "r"(stage + (it * 8 + (lane >> 2)) * 64 + part * 16));
+            *reinterpret_cast<uint4*>(ybase + (static_cast<size_t>(oh) * p.W + cw) * p.Cout) = v;
           }
+          pix += 8;
+          cw += 8;
+          while (cw >= p.Wp) { cw -= p.Wp; ++rr; }
         }
         __syncwarp();
+      };
+      uint32_t ra[32], rb[32];
+      int ch = half;
+      if (ch < nchunks) tmem_ld_32x32b_x32(trow + ch * 32, ra);
+      while (ch < nchunks) {
+        tmem_ld_wait(ra);
+        if (ch + 2 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 2) * 32, rb);
+        process(ra, ch);
+        ch += 2;
+        if (ch >= nchunks) break;
+        tmem_ld_wait(rb);
+        if (ch + 2 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 2) * 32, ra);
+        process(rb, ch);
+        ch += 2;
       }
     }
   }

@@ -95,15 +95,16 @@ __global__ void __launch_bounds__(kPsThreads) premix_small_kernel(PsParams p) {
   }
 }
 
-// Host-side plan: samples per thread chosen so that there are about four
-// threads' worth of items per SM slot, fewer samples per thread when the
-// kernel is small. Returns false when the shape is outside this kernel.
+// Host-side plan: as many samples per thread (up to 16) as keep at least one
+// CTA's worth of items per SM, so that the grid runs in a single wave (fewer
+// samples per thread when the kernel is small). Returns false when the shape
+// is outside this kernel.
 inline bool plan_premix_small(int B, int n, long long wsize, int sms, PsParams* p,
                               unsigned* grid) {
   if (n < 1 || n > kPsMaxExperts || B < 1 || wsize % 8 != 0) return false;
   if (static_cast<long long>(B) * n * 4 > 16384) return false;
   const long long chunks = wsize / 8;
-  const long long target = static_cast<long long>(sms) * 2 * kPsThreads;
+  const long long target = static_cast<long long>(sms) * kPsThreads;
   int sblock = 16;
   while (sblock > 1 && chunks * ((B + sblock - 1) / sblock) < target) sblock >>= 1;
   p->B = B;

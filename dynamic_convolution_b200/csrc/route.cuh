@@ -117,6 +117,8 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
   // the forward kernel may be scheduled as soon as every routing CTA runs; it
   // waits for this grid's completion before it reads alpha
   grid_launch_dependents();
+  // launched with a programmatic edge: the set-up below reads no global
+  // memory; x, Wr, br and alpha are touched only after the wait
 
   extern __shared__ __align__(128) unsigned char route_raw[];
   const int C = p.C;
@@ -165,6 +167,9 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
     mbar_init(wrbar, 1);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  grid_dependency_wait();
+  if (t == 0) {
     if (p.wr_smem) {
       const uint32_t wb = static_cast<uint32_t>(p.n) * C * 4u;
       mbar_arrive_expect_tx(wrbar, wb);
@@ -172,8 +177,6 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
     }
     for (int k = 0; k < npieces && k < 2; ++k) issue(k);
   }
-  if (rank == 0)
-    for (int i = t; i < p.n; i += kRouteThreads) brs[i] = p.br ? p.br[i] : 0.f;
   __syncthreads();
 
   // ---- per-thread channel sums over the slice, fixed order
@@ -213,6 +216,8 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
       for (int j = 0; j < VEC; ++j) partial[static_cast<size_t>(pl) * C + v * VEC + j] = acc[j];
     }
   }
+  if (rank == 0)  // read now: its latency overlaps the reductions below
+    for (int i = t; i < p.n; i += kRouteThreads) brs[i] = p.br ? p.br[i] : 0.f;
   __syncthreads();
   for (int c = t; c < C; c += kRouteThreads) {
     float s = 0.f;
