@@ -14,10 +14,11 @@ over ranks.
 
 Timing: inputs are rotated over enough x/alpha/y buffer sets that their total
 footprint exceeds the 126 MB L2, so each step starts cold in L2. The K timed
-steps run as CUDA-graph replays (8 steps per graph: 8 routing launches, then 8
-forward launches) with CUDA events between the graphs, bracketed by a barrier
-and a device synchronisation; the events also give the per-kernel average
-launch durations used for the roofline.
+steps run as CUDA-graph replays (8 steps per graph, each step routing then
+forward of one set), bracketed by a barrier and a device synchronisation. A
+second timed pass of K/4 steps replays 8 routing launches, then 8 forward
+launches, with CUDA events between the graphs: it gives the per-call average
+durations used for the roofline and the route/forward breakdown.
 """
 from __future__ import annotations
 
@@ -308,11 +309,23 @@ def run_ours(args, cfg):
     st = dc.dynconv_device_status(stream)
     dc.check(st, "device status after warm-up")
 
-    # graphs: all routes of a group of sets, then all forwards of the same group
+    # Timed graphs: each step is route(s) then forward(s) of one input set, as a
+    # layer runs in a network (the forward reads x while the routing kernel
+    # left it in L2; the routing -> mixing edge is programmatic). A second,
+    # shorter timed pass replays all routes of a group, then all forwards, so
+    # that CUDA events between the two graphs give each call's duration.
     G = min(8, nsets)
     groups = [list(range(g, min(g + G, nsets))) for g in range(0, nsets, G)]
-    graphs = []
+    steps_graphs, split_graphs = [], []
     n0 = dc.dynconv_launch_count()
+    for grp in groups:
+        gs = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gs, stream=stream):
+            for s in grp:
+                route(s, stream)
+                forward(s, stream)
+        steps_graphs.append((gs, len(grp)))
+    launches_per_step = (dc.dynconv_launch_count() - n0) / nsets
     for grp in groups:
         gr, gf = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=stream):
@@ -321,17 +334,17 @@ def run_ours(args, cfg):
         with torch.cuda.graph(gf, stream=stream):
             for s in grp:
                 forward(s, stream)
-        graphs.append((gr, gf, len(grp)))
-    launches_per_step = (dc.dynconv_launch_count() - n0) / nsets
+        split_graphs.append((gr, gf, len(grp)))
     tails = {}
     for s in range(nsets):  # single-step graphs for an exact step count
-        gr, gf = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=stream):
+        gt = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gt, stream=stream):
             route(s, stream)
-        with torch.cuda.graph(gf, stream=stream):
             forward(s, stream)
-        tails[s] = (gr, gf)
-    for gr, gf, _ in graphs:  # warm the graphs
+        tails[s] = gt
+    for gs, _ in steps_graphs:  # warm the graphs
+        gs.replay()
+    for gr, gf, _ in split_graphs:
         gr.replay()
         gf.replay()
     torch.cuda.synchronize()
@@ -341,17 +354,16 @@ def run_ours(args, cfg):
     k = 0
     gi = 0
     while k < args.steps:
-        gr, gf, m = graphs[gi % len(graphs)]
+        gs, m = steps_graphs[gi % len(steps_graphs)]
         if k + m <= args.steps:
-            plan.append((gr, gf, m))
+            plan.append(gs)
             k += m
         else:
             for s in range(args.steps - k):
-                trg, tfg = tails[s]
-                plan.append((trg, tfg, 1))
+                plan.append(tails[s])
             k = args.steps
         gi += 1
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(plan) + 1)]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     sampler = ClockSampler(dev)
     if world > 1:
@@ -360,22 +372,41 @@ def run_ours(args, cfg):
     sampler.start()
     time.sleep(0.2)
     with torch.cuda.stream(stream):
-        ev[0].record(stream)
-        for i, (gr, gf, m) in enumerate(plan):
-            gr.replay()
-            ev[2 * i + 1].record(stream)
-            gf.replay()
-            ev[2 * i + 2].record(stream)
+        ev0.record(stream)
+        for gs in plan:
+            gs.replay()
+        ev1.record(stream)
     stream.synchronize()
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    total_ms = ev[0].elapsed_time(ev[-1])
-    route_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(len(plan)))
-    fwd_ms = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(len(plan)))
+    total_ms = ev0.elapsed_time(ev1)
     st = dc.dynconv_device_status(stream)
     dc.check(st, "device status after timing")
+
+    # per-call durations (routing, forward) from the split pass
+    split_groups = max(1, (args.steps // 4) // G)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * split_groups + 1)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        ev[0].record(stream)
+        for i in range(split_groups):
+            gr, gf, m = split_graphs[i % len(split_graphs)]
+            gr.replay()
+            ev[2 * i + 1].record(stream)
+            gf.replay()
+            ev[2 * i + 2].record(stream)
+    stream.synchronize()
+    split_steps = sum(split_graphs[i % len(split_graphs)][2] for i in range(split_groups))
+    route_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(split_groups))
+    fwd_ms = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(split_groups))
+    route_ms *= args.steps / split_steps  # scaled to K steps, like total_ms
+    fwd_ms *= args.steps / split_steps
+    st = dc.dynconv_device_status(stream)
+    dc.check(st, "device status after the split pass")
 
     total_ms, fwd_ms, route_ms = multi.max_over_ranks([total_ms, fwd_ms, route_ms], device="cuda")
 
@@ -408,7 +439,7 @@ def run_ours(args, cfg):
             dist.destroy_process_group()
         return 0
 
-    del graphs, tails
+    del steps_graphs, split_graphs, tails, plan
     peaks, peak_kind = measured_peaks()
     K = args.steps
     value = multi.weak_scaling_rate(cfg.B * K, world, total_ms / 1e3)
