@@ -20,7 +20,7 @@
 #include "direct.cuh"
 #include "premix.cuh"
 #include "premix_small.cuh"
-#include "layer_tc.cuh"
+#include "mixconv.cuh"
 #include "route.cuh"
 
 namespace {
@@ -33,6 +33,8 @@ __device__ int g_device_err;
 // a device address: dynconv_forward_noalloc looks the address up on its first
 // call on each device and keeps it in g_noalloc_ptr.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[DYNCONV_NOALLOC_MAX_BYTES];
+// State slots of the streamed mixing (slice counters), zero between launches.
+static __device__ __align__(256) unsigned int g_mix_state[dc::kMcSlots][dc::kMcStateWords];
 
 constexpr long long kDefaultWaitNs = 500LL * 1000 * 1000;  // 0.5 s
 constexpr int kMaxDevices = 64;
@@ -54,7 +56,7 @@ std::atomic<long long> g_wait_ns{kDefaultWaitNs};
 std::atomic<int> g_inject_skip{0};
 std::atomic<int> g_route_split{0};  // 0: automatic
 std::atomic<int> g_use_pdl{1};      // programmatic launch edges on forward kernels
-std::atomic<int> g_fused_premix{0}; // PREMIX as one persistent kernel (else two kernels)
+std::atomic<int> g_stream_mix{1};   // PREMIX with n <= 8: mixing streamed into the convolution
 std::atomic<int> g_premix_mixer{0};  // 0 automatic, 1 tensor-core GEMM, 2 CUDA cores (n <= 8)
 thread_local char g_last_err[256] = "";
 
@@ -267,15 +269,14 @@ bool depthwise_ok(const dynconv_desc* d) {
          out_size(d->W, d->KW, 1, d->pad) >= 1;
 }
 
-// Workspace of PREMIX: the mixed kernels of every sample, then (256-byte
-// aligned) one word for the fused kernel's grid barrier.
+// Workspace of PREMIX: the mixed kernels of every sample (256-byte aligned).
 size_t premix_wb_bytes(const dynconv_desc* d) {
   return (static_cast<size_t>(d->B) * d->C_out * d->KH * d->KW * d->C_in * 2 + 255) & ~size_t(255);
 }
 size_t premix_workspace(const dynconv_desc* d) {
   if (!tc_shape_ok(d)) return 0;
   if (!dc::premix_shape_ok(d->B, d->n, d->C_out, d->KH * d->KW, d->C_in)) return 0;
-  return premix_wb_bytes(d) + 256;
+  return premix_wb_bytes(d);
 }
 
 // Cost-model choice among the kernels that can run this descriptor.
@@ -370,103 +371,132 @@ int launch_tc(const TcPlan& plan, const CUtensorMap& xmap, const CUtensorMap& wm
   return check_launch("tc_conv_kernel");
 }
 
-// Grid-barrier words already zeroed on some stream (per device and address).
-// Cleared when a bounded wait expires, because an aborted launch can leave
-// the words mid-barrier.
-std::mutex g_bar_mu;
-std::map<std::pair<int, const void*>, bool> g_bar_ready;
 
-bool barrier_words_need_reset(const void* words) {
+// State slot of the streamed mixing for (device, stream): launches on one
+// stream are ordered, so they may share a slot; streams get slots of their
+// own (least recently used first when there are more streams than slots).
+std::mutex g_slot_mu;
+std::map<std::pair<int, void*>, std::pair<int, unsigned long long>> g_slot_of;
+unsigned long long g_slot_tick = 0;
+bool g_slots_dirty[64] = {};  // per device: a bounded wait expired, zero all slots
+
+int mix_state_slot(void* stream, unsigned int** out, cudaStream_t s) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return true;
-  std::lock_guard<std::mutex> lk(g_bar_mu);
-  auto key = std::make_pair(dev, words);
-  if (g_bar_ready.count(key)) return false;
-  g_bar_ready[key] = true;
-  return true;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  void* base = nullptr;
+  e = cudaGetSymbolAddress(&base, g_mix_state);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(mixing state)");
+  std::lock_guard<std::mutex> lk(g_slot_mu);
+  if (dev >= 0 && dev < 64 && g_slots_dirty[dev]) {
+    e = cudaMemsetAsync(base, 0, sizeof(g_mix_state), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(mixing state)");
+    g_slots_dirty[dev] = false;
+  }
+  const auto key = std::make_pair(dev, stream);
+  auto it = g_slot_of.find(key);
+  int slot = -1;
+  if (it != g_slot_of.end()) {
+    slot = it->second.first;
+  } else {
+    bool used[dc::kMcSlots] = {};
+    auto lru = g_slot_of.end();
+    for (auto jt = g_slot_of.begin(); jt != g_slot_of.end(); ++jt) {
+      if (jt->first.first != dev) continue;
+      used[jt->second.first] = true;
+      if (lru == g_slot_of.end() || jt->second.second < lru->second.second) lru = jt;
+    }
+    for (int i = 0; i < dc::kMcSlots && slot < 0; ++i)
+      if (!used[i]) slot = i;
+    if (slot < 0) {
+      slot = lru->second.first;
+      g_slot_of.erase(lru);
+    }
+  }
+  g_slot_of[key] = std::make_pair(slot, ++g_slot_tick);
+  *out = static_cast<unsigned int*>(base) + static_cast<size_t>(slot) * dc::kMcStateWords;
+  return DYNCONV_OK;
 }
 
-void barrier_words_forget_all() {
-  std::lock_guard<std::mutex> lk(g_bar_mu);
-  g_bar_ready.clear();
-}
-
-// PREMIX as one persistent cooperative kernel: returns DYNCONV_ERR_UNSUPPORTED
-// (and launches nothing) when the two phases cannot share one CTA per SM.
-int run_fused_premix(const dynconv_desc* d, const TcPlan& plan_in, const DeviceState* st,
-                     const void* x, const void* experts, const float* alpha, const float* bias,
-                     void* y, void* ws, const CUtensorMap& xmap, const CUtensorMap& wmap,
-                     cudaStream_t stream) {
-  dc::FusedParams fp{};
-  fp.cv = plan_in.p;
-  dc::PremixLaunch pl;
-  int rc = dc::plan_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
-                           static_cast<__nv_bfloat16*>(ws), d->B, d->n,
-                           static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in, st->err,
-                           g_wait_ns.load(), st->sms, g_encode, &pl);
-  if (rc == -2) {
-    std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(premix) failed");
-    return DYNCONV_ERR_CUDA;
-  }
-  if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
-  fp.pm = pl.p;
-  // shared memory: activation stages (own region) | region used by the mixing
-  // phase, then by the convolution's weight stages + epilogue staging | barriers
-  const size_t b_region = static_cast<size_t>(fp.cv.sb) * fp.cv.b_tile_bytes;
-  const size_t fixed = 1024 + 16 + 64;
-  const size_t budget = static_cast<size_t>(st->max_smem_optin) - fixed - b_region;
-  size_t pm_region = 0;
-  for (;; --fp.pm.stages) {  // as many mixing stages as fit (at least 2)
-    pm_region = (static_cast<size_t>(fp.pm.a_bytes) +
-                 static_cast<size_t>(fp.pm.stages) * fp.pm.stage_bytes + 4 * dc::kFusedPmStage +
-                 4 * static_cast<size_t>(d->B) * d->n + 1023) & ~size_t(1023);
-    if (fp.pm.stages <= 2 || pm_region + 8 * 64 <= budget) break;
-  }
-  int sa = fp.cv.sa;
-  size_t cv_region = 0, total = 0;
+// PREMIX with the mixing streamed into the convolution (one persistent
+// cooperative kernel, n <= 8). Returns DYNCONV_ERR_UNSUPPORTED (and launches
+// nothing) when the shape is outside it.
+int run_mixconv(const dynconv_desc* d, const TcPlan& plan_in, const DeviceState* st,
+                const void* experts, const float* alpha, const float* bias, void* y, void* ws,
+                const CUtensorMap& xmap, const CUtensorMap& wmap, cudaStream_t stream) {
+  if (d->n > dc::kMcMaxExperts || plan_in.p.k_steps > dc::kMcMaxSlices) return DYNCONV_ERR_UNSUPPORTED;
+  if (static_cast<size_t>(d->B) * d->n * 4 > 16384 || d->C_in % 8 != 0) return DYNCONV_ERR_UNSUPPORTED;
+  if (!aligned16(experts)) return DYNCONV_ERR_UNSUPPORTED;
+  dc::MixParams mp{};
+  mp.cv = plan_in.p;
+  mp.wsize = static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in;
+  // items: 8 weights x up to 16 samples; fewer samples per item when a whole
+  // grid of mixer threads would otherwise get less than one item
+  const long long threads = static_cast<long long>(st->sms) * 256;
+  int sblock = 16;
+  while (sblock > 1 &&
+         1LL * mp.cv.k_steps * ((d->B + sblock - 1) / sblock) * d->C_out * 8 < threads)
+    sblock >>= 1;
+  sblock = std::min(sblock, d->B);
+  mp.sblock = sblock;
+  mp.nsb = (d->B + sblock - 1) / sblock;
+  mp.ips = mp.nsb * d->C_out * 8;
+  mp.total_items = 1LL * mp.cv.k_steps * mp.ips;
+  mp.units = plan_in.grid;
+  // shared memory from the 1024-aligned base: A stages | B stages | epilogue
+  // staging | alpha | barriers
+  const size_t b_bytes = static_cast<size_t>(mp.cv.sb) * mp.cv.b_tile_bytes;
+  const size_t alpha_bytes = (static_cast<size_t>(d->B) * d->n * 4 + 15) & ~size_t(15);
+  size_t total = 0;
+  int sa = 8;
   for (; sa >= 2; --sa) {
-    cv_region = static_cast<size_t>(sa) * dc::kTcATileBytes + dc::kFusedEpiStage;
-    const size_t region = std::max(pm_region, cv_region);
-    const size_t bars = 8 * (2 * fp.pm.stages + 4 + 2 * sa + 2 * fp.cv.sb + 3);
-    total = fixed + b_region + region + bars;
+    const size_t bar_off = static_cast<size_t>(sa) * dc::kTcATileBytes + b_bytes + dc::kMcEpiStage + alpha_bytes;
+    total = 1024 + bar_off + 8 * (2 * sa + 2 * mp.cv.sb + 3) + 16;
     if (total <= static_cast<size_t>(st->max_smem_optin)) break;
   }
   if (sa < 2) return DYNCONV_ERR_UNSUPPORTED;
-  fp.cv.sa = sa;
-  fp.region_bytes = static_cast<int>(std::max(pm_region, cv_region));
-  fp.cv.experts = static_cast<const __nv_bfloat16*>(experts);
-  fp.cv.alpha = alpha;
-  fp.cv.bias = bias;
-  fp.cv.y = static_cast<__nv_bfloat16*>(y);
-  fp.cv.err = st->err;
-  fp.cv.wait_ns = g_wait_ns.load();
-  fp.units = plan_in.grid;
-  fp.grid_bar = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + premix_wb_bytes(d));
+  mp.cv.sa = sa;
+  mp.stage_off = static_cast<int>(static_cast<size_t>(sa) * dc::kTcATileBytes + b_bytes);
+  mp.alpha_off = mp.stage_off + dc::kMcEpiStage;
+  mp.bar_off = static_cast<int>(mp.alpha_off + alpha_bytes);
+  mp.cv.experts = static_cast<const __nv_bfloat16*>(experts);
+  mp.cv.alpha = alpha;
+  mp.cv.bias = bias;
+  mp.cv.y = static_cast<__nv_bfloat16*>(y);
+  mp.cv.err = st->err;
+  mp.cv.wait_ns = g_wait_ns.load();
+  mp.wb = static_cast<__nv_bfloat16*>(ws);
+  int rc = mix_state_slot(static_cast<void*>(stream), &mp.state, stream);
+  if (rc) return rc;
   cudaError_t e = cudaSuccess;
-  if (barrier_words_need_reset(fp.grid_bar)) {
-    // the barrier resets itself after every use; only a workspace seen for the
-    // first time (or after a timeout) needs its two words zeroed
-    e = cudaMemsetAsync(fp.grid_bar, 0, 2 * sizeof(unsigned int), stream);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(grid barrier words)");
-  }
-  e = ensure_smem(dc::premix_conv_kernel, total);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix_conv)");
+  auto kern = d->n <= 2 ? dc::mixconv_kernel<2>
+              : d->n <= 4 ? dc::mixconv_kernel<4> : dc::mixconv_kernel<8>;
+  e = ensure_smem(kern, total);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(mixconv)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(st->sms);
-  cfg.blockDim = dim3(dc::kFusedThreads);
+  cfg.blockDim = dim3(dc::kMcThreads);
   cfg.dynamicSmemBytes = total;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, dc::premix_conv_kernel, pl.emap, xmap, wmap, fp);
+  cfg.numAttrs = g_use_pdl.load() ? 2 : 1;
+  e = cudaLaunchKernelEx(&cfg, kern, xmap, wmap, mp);
+  if (e != cudaSuccess && cfg.numAttrs == 2) {
+    // a cooperative launch that does not take the programmatic edge: plain order
+    (void)cudaGetLastError();
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, xmap, wmap, mp);
+  }
   if (e != cudaSuccess) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    return cuda_fail(e, "premix_conv_kernel launch");
+    return cuda_fail(e, "mixconv_kernel launch");
   }
-  return check_launch("premix_conv_kernel");
+  return check_launch("mixconv_kernel");
 }
 
 int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void* x,
@@ -493,10 +523,10 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   if (!ws || ws_bytes < need) return DYNCONV_ERR_WORKSPACE;
   if (!aligned16(ws)) return DYNCONV_ERR_MISALIGNED;
   plan.p.inject_skip = 0;
-  if (g_fused_premix.load()) {
+  if (g_stream_mix.load() && g_premix_mixer.load() != 1 && d->n <= dc::kMcMaxExperts) {
     rc = encode_w_map(&wmap, ws, d);
     if (rc) return rc;
-    rc = run_fused_premix(d, plan, st, x, experts, alpha, bias, y, ws, xmap, wmap, stream);
+    rc = run_mixconv(d, plan, st, experts, alpha, bias, y, ws, xmap, wmap, stream);
     if (rc != DYNCONV_ERR_UNSUPPORTED) return rc;
   }
   // few experts: the store-bound CUDA-core mixer (no set-up chain)
@@ -598,7 +628,7 @@ int dynconv_test_hook(int key, long long value) {
   }
   if (key == 6) {
     if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
-    g_fused_premix.store(static_cast<int>(value));
+    g_stream_mix.store(static_cast<int>(value));
     return DYNCONV_OK;
   }
   if (key == 7) {
@@ -877,7 +907,13 @@ int dynconv_device_status(void* stream) {
   e = cudaMemcpyFromSymbol(&word, g_device_err, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e, "read error word");
   if (word != 0) {
-    barrier_words_forget_all();
+    {
+      int dev = 0;
+      if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+        std::lock_guard<std::mutex> lk(g_slot_mu);
+        g_slots_dirty[dev] = true;
+      }
+    }
     const int zero = 0;
     e = cudaMemcpyToSymbol(g_device_err, &zero, sizeof(int));
     if (e != cudaSuccess) return cuda_fail(e, "clear error word");

@@ -118,12 +118,11 @@ int dynconv_route(const dynconv_desc* desc, const void* x, const float* Wr, cons
  *   workspace      device scratch of workspace_bytes bytes, or NULL/0. Only the
  *                  PREMIX variant uses it; AUTO never picks PREMIX unless the
  *                  workspace is large enough. It holds every sample's mixed
- *                  kernel, then (last 256 bytes) the state of a grid barrier:
- *                  the library zeroes that state the first time it sees a
- *                  workspace address on a device (and again after a bounded
- *                  wait expired) and leaves it valid after each call. A caller
- *                  that writes those bytes between calls (reusing the memory for
- *                  other data) zeroes the first 8 of them before the next call.
+ *                  kernel; its contents need not be preserved between calls.
+ *                  (The counters with which the streamed mixing publishes each
+ *                  K slice live in library-owned device memory, one slot per
+ *                  stream, zero between launches; after a bounded wait expired
+ *                  they are re-zeroed when dynconv_device_status reports it.)
  * Precision: bf16 in, fp32 accumulate, the mixed kernel rounded once to bf16
  * (tensor-core variants), y rounded once to bf16. fp32 layers accumulate and
  * mix in fp32.
@@ -207,12 +206,14 @@ unsigned long long dynconv_launch_count(void);
  * stream-serialization edge (they may start while the previous kernel on the
  * stream finishes, and wait for it before reading memory); 0 launches them
  * plainly. For measurements.
- * key 6: 1 runs PREMIX as one persistent cooperative kernel (kernel mixing,
- * grid barrier, convolution); 0 (default) runs it as two kernels.
+ * key 6: 1 (default) runs PREMIX with n <= 8 as one persistent cooperative
+ * kernel that streams the mixing into the convolution (per-K-slice counters in
+ * the workspace); 0 runs it as two kernels (mixing, then convolution).
  * key 7: which kernel mixes the per-sample kernels of the two-kernel PREMIX
  * form: 0 (default) the CUDA-core mixer when n <= 8, else the tensor-core
- * mixing GEMM; 1 always the tensor-core GEMM; 2 the CUDA-core mixer only
- * (forward returns DYNCONV_ERR_UNSUPPORTED when n > 8).
+ * mixing GEMM; 1 always the tensor-core GEMM (and never the streamed kernel of
+ * key 6); 2 the CUDA-core mixer only (forward returns
+ * DYNCONV_ERR_UNSUPPORTED when n > 8).
  * Returns DYNCONV_OK or DYNCONV_ERR_INVALID_ARG. */
 int dynconv_test_hook(int key, long long value);
 

@@ -100,9 +100,9 @@ def test_variant_selection_per_config(lib):
     for name in ("deep_3x3_tau30", "large_n64"):
         d = dc.desc_from_config(synth.CONFIGS[name])
         ws = dc.dynconv_workspace_size(d)
-        # every sample's mixed kernel (256-byte aligned) + 256 bytes of grid-barrier state
+        # every sample's mixed kernel, 256-byte aligned
         wb = (synth.CONFIGS[name].B * synth.CONFIGS[name].weight_elems * 2 + 255) // 256 * 256
-        assert ws == wb + 256
+        assert ws == wb
         assert dc.dynconv_select_variant(d, ws) in (dc.VARIANT_FUSED, dc.VARIANT_OUTSIDE,
                                                      dc.VARIANT_PREMIX)
     # a forced variant is reported as is

@@ -214,11 +214,12 @@ def test_outputs_outside_y_untouched():
     assert torch.all(big[L.y.numel():] == 7.0)
 
 
-@pytest.mark.parametrize("name", ["resnet18_3x3", "effnet_expand_1x1", "large_n64"])
-def test_premix_fused_kernel_equals_two_kernels(name):
-    """PREMIX as one persistent kernel (mixing, grid barrier, convolution; several
-    units per CTA when there are more units than SMs) gives the same bits as the
-    two-kernel form."""
+@pytest.mark.parametrize("name", ["resnet18_3x3", "effnet_expand_1x1"])
+def test_streamed_mixing_equals_two_kernels(name):
+    """PREMIX with the mixing streamed into the convolution (one persistent
+    kernel, per-slice counters) gives the same bits as the two-kernel form with
+    the same CUDA-core mixer, on three consecutive calls (the counters carry
+    over between launches)."""
     inp = layer_inputs(name)
     L = Layer(inp)
     L.route()
@@ -226,17 +227,20 @@ def test_premix_fused_kernel_equals_two_kernels(name):
     ws = torch.zeros(dc.dynconv_workspace_size(d), dtype=torch.uint8, device="cuda")
     outs = []
     try:
-        assert dc.dynconv_test_hook(7, 1) == dc.OK  # both forms mix on tensor cores
-        for fused in (1, 0):
-            assert dc.dynconv_test_hook(6, fused) == dc.OK
-            L.y.fill_(float("nan"))
-            dc.check(dc.dynconv_forward(d, L.x, L.experts, L.alpha, L.bias, L.y, ws, ws.numel()))
-            assert dc.dynconv_device_status(None) == dc.OK
-            outs.append(L.y.clone())
+        for stream_mix, mixer, calls in ((1, 0, 3), (0, 2, 1)):
+            assert dc.dynconv_test_hook(6, stream_mix) == dc.OK
+            assert dc.dynconv_test_hook(7, mixer) == dc.OK
+            for _ in range(calls):
+                L.y.fill_(float("nan"))
+                dc.check(dc.dynconv_forward(d, L.x, L.experts, L.alpha, L.bias, L.y, ws,
+                                            ws.numel()))
+                assert dc.dynconv_device_status(None) == dc.OK
+                outs.append(L.y.clone())
     finally:
-        dc.dynconv_test_hook(6, 0)
+        dc.dynconv_test_hook(6, 1)
         dc.dynconv_test_hook(7, 0)
-    assert torch.equal(outs[0], outs[1])
+    for o in outs[1:]:
+        assert torch.equal(outs[0], o)
     assert torch.isfinite(outs[0].float()).all()
 
 
