@@ -56,7 +56,7 @@ std::atomic<long long> g_wait_ns{kDefaultWaitNs};
 std::atomic<int> g_inject_skip{0};
 std::atomic<int> g_route_split{0};  // 0: automatic
 std::atomic<int> g_use_pdl{1};      // programmatic launch edges on forward kernels
-std::atomic<int> g_stream_mix{1};   // PREMIX with n <= 8: mixing streamed into the convolution
+std::atomic<int> g_stream_mix{0};   // PREMIX with n <= 8: mixing streamed into the convolution
 std::atomic<int> g_premix_mixer{0};  // 0 automatic, 1 tensor-core GEMM, 2 CUDA cores (n <= 8)
 thread_local char g_last_err[256] = "";
 

@@ -206,9 +206,9 @@ unsigned long long dynconv_launch_count(void);
  * stream-serialization edge (they may start while the previous kernel on the
  * stream finishes, and wait for it before reading memory); 0 launches them
  * plainly. For measurements.
- * key 6: 1 (default) runs PREMIX with n <= 8 as one persistent cooperative
- * kernel that streams the mixing into the convolution (per-K-slice counters in
- * the workspace); 0 runs it as two kernels (mixing, then convolution).
+ * key 6: 1 runs PREMIX with n <= 8 as one persistent cooperative kernel that
+ * streams the mixing into the convolution (per-K-slice counters); 0 (default)
+ * runs it as two kernels (mixing, then convolution).
  * key 7: which kernel mixes the per-sample kernels of the two-kernel PREMIX
  * form: 0 (default) the CUDA-core mixer when n <= 8, else the tensor-core
  * mixing GEMM; 1 always the tensor-core GEMM (and never the streamed kernel of

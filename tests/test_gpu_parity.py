@@ -169,6 +169,30 @@ def test_small_structured_all_variants(case, variant):
     assert r["ok"], (name, variant, r)
 
 
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_structured_streamed_mixing(case):
+    """The streamed-mixing PREMIX kernel on the ragged small cases (partial
+    channel chunks and channel tiles, odd expert counts, tiny batches)."""
+    name, B, Cin, Cout, H, W, K, pad, n, mode, tau = case
+    cfg = synth.LayerConfig(name, synth.BF16, B, Cin, Cout, H, W, K, K, 1, pad, 1, n, mode, tau)
+    inp = synth.make_inputs(cfg, seed=4, structured=1.5)
+    L = Layer(inp)
+    a32 = alpha_f32_rounded(oracle.route(inp.x_f64, inp.Wr, inp.br, mode, tau))
+    L.alpha.copy_(torch.from_numpy(a32.astype(np.float32)))
+    ws = torch.empty(dc.dynconv_workspace_size(L.desc(dc.VARIANT_PREMIX)) // 2 + 8,
+                     dtype=torch.bfloat16, device="cuda")
+    try:
+        assert dc.dynconv_test_hook(6, 1) == dc.OK
+        L.forward(dc.VARIANT_PREMIX, workspace=ws)
+        torch.cuda.synchronize()
+        assert dc.dynconv_device_status(None) == dc.OK
+    finally:
+        dc.dynconv_test_hook(6, 0)
+    ref = oracle.forward(inp.x_f64, inp.experts_f64, a32, inp.bias, stride=1, pad=pad)
+    r = compare(from_device(L.y), ref, synth.BF16)
+    assert r["ok"], (name, r)
+
+
 @pytest.mark.parametrize("variant", [dc.VARIANT_FUSED, dc.VARIANT_DIRECT])
 def test_no_bias(variant):
     cfg = synth.LayerConfig("nobias", synth.BF16, 2, 64, 64, 7, 7, 3, 3, 1, 1, 1, 3,
@@ -237,7 +261,7 @@ def test_streamed_mixing_equals_two_kernels(name):
                 assert dc.dynconv_device_status(None) == dc.OK
                 outs.append(L.y.clone())
     finally:
-        dc.dynconv_test_hook(6, 1)
+        dc.dynconv_test_hook(6, 0)
         dc.dynconv_test_hook(7, 0)
     for o in outs[1:]:
         assert torch.equal(outs[0], o)
@@ -245,15 +269,18 @@ def test_streamed_mixing_equals_two_kernels(name):
 
 
 @pytest.mark.parametrize("name", ["resnet18_3x3", "effnet_expand_1x1"])
-@pytest.mark.parametrize("mixer", [1, 2])
+@pytest.mark.parametrize("mixer", [(0, 1), (0, 2), (1, 0)], ids=["gemm", "cuda-core", "streamed"])
 def test_premix_mixers_full_size(name, mixer):
-    """PREMIX with each mixing kernel (1: tensor-core GEMM with a hi/lo split
-    of alpha, 2: CUDA-core fp32 mixer) against the oracle on sampled whole
-    samples."""
+    """PREMIX with each mixing kernel (tensor-core GEMM with a hi/lo split of
+    alpha; CUDA-core fp32 mixer; the mixing streamed into the convolution)
+    against the oracle on sampled whole samples."""
+    stream_mix, which = mixer
     try:
-        assert dc.dynconv_test_hook(7, mixer) == dc.OK
+        assert dc.dynconv_test_hook(6, stream_mix) == dc.OK
+        assert dc.dynconv_test_hook(7, which) == dc.OK
         _forward_case(name, dc.VARIANT_PREMIX, workspace=True)
     finally:
+        dc.dynconv_test_hook(6, 0)
         dc.dynconv_test_hook(7, 0)
 
 
