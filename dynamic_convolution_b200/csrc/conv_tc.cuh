@@ -361,10 +361,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0 && !withhold) mbar_arrive(fullA(s));
       }
     }
+  }
 
-    // ======================= epilogue =======================
-    const int q = warp & 3;                      // TMEM lane quarter
-    const int half = (warp - kTcMixWarp0) >> 2;  // column half
+  // ======================= epilogue (all 12 warps) =======================
+  // Warps 0..2 join once their lane 0 is done with its producer / MMA role,
+  // warp 3 has no other role. Warp w reads TMEM lane quarter w % 4 (output
+  // channels 32*(w%4) ..) and every third 32-pixel chunk from w / 4.
+  __syncwarp();
+  {
+    const int q = warp & 3;   // TMEM lane quarter
+    const int grp = warp >> 2;  // chunk phase 0..2
     const int co = m0 + 32 * q + lane;
     float bb = 0.f;
     if (p.bias != nullptr && co < p.Cout) {
@@ -378,7 +384,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // 2 KB staging tile in the (now idle) A stage buffers, and written as
       // 16-byte NHWC segments. Pixel coordinates on the padded grid advance
       // incrementally (one division per chunk).
-      const uint32_t stage = a_base + (warp - kTcMixWarp0) * 2048;
+      const uint32_t stage = a_base + warp * 2048;
       const int n_pad = p.n_mma0 + p.n_mma1;
       const int nchunks = (n_pad + 31) / 32;
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
@@ -418,18 +424,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
       };
       uint32_t ra[32], rb[32];
-      int ch = half;
+      int ch = grp;
       if (ch < nchunks) tmem_ld_32x32b_x32(trow + ch * 32, ra);
       while (ch < nchunks) {
         tmem_ld_wait(ra);
-        if (ch + 2 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 2) * 32, rb);
+        if (ch + 3 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 3) * 32, rb);
         process(ra, ch);
-        ch += 2;
+        ch += 3;
         if (ch >= nchunks) break;
         tmem_ld_wait(rb);
-        if (ch + 2 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 2) * 32, ra);
+        if (ch + 3 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 3) * 32, ra);
         process(rb, ch);
-        ch += 2;
+        ch += 3;
       }
     }
   }

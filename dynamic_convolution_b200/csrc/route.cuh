@@ -253,6 +253,32 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
   if (rank != 0) return;
 
   const float inv_hw = 1.0f / static_cast<float>(p.HW);
+  float* out = p.alpha + static_cast<size_t>(b) * p.n;
+  if (p.wr_smem && p.n <= 32) {
+    // warp 0 alone: lane i sums expert i's partial logits, then the activation
+    if (warp == 0) {
+      float zi = -INFINITY;
+      if (lane < p.n) {
+        float s = 0.f;
+        for (int r = 0; r < nsplit; ++r) s += recv[static_cast<size_t>(r) * p.n + lane];
+        zi = s * inv_hw + brs[lane];
+      }
+      if (p.mode == 0) {
+        if (lane < p.n) out[lane] = 1.0f / (1.0f + expf(-zi));
+      } else {
+        const float zt = lane < p.n ? zi / p.tau : -INFINITY;
+        float m = zt;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float e = lane < p.n ? expf(zt - m) : 0.f;
+        float s = e;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane < p.n) out[lane] = e * (1.0f / s);
+      }
+    }
+    return;
+  }
   if (p.wr_smem) {
     for (int i = t; i < p.n; i += kRouteThreads) {
       float s = 0.f;
@@ -277,7 +303,6 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
   }
   __syncthreads();
 
-  float* out = p.alpha + static_cast<size_t>(b) * p.n;
   if (p.mode == 0) {
     for (int i = t; i < p.n; i += kRouteThreads) out[i] = 1.0f / (1.0f + expf(-z[i]));
   } else if (warp == 0) {
