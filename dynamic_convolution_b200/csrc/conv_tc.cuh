@@ -75,41 +75,7 @@ struct TcParams {
   int* err;
   long long wait_ns;
   int inject_skip;    // test hook: withhold the first mixer arrival of CTA 0
-  // PREMIX hand-off by slice counters instead of kernel completion (null: off):
-  // slot[1] counts finished CTAs, slot[kSliceWord0 + k] the mixed items of
-  // K step k; slices [0, fa) are complete at ta items, the others at tb
-  unsigned int* slot;
-  int fa;
-  unsigned int ta, tb;
 };
-
-constexpr int kSliceWord0 = 64;
-
-__device__ __forceinline__ unsigned int ld_acquire_gpu_u32(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Bounded spin until slice k of the mixed kernels is complete (acquire), then
-// a proxy fence so that the TMA reads issued next see it.
-__device__ __forceinline__ bool wait_slice(const TcParams& p, int k, const WaitCtl& ctl) {
-  const unsigned int target = k < p.fa ? p.ta : p.tb;
-  const unsigned int* c = p.slot + kSliceWord0 + k;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (ld_acquire_gpu_u32(c) >= target) break;
-    if (*ctl.abort_flag) return false;
-    __nanosleep(64);
-    if ((it & 15u) == 15u && static_cast<long long>(globaltimer_ns() - t0) > ctl.limit_ns) {
-      *ctl.abort_flag = 1;
-      atomicCAS(ctl.err, 0, kErrWaitGrid);
-      return false;
-    }
-  }
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  return true;
-}
 
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, int base_mode) {
   uint64_t d = smem_desc_sw128(saddr);
@@ -178,14 +144,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (VARIANT == kPremix) tma_prefetch_desc(&wmap);
   }
   __syncwarp();
-  // With the slice hand-off the kernel starts while the mixing kernel runs and
-  // reads nothing global before slice 0 is published (which happens after the
-  // mixing kernel's own dependency wait); otherwise the dependency wait.
-  const bool handoff = VARIANT == kPremix && p.slot != nullptr;
-  if (!handoff) grid_dependency_wait();
-  bool slice0 = true;
-  if (threadIdx.x == 32 && handoff) slice0 = wait_slice(p, 0, ctl);
-  if (threadIdx.x == 32 && slice0) {
+  grid_dependency_wait();
+  if (threadIdx.x == 32) {
     // The first loads need nothing but the barriers: issue them now so their
     // latency overlaps the rest of the set-up.
     const int pre_b = p.kc < SB ? p.kc : SB;
@@ -194,7 +154,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tma_load_4d(b_base + cc * p.b_tile_bytes, &xmap, fullB(cc), cc * 64, -p.pad, h0 - p.pad, b);
     }
     if (VARIANT == kPremix) {
-      const int pre_a = handoff ? 1 : (p.k_steps < SA ? p.k_steps : SA);
+      const int pre_a = p.k_steps < SA ? p.k_steps : SA;
       for (int k = 0; k < pre_a; ++k) {
         mbar_arrive_expect_tx(fullA(k), kTcATileBytes);
         tma_load_3d(a_base + k * kTcATileBytes, &wmap, fullA(k), (k / p.spc) * 64, k % p.spc,
@@ -216,9 +176,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ======================= activation producer (TMA) =======================
     if (lane == 0) {
       const int pre_b = p.kc < SB ? p.kc : SB;  // issued during set-up
-      int issued = *abort_flag ? 0 : pre_b;     // none if the set-up gave up
+      int issued = pre_b;
       const uint32_t bytes = 64u * 2u * p.Wp * p.b_box_rows;
-      for (int cc = pre_b; cc < p.kc && issued > 0; ++cc) {
+      for (int cc = pre_b; cc < p.kc; ++cc) {
         const int s = cc % SB;
         const uint32_t ph = static_cast<uint32_t>(cc / SB) & 1u;
         if (!wait_bounded(emptyB(s), ph ^ 1u, ctl, kErrWaitProducer)) break;
@@ -232,13 +192,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == 2) {
     // ======================= weight producer (PREMIX only) =======================
     if (VARIANT == kPremix && lane == 0) {
-      const bool handoff = p.slot != nullptr;
-      const int pre_a = handoff ? 1 : (p.k_steps < SA ? p.k_steps : SA);  // issued during set-up
-      int issued = *abort_flag ? 0 : pre_a;
-      for (int k = pre_a; k < p.k_steps && issued > 0; ++k) {
+      const int pre_a = p.k_steps < SA ? p.k_steps : SA;  // issued during set-up
+      int issued = pre_a;
+      for (int k = pre_a; k < p.k_steps; ++k) {
         const int s = k % SA;
         const uint32_t ph = static_cast<uint32_t>(k / SA) & 1u;
-        if (handoff && !wait_slice(p, k, ctl)) break;
         if (!wait_bounded(emptyA(s), ph ^ 1u, ctl, kErrWaitProducer)) break;
         const int cc = k / p.spc, tap = k % p.spc;
         mbar_arrive_expect_tx(fullA(s), kTcATileBytes);
@@ -488,25 +446,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);
-  }
-  if (VARIANT == kPremix && p.slot != nullptr) {
-    // the last CTA to finish (every slice consumed everywhere) zeroes the
-    // counters for the next launch on this stream
-    volatile int* last_s = reinterpret_cast<volatile int*>(misc + 8);
-    if (threadIdx.x == 0) {
-      int last = 0;
-      if (!*abort_flag) {
-        __threadfence();
-        last = atomicAdd(p.slot + 1, 1u) == gridDim.x - 1;
-      }
-      *last_s = last;
-    }
-    __syncthreads();
-    if (*last_s) {
-      __threadfence();
-      for (int k = threadIdx.x; k < p.k_steps; k += kTcThreads) p.slot[kSliceWord0 + k] = 0u;
-      if (threadIdx.x == 0) p.slot[1] = 0u;
-    }
   }
 }
 

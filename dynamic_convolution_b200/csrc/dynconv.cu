@@ -44,7 +44,6 @@ struct DeviceState {
   int* err = nullptr;  // device address of g_device_err on this device
   int sms = 0;
   int max_smem_optin = 0;
-  int smem_per_sm = 0;
   int cc_major = 0, cc_minor = 0;
 };
 
@@ -59,7 +58,6 @@ std::atomic<int> g_route_split{0};  // 0: automatic
 std::atomic<int> g_use_pdl{1};      // programmatic launch edges on forward kernels
 std::atomic<int> g_stream_mix{0};   // PREMIX with n <= 8: mixing streamed into the convolution
 std::atomic<int> g_premix_mixer{0};  // 0 automatic, 1 tensor-core GEMM, 2 CUDA cores (n <= 8)
-std::atomic<int> g_handoff{1};       // two-kernel PREMIX: hand-off by slice counters (n <= 8)
 thread_local char g_last_err[256] = "";
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -93,7 +91,6 @@ int device_state(DeviceState** out) {
     }
     st.sms = prop.multiProcessorCount;
     st.max_smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
-    st.smem_per_sm = static_cast<int>(prop.sharedMemPerMultiprocessor);
     st.cc_major = prop.major;
     st.cc_minor = prop.minor;
     void* addr = nullptr;
@@ -532,50 +529,6 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
     rc = run_mixconv(d, plan, st, experts, alpha, bias, y, ws, xmap, wmap, stream);
     if (rc != DYNCONV_ERR_UNSUPPORTED) return rc;
   }
-  // few experts, hand-off by slice counters: the convolution starts while the
-  // slice-ordered mixer runs (co-resident) and consumes each K step as soon as
-  // it is published
-  if (g_handoff.load() && g_premix_mixer.load() != 1 && plan.p.k_steps <= dc::kMcMaxSlices &&
-      aligned16(experts)) {
-    dc::PoParams po;
-    unsigned grid = 0;
-    if (dc::plan_premix_ordered(d->B, d->n, d->C_in, d->C_out, d->KH * d->KW, plan.p.k_steps,
-                                st->sms, &po, &grid)) {
-      const size_t po_smem = sizeof(float) * static_cast<size_t>(d->B) * d->n;
-      // one convolution CTA must fit beside one mixing CTA on an SM
-      const size_t limit = static_cast<size_t>(st->smem_per_sm) - 2048 - po_smem;
-      TcPlan hp = plan;
-      while (hp.smem > limit && hp.p.sa > 2) {
-        --hp.p.sa;
-        hp.smem -= dc::kTcATileBytes;
-      }
-      if (hp.smem <= limit) {
-        unsigned int* slot = nullptr;
-        rc = mix_state_slot(static_cast<void*>(stream), &slot, stream);
-        if (rc) return rc;
-        po.experts = static_cast<const __nv_bfloat16*>(experts);
-        po.alpha = alpha;
-        po.out = static_cast<__nv_bfloat16*>(ws);
-        po.counters = slot + dc::kSliceWord0;
-        auto kern = d->n <= 2 ? dc::premix_ordered_kernel<2>
-                    : d->n <= 4 ? dc::premix_ordered_kernel<4> : dc::premix_ordered_kernel<8>;
-        cudaError_t e = launch_pdl(kern, dim3(grid), dim3(dc::kPsThreads), po_smem, stream, po);
-        if (e != cudaSuccess) {
-          g_launches.fetch_add(1, std::memory_order_relaxed);
-          return cuda_fail(e, "premix_ordered_kernel launch");
-        }
-        rc = check_launch("premix_ordered_kernel");
-        if (rc) return rc;
-        rc = encode_w_map(&wmap, ws, d);
-        if (rc) return rc;
-        hp.p.slot = slot;
-        hp.p.fa = po.fa;
-        hp.p.ta = static_cast<unsigned int>(po.ipsA);
-        hp.p.tb = static_cast<unsigned int>(po.ipsB);
-        return launch_tc<dc::kPremix>(hp, xmap, wmap, stream);
-      }
-    }
-  }
   // few experts: the store-bound CUDA-core mixer (no set-up chain)
   if (g_premix_mixer.load() != 1) {
     dc::PsParams ps;
@@ -676,11 +629,6 @@ int dynconv_test_hook(int key, long long value) {
   if (key == 6) {
     if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
     g_stream_mix.store(static_cast<int>(value));
-    return DYNCONV_OK;
-  }
-  if (key == 8) {
-    if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
-    g_handoff.store(static_cast<int>(value));
     return DYNCONV_OK;
   }
   if (key == 7) {

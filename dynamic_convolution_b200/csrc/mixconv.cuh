@@ -37,7 +37,7 @@ constexpr int kMcMixer0 = 4;            // first mixer / epilogue warp
 constexpr int kMcMaxExperts = 8;
 constexpr int kMcStateWords = 1024;     // 4 KB of state per slot
 constexpr int kMcSlots = 64;            // state slots (one per stream in use)
-constexpr int kMcSliceWord0 = kSliceWord0;  // slice counters start here (shared layout)
+constexpr int kMcSliceWord0 = 64;       // slice counters start here
 constexpr int kMcMaxSlices = kMcStateWords - kMcSliceWord0;
 constexpr int kMcEpiStage = 8 * 2048;   // epilogue staging: 2 KB per warp
 

@@ -214,10 +214,6 @@ unsigned long long dynconv_launch_count(void);
  * mixing GEMM; 1 always the tensor-core GEMM (and never the streamed kernel of
  * key 6); 2 the CUDA-core mixer only (forward returns
  * DYNCONV_ERR_UNSUPPORTED when n > 8).
- * key 8: 1 (default) hands the two-kernel PREMIX form with n <= 8 from the
- * mixing kernel to the convolution by per-slice counters (the convolution runs
- * beside the slice-ordered mixer and starts on slice 0); 0 waits for the whole
- * mixing kernel instead.
  * Returns DYNCONV_OK or DYNCONV_ERR_INVALID_ARG. */
 int dynconv_test_hook(int key, long long value);
 
