@@ -25,6 +25,7 @@ OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = -1, -2, -3, -4, -5, -6
 
 SYMBOLS = ("dynconv_route", "dynconv_forward", "dynconv_forward_noalloc",
+           "dynconv_pool_parts", "dynconv_forward_pooled", "dynconv_route_pooled",
            "dynconv_workspace_size", "dynconv_select_variant",
            "dynconv_status_string", "dynconv_last_error", "dynconv_device_status",
            "dynconv_launch_count", "dynconv_test_hook")
@@ -61,6 +62,13 @@ def load():
         lib.dynconv_forward.restype = ctypes.c_int
         lib.dynconv_forward_noalloc.argtypes = [D, P, P, P, P, P, P]
         lib.dynconv_forward_noalloc.restype = ctypes.c_int
+        lib.dynconv_pool_parts.argtypes = [D, ctypes.c_size_t]
+        lib.dynconv_pool_parts.restype = ctypes.c_int
+        lib.dynconv_forward_pooled.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.dynconv_forward_pooled.restype = ctypes.c_int
+        lib.dynconv_route_pooled.argtypes = [D, P, ctypes.c_int, P, P, ctypes.c_int,
+                                             ctypes.c_float, P, P]
+        lib.dynconv_route_pooled.restype = ctypes.c_int
         lib.dynconv_workspace_size.argtypes = [D]
         lib.dynconv_workspace_size.restype = ctypes.c_size_t
         lib.dynconv_select_variant.argtypes = [D, ctypes.c_size_t]
@@ -116,6 +124,26 @@ def dynconv_forward(desc, x, experts, alpha, bias, y, workspace=None, workspace_
     return load().dynconv_forward(ctypes.byref(desc), _ptr(x), _ptr(experts), _ptr(alpha),
                                   _ptr(bias), _ptr(y), _ptr(workspace), int(workspace_bytes),
                                   _stream(stream))
+
+
+def dynconv_pool_parts(desc, workspace_bytes=0) -> int:
+    return int(load().dynconv_pool_parts(ctypes.byref(desc), int(workspace_bytes)))
+
+
+def dynconv_forward_pooled(desc, x, experts, alpha, bias, y, ysum, workspace=None,
+                           workspace_bytes=0, stream=None) -> int:
+    """dynconv_forward that also writes partial channel sums of y (the next
+    layer's routing pool), ysum fp32 [B][P][C_out] with P = dynconv_pool_parts."""
+    return load().dynconv_forward_pooled(ctypes.byref(desc), _ptr(x), _ptr(experts), _ptr(alpha),
+                                         _ptr(bias), _ptr(y), _ptr(ysum), _ptr(workspace),
+                                         int(workspace_bytes), _stream(stream))
+
+
+def dynconv_route_pooled(desc, ysum, parts, Wr, br, mode, tau, alpha, stream=None) -> int:
+    """Routing of the layer `desc` from the previous layer's pooled partial sums."""
+    return load().dynconv_route_pooled(ctypes.byref(desc), _ptr(ysum), int(parts), _ptr(Wr),
+                                       _ptr(br), int(mode), float(tau), _ptr(alpha),
+                                       _stream(stream))
 
 
 # Bytes of the library's built-in scratch array (DYNCONV_NOALLOC_MAX_BYTES).

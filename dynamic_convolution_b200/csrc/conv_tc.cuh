@@ -49,6 +49,9 @@ constexpr int kTcThreads = 384;      // 12 warps
 constexpr int kTcMixWarp0 = 4;       // warps 4..11 mix (FUSED/OUTSIDE) and run the epilogue
 constexpr int kTcMixThreads = 256;
 constexpr int kTcATileBytes = 128 * 128;  // 128 rows x 64 bf16
+// The epilogue stages 12 x 2 KB in the idle A stages; the pooled channel
+// sums (3 x 128 floats) follow them (the A stages hold at least 32 KB).
+constexpr int kTcPoolOff = 12 * 2048;
 
 enum TcVariant { kFused = 1, kOutside = 2, kPremix = 3 };
 
@@ -75,6 +78,7 @@ struct TcParams {
   int* err;
   long long wait_ns;
   int inject_skip;    // test hook: withhold the first mixer arrival of CTA 0
+  float* ysum;        // optional [B][tiles_h][Cout]: per-unit channel sums of y as stored
 };
 
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, int base_mode) {
@@ -392,6 +396,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int c8 = m0 + 32 * q + part * 8;
       const bool c_ok = c8 < p.Cout;
       __nv_bfloat16* ybase = p.y + static_cast<size_t>(b) * p.H * p.W * p.Cout + c8;
+      // optional pooling for the next layer's routing: this thread's 8 output
+      // channels summed over the pixels it stores, in a fixed order
+      const bool pool = p.ysum != nullptr;
+      float ps[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
       auto process = [&](const uint32_t (&r)[32], int ch) {
 #pragma unroll
         for (int jj = 0; jj < 32; jj += 2) {
@@ -416,6 +426,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                          : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                          : "r"(stage + (it * 8 + (lane >> 2)) * 64 + part * 16));
             *reinterpret_cast<uint4*>(ybase + (static_cast<size_t>(oh) * p.W + cw) * p.Cout) = v;
+            if (pool) {
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                ps[2 * e] += bf16lo_to_f32(w4[e]);
+                ps[2 * e + 1] += bf16hi_to_f32(w4[e]);
+              }
+            }
           }
           pix += 8;
           cw += 8;
@@ -437,6 +455,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         process(rb, ch);
         ch += 3;
       }
+      if (pool) {
+        // lanes with the same 16-byte part hold the same channels: fixed tree,
+        // then each (chunk phase, quarter) leaves 32 channel sums in shared memory
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          ps[e] += __shfl_xor_sync(0xffffffffu, ps[e], 4);
+          ps[e] += __shfl_xor_sync(0xffffffffu, ps[e], 8);
+          ps[e] += __shfl_xor_sync(0xffffffffu, ps[e], 16);
+        }
+        if (lane < 4) {
+          float* dst = reinterpret_cast<float*>(base_ptr + kTcPoolOff) + grp * 128 + 32 * q + lane * 8;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dst[e] = ps[e];
+        }
+      }
     }
   }
 
@@ -446,6 +479,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+  if (p.ysum != nullptr && threadIdx.x < 128 && m0 + static_cast<int>(threadIdx.x) < p.Cout &&
+      !*abort_flag) {
+    const float* src = reinterpret_cast<const float*>(base_ptr + kTcPoolOff);
+    const float t = src[threadIdx.x] + src[128 + threadIdx.x] + src[256 + threadIdx.x];
+    p.ysum[(static_cast<size_t>(b) * p.tiles_h + th) * p.Cout + m0 + threadIdx.x] = t;
   }
 }
 

@@ -22,6 +22,7 @@
 #include "premix_small.cuh"
 #include "mixconv.cuh"
 #include "route.cuh"
+#include "pool.cuh"
 
 namespace {
 
@@ -501,9 +502,10 @@ int run_mixconv(const dynconv_desc* d, const TcPlan& plan_in, const DeviceState*
 
 int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void* x,
            const void* experts, const float* alpha, const float* bias, void* y, void* ws,
-           size_t ws_bytes, cudaStream_t stream) {
+           size_t ws_bytes, cudaStream_t stream, float* ysum = nullptr) {
   TcPlan plan;
   if (!tc_plan(d, variant, st->sms, st->max_smem_optin, &plan)) return DYNCONV_ERR_UNSUPPORTED;
+  plan.p.ysum = ysum;
   plan.p.experts = static_cast<const __nv_bfloat16*>(experts);
   plan.p.alpha = alpha;
   plan.p.bias = bias;
@@ -523,7 +525,8 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   if (!ws || ws_bytes < need) return DYNCONV_ERR_WORKSPACE;
   if (!aligned16(ws)) return DYNCONV_ERR_MISALIGNED;
   plan.p.inject_skip = 0;
-  if (g_stream_mix.load() && g_premix_mixer.load() != 1 && d->n <= dc::kMcMaxExperts) {
+  if (g_stream_mix.load() && g_premix_mixer.load() != 1 && d->n <= dc::kMcMaxExperts &&
+      ysum == nullptr) {
     rc = encode_w_map(&wmap, ws, d);
     if (rc) return rc;
     rc = run_mixconv(d, plan, st, experts, alpha, bias, y, ws, xmap, wmap, stream);
@@ -740,9 +743,39 @@ int dynconv_route(const dynconv_desc* desc, const void* x, const float* Wr, cons
   return check_launch("route_kernel");
 }
 
-int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts,
-                    const float* alpha, const float* bias, void* y, void* workspace,
-                    size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The channel sums of y in a second pass (one partial per sample), for the
+// CUDA-core forward kernels.
+int pool_pass(const dynconv_desc* d, const void* y, float* ysum, cudaStream_t s) {
+  const int Ho = out_size(d->H, d->KH, d->stride, d->pad);
+  const int Wo = out_size(d->W, d->KW, d->stride, d->pad);
+  cudaError_t e;
+  if (d->dtype == DYNCONV_F32)
+    e = launch_pdl(dc::pool_sum_kernel<float>, dim3(d->B), dim3(dc::kPoolThreads), 0, s,
+                   static_cast<const float*>(y), Ho * Wo, d->C_out, ysum);
+  else
+    e = launch_pdl(dc::pool_sum_kernel<__nv_bfloat16>, dim3(d->B), dim3(dc::kPoolThreads), 0, s,
+                   static_cast<const __nv_bfloat16*>(y), Ho * Wo, d->C_out, ysum);
+  if (e != cudaSuccess) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_fail(e, "pool_sum_kernel launch");
+  }
+  return check_launch("pool_sum_kernel");
+}
+
+int resolve_variant(const dynconv_desc* desc, size_t ws_bytes, const DeviceState* st) {
+  int variant = desc->variant;
+  if (variant == DYNCONV_VARIANT_AUTO)
+    variant = select_variant(desc, ws_bytes, st->sms, st->max_smem_optin);
+  return variant;
+}
+
+int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
+                 const float* alpha, const float* bias, void* y, void* workspace,
+                 size_t workspace_bytes, void* stream, float* ysum) {
   int rc = validate_desc(desc);
   if (rc) return rc;
   if (!x || !experts || !alpha || !y) return DYNCONV_ERR_INVALID_ARG;
@@ -752,9 +785,7 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  int variant = desc->variant;
-  if (variant == DYNCONV_VARIANT_AUTO)
-    variant = select_variant(desc, workspace ? workspace_bytes : 0, st->sms, st->max_smem_optin);
+  const int variant = resolve_variant(desc, workspace ? workspace_bytes : 0, st);
 
   switch (variant) {
     case DYNCONV_VARIANT_FUSED:
@@ -762,7 +793,8 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
     case DYNCONV_VARIANT_PREMIX: {
       if (!tc_shape_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
       if (!aligned16(x) || !aligned16(experts) || !aligned16(y)) return DYNCONV_ERR_MISALIGNED;
-      return run_tc(desc, variant, st, x, experts, alpha, bias, y, workspace, workspace_bytes, s);
+      return run_tc(desc, variant, st, x, experts, alpha, bias, y, workspace, workspace_bytes, s,
+                    ysum);
     }
     case DYNCONV_VARIANT_DEPTHWISE: {
       if (!depthwise_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
@@ -816,9 +848,10 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
         }
         return check_launch("depthwise_kernel");
       };
-      if (K == 3) return go(dc::depthwise_kernel<3>);
-      if (K == 5) return go(dc::depthwise_kernel<5>);
-      return go(dc::depthwise_kernel<7>);
+      rc = K == 3 ? go(dc::depthwise_kernel<3>)
+           : K == 5 ? go(dc::depthwise_kernel<5>) : go(dc::depthwise_kernel<7>);
+      if (rc || ysum == nullptr) return rc;
+      return pool_pass(desc, y, ysum, s);
     }
     case DYNCONV_VARIANT_DIRECT: {
       const int Cg = desc->C_in / desc->groups;
@@ -848,12 +881,80 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
         }
         return check_launch("direct_conv_kernel");
       };
-      if (desc->dtype == DYNCONV_F32) return go(dc::direct_conv_kernel<float>);
-      return go(dc::direct_conv_kernel<__nv_bfloat16>);
+      rc = desc->dtype == DYNCONV_F32 ? go(dc::direct_conv_kernel<float>)
+                                      : go(dc::direct_conv_kernel<__nv_bfloat16>);
+      if (rc || ysum == nullptr) return rc;
+      return pool_pass(desc, y, ysum, s);
     }
     default:
       return DYNCONV_ERR_INVALID_ARG;
   }
+}
+
+}  // namespace
+
+extern "C" {
+
+int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts,
+                    const float* alpha, const float* bias, void* y, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  return forward_impl(desc, x, experts, alpha, bias, y, workspace, workspace_bytes, stream,
+                      nullptr);
+}
+
+int dynconv_forward_pooled(const dynconv_desc* desc, const void* x, const void* experts,
+                           const float* alpha, const float* bias, void* y, float* ysum,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!ysum) return DYNCONV_ERR_INVALID_ARG;
+  return forward_impl(desc, x, experts, alpha, bias, y, workspace, workspace_bytes, stream, ysum);
+}
+
+int dynconv_pool_parts(const dynconv_desc* desc, size_t workspace_bytes) {
+  int rc = validate_desc(desc);
+  if (rc) return rc;
+  int sms = 148, max_smem = 232448;
+  DeviceState* st = nullptr;
+  if (device_state(&st) == DYNCONV_OK) {
+    sms = st->sms;
+    max_smem = st->max_smem_optin;
+  }
+  int variant = desc->variant;
+  if (variant == DYNCONV_VARIANT_AUTO) variant = select_variant(desc, workspace_bytes, sms, max_smem);
+  if (variant == DYNCONV_VARIANT_FUSED || variant == DYNCONV_VARIANT_OUTSIDE ||
+      variant == DYNCONV_VARIANT_PREMIX) {
+    TcPlan plan;
+    if (!tc_plan(desc, variant, sms, max_smem, &plan)) return DYNCONV_ERR_UNSUPPORTED;
+    return plan.p.tiles_h;
+  }
+  return 1;
+}
+
+int dynconv_route_pooled(const dynconv_desc* desc, const float* ysum, int parts, const float* Wr,
+                         const float* br, int mode, float tau, float* alpha, void* stream) {
+  int rc = validate_desc(desc);
+  if (rc) return rc;
+  if (!ysum || !Wr || !alpha || parts < 1) return DYNCONV_ERR_INVALID_ARG;
+  if (mode != DYNCONV_SIGMOID && mode != DYNCONV_SOFTMAX) return DYNCONV_ERR_INVALID_ARG;
+  if (mode == DYNCONV_SOFTMAX && !(tau > 0.f)) return DYNCONV_ERR_INVALID_ARG;
+  if (desc->n > 1024 || desc->C_in > 16384) return DYNCONV_ERR_UNSUPPORTED;
+  if (desc->B == 0) return DYNCONV_OK;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc) return rc;
+  dc::RoutePooledParams p{desc->B, desc->C_in, desc->H * desc->W, desc->n, parts, mode, tau,
+                          ysum, Wr, br, alpha};
+  const size_t smem = sizeof(float) * (static_cast<size_t>(desc->C_in) + desc->n);
+  if (smem > static_cast<size_t>(st->max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
+  cudaError_t e = cudaSuccess;
+  if (smem > 48 * 1024) e = ensure_smem(dc::route_pooled_kernel, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(route_pooled)");
+  e = launch_pdl(dc::route_pooled_kernel, dim3(desc->B), dim3(dc::kPoolThreads), smem,
+                 static_cast<cudaStream_t>(stream), p);
+  if (e != cudaSuccess) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_fail(e, "route_pooled_kernel launch");
+  }
+  return check_launch("route_pooled_kernel");
 }
 
 int dynconv_forward_noalloc(const dynconv_desc* desc, const void* x, const void* experts,

@@ -132,6 +132,43 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
                     const float* alpha, const float* bias, void* y, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* ---- routing pooled in the previous layer (chained layers) -----------------
+ * When layer L+1's input is layer L's output, the average pool of L+1's
+ * routing step can be taken in L's epilogue, where the output is already in
+ * registers: dynconv_forward_pooled writes, besides y, partial channel sums of
+ * y as stored, and dynconv_route_pooled finishes L+1's routing from them
+ * without reading its input again. (The pages give the attentions as
+ * input-dependent, KernelWarehouse, abstract; the average pool is the reading
+ * taken for the routing step, see dynconv_route.)
+ *
+ * dynconv_pool_parts: the number P >= 1 of partial sums per (sample, channel)
+ * that dynconv_forward_pooled writes for this descriptor and workspace size
+ * (the same inputs dynconv_select_variant takes), or a negative status. Pure
+ * host function.
+ *
+ * dynconv_forward_pooled: as dynconv_forward, and
+ *   ysum  device fp32 [B][P][C_out]: ysum[b][p][c] is the sum, over the p-th of
+ *         P fixed disjoint subsets of the output pixels (together all of them),
+ *         of y[b][h][w][c] as stored (after rounding to desc->dtype); every
+ *         element is written. Deterministic.
+ *   The tensor-core variants add the sums in their epilogue; the CUDA-core
+ *   variants (DIRECT, DEPTHWISE) add them in a second pass over y.
+ * Errors as dynconv_forward; INVALID_ARG if ysum is NULL.
+ *
+ * dynconv_route_pooled: alpha for the layer described by `desc` (desc->C_in =
+ * the previous layer's C_out; desc->H, desc->W = its output size), from `parts`
+ * partial sums per channel: g[b][c] = (sum over p, in order, of
+ * ysum[b][p][c]) / (H*W); then the linear layer and activation exactly as
+ * dynconv_route (same Wr, br, mode, tau, alpha). Deterministic.
+ * Errors: INVALID_ARG (NULL pointers, parts < 1, bad mode or tau),
+ * UNSUPPORTED (n > 1024 or C_in > 16384), CUDA. */
+int dynconv_pool_parts(const dynconv_desc* desc, size_t workspace_bytes);
+int dynconv_forward_pooled(const dynconv_desc* desc, const void* x, const void* experts,
+                           const float* alpha, const float* bias, void* y, float* ysum,
+                           void* workspace, size_t workspace_bytes, void* stream);
+int dynconv_route_pooled(const dynconv_desc* desc, const float* ysum, int parts, const float* Wr,
+                         const float* br, int mode, float tau, float* alpha, void* stream);
+
 /* ---- forward without caller-provided scratch ----------------------------
  * The pages describe no such entry point; it has no counterpart in the method.
  *

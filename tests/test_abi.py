@@ -121,3 +121,19 @@ def test_test_hook_arguments(lib):
     assert dc.dynconv_test_hook(1, 0) == dc.OK
     assert dc.dynconv_test_hook(1, -5) == dc.ERR_INVALID_ARG
     assert dc.dynconv_test_hook(99, 0) == dc.ERR_INVALID_ARG
+
+
+def test_pooled_entry_points_host_side(lib):
+    d = _desc(dtype=dc.BF16)
+    assert dc.dynconv_forward_pooled(d, 16, 16, 16, None, 16, None) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_route_pooled(d, None, 1, 16, None, dc.SIGMOID, 1.0, 16) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_route_pooled(d, 16, 0, 16, None, dc.SIGMOID, 1.0, 16) == dc.ERR_INVALID_ARG
+    for kw in BAD:
+        assert dc.dynconv_pool_parts(_desc(**kw)) == dc.ERR_INVALID_ARG
+    # one partial per sample for the CUDA-core kernels, row blocks for the tensor-core ones
+    assert dc.dynconv_pool_parts(dc.desc_from_config(synth.CONFIGS["tiny_fp32"])) == 1
+    assert dc.dynconv_pool_parts(dc.desc_from_config(synth.CONFIGS["effnet_dw_5x5"])) == 1
+    for name in ("resnet18_3x3", "effnet_expand_1x1"):
+        d = dc.desc_from_config(synth.CONFIGS[name])
+        parts = dc.dynconv_pool_parts(d, dc.dynconv_workspace_size(d))
+        assert 1 <= parts <= synth.CONFIGS[name].H
