@@ -6,6 +6,7 @@ One step = routing + forward of one dynamic-convolution layer over one batch
 n=4 experts, softmax routing). Prints ONE JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--variant V]
+  python bench.py --config effnet_block   # the chained 1x1 -> depthwise block, one GPU
   python bench.py --impl reference ...     # the fp64 CPU oracle on the host cores
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of the
@@ -505,9 +506,98 @@ def run_ours(args, cfg):
     return 0
 
 
+def run_block(args):
+    """The chained EfficientNet-style block (1x1 expand layer, then the depthwise
+    5x5 layer on its output), one GPU. Step = both layers' routing and forward.
+    Times the block with the depthwise layer's routing pooled in the expand
+    layer's epilogue (dynconv_forward_pooled + dynconv_route_pooled) and, for
+    comparison, with the routing kernel reading the intermediate tensor again.
+    CUDA graphs of 8 steps over rotating input sets larger than L2."""
+    import torch
+
+    import dynamic_convolution_b200 as dc
+    from dynamic_convolution_b200 import build, synth
+
+    torch.cuda.set_device(0)
+    build.build()
+    dc.load()
+    up, dw = synth.CONFIGS["effnet_expand_1x1"], synth.CONFIGS["effnet_dw_5x5"]
+    ia, ib = synth.make_inputs(up), synth.make_inputs(dw)
+    bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).cuda()
+    Ea, Eb = bf(ia.experts_store), bf(ib.experts_store)
+    Wra, bra, biasa = (torch.from_numpy(a).cuda() for a in (ia.Wr, ia.br, ia.bias))
+    Wrb, brb, biasb = (torch.from_numpy(a).cuda() for a in (ib.Wr, ib.br, ib.bias))
+    da, db = dc.desc_from_config(up), dc.desc_from_config(dw)
+    wsa = dc.dynconv_workspace_size(da)
+    ws = torch.empty(max(wsa, 16), dtype=torch.uint8, device="cuda")
+    parts = dc.dynconv_pool_parts(da, wsa)
+    x0 = bf(ia.x_store)
+    set_bytes = 2 * x0.numel() * 2 + 2 * up.B * up.H * up.W * up.C_out * 2
+    nsets = max(2, min(64, math.ceil(2 * L2_BYTES / set_bytes)))
+    xs = [x0.clone() for _ in range(nsets)]
+    mids = [torch.empty((up.B, up.H, up.W, up.C_out), dtype=torch.bfloat16, device="cuda")
+            for _ in range(nsets)]
+    outs = [torch.empty_like(m) for m in mids]
+    aa = [torch.empty((up.B, up.n), device="cuda") for _ in range(nsets)]
+    ab = [torch.empty((dw.B, dw.n), device="cuda") for _ in range(nsets)]
+    ysum = [torch.empty((up.B, parts, up.C_out), device="cuda") for _ in range(nsets)]
+    stream = torch.cuda.Stream()
+
+    def step(s, pooled, st):
+        dc.check(dc.dynconv_route(da, xs[s], Wra, bra, up.mode, up.tau, aa[s], st))
+        if pooled:
+            dc.check(dc.dynconv_forward_pooled(da, xs[s], Ea, aa[s], biasa, mids[s], ysum[s], ws,
+                                               wsa, st))
+            dc.check(dc.dynconv_route_pooled(db, ysum[s], parts, Wrb, brb, dw.mode, dw.tau, ab[s],
+                                             st))
+        else:
+            dc.check(dc.dynconv_forward(da, xs[s], Ea, aa[s], biasa, mids[s], ws, wsa, st))
+            dc.check(dc.dynconv_route(db, mids[s], Wrb, brb, dw.mode, dw.tau, ab[s], st))
+        dc.check(dc.dynconv_forward(db, mids[s], Eb, ab[s], biasb, outs[s], None, 0, st))
+
+    res = {}
+    for pooled in (True, False):
+        with torch.cuda.stream(stream):
+            for k in range(max(args.warmup, 3)):
+                step(k % nsets, pooled, stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for s in range(min(8, nsets)):
+                step(s, pooled, stream)
+        reps = max(1, args.steps // min(8, nsets))
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        dc.check(dc.dynconv_device_status(stream), "device status")
+        res[pooled] = e0.elapsed_time(e1) / (reps * min(8, nsets))
+        del g
+    ms = res[True]
+    line = {"metric": "images/s per block (1x1 expand + depthwise 5x5, routing + forward)",
+            "value": up.B / (ms / 1e3), "unit": "images/s", "n_gpus": 1,
+            "steps": reps * min(8, nsets), "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; recipe in DESIGN.md)",
+            "config": {"workload": "effnet_block (effnet_expand_1x1 -> effnet_dw_5x5)",
+                       "routing_pool": "depthwise routing pooled in the expand epilogue",
+                       "l2": f"inputs rotated over {nsets} sets"},
+            "unpooled_ms_per_step": res[False],
+            "unpooled_images_per_s": up.B / (res[False] / 1e3)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     from dynamic_convolution_b200 import synth
+    if args.config == "effnet_block":
+        return run_block(args)
     name = args.config or synth.HEADLINE
     cfg = synth.CONFIGS[name]
     if args.impl == "reference":
