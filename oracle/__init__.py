@@ -51,6 +51,8 @@ def configure(lib):
     lib.oracle_route.restype = i
     lib.oracle_forward.argtypes = [i] * 11 + [dp, dp, dp, dp, i, i, dp, i]
     lib.oracle_forward.restype = i
+    lib.oracle_forward_attn.argtypes = [i] * 11 + [dp, dp, dp, dp, dp, dp, i, i, dp, i]
+    lib.oracle_forward_attn.restype = i
     lib.oracle_forward_rows.argtypes = [i] * 11 + [dp, dp, dp, dp, i, i, i, dp]
     lib.oracle_forward_rows.restype = i
     lib.oracle_assemble.argtypes = [i, ctypes.c_long, dp, dp, dp]
@@ -126,6 +128,36 @@ def forward(x, experts, alpha, bias=None, stride: int = 1, pad: int = 0, groups:
                                 int(nthreads))
     if rc != 0:
         raise ValueError(f"oracle_forward rejected its arguments (rc={rc})")
+    return y
+
+
+def forward_attn(x, experts, alpha, bias, a_in, a_out, stride: int = 1, pad: int = 0,
+                 groups: int = 1, samples: tuple[int, int] | None = None, nthreads: int = 0):
+    """``forward`` with the FMDConv channel attentions: a_in[B][C_in] multiplies
+    every input channel of a sample, a_out[B][C_out] every output channel (bias
+    included); either may be None (all ones)."""
+    x = _f64(x)
+    experts = _f64(experts)
+    alpha = _f64(alpha)
+    bias = _f64(bias)
+    a_in = _f64(a_in)
+    a_out = _f64(a_out)
+    B, H, W, Cin = x.shape
+    n, Cout, KH, KW, Cg = experts.shape
+    assert Cg * groups == Cin, "experts' last dim must be C_in/groups"
+    assert alpha.shape == (B, n)
+    assert bias is None or bias.shape == (n, Cout)
+    assert a_in is None or a_in.shape == (B, Cin)
+    assert a_out is None or a_out.shape == (B, Cout)
+    b0, nb = (0, B) if samples is None else samples
+    Ho = (H + 2 * pad - KH) // stride + 1
+    Wo = (W + 2 * pad - KW) // stride + 1
+    y = np.empty((nb, Ho, Wo, Cout), dtype=np.float64)
+    rc = _load().oracle_forward_attn(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n,
+                                     _dp(x), _dp(experts), _dp(alpha), _dp(bias), _dp(a_in),
+                                     _dp(a_out), b0, nb, _dp(y), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_forward_attn rejected its arguments (rc={rc})")
     return y
 
 

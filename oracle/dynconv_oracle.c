@@ -183,6 +183,8 @@ typedef struct {
   int oh_begin, oh_end;   /* output rows computed, [oh_begin, oh_end) */
   const double *x, *experts, *alpha, *bias;
   double *y;              /* rows oh_begin.. of samples b0.. */
+  const double *a_in;     /* [B][Cin] input (channel) attention, or NULL: all ones */
+  const double *a_out;    /* [B][Cout] output (channel) attention, or NULL: all ones */
 } fwd_ctx;
 
 static void forward_one(void *vctx, int b) {
@@ -196,8 +198,14 @@ static void forward_one(void *vctx, int b) {
   oracle_assemble(f->n, wsize, f->experts, ab, Wb);
   oracle_mix_bias(f->n, f->Cout, f->bias, ab, bb);
 
-  /* Step 5: y[oh,ow,co] = b_b[co] + sum_{kh,kw,ci} xpad[oh*s+kh-p, ow*s+kw-p, g*Cg+ci] W_b[co,kh,kw,ci] */
+  /* Step 5: y[oh,ow,co] = b_b[co] + sum_{kh,kw,ci} xpad[oh*s+kh-p, ow*s+kw-p, g*Cg+ci] W_b[co,kh,kw,ci]
+   * With the FMDConv channel attentions (FMDConv, abstract: input attention and
+   * output attention; no formula on the page, reading: per-channel factors of
+   * the sample): the input factor multiplies x channel by channel, the output
+   * factor multiplies y (bias included) channel by channel. */
   const double *xb = f->x + (size_t)b * f->H * f->W * f->Cin;
+  const double *ain = f->a_in ? f->a_in + (size_t)b * f->Cin : NULL;
+  const double *aout = f->a_out ? f->a_out + (size_t)b * f->Cout : NULL;
   const int nrows = f->oh_end - f->oh_begin;
   double *yb = f->y + (size_t)(b - f->b0) * nrows * f->Wo * f->Cout;
   for (int oh = f->oh_begin; oh < f->oh_end; ++oh)
@@ -213,9 +221,15 @@ static void forward_one(void *vctx, int b) {
             if (iw < 0 || iw >= f->W) continue;        /* zero padding */
             const double *xp = xb + ((size_t)ih * f->W + iw) * f->Cin + (size_t)g * Cg;
             const double *wp = Wb + (((size_t)co * f->KH + kh) * f->KW + kw) * Cg;
-            for (int ci = 0; ci < Cg; ++ci) s += xp[ci] * wp[ci];
+            if (ain) {
+              const double *ap = ain + (size_t)g * Cg;
+              for (int ci = 0; ci < Cg; ++ci) s += (ap[ci] * xp[ci]) * wp[ci];
+            } else {
+              for (int ci = 0; ci < Cg; ++ci) s += xp[ci] * wp[ci];
+            }
           }
         }
+        if (aout) s *= aout[co];
         yb[((size_t)(oh - f->oh_begin) * f->Wo + ow) * f->Cout + co] = s;
       }
   free(Wb);
@@ -241,7 +255,27 @@ int oracle_forward(int B, int Cin, int H, int W, int Cout, int KH, int KW, int s
   if (Ho <= 0 || Wo <= 0) return -1;
   if (nb == 0) return 0;
   fwd_ctx f = {Cin, H, W, Cout, KH, KW, stride, pad, groups, n, Ho, Wo, b0, 0, Ho,
-               x, experts, alpha, bias, y};
+               x, experts, alpha, bias, y, NULL, NULL};
+  return run_samples(forward_one, &f, b0, nb, nthreads);
+}
+
+/* oracle_forward with the FMDConv channel attentions: a_in [B][Cin] multiplies
+ * the input channels of each sample, a_out [B][Cout] its output channels (bias
+ * included); either may be NULL (all ones). */
+int oracle_forward_attn(int B, int Cin, int H, int W, int Cout, int KH, int KW, int stride,
+                        int pad, int groups, int n, const double *x, const double *experts,
+                        const double *alpha, const double *bias, const double *a_in,
+                        const double *a_out, int b0, int nb, double *y, int nthreads) {
+  if (B < 0 || Cin <= 0 || H <= 0 || W <= 0 || Cout <= 0 || KH <= 0 || KW <= 0) return -1;
+  if (stride <= 0 || pad < 0 || groups <= 0 || n <= 0) return -1;
+  if (Cin % groups != 0 || Cout % groups != 0) return -1;
+  if (!x || !experts || !alpha || !y) return -1;
+  if (b0 < 0 || nb < 0 || b0 + nb > B) return -1;
+  const int Ho = oracle_out_size(H, KH, stride, pad), Wo = oracle_out_size(W, KW, stride, pad);
+  if (Ho <= 0 || Wo <= 0) return -1;
+  if (nb == 0) return 0;
+  fwd_ctx f = {Cin, H, W, Cout, KH, KW, stride, pad, groups, n, Ho, Wo, b0, 0, Ho,
+               x, experts, alpha, bias, y, a_in, a_out};
   return run_samples(forward_one, &f, b0, nb, nthreads);
 }
 
@@ -259,7 +293,7 @@ int oracle_forward_rows(int B, int Cin, int H, int W, int Cout, int KH, int KW, 
   if (Ho <= 0 || Wo <= 0 || b < 0 || b >= B || oh0 < 0 || noh < 0 || oh0 + noh > Ho) return -1;
   if (noh == 0) return 0;
   fwd_ctx f = {Cin, H, W, Cout, KH, KW, stride, pad, groups, n, Ho, Wo, b, oh0, oh0 + noh,
-               x, experts, alpha, bias, y};
+               x, experts, alpha, bias, y, NULL, NULL};
   forward_one(&f, b);
   return 0;
 }

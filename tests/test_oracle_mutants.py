@@ -20,13 +20,17 @@ MUTANTS = [
     ("dropped_bias", "double s = bb[co];", "double s = 0.0;"),
     ("alpha_transposed", "const double *ab = f->alpha + (size_t)b * f->n;",
      "const double *ab = f->alpha + (size_t)b;"),
-    ("wrong_group_offset", "+ (size_t)g * Cg;", "+ (size_t)0 * Cg;"),
+    ("wrong_group_offset", "* f->Cin + (size_t)g * Cg;", "* f->Cin + (size_t)0 * Cg;"),
     ("gap_not_averaged", "g[c] = s / (double)(H * W);", "g[c] = s;"),
     ("softmax_without_tau", "den += exp(z[j] / tau);", "den += exp(z[j]);"),
     ("router_bias_dropped", "double s = br ? br[i] : 0.0;", "double s = 0.0;"),
     ("sign_error_in_sigmoid", "1.0 / (1.0 + exp(-z[i]))", "1.0 / (1.0 + exp(z[i]))"),
     ("stride_ignored_in_w", "const int iw = ow * f->stride + kw - f->pad;",
      "const int iw = ow + kw - f->pad;"),
+    ("input_attention_on_wrong_channel", "for (int ci = 0; ci < Cg; ++ci) s += (ap[ci] * xp[ci]) * wp[ci];",
+     "for (int ci = 0; ci < Cg; ++ci) s += (ap[Cg - 1 - ci] * xp[ci]) * wp[ci];"),
+    ("output_attention_before_bias", "double s = bb[co];", "double s = aout ? bb[co] / aout[co] : bb[co];"),
+    ("output_attention_dropped", "if (aout) s *= aout[co];", "if (0) s *= aout[co];"),
 ]
 
 PIN_TESTS = [
@@ -39,6 +43,8 @@ PIN_TESTS = [
     lambda: [pins.test_route_against_library_routines(m, t)
              for m, t in [(0, 1.0), (1, 1.0), (1, 0.3), (1, 30.0)]],
     pins.test_route_invariants,
+    lambda: [pins.test_channel_attention_matches_torch_conv(s) for s in pins.SHAPES],
+    pins.test_channel_attention_zero_input_gives_scaled_bias,
 ]
 
 

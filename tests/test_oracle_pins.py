@@ -355,3 +355,71 @@ def test_row_band_matches_full_forward():
     for b, oh0, noh in [(0, 0, 1), (2, 1, 3), (1, 0, full.shape[1])]:
         band = oracle.forward_rows(x, E, alpha, bias, b, oh0, noh, stride=2, pad=1)
         assert np.array_equal(band, full[b, oh0:oh0 + noh])
+
+
+# ---- FMDConv channel attentions (input attention, output attention: FMDConv,
+# abstract; the page gives no formula, the reading is a per-channel factor of
+# the sample's input and output)
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_channel_attention_matches_torch_conv(shape):
+    """torch conv2d (fp64) on the input scaled by a_in channel by channel, with
+    the mixed kernel and bias, then scaled by a_out channel by channel."""
+    B, Cin, Cout, H, W, K, s, p, g = shape
+    rng = np.random.default_rng(7 + hash(shape) % 2**31)
+    n = 3
+    x, E, alpha, bias = _rand_layer(rng, B, Cin, Cout, H, W, K, s, p, g, n)
+    a_in = rng.uniform(0.05, 1.0, (B, Cin))
+    a_out = rng.uniform(0.05, 1.0, (B, Cout))
+    y = oracle.forward_attn(x, E, alpha, bias, a_in, a_out, stride=s, pad=p, groups=g)
+    for b in range(B):
+        Wb = np.tensordot(alpha[b], E, axes=(0, 0))
+        bb = alpha[b] @ bias
+        xs = x[b:b + 1] * a_in[b][None, None, None, :]
+        ref = _torch_conv(xs, Wb, bb, s, p, g)[0] * a_out[b][None, None, :]
+        assert _rel(y[b], ref) < RTOL
+
+
+def test_channel_attention_absent_or_ones_is_the_plain_forward():
+    rng = np.random.default_rng(11)
+    x, E, alpha, bias = _rand_layer(rng, 2, 4, 6, 6, 5, 3, 1, 1, 1, 2)
+    plain = oracle.forward(x, E, alpha, bias, pad=1)
+    assert np.array_equal(oracle.forward_attn(x, E, alpha, bias, None, None, pad=1), plain)
+    ones = oracle.forward_attn(x, E, alpha, bias, np.ones((2, 4)), np.ones((2, 6)), pad=1)
+    assert _rel(ones, plain) < RTOL
+
+
+def test_channel_attention_scale_invariance_without_bias():
+    """Without bias, c * a_in with a_out / c leaves y unchanged (bilinearity)."""
+    rng = np.random.default_rng(12)
+    x, E, alpha, _ = _rand_layer(rng, 2, 3, 4, 5, 6, 3, 1, 1, 1, 2)
+    a_in = rng.uniform(0.1, 1.0, (2, 3))
+    a_out = rng.uniform(0.1, 1.0, (2, 4))
+    y1 = oracle.forward_attn(x, E, alpha, None, a_in, a_out, pad=1)
+    y2 = oracle.forward_attn(x, E, alpha, None, 2.5 * a_in, a_out / 2.5, pad=1)
+    assert _rel(y2, y1) < RTOL
+
+
+def test_channel_attention_zero_input_gives_scaled_bias():
+    """x = 0: y[b, ., ., co] = a_out[b, co] * sum_i alpha_bi bias_i[co] exactly."""
+    rng = np.random.default_rng(13)
+    _, E, alpha, bias = _rand_layer(rng, 2, 3, 4, 5, 5, 3, 1, 1, 1, 2)
+    x = np.zeros((2, 5, 5, 3))
+    a_in = rng.uniform(0.1, 1.0, (2, 3))
+    a_out = rng.uniform(0.1, 1.0, (2, 4))
+    y = oracle.forward_attn(x, E, alpha, bias, a_in, a_out, pad=1)
+    ref = (a_out * (alpha @ bias))[:, None, None, :]
+    assert np.allclose(y, np.broadcast_to(ref, y.shape), rtol=1e-14, atol=0)
+
+
+def test_channel_attention_routing_is_sigmoid_of_fc_of_gap():
+    """The channel attentions are routing-shaped outputs (sigmoid of a linear
+    layer of the pooled input, one per channel): the oracle's routing with
+    n = channel count gives the library sigmoid of the library mean's FC."""
+    rng = np.random.default_rng(14)
+    x = rng.standard_normal((3, 5, 4, 6))
+    Wi = rng.standard_normal((6, 6)) / np.sqrt(6)
+    bi = rng.standard_normal(6) * 0.1
+    a = oracle.route(x, Wi, bi, oracle.SIGMOID, 1.0)
+    ref = scipy.special.expit(x.mean(axis=(1, 2)) @ Wi.T + bi)
+    assert np.abs(a - ref).max() < 1e-14
