@@ -26,6 +26,7 @@ ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_WOR
 
 SYMBOLS = ("dynconv_route", "dynconv_forward", "dynconv_forward_noalloc",
            "dynconv_pool_parts", "dynconv_forward_pooled", "dynconv_route_pooled",
+           "dynconv_route_channels", "dynconv_forward_attn",
            "dynconv_workspace_size", "dynconv_select_variant",
            "dynconv_status_string", "dynconv_last_error", "dynconv_device_status",
            "dynconv_launch_count", "dynconv_test_hook")
@@ -62,6 +63,10 @@ def load():
         lib.dynconv_forward.restype = ctypes.c_int
         lib.dynconv_forward_noalloc.argtypes = [D, P, P, P, P, P, P]
         lib.dynconv_forward_noalloc.restype = ctypes.c_int
+        lib.dynconv_route_channels.argtypes = [D, P, P, P, P, P, P, P, P]
+        lib.dynconv_route_channels.restype = ctypes.c_int
+        lib.dynconv_forward_attn.argtypes = [D, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.dynconv_forward_attn.restype = ctypes.c_int
         lib.dynconv_pool_parts.argtypes = [D, ctypes.c_size_t]
         lib.dynconv_pool_parts.restype = ctypes.c_int
         lib.dynconv_forward_pooled.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_size_t, P]
@@ -124,6 +129,22 @@ def dynconv_forward(desc, x, experts, alpha, bias, y, workspace=None, workspace_
     return load().dynconv_forward(ctypes.byref(desc), _ptr(x), _ptr(experts), _ptr(alpha),
                                   _ptr(bias), _ptr(y), _ptr(workspace), int(workspace_bytes),
                                   _stream(stream))
+
+
+def dynconv_route_channels(desc, x, Wi, bi, a_in, Wo, bo, a_out, stream=None) -> int:
+    """FMDConv channel attentions a_in [B][C_in], a_out [B][C_out] (sigmoid of a
+    linear layer of the average pool; either pair may be None)."""
+    return load().dynconv_route_channels(ctypes.byref(desc), _ptr(x), _ptr(Wi), _ptr(bi),
+                                         _ptr(a_in), _ptr(Wo), _ptr(bo), _ptr(a_out),
+                                         _stream(stream))
+
+
+def dynconv_forward_attn(desc, x, experts, alpha, bias, a_in, a_out, y, workspace=None,
+                         workspace_bytes=0, stream=None) -> int:
+    """dynconv_forward with the input / output channel attentions (either None)."""
+    return load().dynconv_forward_attn(ctypes.byref(desc), _ptr(x), _ptr(experts), _ptr(alpha),
+                                       _ptr(bias), _ptr(a_in), _ptr(a_out), _ptr(y),
+                                       _ptr(workspace), int(workspace_bytes), _stream(stream))
 
 
 def dynconv_pool_parts(desc, workspace_bytes=0) -> int:

@@ -79,6 +79,7 @@ struct TcParams {
   long long wait_ns;
   int inject_skip;    // test hook: withhold the first mixer arrival of CTA 0
   float* ysum;        // optional [B][tiles_h][Cout]: per-unit channel sums of y as stored
+  const float* a_out; // optional [B][Cout] output channel attention (FMDConv)
 };
 
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, int base_mode) {
@@ -381,6 +382,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float* ab = VARIANT == kPremix ? p.alpha + static_cast<size_t>(b) * p.n : alpha_s;
       for (int i = 0; i < p.n; ++i) bb = fmaf(ab[i], p.bias[static_cast<size_t>(i) * p.Cout + co], bb);
     }
+    // output attention: y = a_out * (conv + mixed bias), channel by channel
+    const float so = (p.a_out != nullptr && co < p.Cout) ? p.a_out[static_cast<size_t>(b) * p.Cout + co] : 1.f;
     if (wait_bounded(accum_bar, 0, ctl, kErrWaitEpilogue)) {
       tc_fence_after();
       // Per warp: chunks of 32 pixels x 32 output channels. The next chunk's
@@ -405,7 +408,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       auto process = [&](const uint32_t (&r)[32], int ch) {
 #pragma unroll
         for (int jj = 0; jj < 32; jj += 2) {
-          const uint32_t w = pack_bf16x2(__uint_as_float(r[jj]) + bb, __uint_as_float(r[jj + 1]) + bb);
+          const uint32_t w = pack_bf16x2((__uint_as_float(r[jj]) + bb) * so,
+                                         (__uint_as_float(r[jj + 1]) + bb) * so);
           asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + jj * 64 + lane * 2),
                        "h"(static_cast<unsigned short>(w & 0xFFFFu))
                        : "memory");

@@ -47,6 +47,8 @@ struct DwParams {
   __nv_bfloat16* y;
   int* err;
   long long wait_ns;
+  const float* a_in;               // [B][C] input channel attention, or null
+  const float* a_out;              // [B][C] output channel attention, or null
 };
 
 template <int K>
@@ -144,11 +146,18 @@ __global__ void __launch_bounds__(kDwThreads, K <= 5 ? 2 : 1)
   const int c = c0 + 2 * cp;
   if (!tile_ok || ct >= p.col_threads || c >= p.C) return;
 
-  // weights of the channel pair, packed (lo = channel c, hi = channel c+1)
+  // weights of the channel pair, packed (lo = channel c, hi = channel c+1);
+  // input attention scales the channel's kernel (depthwise: one input channel)
+  const float ai0 = p.a_in ? p.a_in[static_cast<size_t>(b) * p.C + c] : 1.f;
+  const float ai1 = p.a_in ? p.a_in[static_cast<size_t>(b) * p.C + c + 1] : 1.f;
   uint64_t w2[KK];
 #pragma unroll
-  for (int k = 0; k < KK; ++k) w2[k] = pack_f32x2(w_s[(2 * cp) * KK + k], w_s[(2 * cp + 1) * KK + k]);
+  for (int k = 0; k < KK; ++k)
+    w2[k] = pack_f32x2(w_s[(2 * cp) * KK + k] * ai0, w_s[(2 * cp + 1) * KK + k] * ai1);
   const uint64_t bias2 = pack_f32x2(bias_s[2 * cp], bias_s[2 * cp + 1]);
+  // output attention: y = a_out * (conv + mixed bias)
+  const float ao0 = p.a_out ? p.a_out[static_cast<size_t>(b) * p.C + c] : 1.f;
+  const float ao1 = p.a_out ? p.a_out[static_cast<size_t>(b) * p.C + c + 1] : 1.f;
   __nv_bfloat16* yb = p.y + static_cast<size_t>(b) * p.Ho * p.Wo * p.C;
 
   // this thread's two adjacent output columns
@@ -186,8 +195,14 @@ __global__ void __launch_bounds__(kDwThreads, K <= 5 ? 2 : 1)
           acc[kh % 3][0] = ffma2(win[(j + kh) % K][kw], w, acc[kh % 3][0]);
           acc[kh % 3][1] = ffma2(win[(j + kh) % K][kw + 1], w, acc[kh % 3][1]);
         }
-      const uint64_t s0 = fadd2(fadd2(acc[0][0], acc[1][0]), acc[2][0]);
-      const uint64_t s1 = fadd2(fadd2(acc[0][1], acc[1][1]), acc[2][1]);
+      uint64_t s0 = fadd2(fadd2(acc[0][0], acc[1][0]), acc[2][0]);
+      uint64_t s1 = fadd2(fadd2(acc[0][1], acc[1][1]), acc[2][1]);
+      if (p.a_out) {
+        s0 = pack_f32x2(__uint_as_float(static_cast<uint32_t>(s0)) * ao0,
+                        __uint_as_float(static_cast<uint32_t>(s0 >> 32)) * ao1);
+        s1 = pack_f32x2(__uint_as_float(static_cast<uint32_t>(s1)) * ao0,
+                        __uint_as_float(static_cast<uint32_t>(s1 >> 32)) * ao1);
+      }
       const int oh = oh0 + orow;
       if (oh < p.Ho) {
         __nv_bfloat16* dst = yb + (static_cast<size_t>(oh) * p.Wo + ow) * p.C + c;

@@ -28,6 +28,8 @@ struct DirectParams {
   const float* alpha;
   const float* bias;  // may be null
   void* y;
+  const float* a_in;   // [B][Cin] input channel attention, or null
+  const float* a_out;  // [B][Cout] output channel attention, or null
 };
 
 template <typename T>
@@ -57,6 +59,10 @@ __global__ void __launch_bounds__(kDirectThreads) direct_conv_kernel(DirectParam
     const size_t off = static_cast<size_t>(co0) * wrow + e;
     float s = 0.f;
     for (int i = 0; i < p.n; ++i) s = fmaf(alpha_s[i], to_f32<T>(E[i * wsize + off]), s);
+    if (p.a_in != nullptr) {  // input attention of channel (group of co) * Cg + ci
+      const int cl = e / wrow, ci = e % Cg;
+      s *= p.a_in[static_cast<size_t>(b) * p.Cin + ((co0 + cl) / Coutg) * Cg + ci];
+    }
     w_s[e] = s;
   }
   for (int c = threadIdx.x; c < cob; c += kDirectThreads) {
@@ -91,6 +97,7 @@ __global__ void __launch_bounds__(kDirectThreads) direct_conv_kernel(DirectParam
         for (int ci = 0; ci < Cg; ++ci) acc = fmaf(to_f32<T>(xp[ci]), wp[ci], acc);
       }
     }
+    if (p.a_out != nullptr) acc *= p.a_out[static_cast<size_t>(b) * p.Cout + co];
     yb[static_cast<size_t>(pix) * p.Cout + co] = from_f32<T>(acc);
   }
 }

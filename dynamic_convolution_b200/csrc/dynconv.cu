@@ -502,10 +502,15 @@ int run_mixconv(const dynconv_desc* d, const TcPlan& plan_in, const DeviceState*
 
 int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void* x,
            const void* experts, const float* alpha, const float* bias, void* y, void* ws,
-           size_t ws_bytes, cudaStream_t stream, float* ysum = nullptr) {
+           size_t ws_bytes, cudaStream_t stream, float* ysum = nullptr,
+           const float* a_in = nullptr, const float* a_out = nullptr) {
+  // input attention is folded into the mixed kernel: only the PREMIX variant
+  // with the CUDA-core mixer takes it
+  if (a_in != nullptr && variant != DYNCONV_VARIANT_PREMIX) return DYNCONV_ERR_UNSUPPORTED;
   TcPlan plan;
   if (!tc_plan(d, variant, st->sms, st->max_smem_optin, &plan)) return DYNCONV_ERR_UNSUPPORTED;
   plan.p.ysum = ysum;
+  plan.p.a_out = a_out;
   plan.p.experts = static_cast<const __nv_bfloat16*>(experts);
   plan.p.alpha = alpha;
   plan.p.bias = bias;
@@ -526,7 +531,7 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   if (!aligned16(ws)) return DYNCONV_ERR_MISALIGNED;
   plan.p.inject_skip = 0;
   if (g_stream_mix.load() && g_premix_mixer.load() != 1 && d->n <= dc::kMcMaxExperts &&
-      ysum == nullptr) {
+      ysum == nullptr && a_in == nullptr && a_out == nullptr) {
     rc = encode_w_map(&wmap, ws, d);
     if (rc) return rc;
     rc = run_mixconv(d, plan, st, experts, alpha, bias, y, ws, xmap, wmap, stream);
@@ -543,10 +548,17 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
       ps.experts = static_cast<const __nv_bfloat16*>(experts);
       ps.alpha = alpha;
       ps.out = static_cast<__nv_bfloat16*>(ws);
-      const size_t smem = sizeof(float) * static_cast<size_t>(d->B) * d->n;
+      ps.a_in = a_in;
+      ps.Cin = d->C_in;
+      size_t smem = sizeof(float) * static_cast<size_t>(d->B) * d->n;
+      if (a_in != nullptr) smem += sizeof(float) * static_cast<size_t>(d->B) * d->C_in;
+      if (smem > static_cast<size_t>(st->max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
       auto kern = d->n <= 2 ? dc::premix_small_kernel<2>
                   : d->n <= 4 ? dc::premix_small_kernel<4> : dc::premix_small_kernel<8>;
-      cudaError_t e = launch_pdl(kern, dim3(grid), dim3(dc::kPsThreads), smem, stream, ps);
+      cudaError_t e = cudaSuccess;
+      if (smem > 48 * 1024) e = ensure_smem(kern, smem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix_small)");
+      e = launch_pdl(kern, dim3(grid), dim3(dc::kPsThreads), smem, stream, ps);
       if (e != cudaSuccess) {
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return cuda_fail(e, "premix_small_kernel launch");
@@ -559,6 +571,7 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
     }
     if (g_premix_mixer.load() == 2) return DYNCONV_ERR_UNSUPPORTED;
   }
+  if (a_in != nullptr) return DYNCONV_ERR_UNSUPPORTED;  // the GEMM mixer does not take it
   dc::PremixLaunch pl;
   rc = dc::plan_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
                        static_cast<__nv_bfloat16*>(ws), d->B, d->n,
@@ -775,7 +788,8 @@ int resolve_variant(const dynconv_desc* desc, size_t ws_bytes, const DeviceState
 
 int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
                  const float* alpha, const float* bias, void* y, void* workspace,
-                 size_t workspace_bytes, void* stream, float* ysum) {
+                 size_t workspace_bytes, void* stream, float* ysum,
+                 const float* a_in = nullptr, const float* a_out = nullptr) {
   int rc = validate_desc(desc);
   if (rc) return rc;
   if (!x || !experts || !alpha || !y) return DYNCONV_ERR_INVALID_ARG;
@@ -785,7 +799,15 @@ int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  const int variant = resolve_variant(desc, workspace ? workspace_bytes : 0, st);
+  int variant = resolve_variant(desc, workspace ? workspace_bytes : 0, st);
+  if (a_in != nullptr && desc->variant == DYNCONV_VARIANT_AUTO &&
+      (variant == DYNCONV_VARIANT_FUSED || variant == DYNCONV_VARIANT_OUTSIDE ||
+       (variant == DYNCONV_VARIANT_PREMIX && desc->n > dc::kPsMaxExperts))) {
+    // input attention needs the CUDA-core mixer (PREMIX, n <= 8) or a CUDA-core kernel
+    const bool premix_ok = desc->n <= dc::kPsMaxExperts && workspace != nullptr &&
+                           premix_workspace(desc) != 0 && workspace_bytes >= premix_workspace(desc);
+    variant = premix_ok ? DYNCONV_VARIANT_PREMIX : DYNCONV_VARIANT_DIRECT;
+  }
 
   switch (variant) {
     case DYNCONV_VARIANT_FUSED:
@@ -794,7 +816,7 @@ int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
       if (!tc_shape_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
       if (!aligned16(x) || !aligned16(experts) || !aligned16(y)) return DYNCONV_ERR_MISALIGNED;
       return run_tc(desc, variant, st, x, experts, alpha, bias, y, workspace, workspace_bytes, s,
-                    ysum);
+                    ysum, a_in, a_out);
     }
     case DYNCONV_VARIANT_DEPTHWISE: {
       if (!depthwise_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
@@ -814,6 +836,8 @@ int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
       p.y = static_cast<__nv_bfloat16*>(y);
       p.err = st->err;
       p.wait_ns = g_wait_ns.load();
+      p.a_in = a_in;
+      p.a_out = a_out;
       const int TC = ((p.cols + 1) & ~1) + K - 1, TR = p.rows + K - 1;
       const size_t tile_bytes = static_cast<size_t>(TR) * TC * dc::kDwChunk * 2;
       const size_t smem = 128 + ((tile_bytes + 127) & ~size_t(127)) +
@@ -868,6 +892,7 @@ int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
       p.Wo = out_size(desc->W, desc->KW, desc->stride, desc->pad);
       p.cob = static_cast<int>(cob);
       p.x = x; p.experts = experts; p.alpha = alpha; p.bias = bias; p.y = y;
+      p.a_in = a_in; p.a_out = a_out;
       const size_t smem = sizeof(float) * (desc->n + cob + cob * wrow);
       dim3 grid((p.Ho * p.Wo + dc::kDirectPix - 1) / dc::kDirectPix,
                 static_cast<unsigned>((desc->C_out + cob - 1) / cob), desc->B);
@@ -900,6 +925,37 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
                     size_t workspace_bytes, void* stream) {
   return forward_impl(desc, x, experts, alpha, bias, y, workspace, workspace_bytes, stream,
                       nullptr);
+}
+
+int dynconv_forward_attn(const dynconv_desc* desc, const void* x, const void* experts,
+                         const float* alpha, const float* bias, const float* a_in,
+                         const float* a_out, void* y, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  return forward_impl(desc, x, experts, alpha, bias, y, workspace, workspace_bytes, stream,
+                      nullptr, a_in, a_out);
+}
+
+int dynconv_route_channels(const dynconv_desc* desc, const void* x, const float* Wi,
+                           const float* bi, float* a_in, const float* Wo, const float* bo,
+                           float* a_out, void* stream) {
+  int rc = validate_desc(desc);
+  if (rc) return rc;
+  if (!x || (!Wi && !Wo) || (Wi && !a_in) || (Wo && !a_out)) return DYNCONV_ERR_INVALID_ARG;
+  // each attention is the routing computation with one output per channel
+  // and the sigmoid activation
+  if (Wi) {
+    dynconv_desc di = *desc;
+    di.n = desc->C_in;
+    rc = dynconv_route(&di, x, Wi, bi, DYNCONV_SIGMOID, 1.0f, a_in, stream);
+    if (rc) return rc;
+  }
+  if (Wo) {
+    dynconv_desc dout = *desc;
+    dout.n = desc->C_out;
+    rc = dynconv_route(&dout, x, Wo, bo, DYNCONV_SIGMOID, 1.0f, a_out, stream);
+    if (rc) return rc;
+  }
+  return DYNCONV_OK;
 }
 
 int dynconv_forward_pooled(const dynconv_desc* desc, const void* x, const void* experts,

@@ -33,17 +33,22 @@ struct PsParams {
   const __nv_bfloat16* experts;  // [n][wsize]
   const float* alpha;            // [B][n]
   __nv_bfloat16* out;            // [B][wsize]
+  const float* a_in;             // [B][Cin] input channel attention, or null
+  int Cin;                       // input channels (with a_in: weight w has channel w % Cin)
 };
 
 // NMAX: the expert count rounded up to 2, 4 or 8 (fewer registers for fewer experts)
 template <int NMAX>
 __global__ void __launch_bounds__(kPsThreads) premix_small_kernel(PsParams p) {
-  extern __shared__ float ps_alpha[];  // [B][n]
+  extern __shared__ float ps_alpha[];  // [B][n], then [B][Cin] when a_in is given
+  float* ps_ain = ps_alpha + p.B * p.n;
   // the convolution may be scheduled as soon as every CTA of this grid runs
   grid_launch_dependents();
   grid_dependency_wait();  // alpha comes from the routing kernel
   const int na = p.B * p.n;
   for (int e = threadIdx.x; e < na; e += kPsThreads) ps_alpha[e] = p.alpha[e];
+  if (p.a_in != nullptr)
+    for (int e = threadIdx.x; e < p.B * p.Cin; e += kPsThreads) ps_ain[e] = p.a_in[e];
   __syncthreads();
 
   const long long stride = static_cast<long long>(gridDim.x) * kPsThreads;
@@ -68,6 +73,10 @@ __global__ void __launch_bounds__(kPsThreads) premix_small_kernel(PsParams p) {
     }
     const int b0 = static_cast<int>(sb) * p.sblock;
     const int b1 = min(p.B, b0 + p.sblock);
+    // with input attention: the 8 weights are 8 consecutive input channels of
+    // one (output channel, tap); the factor of channel c scales W_b[., ., c]
+    // (linearity: the same as scaling input channel c of x)
+    const int cin0 = p.a_in != nullptr ? static_cast<int>((ch * 8) % p.Cin) : 0;
 #pragma unroll 2
     for (int b = b0; b < b1; ++b) {
       const float* ab = ps_alpha + b * p.n;
@@ -80,6 +89,13 @@ __global__ void __launch_bounds__(kPsThreads) premix_small_kernel(PsParams p) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) acc[q] = ffma2(a2, ef[i][q], acc[q]);
         }
+      }
+      if (p.a_in != nullptr) {
+        const float* ai = ps_ain + b * p.Cin + cin0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          acc[q] = pack_f32x2(__uint_as_float(static_cast<uint32_t>(acc[q])) * ai[2 * q],
+                              __uint_as_float(static_cast<uint32_t>(acc[q] >> 32)) * ai[2 * q + 1]);
       }
       uint4 o;
       o.x = pack_bf16x2(__uint_as_float(static_cast<uint32_t>(acc[0])),
@@ -103,6 +119,8 @@ inline bool plan_premix_small(int B, int n, long long wsize, int sms, PsParams* 
                               unsigned* grid) {
   if (n < 1 || n > kPsMaxExperts || B < 1 || wsize % 8 != 0) return false;
   if (static_cast<long long>(B) * n * 4 > 16384) return false;
+  p->a_in = nullptr;
+  p->Cin = 0;
   const long long chunks = wsize / 8;
   const long long target = static_cast<long long>(sms) * kPsThreads;
   int sblock = 16;

@@ -132,6 +132,39 @@ int dynconv_forward(const dynconv_desc* desc, const void* x, const void* experts
                     const float* alpha, const float* bias, void* y, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* ---- FMDConv channel attentions ----------------------------------------------
+ * FMDConv combines the kernel attention with an input attention and an output
+ * attention (FMDConv: Fast multi-attention dynamic convolution via
+ * speed-accuracy trade-off, abstract). The page gives no formula; the reading
+ * taken: per-sample, per-channel factors in (0, 1), computed like the kernel
+ * attention from the average pool g_b of the layer input,
+ *   a_in[b][c]  = sigmoid(Wi[c][:] . g_b + bi[c])   (c < C_in),
+ *   a_out[b][o] = sigmoid(Wo[o][:] . g_b + bo[o])   (o < C_out),
+ * and applied as y_b = a_out_b * (conv2d(a_in_b * x_b, W_b) + sum_i alpha_bi bias_i),
+ * each factor multiplying one channel of every pixel.
+ *
+ * dynconv_route_channels: a_in and/or a_out (either pair Wi/a_in or Wo/a_out
+ * may be NULL, not both): Wi fp32 [C_in][C_in], bi fp32 [C_in] or NULL,
+ * a_in fp32 [B][C_in]; Wo fp32 [C_out][C_in], bo [C_out] or NULL, a_out fp32
+ * [B][C_out]; x as dynconv_route. Deterministic.
+ * Errors: INVALID_ARG, UNSUPPORTED (C_in or C_out > 1024), MISALIGNED, CUDA.
+ *
+ * dynconv_forward_attn: dynconv_forward with a_in [B][C_in] and a_out
+ * [B][C_out] (device fp32, either NULL = all ones). The output factor is taken
+ * in every variant's epilogue. The input factor is folded into the mixed
+ * kernel (W_b[o][kh][kw][c] * a_in[b][c], the same by linearity); variants that
+ * take it: PREMIX with the CUDA-core mixer (n <= 8), DEPTHWISE, DIRECT. With
+ * a_in and variant AUTO the choice falls back to those; a forced FUSED or
+ * OUTSIDE variant with a_in returns UNSUPPORTED.
+ * Errors as dynconv_forward. */
+int dynconv_route_channels(const dynconv_desc* desc, const void* x, const float* Wi,
+                           const float* bi, float* a_in, const float* Wo, const float* bo,
+                           float* a_out, void* stream);
+int dynconv_forward_attn(const dynconv_desc* desc, const void* x, const void* experts,
+                         const float* alpha, const float* bias, const float* a_in,
+                         const float* a_out, void* y, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
 /* ---- routing pooled in the previous layer (chained layers) -----------------
  * When layer L+1's input is layer L's output, the average pool of L+1's
  * routing step can be taken in L's epilogue, where the output is already in

@@ -137,3 +137,15 @@ def test_pooled_entry_points_host_side(lib):
         d = dc.desc_from_config(synth.CONFIGS[name])
         parts = dc.dynconv_pool_parts(d, dc.dynconv_workspace_size(d))
         assert 1 <= parts <= synth.CONFIGS[name].H
+
+
+def test_attention_entry_points_host_side(lib):
+    d = _desc(dtype=dc.BF16)
+    # neither attention requested, or an output missing for a given weight
+    assert dc.dynconv_route_channels(d, 16, None, None, None, None, None, None) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_route_channels(d, 16, 16, None, None, None, None, None) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_route_channels(d, None, 16, None, 16, None, None, None) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_forward_attn(d, None, 16, 16, None, 16, 16, 16) == dc.ERR_INVALID_ARG
+    for kw in BAD:
+        assert dc.dynconv_forward_attn(_desc(**kw), 16, 16, 16, None, None, None, 16) == \
+            dc.ERR_INVALID_ARG
