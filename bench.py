@@ -475,20 +475,31 @@ def run_ours(args, cfg):
                   + cfg.n * cfg.weight_elems) * eb
     src_hash = kernel_source_hash()
     variant_name = dc.VARIANT_NAMES.get(chosen, str(chosen))
-    if cfg.dtype == synth.BF16 and cfg.groups == 1:
+    # the bound: tensor cores when the layer's arithmetic intensity (conv FLOP per
+    # algorithmic byte) is above the ridge of the two measured peaks, else HBM
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    tensor_bound = (cfg.dtype == synth.BF16 and cfg.groups == 1
+                    and conv_flops / max(algo_bytes, 1) >= ridge)
+    if variant_name == "premix":
+        mixer = "premix_small_kernel" if cfg.n <= 8 else "premix_kernel"
+        kernel_label = f"forward call: {mixer} + tc_conv_kernel<premix>"
+    elif variant_name in ("fused", "outside"):
+        kernel_label = f"tc_conv_kernel<{variant_name}>"
+    else:
+        kernel_label = f"{variant_name}_kernel"
+    if tensor_bound:
         achieved = conv_flops / (fwd_launch_ms / 1e3) / 1e12
         peak = float(peaks["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "peak_kind": f"bf16 dense burst, {peak_kind}",
-                "kernel": ("forward call: premix_kernel + tc_conv_kernel<premix>"
-                           if variant_name == "premix" else f"tc_conv_kernel<{variant_name}>"),
+                "kernel": kernel_label,
                 "algorithmic": f"{conv_flops} conv FLOP per launch (2*B*HW*Cout*Cin*KH*KW)"}
     else:
         achieved = algo_bytes / (fwd_launch_ms / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": f"HBM copy, {peak_kind}",
-                "kernel": f"{variant_name}_kernel",
+                "kernel": kernel_label,
                 "algorithmic": f"{algo_bytes} bytes per launch (x + y + experts)"}
     roof["traffic"] = profile_traffic(variant_name, cfg.name, src_hash)
     roof["launch_ms"] = fwd_launch_ms
