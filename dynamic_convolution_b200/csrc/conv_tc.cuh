@@ -24,8 +24,8 @@
 // depends on the variant:
 //   FUSED    A = sum_i alpha_{b,i} E_i[co-tile][tap][c-chunk], mixed by 8 warps
 //            on CUDA cores from 16-byte expert loads and rounded once to bf16:
-//            "a linear mixture of n static kernels weighted with their
-//            input-dependent attentions" (KernelWarehouse, abstract), one
+//            the kernel is a weighted sum of n static kernels with weights
+//            that depend on the input (KernelWarehouse, abstract), one
 //            kernel per example (CondConv, abstract);
 //   OUTSIDE  the step also runs over the experts and A = alpha_{b,i} E_i: the
 //            sum over experts happens in the accumulator,

@@ -3,7 +3,7 @@
 // fp32 path and the path for bf16 shapes the tensor-core kernels do not take.
 //
 // y_b = conv2d(x_b, sum_i alpha_{b,i} W_i) + sum_i alpha_{b,i} bias_i: the mixed
-// kernel of "a linear mixture of n static kernels" (KernelWarehouse, abstract)
+// kernel, a weighted sum of n static kernels (KernelWarehouse, abstract),
 // applied per example (CondConv, abstract); cross-correlation with zero
 // padding is the reading taken.
 //

@@ -1,9 +1,9 @@
 // PREMIX with the kernel mixing streamed into the convolution: one persistent
 // cooperative kernel, one CTA per SM, for few experts (n <= 8).
 //
-//   W_b = sum_i alpha[b][i] E_i for every sample b ("a linear mixture of n
-//   static kernels weighted with their input-dependent attentions",
-//   KernelWarehouse, abstract; one kernel per example, CondConv, abstract),
+//   W_b = sum_i alpha[b][i] E_i for every sample b (n static kernels summed
+//   with weights that depend on the input, KernelWarehouse, abstract; one
+//   kernel per example, CondConv, abstract),
 //   then y_b = conv(x_b, W_b) + sum_i alpha[b][i] bias_i.
 //
 // The convolution consumes W_b one K step (one tap of one 64-channel chunk)

@@ -1,6 +1,6 @@
 // Tensor-core kernel mixing: W[b][w] = sum_i alpha[b][i] * E[i][w] for every
-// sample b and every weight element w -- "a linear mixture of n static
-// kernels weighted with their input-dependent attentions" (KernelWarehouse,
+// sample b and every weight element w -- n static kernels summed with weights
+// that depend on the input (KernelWarehouse,
 // abstract), done for all samples at once so that every expert byte is read
 // from HBM once per pass instead of once per sample.
 //

@@ -1,8 +1,8 @@
 // Kernel mixing on CUDA cores for few experts (n <= 8):
 //     W[b][w] = sum_i alpha[b][i] * E[i][w]
-// for every sample b and weight element w -- the per-example "linear mixture
-// of n static kernels weighted with their input-dependent attentions"
-// (KernelWarehouse, abstract; CondConv, abstract: one kernel per example).
+// for every sample b and weight element w -- each example's kernel is n static
+// kernels summed with weights that depend on the input (KernelWarehouse,
+// abstract; CondConv, abstract: one kernel per example).
 //
 // With n <= 8 the mixing costs at most 4 FMAs per output byte, so it is a
 // store-bound stream, not a GEMM: a thread takes 8 consecutive weights (one

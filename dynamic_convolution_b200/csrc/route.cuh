@@ -1,6 +1,6 @@
 // Routing kernel: alpha_b = act(Wr * GAP(x_b) + br).
 //
-// The routing weights are "input-dependent attentions" over n static kernels
+// The routing weights are attentions over n static kernels computed from the input
 // (KernelWarehouse: Rethinking the Design of Dynamic Convolution, abstract),
 // one vector per example (CondConv, abstract), with a temperature on the
 // softmax (FMDConv, abstract: temperature-degraded kernel attention). The

@@ -7,8 +7,8 @@
  *   W_b     = sum_i alpha_{b,i} W_i                 (n static experts W_i)
  *   y_b     = conv2d(x_b, W_b) + sum_i alpha_{b,i} bias_i
  *
- * Sources: the linear mixture of n static kernels weighted with input-dependent
- * attentions is the definition in "KernelWarehouse: Rethinking the Design of
+ * Sources: the kernel as a sum of n static kernels, each weighted by an
+ * attention computed from the input, is the definition in "KernelWarehouse: Rethinking the Design of
  * Dynamic Convolution" (abstract); one specialised kernel per example is
  * "CondConv: Conditionally Parameterized Convolutions for Efficient Inference"
  * (abstract); the temperature on the kernel attention is from "FMDConv: Fast

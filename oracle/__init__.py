@@ -8,9 +8,11 @@ The arithmetic lives in ``dynconv_oracle.c`` (plain C, fp64, direct loops,
 threads over samples only). This module compiles it with gcc and marshals
 numpy arrays in and out; it adds no arithmetic of its own.
 
-Every function here is pinned by ``tests/test_oracle_pins.py`` against closed
-forms, a library convolution (n=1), brute force on tiny inputs and the
-identities that the pages' definition implies.
+Every forward function here is pinned by ``tests/test_oracle_pins.py`` against
+closed forms, a library convolution (n=1), brute force on tiny inputs and the
+identities that the pages' definition implies; the backward functions by
+``tests/test_oracle_backward.py`` against central differences of the pinned
+forward and against torch autograd of the same definition.
 """
 from __future__ import annotations
 
@@ -59,6 +61,15 @@ def configure(lib):
     lib.oracle_assemble.restype = None
     lib.oracle_threads_used.argtypes = [i, i]
     lib.oracle_threads_used.restype = i
+    lib.oracle_weight_grad.argtypes = [i] * 10 + [dp, dp, i, i, dp, dp, i]
+    lib.oracle_weight_grad.restype = i
+    lib.oracle_backward_weight.argtypes = [i] * 11 + [dp, dp, dp, dp, dp, dp, dp, dp, i]
+    lib.oracle_backward_weight.restype = i
+    lib.oracle_route_backward.argtypes = [i, i, i, i, dp, i, dp, dp, dp, i, ctypes.c_double,
+                                          dp, dp, dp]
+    lib.oracle_route_backward.restype = i
+    lib.oracle_backward_data.argtypes = [i] * 11 + [dp, dp, dp, dp, i, i, dp, i]
+    lib.oracle_backward_data.restype = i
     return lib
 
 
@@ -191,3 +202,105 @@ def assemble(experts, alpha_b):
     out = np.empty(experts.shape[1:], dtype=np.float64)
     _load().oracle_assemble(n, wsize, _dp(experts), _dp(alpha_b), _dp(out))
     return out
+
+
+# ------------------------------------------------------------------ backward
+
+
+def weight_grad(x, dy, KH: int, KW: int, stride: int = 1, pad: int = 0, groups: int = 1,
+                samples: tuple[int, int] | None = None, nthreads: int = 0):
+    """Per-sample gradients of the convolution's weight and bias:
+    dW[nb][C_out][KH][KW][C_in/groups] and db[nb][C_out] for samples b0..b0+nb-1."""
+    x = _f64(x)
+    dy = _f64(dy)
+    B, H, W, Cin = x.shape
+    Cout = dy.shape[3]
+    assert dy.shape[:3] == (B, (H + 2 * pad - KH) // stride + 1, (W + 2 * pad - KW) // stride + 1)
+    b0, nb = (0, B) if samples is None else samples
+    dW = np.empty((nb, Cout, KH, KW, Cin // groups), dtype=np.float64)
+    db = np.empty((nb, Cout), dtype=np.float64)
+    rc = _load().oracle_weight_grad(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, _dp(x),
+                                    _dp(dy), b0, nb, _dp(dW), _dp(db), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_weight_grad rejected its arguments (rc={rc})")
+    return dW, db
+
+
+def backward_weight(x, dy, experts, alpha, bias=None, stride: int = 1, pad: int = 0,
+                    groups: int = 1, nthreads: int = 0):
+    """(dexperts[n][C_out][KH][KW][C_in/groups], dbias[n][C_out] or None, dalpha[B][n])."""
+    x = _f64(x)
+    dy = _f64(dy)
+    experts = _f64(experts)
+    alpha = _f64(alpha)
+    bias = _f64(bias)
+    B, H, W, Cin = x.shape
+    n, Cout, KH, KW, Cg = experts.shape
+    assert Cg * groups == Cin and alpha.shape == (B, n)
+    assert bias is None or bias.shape == (n, Cout)
+    assert dy.shape == (B, (H + 2 * pad - KH) // stride + 1, (W + 2 * pad - KW) // stride + 1, Cout)
+    dexperts = np.empty(experts.shape, dtype=np.float64)
+    dbias = None if bias is None else np.empty((n, Cout), dtype=np.float64)
+    dalpha = np.empty((B, n), dtype=np.float64)
+    rc = _load().oracle_backward_weight(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n,
+                                        _dp(x), _dp(dy), _dp(experts), _dp(alpha), _dp(bias),
+                                        _dp(dexperts), _dp(dbias), _dp(dalpha), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_backward_weight rejected its arguments (rc={rc})")
+    return dexperts, dbias, dalpha
+
+
+def route_backward(x, Wr, alpha, dalpha, mode: int, tau: float = 1.0):
+    """(dWr[n][C], dbr[n], dg[B][C]) from dalpha[B][n] through the activation and
+    the linear layer; dg is the gradient of each sample's pooled vector."""
+    x = _f64(x)
+    Wr = _f64(Wr)
+    alpha = _f64(alpha)
+    dalpha = _f64(dalpha)
+    B, H, W, C = x.shape
+    n = Wr.shape[0]
+    assert Wr.shape == (n, C) and alpha.shape == (B, n) and dalpha.shape == (B, n)
+    dWr = np.empty((n, C), dtype=np.float64)
+    dbr = np.empty(n, dtype=np.float64)
+    dg = np.empty((B, C), dtype=np.float64)
+    rc = _load().oracle_route_backward(B, C, H, W, _dp(x), n, _dp(Wr), _dp(alpha), _dp(dalpha),
+                                       int(mode), float(tau), _dp(dWr), _dp(dbr), _dp(dg))
+    if rc != 0:
+        raise ValueError(f"oracle_route_backward rejected its arguments (rc={rc})")
+    return dWr, dbr, dg
+
+
+def backward_data(dy, experts, alpha, dg, H: int, W: int, stride: int = 1, pad: int = 0,
+                  groups: int = 1, samples: tuple[int, int] | None = None, nthreads: int = 0):
+    """dx[nb][H][W][C_in] for samples b0..b0+nb-1: the input gradient through the
+    convolution with W_b, plus dg[b][c]/(H*W) when dg is given (else None)."""
+    dy = _f64(dy)
+    experts = _f64(experts)
+    alpha = _f64(alpha)
+    dg = _f64(dg)
+    B = dy.shape[0]
+    n, Cout, KH, KW, Cg = experts.shape
+    Cin = Cg * groups
+    assert dy.shape == (B, (H + 2 * pad - KH) // stride + 1, (W + 2 * pad - KW) // stride + 1, Cout)
+    assert alpha.shape == (B, n) and (dg is None or dg.shape == (B, Cin))
+    b0, nb = (0, B) if samples is None else samples
+    dx = np.empty((nb, H, W, Cin), dtype=np.float64)
+    rc = _load().oracle_backward_data(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n,
+                                      _dp(dy), _dp(experts), _dp(alpha), _dp(dg), b0, nb,
+                                      _dp(dx), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_backward_data rejected its arguments (rc={rc})")
+    return dx
+
+
+def backward(x, dy, experts, alpha, bias, Wr, mode: int, tau: float = 1.0, stride: int = 1,
+             pad: int = 0, groups: int = 1, nthreads: int = 0):
+    """Every gradient of one layer with its router, given dy: a dict with dx,
+    dexperts, dbias, dalpha, dWr, dbr, dg (the three steps above in order)."""
+    x = _f64(x)
+    H, W = x.shape[1], x.shape[2]
+    dexperts, dbias, dalpha = backward_weight(x, dy, experts, alpha, bias, stride, pad, groups,
+                                              nthreads)
+    dWr, dbr, dg = route_backward(x, Wr, alpha, dalpha, mode, tau)
+    dx = backward_data(dy, experts, alpha, dg, H, W, stride, pad, groups, nthreads=nthreads)
+    return dict(dx=dx, dexperts=dexperts, dbias=dbias, dalpha=dalpha, dWr=dWr, dbr=dbr, dg=dg)

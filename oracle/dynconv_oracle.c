@@ -10,21 +10,21 @@
  * samples only; each sample is computed exactly as a single thread would.
  *
  * What is computed, and where it comes from:
- *   routing   alpha_b = act(FC(GAP(x_b)))  -- "input-dependent attentions"
- *             (KernelWarehouse: Rethinking the Design of Dynamic Convolution,
+ *   routing   alpha_b = act(FC(GAP(x_b)))  -- attentions computed from the
+ *             input (KernelWarehouse: Rethinking the Design of Dynamic Convolution,
  *             abstract), one attention vector per example (CondConv:
  *             Conditionally Parameterized Convolutions for Efficient Inference,
  *             abstract); the temperature divides the logits before the softmax
- *             ("temperature-degraded kernel attention", FMDConv: Fast
+ *             (the kernel attention carries a temperature, FMDConv: Fast
  *             multi-attention dynamic convolution via speed-accuracy trade-off,
  *             abstract). The GAP -> single linear layer -> sigmoid/softmax form
  *             is the reading taken where the pages are silent.
  *   assembly  W_b = sum_i alpha_{b,i} W_i, b_b = sum_i alpha_{b,i} bias_i
- *             ("a linear mixture of n static kernels weighted with their
- *             input-dependent attentions", KernelWarehouse abstract).
+ *             (n static kernels summed with weights that depend on the
+ *             input, KernelWarehouse abstract).
  *   conv      y_b = conv2d(x_b, W_b) + b_b, cross-correlation with zero padding
- *             ("specialized convolutional kernels for each example", CondConv
- *             abstract); orientation and padding are readings, pinned by tests.
+ *             (a kernel specialised to each example, CondConv abstract);
+ *             orientation and padding are readings, pinned by tests.
  *
  * Layouts (all row-major, fastest index last):
  *   x       [B][H][W][C_in]                      (NHWC)
@@ -296,4 +296,223 @@ int oracle_forward_rows(int B, int Cin, int H, int W, int Cout, int KH, int KW, 
                x, experts, alpha, bias, y, NULL, NULL};
   forward_one(&f, b);
   return 0;
+}
+
+/* =============================================================== backward */
+/*
+ * Gradients of a scalar loss through one layer, given dy = dL/dy
+ * [B][Ho][Wo][Cout]. The per-example kernels and the mixture are learned
+ * (CondConv, abstract; KernelWarehouse, abstract), so the layer is trained
+ * through the derivative of the definition above. Each function is that
+ * derivative, one forward step at a time (chain rule), written as plainly as
+ * the forward:
+ *
+ *   conv      dW_b[co,kh,kw,ci] = sum_{oh,ow} dy[b,oh,ow,co] xpad[b, oh*s+kh-p, ow*s+kw-p, g*Cg+ci]
+ *             db_b[co]          = sum_{oh,ow} dy[b,oh,ow,co]
+ *             dx_b              = every dy[b,oh,ow,co] * W_b[co,kh,kw,ci] added back onto the
+ *                                 input element that the forward read with it
+ *   assembly  dexperts_i = sum_b alpha[b,i] dW_b        dbias_i = sum_b alpha[b,i] db_b
+ *             dalpha[b,i] = <dW_b, W_i> + <db_b, bias_i>
+ *   act       sigmoid: dz = dalpha * alpha * (1 - alpha)
+ *             softmax of z/tau: dz_i = alpha_i * (dalpha_i - sum_j alpha_j dalpha_j) / tau
+ *   FC        dWr[i,c] = sum_b dz[b,i] g[b,c],  dbr[i] = sum_b dz[b,i],
+ *             dg[b,c] = sum_i dz[b,i] Wr[i,c]
+ *   GAP       dx[b,h,w,c] += dg[b,c] / (H*W)   (every unpadded pixel)
+ */
+
+typedef struct {
+  int Cin, H, W, Cout, KH, KW, stride, pad, groups, Ho, Wo, b0;
+  const double *x, *dy;
+  double *dW;   /* [nb][Cout][KH][KW][Cg] */
+  double *db;   /* [nb][Cout] */
+} wgrad_ctx;
+
+static void wgrad_one(void *vctx, int b) {
+  wgrad_ctx *f = (wgrad_ctx *)vctx;
+  const int Cg = f->Cin / f->groups, Coutg = f->Cout / f->groups;
+  const long wsize = (long)f->Cout * f->KH * f->KW * Cg;
+  double *dW = f->dW + (size_t)(b - f->b0) * wsize;
+  double *db = f->db + (size_t)(b - f->b0) * f->Cout;
+  memset(dW, 0, sizeof(double) * (size_t)wsize);
+  memset(db, 0, sizeof(double) * (size_t)f->Cout);
+  const double *xb = f->x + (size_t)b * f->H * f->W * f->Cin;
+  const double *dyb = f->dy + (size_t)b * f->Ho * f->Wo * f->Cout;
+  for (int oh = 0; oh < f->Ho; ++oh)
+    for (int ow = 0; ow < f->Wo; ++ow)
+      for (int co = 0; co < f->Cout; ++co) {
+        const double d = dyb[((size_t)oh * f->Wo + ow) * f->Cout + co];
+        const size_t cin0 = (size_t)(co / Coutg) * Cg;   /* first input channel of co's group */
+        db[co] += d;
+        for (int kh = 0; kh < f->KH; ++kh)
+          for (int kw = 0; kw < f->KW; ++kw) {
+            /* the input element the forward multiplied with W_b[co,kh,kw,.] */
+            const int y_in = f->stride * oh - f->pad + kh, x_in = f->stride * ow - f->pad + kw;
+            if (y_in < 0 || y_in >= f->H || x_in < 0 || x_in >= f->W) continue;  /* padding */
+            const double *xp = xb + ((size_t)y_in * f->W + x_in) * f->Cin + cin0;
+            double *gw = dW + ((size_t)(co * f->KH + kh) * f->KW + kw) * Cg;
+            for (int ci = 0; ci < Cg; ++ci) gw[ci] += d * xp[ci];
+          }
+      }
+}
+
+static int bwd_shape_ok(int B, int Cin, int H, int W, int Cout, int KH, int KW, int stride,
+                        int pad, int groups, int n) {
+  if (B < 0 || Cin <= 0 || H <= 0 || W <= 0 || Cout <= 0 || KH <= 0 || KW <= 0) return 0;
+  if (stride <= 0 || pad < 0 || groups <= 0 || n <= 0) return 0;
+  if (Cin % groups != 0 || Cout % groups != 0) return 0;
+  if (oracle_out_size(H, KH, stride, pad) <= 0 || oracle_out_size(W, KW, stride, pad) <= 0)
+    return 0;
+  return 1;
+}
+
+/* Per-sample gradients of the convolution's weight and bias for samples
+ * b0 .. b0+nb-1: dW[nb][Cout][KH][KW][Cin/groups], db[nb][Cout]. */
+int oracle_weight_grad(int B, int Cin, int H, int W, int Cout, int KH, int KW, int stride,
+                       int pad, int groups, const double *x, const double *dy, int b0, int nb,
+                       double *dW, double *db, int nthreads) {
+  if (!bwd_shape_ok(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, 1)) return -1;
+  if (!x || !dy || !dW || !db || b0 < 0 || nb < 0 || b0 + nb > B) return -1;
+  if (nb == 0) return 0;
+  wgrad_ctx f = {Cin, H, W, Cout, KH, KW, stride, pad, groups,
+                 oracle_out_size(H, KH, stride, pad), oracle_out_size(W, KW, stride, pad), b0,
+                 x, dy, dW, db};
+  return run_samples(wgrad_one, &f, b0, nb, nthreads);
+}
+
+/* The assembly step's gradients: dexperts[n][wsize], dbias[n][Cout] (only when
+ * bias is given) and dalpha[B][n], from the per-sample gradients of all B
+ * samples. Sums over samples run in sample order. */
+int oracle_backward_weight(int B, int Cin, int H, int W, int Cout, int KH, int KW, int stride,
+                           int pad, int groups, int n, const double *x, const double *dy,
+                           const double *experts, const double *alpha, const double *bias,
+                           double *dexperts, double *dbias, double *dalpha, int nthreads) {
+  if (!bwd_shape_ok(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n)) return -1;
+  if (!x || !dy || !experts || !alpha || !dexperts || !dalpha || (bias && !dbias)) return -1;
+  const long wsize = (long)Cout * KH * KW * (Cin / groups);
+  double *dW = (double *)malloc(sizeof(double) * (size_t)(B > 0 ? B : 1) * (size_t)wsize);
+  double *db = (double *)malloc(sizeof(double) * (size_t)(B > 0 ? B : 1) * (size_t)Cout);
+  if (!dW || !db) { free(dW); free(db); return -1; }
+  int rc = B > 0 ? oracle_weight_grad(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, x, dy, 0,
+                                      B, dW, db, nthreads)
+                 : 0;
+  if (rc == 0) {
+    for (int b = 0; b < B; ++b)
+      for (int i = 0; i < n; ++i) {
+        double s = 0.0;
+        for (long e = 0; e < wsize; ++e) s += dW[(size_t)b * wsize + e] * experts[(size_t)i * wsize + e];
+        if (bias)
+          for (int co = 0; co < Cout; ++co) s += db[(size_t)b * Cout + co] * bias[(size_t)i * Cout + co];
+        dalpha[(size_t)b * n + i] = s;
+      }
+    for (int i = 0; i < n; ++i) {
+      for (long e = 0; e < wsize; ++e) {
+        double s = 0.0;
+        for (int b = 0; b < B; ++b) s += alpha[(size_t)b * n + i] * dW[(size_t)b * wsize + e];
+        dexperts[(size_t)i * wsize + e] = s;
+      }
+      if (bias)
+        for (int co = 0; co < Cout; ++co) {
+          double s = 0.0;
+          for (int b = 0; b < B; ++b) s += alpha[(size_t)b * n + i] * db[(size_t)b * Cout + co];
+          dbias[(size_t)i * Cout + co] = s;
+        }
+    }
+  }
+  free(dW);
+  free(db);
+  return rc;
+}
+
+/* The router's gradients: dz from dalpha through the activation, then the
+ * linear layer's dWr[n][C], dbr[n] (sums over samples, in sample order) and
+ * dg[B][C], the gradient of the pooled vector g of every sample. */
+int oracle_route_backward(int B, int C, int H, int W, const double *x, int n, const double *Wr,
+                          const double *alpha, const double *dalpha, int mode, double tau,
+                          double *dWr, double *dbr, double *dg) {
+  if (B < 0 || C <= 0 || H <= 0 || W <= 0 || n <= 0) return -1;
+  if (!x || !Wr || !alpha || !dalpha || !dWr || !dbr || !dg) return -1;
+  if (mode != ORACLE_SIGMOID && mode != ORACLE_SOFTMAX) return -1;
+  if (mode == ORACLE_SOFTMAX && !(tau > 0.0)) return -1;
+  double *g = (double *)malloc(sizeof(double) * (size_t)C);
+  double *dz = (double *)malloc(sizeof(double) * (size_t)n);
+  if (!g || !dz) { free(g); free(dz); return -1; }
+  memset(dWr, 0, sizeof(double) * (size_t)n * C);
+  memset(dbr, 0, sizeof(double) * (size_t)n);
+  for (int b = 0; b < B; ++b) {
+    const double *a = alpha + (size_t)b * n, *da = dalpha + (size_t)b * n;
+    if (mode == ORACLE_SIGMOID) {
+      for (int i = 0; i < n; ++i) dz[i] = da[i] * a[i] * (1.0 - a[i]);
+    } else {
+      double dot = 0.0;
+      for (int j = 0; j < n; ++j) dot += a[j] * da[j];
+      for (int i = 0; i < n; ++i) dz[i] = a[i] * (da[i] - dot) / tau;
+    }
+    oracle_gap(C, H, W, x + (size_t)b * H * W * C, g);
+    for (int c = 0; c < C; ++c) {
+      double s = 0.0;
+      for (int i = 0; i < n; ++i) s += dz[i] * Wr[(size_t)i * C + c];
+      dg[(size_t)b * C + c] = s;
+    }
+    for (int i = 0; i < n; ++i) {
+      dbr[i] += dz[i];
+      for (int c = 0; c < C; ++c) dWr[(size_t)i * C + c] += dz[i] * g[c];
+    }
+  }
+  free(g);
+  free(dz);
+  return 0;
+}
+
+typedef struct {
+  int Cin, H, W, Cout, KH, KW, stride, pad, groups, n, Ho, Wo, b0;
+  const double *dy, *experts, *alpha, *dg;
+  double *dx;   /* [nb][H][W][Cin] */
+} dgrad_ctx;
+
+static void dgrad_one(void *vctx, int b) {
+  dgrad_ctx *f = (dgrad_ctx *)vctx;
+  const int Cg = f->Cin / f->groups, Coutg = f->Cout / f->groups;
+  const long wsize = (long)f->Cout * f->KH * f->KW * Cg;
+  double *Wb = (double *)malloc(sizeof(double) * (size_t)wsize);
+  oracle_assemble(f->n, wsize, f->experts, f->alpha + (size_t)b * f->n, Wb);
+  double *dxb = f->dx + (size_t)(b - f->b0) * f->H * f->W * f->Cin;
+  memset(dxb, 0, sizeof(double) * (size_t)f->H * f->W * f->Cin);
+  const double *dyb = f->dy + (size_t)b * f->Ho * f->Wo * f->Cout;
+  for (int oh = 0; oh < f->Ho; ++oh)
+    for (int ow = 0; ow < f->Wo; ++ow)
+      for (int co = 0; co < f->Cout; ++co) {
+        const double d = dyb[((size_t)oh * f->Wo + ow) * f->Cout + co];
+        const size_t cin0 = (size_t)(co / Coutg) * Cg;
+        for (int kh = 0; kh < f->KH; ++kh)
+          for (int kw = 0; kw < f->KW; ++kw) {
+            const int y_in = f->stride * oh - f->pad + kh, x_in = f->stride * ow - f->pad + kw;
+            if (y_in < 0 || y_in >= f->H || x_in < 0 || x_in >= f->W) continue;  /* padding */
+            double *gx = dxb + ((size_t)y_in * f->W + x_in) * f->Cin + cin0;
+            const double *wv = Wb + ((size_t)(co * f->KH + kh) * f->KW + kw) * Cg;
+            for (int ci = 0; ci < Cg; ++ci) gx[ci] += d * wv[ci];
+          }
+      }
+  if (f->dg) {
+    const double *dgb = f->dg + (size_t)b * f->Cin;
+    const double inv = 1.0 / (double)(f->H * f->W);
+    for (long p = 0; p < (long)f->H * f->W; ++p)
+      for (int c = 0; c < f->Cin; ++c) dxb[(size_t)p * f->Cin + c] += dgb[c] * inv;
+  }
+  free(Wb);
+}
+
+/* dx[nb][H][W][Cin] for samples b0 .. b0+nb-1: the convolution's input
+ * gradient with the mixed kernel W_b, plus dg[b,c]/(H*W) on every pixel when
+ * dg [B][Cin] is given (the pooled vector's gradient; NULL: none). */
+int oracle_backward_data(int B, int Cin, int H, int W, int Cout, int KH, int KW, int stride,
+                         int pad, int groups, int n, const double *dy, const double *experts,
+                         const double *alpha, const double *dg, int b0, int nb, double *dx,
+                         int nthreads) {
+  if (!bwd_shape_ok(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n)) return -1;
+  if (!dy || !experts || !alpha || !dx || b0 < 0 || nb < 0 || b0 + nb > B) return -1;
+  if (nb == 0) return 0;
+  dgrad_ctx f = {Cin, H, W, Cout, KH, KW, stride, pad, groups, n,
+                 oracle_out_size(H, KH, stride, pad), oracle_out_size(W, KW, stride, pad), b0,
+                 dy, experts, alpha, dg, dx};
+  return run_samples(dgrad_one, &f, b0, nb, nthreads);
 }

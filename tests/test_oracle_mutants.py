@@ -9,6 +9,7 @@ import pytest
 
 import oracle
 
+from . import test_oracle_backward as bw
 from . import test_oracle_pins as pins
 
 # (name, original text, mutated text) -- each replacement must hit exactly once
@@ -31,6 +32,40 @@ MUTANTS = [
      "for (int ci = 0; ci < Cg; ++ci) s += (ap[Cg - 1 - ci] * xp[ci]) * wp[ci];"),
     ("output_attention_before_bias", "double s = bb[co];", "double s = aout ? bb[co] / aout[co] : bb[co];"),
     ("output_attention_dropped", "if (aout) s *= aout[co];", "if (0) s *= aout[co];"),
+    # backward
+    ("sigmoid_grad_missing_factor", "dz[i] = da[i] * a[i] * (1.0 - a[i]);", "dz[i] = da[i] * a[i];"),
+    ("softmax_grad_missing_tau", "dz[i] = a[i] * (da[i] - dot) / tau;",
+     "dz[i] = a[i] * (da[i] - dot);"),
+    ("softmax_grad_not_centred", "dz[i] = a[i] * (da[i] - dot) / tau;", "dz[i] = a[i] * da[i] / tau;"),
+    ("pool_grad_not_averaged", "dxb[(size_t)p * f->Cin + c] += dgb[c] * inv;",
+     "dxb[(size_t)p * f->Cin + c] += dgb[c];"),
+    ("pool_grad_dropped", "if (f->dg) {", "if (0) {"),
+    ("dalpha_bias_term_dropped",
+     "s += db[(size_t)b * Cout + co] * bias[(size_t)i * Cout + co];",
+     "s += 0.0 * db[(size_t)b * Cout + co];"),
+    ("dexperts_wrong_expert",
+     "for (int b = 0; b < B; ++b) s += alpha[(size_t)b * n + i] * dW[(size_t)b * wsize + e];",
+     "for (int b = 0; b < B; ++b) s += alpha[(size_t)b * n + (n - 1 - i)] * dW[(size_t)b * wsize + e];"),
+    ("dbias_without_alpha",
+     "for (int b = 0; b < B; ++b) s += alpha[(size_t)b * n + i] * db[(size_t)b * Cout + co];",
+     "for (int b = 0; b < B; ++b) s += db[(size_t)b * Cout + co];"),
+    ("weight_grad_channel_reversed", "for (int ci = 0; ci < Cg; ++ci) gw[ci] += d * xp[ci];",
+     "for (int ci = 0; ci < Cg; ++ci) gw[ci] += d * xp[Cg - 1 - ci];"),
+    ("data_grad_kernel_flipped",
+     "const double *wv = Wb + ((size_t)(co * f->KH + kh) * f->KW + kw) * Cg;",
+     "const double *wv = Wb + ((size_t)(co * f->KH + (f->KH - 1 - kh)) * f->KW + (f->KW - 1 - kw)) * Cg;"),
+    ("weight_grad_stride_ignored",
+     "const int y_in = f->stride * oh - f->pad + kh, x_in = f->stride * ow - f->pad + kw;\n"
+     "            if (y_in < 0 || y_in >= f->H || x_in < 0 || x_in >= f->W) continue;  /* padding */\n"
+     "            const double *xp",
+     "const int y_in = oh - f->pad + kh, x_in = ow - f->pad + kw;\n"
+     "            if (y_in < 0 || y_in >= f->H || x_in < 0 || x_in >= f->W) continue;  /* padding */\n"
+     "            const double *xp"),
+    ("router_weight_grad_uses_dalpha",
+     "for (int c = 0; c < C; ++c) dWr[(size_t)i * C + c] += dz[i] * g[c];",
+     "for (int c = 0; c < C; ++c) dWr[(size_t)i * C + c] += da[i] * g[c];"),
+    ("pool_grad_wrong_router_row", "for (int i = 0; i < n; ++i) s += dz[i] * Wr[(size_t)i * C + c];",
+     "for (int i = 0; i < n; ++i) s += dz[i] * Wr[(size_t)(n - 1 - i) * C + c];"),
 ]
 
 PIN_TESTS = [
@@ -45,6 +80,13 @@ PIN_TESTS = [
     pins.test_route_invariants,
     lambda: [pins.test_channel_attention_matches_torch_conv(s) for s in pins.SHAPES],
     pins.test_channel_attention_zero_input_gives_scaled_bias,
+    # backward
+    lambda: [bw.test_central_differences_every_input(c) for c in bw.CASES],
+    lambda: [bw.test_central_differences_attention_as_input(c) for c in bw.CASES[:4]],
+    lambda: [bw.test_matches_torch_autograd(c) for c in bw.CASES],
+    bw.test_softmax_router_gradients_sum_to_zero_over_experts,
+    bw.test_zero_input_leaves_bias_terms,
+    bw.test_pooled_gradient_adds_a_constant_per_channel,
 ]
 
 
@@ -66,6 +108,7 @@ def test_pins_catch_mutant(tmp_path, name, orig, mut):
                 t()
             except (AssertionError, ValueError):
                 failures += 1
+                break  # one failing pin is enough
     finally:
         oracle._lib = saved
     assert failures > 0, f"no pin caught mutant {name}"

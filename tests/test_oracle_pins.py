@@ -5,8 +5,8 @@ a library convolution for n=1, a second brute-force formulation (explicit
 im2col matrix, experts summed on the output side), closed forms (impulse,
 constant input, zero input), library activations, and the identities that the
 definition implies (linearity in the kernel, batch and expert permutation).
-The definition pinned here is the linear mixture of n static kernels weighted
-by input-dependent attentions (KernelWarehouse: Rethinking the Design of
+The definition pinned here is the sum of n static kernels, each weighted by an
+attention computed from the input (KernelWarehouse: Rethinking the Design of
 Dynamic Convolution, abstract), one kernel per example (CondConv:
 Conditionally Parameterized Convolutions for Efficient Inference, abstract),
 and temperature-scaled softmax attention (FMDConv: Fast multi-attention
