@@ -70,6 +70,12 @@ def configure(lib):
     lib.oracle_route_backward.restype = i
     lib.oracle_backward_data.argtypes = [i] * 11 + [dp, dp, dp, dp, i, i, dp, i]
     lib.oracle_backward_data.restype = i
+    lib.oracle_dalpha.argtypes = [i] * 11 + [dp, dp, dp, dp, i, i, dp, i]
+    lib.oracle_dalpha.restype = i
+    lib.oracle_dexperts_at.argtypes = [i] * 11 + [dp, dp, dp, i, ctypes.POINTER(ctypes.c_long), dp]
+    lib.oracle_dexperts_at.restype = i
+    lib.oracle_dbias.argtypes = [i, i, i, i, dp, dp, dp]
+    lib.oracle_dbias.restype = i
     return lib
 
 
@@ -304,3 +310,52 @@ def backward(x, dy, experts, alpha, bias, Wr, mode: int, tau: float = 1.0, strid
     dWr, dbr, dg = route_backward(x, Wr, alpha, dalpha, mode, tau)
     dx = backward_data(dy, experts, alpha, dg, H, W, stride, pad, groups, nthreads=nthreads)
     return dict(dx=dx, dexperts=dexperts, dbias=dbias, dalpha=dalpha, dWr=dWr, dbr=dbr, dg=dg)
+
+
+def dalpha(x, dy, experts, bias, stride: int = 1, pad: int = 0, groups: int = 1,
+           samples: tuple[int, int] | None = None, nthreads: int = 0):
+    """dalpha[nb][n] of samples b0..b0+nb-1 (as backward_weight, restricted)."""
+    x = _f64(x)
+    dy = _f64(dy)
+    experts = _f64(experts)
+    bias = _f64(bias)
+    B, H, W, Cin = x.shape
+    n, Cout, KH, KW, Cg = experts.shape
+    b0, nb = (0, B) if samples is None else samples
+    out = np.empty((nb, n), dtype=np.float64)
+    rc = _load().oracle_dalpha(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n, _dp(x),
+                               _dp(dy), _dp(experts), _dp(bias), b0, nb, _dp(out), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_dalpha rejected its arguments (rc={rc})")
+    return out
+
+
+def dexperts_at(x, dy, alpha, idx, n: int, Cout: int, KH: int, KW: int, stride: int = 1,
+                pad: int = 0, groups: int = 1):
+    """dexperts[i][idx[k]] -> out[n][len(idx)] for flat indices into
+    [C_out][KH][KW][C_in/groups] (as backward_weight, restricted)."""
+    x = _f64(x)
+    dy = _f64(dy)
+    alpha = _f64(alpha)
+    B, H, W, Cin = x.shape
+    idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int64))
+    out = np.empty((n, len(idx)), dtype=np.float64)
+    rc = _load().oracle_dexperts_at(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n, _dp(x),
+                                    _dp(dy), _dp(alpha), len(idx),
+                                    idx.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), _dp(out))
+    if rc != 0:
+        raise ValueError(f"oracle_dexperts_at rejected its arguments (rc={rc})")
+    return out
+
+
+def dbias(dy, alpha):
+    """dbias[n][C_out] = sum_b alpha[b][i] * (dy[b] summed over pixels)."""
+    dy = _f64(dy)
+    alpha = _f64(alpha)
+    B, Ho, Wo, Cout = dy.shape
+    n = alpha.shape[1]
+    out = np.empty((n, Cout), dtype=np.float64)
+    rc = _load().oracle_dbias(B, Ho * Wo, Cout, n, _dp(dy), _dp(alpha), _dp(out))
+    if rc != 0:
+        raise ValueError(f"oracle_dbias rejected its arguments (rc={rc})")
+    return out

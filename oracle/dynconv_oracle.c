@@ -516,3 +516,98 @@ int oracle_backward_data(int B, int Cin, int H, int W, int Cout, int KH, int KW,
                  dy, experts, alpha, dg, dx};
   return run_samples(dgrad_one, &f, b0, nb, nthreads);
 }
+
+/* ------------------------------------------------ restrictions for spot checks
+ * The same definitions as oracle_backward_weight, restricted so that large
+ * layers can be checked without holding every sample's gradient: dalpha of a
+ * range of samples, dexperts at chosen weight elements, and dbias. */
+
+typedef struct {
+  int Cin, H, W, Cout, KH, KW, stride, pad, groups, n;
+  const double *x, *dy, *experts, *bias;
+  double *dalpha;   /* [nb][n] */
+  int b0;
+} dalpha_ctx;
+
+static void dalpha_one(void *vctx, int b) {
+  dalpha_ctx *f = (dalpha_ctx *)vctx;
+  const long wsize = (long)f->Cout * f->KH * f->KW * (f->Cin / f->groups);
+  double *dW = (double *)malloc(sizeof(double) * (size_t)wsize);
+  double *db = (double *)malloc(sizeof(double) * (size_t)f->Cout);
+  wgrad_ctx w = {f->Cin, f->H, f->W, f->Cout, f->KH, f->KW, f->stride, f->pad, f->groups,
+                 oracle_out_size(f->H, f->KH, f->stride, f->pad),
+                 oracle_out_size(f->W, f->KW, f->stride, f->pad), b, f->x, f->dy, dW, db};
+  wgrad_one(&w, b);
+  for (int i = 0; i < f->n; ++i) {
+    double s = 0.0;
+    for (long e = 0; e < wsize; ++e) s += dW[e] * f->experts[(size_t)i * wsize + e];
+    if (f->bias)
+      for (int co = 0; co < f->Cout; ++co) s += db[co] * f->bias[(size_t)i * f->Cout + co];
+    f->dalpha[(size_t)(b - f->b0) * f->n + i] = s;
+  }
+  free(dW);
+  free(db);
+}
+
+/* dalpha[nb][n] of samples b0 .. b0+nb-1. */
+int oracle_dalpha(int B, int Cin, int H, int W, int Cout, int KH, int KW, int stride, int pad,
+                  int groups, int n, const double *x, const double *dy, const double *experts,
+                  const double *bias, int b0, int nb, double *dalpha, int nthreads) {
+  if (!bwd_shape_ok(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n)) return -1;
+  if (!x || !dy || !experts || !dalpha || b0 < 0 || nb < 0 || b0 + nb > B) return -1;
+  if (nb == 0) return 0;
+  dalpha_ctx f = {Cin, H, W, Cout, KH, KW, stride, pad, groups, n, x, dy, experts, bias, dalpha, b0};
+  return run_samples(dalpha_one, &f, b0, nb, nthreads);
+}
+
+/* dexperts[i][idx[k]] for the flat weight indices idx[0 .. nidx-1] (layout
+ * [C_out][KH][KW][C_in/groups]), written to out[n][nidx]: the per-sample
+ * gradient of that one weight, summed over samples in order with alpha. */
+int oracle_dexperts_at(int B, int Cin, int H, int W, int Cout, int KH, int KW, int stride,
+                       int pad, int groups, int n, const double *x, const double *dy,
+                       const double *alpha, int nidx, const long *idx, double *out) {
+  if (!bwd_shape_ok(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, n)) return -1;
+  if (!x || !dy || !alpha || !idx || !out || nidx < 0) return -1;
+  const int Cg = Cin / groups, Coutg = Cout / groups;
+  const int Ho = oracle_out_size(H, KH, stride, pad), Wo = oracle_out_size(W, KW, stride, pad);
+  const long wsize = (long)Cout * KH * KW * Cg;
+  for (int k = 0; k < nidx; ++k) {
+    const long e = idx[k];
+    if (e < 0 || e >= wsize) return -1;
+    const int cil = (int)(e % Cg);
+    const int kw = (int)((e / Cg) % KW), kh = (int)((e / Cg / KW) % KH);
+    const int co = (int)(e / Cg / KW / KH);
+    const int ci = (co / Coutg) * Cg + cil;
+    for (int i = 0; i < n; ++i) out[(size_t)i * nidx + k] = 0.0;
+    for (int b = 0; b < B; ++b) {
+      double g = 0.0;
+      for (int oh = 0; oh < Ho; ++oh)
+        for (int ow = 0; ow < Wo; ++ow) {
+          const int y_in = stride * oh - pad + kh, x_in = stride * ow - pad + kw;
+          if (y_in < 0 || y_in >= H || x_in < 0 || x_in >= W) continue;
+          g += dy[(((size_t)b * Ho + oh) * Wo + ow) * Cout + co] *
+               x[(((size_t)b * H + y_in) * W + x_in) * Cin + ci];
+        }
+      for (int i = 0; i < n; ++i) out[(size_t)i * nidx + k] += alpha[(size_t)b * n + i] * g;
+    }
+  }
+  return 0;
+}
+
+/* dbias[n][Cout] = sum_b alpha[b][i] * (sum over output pixels of dy[b][.][.][co]). */
+int oracle_dbias(int B, int HoWo, int Cout, int n, const double *dy, const double *alpha,
+                 double *dbias) {
+  if (B < 0 || HoWo <= 0 || Cout <= 0 || n <= 0 || !dy || !alpha || !dbias) return -1;
+  double *db = (double *)malloc(sizeof(double) * (size_t)Cout);
+  if (!db) return -1;
+  memset(dbias, 0, sizeof(double) * (size_t)n * Cout);
+  for (int b = 0; b < B; ++b) {
+    for (int co = 0; co < Cout; ++co) db[co] = 0.0;
+    for (long p = 0; p < HoWo; ++p)
+      for (int co = 0; co < Cout; ++co) db[co] += dy[((size_t)b * HoWo + p) * Cout + co];
+    for (int i = 0; i < n; ++i)
+      for (int co = 0; co < Cout; ++co) dbias[(size_t)i * Cout + co] += alpha[(size_t)b * n + i] * db[co];
+  }
+  free(db);
+  return 0;
+}

@@ -209,3 +209,22 @@ def test_sample_ranges_match_full():
     # the per-sample gradients recombine to the mixture's gradients
     dE, dbias, dalpha = oracle.backward_weight(L["x"], L["dy"], L["E"], alpha, L["bias"], s, p, g)
     np.testing.assert_allclose(dE, np.einsum("bi,b...->i...", alpha, dW), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("case", CASES, ids=IDS)
+def test_restrictions_match_the_full_functions(case):
+    """dalpha of a sample range, dexperts at chosen elements and dbias equal the
+    corresponding parts of backward_weight (pinned above)."""
+    B, Cin, Cout, H, W, KH, KW, s, p, g, n, mode, tau = case
+    L = _layer(case, 10)
+    alpha = L["rng"].uniform(0.1, 1, (B, n))
+    dE, dbias, dalpha = oracle.backward_weight(L["x"], L["dy"], L["E"], alpha, L["bias"], s, p, g)
+    np.testing.assert_allclose(oracle.dalpha(L["x"], L["dy"], L["E"], L["bias"], s, p, g),
+                               dalpha, rtol=1e-12, atol=1e-12)
+    b0 = B - 1
+    np.testing.assert_allclose(oracle.dalpha(L["x"], L["dy"], L["E"], L["bias"], s, p, g,
+                                             samples=(b0, 1)), dalpha[b0:], rtol=1e-12, atol=1e-12)
+    idx = L["rng"].choice(dE[0].size, size=min(17, dE[0].size), replace=False)
+    got = oracle.dexperts_at(L["x"], L["dy"], alpha, idx, n, Cout, KH, KW, s, p, g)
+    np.testing.assert_allclose(got, dE.reshape(n, -1)[:, idx], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(oracle.dbias(L["dy"], alpha), dbias, rtol=1e-12, atol=1e-12)
