@@ -28,6 +28,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -52,6 +53,8 @@ def parse():
     ap.add_argument("--variant", default="auto",
                     choices=["auto", "fused", "outside", "premix", "direct", "depthwise"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the layer's backward step (weight, router and input gradients)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--hooks", default="",
                     help="implementation knobs for comparisons, e.g. '6=0,5=0' "
@@ -232,13 +235,23 @@ def profile_traffic(kernel_tag: str, workload: str, src_hash: str):
 
 
 def kernel_source_hash() -> str:
-    h = hashlib.sha256()
+    """Hash of the forward translation unit's sources: dynconv.cu and every
+    csrc header it includes, directly or not (the backward unit compiles
+    separately and cannot change the forward kernels)."""
     csrc = os.path.join(ROOT, "dynamic_convolution_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode())
-                h.update(f.read())
+    seen, todo = set(), ["dynconv.cu"]
+    while todo:
+        fn = todo.pop()
+        if fn in seen or not os.path.exists(os.path.join(csrc, fn)):
+            continue
+        seen.add(fn)
+        with open(os.path.join(csrc, fn)) as f:
+            todo += re.findall(r'^#include "([^"]+)"', f.read(), flags=re.M)
+    h = hashlib.sha256()
+    for fn in sorted(seen):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -628,11 +641,115 @@ def run_block(args):
     return 0
 
 
+def run_backward(args, cfg):
+    """One layer's backward step on one GPU: dynconv_backward_weight,
+    dynconv_route_backward and dynconv_backward_data, with inputs, upstream
+    gradients and dx rotated over sets larger than L2 in total, in CUDA graphs
+    of 8 steps. Also times each call alone (same graphs, one call per step).
+    Effective TFLOP/s counts the two convolution-sized contractions (weight
+    gradient and input gradient): 2 x the forward's conv FLOPs."""
+    import torch
+
+    import dynamic_convolution_b200 as dc
+    from dynamic_convolution_b200 import build, synth
+
+    torch.cuda.set_device(0)
+    build.build()
+    dc.load()
+    inp = synth.make_inputs(cfg)
+    dys, _ = synth.make_upstream_grad(cfg)
+    tdt = torch.bfloat16 if cfg.dtype == synth.BF16 else torch.float32
+    dev = lambda a: (torch.from_numpy(a).view(torch.bfloat16) if cfg.dtype == synth.BF16
+                     else torch.from_numpy(a)).cuda()
+    x0, dy0, E = dev(inp.x_store), dev(dys), dev(inp.experts_store)
+    Wr, br, bias = (torch.from_numpy(a).cuda() for a in (inp.Wr, inp.br, inp.bias))
+    d = dc.desc_from_config(cfg)
+    wsb = dc.dynconv_backward_workspace_size(d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    set_bytes = (2 * x0.numel() + dy0.numel()) * x0.element_size()
+    nsets = max(2, min(64, math.ceil(2 * L2_BYTES / set_bytes)))
+    xs = [x0.clone() for _ in range(nsets)]
+    dys_ = [dy0.clone() for _ in range(nsets)]
+    dxs = [torch.empty_like(x0) for _ in range(nsets)]
+    alphas = [torch.empty((cfg.B, cfg.n), device="cuda") for _ in range(nsets)]
+    for k in range(nsets):
+        dc.check(dc.dynconv_route(d, xs[k], Wr, br, cfg.mode, cfg.tau, alphas[k]))
+    dE = torch.empty(E.shape, dtype=torch.float32, device="cuda")
+    dbias = torch.empty((cfg.n, cfg.C_out), device="cuda")
+    dalpha = torch.empty((cfg.B, cfg.n), device="cuda")
+    dWr = torch.empty((cfg.n, cfg.C_in), device="cuda")
+    dbr = torch.empty(cfg.n, device="cuda")
+    dg = torch.empty((cfg.B, cfg.C_in), device="cuda")
+    stream = torch.cuda.Stream()
+
+    def weight(s, st):
+        dc.check(dc.dynconv_backward_weight(d, xs[s], dys_[s], E, alphas[s], bias, dE, dbias,
+                                            dalpha, ws, wsb, st))
+
+    def router(s, st):
+        dc.check(dc.dynconv_route_backward(d, xs[s], Wr, alphas[s], dalpha, cfg.mode, cfg.tau,
+                                           dWr, dbr, dg, st))
+
+    def data(s, st):
+        dc.check(dc.dynconv_backward_data(d, dys_[s], E, alphas[s], dg, dxs[s], ws, wsb, st))
+
+    def full(s, st):
+        weight(s, st)
+        router(s, st)
+        data(s, st)
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for k in range(max(args.warmup, 3)):
+                fn(k % nsets, stream)
+        stream.synchronize()
+        per = min(8, nsets)
+        g = torch.cuda.CUDAGraph()
+        n0 = dc.dynconv_launch_count()
+        with torch.cuda.graph(g, stream=stream):
+            for k in range(per):
+                fn(k, stream)
+        launches = (dc.dynconv_launch_count() - n0) // per
+        reps = max(1, args.steps // per)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        dc.check(dc.dynconv_device_status(stream), "device status")
+        del g
+        return e0.elapsed_time(e1) / (reps * per), reps * per, launches
+
+    ms, steps, launches = timed(full)
+    parts = {name: round(timed(fn)[0] * 1e3, 2) for name, fn in
+             (("backward_weight", weight), ("route_backward", router), ("backward_data", data))}
+    tflops = 2 * cfg.conv_flops / (ms / 1e3) / 1e12
+    line = {"metric": "images/s (layer backward: expert, bias, attention, router and input "
+                      "gradients)",
+            "value": cfg.B / (ms / 1e3), "unit": "images/s", "n_gpus": 1, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32",
+            "data": "synthetic (seeded; recipe in DESIGN.md)",
+            "config": {"workload": f"{cfg.name} backward", "l2": f"inputs rotated over {nsets} sets"},
+            "effective_tflops": tflops, "us_per_call": parts, "gpu_launches_per_step": launches,
+            "wgrad_kernel": "tcgen05" if dc.VARIANT_AUTO == d.variant and cfg.dtype == synth.BF16
+            and cfg.groups == 1 and cfg.C_in % 8 == 0 and cfg.C_in >= 64 else "cuda-core"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     from dynamic_convolution_b200 import synth
     if args.config == "effnet_block":
         return run_block(args)
+    if args.backward:
+        return run_backward(args, synth.CONFIGS[args.config or synth.HEADLINE])
     name = args.config or synth.HEADLINE
     cfg = synth.CONFIGS[name]
     if args.impl == "reference":

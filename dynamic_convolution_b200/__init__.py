@@ -1,4 +1,5 @@
-"""Python binding of the sm_100a dynamic-convolution C ABI (``include/dynconv.h``).
+"""Python binding of the sm_100a dynamic-convolution C ABI (``include/dynconv.h``,
+``include/dynconv_backward.h``).
 
 Argument marshalling only: every function forwards to the symbol of the same
 name in ``libdynconv.so``; all arithmetic runs in the library's CUDA kernels.
@@ -29,7 +30,10 @@ SYMBOLS = ("dynconv_route", "dynconv_forward", "dynconv_forward_noalloc",
            "dynconv_route_channels", "dynconv_forward_attn",
            "dynconv_workspace_size", "dynconv_select_variant",
            "dynconv_status_string", "dynconv_last_error", "dynconv_device_status",
-           "dynconv_launch_count", "dynconv_test_hook")
+           "dynconv_launch_count", "dynconv_test_hook",
+           # include/dynconv_backward.h
+           "dynconv_backward_workspace_size", "dynconv_backward_weight",
+           "dynconv_route_backward", "dynconv_backward_data")
 
 
 class dynconv_desc(ctypes.Structure):
@@ -88,6 +92,15 @@ def load():
         lib.dynconv_launch_count.restype = ctypes.c_ulonglong
         lib.dynconv_test_hook.argtypes = [ctypes.c_int, ctypes.c_longlong]
         lib.dynconv_test_hook.restype = ctypes.c_int
+        lib.dynconv_backward_workspace_size.argtypes = [D]
+        lib.dynconv_backward_workspace_size.restype = ctypes.c_size_t
+        lib.dynconv_backward_weight.argtypes = [D, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.dynconv_backward_weight.restype = ctypes.c_int
+        lib.dynconv_route_backward.argtypes = [D, P, P, P, P, ctypes.c_int, ctypes.c_float, P, P,
+                                               P, P]
+        lib.dynconv_route_backward.restype = ctypes.c_int
+        lib.dynconv_backward_data.argtypes = [D, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.dynconv_backward_data.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -209,3 +222,36 @@ def dynconv_test_hook(key: int, value: int) -> int:
 def check(status: int, where: str = "dynconv") -> None:
     if status != OK:
         raise DynconvError(status, where)
+
+
+# ------------------------------------------------------------------ backward
+
+
+def dynconv_backward_workspace_size(desc) -> int:
+    return load().dynconv_backward_workspace_size(ctypes.byref(desc))
+
+
+def dynconv_backward_weight(desc, x, dy, experts, alpha, bias, dexperts, dbias, dalpha,
+                            workspace, workspace_bytes, stream=None) -> int:
+    """dexperts [n][C_out][KH][KW][C_in/groups], dbias [n][C_out] (None with no
+    bias), dalpha [B][n], all fp32, from the forward's x, alpha and dy."""
+    return load().dynconv_backward_weight(ctypes.byref(desc), _ptr(x), _ptr(dy), _ptr(experts),
+                                          _ptr(alpha), _ptr(bias), _ptr(dexperts), _ptr(dbias),
+                                          _ptr(dalpha), _ptr(workspace), int(workspace_bytes),
+                                          _stream(stream))
+
+
+def dynconv_route_backward(desc, x, Wr, alpha, dalpha, mode, tau, dWr, dbr, dg,
+                           stream=None) -> int:
+    """dWr [n][C_in], dbr [n] (may be None), dg [B][C_in] (fp32)."""
+    return load().dynconv_route_backward(ctypes.byref(desc), _ptr(x), _ptr(Wr), _ptr(alpha),
+                                         _ptr(dalpha), int(mode), float(tau), _ptr(dWr),
+                                         _ptr(dbr), _ptr(dg), _stream(stream))
+
+
+def dynconv_backward_data(desc, dy, experts, alpha, dg, dx, workspace, workspace_bytes,
+                          stream=None) -> int:
+    """dx [B][H][W][C_in] in the layer's dtype; dg [B][C_in] or None."""
+    return load().dynconv_backward_data(ctypes.byref(desc), _ptr(dy), _ptr(experts), _ptr(alpha),
+                                        _ptr(dg), _ptr(dx), _ptr(workspace),
+                                        int(workspace_bytes), _stream(stream))

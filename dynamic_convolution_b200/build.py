@@ -1,8 +1,9 @@
 """Build the sm_100a C-ABI library ``libdynconv.so`` in-tree with nvcc.
 
 Usage: ``python -m dynamic_convolution_b200.build`` (or ``build()`` from Python).
-The library is one translation unit (``csrc/dynconv.cu`` includes the kernel
-headers); it links the CUDA runtime statically and reaches the driver's
+The library has two translation units: ``csrc/dynconv.cu`` (the forward
+entry points; it includes the forward kernel headers) and ``csrc/backward.cu``
+(the backward entry points and kernels); it links the CUDA runtime statically and reaches the driver's
 tensor-map encoder through the runtime's entry-point query, so it loads on a
 machine without a GPU driver (the calls then fail with DYNCONV_ERR_CUDA).
 """
@@ -19,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdynconv.so")
+UNITS = [os.path.join(CSRC, "dynconv.cu"), os.path.join(CSRC, "backward.cu")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -52,7 +54,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *NVCC_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}",
-           os.path.join(CSRC, "dynconv.cu"), "-o", tmp]
+           *UNITS, "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)

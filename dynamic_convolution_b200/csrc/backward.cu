@@ -1,0 +1,395 @@
+// Host side of the backward entry points declared in include/dynconv_backward.h:
+// argument checks, workspace layout, tensor maps and launches. A translation
+// unit of its own (the forward unit, dynconv.cu, shares device state and
+// error reporting through internal.h); the input gradient reuses the forward
+// entry point on the transposed problem.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+
+#include "dynconv.h"
+#include "dynconv_backward.h"
+#include "internal.h"
+
+#include "backward_kernels.cuh"
+#include "backward_wgrad_tc.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int out_size(int in, int k, int stride, int pad) { return (in + 2 * pad - k) / stride + 1; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+size_t elem_bytes(const dynconv_desc* d) { return d->dtype == DYNCONV_F32 ? 4 : 2; }
+long long wsize_of(const dynconv_desc* d) {
+  return 1LL * d->C_out * d->KH * d->KW * (d->C_in / d->groups);
+}
+
+int launch_error(cudaError_t e, const char* what) {
+  dc_lib::launched(what);
+  return dc_lib::cuda_error(e, what);
+}
+
+// ------------------------------------------------------- workspace layout
+
+struct WeightLayout {
+  size_t dW = 0, db = 0, part = 0, total = 0;
+  int chunks = 0;
+};
+
+WeightLayout weight_layout(const dynconv_desc* d) {
+  WeightLayout L;
+  const long long ws = wsize_of(d);
+  L.chunks = static_cast<int>((ws + dcb::kMgChunk - 1) / dcb::kMgChunk);
+  L.dW = 0;
+  L.db = align256(L.dW + 4ull * d->B * ws);
+  L.part = align256(L.db + 4ull * d->B * d->C_out);
+  L.total = align256(L.part + 4ull * L.chunks * d->B * d->n);
+  return L;
+}
+
+// The input gradient as a forward convolution: stride 1 and one padding
+// value that stays non-negative after the flip (square kernels).
+bool transposed_ok(const dynconv_desc* d) {
+  return d->stride == 1 && d->KH == d->KW && d->KH - 1 - d->pad >= 0;
+}
+
+dynconv_desc transposed_desc(const dynconv_desc* d) {
+  dynconv_desc t = *d;
+  t.C_in = d->C_out;
+  t.C_out = d->C_in;
+  t.H = out_size(d->H, d->KH, 1, d->pad);
+  t.W = out_size(d->W, d->KW, 1, d->pad);
+  t.pad = d->KH - 1 - d->pad;
+  return t;
+}
+
+size_t data_workspace(const dynconv_desc* d) {
+  if (!transposed_ok(d)) return 0;
+  const dynconv_desc t = transposed_desc(d);
+  return align256(static_cast<size_t>(d->n) * wsize_of(d) * elem_bytes(d)) +
+         dynconv_workspace_size(&t);
+}
+
+// ------------------------------------------------- tensor-core weight gradient
+
+bool wgrad_tc_shape_ok(const dynconv_desc* d) {
+  const int Wo = out_size(d->W, d->KW, 1, d->pad);
+  return d->dtype == DYNCONV_BF16 && d->groups == 1 && d->stride == 1 && d->C_in % 8 == 0 &&
+         d->C_out % 8 == 0 && d->C_in >= 64 && d->C_out >= 64 && Wo <= 128;
+}
+
+int encode_4d(EncodeTiledFn enc, CUtensorMap* map, const void* base, int C, int W, int H, int B,
+              int box_w, int box_h) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(W),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * 2,
+                                 static_cast<cuuint64_t>(W) * C * 2,
+                                 static_cast<cuuint64_t>(H) * W * C * 2};
+  const cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(box_w), static_cast<cuuint32_t>(box_h),
+                             1u};
+  const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+  if (enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+          es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return dc_lib::fail(DYNCONV_ERR_CUDA, "cuTensorMapEncodeTiled (weight gradient) failed");
+  return DYNCONV_OK;
+}
+
+int run_wgrad_tc(const dynconv_desc* d, const dc_lib::DeviceInfo& di, const void* x,
+                 const void* dy, float* dW, cudaStream_t s) {
+  const int Ho = out_size(d->H, d->KH, 1, d->pad), Wo = out_size(d->W, d->KW, 1, d->pad);
+  dcb::WgParams p{};
+  p.B = d->B; p.Cin = d->C_in; p.Cout = d->C_out; p.Ho = Ho; p.Wo = Wo;
+  p.KH = d->KH; p.KW = d->KW; p.pad = d->pad;
+  // K tiles of whole output rows, at most 128 pixels, balanced
+  int tiles = (Ho * Wo + 127) / 128;
+  int BH = (Ho + tiles - 1) / tiles;
+  while (BH * Wo > 128) {
+    ++tiles;
+    BH = (Ho + tiles - 1) / tiles;
+  }
+  p.BH = BH;
+  p.ktiles = (Ho + BH - 1) / BH;
+  p.ksteps = (BH * Wo + 15) / 16;
+  p.atom_bytes = p.ksteps * 16 * 128;
+  p.box_bytes = BH * Wo * 128;
+  p.cblk = (d->C_in + 63) / 64;
+  p.natoms = d->KH * d->KW * p.cblk;
+  p.agroups = (p.natoms + dcb::kWgMaxAtoms - 1) / dcb::kWgMaxAtoms;
+  p.co_tiles = (d->C_out + 127) / 128;
+  p.units = 1LL * d->B * p.co_tiles * p.agroups;
+  const int stage_bytes = (2 + dcb::kWgMaxAtoms) * p.atom_bytes;
+  p.stages = std::min(4, (200 * 1024) / stage_bytes);
+  if (p.stages < 2) return dc_lib::fail(DYNCONV_ERR_UNSUPPORTED, "weight-gradient tile too large");
+  p.dW = dW;
+  p.err = di.err;
+  p.wait_ns = di.wait_ns;
+  auto enc = reinterpret_cast<EncodeTiledFn>(di.encode_tiled);
+  CUtensorMap dymap, xmap;
+  int rc = encode_4d(enc, &dymap, dy, d->C_out, Wo, Ho, d->B, Wo, BH);
+  if (rc) return rc;
+  rc = encode_4d(enc, &xmap, x, d->C_in, d->W, d->H, d->B, Wo, BH);
+  if (rc) return rc;
+  // at least 120 KB, so that two CTAs never share an SM (each holds all 512 TMEM columns)
+  const size_t smem = std::max<size_t>(
+      120 * 1024, 1024 + static_cast<size_t>(p.stages) * stage_bytes + 8 * (2 * p.stages + 5) + 16);
+  if (smem > static_cast<size_t>(di.max_smem_optin))
+    return dc_lib::fail(DYNCONV_ERR_UNSUPPORTED, "weight-gradient shared memory");
+  cudaError_t e = dc_lib::set_smem(reinterpret_cast<const void*>(dcb::wgrad_tc_kernel), smem);
+  if (e != cudaSuccess) return dc_lib::cuda_error(e, "cudaFuncSetAttribute(wgrad_tc)");
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(p.units, di.sms));
+  dcb::wgrad_tc_kernel<<<grid, dcb::kWgThreads, smem, s>>>(dymap, xmap, p);
+  return dc_lib::launched("wgrad_tc_kernel");
+}
+
+int run_wgrad_direct(const dynconv_desc* d, const void* x, const void* dy, float* dW,
+                     cudaStream_t s) {
+  dcb::WgdParams p{};
+  p.B = d->B; p.Cin = d->C_in; p.H = d->H; p.W = d->W; p.Cout = d->C_out;
+  p.KH = d->KH; p.KW = d->KW; p.stride = d->stride; p.pad = d->pad; p.groups = d->groups;
+  p.Ho = out_size(d->H, d->KH, d->stride, d->pad);
+  p.Wo = out_size(d->W, d->KW, d->stride, d->pad);
+  p.wsize = wsize_of(d);
+  p.x = x; p.dy = dy; p.dW = dW;
+  const dim3 grid(static_cast<unsigned>((p.wsize + dcb::kBwThreads - 1) / dcb::kBwThreads), d->B);
+  if (d->dtype == DYNCONV_F32)
+    dcb::wgrad_direct_kernel<float><<<grid, dcb::kBwThreads, 0, s>>>(p);
+  else
+    dcb::wgrad_direct_kernel<__nv_bfloat16><<<grid, dcb::kBwThreads, 0, s>>>(p);
+  return dc_lib::launched("wgrad_direct_kernel");
+}
+
+int run_chansum(const dynconv_desc* d, const void* v, int P, int C, float* out, cudaStream_t s) {
+  const dim3 grid((C + 31) / 32, d->B), block(32, 8);
+  if (d->dtype == DYNCONV_F32)
+    dcb::chansum_kernel<float><<<grid, block, 0, s>>>(static_cast<const float*>(v), P, C, out);
+  else
+    dcb::chansum_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(v), P, C, out);
+  return dc_lib::launched("chansum_kernel");
+}
+
+template <typename T>
+int launch_mixgrad(const dcb::MgParams& p, int ne, size_t smem, cudaStream_t s) {
+  const dim3 grid(p.chunks, (p.n + ne - 1) / ne);
+  auto go = [&](auto kern) -> int {
+    if (smem > 48 * 1024) {
+      cudaError_t e = dc_lib::set_smem(reinterpret_cast<const void*>(kern), smem);
+      if (e != cudaSuccess) return dc_lib::cuda_error(e, "cudaFuncSetAttribute(mixgrad)");
+    }
+    kern<<<grid, dcb::kBwThreads, smem, s>>>(p);
+    return dc_lib::launched("mixgrad_kernel");
+  };
+  switch (ne) {
+    case 1: return go(dcb::mixgrad_kernel<T, 1>);
+    case 2: return go(dcb::mixgrad_kernel<T, 2>);
+    case 4: return go(dcb::mixgrad_kernel<T, 4>);
+    default: return go(dcb::mixgrad_kernel<T, 8>);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dynconv_backward_workspace_size(const dynconv_desc* desc) {
+  if (dc_lib::validate(desc) != DYNCONV_OK) return 0;
+  return std::max(weight_layout(desc).total, data_workspace(desc));
+}
+
+int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void* dy,
+                            const void* experts, const float* alpha, const float* bias,
+                            float* dexperts, float* dbias, float* dalpha, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  int rc = dc_lib::validate(desc);
+  if (rc) return rc;
+  if (!x || !dy || !experts || !alpha || !dexperts || !dalpha) return DYNCONV_ERR_INVALID_ARG;
+  if ((bias == nullptr) != (dbias == nullptr)) return DYNCONV_ERR_INVALID_ARG;
+  const dynconv_desc* d = desc;
+  const bool tc_ok = wgrad_tc_shape_ok(d);
+  bool use_tc;
+  switch (d->variant) {
+    case DYNCONV_VARIANT_AUTO: use_tc = tc_ok; break;
+    case DYNCONV_VARIANT_FUSED:
+    case DYNCONV_VARIANT_OUTSIDE:
+    case DYNCONV_VARIANT_PREMIX:
+      if (!tc_ok) return DYNCONV_ERR_UNSUPPORTED;
+      use_tc = true;
+      break;
+    default: use_tc = false; break;
+  }
+  if (use_tc && (!aligned16(x) || !aligned16(dy))) {
+    if (d->variant != DYNCONV_VARIANT_AUTO) return DYNCONV_ERR_MISALIGNED;
+    use_tc = false;
+  }
+  const WeightLayout L = weight_layout(d);
+  const long long ws = wsize_of(d);
+  if (d->B == 0) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(dexperts, 0, 4ull * d->n * ws, s);
+    if (e == cudaSuccess && dbias) e = cudaMemsetAsync(dbias, 0, 4ull * d->n * d->C_out, s);
+    return e == cudaSuccess ? DYNCONV_OK : dc_lib::cuda_error(e, "cudaMemsetAsync");
+  }
+  if (!workspace || workspace_bytes < L.total) return DYNCONV_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DYNCONV_ERR_MISALIGNED;
+  dc_lib::DeviceInfo di;
+  rc = dc_lib::device_info(&di);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* wsb = static_cast<char*>(workspace);
+  float* dW = reinterpret_cast<float*>(wsb + L.dW);
+  float* db = reinterpret_cast<float*>(wsb + L.db);
+  float* part = reinterpret_cast<float*>(wsb + L.part);
+
+  // 1. per-sample weight gradients
+  rc = use_tc ? run_wgrad_tc(d, di, x, dy, dW, s) : run_wgrad_direct(d, x, dy, dW, s);
+  if (rc) return rc;
+  // 2. per-sample bias gradients: channel sums of dy
+  const int Ho = out_size(d->H, d->KH, d->stride, d->pad);
+  const int Wo = out_size(d->W, d->KW, d->stride, d->pad);
+  rc = run_chansum(d, dy, Ho * Wo, d->C_out, db, s);
+  if (rc) return rc;
+  // 3. the experts' gradients and the chunks' shares of dalpha
+  dcb::MgParams mp{};
+  mp.B = d->B; mp.n = d->n; mp.wsize = ws; mp.chunks = L.chunks;
+  mp.vec = (ws % 4 == 0 && aligned16(dexperts)) ? 1 : 0;
+  mp.dW = dW; mp.experts = experts; mp.alpha = alpha; mp.dexperts = dexperts; mp.part = part;
+  const int ne = d->n >= 8 ? 8 : d->n > 2 ? 4 : d->n;
+  const size_t mg_smem = sizeof(float) * (static_cast<size_t>(d->B) * ne +
+                                          (dcb::kBwThreads / 32) * dcb::kMgSampleBlock * ne);
+  if (mg_smem > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
+  rc = d->dtype == DYNCONV_F32 ? launch_mixgrad<float>(mp, ne, mg_smem, s)
+                               : launch_mixgrad<__nv_bfloat16>(mp, ne, mg_smem, s);
+  if (rc) return rc;
+  // 4. dalpha = sum of the chunks' shares + <db_b, bias_i>
+  dcb::dalpha_finish_kernel<<<d->B, dcb::kBwThreads, 0, s>>>(d->B, d->n, d->C_out, L.chunks, part,
+                                                             db, bias, dalpha);
+  rc = dc_lib::launched("dalpha_finish_kernel");
+  if (rc) return rc;
+  // 5. dbias
+  if (dbias) {
+    const int total = d->n * d->C_out;
+    dcb::dbias_kernel<<<(total + dcb::kBwThreads - 1) / dcb::kBwThreads, dcb::kBwThreads, 0, s>>>(
+        d->B, d->n, d->C_out, alpha, db, dbias);
+    rc = dc_lib::launched("dbias_kernel");
+  }
+  return rc;
+}
+
+int dynconv_route_backward(const dynconv_desc* desc, const void* x, const float* Wr,
+                           const float* alpha, const float* dalpha, int mode, float tau,
+                           float* dWr, float* dbr, float* dg, void* stream) {
+  int rc = dc_lib::validate(desc);
+  if (rc) return rc;
+  if (!x || !Wr || !alpha || !dalpha || !dWr || !dg) return DYNCONV_ERR_INVALID_ARG;
+  if (mode != DYNCONV_SIGMOID && mode != DYNCONV_SOFTMAX) return DYNCONV_ERR_INVALID_ARG;
+  if (mode == DYNCONV_SOFTMAX && !(tau > 0.f)) return DYNCONV_ERR_INVALID_ARG;
+  if (desc->n > 1024) return DYNCONV_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int C = desc->C_in, n = desc->n, B = desc->B;
+  if (B == 0) {
+    cudaError_t e = cudaMemsetAsync(dWr, 0, 4ull * n * C, s);
+    if (e == cudaSuccess && dbr) e = cudaMemsetAsync(dbr, 0, 4ull * n, s);
+    return e == cudaSuccess ? DYNCONV_OK : dc_lib::cuda_error(e, "cudaMemsetAsync");
+  }
+  dc_lib::DeviceInfo di;
+  rc = dc_lib::device_info(&di);
+  if (rc) return rc;
+  const size_t smem_param = sizeof(float) * static_cast<size_t>(B);
+  const size_t smem_dg = sizeof(float) * (static_cast<size_t>(n) + dcb::kBwThreads);
+  if (smem_param > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
+  // the channel sums of x go to dg first (scratch), then dg is overwritten
+  rc = run_chansum(desc, x, desc->H * desc->W, C, dg, s);
+  if (rc) return rc;
+  if (smem_param > 48 * 1024) {
+    cudaError_t e = dc_lib::set_smem(reinterpret_cast<const void*>(dcb::route_bwd_param_kernel),
+                                     smem_param);
+    if (e != cudaSuccess) return dc_lib::cuda_error(e, "cudaFuncSetAttribute(route_bwd_param)");
+  }
+  const float inv_hw = 1.f / static_cast<float>(desc->H * desc->W);
+  dcb::route_bwd_param_kernel<<<dim3((C + dcb::kBwThreads - 1) / dcb::kBwThreads, n),
+                                dcb::kBwThreads, smem_param, s>>>(B, C, n, inv_hw, mode, tau,
+                                                                  alpha, dalpha, dg, dWr, dbr);
+  rc = dc_lib::launched("route_bwd_param_kernel");
+  if (rc) return rc;
+  dcb::route_bwd_dg_kernel<<<dim3((C + dcb::kBwThreads - 1) / dcb::kBwThreads, B),
+                             dcb::kBwThreads, smem_dg, s>>>(C, n, mode, tau, alpha, dalpha, Wr,
+                                                            dg);
+  return dc_lib::launched("route_bwd_dg_kernel");
+}
+
+int dynconv_backward_data(const dynconv_desc* desc, const void* dy, const void* experts,
+                          const float* alpha, const float* dg, void* dx, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  int rc = dc_lib::validate(desc);
+  if (rc) return rc;
+  if (!dy || !experts || !alpha || !dx) return DYNCONV_ERR_INVALID_ARG;
+  if (desc->B == 0) return DYNCONV_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const dynconv_desc* d = desc;
+  const float inv_hw = 1.f / static_cast<float>(d->H * d->W);
+  if (transposed_ok(d)) {
+    const size_t et_bytes = align256(static_cast<size_t>(d->n) * wsize_of(d) * elem_bytes(d));
+    if (!workspace || workspace_bytes < et_bytes) return DYNCONV_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DYNCONV_ERR_MISALIGNED;
+    const dynconv_desc t = transposed_desc(d);
+    // refuse what the forward would refuse before anything runs
+    const int v = dynconv_select_variant(&t, workspace_bytes - et_bytes);
+    if (v < 0) return v;
+    dc_lib::DeviceInfo di;
+    rc = dc_lib::device_info(&di);
+    if (rc) return rc;
+    const long long total = 1LL * d->n * wsize_of(d);
+    const unsigned grid = static_cast<unsigned>(
+        std::min<long long>((total + dcb::kBwThreads - 1) / dcb::kBwThreads, 8LL * di.sms));
+    if (d->dtype == DYNCONV_F32)
+      dcb::transpose_experts_kernel<float><<<grid, dcb::kBwThreads, 0, s>>>(
+          d->n, d->C_in, d->C_out, d->KH, d->KW, d->groups, static_cast<const float*>(experts),
+          reinterpret_cast<float*>(workspace));
+    else
+      dcb::transpose_experts_kernel<__nv_bfloat16><<<grid, dcb::kBwThreads, 0, s>>>(
+          d->n, d->C_in, d->C_out, d->KH, d->KW, d->groups,
+          static_cast<const __nv_bfloat16*>(experts), reinterpret_cast<__nv_bfloat16*>(workspace));
+    rc = dc_lib::launched("transpose_experts_kernel");
+    if (rc) return rc;
+    char* rest = static_cast<char*>(workspace) + et_bytes;
+    rc = dynconv_forward(&t, dy, workspace, alpha, nullptr, dx,
+                         workspace_bytes > et_bytes ? rest : nullptr, workspace_bytes - et_bytes,
+                         stream);
+    if (rc || !dg) return rc;
+    const long long n_dx = 1LL * d->B * d->H * d->W * d->C_in;
+    const unsigned g2 = static_cast<unsigned>(
+        std::min<long long>((n_dx + dcb::kBwThreads - 1) / dcb::kBwThreads, 8LL * di.sms));
+    if (d->dtype == DYNCONV_F32)
+      dcb::gap_add_kernel<float><<<g2, dcb::kBwThreads, 0, s>>>(
+          n_dx, d->H * d->W * d->C_in, d->C_in, inv_hw, dg, static_cast<float*>(dx));
+    else
+      dcb::gap_add_kernel<__nv_bfloat16><<<g2, dcb::kBwThreads, 0, s>>>(
+          n_dx, d->H * d->W * d->C_in, d->C_in, inv_hw, dg, static_cast<__nv_bfloat16*>(dx));
+    return dc_lib::launched("gap_add_kernel");
+  }
+  dcb::DgdParams p{};
+  p.B = d->B; p.Cin = d->C_in; p.H = d->H; p.W = d->W; p.Cout = d->C_out;
+  p.KH = d->KH; p.KW = d->KW; p.stride = d->stride; p.pad = d->pad; p.groups = d->groups;
+  p.Ho = out_size(d->H, d->KH, d->stride, d->pad);
+  p.Wo = out_size(d->W, d->KW, d->stride, d->pad);
+  p.n = d->n;
+  p.dy = dy; p.experts = experts; p.alpha = alpha; p.dg = dg; p.inv_hw = inv_hw; p.dx = dx;
+  const long long n_dx = 1LL * d->B * d->H * d->W * d->C_in;
+  const unsigned grid = static_cast<unsigned>((n_dx + dcb::kBwThreads - 1) / dcb::kBwThreads);
+  if (d->dtype == DYNCONV_F32)
+    dcb::dgrad_direct_kernel<float><<<grid, dcb::kBwThreads, 0, s>>>(p);
+  else
+    dcb::dgrad_direct_kernel<__nv_bfloat16><<<grid, dcb::kBwThreads, 0, s>>>(p);
+  return dc_lib::launched("dgrad_direct_kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,413 @@
+// CUDA-core kernels of the layer's backward pass: channel sums, the generic
+// per-sample weight gradient, the mixture's gradients (experts, biases,
+// attentions), the router's gradients, the expert transposition that turns
+// the input gradient into a forward convolution, the generic input gradient,
+// and the pooled vector's share of the input gradient.
+//
+// The gradients are those of the forward definition (chain rule): the
+// per-example kernel is a weighted sum of n learned static kernels
+// (KernelWarehouse, abstract; CondConv, abstract), with the attentions from a
+// softmax with temperature or a sigmoid of a linear layer on the average pool
+// (FMDConv, abstract, for the temperature). Every sum over samples runs in
+// sample order inside one thread, and every other reduction in a fixed tree:
+// results do not depend on scheduling.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace dcb {
+
+using dc::from_f32;
+using dc::to_f32;
+
+constexpr int kBwThreads = 256;
+
+// ------------------------------------------------------------ channel sums
+
+// out[b][c] = sum over p < P of v[b][p][c] (v is [B][P][C]). Block (32, 8):
+// threadIdx.x picks the channel, threadIdx.y strides over pixels; the eight
+// partial sums are added in a fixed order.
+template <typename T>
+__global__ void __launch_bounds__(256) chansum_kernel(const T* __restrict__ v, int P, int C,
+                                                      float* __restrict__ out) {
+  __shared__ float part[8][33];
+  const int c = blockIdx.x * 32 + threadIdx.x;
+  const int b = blockIdx.y;
+  float s = 0.f;
+  if (c < C) {
+    const T* vb = v + static_cast<size_t>(b) * P * C + c;
+    for (int p = threadIdx.y; p < P; p += 8) s += to_f32(vb[static_cast<size_t>(p) * C]);
+  }
+  part[threadIdx.y][threadIdx.x] = s;
+  __syncthreads();
+  if (threadIdx.y == 0 && c < C) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += part[k][threadIdx.x];
+    out[static_cast<size_t>(b) * C + c] = t;
+  }
+}
+
+// ------------------------------------------- per-sample weight gradient
+
+struct WgdParams {
+  int B, Cin, H, W, Cout, KH, KW, stride, pad, groups, Ho, Wo;
+  long long wsize;  // Cout * KH * KW * Cin/groups
+  const void* x;
+  const void* dy;
+  float* dW;        // [B][wsize]
+};
+
+// dW[b][co][kh][kw][ci] = sum over output pixels (oh, ow) of
+// dy[b][oh][ow][co] * x[b][oh*s+kh-p][ow*s+kw-p][g(co)*Cg+ci] (zero outside the
+// image). One thread per weight element of one sample; neighbouring threads
+// take neighbouring input channels, so the x loads of a warp are contiguous
+// and its dy loads are one broadcast.
+template <typename T>
+__global__ void __launch_bounds__(kBwThreads) wgrad_direct_kernel(WgdParams p) {
+  const long long o = static_cast<long long>(blockIdx.x) * kBwThreads + threadIdx.x;
+  const int b = blockIdx.y;
+  if (o >= p.wsize) return;
+  const int Cg = p.Cin / p.groups, Coutg = p.Cout / p.groups;
+  const int cil = static_cast<int>(o % Cg);
+  long long t = o / Cg;
+  const int kw = static_cast<int>(t % p.KW);
+  t /= p.KW;
+  const int kh = static_cast<int>(t % p.KH);
+  const int co = static_cast<int>(t / p.KH);
+  const int ci = (co / Coutg) * Cg + cil;
+  const T* xb = static_cast<const T*>(p.x) + static_cast<size_t>(b) * p.H * p.W * p.Cin + ci;
+  const T* dyb = static_cast<const T*>(p.dy) + static_cast<size_t>(b) * p.Ho * p.Wo * p.Cout + co;
+  float acc = 0.f;
+  for (int oh = 0; oh < p.Ho; ++oh) {
+    const int ih = oh * p.stride + kh - p.pad;
+    if (ih < 0 || ih >= p.H) continue;
+    for (int ow = 0; ow < p.Wo; ++ow) {
+      const int iw = ow * p.stride + kw - p.pad;
+      if (iw < 0 || iw >= p.W) continue;
+      acc = fmaf(to_f32(dyb[(static_cast<size_t>(oh) * p.Wo + ow) * p.Cout]),
+                 to_f32(xb[(static_cast<size_t>(ih) * p.W + iw) * p.Cin]), acc);
+    }
+  }
+  p.dW[static_cast<size_t>(b) * p.wsize + o] = acc;
+}
+
+// ------------------------------------------------ the mixture's gradients
+
+constexpr int kMgMaxExperts = 8;     // experts per CTA at most (grid.y walks the rest)
+constexpr int kMgChunk = 4 * kBwThreads;  // weights per CTA: four per thread
+constexpr int kMgSampleBlock = 32;   // samples per partial-sum round
+
+struct MgParams {
+  int B, n;
+  long long wsize;
+  int chunks;            // ceil(wsize / kMgChunk)
+  int vec;               // wsize % 4 == 0 and 16-byte aligned dW, dexperts
+  const float* dW;       // [B][wsize] per-sample weight gradients
+  const void* experts;   // [n][wsize], T
+  const float* alpha;    // [B][n]
+  float* dexperts;       // [n][wsize]
+  float* part;           // [chunks][B][n]: sum over this chunk of dW[b][w] * E[i][w]
+};
+
+// dexperts[i][w] = sum_b alpha[b][i] dW[b][w] for the CTA's 1024 weights and
+// NE experts (fewer in the last group), and the chunk's share of
+// dalpha[b][i] = <dW_b, E_i>. Each thread holds four weights: per sample one
+// 16-byte load of dW, eight multiply-adds per expert and a warp reduction per
+// expert of the dot product; the warps' sums meet in shared memory and are
+// added in warp order.
+template <typename T, int NE>
+__global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
+  extern __shared__ float mg_smem[];
+  float* alpha_s = mg_smem;                                          // [B][NE]
+  float* red = mg_smem + static_cast<size_t>(p.B) * NE;              // [8][32][NE]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x;
+  const int i0 = blockIdx.y * NE;
+  const int ne = min(NE, p.n - i0);
+  for (int e = threadIdx.x; e < p.B * NE; e += kBwThreads) {
+    const int b = e / NE, i = e - b * NE;
+    alpha_s[e] = i < ne ? p.alpha[static_cast<size_t>(b) * p.n + i0 + i] : 0.f;
+  }
+  const long long w = static_cast<long long>(chunk) * kMgChunk + threadIdx.x * 4;
+  const T* E = static_cast<const T*>(p.experts);
+  float ev[NE][4];
+#pragma unroll
+  for (int i = 0; i < NE; ++i)
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      ev[i][k] = (i < ne && w + k < p.wsize)
+                     ? to_f32(E[static_cast<size_t>(i0 + i) * p.wsize + w + k])
+                     : 0.f;
+  float dex[NE][4];
+#pragma unroll
+  for (int i = 0; i < NE; ++i)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dex[i][k] = 0.f;
+  __syncthreads();
+
+  for (int b0 = 0; b0 < p.B; b0 += kMgSampleBlock) {
+    const int nbb = min(kMgSampleBlock, p.B - b0);
+    for (int bb = 0; bb < nbb; ++bb) {
+      const int b = b0 + bb;
+      float v[4];
+      const float* src = p.dW + static_cast<size_t>(b) * p.wsize + w;
+      if (p.vec && w < p.wsize) {
+        const float4 q = *reinterpret_cast<const float4*>(src);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[k] = w + k < p.wsize ? src[k] : 0.f;
+      }
+      const float* ab = alpha_s + static_cast<size_t>(b) * NE;
+#pragma unroll
+      for (int i = 0; i < NE; ++i) {
+        const float a = ab[i];
+        float d = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          dex[i][k] = fmaf(a, v[k], dex[i][k]);
+          d = fmaf(v[k], ev[i][k], d);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        if (lane == 0) red[(warp * kMgSampleBlock + bb) * NE + i] = d;
+      }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < nbb * ne; e += kBwThreads) {
+      const int bb = e / ne, i = e - bb * ne;
+      float s = 0.f;
+      for (int wp = 0; wp < kBwThreads / 32; ++wp) s += red[(wp * kMgSampleBlock + bb) * NE + i];
+      p.part[(static_cast<size_t>(chunk) * p.B + b0 + bb) * p.n + i0 + i] = s;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    if (i < ne) {
+      float* dst = p.dexperts + static_cast<size_t>(i0 + i) * p.wsize + w;
+      if (p.vec && w < p.wsize) {
+        *reinterpret_cast<float4*>(dst) = make_float4(dex[i][0], dex[i][1], dex[i][2], dex[i][3]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (w + k < p.wsize) dst[k] = dex[i][k];
+      }
+    }
+  }
+}
+
+// dalpha[b][i] = sum over chunks (in order) of part[chunk][b][i]
+//              + sum_co db[b][co] * bias[i][co]    (bias may be NULL).
+// One CTA per sample, one thread per expert.
+__global__ void __launch_bounds__(kBwThreads)
+    dalpha_finish_kernel(int B, int n, int Cout, int chunks, const float* __restrict__ part,
+                         const float* __restrict__ db, const float* __restrict__ bias,
+                         float* __restrict__ dalpha) {
+  const int b = blockIdx.x;
+  for (int i = threadIdx.x; i < n; i += kBwThreads) {
+    float s = 0.f;
+    for (int c = 0; c < chunks; ++c) s += part[(static_cast<size_t>(c) * B + b) * n + i];
+    if (bias) {
+      float t = 0.f;
+      for (int co = 0; co < Cout; ++co)
+        t = fmaf(db[static_cast<size_t>(b) * Cout + co], bias[static_cast<size_t>(i) * Cout + co], t);
+      s += t;
+    }
+    dalpha[static_cast<size_t>(b) * n + i] = s;
+  }
+}
+
+// dbias[i][co] = sum_b alpha[b][i] * db[b][co], one thread per element.
+__global__ void __launch_bounds__(kBwThreads)
+    dbias_kernel(int B, int n, int Cout, const float* __restrict__ alpha,
+                 const float* __restrict__ db, float* __restrict__ dbias) {
+  const int e = blockIdx.x * kBwThreads + threadIdx.x;
+  if (e >= n * Cout) return;
+  const int i = e / Cout, co = e - i * Cout;
+  float s = 0.f;
+  for (int b = 0; b < B; ++b)
+    s = fmaf(alpha[static_cast<size_t>(b) * n + i], db[static_cast<size_t>(b) * Cout + co], s);
+  dbias[e] = s;
+}
+
+// ------------------------------------------------------ router gradients
+
+// dz[b][i] from the attention's gradient through the activation:
+// sigmoid: dalpha * alpha * (1 - alpha); softmax of z/tau:
+// alpha_i * (dalpha_i - sum_j alpha_j dalpha_j) / tau, the sum over j in order.
+__device__ __forceinline__ float dz_of(const float* a, const float* da, int n, int i, int mode,
+                                       float tau) {
+  if (mode == 0) return da[i] * a[i] * (1.f - a[i]);
+  float dot = 0.f;
+  for (int j = 0; j < n; ++j) dot = fmaf(a[j], da[j], dot);
+  return a[i] * (da[i] - dot) / tau;
+}
+
+// Router parameters: dWr[i][c] = sum_b dz[b][i] * gsum[b][c] / HW and
+// dbr[i] = sum_b dz[b][i]. Grid (ceil(C / 256), n): the CTA first takes
+// dz[b][i] for every sample into shared memory (one thread per sample).
+__global__ void __launch_bounds__(kBwThreads)
+    route_bwd_param_kernel(int B, int C, int n, float inv_hw, int mode, float tau,
+                           const float* __restrict__ alpha, const float* __restrict__ dalpha,
+                           const float* __restrict__ gsum, float* __restrict__ dWr,
+                           float* __restrict__ dbr) {
+  extern __shared__ float dz_s[];  // [B]
+  const int i = blockIdx.y;
+  for (int b = threadIdx.x; b < B; b += kBwThreads)
+    dz_s[b] = dz_of(alpha + static_cast<size_t>(b) * n, dalpha + static_cast<size_t>(b) * n, n,
+                    i, mode, tau);
+  __syncthreads();
+  const int c = blockIdx.x * kBwThreads + threadIdx.x;
+  if (c < C) {
+    float s = 0.f;
+    for (int b = 0; b < B; ++b) s = fmaf(dz_s[b], gsum[static_cast<size_t>(b) * C + c], s);
+    dWr[static_cast<size_t>(i) * C + c] = s * inv_hw;
+  }
+  if (dbr && blockIdx.x == 0 && threadIdx.x == 0) {
+    float s = 0.f;
+    for (int b = 0; b < B; ++b) s += dz_s[b];
+    dbr[i] = s;
+  }
+}
+
+// The pooled vector's gradient: dg[b][c] = sum_i dz[b][i] * Wr[i][c]. Grid
+// (ceil(C / 256), B); dz of the sample goes to shared memory first (the
+// softmax's sum over j by a fixed tree).
+__global__ void __launch_bounds__(kBwThreads)
+    route_bwd_dg_kernel(int C, int n, int mode, float tau, const float* __restrict__ alpha,
+                        const float* __restrict__ dalpha, const float* __restrict__ Wr,
+                        float* __restrict__ dg) {
+  extern __shared__ float rd_s[];  // dz [n] then the tree [256]
+  float* dz = rd_s;
+  float* tree = rd_s + n;
+  const int b = blockIdx.y;
+  const float* a = alpha + static_cast<size_t>(b) * n;
+  const float* da = dalpha + static_cast<size_t>(b) * n;
+  float dot = 0.f;
+  if (mode == 1) {
+    float s = 0.f;
+    for (int j = threadIdx.x; j < n; j += kBwThreads) s = fmaf(a[j], da[j], s);
+    tree[threadIdx.x] = s;
+    __syncthreads();
+    for (int off = kBwThreads / 2; off > 0; off >>= 1) {
+      if (threadIdx.x < off) tree[threadIdx.x] += tree[threadIdx.x + off];
+      __syncthreads();
+    }
+    dot = tree[0];
+  }
+  for (int i = threadIdx.x; i < n; i += kBwThreads)
+    dz[i] = mode == 0 ? da[i] * a[i] * (1.f - a[i]) : a[i] * (da[i] - dot) / tau;
+  __syncthreads();
+  const int c = blockIdx.x * kBwThreads + threadIdx.x;
+  if (c < C) {
+    float s = 0.f;
+    for (int i = 0; i < n; ++i) s = fmaf(dz[i], Wr[static_cast<size_t>(i) * C + c], s);
+    dg[static_cast<size_t>(b) * C + c] = s;
+  }
+}
+
+// ------------------------------------------------------- input gradient
+
+// Et[i][ci][kh][kw][col] = E[i][g*Coutg + col][KH-1-kh][KW-1-kw][ci - g*Cg],
+// g = ci / Cg: every expert with input and output channels swapped within
+// its group and flipped in both spatial axes, so that the input gradient of
+// the convolution is a forward convolution of dy with the same attentions.
+// One thread per output element (grid-stride), writes contiguous.
+template <typename T>
+__global__ void __launch_bounds__(kBwThreads)
+    transpose_experts_kernel(int n, int Cin, int Cout, int KH, int KW, int groups,
+                             const T* __restrict__ E, T* __restrict__ Et) {
+  const int Cg = Cin / groups, Coutg = Cout / groups;
+  const long long total = 1LL * n * Cin * KH * KW * Coutg;
+  for (long long o = static_cast<long long>(blockIdx.x) * kBwThreads + threadIdx.x; o < total;
+       o += static_cast<long long>(gridDim.x) * kBwThreads) {
+    long long t = o;
+    const int col = static_cast<int>(t % Coutg);
+    t /= Coutg;
+    const int kw = static_cast<int>(t % KW);
+    t /= KW;
+    const int kh = static_cast<int>(t % KH);
+    t /= KH;
+    const int ci = static_cast<int>(t % Cin);
+    const long long i = t / Cin;
+    const int g = ci / Cg;
+    const int co = g * Coutg + col;
+    const size_t src = ((((static_cast<size_t>(i) * Cout + co) * KH + (KH - 1 - kh)) * KW +
+                         (KW - 1 - kw)) * Cg) + (ci - g * Cg);
+    Et[o] = E[src];
+  }
+}
+
+struct DgdParams {
+  int B, Cin, H, W, Cout, KH, KW, stride, pad, groups, Ho, Wo, n;
+  const void* dy;
+  const void* experts;
+  const float* alpha;
+  const float* dg;   // [B][Cin] or NULL
+  float inv_hw;
+  void* dx;
+};
+
+// Generic input gradient (any stride, padding, groups): one thread per
+// element of dx, summing dy * W_b over the (output pixel, tap) pairs that
+// read it, W_b mixed on the fly from the experts; plus dg/(H*W); rounded once.
+template <typename T>
+__global__ void __launch_bounds__(kBwThreads) dgrad_direct_kernel(DgdParams p) {
+  const long long total = 1LL * p.B * p.H * p.W * p.Cin;
+  const long long o = static_cast<long long>(blockIdx.x) * kBwThreads + threadIdx.x;
+  if (o >= total) return;
+  const int ci = static_cast<int>(o % p.Cin);
+  long long t = o / p.Cin;
+  const int iw = static_cast<int>(t % p.W);
+  t /= p.W;
+  const int ih = static_cast<int>(t % p.H);
+  const int b = static_cast<int>(t / p.H);
+  const int Cg = p.Cin / p.groups, Coutg = p.Cout / p.groups;
+  const int g = ci / Cg, cil = ci - g * Cg;
+  const T* E = static_cast<const T*>(p.experts);
+  const T* dyb = static_cast<const T*>(p.dy) + static_cast<size_t>(b) * p.Ho * p.Wo * p.Cout;
+  const float* ab = p.alpha + static_cast<size_t>(b) * p.n;
+  const size_t wsize = static_cast<size_t>(p.Cout) * p.KH * p.KW * Cg;
+  float acc = 0.f;
+  for (int kh = 0; kh < p.KH; ++kh) {
+    const int th = ih + p.pad - kh;
+    if (th < 0 || th % p.stride) continue;
+    const int oh = th / p.stride;
+    if (oh >= p.Ho) continue;
+    for (int kw = 0; kw < p.KW; ++kw) {
+      const int tw = iw + p.pad - kw;
+      if (tw < 0 || tw % p.stride) continue;
+      const int ow = tw / p.stride;
+      if (ow >= p.Wo) continue;
+      for (int col = 0; col < Coutg; ++col) {
+        const int co = g * Coutg + col;
+        const size_t widx = ((static_cast<size_t>(co) * p.KH + kh) * p.KW + kw) * Cg + cil;
+        float wv = 0.f;
+        for (int i = 0; i < p.n; ++i) wv = fmaf(ab[i], to_f32(E[i * wsize + widx]), wv);
+        acc = fmaf(to_f32(dyb[(static_cast<size_t>(oh) * p.Wo + ow) * p.Cout + co]), wv, acc);
+      }
+    }
+  }
+  if (p.dg) acc += p.dg[static_cast<size_t>(b) * p.Cin + ci] * p.inv_hw;
+  static_cast<T*>(p.dx)[o] = from_f32<T>(acc);
+}
+
+// dx[b][p][c] += dg[b][c] * inv_hw in place (dx in T, one rounding).
+template <typename T>
+__global__ void __launch_bounds__(kBwThreads)
+    gap_add_kernel(long long total, int HWC, int C, float inv_hw, const float* __restrict__ dg,
+                   T* __restrict__ dx) {
+  for (long long o = static_cast<long long>(blockIdx.x) * kBwThreads + threadIdx.x; o < total;
+       o += static_cast<long long>(gridDim.x) * kBwThreads) {
+    const long long b = o / HWC;
+    const int c = static_cast<int>(o % C);
+    dx[o] = from_f32<T>(to_f32(dx[o]) + dg[b * C + c] * inv_hw);
+  }
+}
+
+}  // namespace dcb

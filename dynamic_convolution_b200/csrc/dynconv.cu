@@ -13,6 +13,7 @@
 #include <utility>
 
 #include "dynconv.h"
+#include "internal.h"
 
 #include "common.cuh"
 #include "conv_tc.cuh"
@@ -1081,3 +1082,46 @@ int dynconv_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ============================================== helpers for the other units
+
+namespace dc_lib {
+
+int device_info(DeviceInfo* out) {
+  DeviceState* st = nullptr;
+  const int rc = device_state(&st);
+  if (rc) return rc;
+  out->err = st->err;
+  out->sms = st->sms;
+  out->max_smem_optin = st->max_smem_optin;
+  out->wait_ns = g_wait_ns.load();
+  out->encode_tiled = reinterpret_cast<void*>(g_encode);
+  return DYNCONV_OK;
+}
+
+int fail(int status, const char* msg) {
+  std::snprintf(g_last_err, sizeof(g_last_err), "%s", msg);
+  return status;
+}
+
+int cuda_error(cudaError_t e, const char* what) { return cuda_fail(e, what); }
+
+int launched(const char* what) { return check_launch(what); }
+
+int validate(const dynconv_desc* desc) { return validate_desc(desc); }
+
+cudaError_t set_smem(const void* kernel, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const auto key = std::make_pair(dev, kernel);
+  std::lock_guard<std::mutex> lk(g_smem_mu);
+  auto it = g_smem_set.find(key);
+  if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes));
+  if (e == cudaSuccess) g_smem_set[key] = bytes;
+  return e;
+}
+
+}  // namespace dc_lib

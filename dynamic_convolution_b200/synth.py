@@ -161,3 +161,10 @@ def make_inputs(cfg: LayerConfig, seed: int = 0, structured: float = 0.0) -> Lay
     es, ef = _round(experts, cfg.dtype)
     return LayerInputs(cfg, xs, xf, es, ef, Wr.astype(np.float32), br.astype(np.float32),
                        bias.astype(np.float32))
+
+
+def make_upstream_grad(cfg: LayerConfig, seed: int = 1):
+    """A seeded upstream gradient dy[B][H_out][W_out][C_out] ~ N(0, 1), rounded to
+    the layer dtype: (device storage, the same values as float64)."""
+    rng = np.random.default_rng(seed)
+    return _round(rng.standard_normal((cfg.B, cfg.H_out, cfg.W_out, cfg.C_out)), cfg.dtype)

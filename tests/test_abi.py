@@ -13,7 +13,8 @@ import dynamic_convolution_b200 as dc
 from dynamic_convolution_b200 import build as dcbuild
 from dynamic_convolution_b200 import synth
 
-HEADER = os.path.join(dcbuild.ROOT, "include", "dynconv.h")
+HEADERS = [os.path.join(dcbuild.ROOT, "include", h)
+           for h in ("dynconv.h", "dynconv_backward.h")]
 
 
 @pytest.fixture(scope="module")
@@ -23,7 +24,7 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(dynconv_[a-z_]+)\s*\(", text)))
 
@@ -149,3 +150,40 @@ def test_attention_entry_points_host_side(lib):
     for kw in BAD:
         assert dc.dynconv_forward_attn(_desc(**kw), 16, 16, 16, None, None, None, 16) == \
             dc.ERR_INVALID_ARG
+
+
+def test_backward_entry_points_host_side(lib):
+    """Argument checks of the backward calls, the workspace size (per-sample
+    fp32 weight gradients, or transposed experts plus the transposed forward's
+    own scratch, whichever is larger), and the loud failure with no device."""
+    cfg = synth.CONFIGS["resnet18_3x3"]
+    d = dc.desc_from_config(cfg)
+    wsize = cfg.C_out * cfg.KH * cfg.KW * cfg.C_in
+    need = dc.dynconv_backward_workspace_size(d)
+    assert need >= 4 * cfg.B * wsize + 4 * cfg.B * cfg.C_out
+    t = dc.make_desc(cfg.B, cfg.C_out, cfg.H, cfg.W, cfg.C_in, 3, 3, 1, 1, 1, cfg.n, cfg.dtype)
+    assert need >= 2 * cfg.n * wsize + dc.dynconv_workspace_size(t)
+    assert dc.dynconv_backward_workspace_size(dc.make_desc(0, 0, 1, 1, 1, 1, 1)) == 0
+    P, ws = 256, need
+    bw = dc.dynconv_backward_weight
+    assert bw(d, None, P, P, P, P, P, P, P, P, ws) == dc.ERR_INVALID_ARG      # no x
+    assert bw(d, P, P, P, P, P, P, None, P, P, ws) == dc.ERR_INVALID_ARG      # bias without dbias
+    assert bw(d, P, P, P, P, None, P, P, P, P, ws) == dc.ERR_INVALID_ARG      # dbias without bias
+    assert bw(d, P, P, P, P, P, P, P, P, P, ws - 256) == dc.ERR_WORKSPACE
+    assert bw(d, P, P, P, P, P, P, P, P, P + 16, ws) == dc.ERR_MISALIGNED     # workspace alignment
+    s2 = dc.make_desc(cfg.B, cfg.C_in, cfg.H, cfg.W, cfg.C_out, 3, 3, 2, 1, 1, cfg.n, cfg.dtype,
+                      dc.VARIANT_PREMIX)
+    assert bw(s2, P, P, P, P, P, P, P, P, P, ws) == dc.ERR_UNSUPPORTED       # forced TC, stride 2
+    assert bw(d, P, P, P, P, P, P, P, P, P, ws) == dc.ERR_CUDA               # no device: loud
+    rb = dc.dynconv_route_backward
+    assert rb(d, P, P, P, P, 2, 1.0, P, P, P) == dc.ERR_INVALID_ARG          # bad mode
+    assert rb(d, P, P, P, P, dc.SOFTMAX, 0.0, P, P, P) == dc.ERR_INVALID_ARG
+    assert rb(d, P, None, P, P, dc.SOFTMAX, 1.0, P, P, P) == dc.ERR_INVALID_ARG
+    assert rb(d, P, P, P, P, dc.SOFTMAX, 1.0, P, None, P) == dc.ERR_CUDA     # dbr optional
+    bd = dc.dynconv_backward_data
+    assert bd(d, None, P, P, None, P, P, ws) == dc.ERR_INVALID_ARG
+    assert bd(d, P, P, P, None, P, P, 1024) == dc.ERR_WORKSPACE              # no room for experts
+    assert bd(d, P, P, P, None, P, P, ws) == dc.ERR_CUDA
+    # shapes off the transposed path take the CUDA-core kernel and need no workspace
+    assert bd(s2, P, P, P, None, P, None, 0) == dc.ERR_CUDA
+    assert dc.dynconv_last_error() != ""
