@@ -737,8 +737,11 @@ def run_backward(args, cfg):
             "data": "synthetic (seeded; recipe in DESIGN.md)",
             "config": {"workload": f"{cfg.name} backward", "l2": f"inputs rotated over {nsets} sets"},
             "effective_tflops": tflops, "us_per_call": parts, "gpu_launches_per_step": launches,
-            "wgrad_kernel": "tcgen05" if dc.VARIANT_AUTO == d.variant and cfg.dtype == synth.BF16
-            and cfg.groups == 1 and cfg.C_in % 8 == 0 and cfg.C_in >= 64 else "cuda-core"}
+            "wgrad_kernel": ("tcgen05" if cfg.dtype == synth.BF16 and cfg.groups == 1
+                             and cfg.stride == 1 and cfg.C_in % 8 == 0 and cfg.C_out % 8 == 0
+                             else "cuda-core depthwise" if cfg.dtype == synth.BF16
+                             and cfg.groups == cfg.C_in == cfg.C_out and cfg.C_in % 8 == 0
+                             else "cuda-core")}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -83,7 +83,7 @@ size_t data_workspace(const dynconv_desc* d) {
 bool wgrad_tc_shape_ok(const dynconv_desc* d) {
   const int Wo = out_size(d->W, d->KW, 1, d->pad);
   return d->dtype == DYNCONV_BF16 && d->groups == 1 && d->stride == 1 && d->C_in % 8 == 0 &&
-         d->C_out % 8 == 0 && d->C_in >= 64 && d->C_out >= 64 && Wo <= 128;
+         d->C_out % 8 == 0 && Wo <= 128;
 }
 
 int encode_4d(EncodeTiledFn enc, CUtensorMap* map, const void* base, int C, int W, int H, int B,
@@ -99,7 +99,8 @@ int encode_4d(EncodeTiledFn enc, CUtensorMap* map, const void* base, int C, int 
   if (enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
           es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return dc_lib::fail(DYNCONV_ERR_CUDA, "cuTensorMapEncodeTiled (weight gradient) failed");
+    return dc_lib::fail(DYNCONV_ERR_UNSUPPORTED,
+                        "cuTensorMapEncodeTiled (weight gradient) refused the shape");
   return DYNCONV_OK;
 }
 
@@ -127,7 +128,7 @@ int run_wgrad_tc(const dynconv_desc* d, const dc_lib::DeviceInfo& di, const void
   p.co_tiles = (d->C_out + 127) / 128;
   p.units = 1LL * d->B * p.co_tiles * p.agroups;
   const int stage_bytes = (2 + dcb::kWgMaxAtoms) * p.atom_bytes;
-  p.stages = std::min(4, (200 * 1024) / stage_bytes);
+  p.stages = std::min(4, (210 * 1024 - 4 * dcb::kWgStageBytes) / stage_bytes);
   if (p.stages < 2) return dc_lib::fail(DYNCONV_ERR_UNSUPPORTED, "weight-gradient tile too large");
   p.dW = dW;
   p.err = di.err;
@@ -140,7 +141,8 @@ int run_wgrad_tc(const dynconv_desc* d, const dc_lib::DeviceInfo& di, const void
   if (rc) return rc;
   // at least 120 KB, so that two CTAs never share an SM (each holds all 512 TMEM columns)
   const size_t smem = std::max<size_t>(
-      120 * 1024, 1024 + static_cast<size_t>(p.stages) * stage_bytes + 8 * (2 * p.stages + 5) + 16);
+      120 * 1024, 1024 + static_cast<size_t>(p.stages) * stage_bytes + 4 * dcb::kWgStageBytes +
+                      8 * (2 * p.stages + 5) + 16);
   if (smem > static_cast<size_t>(di.max_smem_optin))
     return dc_lib::fail(DYNCONV_ERR_UNSUPPORTED, "weight-gradient shared memory");
   cudaError_t e = dc_lib::set_smem(reinterpret_cast<const void*>(dcb::wgrad_tc_kernel), smem);
@@ -167,13 +169,70 @@ int run_wgrad_direct(const dynconv_desc* d, const void* x, const void* dy, float
   return dc_lib::launched("wgrad_direct_kernel");
 }
 
+bool wgrad_dw_ok(const dynconv_desc* d) {
+  return d->dtype == DYNCONV_BF16 && d->groups == d->C_in && d->C_in == d->C_out &&
+         d->stride == 1 && d->KH == d->KW && (d->KH == 3 || d->KH == 5 || d->KH == 7) &&
+         d->C_in % 8 == 0;
+}
+
+// Bands of output rows small enough for ~3 CTAs per SM (at most 80 KB), or
+// 0 when even one row does not fit.
+int wgrad_dw_band(const dynconv_desc* d, int max_smem, size_t* smem_out) {
+  const int K = d->KH;
+  const int Ho = out_size(d->H, K, 1, d->pad), Wo = out_size(d->W, K, 1, d->pad);
+  const int Wp = Wo + K - 1;
+  auto bytes = [&](int band) {
+    return static_cast<size_t>((band + K - 1) * Wp + band * Wo) * dcb::kDwgChunk * 2;
+  };
+  int band = Ho;
+  while (band > 1 && bytes(band) > 80 * 1024) band = (band + 1) / 2;
+  if (bytes(band) > static_cast<size_t>(max_smem)) return 0;
+  *smem_out = bytes(band);
+  return band;
+}
+
+int run_wgrad_dw(const dynconv_desc* d, int band, size_t smem, const void* x, const void* dy,
+                 float* dW, cudaStream_t s) {
+  dcb::DwgParams p{};
+  p.B = d->B; p.C = d->C_in; p.H = d->H; p.W = d->W; p.pad = d->pad; p.band = band;
+  p.Ho = out_size(d->H, d->KH, 1, d->pad);
+  p.Wo = out_size(d->W, d->KW, 1, d->pad);
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.dy = static_cast<const __nv_bfloat16*>(dy);
+  p.dW = dW;
+  const dim3 grid((d->C_in + dcb::kDwgChunk - 1) / dcb::kDwgChunk, d->B);
+  auto go = [&](auto kern, int K) -> int {
+    if (smem > 48 * 1024) {
+      cudaError_t e = dc_lib::set_smem(reinterpret_cast<const void*>(kern), smem);
+      if (e != cudaSuccess) return dc_lib::cuda_error(e, "cudaFuncSetAttribute(wgrad_dw)");
+    }
+    kern<<<grid, dim3(32, K), smem, s>>>(p);
+    return dc_lib::launched("wgrad_dw_kernel");
+  };
+  return d->KH == 3 ? go(dcb::wgrad_dw_kernel<3>, 3)
+         : d->KH == 5 ? go(dcb::wgrad_dw_kernel<5>, 5) : go(dcb::wgrad_dw_kernel<7>, 7);
+}
+
 int run_chansum(const dynconv_desc* d, const void* v, int P, int C, float* out, cudaStream_t s) {
-  const dim3 grid((C + 31) / 32, d->B), block(32, 8);
-  if (d->dtype == DYNCONV_F32)
-    dcb::chansum_kernel<float><<<grid, block, 0, s>>>(static_cast<const float*>(v), P, C, out);
-  else
-    dcb::chansum_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(v), P, C, out);
+  const bool bf = d->dtype == DYNCONV_BF16;
+  const int vec = bf ? 8 : 4;
+  const bool vok = C % vec == 0 && aligned16(v);
+  const size_t smem = sizeof(float) * dcb::kBwThreads * (vok ? vec : 1);
+  if (bf) {
+    if (vok)
+      dcb::chansum_kernel<__nv_bfloat16, 8><<<d->B, dcb::kBwThreads, smem, s>>>(
+          static_cast<const __nv_bfloat16*>(v), P, C, out);
+    else
+      dcb::chansum_kernel<__nv_bfloat16, 1><<<d->B, dcb::kBwThreads, smem, s>>>(
+          static_cast<const __nv_bfloat16*>(v), P, C, out);
+  } else {
+    if (vok)
+      dcb::chansum_kernel<float, 4><<<d->B, dcb::kBwThreads, smem, s>>>(
+          static_cast<const float*>(v), P, C, out);
+    else
+      dcb::chansum_kernel<float, 1><<<d->B, dcb::kBwThreads, smem, s>>>(
+          static_cast<const float*>(v), P, C, out);
+  }
   return dc_lib::launched("chansum_kernel");
 }
 
@@ -192,7 +251,8 @@ int launch_mixgrad(const dcb::MgParams& p, int ne, size_t smem, cudaStream_t s) 
     case 1: return go(dcb::mixgrad_kernel<T, 1>);
     case 2: return go(dcb::mixgrad_kernel<T, 2>);
     case 4: return go(dcb::mixgrad_kernel<T, 4>);
-    default: return go(dcb::mixgrad_kernel<T, 8>);
+    case 8: return go(dcb::mixgrad_kernel<T, 8>);
+    default: return go(dcb::mixgrad_kernel<T, 16>);
   }
 }
 
@@ -250,8 +310,22 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
   float* part = reinterpret_cast<float*>(wsb + L.part);
 
   // 1. per-sample weight gradients
-  rc = use_tc ? run_wgrad_tc(d, di, x, dy, dW, s) : run_wgrad_direct(d, x, dy, dW, s);
-  if (rc) return rc;
+  if (use_tc) {
+    rc = run_wgrad_tc(d, di, x, dy, dW, s);
+    if (rc == DYNCONV_ERR_UNSUPPORTED && d->variant == DYNCONV_VARIANT_AUTO) use_tc = false;
+    else if (rc) return rc;
+  }
+  if (!use_tc) {
+    size_t dw_smem = 0;
+    const int band = (wgrad_dw_ok(d) && aligned16(x) && aligned16(dy) &&
+                      d->variant != DYNCONV_VARIANT_DIRECT)
+                         ? wgrad_dw_band(d, di.max_smem_optin, &dw_smem)
+                         : 0;
+    if (d->variant == DYNCONV_VARIANT_DEPTHWISE && band == 0) return DYNCONV_ERR_UNSUPPORTED;
+    rc = band > 0 ? run_wgrad_dw(d, band, dw_smem, x, dy, dW, s)
+                  : run_wgrad_direct(d, x, dy, dW, s);
+    if (rc) return rc;
+  }
   // 2. per-sample bias gradients: channel sums of dy
   const int Ho = out_size(d->H, d->KH, d->stride, d->pad);
   const int Wo = out_size(d->W, d->KW, d->stride, d->pad);
@@ -262,7 +336,8 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
   mp.B = d->B; mp.n = d->n; mp.wsize = ws; mp.chunks = L.chunks;
   mp.vec = (ws % 4 == 0 && aligned16(dexperts)) ? 1 : 0;
   mp.dW = dW; mp.experts = experts; mp.alpha = alpha; mp.dexperts = dexperts; mp.part = part;
-  const int ne = d->n >= 8 ? 8 : d->n > 2 ? 4 : d->n;
+  // experts per CTA: every sample's dW is read ceil(n / ne) times
+  const int ne = d->n >= 16 ? 16 : d->n > 4 ? 8 : d->n > 2 ? 4 : d->n;
   const size_t mg_smem = sizeof(float) * (static_cast<size_t>(d->B) * ne +
                                           (dcb::kBwThreads / 32) * dcb::kMgSampleBlock * ne);
   if (mg_smem > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
@@ -347,17 +422,34 @@ int dynconv_backward_data(const dynconv_desc* desc, const void* dy, const void* 
     dc_lib::DeviceInfo di;
     rc = dc_lib::device_info(&di);
     if (rc) return rc;
-    const long long total = 1LL * d->n * wsize_of(d);
-    const unsigned grid = static_cast<unsigned>(
-        std::min<long long>((total + dcb::kBwThreads - 1) / dcb::kBwThreads, 8LL * di.sms));
-    if (d->dtype == DYNCONV_F32)
-      dcb::transpose_experts_kernel<float><<<grid, dcb::kBwThreads, 0, s>>>(
-          d->n, d->C_in, d->C_out, d->KH, d->KW, d->groups, static_cast<const float*>(experts),
-          reinterpret_cast<float*>(workspace));
-    else
-      dcb::transpose_experts_kernel<__nv_bfloat16><<<grid, dcb::kBwThreads, 0, s>>>(
-          d->n, d->C_in, d->C_out, d->KH, d->KW, d->groups,
-          static_cast<const __nv_bfloat16*>(experts), reinterpret_cast<__nv_bfloat16*>(workspace));
+    const int Cg = d->C_in / d->groups, Coutg = d->C_out / d->groups;
+    const int taps_groups = d->KH * d->KW * d->groups;
+    if (Cg >= 8 && Coutg >= 8 && taps_groups <= 65535 && d->n <= 65535) {
+      // 32 x 32 tiles of each group's [Coutg][Cg] matrix per (tap, group, expert)
+      const dim3 grid(((Cg + 31) / 32) * ((Coutg + 31) / 32), taps_groups, d->n), block(32, 8);
+      if (d->dtype == DYNCONV_F32)
+        dcb::transpose_experts_tiled_kernel<float><<<grid, block, 0, s>>>(
+            d->C_in, d->C_out, d->KH, d->KW, d->groups, static_cast<const float*>(experts),
+            reinterpret_cast<float*>(workspace));
+      else
+        dcb::transpose_experts_tiled_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
+            d->C_in, d->C_out, d->KH, d->KW, d->groups,
+            static_cast<const __nv_bfloat16*>(experts),
+            reinterpret_cast<__nv_bfloat16*>(workspace));
+    } else {
+      const long long total = 1LL * d->n * wsize_of(d);
+      const unsigned grid = static_cast<unsigned>(
+          std::min<long long>((total + dcb::kBwThreads - 1) / dcb::kBwThreads, 8LL * di.sms));
+      if (d->dtype == DYNCONV_F32)
+        dcb::transpose_experts_kernel<float><<<grid, dcb::kBwThreads, 0, s>>>(
+            d->n, d->C_in, d->C_out, d->KH, d->KW, d->groups, static_cast<const float*>(experts),
+            reinterpret_cast<float*>(workspace));
+      else
+        dcb::transpose_experts_kernel<__nv_bfloat16><<<grid, dcb::kBwThreads, 0, s>>>(
+            d->n, d->C_in, d->C_out, d->KH, d->KW, d->groups,
+            static_cast<const __nv_bfloat16*>(experts),
+            reinterpret_cast<__nv_bfloat16*>(workspace));
+    }
     rc = dc_lib::launched("transpose_experts_kernel");
     if (rc) return rc;
     char* rest = static_cast<char*>(workspace) + et_bytes;
@@ -366,14 +458,24 @@ int dynconv_backward_data(const dynconv_desc* desc, const void* dy, const void* 
                          stream);
     if (rc || !dg) return rc;
     const long long n_dx = 1LL * d->B * d->H * d->W * d->C_in;
+    const bool bf = d->dtype == DYNCONV_BF16;
+    const int vec = (d->C_in % (bf ? 8 : 4) == 0 && aligned16(dx)) ? (bf ? 8 : 4) : 1;
+    const long long nvec = n_dx / vec;
     const unsigned g2 = static_cast<unsigned>(
-        std::min<long long>((n_dx + dcb::kBwThreads - 1) / dcb::kBwThreads, 8LL * di.sms));
-    if (d->dtype == DYNCONV_F32)
-      dcb::gap_add_kernel<float><<<g2, dcb::kBwThreads, 0, s>>>(
-          n_dx, d->H * d->W * d->C_in, d->C_in, inv_hw, dg, static_cast<float*>(dx));
+        std::min<long long>((nvec + dcb::kBwThreads - 1) / dcb::kBwThreads, 16LL * di.sms));
+    const int hwc = d->H * d->W * d->C_in;
+    if (!bf && vec == 4)
+      dcb::gap_add_kernel<float, 4><<<g2, dcb::kBwThreads, 0, s>>>(nvec, hwc, d->C_in, inv_hw, dg,
+                                                                   static_cast<float*>(dx));
+    else if (!bf)
+      dcb::gap_add_kernel<float, 1><<<g2, dcb::kBwThreads, 0, s>>>(nvec, hwc, d->C_in, inv_hw, dg,
+                                                                   static_cast<float*>(dx));
+    else if (vec == 8)
+      dcb::gap_add_kernel<__nv_bfloat16, 8><<<g2, dcb::kBwThreads, 0, s>>>(
+          nvec, hwc, d->C_in, inv_hw, dg, static_cast<__nv_bfloat16*>(dx));
     else
-      dcb::gap_add_kernel<__nv_bfloat16><<<g2, dcb::kBwThreads, 0, s>>>(
-          n_dx, d->H * d->W * d->C_in, d->C_in, inv_hw, dg, static_cast<__nv_bfloat16*>(dx));
+      dcb::gap_add_kernel<__nv_bfloat16, 1><<<g2, dcb::kBwThreads, 0, s>>>(
+          nvec, hwc, d->C_in, inv_hw, dg, static_cast<__nv_bfloat16*>(dx));
     return dc_lib::launched("gap_add_kernel");
   }
   dcb::DgdParams p{};

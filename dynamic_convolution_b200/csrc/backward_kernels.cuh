@@ -27,27 +27,60 @@ constexpr int kBwThreads = 256;
 
 // ------------------------------------------------------------ channel sums
 
-// out[b][c] = sum over p < P of v[b][p][c] (v is [B][P][C]). Block (32, 8):
-// threadIdx.x picks the channel, threadIdx.y strides over pixels; the eight
-// partial sums are added in a fixed order.
-template <typename T>
-__global__ void __launch_bounds__(256) chansum_kernel(const T* __restrict__ v, int P, int C,
-                                                      float* __restrict__ out) {
-  __shared__ float part[8][33];
-  const int c = blockIdx.x * 32 + threadIdx.x;
-  const int b = blockIdx.y;
-  float s = 0.f;
-  if (c < C) {
-    const T* vb = v + static_cast<size_t>(b) * P * C + c;
-    for (int p = threadIdx.y; p < P; p += 8) s += to_f32(vb[static_cast<size_t>(p) * C]);
-  }
-  part[threadIdx.y][threadIdx.x] = s;
-  __syncthreads();
-  if (threadIdx.y == 0 && c < C) {
-    float t = 0.f;
+// out[b][c] = sum over p < P of v[b][p][c] (v is [B][P][C]). One CTA per
+// sample: thread t takes the VEC channels of vector t % cv (cv = C / VEC
+// vectors per pixel) and the pixels t / cv, t / cv + L, ... (L = 256 / cv pixel
+// lanes), four 16-byte loads in flight; the L lane sums are then added in
+// lane order. VEC = 1 is the unvectorised form (any C, any alignment).
+template <typename T, int VEC>
+__global__ void __launch_bounds__(kBwThreads) chansum_kernel(const T* __restrict__ v, int P, int C,
+                                                             float* __restrict__ out) {
+  extern __shared__ float cs_part[];  // [L][C]
+  const int b = blockIdx.x;
+  const int cv = C / VEC;
+  const T* vb = v + static_cast<size_t>(b) * P * C;
+  for (int v0 = 0; v0 < cv; v0 += kBwThreads) {
+    const int nvec = min(kBwThreads, cv - v0);
+    const int L = kBwThreads / nvec;
+    const int t = threadIdx.x;
+    const int vi = v0 + t % nvec, lane_p = t / nvec;
+    float acc[VEC];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) t += part[k][threadIdx.x];
-    out[static_cast<size_t>(b) * C + c] = t;
+    for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
+    if (lane_p < L) {
+      int p = lane_p;
+      for (; p + 3 * L < P; p += 4 * L) {
+        alignas(16) T q[4][VEC];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const T* src = vb + static_cast<size_t>(p + u * L) * C + static_cast<size_t>(vi) * VEC;
+          if constexpr (VEC * sizeof(T) == 16)
+            *reinterpret_cast<uint4*>(q[u]) = *reinterpret_cast<const uint4*>(src);
+          else
+#pragma unroll
+            for (int k = 0; k < VEC; ++k) q[u][k] = src[k];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int k = 0; k < VEC; ++k) acc[k] += to_f32(q[u][k]);
+      }
+      for (; p < P; p += L) {
+        const T* src = vb + static_cast<size_t>(p) * C + static_cast<size_t>(vi) * VEC;
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) acc[k] += to_f32(src[k]);
+      }
+    }
+    __syncthreads();
+    if (lane_p < L)
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) cs_part[lane_p * (nvec * VEC) + (t % nvec) * VEC + k] = acc[k];
+    __syncthreads();
+    for (int e = t; e < nvec * VEC; e += kBwThreads) {
+      float s = 0.f;
+      for (int l = 0; l < L; ++l) s += cs_part[l * (nvec * VEC) + e];
+      out[static_cast<size_t>(b) * C + static_cast<size_t>(v0) * VEC + e] = s;
+    }
   }
 }
 
@@ -63,9 +96,10 @@ struct WgdParams {
 
 // dW[b][co][kh][kw][ci] = sum over output pixels (oh, ow) of
 // dy[b][oh][ow][co] * x[b][oh*s+kh-p][ow*s+kw-p][g(co)*Cg+ci] (zero outside the
-// image). One thread per weight element of one sample; neighbouring threads
-// take neighbouring input channels, so the x loads of a warp are contiguous
-// and its dy loads are one broadcast.
+// image). One thread per weight element of one sample, threads ordered input
+// channel fastest, then output channel, then tap: in a dense layer a warp's x
+// loads are contiguous and its dy loads one broadcast; in a depthwise layer
+// (one input channel per output channel) both are contiguous runs of channels.
 template <typename T>
 __global__ void __launch_bounds__(kBwThreads) wgrad_direct_kernel(WgdParams p) {
   const long long o = static_cast<long long>(blockIdx.x) * kBwThreads + threadIdx.x;
@@ -73,11 +107,10 @@ __global__ void __launch_bounds__(kBwThreads) wgrad_direct_kernel(WgdParams p) {
   if (o >= p.wsize) return;
   const int Cg = p.Cin / p.groups, Coutg = p.Cout / p.groups;
   const int cil = static_cast<int>(o % Cg);
-  long long t = o / Cg;
-  const int kw = static_cast<int>(t % p.KW);
-  t /= p.KW;
-  const int kh = static_cast<int>(t % p.KH);
-  const int co = static_cast<int>(t / p.KH);
+  const long long t = o / Cg;
+  const int co = static_cast<int>(t % p.Cout);
+  const int tap = static_cast<int>(t / p.Cout);
+  const int kh = tap / p.KW, kw = tap - kh * p.KW;
   const int ci = (co / Coutg) * Cg + cil;
   const T* xb = static_cast<const T*>(p.x) + static_cast<size_t>(b) * p.H * p.W * p.Cin + ci;
   const T* dyb = static_cast<const T*>(p.dy) + static_cast<size_t>(b) * p.Ho * p.Wo * p.Cout + co;
@@ -92,12 +125,94 @@ __global__ void __launch_bounds__(kBwThreads) wgrad_direct_kernel(WgdParams p) {
                  to_f32(xb[(static_cast<size_t>(ih) * p.W + iw) * p.Cin]), acc);
     }
   }
-  p.dW[static_cast<size_t>(b) * p.wsize + o] = acc;
+  p.dW[static_cast<size_t>(b) * p.wsize + (static_cast<size_t>(co) * p.KH * p.KW + tap) * Cg +
+       cil] = acc;
+}
+
+// Depthwise per-sample weight gradient (groups = C_in = C_out, stride 1,
+// square K x K, bf16): dW[b][c][kh][kw] = sum over output pixels of
+// dy[b][oh][ow][c] * x[b][oh+kh-p][ow+kw-p][c]. CTA = (32 channels, sample);
+// bands of output rows are staged in shared memory (x with its K-1 halo rows
+// and columns, zero outside the image, and dy), 16-byte loads. Thread = (lane:
+// channel, threadIdx.y: kh): it slides a K-wide register window of x along each
+// output row, so each output pixel costs two shared loads and K multiply-adds.
+constexpr int kDwgChunk = 32;
+
+struct DwgParams {
+  int B, C, H, W, Ho, Wo, pad, band;
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* dy;
+  float* dW;  // [B][C][K][K]
+};
+
+template <int K>
+__global__ void __launch_bounds__(32 * K) wgrad_dw_kernel(DwgParams p) {
+  extern __shared__ __align__(16) unsigned char dwg_smem[];
+  const int Wp = p.Wo + K - 1;
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(dwg_smem);
+  __nv_bfloat16* ds = xs + static_cast<size_t>(p.band + K - 1) * Wp * kDwgChunk;
+  const int lane = threadIdx.x, kh = threadIdx.y;
+  const int tid = kh * 32 + lane;
+  const int c0 = blockIdx.x * kDwgChunk, b = blockIdx.y;
+  float acc[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) acc[k] = 0.f;
+  for (int oh0 = 0; oh0 < p.Ho; oh0 += p.band) {
+    const int R = min(p.band, p.Ho - oh0);
+    __syncthreads();  // the previous band's readers are done
+    const int xrows = R + K - 1;
+    for (int e = tid; e < xrows * Wp * 4; e += 32 * K) {
+      const int v = e & 3, pix = e >> 2;
+      const int r = pix / Wp, col = pix - r * Wp;
+      const int ih = oh0 + r - p.pad, iw = col - p.pad, c = c0 + v * 8;
+      uint4 q = make_uint4(0u, 0u, 0u, 0u);
+      if (ih >= 0 && ih < p.H && iw >= 0 && iw < p.W && c < p.C)
+        q = *reinterpret_cast<const uint4*>(
+            p.x + ((static_cast<size_t>(b) * p.H + ih) * p.W + iw) * p.C + c);
+      *reinterpret_cast<uint4*>(xs + static_cast<size_t>(pix) * kDwgChunk + v * 8) = q;
+    }
+    for (int e = tid; e < R * p.Wo * 4; e += 32 * K) {
+      const int v = e & 3, pix = e >> 2;
+      const int r = pix / p.Wo, ow = pix - r * p.Wo, c = c0 + v * 8;
+      uint4 q = make_uint4(0u, 0u, 0u, 0u);
+      if (c < p.C)
+        q = *reinterpret_cast<const uint4*>(
+            p.dy + ((static_cast<size_t>(b) * p.Ho + oh0 + r) * p.Wo + ow) * p.C + c);
+      *reinterpret_cast<uint4*>(ds + static_cast<size_t>(pix) * kDwgChunk + v * 8) = q;
+    }
+    __syncthreads();
+    for (int r = 0; r < R; ++r) {
+      // x row r + kh of the band, halo column q holds input column q - pad
+      const __nv_bfloat16* xr = xs + static_cast<size_t>(r + kh) * Wp * kDwgChunk + lane;
+      const __nv_bfloat16* dr = ds + static_cast<size_t>(r) * p.Wo * kDwgChunk + lane;
+      // ring of K values: halo column q sits at index q % K
+      float win[K];
+#pragma unroll
+      for (int k = 0; k < K - 1; ++k) win[k] = __bfloat162float(xr[k * kDwgChunk]);
+      for (int ow0 = 0; ow0 < p.Wo; ow0 += K) {
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+          const int ow = ow0 + j;
+          if (ow < p.Wo) {
+            win[(j + K - 1) % K] = __bfloat162float(xr[(ow + K - 1) * kDwgChunk]);
+            const float d = __bfloat162float(dr[ow * kDwgChunk]);
+#pragma unroll
+            for (int k = 0; k < K; ++k) acc[k] = fmaf(d, win[(j + k) % K], acc[k]);
+          }
+        }
+      }
+    }
+  }
+  const int c = c0 + lane;
+  if (c < p.C)
+#pragma unroll
+    for (int kw = 0; kw < K; ++kw)
+      p.dW[((static_cast<size_t>(b) * p.C + c) * K + kh) * K + kw] = acc[kw];
 }
 
 // ------------------------------------------------ the mixture's gradients
 
-constexpr int kMgMaxExperts = 8;     // experts per CTA at most (grid.y walks the rest)
+constexpr int kMgMaxExperts = 16;    // experts per CTA at most (grid.y walks the rest)
 constexpr int kMgChunk = 4 * kBwThreads;  // weights per CTA: four per thread
 constexpr int kMgSampleBlock = 32;   // samples per partial-sum round
 
@@ -151,30 +266,41 @@ __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
 
   for (int b0 = 0; b0 < p.B; b0 += kMgSampleBlock) {
     const int nbb = min(kMgSampleBlock, p.B - b0);
-    for (int bb = 0; bb < nbb; ++bb) {
-      const int b = b0 + bb;
-      float v[4];
-      const float* src = p.dW + static_cast<size_t>(b) * p.wsize + w;
-      if (p.vec && w < p.wsize) {
-        const float4 q = *reinterpret_cast<const float4*>(src);
-        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-      } else {
+    // four samples per round: their loads are all in flight before the math
+    for (int bb0 = 0; bb0 < nbb; bb0 += 4) {
+      float v[4][4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = w + k < p.wsize ? src[k] : 0.f;
-      }
-      const float* ab = alpha_s + static_cast<size_t>(b) * NE;
+      for (int u = 0; u < 4; ++u) {
+        const float* src = p.dW + static_cast<size_t>(b0 + bb0 + u) * p.wsize + w;
+        if (bb0 + u >= nbb || w >= p.wsize) {
 #pragma unroll
-      for (int i = 0; i < NE; ++i) {
-        const float a = ab[i];
-        float d = 0.f;
+          for (int k = 0; k < 4; ++k) v[u][k] = 0.f;
+        } else if (p.vec) {
+          const float4 q = *reinterpret_cast<const float4*>(src);
+          v[u][0] = q.x; v[u][1] = q.y; v[u][2] = q.z; v[u][3] = q.w;
+        } else {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          dex[i][k] = fmaf(a, v[k], dex[i][k]);
-          d = fmaf(v[k], ev[i][k], d);
+          for (int k = 0; k < 4; ++k) v[u][k] = w + k < p.wsize ? src[k] : 0.f;
         }
+      }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-        if (lane == 0) red[(warp * kMgSampleBlock + bb) * NE + i] = d;
+      for (int u = 0; u < 4; ++u) {
+        const int bb = bb0 + u;
+        if (bb >= nbb) break;  // the same for every thread of the CTA
+        const float* ab = alpha_s + static_cast<size_t>(b0 + bb) * NE;
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+          const float a = ab[i];
+          float d = 0.f;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            dex[i][k] = fmaf(a, v[u][k], dex[i][k]);
+            d = fmaf(v[u][k], ev[i][k], d);
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+          if (lane == 0) red[(warp * kMgSampleBlock + bb) * NE + i] = d;
+        }
       }
     }
     __syncthreads();
@@ -201,24 +327,40 @@ __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
   }
 }
 
-// dalpha[b][i] = sum over chunks (in order) of part[chunk][b][i]
+// dalpha[b][i] = sum over chunks of part[chunk][b][i]
 //              + sum_co db[b][co] * bias[i][co]    (bias may be NULL).
-// One CTA per sample, one thread per expert.
+// One CTA per sample. With n < 256 the chunks are split into S = 256 / n
+// interleaved slices (thread t: expert t % n, slice t / n), each summed in
+// order by one thread; the slice sums are then added in slice order.
 __global__ void __launch_bounds__(kBwThreads)
     dalpha_finish_kernel(int B, int n, int Cout, int chunks, const float* __restrict__ part,
                          const float* __restrict__ db, const float* __restrict__ bias,
                          float* __restrict__ dalpha) {
+  __shared__ float slice_sum[kBwThreads];
   const int b = blockIdx.x;
-  for (int i = threadIdx.x; i < n; i += kBwThreads) {
+  const int S = n < kBwThreads ? kBwThreads / n : 1;
+  for (int i0 = 0; i0 < n; i0 += kBwThreads) {
+    const int i = i0 + (S > 1 ? static_cast<int>(threadIdx.x) % n : static_cast<int>(threadIdx.x));
+    const int sl = S > 1 ? static_cast<int>(threadIdx.x) / n : 0;
     float s = 0.f;
-    for (int c = 0; c < chunks; ++c) s += part[(static_cast<size_t>(c) * B + b) * n + i];
-    if (bias) {
-      float t = 0.f;
-      for (int co = 0; co < Cout; ++co)
-        t = fmaf(db[static_cast<size_t>(b) * Cout + co], bias[static_cast<size_t>(i) * Cout + co], t);
-      s += t;
+    if (i < n && sl < S)
+#pragma unroll 8
+      for (int c = sl; c < chunks; c += S) s += part[(static_cast<size_t>(c) * B + b) * n + i];
+    slice_sum[threadIdx.x] = s;
+    __syncthreads();
+    if (sl == 0 && i < n) {
+      float tot = 0.f;
+      for (int k = 0; k < S; ++k) tot += slice_sum[k * (S > 1 ? n : 0) + threadIdx.x];
+      if (bias) {
+        float t = 0.f;
+#pragma unroll 8
+        for (int co = 0; co < Cout; ++co)
+          t = fmaf(db[static_cast<size_t>(b) * Cout + co], bias[static_cast<size_t>(i) * Cout + co], t);
+        tot += t;
+      }
+      dalpha[static_cast<size_t>(b) * n + i] = tot;
     }
-    dalpha[static_cast<size_t>(b) * n + i] = s;
+    __syncthreads();
   }
 }
 
@@ -230,6 +372,7 @@ __global__ void __launch_bounds__(kBwThreads)
   if (e >= n * Cout) return;
   const int i = e / Cout, co = e - i * Cout;
   float s = 0.f;
+#pragma unroll 8
   for (int b = 0; b < B; ++b)
     s = fmaf(alpha[static_cast<size_t>(b) * n + i], db[static_cast<size_t>(b) * Cout + co], s);
   dbias[e] = s;
@@ -397,16 +540,65 @@ __global__ void __launch_bounds__(kBwThreads) dgrad_direct_kernel(DgdParams p) {
   static_cast<T*>(p.dx)[o] = from_f32<T>(acc);
 }
 
-// dx[b][p][c] += dg[b][c] * inv_hw in place (dx in T, one rounding).
-template <typename T>
+// dx[b][p][c] += dg[b][c] * inv_hw in place (dx in T, one rounding). VEC
+// consecutive channels per thread (one 16-byte access when VEC * sizeof(T)
+// is 16; C % VEC == 0).
+template <typename T, int VEC>
 __global__ void __launch_bounds__(kBwThreads)
-    gap_add_kernel(long long total, int HWC, int C, float inv_hw, const float* __restrict__ dg,
+    gap_add_kernel(long long nvec, int HWC, int C, float inv_hw, const float* __restrict__ dg,
                    T* __restrict__ dx) {
-  for (long long o = static_cast<long long>(blockIdx.x) * kBwThreads + threadIdx.x; o < total;
+  for (long long o = static_cast<long long>(blockIdx.x) * kBwThreads + threadIdx.x; o < nvec;
        o += static_cast<long long>(gridDim.x) * kBwThreads) {
-    const long long b = o / HWC;
-    const int c = static_cast<int>(o % C);
-    dx[o] = from_f32<T>(to_f32(dx[o]) + dg[b * C + c] * inv_hw);
+    const long long e = o * VEC;
+    const long long b = e / HWC;
+    const int c = static_cast<int>(e % C);
+    alignas(16) T q[VEC];
+    if constexpr (VEC * sizeof(T) == 16)
+      *reinterpret_cast<uint4*>(q) = *reinterpret_cast<const uint4*>(dx + e);
+    else
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) q[k] = dx[e + k];
+    const float* g = dg + b * C + c;
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) q[k] = from_f32<T>(to_f32(q[k]) + g[k] * inv_hw);
+    if constexpr (VEC * sizeof(T) == 16)
+      *reinterpret_cast<uint4*>(dx + e) = *reinterpret_cast<const uint4*>(q);
+    else
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) dx[e + k] = q[k];
+  }
+}
+
+// Et = every expert transposed within its group and flipped in both spatial
+// axes, as transpose_experts_kernel, through 32 x 32 tiles of shared memory
+// so that both the reads (input channels contiguous) and the writes (output
+// channels contiguous) are coalesced. Grid (tiles of the group's [Coutg][Cg]
+// matrix, taps * groups, n); block (32, 8).
+template <typename T>
+__global__ void __launch_bounds__(256)
+    transpose_experts_tiled_kernel(int Cin, int Cout, int KH, int KW, int groups,
+                                   const T* __restrict__ E, T* __restrict__ Et) {
+  __shared__ T tile[32][33];
+  const int Cg = Cin / groups, Coutg = Cout / groups;
+  const int tiles_c = (Cg + 31) / 32;
+  const int cil0 = (blockIdx.x % tiles_c) * 32, col0 = (blockIdx.x / tiles_c) * 32;
+  const int taps = KH * KW;
+  const int tap = blockIdx.y % taps, g = blockIdx.y / taps;
+  const int kh = tap / KW, kw = tap - kh * KW;
+  const int tap_src = (KH - 1 - kh) * KW + (KW - 1 - kw);
+  const size_t i = blockIdx.z;
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int col = col0 + r, cil = cil0 + threadIdx.x;
+    T v = from_f32<T>(0.f);
+    if (col < Coutg && cil < Cg)
+      v = E[((i * Cout + g * Coutg + col) * taps + tap_src) * Cg + cil];
+    tile[r][threadIdx.x] = v;
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int cil = cil0 + r, col = col0 + threadIdx.x;
+    if (col < Coutg && cil < Cg)
+      Et[((i * Cin + g * Cg + cil) * taps + tap) * Coutg + col] = tile[threadIdx.x][r];
   }
 }
 

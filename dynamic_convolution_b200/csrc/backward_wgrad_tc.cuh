@@ -33,6 +33,7 @@ namespace dcb {
 
 constexpr int kWgThreads = 192;
 constexpr int kWgMaxAtoms = 4;
+constexpr int kWgStageBytes = 32 * 32 * 4;  // one warp's 32 rows x 32 fp32
 
 // Shared-memory matrix descriptor of an MN-major operand in the 128-byte
 // swizzle: rows of 64 bf16 along M (or N), one row per K index; 64-element
@@ -78,7 +79,8 @@ __global__ void __launch_bounds__(kWgThreads, 1)
   const int S = p.stages;
   const uint32_t ab_bytes = static_cast<uint32_t>(p.atom_bytes);
   const uint32_t stage_bytes = (2 + kWgMaxAtoms) * ab_bytes;
-  const uint32_t bar_base = base + S * stage_bytes;
+  const uint32_t stg_base = base + S * stage_bytes;  // epilogue staging: 4 warps x 4 KB
+  const uint32_t bar_base = stg_base + 4 * kWgStageBytes;
   auto full = [&](int s) { return bar_base + 8u * s; };
   auto empty = [&](int s) { return bar_base + 8u * (S + s); };
   auto tfull = [&](int a) { return bar_base + 8u * (2 * S + a); };
@@ -202,8 +204,11 @@ __global__ void __launch_bounds__(kWgThreads, 1)
     }
   } else {
     // warps 2..5: warp w reads TMEM lanes 32*(w%4) .. +31, output channels
-    // co0 + 32*(w%4) + lane; each thread stores 32 contiguous fp32 per load.
+    // co0 + 32*(w%4) + lane. Each 32 x 32 fp32 block goes through shared
+    // memory (16-byte slots XOR-ed with the row, conflict-free both ways) so
+    // that every store instruction writes four whole 128-byte rows of dW.
     const int q = warp & 3;
+    const uint32_t stg = stg_base + (warp - 2) * kWgStageBytes;
     for (long long j = 0; j < my_units; ++j) {
       const long long u = blockIdx.x + j * gridDim.x;
       const int ag = static_cast<int>(u % p.agroups);
@@ -214,7 +219,6 @@ __global__ void __launch_bounds__(kWgThreads, 1)
       const int ab = static_cast<int>(j & 1);
       if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j >> 1) & 1), ctl, kErrWaitEpilogue)) break;
       tc_fence_after();
-      const int co = cot * 128 + 32 * q + lane;
       for (int a = 0; a < nat; ++a) {
         const int atom = ag * kWgMaxAtoms + a;
         const int tap = atom / p.cblk, cb = atom - tap * p.cblk;
@@ -225,16 +229,25 @@ __global__ void __launch_bounds__(kWgThreads, 1)
                                  a * 64 + h * 32,
                              r);
           tmem_ld_wait(r);
-          const int ci = cb * 64 + h * 32;
-          if (co < p.Cout) {
-            float* dst = p.dW + ((static_cast<size_t>(b) * p.Cout + co) * taps + tap) * p.Cin + ci;
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              if (ci + 4 * v < p.Cin)
-                *reinterpret_cast<float4*>(dst + 4 * v) =
-                    make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          for (int v = 0; v < 8; ++v)
+            st_shared_v4(stg + lane * 128 + ((v ^ (lane & 7)) << 4),
+                         make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]));
+          __syncwarp();
+          const int ci = cb * 64 + h * 32 + 4 * (lane & 7);
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int row = 4 * it + (lane >> 3);
+            uint4 v;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(stg + row * 128 + (((lane & 7) ^ (row & 7)) << 4)));
+            const int co_r = cot * 128 + 32 * q + row;
+            if (co_r < p.Cout && ci < p.Cin)
+              *reinterpret_cast<uint4*>(
+                  p.dW + ((static_cast<size_t>(b) * p.Cout + co_r) * taps + tap) * p.Cin + ci) = v;
           }
+          __syncwarp();
         }
       }
       tc_fence_before();

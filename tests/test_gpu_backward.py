@@ -153,8 +153,15 @@ OTHER = [
     # strided and grouped: the generic input-gradient kernel
     LC("bw_s2g2", synth.BF16, 2, 32, 48, 9, 7, 3, 3, 2, 1, 2, 3, synth.SOFTMAX, 0.7),
     LC("bw_f32_s2", synth.F32, 2, 6, 10, 9, 8, 3, 3, 2, 0, 1, 3, synth.SIGMOID, 1.0),
-    # 1x1 with 40 input channels: the CUDA-core weight gradient under AUTO
+    # 1x1 with 40 input channels and 48 output channels: tcgen05 boxes wider than
+    # the tensor's channel extent (zero fill)
     LC("bw_c40", synth.BF16, 3, 40, 48, 10, 10, 1, 1, 1, 0, 1, 8, synth.SIGMOID, 1.0),
+    # 16 output channels; 20 experts (a group of 16 and a partial group of 4)
+    LC("bw_c16out", synth.BF16, 2, 64, 16, 9, 9, 3, 3, 1, 1, 1, 20, synth.SOFTMAX, 1.0),
+    # grouped, stride 1: tiled expert transposition with groups, CUDA-core forward
+    LC("bw_g4", synth.BF16, 2, 64, 64, 8, 8, 3, 3, 1, 1, 4, 3, synth.SIGMOID, 1.0),
+    # 12 input channels: rows not a 16-byte multiple (unvectorised sums and adds)
+    LC("bw_c12", synth.BF16, 2, 12, 16, 6, 6, 3, 3, 1, 1, 1, 2, synth.SIGMOID, 1.0),
 ]
 
 
@@ -163,6 +170,14 @@ OTHER = [
 def test_backward_cuda_core_paths(cfg):
     c = Case(cfg)
     _check_all(c.run(), c.reference(), cfg)
+
+
+@pytest.mark.parametrize("cfg,wg", [(OTHER[0], dc.VARIANT_DIRECT), (OTHER[1], dc.VARIANT_DEPTHWISE),
+                                    (OTHER[4], dc.VARIANT_DIRECT)],
+                         ids=["depthwise-generic", "depthwise-forced", "c40-cuda-core"])
+def test_backward_forced_weight_kernels(cfg, wg):
+    c = Case(cfg)
+    _check_all(c.run(wg_variant=wg), c.reference(), cfg)
 
 
 def test_backward_without_bias():
