@@ -688,7 +688,7 @@ def run_backward(args, cfg):
 
     def router(s, st):
         dc.check(dc.dynconv_route_backward(d, xs[s], Wr, alphas[s], dalpha, cfg.mode, cfg.tau,
-                                           dWr, dbr, dg, st))
+                                           dWr, dbr, dg, ws, wsb, st))
 
     def data(s, st):
         dc.check(dc.dynconv_backward_data(d, dys_[s], E, alphas[s], dg, dxs[s], ws, wsb, st))

@@ -97,7 +97,7 @@ def load():
         lib.dynconv_backward_weight.argtypes = [D, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.dynconv_backward_weight.restype = ctypes.c_int
         lib.dynconv_route_backward.argtypes = [D, P, P, P, P, ctypes.c_int, ctypes.c_float, P, P,
-                                               P, P]
+                                               P, P, ctypes.c_size_t, P]
         lib.dynconv_route_backward.restype = ctypes.c_int
         lib.dynconv_backward_data.argtypes = [D, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.dynconv_backward_data.restype = ctypes.c_int
@@ -242,11 +242,12 @@ def dynconv_backward_weight(desc, x, dy, experts, alpha, bias, dexperts, dbias, 
 
 
 def dynconv_route_backward(desc, x, Wr, alpha, dalpha, mode, tau, dWr, dbr, dg,
-                           stream=None) -> int:
+                           workspace=None, workspace_bytes=0, stream=None) -> int:
     """dWr [n][C_in], dbr [n] (may be None), dg [B][C_in] (fp32)."""
     return load().dynconv_route_backward(ctypes.byref(desc), _ptr(x), _ptr(Wr), _ptr(alpha),
                                          _ptr(dalpha), int(mode), float(tau), _ptr(dWr),
-                                         _ptr(dbr), _ptr(dg), _stream(stream))
+                                         _ptr(dbr), _ptr(dg), _ptr(workspace),
+                                         int(workspace_bytes), _stream(stream))
 
 
 def dynconv_backward_data(desc, dy, experts, alpha, dg, dx, workspace, workspace_bytes,

@@ -32,15 +32,16 @@ long long wsize_of(const dynconv_desc* d) {
   return 1LL * d->C_out * d->KH * d->KW * (d->C_in / d->groups);
 }
 
-int launch_error(cudaError_t e, const char* what) {
-  dc_lib::launched(what);
-  return dc_lib::cuda_error(e, what);
-}
-
 // ------------------------------------------------------- workspace layout
 
+// Slices of the channel sums are sized for at most this many SMs (the
+// workspace size is a pure host function).
+constexpr int kMaxSms = 160;
+
+int chansum_slices(int B, int P, int sms);
+
 struct WeightLayout {
-  size_t dW = 0, db = 0, part = 0, total = 0;
+  size_t dW = 0, db = 0, part = 0, cs = 0, total = 0;
   int chunks = 0;
 };
 
@@ -51,7 +52,9 @@ WeightLayout weight_layout(const dynconv_desc* d) {
   L.dW = 0;
   L.db = align256(L.dW + 4ull * d->B * ws);
   L.part = align256(L.db + 4ull * d->B * d->C_out);
-  L.total = align256(L.part + 4ull * L.chunks * d->B * d->n);
+  L.cs = align256(L.part + 4ull * L.chunks * d->B * d->n);
+  const int Ho = out_size(d->H, d->KH, d->stride, d->pad), Wo = out_size(d->W, d->KW, d->stride, d->pad);
+  L.total = align256(L.cs + 4ull * d->B * d->C_out * chansum_slices(d->B, Ho * Wo, kMaxSms));
   return L;
 }
 
@@ -213,27 +216,45 @@ int run_wgrad_dw(const dynconv_desc* d, int band, size_t smem, const void* x, co
          : d->KH == 5 ? go(dcb::wgrad_dw_kernel<5>, 5) : go(dcb::wgrad_dw_kernel<7>, 7);
 }
 
-int run_chansum(const dynconv_desc* d, const void* v, int P, int C, float* out, cudaStream_t s) {
+// Pixel slices per sample for the channel sums: about four CTAs per SM in
+// all, at least 32 pixels per slice.
+int chansum_slices(int B, int P, int sms) {
+  const int want = std::max(1, (4 * sms + B - 1) / std::max(B, 1));
+  return std::max(1, std::min(want, P / 32));
+}
+
+// out[b][c] = sum over pixels of v; `scratch` holds B * slices * C floats.
+int run_chansum(const dynconv_desc* d, int sms, const void* v, int P, int C, float* scratch,
+                float* out, cudaStream_t s) {
   const bool bf = d->dtype == DYNCONV_BF16;
   const int vec = bf ? 8 : 4;
   const bool vok = C % vec == 0 && aligned16(v);
   const size_t smem = sizeof(float) * dcb::kBwThreads * (vok ? vec : 1);
+  const int slices = scratch ? chansum_slices(d->B, P, sms) : 1;
+  if (slices == 1) scratch = out;  // one slice: the partial is the sum
+  const int Ps = (P + slices - 1) / slices;
+  const dim3 grid(slices, d->B);
   if (bf) {
     if (vok)
-      dcb::chansum_kernel<__nv_bfloat16, 8><<<d->B, dcb::kBwThreads, smem, s>>>(
-          static_cast<const __nv_bfloat16*>(v), P, C, out);
+      dcb::chansum_kernel<__nv_bfloat16, 8><<<grid, dcb::kBwThreads, smem, s>>>(
+          static_cast<const __nv_bfloat16*>(v), P, C, Ps, scratch);
     else
-      dcb::chansum_kernel<__nv_bfloat16, 1><<<d->B, dcb::kBwThreads, smem, s>>>(
-          static_cast<const __nv_bfloat16*>(v), P, C, out);
+      dcb::chansum_kernel<__nv_bfloat16, 1><<<grid, dcb::kBwThreads, smem, s>>>(
+          static_cast<const __nv_bfloat16*>(v), P, C, Ps, scratch);
   } else {
     if (vok)
-      dcb::chansum_kernel<float, 4><<<d->B, dcb::kBwThreads, smem, s>>>(
-          static_cast<const float*>(v), P, C, out);
+      dcb::chansum_kernel<float, 4><<<grid, dcb::kBwThreads, smem, s>>>(
+          static_cast<const float*>(v), P, C, Ps, scratch);
     else
-      dcb::chansum_kernel<float, 1><<<d->B, dcb::kBwThreads, smem, s>>>(
-          static_cast<const float*>(v), P, C, out);
+      dcb::chansum_kernel<float, 1><<<grid, dcb::kBwThreads, smem, s>>>(
+          static_cast<const float*>(v), P, C, Ps, scratch);
   }
-  return dc_lib::launched("chansum_kernel");
+  int rc = dc_lib::launched("chansum_kernel");
+  if (rc || slices == 1) return rc;
+  const long long total = 1LL * d->B * C;
+  dcb::chansum_finish_kernel<<<static_cast<unsigned>((total + dcb::kBwThreads - 1) / dcb::kBwThreads),
+                               dcb::kBwThreads, 0, s>>>(d->B, C, slices, scratch, out);
+  return dc_lib::launched("chansum_finish_kernel");
 }
 
 template <typename T>
@@ -251,8 +272,7 @@ int launch_mixgrad(const dcb::MgParams& p, int ne, size_t smem, cudaStream_t s) 
     case 1: return go(dcb::mixgrad_kernel<T, 1>);
     case 2: return go(dcb::mixgrad_kernel<T, 2>);
     case 4: return go(dcb::mixgrad_kernel<T, 4>);
-    case 8: return go(dcb::mixgrad_kernel<T, 8>);
-    default: return go(dcb::mixgrad_kernel<T, 16>);
+    default: return go(dcb::mixgrad_kernel<T, 8>);
   }
 }
 
@@ -262,7 +282,9 @@ extern "C" {
 
 size_t dynconv_backward_workspace_size(const dynconv_desc* desc) {
   if (dc_lib::validate(desc) != DYNCONV_OK) return 0;
-  return std::max(weight_layout(desc).total, data_workspace(desc));
+  const size_t route = align256(4ull * desc->B * desc->C_in *
+                                chansum_slices(desc->B, desc->H * desc->W, kMaxSms));
+  return std::max({weight_layout(desc).total, data_workspace(desc), route});
 }
 
 int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void* dy,
@@ -329,7 +351,8 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
   // 2. per-sample bias gradients: channel sums of dy
   const int Ho = out_size(d->H, d->KH, d->stride, d->pad);
   const int Wo = out_size(d->W, d->KW, d->stride, d->pad);
-  rc = run_chansum(d, dy, Ho * Wo, d->C_out, db, s);
+  rc = run_chansum(d, std::min(di.sms, kMaxSms), dy, Ho * Wo, d->C_out,
+                   reinterpret_cast<float*>(wsb + L.cs), db, s);
   if (rc) return rc;
   // 3. the experts' gradients and the chunks' shares of dalpha
   dcb::MgParams mp{};
@@ -337,7 +360,7 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
   mp.vec = (ws % 4 == 0 && aligned16(dexperts)) ? 1 : 0;
   mp.dW = dW; mp.experts = experts; mp.alpha = alpha; mp.dexperts = dexperts; mp.part = part;
   // experts per CTA: every sample's dW is read ceil(n / ne) times
-  const int ne = d->n >= 16 ? 16 : d->n > 4 ? 8 : d->n > 2 ? 4 : d->n;
+  const int ne = d->n > 4 ? 8 : d->n > 2 ? 4 : d->n;
   const size_t mg_smem = sizeof(float) * (static_cast<size_t>(d->B) * ne +
                                           (dcb::kBwThreads / 32) * dcb::kMgSampleBlock * ne);
   if (mg_smem > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
@@ -351,8 +374,7 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
   if (rc) return rc;
   // 5. dbias
   if (dbias) {
-    const int total = d->n * d->C_out;
-    dcb::dbias_kernel<<<(total + dcb::kBwThreads - 1) / dcb::kBwThreads, dcb::kBwThreads, 0, s>>>(
+    dcb::dbias_kernel<<<dim3((d->C_out + 31) / 32, (d->n + 7) / 8), dim3(32, 8), 0, s>>>(
         d->B, d->n, d->C_out, alpha, db, dbias);
     rc = dc_lib::launched("dbias_kernel");
   }
@@ -361,7 +383,8 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
 
 int dynconv_route_backward(const dynconv_desc* desc, const void* x, const float* Wr,
                            const float* alpha, const float* dalpha, int mode, float tau,
-                           float* dWr, float* dbr, float* dg, void* stream) {
+                           float* dWr, float* dbr, float* dg, void* workspace,
+                           size_t workspace_bytes, void* stream) {
   int rc = dc_lib::validate(desc);
   if (rc) return rc;
   if (!x || !Wr || !alpha || !dalpha || !dWr || !dg) return DYNCONV_ERR_INVALID_ARG;
@@ -381,8 +404,16 @@ int dynconv_route_backward(const dynconv_desc* desc, const void* x, const float*
   const size_t smem_param = sizeof(float) * static_cast<size_t>(B);
   const size_t smem_dg = sizeof(float) * (static_cast<size_t>(n) + dcb::kBwThreads);
   if (smem_param > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
-  // the channel sums of x go to dg first (scratch), then dg is overwritten
-  rc = run_chansum(desc, x, desc->H * desc->W, C, dg, s);
+  // the channel sums of x go to dg first (scratch), then dg is overwritten;
+  // their pixel slices use the workspace when it has room
+  const int sms = std::min(di.sms, kMaxSms);
+  const size_t cs_bytes =
+      4ull * B * C * chansum_slices(B, desc->H * desc->W, sms);
+  float* cs = (workspace && workspace_bytes >= cs_bytes &&
+               (reinterpret_cast<uintptr_t>(workspace) & 15u) == 0)
+                  ? static_cast<float*>(workspace)
+                  : nullptr;
+  rc = run_chansum(desc, sms, x, desc->H * desc->W, C, cs, dg, s);
   if (rc) return rc;
   if (smem_param > 48 * 1024) {
     cudaError_t e = dc_lib::set_smem(reinterpret_cast<const void*>(dcb::route_bwd_param_kernel),

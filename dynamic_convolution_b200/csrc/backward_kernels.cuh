@@ -27,16 +27,20 @@ constexpr int kBwThreads = 256;
 
 // ------------------------------------------------------------ channel sums
 
-// out[b][c] = sum over p < P of v[b][p][c] (v is [B][P][C]). One CTA per
-// sample: thread t takes the VEC channels of vector t % cv (cv = C / VEC
-// vectors per pixel) and the pixels t / cv, t / cv + L, ... (L = 256 / cv pixel
-// lanes), four 16-byte loads in flight; the L lane sums are then added in
-// lane order. VEC = 1 is the unvectorised form (any C, any alignment).
+// Channel sums in two passes. chansum_kernel: CTA (slice, sample) sums the
+// pixels [slice * P_s, (slice + 1) * P_s) of v[b][p][c] (v is [B][P][C]) into
+// part[b][slice][c]: thread t takes the VEC channels of vector t % cv (cv =
+// C / VEC vectors per pixel) and every L-th pixel of the slice (L = 256 / cv
+// pixel lanes), four 16-byte loads in flight; the L lane sums are added in
+// lane order. chansum_finish_kernel adds the slices in order. VEC = 1 is the
+// unvectorised form (any C, any alignment).
 template <typename T, int VEC>
 __global__ void __launch_bounds__(kBwThreads) chansum_kernel(const T* __restrict__ v, int P, int C,
-                                                             float* __restrict__ out) {
+                                                             int Ps, float* __restrict__ part) {
   extern __shared__ float cs_part[];  // [L][C]
-  const int b = blockIdx.x;
+  const int b = blockIdx.y, slice = blockIdx.x;
+  const int nslices = gridDim.x;
+  const int p_begin = slice * Ps, p_end = min(P, p_begin + Ps);
   const int cv = C / VEC;
   const T* vb = v + static_cast<size_t>(b) * P * C;
   for (int v0 = 0; v0 < cv; v0 += kBwThreads) {
@@ -48,8 +52,8 @@ __global__ void __launch_bounds__(kBwThreads) chansum_kernel(const T* __restrict
 #pragma unroll
     for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
     if (lane_p < L) {
-      int p = lane_p;
-      for (; p + 3 * L < P; p += 4 * L) {
+      int p = p_begin + lane_p;
+      for (; p + 3 * L < p_end; p += 4 * L) {
         alignas(16) T q[4][VEC];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -65,7 +69,7 @@ __global__ void __launch_bounds__(kBwThreads) chansum_kernel(const T* __restrict
 #pragma unroll
           for (int k = 0; k < VEC; ++k) acc[k] += to_f32(q[u][k]);
       }
-      for (; p < P; p += L) {
+      for (; p < p_end; p += L) {
         const T* src = vb + static_cast<size_t>(p) * C + static_cast<size_t>(vi) * VEC;
 #pragma unroll
         for (int k = 0; k < VEC; ++k) acc[k] += to_f32(src[k]);
@@ -79,9 +83,23 @@ __global__ void __launch_bounds__(kBwThreads) chansum_kernel(const T* __restrict
     for (int e = t; e < nvec * VEC; e += kBwThreads) {
       float s = 0.f;
       for (int l = 0; l < L; ++l) s += cs_part[l * (nvec * VEC) + e];
-      out[static_cast<size_t>(b) * C + static_cast<size_t>(v0) * VEC + e] = s;
+      part[(static_cast<size_t>(b) * nslices + slice) * C + static_cast<size_t>(v0) * VEC + e] = s;
     }
   }
+}
+
+// out[b][c] = sum over slices, in order, of part[b][slice][c].
+__global__ void __launch_bounds__(kBwThreads)
+    chansum_finish_kernel(int B, int C, int nslices, const float* __restrict__ part,
+                          float* __restrict__ out) {
+  const long long e = static_cast<long long>(blockIdx.x) * kBwThreads + threadIdx.x;
+  if (e >= 1LL * B * C) return;
+  const long long b = e / C;
+  const int c = static_cast<int>(e - b * C);
+  float s = 0.f;
+#pragma unroll 4
+  for (int k = 0; k < nslices; ++k) s += part[(b * nslices + k) * C + c];
+  out[e] = s;
 }
 
 // ------------------------------------------- per-sample weight gradient
@@ -212,7 +230,7 @@ __global__ void __launch_bounds__(32 * K) wgrad_dw_kernel(DwgParams p) {
 
 // ------------------------------------------------ the mixture's gradients
 
-constexpr int kMgMaxExperts = 16;    // experts per CTA at most (grid.y walks the rest)
+constexpr int kMgMaxExperts = 8;     // experts per CTA at most (grid.y walks the rest)
 constexpr int kMgChunk = 4 * kBwThreads;  // weights per CTA: four per thread
 constexpr int kMgSampleBlock = 32;   // samples per partial-sum round
 
@@ -266,11 +284,11 @@ __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
 
   for (int b0 = 0; b0 < p.B; b0 += kMgSampleBlock) {
     const int nbb = min(kMgSampleBlock, p.B - b0);
-    // four samples per round: their loads are all in flight before the math
-    for (int bb0 = 0; bb0 < nbb; bb0 += 4) {
-      float v[4][4];
+    // eight samples per round: their loads are all in flight before the math
+    for (int bb0 = 0; bb0 < nbb; bb0 += 8) {
+      float v[8][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const float* src = p.dW + static_cast<size_t>(b0 + bb0 + u) * p.wsize + w;
         if (bb0 + u >= nbb || w >= p.wsize) {
 #pragma unroll
@@ -284,7 +302,7 @@ __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int bb = bb0 + u;
         if (bb >= nbb) break;  // the same for every thread of the CTA
         const float* ab = alpha_s + static_cast<size_t>(b0 + bb) * NE;
@@ -329,9 +347,10 @@ __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
 
 // dalpha[b][i] = sum over chunks of part[chunk][b][i]
 //              + sum_co db[b][co] * bias[i][co]    (bias may be NULL).
-// One CTA per sample. With n < 256 the chunks are split into S = 256 / n
-// interleaved slices (thread t: expert t % n, slice t / n), each summed in
-// order by one thread; the slice sums are then added in slice order.
+// One CTA per sample. With n < 256 the chunks and the output channels are
+// split into S = 256 / n interleaved slices (thread t: expert t % n, slice
+// t / n), each summed in order by one thread; the slice sums are then added
+// in slice order.
 __global__ void __launch_bounds__(kBwThreads)
     dalpha_finish_kernel(int B, int n, int Cout, int chunks, const float* __restrict__ part,
                          const float* __restrict__ db, const float* __restrict__ bias,
@@ -343,39 +362,58 @@ __global__ void __launch_bounds__(kBwThreads)
     const int i = i0 + (S > 1 ? static_cast<int>(threadIdx.x) % n : static_cast<int>(threadIdx.x));
     const int sl = S > 1 ? static_cast<int>(threadIdx.x) / n : 0;
     float s = 0.f;
-    if (i < n && sl < S)
+    if (i < n && sl < S) {
 #pragma unroll 8
       for (int c = sl; c < chunks; c += S) s += part[(static_cast<size_t>(c) * B + b) * n + i];
+      if (bias) {
+        // this slice's share of <db_b, bias_i>
+        float t = 0.f;
+#pragma unroll 8
+        for (int co = sl; co < Cout; co += S)
+          t = fmaf(db[static_cast<size_t>(b) * Cout + co], bias[static_cast<size_t>(i) * Cout + co], t);
+        s += t;
+      }
+    }
     slice_sum[threadIdx.x] = s;
     __syncthreads();
     if (sl == 0 && i < n) {
       float tot = 0.f;
       for (int k = 0; k < S; ++k) tot += slice_sum[k * (S > 1 ? n : 0) + threadIdx.x];
-      if (bias) {
-        float t = 0.f;
-#pragma unroll 8
-        for (int co = 0; co < Cout; ++co)
-          t = fmaf(db[static_cast<size_t>(b) * Cout + co], bias[static_cast<size_t>(i) * Cout + co], t);
-        tot += t;
-      }
       dalpha[static_cast<size_t>(b) * n + i] = tot;
     }
     __syncthreads();
   }
 }
 
-// dbias[i][co] = sum_b alpha[b][i] * db[b][co], one thread per element.
-__global__ void __launch_bounds__(kBwThreads)
+// dbias[i][co] = sum_b alpha[b][i] * db[b][co]. CTA = (32 channels, up to 8
+// experts); thread (lane: channel, y: one of 8 interleaved sample slices)
+// sums its slice for each expert; the slices are added in order.
+__global__ void __launch_bounds__(256)
     dbias_kernel(int B, int n, int Cout, const float* __restrict__ alpha,
                  const float* __restrict__ db, float* __restrict__ dbias) {
-  const int e = blockIdx.x * kBwThreads + threadIdx.x;
-  if (e >= n * Cout) return;
-  const int i = e / Cout, co = e - i * Cout;
-  float s = 0.f;
-#pragma unroll 8
-  for (int b = 0; b < B; ++b)
-    s = fmaf(alpha[static_cast<size_t>(b) * n + i], db[static_cast<size_t>(b) * Cout + co], s);
-  dbias[e] = s;
+  __shared__ float red[8][8][33];  // [slice][expert][channel]
+  const int co = blockIdx.x * 32 + threadIdx.x;
+  const int i0 = blockIdx.y * 8, ne = min(8, n - i0);
+  float acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+  if (co < Cout)
+    for (int b = threadIdx.y; b < B; b += 8) {
+      const float d = db[static_cast<size_t>(b) * Cout + co];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (k < ne) acc[k] = fmaf(alpha[static_cast<size_t>(b) * n + i0 + k], d, acc[k]);
+    }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) red[threadIdx.y][k][threadIdx.x] = acc[k];
+  __syncthreads();
+  if (threadIdx.y < ne && co < Cout) {
+    const int k = threadIdx.y;
+    float s = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < 8; ++sl) s += red[sl][k][threadIdx.x];
+    dbias[static_cast<size_t>(i0 + k) * Cout + co] = s;
+  }
 }
 
 // ------------------------------------------------------ router gradients

@@ -32,8 +32,9 @@
  * [B][H_out][W_out][C_out] in desc->dtype; experts [n][C_out][KH][KW][C_in/groups]
  * in desc->dtype; alpha, bias, Wr as in dynconv.h (fp32). Every gradient is
  * fp32 and in the layout of the value it belongs to, except dx, which is in
- * desc->dtype (rounded once after the convolution's input gradient, and once
- * more after dg/(H*W) is added). Outputs are overwritten, not accumulated.
+ * desc->dtype: rounded once after the convolution's input gradient and once
+ * more after dg/(H*W) is added when it runs on the forward kernels, once when
+ * it runs on the generic kernel. Outputs are overwritten, not accumulated.
  * All results are deterministic (no floating-point atomics).
  *
  * Ownership: the caller allocates every buffer (device memory) and the
@@ -51,9 +52,9 @@
 extern "C" {
 #endif
 
-/* Bytes of device workspace that dynconv_backward_weight and
- * dynconv_backward_data need for this descriptor (one buffer serves both; 0
- * on an invalid descriptor). Pure host function. */
+/* Bytes of device workspace that the three backward calls need for this
+ * descriptor (one buffer serves all three, in turn; 0 on an invalid
+ * descriptor). Pure host function. */
 size_t dynconv_backward_workspace_size(const dynconv_desc* desc);
 
 /* Gradients of the experts, their biases and the attentions.
@@ -71,8 +72,11 @@ size_t dynconv_backward_workspace_size(const dynconv_desc* desc);
  * The per-sample gradients dW_b are computed by the tcgen05 weight-gradient
  * kernel when desc->variant is AUTO or a tensor-core variant and the shape
  * allows it (bf16, groups 1, stride 1, C_in and C_out multiples of 8,
- * W_out <= 128), else by the CUDA-core kernel (desc->variant DIRECT forces
- * it); a forced tensor-core variant on another shape returns UNSUPPORTED.
+ * W_out <= 128); else, for a bf16 depthwise layer (groups = C_in = C_out,
+ * stride 1, square 3x3, 5x5 or 7x7, C_in a multiple of 8), by the depthwise
+ * CUDA-core kernel (desc->variant DEPTHWISE forces it); else by the generic
+ * CUDA-core kernel (desc->variant DIRECT forces it). A forced variant on a
+ * shape its kernel does not take returns UNSUPPORTED.
  * Errors: INVALID_ARG (NULL pointer, bias/dbias mismatch, bad descriptor),
  * UNSUPPORTED, MISALIGNED (x, dy or workspace not 16-byte aligned on the
  * tensor-core path), WORKSPACE, CUDA. */
@@ -88,12 +92,16 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
  *   alpha    fp32 [B][n], dalpha fp32 [B][n] (from dynconv_backward_weight)
  *   mode, tau: as in dynconv_route
  *   dWr fp32 [n][C_in], dbr fp32 [n], dg fp32 [B][C_in]  (out; dbr may be NULL)
- * dg is first used as scratch for the channel sums of x.
+ *   workspace, workspace_bytes: as for dynconv_backward_weight (the same
+ *            buffer serves all three calls); may be NULL, the channel sums of
+ *            x then run with less parallelism.
+ * dg is also used as scratch for the channel sums of x.
  * Errors: INVALID_ARG (NULL pointers, bad mode or tau), UNSUPPORTED
  * (n > 1024), CUDA. */
 int dynconv_route_backward(const dynconv_desc* desc, const void* x, const float* Wr,
                            const float* alpha, const float* dalpha, int mode, float tau,
-                           float* dWr, float* dbr, float* dg, void* stream);
+                           float* dWr, float* dbr, float* dg, void* workspace,
+                           size_t workspace_bytes, void* stream);
 
 /* Gradient of the layer's input.
  *   dy, experts, alpha: as for dynconv_backward_weight
@@ -109,7 +117,9 @@ int dynconv_route_backward(const dynconv_desc* desc, const void* x, const float*
  * workspace. Other shapes run a CUDA-core kernel. dg/(H*W) is then added in
  * place.
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA, and those of
- * dynconv_forward for the transposed shape. */
+ * dynconv_forward for the transposed shape; an error of that forward call (a
+ * forced variant that cannot take the transposed shape) comes after the
+ * transposition kernel has run: dx is then not written. */
 int dynconv_backward_data(const dynconv_desc* desc, const void* dy, const void* experts,
                           const float* alpha, const float* dg, void* dx, void* workspace,
                           size_t workspace_bytes, void* stream);

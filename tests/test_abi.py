@@ -176,10 +176,11 @@ def test_backward_entry_points_host_side(lib):
     assert bw(s2, P, P, P, P, P, P, P, P, P, ws) == dc.ERR_UNSUPPORTED       # forced TC, stride 2
     assert bw(d, P, P, P, P, P, P, P, P, P, ws) == dc.ERR_CUDA               # no device: loud
     rb = dc.dynconv_route_backward
-    assert rb(d, P, P, P, P, 2, 1.0, P, P, P) == dc.ERR_INVALID_ARG          # bad mode
-    assert rb(d, P, P, P, P, dc.SOFTMAX, 0.0, P, P, P) == dc.ERR_INVALID_ARG
-    assert rb(d, P, None, P, P, dc.SOFTMAX, 1.0, P, P, P) == dc.ERR_INVALID_ARG
-    assert rb(d, P, P, P, P, dc.SOFTMAX, 1.0, P, None, P) == dc.ERR_CUDA     # dbr optional
+    assert rb(d, P, P, P, P, 2, 1.0, P, P, P, P, ws) == dc.ERR_INVALID_ARG          # bad mode
+    assert rb(d, P, P, P, P, dc.SOFTMAX, 0.0, P, P, P, P, ws) == dc.ERR_INVALID_ARG
+    assert rb(d, P, None, P, P, dc.SOFTMAX, 1.0, P, P, P, P, ws) == dc.ERR_INVALID_ARG
+    assert rb(d, P, P, P, P, dc.SOFTMAX, 1.0, P, None, P, P, ws) == dc.ERR_CUDA     # dbr optional
+    assert rb(d, P, P, P, P, dc.SOFTMAX, 1.0, P, P, P) == dc.ERR_CUDA               # no workspace
     bd = dc.dynconv_backward_data
     assert bd(d, None, P, P, None, P, P, ws) == dc.ERR_INVALID_ARG
     assert bd(d, P, P, P, None, P, P, 1024) == dc.ERR_WORKSPACE              # no room for experts

@@ -78,7 +78,7 @@ class Case:
                  "dynconv_backward_weight")
         dWr, dbr, dg = nan(cfg.n, cfg.C_in), nan(cfg.n), nan(cfg.B, cfg.C_in)
         dc.check(dc.dynconv_route_backward(d, L.x, L.Wr, L.alpha, dalpha, cfg.mode, cfg.tau,
-                                           dWr, dbr, dg), "dynconv_route_backward")
+                                           dWr, dbr, dg, ws, wsb), "dynconv_route_backward")
         dx = torch.full_like(L.x, float("nan"))
         dc.check(dc.dynconv_backward_data(dc.desc_from_config(cfg, dx_variant), self.dy,
                                           L.experts, L.alpha, dg, dx, ws, wsb),
