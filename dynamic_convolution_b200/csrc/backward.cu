@@ -41,9 +41,19 @@ constexpr int kMaxSms = 160;
 int chansum_slices(int B, int P, int sms);
 
 struct WeightLayout {
-  size_t dW = 0, db = 0, part = 0, cs = 0, total = 0;
+  size_t dW = 0, db = 0, part = 0, cs = 0, dex = 0, total = 0;
   int chunks = 0;
+  int bsplit = 1;  // sample groups of the mixing gradient (partial dexperts when > 1)
 };
+
+// Sample groups for the mixing gradient: about two CTAs per SM in all, at
+// least 8 samples per group.
+int mix_bsplit(const dynconv_desc* d, int chunks) {
+  const int ne = d->n > 4 ? 8 : d->n > 2 ? 4 : d->n;
+  const long long ctas = 1LL * chunks * ((d->n + ne - 1) / ne);
+  const long long want = (2LL * kMaxSms + ctas - 1) / ctas;
+  return static_cast<int>(std::max<long long>(1, std::min<long long>(want, d->B / 8)));
+}
 
 WeightLayout weight_layout(const dynconv_desc* d) {
   WeightLayout L;
@@ -54,7 +64,9 @@ WeightLayout weight_layout(const dynconv_desc* d) {
   L.part = align256(L.db + 4ull * d->B * d->C_out);
   L.cs = align256(L.part + 4ull * L.chunks * d->B * d->n);
   const int Ho = out_size(d->H, d->KH, d->stride, d->pad), Wo = out_size(d->W, d->KW, d->stride, d->pad);
-  L.total = align256(L.cs + 4ull * d->B * d->C_out * chansum_slices(d->B, Ho * Wo, kMaxSms));
+  L.dex = align256(L.cs + 4ull * d->B * d->C_out * chansum_slices(d->B, Ho * Wo, kMaxSms));
+  L.bsplit = mix_bsplit(d, L.chunks);
+  L.total = align256(L.dex + (L.bsplit > 1 ? 4ull * L.bsplit * d->n * ws : 0));
   return L;
 }
 
@@ -259,7 +271,7 @@ int run_chansum(const dynconv_desc* d, int sms, const void* v, int P, int C, flo
 
 template <typename T>
 int launch_mixgrad(const dcb::MgParams& p, int ne, size_t smem, cudaStream_t s) {
-  const dim3 grid(p.chunks, (p.n + ne - 1) / ne);
+  const dim3 grid(p.chunks, (p.n + ne - 1) / ne, p.bsplit);
   auto go = [&](auto kern) -> int {
     if (smem > 48 * 1024) {
       cudaError_t e = dc_lib::set_smem(reinterpret_cast<const void*>(kern), smem);
@@ -358,7 +370,11 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
   dcb::MgParams mp{};
   mp.B = d->B; mp.n = d->n; mp.wsize = ws; mp.chunks = L.chunks;
   mp.vec = (ws % 4 == 0 && aligned16(dexperts)) ? 1 : 0;
-  mp.dW = dW; mp.experts = experts; mp.alpha = alpha; mp.dexperts = dexperts; mp.part = part;
+  mp.dW = dW; mp.experts = experts; mp.alpha = alpha; mp.part = part;
+  mp.bsplit = L.bsplit;
+  mp.bs = (d->B + L.bsplit - 1) / L.bsplit;
+  mp.dexperts = L.bsplit > 1 ? reinterpret_cast<float*>(wsb + L.dex) : dexperts;
+  if (L.bsplit > 1) mp.vec = ws % 4 == 0 ? 1 : 0;
   // experts per CTA: every sample's dW is read ceil(n / ne) times
   const int ne = d->n > 4 ? 8 : d->n > 2 ? 4 : d->n;
   const size_t mg_smem = sizeof(float) * (static_cast<size_t>(d->B) * ne +
@@ -367,6 +383,15 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
   rc = d->dtype == DYNCONV_F32 ? launch_mixgrad<float>(mp, ne, mg_smem, s)
                                : launch_mixgrad<__nv_bfloat16>(mp, ne, mg_smem, s);
   if (rc) return rc;
+  if (L.bsplit > 1) {
+    const long long total = 1LL * d->n * ws;
+    const unsigned g = static_cast<unsigned>(
+        std::min<long long>((total / 4 + dcb::kBwThreads) / dcb::kBwThreads, 16LL * di.sms));
+    dcb::dexperts_finish_kernel<<<g, dcb::kBwThreads, 0, s>>>(total, L.bsplit, mp.dexperts,
+                                                              dexperts);
+    rc = dc_lib::launched("dexperts_finish_kernel");
+    if (rc) return rc;
+  }
   // 4. dalpha = sum of the chunks' shares + <db_b, bias_i>
   dcb::dalpha_finish_kernel<<<d->B, dcb::kBwThreads, 0, s>>>(d->B, d->n, d->C_out, L.chunks, part,
                                                              db, bias, dalpha);

@@ -25,6 +25,19 @@ using dc::to_f32;
 
 constexpr int kBwThreads = 256;
 
+// 16-byte asynchronous copy global -> shared (cp.async, L2 only); with
+// valid == false nothing is read and the 16 bytes are zero-filled (src must
+// still be a mapped address).
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+// Wait for every cp.async this thread issued.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // ------------------------------------------------------------ channel sums
 
 // Channel sums in two passes. chansum_kernel: CTA (slice, sample) sums the
@@ -179,25 +192,26 @@ __global__ void __launch_bounds__(32 * K) wgrad_dw_kernel(DwgParams p) {
     const int R = min(p.band, p.Ho - oh0);
     __syncthreads();  // the previous band's readers are done
     const int xrows = R + K - 1;
+    // asynchronous 16-byte copies (all in flight at once), zero-filled outside
+    // the image and past the last channel
     for (int e = tid; e < xrows * Wp * 4; e += 32 * K) {
       const int v = e & 3, pix = e >> 2;
       const int r = pix / Wp, col = pix - r * Wp;
       const int ih = oh0 + r - p.pad, iw = col - p.pad, c = c0 + v * 8;
-      uint4 q = make_uint4(0u, 0u, 0u, 0u);
-      if (ih >= 0 && ih < p.H && iw >= 0 && iw < p.W && c < p.C)
-        q = *reinterpret_cast<const uint4*>(
-            p.x + ((static_cast<size_t>(b) * p.H + ih) * p.W + iw) * p.C + c);
-      *reinterpret_cast<uint4*>(xs + static_cast<size_t>(pix) * kDwgChunk + v * 8) = q;
+      const bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W && c < p.C;
+      const __nv_bfloat16* src =
+          ok ? p.x + ((static_cast<size_t>(b) * p.H + ih) * p.W + iw) * p.C + c : p.x;
+      cp_async_16(dc::smem_u32(xs + static_cast<size_t>(pix) * kDwgChunk + v * 8), src, ok);
     }
     for (int e = tid; e < R * p.Wo * 4; e += 32 * K) {
       const int v = e & 3, pix = e >> 2;
       const int r = pix / p.Wo, ow = pix - r * p.Wo, c = c0 + v * 8;
-      uint4 q = make_uint4(0u, 0u, 0u, 0u);
-      if (c < p.C)
-        q = *reinterpret_cast<const uint4*>(
-            p.dy + ((static_cast<size_t>(b) * p.Ho + oh0 + r) * p.Wo + ow) * p.C + c);
-      *reinterpret_cast<uint4*>(ds + static_cast<size_t>(pix) * kDwgChunk + v * 8) = q;
+      const bool ok = c < p.C;
+      const __nv_bfloat16* src =
+          ok ? p.dy + ((static_cast<size_t>(b) * p.Ho + oh0 + r) * p.Wo + ow) * p.C + c : p.dy;
+      cp_async_16(dc::smem_u32(ds + static_cast<size_t>(pix) * kDwgChunk + v * 8), src, ok);
     }
+    cp_async_wait_all();
     __syncthreads();
     for (int r = 0; r < R; ++r) {
       // x row r + kh of the band, halo column q holds input column q - pad
@@ -242,8 +256,10 @@ struct MgParams {
   const float* dW;       // [B][wsize] per-sample weight gradients
   const void* experts;   // [n][wsize], T
   const float* alpha;    // [B][n]
-  float* dexperts;       // [n][wsize]
+  float* dexperts;       // [n][wsize], or with bsplit > 1 partials [bsplit][n][wsize]
   float* part;           // [chunks][B][n]: sum over this chunk of dW[b][w] * E[i][w]
+  int bsplit;            // sample groups (grid.z), each of bs samples
+  int bs;
 };
 
 // dexperts[i][w] = sum_b alpha[b][i] dW[b][w] for the CTA's 1024 weights and
@@ -282,8 +298,9 @@ __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
     for (int k = 0; k < 4; ++k) dex[i][k] = 0.f;
   __syncthreads();
 
-  for (int b0 = 0; b0 < p.B; b0 += kMgSampleBlock) {
-    const int nbb = min(kMgSampleBlock, p.B - b0);
+  const int b_begin = blockIdx.z * p.bs, b_end = min(p.B, b_begin + p.bs);
+  for (int b0 = b_begin; b0 < b_end; b0 += kMgSampleBlock) {
+    const int nbb = min(kMgSampleBlock, b_end - b0);
     // eight samples per round: their loads are all in flight before the math
     for (int bb0 = 0; bb0 < nbb; bb0 += 8) {
       float v[8][4];
@@ -333,7 +350,7 @@ __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
 #pragma unroll
   for (int i = 0; i < NE; ++i) {
     if (i < ne) {
-      float* dst = p.dexperts + static_cast<size_t>(i0 + i) * p.wsize + w;
+      float* dst = p.dexperts + (static_cast<size_t>(blockIdx.z) * p.n + i0 + i) * p.wsize + w;
       if (p.vec && w < p.wsize) {
         *reinterpret_cast<float4*>(dst) = make_float4(dex[i][0], dex[i][1], dex[i][2], dex[i][3]);
       } else {
@@ -342,6 +359,24 @@ __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
           if (w + k < p.wsize) dst[k] = dex[i][k];
       }
     }
+  }
+}
+
+// dexperts[e] = sum over sample groups, in order, of part[g][e] (e over
+// n * wsize), four elements per thread.
+__global__ void __launch_bounds__(kBwThreads)
+    dexperts_finish_kernel(long long total, int groups, const float* __restrict__ part,
+                           float* __restrict__ dexperts) {
+  for (long long e = (static_cast<long long>(blockIdx.x) * kBwThreads + threadIdx.x) * 4; e < total;
+       e += static_cast<long long>(gridDim.x) * kBwThreads * 4) {
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int g = 0; g < groups; ++g)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (e + k < total) s[k] += part[static_cast<size_t>(g) * total + e + k];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (e + k < total) dexperts[e + k] = s[k];
   }
 }
 

@@ -160,6 +160,9 @@ OTHER = [
     LC("bw_c16out", synth.BF16, 2, 64, 16, 9, 9, 3, 3, 1, 1, 1, 20, synth.SOFTMAX, 1.0),
     # grouped, stride 1: tiled expert transposition with groups, CUDA-core forward
     LC("bw_g4", synth.BF16, 2, 64, 64, 8, 8, 3, 3, 1, 1, 4, 3, synth.SIGMOID, 1.0),
+    # 16 samples: the mixing gradient splits the samples into groups (partial
+    # dexperts added in order)
+    LC("bw_b16", synth.BF16, 16, 64, 64, 6, 6, 3, 3, 1, 1, 1, 3, synth.SOFTMAX, 1.0),
     # 12 input channels: rows not a 16-byte multiple (unvectorised sums and adds)
     LC("bw_c12", synth.BF16, 2, 12, 16, 6, 6, 3, 3, 1, 1, 1, 2, synth.SIGMOID, 1.0),
 ]
