@@ -378,7 +378,8 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
   // experts per CTA: every sample's dW is read ceil(n / ne) times
   const int ne = d->n > 4 ? 8 : d->n > 2 ? 4 : d->n;
   const size_t mg_smem = sizeof(float) * (static_cast<size_t>(d->B) * ne +
-                                          (dcb::kBwThreads / 32) * dcb::kMgSampleBlock * ne);
+                                          (dcb::kBwThreads / 32) * dcb::kMgSampleBlock * ne +
+                                          (dcb::kBwThreads / 32) * 32 * 33);
   if (mg_smem > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
   rc = d->dtype == DYNCONV_F32 ? launch_mixgrad<float>(mp, ne, mg_smem, s)
                                : launch_mixgrad<__nv_bfloat16>(mp, ne, mg_smem, s);

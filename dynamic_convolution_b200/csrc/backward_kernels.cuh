@@ -263,17 +263,23 @@ struct MgParams {
 };
 
 // dexperts[i][w] = sum_b alpha[b][i] dW[b][w] for the CTA's 1024 weights and
-// NE experts (fewer in the last group), and the chunk's share of
-// dalpha[b][i] = <dW_b, E_i>. Each thread holds four weights: per sample one
-// 16-byte load of dW, eight multiply-adds per expert and a warp reduction per
-// expert of the dot product; the warps' sums meet in shared memory and are
-// added in warp order.
+// NE experts (fewer in the last group), over the CTA's group of samples, and
+// the chunk's share of dalpha[b][i] = <dW_b, E_i>. Each thread holds four
+// weights: per sample one 16-byte load of dW (eight samples' loads in flight),
+// four multiply-adds per expert into dexperts and four into the dot product.
+// The dot products of SU samples x NE experts (32 values per lane) are summed
+// over the warp by a transpose through shared memory: lane l writes its values
+// as row l of a 32 x 33 tile, lane j adds column j in row order. The warps'
+// sums meet in shared memory and are added in warp order.
 template <typename T, int NE>
 __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
+  constexpr int SU = (32 / NE) < 8 ? (32 / NE) : 8;  // samples per reduction
   extern __shared__ float mg_smem[];
   float* alpha_s = mg_smem;                                          // [B][NE]
-  float* red = mg_smem + static_cast<size_t>(p.B) * NE;              // [8][32][NE]
+  float* red = alpha_s + static_cast<size_t>(p.B) * NE;              // [8][32][NE]
+  float* tiles = red + (kBwThreads / 32) * kMgSampleBlock * NE;      // [8][32][33]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* tl = tiles + warp * (32 * 33);
   const int chunk = blockIdx.x;
   const int i0 = blockIdx.y * NE;
   const int ne = min(NE, p.n - i0);
@@ -301,8 +307,8 @@ __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
   const int b_begin = blockIdx.z * p.bs, b_end = min(p.B, b_begin + p.bs);
   for (int b0 = b_begin; b0 < b_end; b0 += kMgSampleBlock) {
     const int nbb = min(kMgSampleBlock, b_end - b0);
-    // eight samples per round: their loads are all in flight before the math
     for (int bb0 = 0; bb0 < nbb; bb0 += 8) {
+      // eight samples' loads in flight before the math
       float v[8][4];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -319,23 +325,33 @@ __global__ void __launch_bounds__(kBwThreads) mixgrad_kernel(MgParams p) {
         }
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int bb = bb0 + u;
-        if (bb >= nbb) break;  // the same for every thread of the CTA
-        const float* ab = alpha_s + static_cast<size_t>(b0 + bb) * NE;
+      for (int h = 0; h < 8; h += SU) {
 #pragma unroll
-        for (int i = 0; i < NE; ++i) {
-          const float a = ab[i];
-          float d = 0.f;
+        for (int u = 0; u < SU; ++u) {
+          // samples past the group have v = 0 and alpha rows that are not read
+          const int bq = min(b0 + bb0 + h + u, p.B - 1);
+          const float* ab = alpha_s + static_cast<size_t>(bq) * NE;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            dex[i][k] = fmaf(a, v[u][k], dex[i][k]);
-            d = fmaf(v[u][k], ev[i][k], d);
+          for (int i = 0; i < NE; ++i) {
+            const float a = ab[i];
+            float d = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              dex[i][k] = fmaf(a, v[h + u][k], dex[i][k]);
+              d = fmaf(v[h + u][k], ev[i][k], d);
+            }
+            tl[lane * 33 + u * NE + i] = d;
           }
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-          if (lane == 0) red[(warp * kMgSampleBlock + bb) * NE + i] = d;
         }
+        __syncwarp();
+        if (lane < SU * NE) {
+          float sum = 0.f;
+#pragma unroll 8
+          for (int l = 0; l < 32; ++l) sum += tl[l * 33 + lane];
+          const int bb = bb0 + h + lane / NE;
+          if (bb < nbb) red[(warp * kMgSampleBlock + bb) * NE + lane % NE] = sum;
+        }
+        __syncwarp();
       }
     }
     __syncthreads();
@@ -481,6 +497,7 @@ __global__ void __launch_bounds__(kBwThreads)
   const int c = blockIdx.x * kBwThreads + threadIdx.x;
   if (c < C) {
     float s = 0.f;
+#pragma unroll 8
     for (int b = 0; b < B; ++b) s = fmaf(dz_s[b], gsum[static_cast<size_t>(b) * C + c], s);
     dWr[static_cast<size_t>(i) * C + c] = s * inv_hw;
   }
