@@ -76,6 +76,12 @@ def configure(lib):
     lib.oracle_dexperts_at.restype = i
     lib.oracle_dbias.argtypes = [i, i, i, i, dp, dp, dp]
     lib.oracle_dbias.restype = i
+    lib.oracle_assemble_cells.argtypes = [i, i, ctypes.c_long, dp, dp, dp]
+    lib.oracle_assemble_cells.restype = None
+    lib.oracle_route_cells.argtypes = [i, i, i, i, dp, i, i, dp, dp, i, ctypes.c_double, dp]
+    lib.oracle_route_cells.restype = i
+    lib.oracle_forward_cells.argtypes = [i] * 12 + [dp, dp, dp, dp, i, i, dp]
+    lib.oracle_forward_cells.restype = i
     return lib
 
 
@@ -359,3 +365,60 @@ def dbias(dy, alpha):
     if rc != 0:
         raise ValueError(f"oracle_dbias rejected its arguments (rc={rc})")
     return out
+
+
+# ------------------------------------------------------------- kernel cells
+
+
+def route_cells(x, Wr, br, m: int, mode: int, tau: float = 1.0):
+    """alpha[B][m][n]: the router with m*n outputs (Wr[m*n][C], br[m*n] or None),
+    its activation taken per cell of n values."""
+    x = _f64(x)
+    Wr = _f64(Wr)
+    br = _f64(br)
+    B, H, W, C = x.shape
+    assert Wr.shape[0] % m == 0 and Wr.shape[1] == C
+    n = Wr.shape[0] // m
+    alpha = np.empty((B, m, n), dtype=np.float64)
+    rc = _load().oracle_route_cells(B, C, H, W, _dp(x), m, n, _dp(Wr), _dp(br), int(mode),
+                                    float(tau), _dp(alpha))
+    if rc != 0:
+        raise ValueError(f"oracle_route_cells rejected its arguments (rc={rc})")
+    return alpha
+
+
+def assemble_cells(warehouse, alpha_b):
+    """W_b (flat, m*s elements) from warehouse[n][s] and alpha_b[m][n]."""
+    warehouse = _f64(warehouse)
+    alpha_b = _f64(alpha_b)
+    n, s = warehouse.shape
+    m = alpha_b.shape[0]
+    assert alpha_b.shape == (m, n)
+    out = np.empty(m * s, dtype=np.float64)
+    _load().oracle_assemble_cells(m, n, s, _dp(warehouse), _dp(alpha_b), _dp(out))
+    return out
+
+
+def forward_cells(x, warehouse, alpha, bias, Cout: int, KH: int, KW: int, stride: int = 1,
+                  pad: int = 0, groups: int = 1, samples: tuple[int, int] | None = None):
+    """y with the kernel assembled from cells: warehouse[n][s], alpha[B][m][n],
+    bias[C_out] static (or None); the layer's kernel has m*s elements."""
+    x = _f64(x)
+    warehouse = _f64(warehouse)
+    alpha = _f64(alpha)
+    bias = _f64(bias)
+    B, H, W, Cin = x.shape
+    n, s = warehouse.shape
+    m = alpha.shape[1]
+    assert alpha.shape == (B, m, n) and m * s == Cout * KH * KW * (Cin // groups)
+    assert bias is None or bias.shape == (Cout,)
+    b0, nb = (0, B) if samples is None else samples
+    Ho = (H + 2 * pad - KH) // stride + 1
+    Wo = (W + 2 * pad - KW) // stride + 1
+    y = np.empty((nb, Ho, Wo, Cout), dtype=np.float64)
+    rc = _load().oracle_forward_cells(B, Cin, H, W, Cout, KH, KW, stride, pad, groups, m, n,
+                                      _dp(x), _dp(warehouse), _dp(alpha), _dp(bias), b0, nb,
+                                      _dp(y))
+    if rc != 0:
+        raise ValueError(f"oracle_forward_cells rejected its arguments (rc={rc})")
+    return y

@@ -611,3 +611,80 @@ int oracle_dbias(int B, int HoWo, int Cout, int n, const double *dy, const doubl
   free(db);
   return 0;
 }
+
+/* =========================================================== kernel cells */
+/*
+ * Kernel cells shared through a warehouse (KernelWarehouse: Rethinking the
+ * Design of Dynamic Convolution, abstract: the page redefines the kernel, its
+ * assembly and the attention function so that n can exceed 100, by sharing
+ * parameters within a layer and across neighbouring layers; it gives no
+ * formula). Reading taken: the layer's kernel, flattened in the layout
+ * [C_out][KH][KW][C_in/groups], is split into m contiguous cells of s
+ * elements; a warehouse holds n cells E[n][s] (one warehouse may serve several
+ * layers); every kernel cell j of sample b is its own mixture
+ *     W_b[j*s + e] = sum_i alpha[b][j][i] * E[i][e],
+ * with the attentions from the same router (average pool, one linear layer
+ * with m*n outputs) normalised per cell: softmax over the n values of each
+ * cell (z / tau), or an elementwise sigmoid. With m = 1 this is the ordinary
+ * mixture of n kernels.
+ */
+
+/* W_b of one sample from its cell attentions alpha_b[m][n]. */
+void oracle_assemble_cells(int m, int n, long s, const double *warehouse,
+                           const double *alpha_b, double *Wb) {
+  for (int j = 0; j < m; ++j)
+    for (long e = 0; e < s; ++e) {
+      double acc = 0.0;
+      for (int i = 0; i < n; ++i) acc += alpha_b[(size_t)j * n + i] * warehouse[(size_t)i * s + e];
+      Wb[(size_t)j * s + e] = acc;
+    }
+}
+
+/* alpha[B][m][n]: the router with m*n outputs, its activation taken per cell. */
+int oracle_route_cells(int B, int C, int H, int W, const double *x, int m, int n,
+                       const double *Wr, const double *br, int mode, double tau, double *alpha) {
+  if (B < 0 || C <= 0 || H <= 0 || W <= 0 || m <= 0 || n <= 0 || !x || !Wr || !alpha) return -1;
+  if (mode != ORACLE_SIGMOID && mode != ORACLE_SOFTMAX) return -1;
+  if (mode == ORACLE_SOFTMAX && !(tau > 0.0)) return -1;
+  double *g = (double *)malloc(sizeof(double) * (size_t)C);
+  double *z = (double *)malloc(sizeof(double) * (size_t)m * n);
+  if (!g || !z) { free(g); free(z); return -1; }
+  for (int b = 0; b < B; ++b) {
+    oracle_gap(C, H, W, x + (size_t)b * H * W * C, g);
+    oracle_fc(C, m * n, Wr, br, g, z);
+    for (int j = 0; j < m; ++j)
+      oracle_act(n, z + (size_t)j * n, mode, tau, alpha + ((size_t)b * m + j) * n);
+  }
+  free(g);
+  free(z);
+  return 0;
+}
+
+/* y of samples b0 .. b0+nb-1 with the kernel assembled from cells, plus an
+ * optional static bias[C_out] (not mixed): the convolution is oracle_forward
+ * of one sample with W_b as its only expert and attention 1. */
+int oracle_forward_cells(int B, int Cin, int H, int W, int Cout, int KH, int KW, int stride,
+                         int pad, int groups, int m, int n, const double *x,
+                         const double *warehouse, const double *alpha, const double *bias,
+                         int b0, int nb, double *y) {
+  if (B < 0 || Cin <= 0 || H <= 0 || W <= 0 || Cout <= 0 || KH <= 0 || KW <= 0) return -1;
+  if (m <= 0 || n <= 0 || groups <= 0 || Cin % groups || Cout % groups) return -1;
+  if (!x || !warehouse || !alpha || !y || b0 < 0 || nb < 0 || b0 + nb > B) return -1;
+  const long wsize = (long)Cout * KH * KW * (Cin / groups);
+  if (wsize % m != 0) return -1;
+  const long s = wsize / m;
+  const int Ho = oracle_out_size(H, KH, stride, pad), Wo = oracle_out_size(W, KW, stride, pad);
+  if (Ho <= 0 || Wo <= 0) return -1;
+  double *Wb = (double *)malloc(sizeof(double) * (size_t)wsize);
+  if (!Wb) return -1;
+  const double one = 1.0;
+  int rc = 0;
+  for (int b = b0; b < b0 + nb && rc == 0; ++b) {
+    oracle_assemble_cells(m, n, s, warehouse, alpha + (size_t)b * m * n, Wb);
+    rc = oracle_forward(1, Cin, H, W, Cout, KH, KW, stride, pad, groups, 1,
+                        x + (size_t)b * H * W * Cin, Wb, &one, bias, 0, 1,
+                        y + (size_t)(b - b0) * Ho * Wo * Cout, 1);
+  }
+  free(Wb);
+  return rc;
+}

@@ -10,6 +10,7 @@ import pytest
 import oracle
 
 from . import test_oracle_backward as bw
+from . import test_oracle_cells as cells
 from . import test_oracle_pins as pins
 
 # (name, original text, mutated text) -- each replacement must hit exactly once
@@ -66,6 +67,12 @@ MUTANTS = [
      "for (int c = 0; c < C; ++c) dWr[(size_t)i * C + c] += da[i] * g[c];"),
     ("pool_grad_wrong_router_row", "for (int i = 0; i < n; ++i) s += dz[i] * Wr[(size_t)i * C + c];",
      "for (int i = 0; i < n; ++i) s += dz[i] * Wr[(size_t)(n - 1 - i) * C + c];"),
+    # kernel cells
+    ("cells_share_first_cells_attention", "acc += alpha_b[(size_t)j * n + i] * warehouse[(size_t)i * s + e];",
+     "acc += alpha_b[i] * warehouse[(size_t)i * s + e];"),
+    ("cells_written_over_each_other", "Wb[(size_t)j * s + e] = acc;", "Wb[e] = acc;"),
+    ("cells_activation_on_first_block", "oracle_act(n, z + (size_t)j * n, mode, tau,",
+     "oracle_act(n, z, mode, tau,"),
 ]
 
 PIN_TESTS = [
@@ -87,6 +94,11 @@ PIN_TESTS = [
     bw.test_softmax_router_gradients_sum_to_zero_over_experts,
     bw.test_zero_input_leaves_bias_terms,
     bw.test_pooled_gradient_adds_a_constant_per_channel,
+    # kernel cells
+    lambda: [cells.test_one_hot_attentions_pick_whole_cells(sh) for sh in cells.SHAPES],
+    lambda: [cells.test_cell_routing_is_the_routing_per_cell(m, t)
+             for m, t in [(0, 1.0), (1, 1.0), (1, 3.0)]],
+    cells.test_a_cell_changes_only_its_output_channels,
 ]
 
 
