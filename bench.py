@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="time the layer's backward step (weight, router and input gradients)")
+    ap.add_argument("--cells", type=int, default=0,
+                    help="time the layer with its kernel assembled from this many warehouse cells")
+    ap.add_argument("--warehouse", type=int, default=128, help="warehouse cells for --cells")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--hooks", default="",
                     help="implementation knobs for comparisons, e.g. '6=0,5=0' "
@@ -746,6 +749,82 @@ def run_backward(args, cfg):
     return 0
 
 
+def run_cells(args, cfg):
+    """The layer with its kernel assembled from warehouse cells, one GPU: step =
+    dynconv_route_cells + dynconv_forward_cells of one batch, CUDA graphs of 8
+    steps, inputs rotated over sets larger than L2 in total."""
+    import torch
+
+    import dynamic_convolution_b200 as dc
+    from dynamic_convolution_b200 import build, synth
+
+    torch.cuda.set_device(0)
+    build.build()
+    dc.load()
+    cells, n = args.cells, args.warehouse
+    ci = synth.make_cell_inputs(cfg, cells, n)
+    dev = lambda a: (torch.from_numpy(a).view(torch.bfloat16) if cfg.dtype == synth.BF16
+                     else torch.from_numpy(a)).cuda()
+    x0, E = dev(ci.x_store), dev(ci.warehouse_store)
+    Wr, br, bias = (torch.from_numpy(a).cuda() for a in (ci.Wr, ci.br, ci.bias))
+    d = dc.make_desc(cfg.B, cfg.C_in, cfg.H, cfg.W, cfg.C_out, cfg.KH, cfg.KW, cfg.stride,
+                     cfg.pad, cfg.groups, n, cfg.dtype)
+    wsb = dc.dynconv_cells_workspace_size(d, cells)
+    if wsb == 0:
+        raise SystemExit(f"{cfg.name}: {cells} cells do not divide the kernel into 16-byte cells")
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    tdt = torch.bfloat16 if cfg.dtype == synth.BF16 else torch.float32
+    set_bytes = x0.numel() * x0.element_size() + cfg.B * cfg.H_out * cfg.W_out * cfg.C_out * 2
+    nsets = max(2, min(64, math.ceil(2 * L2_BYTES / set_bytes)))
+    xs = [x0.clone() for _ in range(nsets)]
+    ys = [torch.empty((cfg.B, cfg.H_out, cfg.W_out, cfg.C_out), dtype=tdt, device="cuda")
+          for _ in range(nsets)]
+    alphas = [torch.empty((cfg.B, cells, n), device="cuda") for _ in range(nsets)]
+    stream = torch.cuda.Stream()
+
+    def step(k, st):
+        dc.check(dc.dynconv_route_cells(d, cells, xs[k], Wr, br, cfg.mode, cfg.tau, alphas[k], st))
+        dc.check(dc.dynconv_forward_cells(d, cells, xs[k], E, alphas[k], bias, ys[k], ws, wsb, st))
+
+    with torch.cuda.stream(stream):
+        for k in range(max(args.warmup, 3)):
+            step(k % nsets, stream)
+    stream.synchronize()
+    per = min(8, nsets)
+    g = torch.cuda.CUDAGraph()
+    n0 = dc.dynconv_launch_count()
+    with torch.cuda.graph(g, stream=stream):
+        for k in range(per):
+            step(k, stream)
+    launches = (dc.dynconv_launch_count() - n0) // per
+    reps = max(1, args.steps // per)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    dc.check(dc.dynconv_device_status(stream), "device status")
+    ms = e0.elapsed_time(e1) / (reps * per)
+    del g
+    mix_flops = 2.0 * cfg.B * cfg.C_out * cfg.KH * cfg.KW * cfg.Cg * n
+    line = {"metric": "images/s (warehouse cells: route + forward)",
+            "value": cfg.B / (ms / 1e3), "unit": "images/s", "n_gpus": 1, "steps": reps * per,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32",
+            "data": "synthetic (seeded; recipe in DESIGN.md)",
+            "config": {"workload": f"{cfg.name} from {cells} cells, warehouse of {n} cells",
+                       "l2": f"inputs rotated over {nsets} sets"},
+            "conv_tflops": cfg.conv_flops / (ms / 1e3) / 1e12,
+            "mixing_gflop": mix_flops / 1e9, "gpu_launches_per_step": launches}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     from dynamic_convolution_b200 import synth
@@ -753,6 +832,8 @@ def main():
         return run_block(args)
     if args.backward:
         return run_backward(args, synth.CONFIGS[args.config or synth.HEADLINE])
+    if args.cells:
+        return run_cells(args, synth.CONFIGS[args.config or synth.HEADLINE])
     name = args.config or synth.HEADLINE
     cfg = synth.CONFIGS[name]
     if args.impl == "reference":

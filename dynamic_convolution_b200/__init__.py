@@ -1,5 +1,5 @@
 """Python binding of the sm_100a dynamic-convolution C ABI (``include/dynconv.h``,
-``include/dynconv_backward.h``).
+``include/dynconv_backward.h``, ``include/dynconv_cells.h``).
 
 Argument marshalling only: every function forwards to the symbol of the same
 name in ``libdynconv.so``; all arithmetic runs in the library's CUDA kernels.
@@ -33,7 +33,9 @@ SYMBOLS = ("dynconv_route", "dynconv_forward", "dynconv_forward_noalloc",
            "dynconv_launch_count", "dynconv_test_hook",
            # include/dynconv_backward.h
            "dynconv_backward_workspace_size", "dynconv_backward_weight",
-           "dynconv_route_backward", "dynconv_backward_data")
+           "dynconv_route_backward", "dynconv_backward_data",
+           # include/dynconv_cells.h
+           "dynconv_route_cells", "dynconv_cells_workspace_size", "dynconv_forward_cells")
 
 
 class dynconv_desc(ctypes.Structure):
@@ -101,6 +103,13 @@ def load():
         lib.dynconv_route_backward.restype = ctypes.c_int
         lib.dynconv_backward_data.argtypes = [D, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.dynconv_backward_data.restype = ctypes.c_int
+        lib.dynconv_route_cells.argtypes = [D, ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_float,
+                                            P, P]
+        lib.dynconv_route_cells.restype = ctypes.c_int
+        lib.dynconv_cells_workspace_size.argtypes = [D, ctypes.c_int]
+        lib.dynconv_cells_workspace_size.restype = ctypes.c_size_t
+        lib.dynconv_forward_cells.argtypes = [D, ctypes.c_int, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.dynconv_forward_cells.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -255,4 +264,26 @@ def dynconv_backward_data(desc, dy, experts, alpha, dg, dx, workspace, workspace
     """dx [B][H][W][C_in] in the layer's dtype; dg [B][C_in] or None."""
     return load().dynconv_backward_data(ctypes.byref(desc), _ptr(dy), _ptr(experts), _ptr(alpha),
                                         _ptr(dg), _ptr(dx), _ptr(workspace),
+                                        int(workspace_bytes), _stream(stream))
+
+
+# ------------------------------------------------------------- kernel cells
+
+
+def dynconv_route_cells(desc, cells, x, Wr, br, mode, tau, alpha, stream=None) -> int:
+    """alpha [B][cells][n] (fp32) from Wr [cells*n][C_in], br [cells*n] (or None)."""
+    return load().dynconv_route_cells(ctypes.byref(desc), int(cells), _ptr(x), _ptr(Wr), _ptr(br),
+                                      int(mode), float(tau), _ptr(alpha), _stream(stream))
+
+
+def dynconv_cells_workspace_size(desc, cells) -> int:
+    return load().dynconv_cells_workspace_size(ctypes.byref(desc), int(cells))
+
+
+def dynconv_forward_cells(desc, cells, x, warehouse, alpha, bias, y, workspace, workspace_bytes,
+                          stream=None) -> int:
+    """y with the kernel assembled from `cells` cells of the warehouse [n][s];
+    bias [C_out] static (or None)."""
+    return load().dynconv_forward_cells(ctypes.byref(desc), int(cells), _ptr(x), _ptr(warehouse),
+                                        _ptr(alpha), _ptr(bias), _ptr(y), _ptr(workspace),
                                         int(workspace_bytes), _stream(stream))

@@ -1,9 +1,10 @@
 """Build the sm_100a C-ABI library ``libdynconv.so`` in-tree with nvcc.
 
 Usage: ``python -m dynamic_convolution_b200.build`` (or ``build()`` from Python).
-The library has two translation units: ``csrc/dynconv.cu`` (the forward
-entry points; it includes the forward kernel headers) and ``csrc/backward.cu``
-(the backward entry points and kernels); it links the CUDA runtime statically and reaches the driver's
+The library has three translation units: ``csrc/dynconv.cu`` (the forward
+entry points; it includes the forward kernel headers), ``csrc/backward.cu``
+(the backward entry points and kernels) and ``csrc/cells.cu`` (warehouse
+cells); it links the CUDA runtime statically and reaches the driver's
 tensor-map encoder through the runtime's entry-point query, so it loads on a
 machine without a GPU driver (the calls then fail with DYNCONV_ERR_CUDA).
 """
@@ -20,7 +21,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdynconv.so")
-UNITS = [os.path.join(CSRC, "dynconv.cu"), os.path.join(CSRC, "backward.cu")]
+UNITS = [os.path.join(CSRC, "dynconv.cu"), os.path.join(CSRC, "backward.cu"),
+         os.path.join(CSRC, "cells.cu")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -39,7 +41,7 @@ def _nvcc() -> str:
 
 def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + [os.path.join(INCLUDE, "dynconv.h")])
+                  + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def is_stale() -> bool:

@@ -168,3 +168,32 @@ def make_upstream_grad(cfg: LayerConfig, seed: int = 1):
     the layer dtype: (device storage, the same values as float64)."""
     rng = np.random.default_rng(seed)
     return _round(rng.standard_normal((cfg.B, cfg.H_out, cfg.W_out, cfg.C_out)), cfg.dtype)
+
+
+@dataclasses.dataclass
+class CellInputs:
+    """Host arrays of one layer built from warehouse cells: the layer's x (as
+    make_inputs draws it), a warehouse of n cells of s elements each drawn like
+    one expert's elements, the router of cells * n outputs and a static bias."""
+    x_store: np.ndarray
+    x_f64: np.ndarray
+    warehouse_store: np.ndarray   # [n][s]
+    warehouse_f64: np.ndarray
+    Wr: np.ndarray                # float32 [cells * n][C_in]
+    br: np.ndarray                # float32 [cells * n]
+    bias: np.ndarray              # float32 [C_out]
+
+
+def make_cell_inputs(cfg: LayerConfig, cells: int, n: int, seed: int = 0,
+                     structured: float = 0.0) -> CellInputs:
+    base = make_inputs(cfg, seed=seed, structured=structured)
+    rng = np.random.default_rng(seed + 1000)
+    wsize = cfg.C_out * cfg.KH * cfg.KW * cfg.Cg
+    assert wsize % cells == 0
+    std = math.sqrt(2.0 / (cfg.Cg * cfg.KH * cfg.KW)) * cfg.expert_scale
+    ws, wf = _round(rng.standard_normal((n, wsize // cells)) * std, cfg.dtype)
+    Wr = rng.standard_normal((cells * n, cfg.C_in)) * math.sqrt(1.0 / cfg.C_in)
+    br = rng.standard_normal(cells * n) * 0.1
+    bias = rng.standard_normal(cfg.C_out) * 0.1
+    return CellInputs(base.x_store, base.x_f64, ws, wf, Wr.astype(np.float32),
+                      br.astype(np.float32), bias.astype(np.float32))

@@ -14,7 +14,7 @@ from dynamic_convolution_b200 import build as dcbuild
 from dynamic_convolution_b200 import synth
 
 HEADERS = [os.path.join(dcbuild.ROOT, "include", h)
-           for h in ("dynconv.h", "dynconv_backward.h")]
+           for h in ("dynconv.h", "dynconv_backward.h", "dynconv_cells.h")]
 
 
 @pytest.fixture(scope="module")
@@ -188,3 +188,30 @@ def test_backward_entry_points_host_side(lib):
     # shapes off the transposed path take the CUDA-core kernel and need no workspace
     assert bd(s2, P, P, P, None, P, None, 0) == dc.ERR_CUDA
     assert dc.dynconv_last_error() != ""
+
+
+def test_cells_entry_points_host_side(lib):
+    """Shapes the cell path takes, its workspace, argument checks, and the loud
+    failure with no device."""
+    cfg = synth.CONFIGS["resnet18_3x3"]
+    d = dc.make_desc(cfg.B, cfg.C_in, cfg.H, cfg.W, cfg.C_out, 3, 3, 1, 1, 1, 128, cfg.dtype)
+    wsize = cfg.C_out * 9 * cfg.C_in
+    need = dc.dynconv_cells_workspace_size(d, 16)
+    assert need >= 2 * cfg.B * wsize                       # every sample's kernel
+    assert dc.dynconv_cells_workspace_size(d, 7) == 0      # cells must divide the kernel
+    assert dc.dynconv_cells_workspace_size(d, wsize // 4) == 0   # cells of 4 elements: not 16 bytes
+    big = dc.make_desc(cfg.B, cfg.C_in, cfg.H, cfg.W, cfg.C_out, 3, 3, 1, 1, 1, 2048, cfg.dtype)
+    assert dc.dynconv_cells_workspace_size(big, 16) == 0   # warehouse above 1024 cells
+    P = 256
+    fc = dc.dynconv_forward_cells
+    assert fc(d, 0, P, P, P, None, P, P, need) == dc.ERR_INVALID_ARG
+    assert fc(d, 16, None, P, P, None, P, P, need) == dc.ERR_INVALID_ARG
+    assert fc(d, 7, P, P, P, None, P, P, need) == dc.ERR_UNSUPPORTED
+    assert fc(d, 16, P, P, P, None, P, P, need - 256) == dc.ERR_WORKSPACE
+    assert fc(d, 16, P, P + 2, P, None, P, P, need) == dc.ERR_MISALIGNED
+    assert fc(d, 16, P, P, P, None, P, P, need) == dc.ERR_CUDA
+    rc = dc.dynconv_route_cells
+    assert rc(d, 16, P, P, None, 2, 1.0, P) == dc.ERR_INVALID_ARG
+    assert rc(d, 16, P, P, None, dc.SOFTMAX, 0.0, P) == dc.ERR_INVALID_ARG
+    assert rc(d, 64, P, P, None, dc.SOFTMAX, 1.0, P) == dc.ERR_UNSUPPORTED   # 64 * 128 logits
+    assert rc(d, 16, P, P, None, dc.SOFTMAX, 1.0, P) == dc.ERR_CUDA
