@@ -783,7 +783,8 @@ def run_cells(args, cfg):
     stream = torch.cuda.Stream()
 
     def step(k, st):
-        dc.check(dc.dynconv_route_cells(d, cells, xs[k], Wr, br, cfg.mode, cfg.tau, alphas[k], st))
+        dc.check(dc.dynconv_route_cells(d, cells, xs[k], Wr, br, cfg.mode, cfg.tau, alphas[k],
+                                        ws, wsb, st))
         dc.check(dc.dynconv_forward_cells(d, cells, xs[k], E, alphas[k], bias, ys[k], ws, wsb, st))
 
     with torch.cuda.stream(stream):

@@ -104,7 +104,7 @@ def load():
         lib.dynconv_backward_data.argtypes = [D, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.dynconv_backward_data.restype = ctypes.c_int
         lib.dynconv_route_cells.argtypes = [D, ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_float,
-                                            P, P]
+                                            P, P, ctypes.c_size_t, P]
         lib.dynconv_route_cells.restype = ctypes.c_int
         lib.dynconv_cells_workspace_size.argtypes = [D, ctypes.c_int]
         lib.dynconv_cells_workspace_size.restype = ctypes.c_size_t
@@ -270,10 +270,12 @@ def dynconv_backward_data(desc, dy, experts, alpha, dg, dx, workspace, workspace
 # ------------------------------------------------------------- kernel cells
 
 
-def dynconv_route_cells(desc, cells, x, Wr, br, mode, tau, alpha, stream=None) -> int:
+def dynconv_route_cells(desc, cells, x, Wr, br, mode, tau, alpha, workspace, workspace_bytes,
+                        stream=None) -> int:
     """alpha [B][cells][n] (fp32) from Wr [cells*n][C_in], br [cells*n] (or None)."""
     return load().dynconv_route_cells(ctypes.byref(desc), int(cells), _ptr(x), _ptr(Wr), _ptr(br),
-                                      int(mode), float(tau), _ptr(alpha), _stream(stream))
+                                      int(mode), float(tau), _ptr(alpha), _ptr(workspace),
+                                      int(workspace_bytes), _stream(stream))
 
 
 def dynconv_cells_workspace_size(desc, cells) -> int:

@@ -58,6 +58,16 @@ int conv_variant(const dynconv_desc* d) {
   return depthwise_shape(d) ? DYNCONV_VARIANT_DEPTHWISE : DYNCONV_VARIANT_DIRECT;
 }
 
+// Pixel slices of the routing's average pool: about four CTAs per SM in all
+// (for at most 160 SMs), at least 32 pixels per slice.
+int pool_slices(int B, int HW) {
+  const int want = std::max(1, (4 * 160 + B - 1) / std::max(B, 1));
+  return std::max(1, std::min(want, HW / 32));
+}
+size_t pool_bytes(const dynconv_desc* d) {
+  return align256(4ull * d->B * d->C_in * pool_slices(d->B, d->H * d->W));
+}
+
 struct CellsLayout {
   size_t wb = 0, ident = 0, ident_tail = 0, bias_rows = 0, conv = 0, total = 0;
 };
@@ -83,7 +93,7 @@ CellsLayout cells_layout(const dynconv_desc* d, int cells) {
     dynconv_desc c = chunk_desc(d, bc, DYNCONV_VARIANT_PREMIX);
     conv = dynconv_workspace_size(&c);
   }
-  L.total = align256(L.conv + conv);
+  L.total = std::max(align256(L.conv + conv), pool_bytes(d));
   (void)cells;
   return L;
 }
@@ -106,7 +116,8 @@ int launch_mix(const dcc::CmParams& p, int vec, size_t smem, cudaStream_t s) {
 extern "C" {
 
 int dynconv_route_cells(const dynconv_desc* desc, int cells, const void* x, const float* Wr,
-                        const float* br, int mode, float tau, float* alpha, void* stream) {
+                        const float* br, int mode, float tau, float* alpha, void* workspace,
+                        size_t workspace_bytes, void* stream) {
   int rc = dc_lib::validate(desc);
   if (rc) return rc;
   if (!x || !Wr || !alpha || cells < 1) return DYNCONV_ERR_INVALID_ARG;
@@ -114,25 +125,35 @@ int dynconv_route_cells(const dynconv_desc* desc, int cells, const void* x, cons
   if (mode == DYNCONV_SOFTMAX && !(tau > 0.f)) return DYNCONV_ERR_INVALID_ARG;
   if (1LL * cells * desc->n > 4096 || desc->C_in > 16384) return DYNCONV_ERR_UNSUPPORTED;
   if (desc->B == 0) return DYNCONV_OK;
+  const int HW = desc->H * desc->W;
+  const int S = pool_slices(desc->B, HW);
+  if (!workspace || workspace_bytes < pool_bytes(desc)) return DYNCONV_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DYNCONV_ERR_MISALIGNED;
   dc_lib::DeviceInfo di;
   rc = dc_lib::device_info(&di);
   if (rc) return rc;
-  const size_t smem = sizeof(float) * (static_cast<size_t>(desc->C_in) + cells * desc->n +
-                                       dcc::kCellThreads);
+  const size_t smem = sizeof(float) * (static_cast<size_t>(desc->C_in) +
+                                       static_cast<size_t>(dcc::kCellsPerCta) * desc->n);
   if (smem > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  auto go = [&](auto kern, const auto* xp) -> int {
-    if (smem > 48 * 1024) {
-      cudaError_t e = dc_lib::set_smem(reinterpret_cast<const void*>(kern), smem);
-      if (e != cudaSuccess) return dc_lib::cuda_error(e, "cudaFuncSetAttribute(route_cells)");
-    }
-    kern<<<desc->B, dcc::kCellThreads, smem, s>>>(desc->C_in, desc->H * desc->W, cells, desc->n,
-                                                   mode, tau, xp, Wr, br, alpha);
-    return dc_lib::launched("route_cells_kernel");
-  };
+  float* part = static_cast<float*>(workspace);
+  const int Ps = (HW + S - 1) / S;
   if (desc->dtype == DYNCONV_F32)
-    return go(dcc::route_cells_kernel<float>, static_cast<const float*>(x));
-  return go(dcc::route_cells_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16*>(x));
+    dcc::cells_pool_kernel<float><<<dim3(S, desc->B), dcc::kCellThreads, 0, s>>>(
+        desc->C_in, HW, Ps, static_cast<const float*>(x), part);
+  else
+    dcc::cells_pool_kernel<__nv_bfloat16><<<dim3(S, desc->B), dcc::kCellThreads, 0, s>>>(
+        desc->C_in, HW, Ps, static_cast<const __nv_bfloat16*>(x), part);
+  rc = dc_lib::launched("cells_pool_kernel");
+  if (rc) return rc;
+  if (smem > 48 * 1024) {
+    cudaError_t e = dc_lib::set_smem(reinterpret_cast<const void*>(dcc::route_cells_kernel), smem);
+    if (e != cudaSuccess) return dc_lib::cuda_error(e, "cudaFuncSetAttribute(route_cells)");
+  }
+  dcc::route_cells_kernel<<<dim3((cells + dcc::kCellsPerCta - 1) / dcc::kCellsPerCta, desc->B),
+                            dcc::kCellThreads, smem, s>>>(desc->C_in, HW, S, cells, desc->n, mode,
+                                                          tau, part, Wr, br, alpha);
+  return dc_lib::launched("route_cells_kernel");
 }
 
 size_t dynconv_cells_workspace_size(const dynconv_desc* desc, int cells) {
@@ -158,7 +179,7 @@ int dynconv_forward_cells(const dynconv_desc* desc, int cells, const void* x,
   dc_lib::DeviceInfo di;
   rc = dc_lib::device_info(&di);
   if (rc) return rc;
-  const size_t mix_smem = sizeof(float) * kMixSamples * static_cast<size_t>(desc->n);
+  const size_t mix_smem = sizeof(float) * kMixSamples * static_cast<size_t>(desc->n);  // [n][SB]
   if (mix_smem > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* wsb = static_cast<char*>(workspace);

@@ -36,16 +36,21 @@
 extern "C" {
 #endif
 
-/* alpha[B][m][n] for m = cells, n = desc->n. One CTA per sample: the average
- * pool (fp32), the linear layer (one warp per output, fixed-order sums), the
- * activation per cell (softmax: the cell's maximum subtracted).
+/* alpha[B][m][n] for m = cells, n = desc->n: the average pool (fp32, pixel
+ * slices summed into the workspace, then added in order), the linear layer
+ * (eight outputs per warp at a time, fixed-order sums) and the activation per
+ * cell (softmax: the cell's maximum subtracted), two cells per CTA.
+ *   workspace, workspace_bytes: at least dynconv_cells_workspace_size(desc,
+ *   cells) bytes, 256-byte aligned (the same buffer as the forward call's).
  * Errors: INVALID_ARG (NULL pointers, cells < 1, bad mode or tau),
- * UNSUPPORTED (m*n > 4096 or C_in > 16384), CUDA. */
+ * UNSUPPORTED (m*n > 4096 or C_in > 16384), WORKSPACE, MISALIGNED, CUDA. */
 int dynconv_route_cells(const dynconv_desc* desc, int cells, const void* x, const float* Wr,
-                        const float* br, int mode, float tau, float* alpha, void* stream);
+                        const float* br, int mode, float tau, float* alpha, void* workspace,
+                        size_t workspace_bytes, void* stream);
 
-/* Workspace bytes of dynconv_forward_cells for this descriptor and cell count
- * (0 if the shape is not taken). Pure host function. */
+/* Workspace bytes of dynconv_route_cells and dynconv_forward_cells for this
+ * descriptor and cell count (one buffer serves both; 0 if the shape is not
+ * taken). Pure host function. */
 size_t dynconv_cells_workspace_size(const dynconv_desc* desc, int cells);
 
 /* y for the layer in `desc` (desc->n = warehouse cells n <= 1024) with the

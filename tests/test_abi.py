@@ -211,7 +211,8 @@ def test_cells_entry_points_host_side(lib):
     assert fc(d, 16, P, P + 2, P, None, P, P, need) == dc.ERR_MISALIGNED
     assert fc(d, 16, P, P, P, None, P, P, need) == dc.ERR_CUDA
     rc = dc.dynconv_route_cells
-    assert rc(d, 16, P, P, None, 2, 1.0, P) == dc.ERR_INVALID_ARG
-    assert rc(d, 16, P, P, None, dc.SOFTMAX, 0.0, P) == dc.ERR_INVALID_ARG
-    assert rc(d, 64, P, P, None, dc.SOFTMAX, 1.0, P) == dc.ERR_UNSUPPORTED   # 64 * 128 logits
-    assert rc(d, 16, P, P, None, dc.SOFTMAX, 1.0, P) == dc.ERR_CUDA
+    assert rc(d, 16, P, P, None, 2, 1.0, P, P, need) == dc.ERR_INVALID_ARG
+    assert rc(d, 16, P, P, None, dc.SOFTMAX, 0.0, P, P, need) == dc.ERR_INVALID_ARG
+    assert rc(d, 64, P, P, None, dc.SOFTMAX, 1.0, P, P, need) == dc.ERR_UNSUPPORTED  # 64 * 128
+    assert rc(d, 16, P, P, None, dc.SOFTMAX, 1.0, P, None, 0) == dc.ERR_WORKSPACE
+    assert rc(d, 16, P, P, None, dc.SOFTMAX, 1.0, P, P, need) == dc.ERR_CUDA

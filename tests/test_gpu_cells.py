@@ -32,7 +32,11 @@ def _run(cfg, cells, n, bias=True, samples=None, seed=5):
     E = to_device(ci.warehouse_store, cfg.dtype)
     Wr, br = torch.from_numpy(ci.Wr).cuda(), torch.from_numpy(ci.br).cuda()
     alpha = torch.full((cfg.B, cells, n), float("nan"), device="cuda")
-    dc.check(dc.dynconv_route_cells(d, cells, x, Wr, br, cfg.mode, cfg.tau, alpha), "route_cells")
+    wsb = dc.dynconv_cells_workspace_size(d, cells)
+    assert wsb > 0
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    dc.check(dc.dynconv_route_cells(d, cells, x, Wr, br, cfg.mode, cfg.tau, alpha, ws, wsb),
+             "route_cells")
     torch.cuda.synchronize()
     a_ref = oracle.route_cells(ci.x_f64, ci.Wr, ci.br, cells, cfg.mode, cfg.tau)
     a_got = from_device(alpha)
@@ -40,9 +44,6 @@ def _run(cfg, cells, n, bias=True, samples=None, seed=5):
     # the forward with the oracle's attentions, as fp32
     a32 = alpha_f32_rounded(a_ref)
     alpha.copy_(torch.from_numpy(a32.astype(np.float32)))
-    wsb = dc.dynconv_cells_workspace_size(d, cells)
-    assert wsb > 0
-    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
     tdt = torch.bfloat16 if cfg.dtype == synth.BF16 else torch.float32
     y = torch.full((cfg.B, cfg.H_out, cfg.W_out, cfg.C_out), float("nan"), dtype=tdt, device="cuda")
     b = torch.from_numpy(ci.bias).cuda() if bias else None
