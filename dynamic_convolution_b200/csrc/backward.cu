@@ -343,6 +343,14 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
   float* db = reinterpret_cast<float*>(wsb + L.db);
   float* part = reinterpret_cast<float*>(wsb + L.part);
 
+  // experts per CTA of the mixing gradient: every sample's dW is read
+  // ceil(n / ne) times; its shared memory is checked before anything runs
+  const int ne = d->n > 4 ? 8 : d->n > 2 ? 4 : d->n;
+  const size_t mg_smem = sizeof(float) * (static_cast<size_t>(d->B) * ne +
+                                          (dcb::kBwThreads / 32) * dcb::kMgSampleBlock * ne +
+                                          (dcb::kBwThreads / 32) * 32 * 33);
+  if (mg_smem > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
+
   // 1. per-sample weight gradients
   if (use_tc) {
     rc = run_wgrad_tc(d, di, x, dy, dW, s);
@@ -375,12 +383,6 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
   mp.bs = (d->B + L.bsplit - 1) / L.bsplit;
   mp.dexperts = L.bsplit > 1 ? reinterpret_cast<float*>(wsb + L.dex) : dexperts;
   if (L.bsplit > 1) mp.vec = ws % 4 == 0 ? 1 : 0;
-  // experts per CTA: every sample's dW is read ceil(n / ne) times
-  const int ne = d->n > 4 ? 8 : d->n > 2 ? 4 : d->n;
-  const size_t mg_smem = sizeof(float) * (static_cast<size_t>(d->B) * ne +
-                                          (dcb::kBwThreads / 32) * dcb::kMgSampleBlock * ne +
-                                          (dcb::kBwThreads / 32) * 32 * 33);
-  if (mg_smem > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
   rc = d->dtype == DYNCONV_F32 ? launch_mixgrad<float>(mp, ne, mg_smem, s)
                                : launch_mixgrad<__nv_bfloat16>(mp, ne, mg_smem, s);
   if (rc) return rc;
