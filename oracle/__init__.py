@@ -12,7 +12,10 @@ Every forward function here is pinned by ``tests/test_oracle_pins.py`` against
 closed forms, a library convolution (n=1), brute force on tiny inputs and the
 identities that the pages' definition implies; the backward functions by
 ``tests/test_oracle_backward.py`` against central differences of the pinned
-forward and against torch autograd of the same definition.
+forward and against torch autograd of the same definition; the warehouse
+cells by ``tests/test_oracle_cells.py`` against the pinned ordinary mixture
+(one cell), the pinned routing (per cell), torch conv2d (one-hot cells) and
+per-cell locality.
 """
 from __future__ import annotations
 
