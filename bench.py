@@ -223,6 +223,40 @@ def cpu_baseline(cfg, inp):
                       f"threads over images"}
 
 
+def cpu_baseline_backward(cfg, inp, dy_f64, nb=None):
+    """The oracle's backward step (expert, bias, attention, router and input
+    gradients) on a bounded sample of the batch, timed on the host cores."""
+    import oracle
+    cores = os.cpu_count() or 1
+    nb = nb or min(cfg.B, max(2, min(cores, 8)))
+    x, dy = inp.x_f64[:nb], dy_f64[:nb]
+    a = oracle.route(x, inp.Wr, inp.br, cfg.mode, cfg.tau)
+    t0 = time.perf_counter()
+    oracle.backward(x, dy, inp.experts_f64, a, inp.bias, inp.Wr, cfg.mode, cfg.tau,
+                    stride=cfg.stride, pad=cfg.pad, groups=cfg.groups)
+    dt = time.perf_counter() - t0
+    return {"value": nb / dt, "unit": "images/s", "cores": oracle.threads_used(0, nb),
+            "kind": "oracle",
+            "sample": f"backward of {nb} of the {cfg.B} images (fp64 C oracle; weight and input "
+                      f"gradients threaded over images, router gradients and sums over images "
+                      f"on one thread)"}
+
+
+def cpu_baseline_cells(cfg, ci, cells, n, nb=None):
+    """The oracle's cell routing and forward on a bounded sample of the batch."""
+    import oracle
+    nb = nb or min(cfg.B, 4)
+    x = ci.x_f64[:nb]
+    t0 = time.perf_counter()
+    a = oracle.route_cells(x, ci.Wr, ci.br, cells, cfg.mode, cfg.tau)
+    oracle.forward_cells(x, ci.warehouse_f64, a, ci.bias, cfg.C_out, cfg.KH, cfg.KW, cfg.stride,
+                         cfg.pad, cfg.groups)
+    dt = time.perf_counter() - t0
+    return {"value": nb / dt, "unit": "images/s", "cores": 1, "kind": "oracle",
+            "sample": f"cell routing + forward of {nb} of the {cfg.B} images "
+                      f"(fp64 C oracle, one thread)"}
+
+
 def profile_traffic(kernel_tag: str, workload: str, src_hash: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on the
     current kernel source; else None."""
@@ -237,11 +271,11 @@ def profile_traffic(kernel_tag: str, workload: str, src_hash: str):
     return d.get("dram_bytes_per_launch")
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(csrc: str | None = None) -> str:
     """Hash of the forward translation unit's sources: dynconv.cu and every
-    csrc header it includes, directly or not (the backward unit compiles
-    separately and cannot change the forward kernels)."""
-    csrc = os.path.join(ROOT, "dynamic_convolution_b200", "csrc")
+    csrc header it includes, directly or not (the backward and cell units
+    compile separately and cannot change the forward kernels)."""
+    csrc = csrc or os.path.join(ROOT, "dynamic_convolution_b200", "csrc")
     seen, todo = set(), ["dynconv.cu"]
     while todo:
         fn = todo.pop()
@@ -740,6 +774,8 @@ def run_backward(args, cfg):
             "data": "synthetic (seeded; recipe in DESIGN.md)",
             "config": {"workload": f"{cfg.name} backward", "l2": f"inputs rotated over {nsets} sets"},
             "effective_tflops": tflops, "us_per_call": parts, "gpu_launches_per_step": launches,
+            "cpu_baseline": None if args.no_cpu_baseline else cpu_baseline_backward(
+                cfg, inp, synth.make_upstream_grad(cfg)[1]),
             "wgrad_kernel": ("tcgen05" if cfg.dtype == synth.BF16 and cfg.groups == 1
                              and cfg.stride == 1 and cfg.C_in % 8 == 0 and cfg.C_out % 8 == 0
                              else "cuda-core depthwise" if cfg.dtype == synth.BF16
@@ -821,7 +857,8 @@ def run_cells(args, cfg):
             "config": {"workload": f"{cfg.name} from {cells} cells, warehouse of {n} cells",
                        "l2": f"inputs rotated over {nsets} sets"},
             "conv_tflops": cfg.conv_flops / (ms / 1e3) / 1e12,
-            "mixing_gflop": mix_flops / 1e9, "gpu_launches_per_step": launches}
+            "mixing_gflop": mix_flops / 1e9, "gpu_launches_per_step": launches,
+            "cpu_baseline": None if args.no_cpu_baseline else cpu_baseline_cells(cfg, ci, cells, n)}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -1,0 +1,39 @@
+"""Host-side pieces of bench.py that need no GPU: the CPU baselines of the
+backward and cell modes (bounded oracle samples), and the source hash that
+ties a committed profile to the forward kernels."""
+import os
+import shutil
+
+import bench
+from dynamic_convolution_b200 import synth
+
+
+def test_cpu_baseline_backward_small():
+    cfg = synth.CONFIGS["tiny_fp32"]
+    inp = synth.make_inputs(cfg)
+    r = bench.cpu_baseline_backward(cfg, inp, synth.make_upstream_grad(cfg)[1], nb=2)
+    assert r["value"] > 0 and r["kind"] == "oracle" and r["unit"] == "images/s"
+
+
+def test_cpu_baseline_cells_small():
+    cfg = synth.CONFIGS["tiny_fp32"]
+    ci = synth.make_cell_inputs(cfg, 4, 6)
+    r = bench.cpu_baseline_cells(cfg, ci, 4, 6, nb=2)
+    assert r["value"] > 0 and r["cores"] == 1
+
+
+def test_source_hash_covers_the_forward_unit_only(tmp_path):
+    """On a copy of the sources: the hash changes with a forward header and not
+    with a backward or cell source (those compile in other translation units)."""
+    src = os.path.join(bench.ROOT, "dynamic_convolution_b200", "csrc")
+    dst = tmp_path / "csrc"
+    shutil.copytree(src, dst)
+    base = bench.kernel_source_hash(str(dst))
+    assert base == bench.kernel_source_hash()
+    for fn, changes in (("conv_tc.cuh", True), ("internal.h", True), ("backward.cu", False),
+                        ("backward_kernels.cuh", False), ("cells_kernels.cuh", False)):
+        path = dst / fn
+        orig = path.read_bytes()
+        path.write_bytes(orig + b"\n// probe\n")
+        assert (bench.kernel_source_hash(str(dst)) != base) == changes, fn
+        path.write_bytes(orig)
