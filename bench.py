@@ -563,7 +563,7 @@ def run_ours(args, cfg):
         "value": value, "unit": "images/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32",
-        "data": "synthetic (seeded; recipe in DESIGN.md)",
+        "data": "synthetic (seeded normal draws, layer shapes of the configuration)",
         "config": config_dict(cfg, {"variant": variant_name,
                                     "l2": f"inputs rotated over {nsets} x/y sets "
                                           f"({nsets * set_bytes / 2**20:.0f} MiB > 126 MiB L2)",
@@ -668,7 +668,7 @@ def run_block(args):
             "value": up.B / (ms / 1e3), "unit": "images/s", "n_gpus": 1,
             "steps": reps * min(8, nsets), "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded; recipe in DESIGN.md)",
+            "data": "synthetic (seeded normal draws, layer shapes of the configuration)",
             "config": {"workload": "effnet_block (effnet_expand_1x1 -> effnet_dw_5x5)",
                        "routing_pool": "depthwise routing pooled in the expand epilogue",
                        "l2": f"inputs rotated over {nsets} sets"},
@@ -771,7 +771,7 @@ def run_backward(args, cfg):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32",
-            "data": "synthetic (seeded; recipe in DESIGN.md)",
+            "data": "synthetic (seeded normal draws, layer shapes of the configuration)",
             "config": {"workload": f"{cfg.name} backward", "l2": f"inputs rotated over {nsets} sets"},
             "effective_tflops": tflops, "us_per_call": parts, "gpu_launches_per_step": launches,
             "cpu_baseline": None if args.no_cpu_baseline else cpu_baseline_backward(
@@ -853,7 +853,7 @@ def run_cells(args, cfg):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32",
-            "data": "synthetic (seeded; recipe in DESIGN.md)",
+            "data": "synthetic (seeded normal draws, layer shapes of the configuration)",
             "config": {"workload": f"{cfg.name} from {cells} cells, warehouse of {n} cells",
                        "l2": f"inputs rotated over {nsets} sets"},
             "conv_tflops": cfg.conv_flops / (ms / 1e3) / 1e12,

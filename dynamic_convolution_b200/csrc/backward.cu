@@ -512,30 +512,11 @@ int dynconv_backward_data(const dynconv_desc* desc, const void* dy, const void* 
     rc = dc_lib::launched("transpose_experts_kernel");
     if (rc) return rc;
     char* rest = static_cast<char*>(workspace) + et_bytes;
-    rc = dynconv_forward(&t, dy, workspace, alpha, nullptr, dx,
-                         workspace_bytes > et_bytes ? rest : nullptr, workspace_bytes - et_bytes,
-                         stream);
-    if (rc || !dg) return rc;
-    const long long n_dx = 1LL * d->B * d->H * d->W * d->C_in;
-    const bool bf = d->dtype == DYNCONV_BF16;
-    const int vec = (d->C_in % (bf ? 8 : 4) == 0 && aligned16(dx)) ? (bf ? 8 : 4) : 1;
-    const long long nvec = n_dx / vec;
-    const unsigned g2 = static_cast<unsigned>(
-        std::min<long long>((nvec + dcb::kBwThreads - 1) / dcb::kBwThreads, 16LL * di.sms));
-    const int hwc = d->H * d->W * d->C_in;
-    if (!bf && vec == 4)
-      dcb::gap_add_kernel<float, 4><<<g2, dcb::kBwThreads, 0, s>>>(nvec, hwc, d->C_in, inv_hw, dg,
-                                                                   static_cast<float*>(dx));
-    else if (!bf)
-      dcb::gap_add_kernel<float, 1><<<g2, dcb::kBwThreads, 0, s>>>(nvec, hwc, d->C_in, inv_hw, dg,
-                                                                   static_cast<float*>(dx));
-    else if (vec == 8)
-      dcb::gap_add_kernel<__nv_bfloat16, 8><<<g2, dcb::kBwThreads, 0, s>>>(
-          nvec, hwc, d->C_in, inv_hw, dg, static_cast<__nv_bfloat16*>(dx));
-    else
-      dcb::gap_add_kernel<__nv_bfloat16, 1><<<g2, dcb::kBwThreads, 0, s>>>(
-          nvec, hwc, d->C_in, inv_hw, dg, static_cast<__nv_bfloat16*>(dx));
-    return dc_lib::launched("gap_add_kernel");
+    // dx = (transposed convolution of dy) + dg / (H W), added before the
+    // convolution's single rounding of dx
+    return dc_lib::forward_add(&t, dy, workspace, alpha, nullptr, dx,
+                               workspace_bytes > et_bytes ? rest : nullptr,
+                               workspace_bytes - et_bytes, stream, dg, inv_hw);
   }
   dcb::DgdParams p{};
   p.B = d->B; p.Cin = d->C_in; p.H = d->H; p.W = d->W; p.Cout = d->C_out;

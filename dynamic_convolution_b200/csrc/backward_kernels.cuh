@@ -630,35 +630,6 @@ __global__ void __launch_bounds__(kBwThreads) dgrad_direct_kernel(DgdParams p) {
   static_cast<T*>(p.dx)[o] = from_f32<T>(acc);
 }
 
-// dx[b][p][c] += dg[b][c] * inv_hw in place (dx in T, one rounding). VEC
-// consecutive channels per thread (one 16-byte access when VEC * sizeof(T)
-// is 16; C % VEC == 0).
-template <typename T, int VEC>
-__global__ void __launch_bounds__(kBwThreads)
-    gap_add_kernel(long long nvec, int HWC, int C, float inv_hw, const float* __restrict__ dg,
-                   T* __restrict__ dx) {
-  for (long long o = static_cast<long long>(blockIdx.x) * kBwThreads + threadIdx.x; o < nvec;
-       o += static_cast<long long>(gridDim.x) * kBwThreads) {
-    const long long e = o * VEC;
-    const long long b = e / HWC;
-    const int c = static_cast<int>(e % C);
-    alignas(16) T q[VEC];
-    if constexpr (VEC * sizeof(T) == 16)
-      *reinterpret_cast<uint4*>(q) = *reinterpret_cast<const uint4*>(dx + e);
-    else
-#pragma unroll
-      for (int k = 0; k < VEC; ++k) q[k] = dx[e + k];
-    const float* g = dg + b * C + c;
-#pragma unroll
-    for (int k = 0; k < VEC; ++k) q[k] = from_f32<T>(to_f32(q[k]) + g[k] * inv_hw);
-    if constexpr (VEC * sizeof(T) == 16)
-      *reinterpret_cast<uint4*>(dx + e) = *reinterpret_cast<const uint4*>(q);
-    else
-#pragma unroll
-      for (int k = 0; k < VEC; ++k) dx[e + k] = q[k];
-  }
-}
-
 // Et = every expert transposed within its group and flipped in both spatial
 // axes, as transpose_experts_kernel, through 32 x 32 tiles of shared memory
 // so that both the reads (input channels contiguous) and the writes (output

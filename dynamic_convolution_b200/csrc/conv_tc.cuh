@@ -80,6 +80,8 @@ struct TcParams {
   int inject_skip;    // test hook: withhold the first mixer arrival of CTA 0
   float* ysum;        // optional [B][tiles_h][Cout]: per-unit channel sums of y as stored
   const float* a_out; // optional [B][Cout] output channel attention (FMDConv)
+  const float* chan_add;  // optional [B][Cout]: chan_scale * chan_add[b][co] joins the mixed
+  float chan_scale;       // bias before the single rounding of y
 };
 
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, int base_mode) {
@@ -382,6 +384,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float* ab = VARIANT == kPremix ? p.alpha + static_cast<size_t>(b) * p.n : alpha_s;
       for (int i = 0; i < p.n; ++i) bb = fmaf(ab[i], p.bias[static_cast<size_t>(i) * p.Cout + co], bb);
     }
+    if (p.chan_add != nullptr && co < p.Cout)
+      bb = fmaf(p.chan_add[static_cast<size_t>(b) * p.Cout + co], p.chan_scale, bb);
     // output attention: y = a_out * (conv + mixed bias), channel by channel
     const float so = (p.a_out != nullptr && co < p.Cout) ? p.a_out[static_cast<size_t>(b) * p.Cout + co] : 1.f;
     if (wait_bounded(accum_bar, 0, ctl, kErrWaitEpilogue)) {

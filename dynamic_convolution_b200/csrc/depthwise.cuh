@@ -49,6 +49,8 @@ struct DwParams {
   long long wait_ns;
   const float* a_in;               // [B][C] input channel attention, or null
   const float* a_out;              // [B][C] output channel attention, or null
+  const float* chan_add;           // [B][C] or null: chan_scale * chan_add joins the mixed bias
+  float chan_scale;
 };
 
 template <int K>
@@ -136,6 +138,7 @@ __global__ void __launch_bounds__(kDwThreads, K <= 5 ? 2 : 1)
         for (int q = 0; q < 8; ++q) if (i + q < p.n) s = fmaf(alpha_s[i + q], v[q], s);
       }
     }
+    if (p.chan_add && c < p.C) s = fmaf(p.chan_add[static_cast<size_t>(b) * p.C + c], p.chan_scale, s);
     bias_s[t] = s;
   }
   __syncthreads();

@@ -30,6 +30,8 @@ struct DirectParams {
   void* y;
   const float* a_in;   // [B][Cin] input channel attention, or null
   const float* a_out;  // [B][Cout] output channel attention, or null
+  const float* chan_add;  // [B][Cout] or null: chan_scale * chan_add joins the mixed bias
+  float chan_scale;
 };
 
 template <typename T>
@@ -70,6 +72,8 @@ __global__ void __launch_bounds__(kDirectThreads) direct_conv_kernel(DirectParam
     if (p.bias)
       for (int i = 0; i < p.n; ++i)
         s = fmaf(alpha_s[i], p.bias[static_cast<size_t>(i) * p.Cout + co0 + c], s);
+    if (p.chan_add)
+      s = fmaf(p.chan_add[static_cast<size_t>(b) * p.Cout + co0 + c], p.chan_scale, s);
     bias_s[c] = s;
   }
   __syncthreads();

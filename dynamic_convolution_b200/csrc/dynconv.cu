@@ -375,11 +375,13 @@ int launch_tc(const TcPlan& plan, const CUtensorMap& xmap, const CUtensorMap& wm
 
 
 // State slot of the streamed mixing for (device, stream): launches on one
-// stream are ordered, so they may share a slot; streams get slots of their
-// own (least recently used first when there are more streams than slots).
+// stream are ordered, so they may share a slot; every stream gets a slot of
+// its own, kept for the life of the process. When all kMcSlots slots of the
+// device belong to other streams, a slot is never taken from one of them (its
+// kernel may still be running on those counters): the call returns
+// DYNCONV_ERR_UNSUPPORTED and the caller runs the two-kernel PREMIX form.
 std::mutex g_slot_mu;
-std::map<std::pair<int, void*>, std::pair<int, unsigned long long>> g_slot_of;
-unsigned long long g_slot_tick = 0;
+std::map<std::pair<int, void*>, int> g_slot_of;
 bool g_slots_dirty[64] = {};  // per device: a bounded wait expired, zero all slots
 
 int mix_state_slot(void* stream, unsigned int** out, cudaStream_t s) {
@@ -399,23 +401,16 @@ int mix_state_slot(void* stream, unsigned int** out, cudaStream_t s) {
   auto it = g_slot_of.find(key);
   int slot = -1;
   if (it != g_slot_of.end()) {
-    slot = it->second.first;
+    slot = it->second;
   } else {
     bool used[dc::kMcSlots] = {};
-    auto lru = g_slot_of.end();
-    for (auto jt = g_slot_of.begin(); jt != g_slot_of.end(); ++jt) {
-      if (jt->first.first != dev) continue;
-      used[jt->second.first] = true;
-      if (lru == g_slot_of.end() || jt->second.second < lru->second.second) lru = jt;
-    }
+    for (auto jt = g_slot_of.begin(); jt != g_slot_of.end(); ++jt)
+      if (jt->first.first == dev) used[jt->second] = true;
     for (int i = 0; i < dc::kMcSlots && slot < 0; ++i)
       if (!used[i]) slot = i;
-    if (slot < 0) {
-      slot = lru->second.first;
-      g_slot_of.erase(lru);
-    }
+    if (slot < 0) return DYNCONV_ERR_UNSUPPORTED;  // every slot belongs to another stream
+    g_slot_of[key] = slot;
   }
-  g_slot_of[key] = std::make_pair(slot, ++g_slot_tick);
   *out = static_cast<unsigned int*>(base) + static_cast<size_t>(slot) * dc::kMcStateWords;
   return DYNCONV_OK;
 }
@@ -469,7 +464,7 @@ int run_mixconv(const dynconv_desc* d, const TcPlan& plan_in, const DeviceState*
   mp.cv.wait_ns = g_wait_ns.load();
   mp.wb = static_cast<__nv_bfloat16*>(ws);
   int rc = mix_state_slot(static_cast<void*>(stream), &mp.state, stream);
-  if (rc) return rc;
+  if (rc) return rc;  // UNSUPPORTED when no slot is free: the two-kernel form runs
   cudaError_t e = cudaSuccess;
   auto kern = d->n <= 2 ? dc::mixconv_kernel<2>
               : d->n <= 4 ? dc::mixconv_kernel<4> : dc::mixconv_kernel<8>;
@@ -504,7 +499,8 @@ int run_mixconv(const dynconv_desc* d, const TcPlan& plan_in, const DeviceState*
 int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void* x,
            const void* experts, const float* alpha, const float* bias, void* y, void* ws,
            size_t ws_bytes, cudaStream_t stream, float* ysum = nullptr,
-           const float* a_in = nullptr, const float* a_out = nullptr) {
+           const float* a_in = nullptr, const float* a_out = nullptr,
+           const float* chan_add = nullptr, float chan_scale = 0.f) {
   // input attention is folded into the mixed kernel: only the PREMIX variant
   // with the CUDA-core mixer takes it
   if (a_in != nullptr && variant != DYNCONV_VARIANT_PREMIX) return DYNCONV_ERR_UNSUPPORTED;
@@ -512,6 +508,8 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   if (!tc_plan(d, variant, st->sms, st->max_smem_optin, &plan)) return DYNCONV_ERR_UNSUPPORTED;
   plan.p.ysum = ysum;
   plan.p.a_out = a_out;
+  plan.p.chan_add = chan_add;
+  plan.p.chan_scale = chan_scale;
   plan.p.experts = static_cast<const __nv_bfloat16*>(experts);
   plan.p.alpha = alpha;
   plan.p.bias = bias;
@@ -532,7 +530,7 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   if (!aligned16(ws)) return DYNCONV_ERR_MISALIGNED;
   plan.p.inject_skip = 0;
   if (g_stream_mix.load() && g_premix_mixer.load() != 1 && d->n <= dc::kMcMaxExperts &&
-      ysum == nullptr && a_in == nullptr && a_out == nullptr) {
+      ysum == nullptr && a_in == nullptr && a_out == nullptr && chan_add == nullptr) {
     rc = encode_w_map(&wmap, ws, d);
     if (rc) return rc;
     rc = run_mixconv(d, plan, st, experts, alpha, bias, y, ws, xmap, wmap, stream);
@@ -790,7 +788,8 @@ int resolve_variant(const dynconv_desc* desc, size_t ws_bytes, const DeviceState
 int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
                  const float* alpha, const float* bias, void* y, void* workspace,
                  size_t workspace_bytes, void* stream, float* ysum,
-                 const float* a_in = nullptr, const float* a_out = nullptr) {
+                 const float* a_in = nullptr, const float* a_out = nullptr,
+                 const float* chan_add = nullptr, float chan_scale = 0.f) {
   int rc = validate_desc(desc);
   if (rc) return rc;
   if (!x || !experts || !alpha || !y) return DYNCONV_ERR_INVALID_ARG;
@@ -817,7 +816,7 @@ int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
       if (!tc_shape_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
       if (!aligned16(x) || !aligned16(experts) || !aligned16(y)) return DYNCONV_ERR_MISALIGNED;
       return run_tc(desc, variant, st, x, experts, alpha, bias, y, workspace, workspace_bytes, s,
-                    ysum, a_in, a_out);
+                    ysum, a_in, a_out, chan_add, chan_scale);
     }
     case DYNCONV_VARIANT_DEPTHWISE: {
       if (!depthwise_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
@@ -839,6 +838,8 @@ int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
       p.wait_ns = g_wait_ns.load();
       p.a_in = a_in;
       p.a_out = a_out;
+      p.chan_add = chan_add;
+      p.chan_scale = chan_scale;
       const int TC = ((p.cols + 1) & ~1) + K - 1, TR = p.rows + K - 1;
       const size_t tile_bytes = static_cast<size_t>(TR) * TC * dc::kDwChunk * 2;
       const size_t smem = 128 + ((tile_bytes + 127) & ~size_t(127)) +
@@ -894,6 +895,7 @@ int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
       p.cob = static_cast<int>(cob);
       p.x = x; p.experts = experts; p.alpha = alpha; p.bias = bias; p.y = y;
       p.a_in = a_in; p.a_out = a_out;
+      p.chan_add = chan_add; p.chan_scale = chan_scale;
       const size_t smem = sizeof(float) * (desc->n + cob + cob * wrow);
       dim3 grid((p.Ho * p.Wo + dc::kDirectPix - 1) / dc::kDirectPix,
                 static_cast<unsigned>((desc->C_out + cob - 1) / cob), desc->B);
@@ -1109,6 +1111,13 @@ int cuda_error(cudaError_t e, const char* what) { return cuda_fail(e, what); }
 int launched(const char* what) { return check_launch(what); }
 
 int validate(const dynconv_desc* desc) { return validate_desc(desc); }
+
+int forward_add(const dynconv_desc* desc, const void* x, const void* experts, const float* alpha,
+                const float* bias, void* y, void* workspace, size_t workspace_bytes, void* stream,
+                const float* chan_add, float chan_scale) {
+  return forward_impl(desc, x, experts, alpha, bias, y, workspace, workspace_bytes, stream,
+                      nullptr, nullptr, nullptr, chan_add, chan_scale);
+}
 
 cudaError_t set_smem(const void* kernel, size_t bytes) {
   int dev = 0;

@@ -33,5 +33,12 @@ DC_HIDDEN cudaError_t set_smem(const void* kernel, size_t bytes);
 // The descriptor checks every entry point makes (DYNCONV_OK or INVALID_ARG /
 // UNSUPPORTED).
 DC_HIDDEN int validate(const dynconv_desc* desc);
+// dynconv_forward with one more per-(sample, output channel) term:
+// chan_scale * chan_add[b][co] is added to the mixed bias, so that it joins
+// the convolution before the single rounding of y (chan_add may be null).
+DC_HIDDEN int forward_add(const dynconv_desc* desc, const void* x, const void* experts,
+                          const float* alpha, const float* bias, void* y, void* workspace,
+                          size_t workspace_bytes, void* stream, const float* chan_add,
+                          float chan_scale);
 
 }  // namespace dc_lib

@@ -71,8 +71,10 @@ typedef enum { DYNCONV_SIGMOID = 0, DYNCONV_SOFTMAX = 1 } dynconv_mode;
  *  OUTSIDE - output-side mixing: y_b = sum_i alpha_{b,i} (x_b conv W_i) + b_b as
  *            one K-stacked tensor-core GEMM over (expert, tap, channel) with the
  *            operand alpha_{b,i} W_i (bf16 only; n times the conv work);
- *  PREMIX  - W_b for all samples is mixed first by a tensor-core GEMM into the
- *            workspace (bf16), then a tensor-core convolution reads it
+ *  PREMIX  - W_b for all samples is mixed first into the workspace (bf16),
+ *            on CUDA cores when n <= 8 (a store-bound stream of at most 8
+ *            multiply-adds per weight) and by a tcgen05 GEMM over the experts
+ *            when n > 8; then a tensor-core convolution TMA-loads it
  *            (bf16 only; needs dynconv_workspace_size bytes);
  *  DIRECT  - CUDA-core direct convolution, fp32 accumulation, any shape
  *            (the fp32 path; also bf16 shapes the tensor-core kernels reject);
@@ -210,8 +212,9 @@ int dynconv_route_pooled(const dynconv_desc* desc, const float* ysum, int parts,
  * device memory and hands out no workspace, or code that must not call
  * cudaMalloc after start-up (cudaMalloc synchronises the device and can fail
  * once memory is committed). It computes exactly what dynconv_forward with the
- * PREMIX variant computes (tensor-core kernel mixing, then the tensor-core
- * convolution), but its scratch is a fixed array that the library itself
+ * PREMIX variant computes, bit for bit: the same mixer PREMIX selects (CUDA
+ * cores for n <= 8, the tcgen05 mixing GEMM above), then the tensor-core
+ * convolution; but its scratch is a fixed array that the library itself
  * defines in device memory: DYNCONV_NOALLOC_MAX_BYTES bytes, reserved on every
  * GPU on which the library's kernels are loaded, for the life of the process.
  *
@@ -278,7 +281,9 @@ unsigned long long dynconv_launch_count(void);
  * plainly. For measurements.
  * key 6: 1 runs PREMIX with n <= 8 as one persistent cooperative kernel that
  * streams the mixing into the convolution (per-K-slice counters); 0 (default)
- * runs it as two kernels (mixing, then convolution).
+ * runs it as two kernels (mixing, then convolution). The counters live in a
+ * few fixed slots per device, one per stream for the life of the process;
+ * calls on further streams run the two-kernel form.
  * key 7: which kernel mixes the per-sample kernels of the two-kernel PREMIX
  * form: 0 (default) the CUDA-core mixer when n <= 8, else the tensor-core
  * mixing GEMM; 1 always the tensor-core GEMM (and never the streamed kernel of

@@ -32,9 +32,10 @@
  * [B][H_out][W_out][C_out] in desc->dtype; experts [n][C_out][KH][KW][C_in/groups]
  * in desc->dtype; alpha, bias, Wr as in dynconv.h (fp32). Every gradient is
  * fp32 and in the layout of the value it belongs to, except dx, which is in
- * desc->dtype: rounded once after the convolution's input gradient and once
- * more after dg/(H*W) is added when it runs on the forward kernels, once when
- * it runs on the generic kernel. Outputs are overwritten, not accumulated.
+ * desc->dtype, rounded once: dg/(H*W) is added to the convolution's input
+ * gradient in fp32 before the rounding, on the forward kernels (through their
+ * epilogue's per-channel term) and on the generic kernel alike. Outputs are
+ * overwritten, not accumulated.
  * All results are deterministic (no floating-point atomics).
  *
  * Ownership: the caller allocates every buffer (device memory) and the
