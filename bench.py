@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--config", default=None)
     ap.add_argument("--variant", default="auto",
                     choices=["auto", "fused", "outside", "premix", "direct", "depthwise"])
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the configuration's batch size (small profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="time the layer's backward step (weight, router and input gradients)")
@@ -59,6 +61,9 @@ def parse():
                     help="time the layer with its kernel assembled from this many warehouse cells")
     ap.add_argument("--warehouse", type=int, default=128, help="warehouse cells for --cells")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--per-config", default="all",
+                    help="comma-separated configurations measured into the line's per_config "
+                         "object ('all', or 'none' to skip); one GPU only")
     ap.add_argument("--hooks", default="",
                     help="implementation knobs for comparisons, e.g. '6=0,5=0' "
                          "(see dynconv_test_hook in include/dynconv.h)")
@@ -290,6 +295,269 @@ def kernel_source_hash(csrc: str | None = None) -> str:
             h.update(fn.encode())
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def bound_of(cfg, peaks):
+    """Roofline bound of a layer: tensor cores when its arithmetic intensity
+    (conv FLOP per algorithmic byte, x + y + experts) is above the ridge of the
+    two measured peaks and it is a dense bf16 layer, else HBM."""
+    from dynamic_convolution_b200 import synth
+    algo_bytes = (cfg.B * cfg.H * cfg.W * cfg.C_in + cfg.B * cfg.H_out * cfg.W_out * cfg.C_out
+                  + cfg.n * cfg.weight_elems) * cfg.elem_bytes
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    tensor = (cfg.dtype == synth.BF16 and cfg.groups == 1
+              and cfg.conv_flops / max(algo_bytes, 1) >= ridge)
+    return ("tensor" if tensor else "hbm"), algo_bytes
+
+
+def roofline_entry(cfg, launch_ms, kernel_label, peaks, peak_kind, traffic):
+    bound, algo_bytes = bound_of(cfg, peaks)
+    if bound == "tensor":
+        achieved = cfg.conv_flops / (launch_ms / 1e3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_kind": f"bf16 dense burst, {peak_kind}",
+                "kernel": kernel_label, "traffic": traffic, "launch_ms": launch_ms,
+                "algorithmic": f"{cfg.conv_flops} conv FLOP per launch (2*B*HW*Cout*Cin*KH*KW)"}
+    achieved = algo_bytes / (launch_ms / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_kind": f"HBM copy, {peak_kind}",
+            "kernel": kernel_label, "traffic": traffic, "launch_ms": launch_ms,
+            "algorithmic": f"{algo_bytes} bytes per launch (x + y + experts)"}
+
+
+def kernel_label_of(variant_name, cfg):
+    if variant_name == "premix":
+        mixer = "premix_small_kernel" if cfg.n <= 8 else "premix_kernel"
+        return f"forward call: {mixer} + tc_conv_kernel<premix>"
+    if variant_name in ("fused", "outside"):
+        return f"tc_conv_kernel<{variant_name}>"
+    return f"{variant_name}_kernel"
+
+
+class GraphTimer:
+    """Per-call device times of captured calls: each call is one CUDA graph;
+    cold reps first READ a buffer of twice the L2 size (every input, expert and
+    workspace byte of the call then comes from HBM; a read leaves no dirty
+    lines that would drain to HBM during the timed call, as a write would),
+    warm reps repeat the call back to back. Events are recorded on the stream
+    the graphs replay on."""
+
+    def __init__(self, torch, stream):
+        self.torch = torch
+        self.stream = stream
+        self.flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.int32, device="cuda")
+        self.sink = None
+
+    def capture(self, fn):
+        g = self.torch.cuda.CUDAGraph()
+        with self.torch.cuda.graph(g, stream=self.stream):
+            fn(self.stream)
+        return g
+
+    def median_ms(self, g, reps, cold):
+        torch = self.torch
+        g.replay()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        with torch.cuda.stream(self.stream):
+            for k, (e0, e1) in enumerate(evs):
+                if cold:
+                    self.sink = self.flush.sum()
+                e0.record(self.stream)
+                g.replay()
+                e1.record(self.stream)
+        self.stream.synchronize()
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+
+
+def measure_config(name, args, peaks, peak_kind, src_hash):
+    """One layer configuration on one GPU, for the line's per_config object:
+    steps of routing + forward as CUDA-graph replays over rotating input sets
+    (ms_per_step, with the clocks sampled meanwhile), the median of >= 50 cold
+    and of >= 50 warm per-call times of the routing and the forward call (the
+    roofline uses the cold forward median), the forward of every variant that
+    takes the shape, the oracle on a bounded sample of the batch, and the
+    end-to-end rate through the public calls with host buffers."""
+    import torch
+
+    import dynamic_convolution_b200 as dc
+    from dynamic_convolution_b200 import synth
+
+    cfg = synth.CONFIGS[name]
+    reps = max(args.steps, 50)
+    inp = synth.make_inputs(cfg)
+    tdt = torch.bfloat16 if cfg.dtype == synth.BF16 else torch.float32
+    dev = lambda a: (torch.from_numpy(a).view(torch.bfloat16) if cfg.dtype == synth.BF16
+                     else torch.from_numpy(a)).cuda()
+    x0, E = dev(inp.x_store), dev(inp.experts_store)
+    Wr, br, bias = (torch.from_numpy(a).cuda() for a in (inp.Wr, inp.br, inp.bias))
+    desc = dc.desc_from_config(cfg)
+    ws_bytes = dc.dynconv_workspace_size(desc)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    chosen = dc.dynconv_select_variant(desc, ws_bytes)
+    vname = dc.VARIANT_NAMES.get(chosen, str(chosen))
+    set_bytes = 2 * x0.numel() * x0.element_size()
+    nsets = max(2, min(64, math.ceil(2 * L2_BYTES / set_bytes)))
+    xs = [x0] + [x0.clone() for _ in range(nsets - 1)]
+    ys = [torch.empty((cfg.B, cfg.H_out, cfg.W_out, cfg.C_out), dtype=tdt, device="cuda")
+          for _ in range(nsets)]
+    alphas = [torch.empty((cfg.B, cfg.n), device="cuda") for _ in range(nsets)]
+    stream = torch.cuda.Stream()
+    timer = GraphTimer(torch, stream)
+
+    def route(s, st, d=desc):
+        dc.check(dc.dynconv_route(d, xs[s], Wr, br, cfg.mode, cfg.tau, alphas[s], st), "route")
+
+    def forward(s, st, d=desc):
+        dc.check(dc.dynconv_forward(d, xs[s], E, alphas[s], bias, ys[s], ws, ws_bytes, st),
+                 "forward")
+
+    with torch.cuda.stream(stream):
+        for k in range(max(args.warmup, 10)):
+            route(k % nsets, stream)
+            forward(k % nsets, stream)
+    stream.synchronize()
+    dc.check(dc.dynconv_device_status(stream), f"{name}: device status after warm-up")
+
+    # steps: graphs of up to 8 (route, forward) pairs over rotating sets
+    G = min(8, nsets)
+    n0 = dc.dynconv_launch_count()
+    graphs = []
+    for g0 in range(0, nsets - G + 1, G):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for s in range(g0, g0 + G):
+                route(s, stream)
+                forward(s, stream)
+        graphs.append(g)
+    launches_per_step = (dc.dynconv_launch_count() - n0) / (len(graphs) * G)
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    graphs[0].replay()
+    torch.cuda.synchronize()
+    est = max(time.perf_counter() - t0, 1e-6)
+    n_rep = max(math.ceil(reps / G), min(4000, math.ceil(0.25 / est)))
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.1)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(n_rep):
+            graphs[i % len(graphs)].replay()
+        e1.record(stream)
+    stream.synchronize()
+    clocks = sampler.stop()
+    step_ms = e0.elapsed_time(e1) / (n_rep * G)
+    del graphs
+
+    # per-call medians, cold (L2 flushed first) and warm
+    g_route = timer.capture(lambda st: route(0, st))
+    g_fwd = timer.capture(lambda st: forward(0, st))
+    route_cold = timer.median_ms(g_route, reps, True)
+    fwd_cold = timer.median_ms(g_fwd, reps, True)
+    route_warm = timer.median_ms(g_route, reps, False)
+    fwd_warm = timer.median_ms(g_fwd, reps, False)
+    del g_route, g_fwd
+    dc.check(dc.dynconv_device_status(stream), f"{name}: device status after timing")
+
+    # every variant that takes the shape (cold forward medians)
+    variants = {}
+    cand = ([dc.VARIANT_FUSED, dc.VARIANT_OUTSIDE, dc.VARIANT_PREMIX]
+            if cfg.dtype == synth.BF16 and cfg.groups == 1 else
+            [dc.VARIANT_DEPTHWISE] if cfg.groups > 1 else [dc.VARIANT_DIRECT])
+    for v in cand:
+        dv = dc.desc_from_config(cfg, v)
+        # a plain call first: a variant that refuses the shape is skipped
+        # (it returns before launching anything)
+        if dc.dynconv_forward(dv, xs[0], E, alphas[0], bias, ys[0], ws, ws_bytes, stream) != 0:
+            continue
+        stream.synchronize()
+        g = timer.capture(lambda st, dv=dv: forward(0, st, dv))
+        variants[dc.VARIANT_NAMES[v]] = timer.median_ms(g, reps, True)
+        del g
+    dc.check(dc.dynconv_device_status(stream), f"{name}: device status after variants")
+
+    # end to end: host x in, y out, copies inside the timed region
+    e2e = measure_e2e(torch, dc, cfg, inp, desc, xs, alphas, ys, Wr, br, E, bias, ws_bytes,
+                      max(20, min(reps, 200)), tdt, nsets)
+
+    cpu = None if args.no_cpu_baseline else cpu_baseline(cfg, inp)
+    traffic = profile_traffic(vname, cfg.name, src_hash)
+    label = kernel_label_of(vname, cfg)
+    entry = {
+        "variant": vname, "dtype": "bf16" if cfg.dtype == synth.BF16 else "f32",
+        "ms_per_step": step_ms, "images_per_s": cfg.B / (step_ms / 1e3),
+        "forward_ms": fwd_cold, "route_ms": route_cold,
+        "forward_ms_warm_l2": fwd_warm, "route_ms_warm_l2": route_warm,
+        "forward_images_per_s": cfg.B / (fwd_cold / 1e3),
+        "forward_eff_tflops": cfg.conv_flops / (fwd_cold / 1e3) / 1e12,
+        "roofline": roofline_entry(cfg, fwd_cold, label, peaks, peak_kind, traffic),
+        "variants_forward_ms": variants,
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "gpu_launches_per_step": launches_per_step,
+        "timing": (f"ms_per_step: mean over {n_rep * G} graph-replayed steps over {nsets} input "
+                   f"sets; *_ms: median of {reps} calls, cold = after reading "
+                   f"{2 * L2_BYTES >> 20} MiB (2x L2), warm = back to back"),
+    }
+    if cfg.dtype == synth.BF16 and cfg.groups == 1:
+        entry["mixing_gflop"] = 2.0 * cfg.B * cfg.n * cfg.weight_elems / 1e9
+    del xs, ys, alphas, E, ws, timer
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry
+
+
+def measure_e2e(torch, dc, cfg, inp, desc, xs, alphas, ys, Wr, br, E, bias, ws_bytes, steps,
+                tdt, nsets):
+    """Routing + forward through the public calls with the input copied in from
+    pinned host memory and the output copied back every step, alternating over
+    two streams (own buffers and workspace each) so that copies in, kernels and
+    copies out of neighbouring steps overlap."""
+    from dynamic_convolution_b200 import synth
+    xh = torch.from_numpy(inp.x_store).pin_memory()
+    if cfg.dtype == synth.BF16:
+        xh = xh.view(torch.bfloat16)
+    n_e2e = 2
+    streams = [torch.cuda.Stream() for _ in range(n_e2e)]
+    yhs = [torch.empty(ys[0].shape, dtype=tdt).pin_memory() for _ in range(n_e2e)]
+    wss = [torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda") for _ in range(n_e2e)]
+    per = max(1, nsets // n_e2e)
+
+    def step(k):
+        j = k % n_e2e
+        st, s = streams[j], k % (n_e2e * per)
+        with torch.cuda.stream(st):
+            xs[s].copy_(xh, non_blocking=True)
+            dc.check(dc.dynconv_route(desc, xs[s], Wr, br, cfg.mode, cfg.tau, alphas[s], st))
+            dc.check(dc.dynconv_forward(desc, xs[s], E, alphas[s], bias, ys[s], wss[j], ws_bytes,
+                                        st))
+            yhs[j].copy_(ys[s], non_blocking=True)
+
+    for k in range(2 * n_e2e):
+        step(k)
+    torch.cuda.synchronize()
+    main = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for st in streams:
+        st.wait_event(e0)
+    for k in range(steps):
+        step(k)
+    for st in streams:
+        main.wait_stream(st)
+    e1.record(main)
+    main.synchronize()
+    ms = e0.elapsed_time(e1)
+    return {"value": cfg.B * steps / (ms / 1e3), "unit": "images/s",
+            "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
+            "d2h_bytes_per_step": int(yhs[0].numel() * yhs[0].element_size()),
+            "streams": n_e2e, "steps": steps}
 
 
 def run_ours(args, cfg):
@@ -585,6 +853,10 @@ def run_ours(args, cfg):
         "source_hash": src_hash,
         "hooks": hooks or None,
     }
+    if world == 1 and args.per_config != "none":
+        names = list(synth.CONFIGS) if args.per_config == "all" else args.per_config.split(",")
+        line["per_config"] = {nm: measure_config(nm, args, peaks, peak_kind, src_hash)
+                              for nm in names}
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -874,6 +1146,8 @@ def main():
         return run_cells(args, synth.CONFIGS[args.config or synth.HEADLINE])
     name = args.config or synth.HEADLINE
     cfg = synth.CONFIGS[name]
+    if args.batch > 0:
+        cfg = cfg.scaled(B=args.batch, name=f"{cfg.name}_b{args.batch}")
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

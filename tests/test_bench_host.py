@@ -37,3 +37,24 @@ def test_source_hash_covers_the_forward_unit_only(tmp_path):
         path.write_bytes(orig + b"\n// probe\n")
         assert (bench.kernel_source_hash(str(dst)) != base) == changes, fn
         path.write_bytes(orig)
+
+
+def test_roofline_bound_per_configuration():
+    """Tensor-bound only where the conv FLOP per algorithmic byte exceeds the
+    ridge of the two peaks (dense bf16 layers); the fraction is achieved / peak."""
+    peaks = {"hbm_gbs": 6553.6, "bf16_tflops": 1672.7}
+    want = {"tiny_fp32": "hbm", "resnet18_3x3": "tensor", "effnet_expand_1x1": "hbm",
+            "effnet_dw_5x5": "hbm", "deep_3x3_tau30": "tensor", "large_n64": "hbm"}
+    for name, bound in want.items():
+        cfg = synth.CONFIGS[name]
+        got, algo = bench.bound_of(cfg, peaks)
+        assert got == bound, name
+        r = bench.roofline_entry(cfg, 0.05, "k", peaks, "measured", None)
+        if bound == "tensor":
+            assert abs(r["achieved"] - cfg.conv_flops / 5e-5 / 1e12) < 1e-6 * r["achieved"]
+        else:
+            assert abs(r["achieved"] - algo / 5e-5 / 1e9) < 1e-6 * r["achieved"]
+        assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
+    # the algorithmic bytes of the deep 3x3 layer: x + y + experts, bf16
+    cfg = synth.CONFIGS["deep_3x3_tau30"]
+    assert bench.bound_of(cfg, peaks)[1] == 2 * (2 * 256 * 14 * 14 * 256 + 16 * 256 * 9 * 256)
