@@ -16,6 +16,7 @@
 
 #include "backward_kernels.cuh"
 #include "backward_wgrad_tc.cuh"
+#include "backward_mixgrad_tc.cuh"
 
 namespace {
 
@@ -120,7 +121,7 @@ int encode_4d(EncodeTiledFn enc, CUtensorMap* map, const void* base, int C, int 
 }
 
 int run_wgrad_tc(const dynconv_desc* d, const dc_lib::DeviceInfo& di, const void* x,
-                 const void* dy, float* dW, cudaStream_t s) {
+                 const void* dy, float* dW, cudaStream_t s, bool hilo = false) {
   const int Ho = out_size(d->H, d->KH, 1, d->pad), Wo = out_size(d->W, d->KW, 1, d->pad);
   dcb::WgParams p{};
   p.B = d->B; p.Cin = d->C_in; p.Cout = d->C_out; p.Ho = Ho; p.Wo = Wo;
@@ -146,6 +147,7 @@ int run_wgrad_tc(const dynconv_desc* d, const dc_lib::DeviceInfo& di, const void
   p.stages = std::min(4, (210 * 1024 - 4 * dcb::kWgStageBytes) / stage_bytes);
   if (p.stages < 2) return dc_lib::fail(DYNCONV_ERR_UNSUPPORTED, "weight-gradient tile too large");
   p.dW = dW;
+  p.hilo = hilo ? 1 : 0;
   p.err = di.err;
   p.wait_ns = di.wait_ns;
   auto enc = reinterpret_cast<EncodeTiledFn>(di.encode_tiled);
@@ -269,6 +271,63 @@ int run_chansum(const dynconv_desc* d, int sms, const void* v, int P, int C, flo
   return dc_lib::launched("chansum_finish_kernel");
 }
 
+// The tensor-core mixing gradient applies to dW from the tcgen05 weight
+// gradient (written as bf16 hi / lo planes) with at most 256 samples, 32
+// experts and kernels of a multiple of 128 weights.
+bool mixgrad_tc_ok(const dynconv_desc* d) {
+  return dc_lib::mixgrad_tc_enabled() && d->dtype == DYNCONV_BF16 && d->B >= 1 && d->B <= 256 &&
+         d->n <= 32 && wsize_of(d) % dcb::kMtTile == 0;
+}
+
+// dexperts (complete) and one dalpha partial per CTA; returns the number of
+// partials in `part` through *nparts.
+int run_mixgrad_tc(const dynconv_desc* d, const dc_lib::DeviceInfo& di, const void* planes,
+                   const void* experts, const float* alpha, float* dexperts, float* part,
+                   int max_parts, int* nparts, cudaStream_t s) {
+  const long long ws = wsize_of(d);
+  dcb::MtParams p{};
+  p.B = d->B; p.n = d->n; p.nk = d->n <= 16 ? 16 : 32;
+  p.halves = (d->B + 127) / 128;
+  p.wsize = ws;
+  p.tiles = ws / dcb::kMtTile;
+  p.plane_bytes = 2 * 128 * 128;
+  p.e_bytes = 2 * p.nk * 128;
+  p.stage_bytes = 2 * p.plane_bytes + p.e_bytes;
+  p.b_bytes = p.halves * 2 * 2 * p.nk * 128;
+  const size_t fixed = 1024 + static_cast<size_t>(p.b_bytes) + 8 * 32 + 16;
+  p.stages = static_cast<int>(std::min<size_t>(3, (di.max_smem_optin - fixed) / p.stage_bytes));
+  if (p.stages < 2) return DYNCONV_ERR_UNSUPPORTED;
+  p.alpha = alpha;
+  p.dexperts = dexperts;
+  p.part = part;
+  p.err = di.err;
+  p.wait_ns = di.wait_ns;
+  auto enc = reinterpret_cast<EncodeTiledFn>(di.encode_tiled);
+  auto map2d = [&](CUtensorMap* m, const void* base, long long inner, int rows, int box_rows) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner) * 2};
+    const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t es[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  CUtensorMap himap, lomap, emap;
+  const __nv_bfloat16* hi = static_cast<const __nv_bfloat16*>(planes);
+  const __nv_bfloat16* lo = hi + static_cast<size_t>(d->B) * ws;
+  if (!map2d(&himap, hi, ws, d->B, 128) || !map2d(&lomap, lo, ws, d->B, 128) ||
+      !map2d(&emap, experts, ws, d->n, p.nk))
+    return dc_lib::fail(DYNCONV_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled (mixing gradient)");
+  const size_t smem = fixed + static_cast<size_t>(p.stages) * p.stage_bytes;
+  cudaError_t e = dc_lib::set_smem(reinterpret_cast<const void*>(dcb::mixgrad_tc_kernel), smem);
+  if (e != cudaSuccess) return dc_lib::cuda_error(e, "cudaFuncSetAttribute(mixgrad_tc)");
+  const int grid = static_cast<int>(std::min<long long>({p.tiles, static_cast<long long>(di.sms),
+                                                         static_cast<long long>(max_parts)}));
+  dcb::mixgrad_tc_kernel<<<grid, dcb::kMtThreads, smem, s>>>(himap, lomap, emap, p);
+  *nparts = grid;
+  return dc_lib::launched("mixgrad_tc_kernel");
+}
+
 template <typename T>
 int launch_mixgrad(const dcb::MgParams& p, int ne, size_t smem, cudaStream_t s) {
   const dim3 grid(p.chunks, (p.n + ne - 1) / ne, p.bsplit);
@@ -351,9 +410,11 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
                                           (dcb::kBwThreads / 32) * 32 * 33);
   if (mg_smem > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
 
-  // 1. per-sample weight gradients
+  // 1. per-sample weight gradients (as bf16 hi / lo planes when the
+  // tensor-core mixing gradient reads them)
+  const bool mg_tc = use_tc && mixgrad_tc_ok(d) && aligned16(experts);
   if (use_tc) {
-    rc = run_wgrad_tc(d, di, x, dy, dW, s);
+    rc = run_wgrad_tc(d, di, x, dy, dW, s, mg_tc);
     if (rc == DYNCONV_ERR_UNSUPPORTED && d->variant == DYNCONV_VARIANT_AUTO) use_tc = false;
     else if (rc) return rc;
   }
@@ -375,6 +436,11 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
                    reinterpret_cast<float*>(wsb + L.cs), db, s);
   if (rc) return rc;
   // 3. the experts' gradients and the chunks' shares of dalpha
+  int nparts = L.chunks;
+  if (use_tc && mg_tc) {
+    rc = run_mixgrad_tc(d, di, dW, experts, alpha, dexperts, part, L.chunks, &nparts, s);
+    if (rc) return rc;
+  } else {
   dcb::MgParams mp{};
   mp.B = d->B; mp.n = d->n; mp.wsize = ws; mp.chunks = L.chunks;
   mp.vec = (ws % 4 == 0 && aligned16(dexperts)) ? 1 : 0;
@@ -395,8 +461,9 @@ int dynconv_backward_weight(const dynconv_desc* desc, const void* x, const void*
     rc = dc_lib::launched("dexperts_finish_kernel");
     if (rc) return rc;
   }
-  // 4. dalpha = sum of the chunks' shares + <db_b, bias_i>
-  dcb::dalpha_finish_kernel<<<d->B, dcb::kBwThreads, 0, s>>>(d->B, d->n, d->C_out, L.chunks, part,
+  }
+  // 4. dalpha = sum of the partial shares + <db_b, bias_i>
+  dcb::dalpha_finish_kernel<<<d->B, dcb::kBwThreads, 0, s>>>(d->B, d->n, d->C_out, nparts, part,
                                                              db, bias, dalpha);
   rc = dc_lib::launched("dalpha_finish_kernel");
   if (rc) return rc;

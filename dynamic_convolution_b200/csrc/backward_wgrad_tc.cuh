@@ -62,7 +62,8 @@ struct WgParams {
   int co_tiles;     // ceil(Cout / 128)
   int stages;
   long long units;  // B * co_tiles * agroups
-  float* dW;
+  float* dW;        // fp32 [B][Cout][KH][KW][Cin] -- or, with hilo, two bf16 planes there
+  int hilo;         // 1: dW as bf16 hi = bf16(v) and lo = bf16(v - hi), planes [B][wsize] each
   int* err;
   long long wait_ns;
 };
@@ -229,6 +230,51 @@ __global__ void __launch_bounds__(kWgThreads, 1)
                                  a * 64 + h * 32,
                              r);
           tmem_ld_wait(r);
+          if (p.hilo) {
+            // hi / lo planes: each lane (row) stages its 32 values twice as
+            // 64 bf16 bytes (16-byte chunks XOR-ed with the row's low bits);
+            // every store instruction then writes 8 whole 64-byte row pieces
+            const long long wsize = static_cast<long long>(p.Cout) * taps * p.Cin;
+            __nv_bfloat16* hi_plane = reinterpret_cast<__nv_bfloat16*>(p.dW);
+            __nv_bfloat16* lo_plane = hi_plane + static_cast<size_t>(p.B) * wsize;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint32_t hw[4], lw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float f0 = __uint_as_float(r[8 * v + 2 * e]);
+                const float f1 = __uint_as_float(r[8 * v + 2 * e + 1]);
+                hw[e] = pack_bf16x2(f0, f1);
+                lw[e] = pack_bf16x2(f0 - bf16lo_to_f32(hw[e]), f1 - bf16hi_to_f32(hw[e]));
+              }
+              const uint32_t slot = ((v ^ (lane & 3)) << 4);
+              st_shared_v4(stg + lane * 64 + slot, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+              st_shared_v4(stg + 2048 + lane * 64 + slot, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+            }
+            __syncwarp();
+            const int ci = cb * 64 + h * 32 + 8 * (lane & 3);
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int row = 8 * it + (lane >> 2);
+              const uint32_t off = row * 64 + (((lane & 3) ^ (row & 3)) << 4);
+              uint4 vh, vl;
+              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(vh.x), "=r"(vh.y), "=r"(vh.z), "=r"(vh.w)
+                           : "r"(stg + off));
+              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(vl.x), "=r"(vl.y), "=r"(vl.z), "=r"(vl.w)
+                           : "r"(stg + 2048 + off));
+              const int co_r = cot * 128 + 32 * q + row;
+              if (co_r < p.Cout && ci < p.Cin) {
+                const size_t e = (static_cast<size_t>(b) * p.Cout + co_r) * taps * p.Cin +
+                                 static_cast<size_t>(tap) * p.Cin + ci;
+                *reinterpret_cast<uint4*>(hi_plane + e) = vh;
+                *reinterpret_cast<uint4*>(lo_plane + e) = vl;
+              }
+            }
+            __syncwarp();
+            continue;
+          }
 #pragma unroll
           for (int v = 0; v < 8; ++v)
             st_shared_v4(stg + lane * 128 + ((v ^ (lane & 7)) << 4),

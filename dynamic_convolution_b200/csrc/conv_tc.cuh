@@ -82,6 +82,9 @@ struct TcParams {
   const float* a_out; // optional [B][Cout] output channel attention (FMDConv)
   const float* chan_add;  // optional [B][Cout]: chan_scale * chan_add[b][co] joins the mixed
   float chan_scale;       // bias before the single rounding of y
+  int co_base;            // persistent kernel: channel offset of this launch in y and the biases
+  int ld_c;               // persistent kernel: channel stride of y and bias rows (0: Cout)
+  int x_early;            // persistent kernel: first x boxes may load before the grid wait
 };
 
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, int base_mode) {
@@ -493,6 +496,312 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const float* src = reinterpret_cast<const float*>(base_ptr + kTcPoolOff);
     const float t = src[threadIdx.x] + src[128 + threadIdx.x] + src[256 + threadIdx.x];
     p.ysum[(static_cast<size_t>(b) * p.tiles_h + th) * p.Cout + m0 + threadIdx.x] = t;
+  }
+}
+
+}  // namespace dc
+
+namespace dc {
+
+// ---------------------------------------------------------------------------
+// Persistent form of the PREMIX convolution: one CTA per SM walks the units
+// (sample, row block, 128-channel tile) blockIdx.x, +gridDim.x, ... with two
+// TMEM accumulators, so that the epilogue of one unit (TMEM -> bias, rounding
+// -> shared-memory transpose -> NHWC stores) runs while the MMAs of the next
+// unit accumulate into the other buffer, and the TMA producers load the next
+// unit's activations and mixed-kernel tiles meanwhile. Roles: warp 0 loads
+// activation boxes, warp 2 loads mixed-kernel tiles, warp 1 issues the MMAs,
+// warps 4..11 run the epilogue (two warps per TMEM lane quarter, alternate
+// 32-pixel chunks). A launch may cover a slice of the output channels
+// (co_base, with ld_c the full channel count) when the mixed kernels of one
+// 128-channel group at a time are in the workspace.
+// Same arithmetic, rounding and outputs as tc_conv_kernel
+// with VARIANT = kPremix; the pooled channel sums of the chained-block forward
+// are not produced here (that call runs tc_conv_kernel).
+// ---------------------------------------------------------------------------
+
+constexpr int kTpEpiWarp0 = 4;
+constexpr int kTpEpiWarps = 8;
+constexpr int kTpStageBytes = kTpEpiWarps * 2048;  // epilogue transpose tiles
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_conv_persist_kernel(const __grid_constant__ CUtensorMap xmap,
+                           const __grid_constant__ CUtensorMap wmap, TcParams p) {
+  extern __shared__ __align__(1024) unsigned char tp_smem_raw[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const uint32_t raw = smem_u32(tp_smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* base_ptr = tp_smem_raw + (base - raw);
+  const int SA = p.sa, SB = p.sb;
+  const uint32_t a_base = base;
+  const uint32_t b_base = a_base + SA * kTcATileBytes;
+  const uint32_t epi_base = b_base + SB * p.b_tile_bytes;  // 8 x 2 KB
+  const uint32_t bar_base = epi_base + kTpStageBytes;
+  auto fullA = [&](int s) { return bar_base + 8u * s; };
+  auto emptyA = [&](int s) { return bar_base + 8u * (SA + s); };
+  auto fullB = [&](int s) { return bar_base + 8u * (2 * SA + s); };
+  auto emptyB = [&](int s) { return bar_base + 8u * (2 * SA + SB + s); };
+  auto tfull = [&](int a) { return bar_base + 8u * (2 * SA + 2 * SB + a); };
+  auto tempty = [&](int a) { return bar_base + 8u * (2 * SA + 2 * SB + 2 + a); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * SA + 2 * SB + 4);
+  unsigned char* misc = base_ptr + (bar_base - base) + 8u * (2 * SA + 2 * SB + 5);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
+
+  const int units = p.B * p.tiles_h * p.m_tiles;
+  const int my_units = static_cast<int>(blockIdx.x) < units
+                           ? (units - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x
+                           : 0;
+  auto decode = [&](int i, int& b, int& h0, int& m0, int& th) {
+    int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    const int mt = u % p.m_tiles;
+    u /= p.m_tiles;
+    th = u % p.tiles_h;
+    b = u / p.tiles_h;
+    m0 = mt * 128;
+    h0 = th * p.R;
+  };
+
+  if (warp == 0) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), p.tmem_cols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(fullA(s), 1);
+      mbar_init(emptyA(s), 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(fullB(s), 1);
+      mbar_init(emptyB(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), kTpEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&xmap);
+    tma_prefetch_desc(&wmap);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // The mixing kernel this convolution follows signals its dependents only
+  // once all of its CTAs are past their own wait, so whatever wrote x has
+  // completed: the first activation boxes are loaded before this kernel's
+  // wait, overlapping the mixing kernel's tail. The mixed kernels are read
+  // only after the wait. (p.x_early is 0 when the previous kernel on the
+  // stream is not such a mixing kernel.)
+  const int pre_x = (p.x_early && my_units > 0) ? (p.kc < SB ? p.kc : SB) : 0;
+  if (warp == 0 && lane == 0 && pre_x > 0) {
+    int b, h0, m0, th;
+    decode(0, b, h0, m0, th);
+    for (int cc = 0; cc < pre_x; ++cc) {
+      mbar_arrive_expect_tx(fullB(cc), 64u * 2u * p.Wp * p.b_box_rows);
+      tma_load_4d(b_base + cc * p.b_tile_bytes, &xmap, fullB(cc), cc * 64, -p.pad, h0 - p.pad, b);
+    }
+  }
+  grid_dependency_wait();
+  const int taps = p.KH * p.KW;
+  const uint32_t acc_cols = p.tmem_cols >> 1;
+
+  if (warp == 0) {
+    // ==================== activation producer (TMA) ====================
+    if (lane == 0) {
+      const uint32_t bytes = 64u * 2u * p.Wp * p.b_box_rows;
+      int issued = 0;
+      bool ok = true;
+      for (int i = 0; i < my_units && ok; ++i) {
+        int b, h0, m0, th;
+        decode(i, b, h0, m0, th);
+        for (int cc = 0; cc < p.kc; ++cc, ++issued) {
+          if (issued < pre_x) continue;  // loaded before the wait
+          const int s = issued % SB;
+          const uint32_t ph = static_cast<uint32_t>(issued / SB) & 1u;
+          if (!wait_bounded(emptyB(s), ph ^ 1u, ctl, kErrWaitProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(fullB(s), bytes);
+          tma_load_4d(b_base + s * p.b_tile_bytes, &xmap, fullB(s), cc * 64, -p.pad, h0 - p.pad, b);
+        }
+      }
+      for (int j = (issued > SB ? issued - SB : 0); j < issued; ++j)
+        wait_drain(fullB(j % SB), static_cast<uint32_t>(j / SB) & 1u, p.wait_ns, p.err);
+    }
+  } else if (warp == 2) {
+    // ==================== mixed-kernel producer (TMA) ====================
+    if (lane == 0) {
+      int issued = 0;
+      bool ok = true;
+      for (int i = 0; i < my_units && ok; ++i) {
+        int b, h0, m0, th;
+        decode(i, b, h0, m0, th);
+        int cc = 0, tap = 0;
+        for (int k = 0; k < p.k_steps; ++k, ++issued) {
+          const int s = issued % SA;
+          const uint32_t ph = static_cast<uint32_t>(issued / SA) & 1u;
+          if (!wait_bounded(emptyA(s), ph ^ 1u, ctl, kErrWaitProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(fullA(s), kTcATileBytes);
+          tma_load_3d(a_base + s * kTcATileBytes, &wmap, fullA(s), cc * 64, tap, b * p.Cout + m0);
+          if (++tap == p.spc) { tap = 0; ++cc; }
+        }
+      }
+      for (int j = (issued > SA ? issued - SA : 0); j < issued; ++j)
+        wait_drain(fullA(j % SA), static_cast<uint32_t>(j / SA) & 1u, p.wait_ns, p.err);
+    }
+  } else if (warp == 1) {
+    // ============================ MMA issuer ============================
+    if (lane == 0) {
+      const uint32_t idesc0 = idesc_bf16_f32(128, p.n_mma0);
+      const uint64_t a_desc0 = tc_desc(a_base, 0);
+      const uint64_t b_desc0 = tc_desc(b_base, p.desc_base_mode);
+      const uint64_t b_stage = static_cast<uint64_t>(p.b_tile_bytes) >> 4;
+      const uint64_t row_skip = static_cast<uint64_t>(p.Wp - p.KW + 1) * 8u;
+      uint32_t s = 0, ph = 0, sbi = 0, phb = 0;
+      bool ok = true;
+      for (int i = 0; i < my_units && ok; ++i) {
+        const int ab = i & 1;
+        const uint32_t d = tmem_base + ab * acc_cols;
+        if (!wait_bounded(tempty(ab), (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u, ctl, kErrWaitMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        int t = 0, tap = 0, kw = 0;
+        uint64_t tap_off = 0;
+        if (!wait_bounded(fullB(sbi), phb, ctl, kErrWaitMma) ||
+            !wait_bounded(fullA(s), ph, ctl, kErrWaitMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int k = 0; k < p.k_steps && ok; ++k) {
+          const uint64_t ad = a_desc0 + s * (kTcATileBytes >> 4);
+          const uint64_t bd = b_desc0 + sbi * b_stage + tap_off;
+          tc_mma_f16(d, ad, bd, idesc0, k > 0 ? 1u : 0u);
+#pragma unroll
+          for (int q = 1; q < 3; ++q) tc_mma_f16(d, ad + 2 * q, bd + 2 * q, idesc0, 1u);
+          const uint32_t s_cur = s, sbi_cur = sbi;
+          bool chunk_end = false;
+          if (++tap == taps) {
+            tap = 0; kw = 0; tap_off = 0;
+          } else if (++kw == p.KW) {
+            kw = 0; tap_off += row_skip;
+          } else {
+            tap_off += 8u;
+          }
+          if (++t == p.spc) {
+            t = 0;
+            chunk_end = true;
+            if (++sbi == static_cast<uint32_t>(SB)) { sbi = 0; phb ^= 1u; }
+          }
+          if (++s == static_cast<uint32_t>(SA)) { s = 0; ph ^= 1u; }
+          if (k + 1 < p.k_steps) {
+            if (chunk_end && !wait_bounded(fullB(sbi), phb, ctl, kErrWaitMma)) ok = false;
+            if (ok && !wait_bounded(fullA(s), ph, ctl, kErrWaitMma)) ok = false;
+            if (ok) tc_fence_after();
+          }
+          tc_mma_f16(d, ad + 6, bd + 6, idesc0, 1u);
+          tc_commit(emptyA(s_cur));
+          if (chunk_end) tc_commit(emptyB(sbi_cur));
+        }
+        if (ok) tc_commit(tfull(ab));
+      }
+      if (!ok) {
+        tc_commit(drain_bar);
+        wait_drain(drain_bar, 0, p.wait_ns, p.err);
+      }
+    }
+  } else if (warp >= kTpEpiWarp0) {
+    // ============================= epilogue =============================
+    const int q = warp & 3;                    // TMEM lane quarter
+    const int grp = (warp - kTpEpiWarp0) >> 2;  // chunk phase 0..1
+    const uint32_t stage = epi_base + (warp - kTpEpiWarp0) * 2048;
+    const int part = lane & 3;
+    const int nchunks = (p.n_mma0 + 31) / 32;
+    const int ldc = p.ld_c > 0 ? p.ld_c : p.Cout;  // channel stride of y and bias rows
+    const int cb = p.co_base;                       // channel offset of this launch
+    for (int i = 0; i < my_units; ++i) {
+      const int ab = i & 1;
+      int b, h0, m0, th;
+      decode(i, b, h0, m0, th);
+      const int co = m0 + 32 * q + lane;  // channel of this launch; cb + co in y and the biases
+      float bb = 0.f;
+      if (p.bias != nullptr && co < p.Cout) {
+        const float* al = p.alpha + static_cast<size_t>(b) * p.n;
+        for (int e = 0; e < p.n; ++e) bb = fmaf(al[e], p.bias[static_cast<size_t>(e) * ldc + cb + co], bb);
+      }
+      if (p.chan_add != nullptr && co < p.Cout)
+        bb = fmaf(p.chan_add[static_cast<size_t>(b) * ldc + cb + co], p.chan_scale, bb);
+      const float so = (p.a_out != nullptr && co < p.Cout) ? p.a_out[static_cast<size_t>(b) * ldc + cb + co] : 1.f;
+      if (!wait_bounded(tfull(ab), static_cast<uint32_t>(i >> 1) & 1u, ctl, kErrWaitEpilogue)) break;
+      tc_fence_after();
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * acc_cols;
+      const int c8 = m0 + 32 * q + part * 8;
+      const bool c_ok = c8 < p.Cout;
+      __nv_bfloat16* ybase = p.y + static_cast<size_t>(b) * p.H * p.W * ldc + cb + c8;
+      auto process = [&](const uint32_t (&r)[32], int ch) {
+#pragma unroll
+        for (int jj = 0; jj < 32; jj += 2) {
+          const uint32_t w = pack_bf16x2((__uint_as_float(r[jj]) + bb) * so,
+                                         (__uint_as_float(r[jj + 1]) + bb) * so);
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + jj * 64 + lane * 2),
+                       "h"(static_cast<unsigned short>(w & 0xFFFFu))
+                       : "memory");
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + (jj + 1) * 64 + lane * 2),
+                       "h"(static_cast<unsigned short>(w >> 16))
+                       : "memory");
+        }
+        __syncwarp();
+        int pix = ch * 32 + (lane >> 2);
+        int rr = pix / p.Wp;
+        int cw = pix - rr * p.Wp;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int oh = h0 + rr;
+          if (c_ok && pix < p.n_virt && cw < p.W && oh < p.H) {
+            uint4 v;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(stage + (it * 8 + (lane >> 2)) * 64 + part * 16));
+            *reinterpret_cast<uint4*>(ybase + (static_cast<size_t>(oh) * p.W + cw) * ldc) = v;
+          }
+          pix += 8;
+          cw += 8;
+          while (cw >= p.Wp) { cw -= p.Wp; ++rr; }
+        }
+        __syncwarp();
+      };
+      uint32_t ra[32], rb[32];
+      int ch = grp;
+      if (ch < nchunks) tmem_ld_32x32b_x32(trow + ch * 32, ra);
+      while (ch < nchunks) {
+        tmem_ld_wait(ra);
+        if (ch + 2 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 2) * 32, rb);
+        process(ra, ch);
+        ch += 2;
+        if (ch >= nchunks) break;
+        tmem_ld_wait(rb);
+        if (ch + 2 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 2) * 32, ra);
+        process(rb, ch);
+        ch += 2;
+      }
+      // this warp's reads of the accumulator are complete: release it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty(ab));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 

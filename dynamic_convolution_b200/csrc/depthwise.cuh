@@ -25,6 +25,8 @@
 //    are conflict-free and the NHWC stores coalesce.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace dc {
@@ -218,6 +220,302 @@ __global__ void __launch_bounds__(kDwThreads, K <= 5 ? 2 : 1)
                           __uint_as_float(static_cast<uint32_t>(s1 >> 32)));
       }
     }
+  }
+}
+
+}  // namespace dc
+
+namespace dc {
+
+// ---------------------------------------------------------------------------
+// Pipelined depthwise kernel (the default when the expert slab fits).
+//
+// The same layer arithmetic as depthwise_kernel above, organised so that HBM
+// and the FMA pipe stay busy together:
+//  * persistent CTAs, one per SM; CTA i owns the channel chunk i % nchunks for
+//    its whole life and walks the tiles (sample, row band, column band) of that
+//    chunk with stride = the number of CTAs sharing the chunk;
+//  * the chunk's expert slabs [n][CC][K*K] (and bias slabs) are copied into
+//    shared memory once per CTA by bulk copies and stay resident;
+//  * a producer warp keeps S tiles in flight: per tile one 4-D TMA box of the
+//    zero-padded input window {CC channels, CB+K-1 columns, RB+K-1 rows}, plus
+//    the sample's attentions (and channel factors) stored by its lanes;
+//  * the compute warps first mix the tile's kernels together (CC*K*K weights,
+//    CC biases, fp32, from the resident slabs) into the stage, then each thread
+//    takes TWO adjacent output columns of ONE channel pair and walks the input
+//    rows of the band: for every input row it loads K+1 packed pairs and adds
+//    them into the K output rows (x 2 columns) that use that input row
+//    (vertical accumulators, packed fp32x2 FMAs: 2*K*K per row for K+1 loads);
+//    an output row is stored when its last input row is in. The rows are
+//    walked in groups of K with every accumulator slot a compile-time
+//    register; only the first and the last groups carry the band-edge tests.
+//    Consecutive threads take consecutive channel pairs of one column pair,
+//    so with 32 or 64 pairs per chunk a warp's loads are conflict-free.
+// Every wait is bounded (mbarriers only, no named barriers); on expiry the
+// CTA raises its abort flag, the producer drains its in-flight copies, and
+// all warps leave.
+// ---------------------------------------------------------------------------
+
+template <int K>
+struct DwpShape;
+// Compute threads per CTA and the register cap that fits them (plus the
+// producer warp) in one SM's 64 K registers -- registers are granted to warps
+// in groups of four, so the cap is 64 K / (32 * warps rounded up to 4),
+// rounded down to 8: the K*K packed weights stay in registers for the whole
+// tile.
+template <>
+struct DwpShape<3> { static constexpr int kComp = 992; static constexpr int kRegs = 64; };
+template <>
+struct DwpShape<5> { static constexpr int kComp = 480; static constexpr int kRegs = 128; };
+template <>
+struct DwpShape<7> { static constexpr int kComp = 352; static constexpr int kRegs = 168; };
+
+constexpr int kDwpMaxStages = 4;
+constexpr int kErrWaitDwp = 0x108;
+
+struct DwpParams {
+  int B, C, H, W, pad, n, Ho, Wo;
+  int CC;           // channels per chunk (multiple of 8)
+  int CB;           // output columns per tile
+  int RB;           // output rows per tile
+  int nchunks, bands, cbands;
+  int S;            // stages in flight
+  int stage_bytes;  // one stage: box | weights | misc (128-aligned)
+  int box_bytes;    // (RB+K-1) * (even(CB)+K-1) * CC * 2
+  int wst_off;      // weights [K*K][CC/2] packed pairs, from the stage base
+  int misc_off;     // alpha[n] | a_in[CC] | a_out[CC] | chan_add[CC], from the stage base
+  int e_off;        // resident expert slabs [n][CC][K*K] bf16
+  int eb_off;       // resident bias slabs [n][CC] fp32
+  int bar_off;
+  const __nv_bfloat16* experts;  // [n][C][K][K]
+  const float* alpha;            // [B][n]
+  const float* bias;             // [n][C] or null
+  __nv_bfloat16* y;
+  const float* a_in;             // [B][C] or null
+  const float* a_out;            // [B][C] or null
+  const float* chan_add;         // [B][C] or null
+  float chan_scale;
+  int* err;
+  long long wait_ns;
+};
+
+template <int K>
+__global__ void __maxnreg__(DwpShape<K>::kRegs)
+    depthwise_pipe_kernel(const __grid_constant__ CUtensorMap xmap, DwpParams p) {
+  constexpr int KK = K * K;
+  constexpr int NCOMP = DwpShape<K>::kComp;
+  constexpr int NWARP_C = NCOMP / 32;
+  extern __shared__ __align__(128) unsigned char dwp_raw[];
+  unsigned char* sm = dwp_raw + ((128u - (smem_u32(dwp_raw) & 127u)) & 127u);
+  const int t = threadIdx.x;
+  const int warp = t >> 5, lane = t & 31;
+  const int CCp = p.CC >> 1;
+  const int TC = ((p.CB + 1) & ~1) + K - 1;  // staged columns: even tile width + halo
+
+  // this CTA's chunk and its share of the chunk's tiles
+  const int chunk = blockIdx.x % p.nchunks;
+  const int local = blockIdx.x / p.nchunks;
+  const int sharers = (gridDim.x - chunk + p.nchunks - 1) / p.nchunks;
+  const int c0 = chunk * p.CC;
+  const int cc_valid = min(p.CC, p.C - c0);
+  const int tiles = p.B * p.bands * p.cbands;
+  const int my_tiles = local < tiles ? (tiles - local + sharers - 1) / sharers : 0;
+
+  const uint32_t bar0 = smem_u32(sm + p.bar_off);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (kDwpMaxStages + s); };
+  auto mixed = [&](int s) { return bar0 + 8u * (2 * kDwpMaxStages + s); };
+  const uint32_t ebar = bar0 + 8u * (3 * kDwpMaxStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.bar_off + 8 * (3 * kDwpMaxStages + 1));
+  const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
+  const __nv_bfloat16* ebuf = reinterpret_cast<const __nv_bfloat16*>(sm + p.e_off);
+  const float* ebias = reinterpret_cast<const float*>(sm + p.eb_off);
+
+  if (t == 0) {
+    for (int s = 0; s < kDwpMaxStages; ++s) {
+      mbar_init(full(s), 33);        // producer lane 0's expect-tx arrive + 32 lane arrives
+      mbar_init(empty(s), NWARP_C);  // one arrive per compute warp
+      mbar_init(mixed(s), NWARP_C);
+    }
+    mbar_init(ebar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&xmap);
+  }
+  __syncthreads();
+  grid_dependency_wait();  // alpha (and x) come from earlier kernels
+
+  auto tile_coords = [&](int k, int& b, int& oh0, int& ow0) {
+    int u = local + k * sharers;
+    const int cb = u % p.cbands;
+    u /= p.cbands;
+    const int band = u % p.bands;
+    b = u / p.bands;
+    oh0 = band * p.RB;
+    ow0 = cb * p.CB;
+  };
+
+  if (warp == NWARP_C) {
+    // =============================== producer ===============================
+    if (my_tiles > 0 && lane == 0) {
+      const uint32_t eb = static_cast<uint32_t>(cc_valid) * KK * 2;
+      const uint32_t bb = p.bias ? static_cast<uint32_t>(cc_valid) * 4 : 0u;
+      mbar_arrive_expect_tx(ebar, static_cast<uint32_t>(p.n) * (eb + bb));
+      for (int i = 0; i < p.n; ++i) {
+        bulk_load(smem_u32(sm + p.e_off) + static_cast<uint32_t>(i) * p.CC * KK * 2,
+                  p.experts + (static_cast<size_t>(i) * p.C + c0) * KK, eb, ebar);
+        if (p.bias)
+          bulk_load(smem_u32(sm + p.eb_off) + static_cast<uint32_t>(i) * p.CC * 4,
+                    p.bias + static_cast<size_t>(i) * p.C + c0, bb, ebar);
+      }
+    }
+    int issued = 0;
+    for (int k = 0; k < my_tiles; ++k) {
+      const int s = k % p.S;
+      const uint32_t ph = static_cast<uint32_t>(k / p.S) & 1u;
+      if (!wait_bounded(empty(s), ph ^ 1u, ctl, kErrWaitDwp)) break;
+      int b, oh0, ow0;
+      tile_coords(k, b, oh0, ow0);
+      unsigned char* st = sm + static_cast<size_t>(s) * p.stage_bytes;
+      float* misc = reinterpret_cast<float*>(st + p.misc_off);
+      for (int j = lane; j < p.n; j += 32) misc[j] = p.alpha[static_cast<size_t>(b) * p.n + j];
+      float* fin = misc + p.n;
+      for (int c = lane; c < cc_valid; c += 32) {
+        const size_t o = static_cast<size_t>(b) * p.C + c0 + c;
+        fin[c] = p.a_in ? p.a_in[o] : 1.f;
+        fin[p.CC + c] = p.a_out ? p.a_out[o] : 1.f;
+        fin[2 * p.CC + c] = p.chan_add ? p.chan_add[o] * p.chan_scale : 0.f;
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(full(s), static_cast<uint32_t>(p.box_bytes));
+        tma_load_4d(smem_u32(st), &xmap, full(s), c0, ow0 - p.pad, oh0 - p.pad, b);
+      }
+      __syncwarp();
+      mbar_arrive(full(s));
+      ++issued;
+    }
+    if (lane == 0) {
+      // leave no copy in flight: the last S issued tiles (the compute warps
+      // consumed the rest), and the resident slabs
+      for (int j = (issued > p.S ? issued - p.S : 0); j < issued; ++j)
+        wait_drain(full(j % p.S), static_cast<uint32_t>(j / p.S) & 1u, p.wait_ns, p.err);
+      if (my_tiles > 0) wait_drain(ebar, 0, p.wait_ns, p.err);
+    }
+    return;
+  }
+
+  // ================================ compute ================================
+  if (my_tiles == 0) return;
+  if (!wait_bounded(ebar, 0, ctl, kErrWaitDwp)) return;
+  const int cpair = t / CCp, pair = t - (t / CCp) * CCp;
+  const int col = 2 * cpair;  // this thread's output columns col, col + 1 in the tile
+  for (int k = 0; k < my_tiles; ++k) {
+    const int s = k % p.S;
+    const uint32_t ph = static_cast<uint32_t>(k / p.S) & 1u;
+    if (!wait_bounded(full(s), ph, ctl, kErrWaitDwp)) return;
+    int b, oh0, ow0;
+    tile_coords(k, b, oh0, ow0);
+    unsigned char* st = sm + static_cast<size_t>(s) * p.stage_bytes;
+    const float* misc = reinterpret_cast<const float*>(st + p.misc_off);
+    const float* fin = misc + p.n;
+    float* wst = reinterpret_cast<float*>(st + p.wst_off);  // [KK][CCp][2]
+    float* bst = wst + KK * p.CC;                            // [CC] mixed bias (+ term)
+
+    // ---- mix this tile's kernels: tap-major items, consecutive channels
+    for (int it = t; it < (KK + 1) * p.CC; it += NCOMP) {
+      const int tap = it / p.CC, c = it - (it / p.CC) * p.CC;
+      if (c >= cc_valid) continue;
+      float sacc = 0.f;
+      if (tap < KK) {
+        for (int j = 0; j < p.n; ++j)
+          sacc = fmaf(misc[j], __bfloat162float(ebuf[(static_cast<size_t>(j) * p.CC + c) * KK + tap]),
+                      sacc);
+        wst[tap * p.CC + c] = sacc * fin[c];  // input attention folded (depthwise: one channel)
+      } else {
+        if (p.bias)
+          for (int j = 0; j < p.n; ++j) sacc = fmaf(misc[j], ebias[j * p.CC + c], sacc);
+        bst[c] = sacc + fin[2 * p.CC + c];
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(mixed(s));
+    if (!wait_bounded(mixed(s), ph, ctl, kErrWaitDwp)) return;
+
+    const int ow = ow0 + col;
+    const int c = c0 + 2 * pair;
+    const bool active = col < p.CB && ow < p.Wo && c < p.C;
+    if (active) {
+      uint64_t w2[KK];
+#pragma unroll
+      for (int q = 0; q < KK; ++q)
+        w2[q] = *reinterpret_cast<const uint64_t*>(wst + q * p.CC + 2 * pair);
+      const uint64_t bias2 = *reinterpret_cast<const uint64_t*>(bst + 2 * pair);
+      const float ao0 = fin[p.CC + 2 * pair], ao1 = fin[p.CC + 2 * pair + 1];
+      const bool scale_out = p.a_out != nullptr;
+      const bool second = col + 1 < p.CB && ow + 1 < p.Wo;  // the column pair's second column
+      const uint32_t* xw = reinterpret_cast<const uint32_t*>(st) + col * CCp + pair;
+      const int row_words = TC * CCp;
+      __nv_bfloat16* yb = p.y + (static_cast<size_t>(b) * p.Ho * p.Wo + ow) * p.C + c;
+      const int rows_in = p.RB + K - 1;
+      uint64_t acc[K][2];
+#pragma unroll
+      for (int q = 0; q < K; ++q) acc[q][0] = acc[q][1] = bias2;
+      auto store_row = [&](uint64_t (&a)[2], int o) {
+        const int oh = oh0 + o;
+        if (oh < p.Ho) {
+          __nv_bfloat16* dst = yb + static_cast<size_t>(oh) * p.Wo * p.C;
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            float lo = __uint_as_float(static_cast<uint32_t>(a[v]));
+            float hi = __uint_as_float(static_cast<uint32_t>(a[v] >> 32));
+            if (scale_out) { lo *= ao0; hi *= ao1; }
+            if (v == 0 || second)
+              *reinterpret_cast<uint32_t*>(dst + v * p.C) = pack_bf16x2(lo, hi);
+          }
+        }
+      };
+      // One group of K input rows starting at ir0 (a multiple of K): for input
+      // row ir the output rows o = ir - kh; row ir - (K-1) completes. GUARDED
+      // groups test the band edges (o < 0, o >= RB, ir >= rows_in).
+      auto group = [&](int ir0, auto guarded) {
+        constexpr bool G = decltype(guarded)::value;
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+          const int ir = ir0 + j;
+          if (G && ir >= rows_in) break;
+          const uint32_t* xr = xw + ir * row_words;
+          uint64_t xv[K + 1];
+#pragma unroll
+          for (int kw = 0; kw <= K; ++kw) xv[kw] = bf16x2_to_f32x2(xr[kw * CCp]);
+#pragma unroll
+          for (int kh = K - 1; kh >= 0; --kh) {
+            const int o = ir - kh;
+            if (G && (o < 0 || o >= p.RB)) continue;
+            const int slot = (j - kh + K) % K;  // o % K
+#pragma unroll
+            for (int kw = 0; kw < K; ++kw) {
+              acc[slot][0] = ffma2(xv[kw], w2[kh * K + kw], acc[slot][0]);
+              acc[slot][1] = ffma2(xv[kw + 1], w2[kh * K + kw], acc[slot][1]);
+            }
+            if (kh == K - 1) {
+              store_row(acc[slot], o);
+              acc[slot][0] = acc[slot][1] = bias2;
+            }
+          }
+        }
+      };
+      // groups wholly inside the band (every o in [0, RB)): ir0 >= K and
+      // ir0 + K - 1 < RB; the others are guarded
+      const int inner_end = p.RB >= K ? (p.RB - K + 1 + K - 1) / K * K : K;  // first ir0 > RB - K
+      group(0, std::true_type{});
+#pragma unroll 1
+      for (int ir0 = K; ir0 < inner_end && ir0 <= p.RB - K; ir0 += K) group(ir0, std::false_type{});
+#pragma unroll 1
+      for (int ir0 = (inner_end > K ? inner_end : K); ir0 < rows_in; ir0 += K)
+        group(ir0, std::true_type{});
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty(s));
   }
 }
 

@@ -11,6 +11,7 @@
 #include <map>
 #include <mutex>
 #include <utility>
+#include <vector>
 
 #include "dynconv.h"
 #include "internal.h"
@@ -21,6 +22,7 @@
 #include "direct.cuh"
 #include "premix.cuh"
 #include "premix_small.cuh"
+#include "premix_t.cuh"
 #include "mixconv.cuh"
 #include "route.cuh"
 #include "pool.cuh"
@@ -60,6 +62,12 @@ std::atomic<int> g_route_split{0};  // 0: automatic
 std::atomic<int> g_use_pdl{1};      // programmatic launch edges on forward kernels
 std::atomic<int> g_stream_mix{0};   // PREMIX with n <= 8: mixing streamed into the convolution
 std::atomic<int> g_premix_mixer{0};  // 0 automatic, 1 tensor-core GEMM, 2 CUDA cores (n <= 8)
+std::atomic<int> g_dw_kernel{0};     // 0 pipelined depthwise kernel when it fits, 1 the per-tile one
+std::atomic<int> g_conv_persist{1};  // PREMIX convolution: 1 persistent kernel when it fits, 0 one CTA per unit
+std::atomic<int> g_group_mix{1};     // PREMIX, n > 8, large B*|W|: 1 grouped mixing pipeline, 0 one pass
+std::atomic<int> g_mixgrad_tc{1};    // backward: 1 tensor-core mixing gradient when it fits, 0 CUDA cores
+std::atomic<long long> g_group_bytes{40LL << 20};  // target bytes of one group's mixed kernels
+std::atomic<long long> g_group_min{64LL << 20};    // below this B*|W| the one-pass form is used
 thread_local char g_last_err[256] = "";
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -264,11 +272,151 @@ bool tc_plan(const dynconv_desc* d, int variant, int sms, int max_smem, TcPlan* 
   return true;
 }
 
+// Plan of the persistent PREMIX convolution (tc_conv_persist_kernel): two
+// TMEM accumulators of up to 256 columns each, so row blocks of at most 256
+// padded pixels; one CTA per SM. Cost (cycles of the busiest CTA): its units
+// times the slowest of MMA issue (2 * N_pad per K step), operand bytes
+// (16 KB per step at ~20 B/clk from L2), the epilogue (~4 cycles per padded
+// pixel column) and the unit's HBM bytes at its share of the bandwidth
+// (~23 B/clk per SM); plus one epilogue and a fixed set-up.
+bool tc_plan_persist(const dynconv_desc* d, int sms, int max_smem, TcPlan* out) {
+  if (!tc_shape_ok(d)) return false;
+  const int taps = d->KH * d->KW;
+  const int kc = (d->C_in + 63) / 64;
+  const int m_tiles = (d->C_out + 127) / 128;
+  const int k_steps = kc * taps;
+  const int Wp = d->W + d->KW - 1;
+  if (Wp > 256) return false;
+  const int s_tap_max = (d->KH - 1) * Wp + (d->KW - 1);
+  bool found = false;
+  TcPlan best;
+  for (int R = 1; R <= d->H; ++R) {
+    const int n_virt = R * Wp;
+    const int n_pad = (n_virt + 15) / 16 * 16;
+    if (n_pad > 256) break;
+    const int box_rows = R + d->KH - 1;
+    if (box_rows > 256) break;
+    const int rows = std::max(box_rows * Wp, s_tap_max + n_pad);
+    const int b_tile = (rows * 128 + 1023) / 1024 * 1024;
+    const size_t fixed = 1024 + dc::kTpStageBytes + 8 * 64 + 16;
+    const int sb = kc > 1 ? 2 : 1;
+    if (fixed + sb * static_cast<size_t>(b_tile) + 2 * dc::kTcATileBytes > static_cast<size_t>(max_smem))
+      continue;
+    int sa = static_cast<int>((max_smem - fixed - sb * static_cast<size_t>(b_tile)) / dc::kTcATileBytes);
+    sa = std::min(sa, std::max(2, std::min(8, k_steps + 2)));
+    const int tiles_h = (d->H + R - 1) / R;
+    const long long units = 1LL * d->B * tiles_h * m_tiles;
+    const long long grid = std::min<long long>(units, sms);
+    const long long per_cta = (units + grid - 1) / grid;
+    const double mma = k_steps * std::max(2.0 * n_pad, 16384.0 / 20.0);
+    const double epi = 4.0 * n_pad;
+    const double bytes = 2.0 * (static_cast<double>(kc) * 64 * Wp * box_rows + 128.0 * R * d->W) +
+                         16384.0 * k_steps;
+    const double t_unit = std::max({mma, epi, bytes / 23.0});
+    const double cost = per_cta * t_unit + epi + 3000.0;
+    if (!found || cost < best.cost) {
+      found = true;
+      best.cost = cost;
+      best.grid = static_cast<int>(grid);
+      best.smem = fixed + sb * static_cast<size_t>(b_tile) + sa * static_cast<size_t>(dc::kTcATileBytes);
+      dc::TcParams& p = best.p;
+      std::memset(&p, 0, sizeof(p));
+      p.B = d->B; p.H = d->H; p.W = d->W; p.Cin = d->C_in; p.Cout = d->C_out;
+      p.KH = d->KH; p.KW = d->KW; p.pad = d->pad; p.n = d->n;
+      p.R = R; p.tiles_h = tiles_h; p.m_tiles = m_tiles; p.Wp = Wp; p.n_virt = n_virt;
+      p.n_mma0 = n_pad; p.n_mma1 = 0; p.kc = kc; p.spc = taps; p.k_steps = k_steps;
+      p.sa = sa; p.sb = sb; p.b_tile_bytes = b_tile; p.b_box_rows = box_rows;
+      p.desc_base_mode = g_desc_base_mode;
+      uint32_t cols = 32;
+      while (cols < static_cast<uint32_t>(n_pad)) cols <<= 1;
+      p.tmem_cols = 2 * cols;
+    }
+  }
+  if (!found || best.grid <= 0) return false;
+  *out = best;
+  return true;
+}
+
 bool depthwise_ok(const dynconv_desc* d) {
   return d->dtype == DYNCONV_BF16 && d->groups == d->C_in && d->C_in == d->C_out &&
          d->stride == 1 && d->KH == d->KW && (d->KH == 3 || d->KH == 5 || d->KH == 7) &&
          d->C_in % 8 == 0 && d->n <= 4096 && out_size(d->H, d->KH, 1, d->pad) >= 1 &&
          out_size(d->W, d->KW, 1, d->pad) >= 1;
+}
+
+// Plan of the pipelined depthwise kernel (depthwise_pipe_kernel): chunk width
+// CC and tile width CB so that the CC/2 x CB compute threads fill the kernel's
+// thread count with the least waste (idle threads, channels past C, columns
+// past W_out); then the tallest row band RB for which three stages, the
+// resident expert and bias slabs and the barriers fit in shared memory (two
+// stages when three do not fit). False when the shape does not fit.
+bool dwp_plan(const dynconv_desc* d, int sms, int max_smem, bool has_bias, dc::DwpParams* p,
+              int* grid, size_t* smem_out) {
+  const int K = d->KH, KK = K * K;
+  const int ncomp = K == 3 ? dc::DwpShape<3>::kComp : K == 5 ? dc::DwpShape<5>::kComp
+                                                            : dc::DwpShape<7>::kComp;
+  const int Ho = out_size(d->H, K, 1, d->pad), Wo = out_size(d->W, K, 1, d->pad);
+  const int C = d->C_in;
+  double best = -1;
+  int bCC = 0, bCB = 0;
+  for (int CC = 8; CC <= std::min(256, (C + 7) / 8 * 8); CC += 8) {
+    const int nch = (C + CC - 1) / CC;
+    for (int CB = 1; CB <= std::min(Wo, 254 - (K - 1)); ++CB) {
+      const int thr = CC / 2 * ((CB + 1) / 2);  // one thread per channel pair and column pair
+      if (thr > ncomp) break;
+      const int cbands = (Wo + CB - 1) / CB;
+      // the halo columns are staged for every tile: a mild preference for wide
+      // tiles; a warp of 32 consecutive pairs of one column pair reads without
+      // bank conflicts, other chunk widths with some
+      const double eff = static_cast<double>(thr) / ncomp * C / (nch * CC) * Wo / (cbands * CB) *
+                         (1.0 - 0.25 * (K - 1) / (CB + K - 1.0)) *
+                         ((CC / 2) % 32 == 0 ? 1.0 : 0.85);
+      if (eff > best + 1e-9) { best = eff; bCC = CC; bCB = CB; }
+    }
+  }
+  if (bCC == 0) return false;
+  const int CC = bCC, CB = bCB;
+  auto a128 = [](size_t v) { return (v + 127) / 128 * 128; };
+  const size_t e_bytes = a128(static_cast<size_t>(d->n) * CC * KK * 2);
+  const size_t eb_bytes = has_bias ? a128(static_cast<size_t>(d->n) * CC * 4) : 0;
+  const size_t wst_bytes = a128(static_cast<size_t>(KK + 1) * CC * 4);
+  const size_t misc_bytes = a128(static_cast<size_t>(d->n + 3 * CC) * 4);
+  const size_t bars = 8 * (3 * dc::kDwpMaxStages + 1) + 16;
+  const int TC = ((CB + 1) & ~1) + K - 1;  // staged columns
+  auto stage_of = [&](int RB) {
+    return a128(static_cast<size_t>(RB + K - 1) * TC * CC * 2) + wst_bytes + misc_bytes;
+  };
+  int S = 0, RBmax = 0;
+  for (int st : {3, 2}) {
+    int rb = std::min(Ho, 256 - (K - 1));
+    while (rb > 0 && 128 + st * stage_of(rb) + e_bytes + eb_bytes + bars >
+                         static_cast<size_t>(max_smem))
+      --rb;
+    if (rb > 0 && (rb >= std::min(Ho, 8) || st == 2)) { S = st; RBmax = rb; break; }
+  }
+  if (S == 0 || RBmax == 0) return false;
+  const int bands = (Ho + RBmax - 1) / RBmax;
+  const int RB = (Ho + bands - 1) / bands;
+  std::memset(p, 0, sizeof(*p));
+  p->B = d->B; p->C = C; p->H = d->H; p->W = d->W; p->pad = d->pad; p->n = d->n;
+  p->Ho = Ho; p->Wo = Wo; p->CC = CC; p->CB = CB; p->RB = RB;
+  p->nchunks = (C + CC - 1) / CC;
+  p->bands = bands;
+  p->cbands = (Wo + CB - 1) / CB;
+  p->S = S;
+  p->box_bytes = (RB + K - 1) * TC * CC * 2;
+  p->wst_off = static_cast<int>(a128(static_cast<size_t>(p->box_bytes)));
+  p->misc_off = p->wst_off + static_cast<int>(wst_bytes);
+  p->stage_bytes = p->misc_off + static_cast<int>(misc_bytes);
+  p->e_off = S * p->stage_bytes;
+  p->eb_off = p->e_off + static_cast<int>(e_bytes);
+  p->bar_off = p->eb_off + static_cast<int>(eb_bytes);
+  const long long tiles_per_chunk = 1LL * d->B * p->bands * p->cbands;
+  const long long g = std::min<long long>(std::max(sms, p->nchunks), p->nchunks * tiles_per_chunk);
+  if (g <= 0 || g > (1 << 30)) return false;
+  *grid = static_cast<int>(g);
+  *smem_out = 128 + static_cast<size_t>(p->bar_off) + bars;
+  return *smem_out <= static_cast<size_t>(max_smem);
 }
 
 // Workspace of PREMIX: the mixed kernels of every sample (256-byte aligned).
@@ -373,6 +521,242 @@ int launch_tc(const TcPlan& plan, const CUtensorMap& xmap, const CUtensorMap& wm
   return check_launch("tc_conv_kernel");
 }
 
+
+// The PREMIX convolution on mixed kernels already in the workspace: the
+// persistent kernel when its plan exists, no pooled sums are asked for and it
+// pays -- a CTA gets three or more units, or a unit has at most four K steps
+// (its epilogue, not its MMAs, is then the unit's cost). With one or two
+// MMA-bound units per CTA the persistent kernel issues as many MMAs per CTA as
+// one CTA per (larger) unit does, while the epilogue of the first unit runs
+// beside the MMA-issuing thread of the second and delays it; measured on the
+// 3x3 layer (B=64, 128 channels, 28x28): 30.1 us against 26.4 us per forward.
+// Else one CTA per unit.
+int launch_premix_conv(const dynconv_desc* d, const TcPlan& plan, const DeviceState* st,
+                       const void* x, const CUtensorMap& xmap, const CUtensorMap& wmap,
+                       cudaStream_t stream) {
+  TcPlan pp;
+  const bool have = g_conv_persist.load() && plan.p.ysum == nullptr &&
+                    tc_plan_persist(d, st->sms, st->max_smem_optin, &pp);
+  const int units = have ? pp.p.B * pp.p.tiles_h * pp.p.m_tiles : 0;
+  const bool pays = have && ((units + pp.grid - 1) / pp.grid >= 3 || pp.p.k_steps <= 4);
+  if (pays || (have && g_conv_persist.load() == 2)) {
+    const dc::TcParams& q = plan.p;
+    pp.p.experts = q.experts; pp.p.alpha = q.alpha; pp.p.bias = q.bias; pp.p.y = q.y;
+    pp.p.err = q.err; pp.p.wait_ns = q.wait_ns; pp.p.a_out = q.a_out;
+    pp.p.chan_add = q.chan_add; pp.p.chan_scale = q.chan_scale;
+    // launched right after one of this library's mixing kernels (they signal
+    // dependents only past their own wait), with a programmatic edge
+    pp.p.x_early = g_use_pdl.load() ? 1 : 0;
+    CUtensorMap pxmap;
+    int rc = encode_x_map(&pxmap, x, d, pp.p.Wp, pp.p.b_box_rows);
+    if (rc) return rc;
+    cudaError_t e = ensure_smem(dc::tc_conv_persist_kernel, pp.smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc_conv_persist)");
+    e = launch_pdl(dc::tc_conv_persist_kernel, dim3(pp.grid), dim3(dc::kTcThreads), pp.smem,
+                   stream, pxmap, wmap, pp.p);
+    if (e != cudaSuccess) {
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      return cuda_fail(e, "tc_conv_persist_kernel launch");
+    }
+    return check_launch("tc_conv_persist_kernel");
+  }
+  return launch_tc<dc::kPremix>(plan, xmap, wmap, stream);
+}
+
+// ------------------------------------------------------------ grouped PREMIX
+// When every sample's mixed kernel together (B*|W| bf16) is far larger than
+// the L2 and the mixing runs on the tensor-core GEMM (n > 8), the mixed
+// kernels are made and consumed one group at a time through two workspace
+// slots: the mixing GEMM of group g+1 runs on an internal stream while the
+// persistent convolution consumes group g on the caller's stream, so a
+// group's mixed kernels are read back while they are still in L2 instead of
+// making a round trip through HBM. A group is either a run of samples (the
+// experts, read once per group, stay in L2) or, when all samples' kernels for
+// a run of 128-channel tiles fit, a run of output-channel tiles (every expert
+// byte is read once in total). Event edges order the two streams; a stream
+// capture records them as graph edges.
+constexpr size_t kGroupExpertL2 = 48u << 20;  // sample groups: the experts must stay in L2
+constexpr int kGroupTransposedMax = 64;       // groups of at most this many samples mix with premix_t
+
+struct GroupPlan {
+  int kind = 0;     // 0 none, 1 runs of samples, 2 runs of 128-channel tiles
+  int groups = 0;
+  int per = 0;      // samples (kind 1) or channels (kind 2) per group
+  size_t slot = 0;  // bytes of one slot (256-aligned)
+};
+
+GroupPlan group_plan(const dynconv_desc* d) {
+  GroupPlan g;
+  if (d->n <= dc::kPsMaxExperts || !tc_shape_ok(d)) return g;
+  const size_t taps_cin = static_cast<size_t>(d->KH) * d->KW * d->C_in;
+  const size_t wsize = d->C_out * taps_cin;
+  const size_t group_bytes = static_cast<size_t>(g_group_bytes.load());
+  if (static_cast<size_t>(d->B) * wsize * 2 < static_cast<size_t>(g_group_min.load())) return g;
+  const int m_tiles = (d->C_out + 127) / 128;
+  const size_t per_tile = static_cast<size_t>(d->B) * 128 * taps_cin * 2;
+  if (m_tiles >= 2 && per_tile <= group_bytes &&
+      dc::premix_shape_ok(d->B, d->n, 128, d->KH * d->KW, d->C_in)) {
+    const int mg = static_cast<int>(std::min<size_t>(m_tiles - 1, group_bytes / per_tile));
+    g.kind = 2;
+    g.per = mg * 128;
+    g.groups = (d->C_out + g.per - 1) / g.per;
+    g.slot = (static_cast<size_t>(d->B) * g.per * taps_cin * 2 + 255) & ~size_t(255);
+    return g;
+  }
+  if (static_cast<size_t>(d->n) * wsize * 2 > kGroupExpertL2) return g;
+  const int bg = static_cast<int>(std::max<size_t>(1, group_bytes / (wsize * 2)));
+  if (bg >= d->B) return g;
+  g.groups = (d->B + bg - 1) / bg;
+  g.per = (d->B + g.groups - 1) / g.groups;  // balanced runs of samples
+  if (!dc::premix_shape_ok(g.per, d->n, d->C_out, d->KH * d->KW, d->C_in)) return GroupPlan{};
+  g.kind = 1;
+  g.slot = (static_cast<size_t>(bg) * wsize * 2 + 255) & ~size_t(255);
+  return g;
+}
+
+// The internal stream and events of one (device, caller stream), created on
+// first use and kept for the life of the process.
+struct AuxStream {
+  cudaStream_t aux = nullptr;
+  cudaEvent_t start = nullptr, mixed[2] = {nullptr, nullptr}, used[2] = {nullptr, nullptr};
+};
+std::mutex g_aux_mu;
+std::map<std::pair<int, void*>, AuxStream> g_aux;
+
+int aux_stream(cudaStream_t caller, AuxStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_aux_mu);
+  const auto key = std::make_pair(dev, static_cast<void*>(caller));
+  auto it = g_aux.find(key);
+  if (it != g_aux.end()) {
+    *out = &it->second;
+    return DYNCONV_OK;
+  }
+  AuxStream a;
+  int prio = 0;
+  if (caller != nullptr && cudaStreamGetPriority(caller, &prio) != cudaSuccess) prio = 0;
+  e = cudaStreamCreateWithPriority(&a.aux, cudaStreamNonBlocking, prio);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreateWithPriority (internal stream)");
+  cudaEvent_t* evs[5] = {&a.start, &a.mixed[0], &a.mixed[1], &a.used[0], &a.used[1]};
+  for (cudaEvent_t* ev : evs) {
+    e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreateWithFlags (internal event)");
+  }
+  auto ins = g_aux.emplace(key, a);
+  *out = &ins.first->second;
+  return DYNCONV_OK;
+}
+
+// PREMIX through the grouped pipeline (see group_plan). DYNCONV_ERR_UNSUPPORTED
+// when a group's convolution has no persistent plan (nothing launched then).
+int run_grouped(const dynconv_desc* d, const GroupPlan& gp, const DeviceState* st, const void* x,
+                const void* experts, const float* alpha, const float* bias, void* y, void* ws,
+                const float* a_out, const float* chan_add, float chan_scale, cudaStream_t stream) {
+  const size_t taps_cin = static_cast<size_t>(d->KH) * d->KW * d->C_in;
+  const size_t wsize = d->C_out * taps_cin;
+  // every group's convolution must have a persistent plan before anything runs
+  std::vector<TcPlan> plans(gp.groups);
+  std::vector<dynconv_desc> subs(gp.groups);
+  for (int g = 0; g < gp.groups; ++g) {
+    dynconv_desc s = *d;
+    if (gp.kind == 1) s.B = std::min(gp.per, d->B - g * gp.per);
+    else s.C_out = std::min(gp.per, d->C_out - g * gp.per);
+    subs[g] = s;
+    if (!tc_plan_persist(&s, st->sms, st->max_smem_optin, &plans[g])) return DYNCONV_ERR_UNSUPPORTED;
+  }
+  AuxStream* ax = nullptr;
+  int rc = aux_stream(stream, &ax);
+  if (rc) return rc;
+  cudaError_t e = cudaEventRecord(ax->start, stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ax->aux, ax->start, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "grouped mixing: stream edge");
+  const __nv_bfloat16* E = static_cast<const __nv_bfloat16*>(experts);
+  for (int g = 0; g < gp.groups; ++g) {
+    const int slot = g & 1;
+    void* wsl = static_cast<char*>(ws) + slot * gp.slot;
+    const dynconv_desc& s = subs[g];
+    const size_t b0 = gp.kind == 1 ? static_cast<size_t>(g) * gp.per : 0;
+    const size_t c0 = gp.kind == 2 ? static_cast<size_t>(g) * gp.per : 0;
+    // ---- mixing of group g on the internal stream, once its slot is free
+    if (g >= 2) {
+      e = cudaStreamWaitEvent(ax->aux, ax->used[slot], 0);
+      if (e != cudaSuccess) return cuda_fail(e, "grouped mixing: slot edge");
+    }
+    const long long wg = static_cast<long long>(s.C_out) * static_cast<long long>(taps_cin);
+    // later groups share the GPU with the previous group's convolution
+    const int mix_sms = g == 0 ? st->sms : std::max(16, st->sms - plans[g - 1].grid);
+    if (s.B <= kGroupTransposedMax) {
+      // few samples: M = weights, N = samples (every epilogue warp busy)
+      dc::PremixTLaunch pl;
+      rc = dc::plan_premix_t(E + c0 * taps_cin, static_cast<long long>(wsize), alpha + b0 * d->n,
+                             static_cast<__nv_bfloat16*>(wsl), s.B, d->n, wg, st->err,
+                             g_wait_ns.load(), mix_sms, g_encode, &pl);
+      if (rc == -2) {
+        std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(grouped premix) failed");
+        return DYNCONV_ERR_CUDA;
+      }
+      if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
+      e = ensure_smem(dc::premix_t_kernel, pl.smem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix_t)");
+      dc::premix_t_kernel<<<pl.grid, dc::kPtThreads, pl.smem, ax->aux>>>(pl.emap, pl.p);
+      rc = check_launch("premix_t_kernel (grouped)");
+    } else {
+      dc::PremixLaunch pl;
+      rc = dc::plan_premix(E + c0 * taps_cin, alpha + b0 * d->n, static_cast<__nv_bfloat16*>(wsl),
+                           s.B, d->n, wg, st->err, g_wait_ns.load(), mix_sms, g_encode, &pl,
+                           static_cast<long long>(wsize));
+      if (rc == -2) {
+        std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(grouped premix) failed");
+        return DYNCONV_ERR_CUDA;
+      }
+      if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
+      e = ensure_smem(dc::premix_kernel, pl.smem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
+      dc::premix_kernel<<<pl.grid, dc::kPmThreads, pl.smem, ax->aux>>>(pl.emap, pl.p);
+      rc = check_launch("premix_kernel (grouped)");
+    }
+    if (rc) return rc;
+    e = cudaEventRecord(ax->mixed[slot], ax->aux);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, ax->mixed[slot], 0);
+    if (e != cudaSuccess) return cuda_fail(e, "grouped mixing: mixed edge");
+    // ---- convolution of group g on the caller's stream
+    TcPlan& pp = plans[g];
+    const size_t xoff = b0 * d->H * d->W * d->C_in;
+    const size_t yoff = b0 * d->H * d->W * d->C_out;
+    pp.p.experts = E;
+    pp.p.alpha = alpha + b0 * d->n;
+    pp.p.bias = bias;
+    pp.p.y = static_cast<__nv_bfloat16*>(y) + yoff;
+    pp.p.err = st->err;
+    pp.p.wait_ns = g_wait_ns.load();
+    pp.p.a_out = a_out ? a_out + b0 * d->C_out : nullptr;
+    pp.p.chan_add = chan_add ? chan_add + b0 * d->C_out : nullptr;
+    pp.p.chan_scale = chan_scale;
+    pp.p.co_base = static_cast<int>(c0);
+    pp.p.ld_c = d->C_out;
+    CUtensorMap xmap, wmap;
+    rc = encode_x_map(&xmap, static_cast<const __nv_bfloat16*>(x) + xoff, &s, pp.p.Wp,
+                      pp.p.b_box_rows);
+    if (rc) return rc;
+    rc = encode_w_map(&wmap, wsl, &s);
+    if (rc) return rc;
+    e = ensure_smem(dc::tc_conv_persist_kernel, pp.smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc_conv_persist)");
+    e = launch_pdl(dc::tc_conv_persist_kernel, dim3(pp.grid), dim3(dc::kTcThreads), pp.smem,
+                   stream, xmap, wmap, pp.p);
+    if (e != cudaSuccess) {
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      return cuda_fail(e, "tc_conv_persist_kernel launch (grouped)");
+    }
+    rc = check_launch("tc_conv_persist_kernel (grouped)");
+    if (rc) return rc;
+    e = cudaEventRecord(ax->used[slot], stream);
+    if (e != cudaSuccess) return cuda_fail(e, "grouped mixing: slot release");
+  }
+  return DYNCONV_OK;
+}
 
 // State slot of the streamed mixing for (device, stream): launches on one
 // stream are ordered, so they may share a slot; every stream gets a slot of
@@ -536,6 +920,15 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
     rc = run_mixconv(d, plan, st, experts, alpha, bias, y, ws, xmap, wmap, stream);
     if (rc != DYNCONV_ERR_UNSUPPORTED) return rc;
   }
+  // large B*|W| with the tensor-core mixer: the grouped pipeline through L2
+  if (g_group_mix.load() && ysum == nullptr && a_in == nullptr && g_premix_mixer.load() != 2) {
+    const GroupPlan gp = group_plan(d);
+    if (gp.kind != 0 && ws_bytes >= 2 * gp.slot && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0) {
+      rc = run_grouped(d, gp, st, x, experts, alpha, bias, y, ws, a_out, chan_add, chan_scale,
+                       stream);
+      if (rc != DYNCONV_ERR_UNSUPPORTED) return rc;
+    }
+  }
   // few experts: the store-bound CUDA-core mixer (no set-up chain)
   if (g_premix_mixer.load() != 1) {
     dc::PsParams ps;
@@ -566,7 +959,7 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
       if (rc) return rc;
       rc = encode_w_map(&wmap, ws, d);
       if (rc) return rc;
-      return launch_tc<dc::kPremix>(plan, xmap, wmap, stream);
+      return launch_premix_conv(d, plan, st, x, xmap, wmap, stream);
     }
     if (g_premix_mixer.load() == 2) return DYNCONV_ERR_UNSUPPORTED;
   }
@@ -595,7 +988,7 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   }
   rc = encode_w_map(&wmap, ws, d);
   if (rc) return rc;
-  return launch_tc<dc::kPremix>(plan, xmap, wmap, stream);
+  return launch_premix_conv(d, plan, st, x, xmap, wmap, stream);
 }
 
 }  // namespace
@@ -654,6 +1047,28 @@ int dynconv_test_hook(int key, long long value) {
   if (key == 3) {
     if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
     g_desc_base_mode = static_cast<int>(value);
+    return DYNCONV_OK;
+  }
+  if (key == 8) {
+    if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
+    g_dw_kernel.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
+  if (key == 9) {
+    if (value < 0 || value > 2) return DYNCONV_ERR_INVALID_ARG;
+    g_conv_persist.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
+  if (key == 11) {
+    if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
+    g_mixgrad_tc.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
+  if (key == 10) {
+    if (value < 0 || (value > 1 && value < 4096)) return DYNCONV_ERR_INVALID_ARG;
+    g_group_mix.store(value != 0 ? 1 : 0);
+    g_group_bytes.store(value >= 4096 ? value : (40LL << 20));
+    g_group_min.store(value >= 4096 ? 0 : (64LL << 20));
     return DYNCONV_OK;
   }
   return DYNCONV_ERR_INVALID_ARG;
@@ -778,6 +1193,67 @@ int pool_pass(const dynconv_desc* d, const void* y, float* ysum, cudaStream_t s)
   return check_launch("pool_sum_kernel");
 }
 
+// The pipelined depthwise kernel; DYNCONV_ERR_UNSUPPORTED (nothing launched)
+// when the shape does not fit its plan.
+int run_depthwise_pipe(const dynconv_desc* d, const DeviceState* st, const void* x,
+                       const void* experts, const float* alpha, const float* bias, void* y,
+                       const float* a_in, const float* a_out, const float* chan_add,
+                       float chan_scale, cudaStream_t s) {
+  dc::DwpParams p;
+  int grid = 0;
+  size_t smem = 0;
+  if (!dwp_plan(d, st->sms, st->max_smem_optin, bias != nullptr, &p, &grid, &smem))
+    return DYNCONV_ERR_UNSUPPORTED;
+  const int K = d->KH;
+  p.experts = static_cast<const __nv_bfloat16*>(experts);
+  p.alpha = alpha;
+  p.bias = bias;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.a_in = a_in;
+  p.a_out = a_out;
+  p.chan_add = chan_add;
+  p.chan_scale = chan_scale;
+  p.err = st->err;
+  p.wait_ns = g_wait_ns.load();
+  CUtensorMap xmap;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d->C_in), static_cast<cuuint64_t>(d->W),
+                              static_cast<cuuint64_t>(d->H), static_cast<cuuint64_t>(d->B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d->C_in) * 2,
+                                 static_cast<cuuint64_t>(d->W) * d->C_in * 2,
+                                 static_cast<cuuint64_t>(d->H) * d->W * d->C_in * 2};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(p.CC),
+                             static_cast<cuuint32_t>(((p.CB + 1) & ~1) + K - 1),
+                             static_cast<cuuint32_t>(p.RB + K - 1), 1u};
+  const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+  if (g_encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+    std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(depthwise pipe) failed");
+    return DYNCONV_ERR_CUDA;
+  }
+  auto go = [&](auto kern, int threads) -> int {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(depthwise pipe)");
+    if (fa.maxThreadsPerBlock < threads) return DYNCONV_ERR_UNSUPPORTED;  // the per-tile kernel runs
+    e = ensure_smem(kern, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(depthwise pipe)");
+    e = launch_pdl(kern, dim3(grid), dim3(threads), smem, s, xmap, p);
+    if (e != cudaSuccess) {
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      char what[160];
+      std::snprintf(what, sizeof(what),
+                    "depthwise_pipe_kernel launch (grid %d, %d threads, %zu B shared, %d regs)",
+                    grid, threads, smem, fa.numRegs);
+      return cuda_fail(e, what);
+    }
+    return check_launch("depthwise_pipe_kernel");
+  };
+  if (K == 3) return go(dc::depthwise_pipe_kernel<3>, dc::DwpShape<3>::kComp + 32);
+  if (K == 5) return go(dc::depthwise_pipe_kernel<5>, dc::DwpShape<5>::kComp + 32);
+  return go(dc::depthwise_pipe_kernel<7>, dc::DwpShape<7>::kComp + 32);
+}
+
 int resolve_variant(const dynconv_desc* desc, size_t ws_bytes, const DeviceState* st) {
   int variant = desc->variant;
   if (variant == DYNCONV_VARIANT_AUTO)
@@ -821,6 +1297,14 @@ int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
     case DYNCONV_VARIANT_DEPTHWISE: {
       if (!depthwise_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
       if (!aligned16(x) || !aligned16(y)) return DYNCONV_ERR_MISALIGNED;
+      if (g_dw_kernel.load() == 0 && aligned16(experts) && (bias == nullptr || aligned16(bias))) {
+        rc = run_depthwise_pipe(desc, st, x, experts, alpha, bias, y, a_in, a_out, chan_add,
+                                chan_scale, s);
+        if (rc != DYNCONV_ERR_UNSUPPORTED) {
+          if (rc || ysum == nullptr) return rc;
+          return pool_pass(desc, y, ysum, s);
+        }
+      }
       dc::DwParams p{};
       const int K = desc->KH;
       p.B = desc->B; p.C = desc->C_in; p.H = desc->H; p.W = desc->W; p.pad = desc->pad;
@@ -1111,6 +1595,8 @@ int cuda_error(cudaError_t e, const char* what) { return cuda_fail(e, what); }
 int launched(const char* what) { return check_launch(what); }
 
 int validate(const dynconv_desc* desc) { return validate_desc(desc); }
+
+bool mixgrad_tc_enabled() { return g_mixgrad_tc.load() != 0; }
 
 int forward_add(const dynconv_desc* desc, const void* x, const void* experts, const float* alpha,
                 const float* bias, void* y, void* workspace, size_t workspace_bytes, void* stream,

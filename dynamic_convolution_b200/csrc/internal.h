@@ -33,6 +33,8 @@ DC_HIDDEN cudaError_t set_smem(const void* kernel, size_t bytes);
 // The descriptor checks every entry point makes (DYNCONV_OK or INVALID_ARG /
 // UNSUPPORTED).
 DC_HIDDEN int validate(const dynconv_desc* desc);
+// Test hook 11: whether the backward may run the tensor-core mixing gradient.
+DC_HIDDEN bool mixgrad_tc_enabled();
 // dynconv_forward with one more per-(sample, output channel) term:
 // chan_scale * chan_add[b][co] is added to the mixed bias, so that it joins
 // the convolution before the single rounding of y (chan_add may be null).

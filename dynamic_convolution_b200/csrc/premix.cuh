@@ -15,7 +15,9 @@
 //    LBO = K*128 bytes apart, 8-expert groups SBO = 1024 bytes apart.
 //  * D (fp32) lives in TMEM, double-buffered (2 x 256 columns) so the
 //    epilogue of one tile overlaps the MMAs of the next; the epilogue rounds to
-//    bf16 and each thread (one sample) stores 64 contiguous bytes per chunk.
+//    bf16 and each thread (one sample) stores 64 contiguous bytes per chunk,
+//    straight from registers as two whole 32-byte sectors when every kernel
+//    is a multiple of 16 weights, else through an XOR-staged shared tile.
 // Persistent: one CTA per SM walks the (weight-tile, sample-tile) space.
 #pragma once
 
@@ -48,6 +50,7 @@ struct PmParams {
   long long tiles;       // n_tiles * m_tiles
   int a_bytes;           // bytes of all A operands
   int stage_bytes;       // bytes of one expert stage
+  int direct_store;      // 1: epilogue stores from registers (wsize % 16 == 0, out 32-byte aligned)
   const float* alpha;
   __nv_bfloat16* out;    // [B][wsize]
   int* err;
@@ -76,7 +79,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   const uint32_t a_base = base;                         // [m_tile][hi/lo][kcol][128 rows x 128 B]
   const uint32_t e_base = a_base + p.a_bytes;           // [stage][4 atoms][nk rows x 128 B]
   const uint32_t st_base = e_base + S * p.stage_bytes;  // epilogue staging: 4 warps x 16 KB
-  const uint32_t bar_base = st_base + 4 * kPmStageBytes;
+  const uint32_t bar_base = st_base + (p.direct_store ? 0u : 4u * kPmStageBytes);
   auto full = [&](int s) { return bar_base + 8u * s; };
   auto empty = [&](int s) { return bar_base + 8u * (S + s); };
   auto tfull = [&](int a) { return bar_base + 8u * (2 * S + a); };
@@ -87,13 +90,15 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
 
-  // the convolution may be scheduled as soon as every CTA of this grid runs
-  grid_launch_dependents();
   if (warp == 0) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), 512);
     tmem_relinquish();
   }
   grid_dependency_wait();  // alpha comes from the routing kernel
+  // The convolution may be scheduled once every CTA of this grid is past its
+  // wait: everything launched before this kernel has then completed, so the
+  // convolution may load x (not the mixed kernels) before its own wait.
+  grid_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full(s), 1);
@@ -215,6 +220,56 @@ __global__ void __launch_bounds__(kPmThreads, 1)
         wait_drain(drain_bar, 0, p.wait_ns, p.err);
       }
     }
+  } else if (p.direct_store) {
+    // Epilogue, direct form (every sample's kernel a multiple of 16 weights,
+    // workspace 32-byte aligned): warp w reads TMEM lanes 32*(w%4) .. +31 (=
+    // 32 samples of the tile) 32 columns at a time, the next load in flight
+    // while the current one is rounded to bf16, and each lane writes its
+    // sample's 64 contiguous bytes as two 32-byte stores: whole sectors, no
+    // shared-memory round trip.
+    const int q = warp & 3;
+    long long ntile = ntile0;
+    int mt = mt0;
+    for (long long j = 0; j < my_tiles; ++j) {
+      const int ab = static_cast<int>(j & 1);
+      if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j >> 1) & 1), ctl, kErrWaitEpilogue)) break;
+      tc_fence_after();
+      const int row0 = mt * 128 + 32 * q;
+      if (row0 < p.B) {
+        const int b = row0 + lane;
+        const long long w0 = ntile * kPmN;
+        __nv_bfloat16* dst = p.out + static_cast<size_t>(b < p.B ? b : 0) * p.wsize + w0;
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * kPmN;
+        uint32_t ra[32], rb[32];
+        auto emit = [&](const uint32_t (&r)[32], int ch) {
+          uint32_t o[16];
+#pragma unroll
+          for (int v = 0; v < 16; ++v)
+            o[v] = pack_bf16x2(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (b < p.B && w0 + ch * 32 + h * 16 < p.wsize) st_global_v8(dst + ch * 32 + h * 16, o + 8 * h);
+          }
+        };
+        tmem_ld_32x32b_x32(taddr, ra);
+#pragma unroll 1
+        for (int ch = 0; ch < kPmN / 32; ch += 2) {
+          tmem_ld_wait(ra);
+          tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, rb);
+          emit(ra, ch);
+          tmem_ld_wait(rb);
+          if (ch + 2 < kPmN / 32) tmem_ld_32x32b_x32(taddr + (ch + 2) * 32, ra);
+          emit(rb, ch + 1);
+        }
+      }
+      // the TMEM buffer is free once every lane's loads completed
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty(ab));
+      ntile += dn;
+      mt += dm;
+      if (mt >= p.m_tiles) { mt -= p.m_tiles; ++ntile; }
+    }
   } else {
     // Epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 (= 32 samples of the
     // tile), rounds to bf16 and stages its 32 x 256 block in shared memory with
@@ -291,7 +346,9 @@ struct PremixLaunch {
 template <typename EncodeFn>
 inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bfloat16* out_ws,
                        int B, int n, long long wsize, int* err, long long wait_ns, int sms,
-                       EncodeFn encode, PremixLaunch* out) {
+                       EncodeFn encode, PremixLaunch* out, long long estride = 0) {
+  // estride: elements from one expert to the next (default wsize); a larger
+  // stride mixes a contiguous slice of wsize elements of every expert
   PmParams& p = out->p;
   p = PmParams{};
   p.B = B;
@@ -303,7 +360,9 @@ inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bf
   p.tiles = n_tiles * p.m_tiles;
   p.a_bytes = 2 * p.m_tiles * pm_kcols(n) * 16384;
   p.stage_bytes = p.nk * 512;
-  const int budget = 200 * 1024 - p.a_bytes - 4 * kPmStageBytes - 4 * B * n;
+  p.direct_store = (wsize % 16 == 0 && (reinterpret_cast<uintptr_t>(out_ws) & 31u) == 0) ? 1 : 0;
+  const int staging = p.direct_store ? 0 : 4 * kPmStageBytes;
+  const int budget = 200 * 1024 - p.a_bytes - staging - 4 * B * n;
   p.stages = std::min(4, budget / p.stage_bytes);
   if (p.stages < 2) return -3;
   p.alpha = alpha;
@@ -311,7 +370,7 @@ inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bf
   p.err = err;
   p.wait_ns = wait_ns;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(wsize), static_cast<cuuint64_t>(n)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(wsize) * 2};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(estride > 0 ? estride : wsize) * 2};
   const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(p.nk)};
   const cuuint32_t es[2] = {1u, 1u};
   if (encode(&out->emap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(experts),
@@ -321,7 +380,7 @@ inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bf
   // at least 120 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
   out->smem = std::max<size_t>(120 * 1024, 1024 + static_cast<size_t>(p.a_bytes) +
                                                static_cast<size_t>(p.stages) * p.stage_bytes +
-                                               4 * kPmStageBytes + 8 * (2 * p.stages + 5) + 16 +
+                                               staging + 8 * (2 * p.stages + 5) + 16 +
                                                4 * static_cast<size_t>(B) * n);
   out->grid = static_cast<unsigned>(std::min<long long>(p.tiles, sms));
   return 0;

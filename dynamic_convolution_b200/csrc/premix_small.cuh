@@ -42,9 +42,11 @@ template <int NMAX>
 __global__ void __launch_bounds__(kPsThreads) premix_small_kernel(PsParams p) {
   extern __shared__ float ps_alpha[];  // [B][n], then [B][Cin] when a_in is given
   float* ps_ain = ps_alpha + p.B * p.n;
-  // the convolution may be scheduled as soon as every CTA of this grid runs
-  grid_launch_dependents();
   grid_dependency_wait();  // alpha comes from the routing kernel
+  // The convolution may be scheduled once every CTA of this grid is past its
+  // wait: everything launched before this kernel (the writer of x included)
+  // has then completed, so the convolution may load x before its own wait.
+  grid_launch_dependents();
   const int na = p.B * p.n;
   for (int e = threadIdx.x; e < na; e += kPsThreads) ps_alpha[e] = p.alpha[e];
   if (p.a_in != nullptr)

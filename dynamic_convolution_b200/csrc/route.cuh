@@ -20,8 +20,11 @@
 //    memory (distributed shared memory); after the one cluster barrier rank 0
 //    adds nsplit x n numbers, scales by 1/HW, adds br and applies the
 //    activation.
-// When Wr does not fit in shared memory the CTAs push per-channel sums and
-// rank 0 runs the linear layer reading Wr from global memory. When a pixel's
+// When Wr does not fit in shared memory the CTAs push per-channel sums to
+// rank 0; after the barrier every rank reads them back (DSMEM, rank order),
+// computes the logits of every nsplit-th expert from Wr rows in global
+// memory and pushes them to rank 0, which after a second cluster barrier adds
+// br and applies the activation. When a pixel's
 // channels are not a multiple of 16 bytes the threads load the pixels
 // themselves (no bulk copy). No global scratch, no atomics, deterministic.
 #pragma once
@@ -243,16 +246,43 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
     float* dst = cluster.map_shared_rank(recv, 0) + static_cast<size_t>(rank) * C;
     for (int c = t; c < C; c += kRouteThreads) dst[c] = g[c];
   }
-  cluster.sync();  // remote stores visible to rank 0; peers may exit after this
+  cluster.sync();  // remote stores visible to rank 0; with Wr staged, peers may exit after this
   if (*abort_flag && t == 0) {
     // a bounded wait gave up: let the copies still in flight land before exit
     for (int k = (issued > 2 ? issued - 2 : 0); k < issued; ++k)
       wait_drain(bar0 + 8u * (k & 1), static_cast<uint32_t>(k >> 1) & 1u, p.wait_ns, p.err);
     if (p.wr_smem) wait_drain(wrbar, 0, p.wait_ns, p.err);
   }
-  if (rank != 0) return;
-
   const float inv_hw = 1.0f / static_cast<float>(p.HW);
+  if (!p.wr_smem) {
+    // Wr too large to stage: the linear layer is split over the ranks by
+    // expert. Every rank adds the ranks' channel sums held by rank 0 (DSMEM
+    // reads, rank order) into the mean, computes the logits of experts
+    // rank, rank + nsplit, ... (one warp per expert, Wr rows read from L2) and
+    // pushes them into rank 0's z; every rank reaches both cluster barriers.
+    const float* r0 = cluster.map_shared_rank(recv, 0);
+    for (int c = t; c < C; c += kRouteThreads) {
+      float s = 0.f;
+      for (int r = 0; r < nsplit; ++r) s += r0[static_cast<size_t>(r) * C + c];
+      g[c] = s * inv_hw;
+    }
+    __syncthreads();
+    float* zdst = cluster.map_shared_rank(z, 0);
+    for (int i = rank + warp * nsplit; i < p.n; i += (kRouteThreads / 32) * nsplit) {
+      const float* wr = p.Wr + static_cast<size_t>(i) * C;
+      float s = 0.f;
+      for (int c = lane; c < C; c += 32) s = fmaf(wr[c], g[c], s);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) zdst[i] = s;
+    }
+    cluster.sync();  // logits at rank 0; nobody reads rank 0's channel sums any more
+    if (rank != 0) return;
+    for (int i = t; i < p.n; i += kRouteThreads) z[i] += brs[i];
+    __syncthreads();
+  } else if (rank != 0) {
+    return;
+  }
   float* out = p.alpha + static_cast<size_t>(b) * p.n;
   if (p.wr_smem && p.n <= 32) {
     // warp 0 alone: lane i sums expert i's partial logits, then the activation
@@ -284,21 +314,6 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
       float s = 0.f;
       for (int r = 0; r < nsplit; ++r) s += recv[static_cast<size_t>(r) * p.n + i];
       z[i] = s * inv_hw + brs[i];
-    }
-  } else {
-    for (int c = t; c < C; c += kRouteThreads) {
-      float s = 0.f;
-      for (int r = 0; r < nsplit; ++r) s += recv[static_cast<size_t>(r) * C + c];
-      g[c] = s * inv_hw;
-    }
-    __syncthreads();
-    for (int i = warp; i < p.n; i += kRouteThreads / 32) {
-      const float* wr = p.Wr + static_cast<size_t>(i) * C;
-      float s = 0.f;
-      for (int c = lane; c < C; c += 32) s = fmaf(wr[c], g[c], s);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) z[i] = s + brs[i];
     }
   }
   __syncthreads();

@@ -90,22 +90,35 @@ def test_no_device_fails_loudly(lib):
     assert dc.dynconv_last_error() != ""
 
 
+# The forward variant measured fastest on each layer by bench.py's
+# per_config.variants_forward_ms (median of 50 cold calls, one B200): with a
+# workspace, PREMIX on every dense layer (e.g. 30.7 us against FUSED 55.2 and
+# OUTSIDE 96.1 on the 3x3 layer; 184 us against 1933 and 5066 on the n=64
+# layer); without one, FUSED before OUTSIDE on every dense layer.
+MEASURED_BEST = {
+    "tiny_fp32": ("direct", "direct"),
+    "resnet18_3x3": ("premix", "fused"),
+    "effnet_expand_1x1": ("premix", "fused"),
+    "effnet_dw_5x5": ("depthwise", "depthwise"),
+    "deep_3x3_tau30": ("premix", "fused"),
+    "large_n64": ("premix", "fused"),
+}
+
+
 def test_variant_selection_per_config(lib):
-    sel = {name: dc.dynconv_select_variant(dc.desc_from_config(cfg)) for name, cfg in
-           synth.CONFIGS.items()}
-    assert sel["tiny_fp32"] == dc.VARIANT_DIRECT
-    assert sel["effnet_dw_5x5"] == dc.VARIANT_DEPTHWISE
-    for name in ("resnet18_3x3", "effnet_expand_1x1", "deep_3x3_tau30", "large_n64"):
-        assert sel[name] in (dc.VARIANT_FUSED, dc.VARIANT_OUTSIDE), name
-    # with a large enough workspace the premix variant becomes a candidate
+    """AUTO resolves to the measured fastest variant on every layer, with the
+    workspace dynconv_workspace_size asks for and with none."""
+    for name, cfg in synth.CONFIGS.items():
+        d = dc.desc_from_config(cfg)
+        ws = dc.dynconv_workspace_size(d)
+        with_ws, without = MEASURED_BEST[name]
+        assert dc.VARIANT_NAMES[dc.dynconv_select_variant(d, ws)] == with_ws, name
+        assert dc.VARIANT_NAMES[dc.dynconv_select_variant(d, 0)] == without, name
     for name in ("deep_3x3_tau30", "large_n64"):
         d = dc.desc_from_config(synth.CONFIGS[name])
-        ws = dc.dynconv_workspace_size(d)
         # every sample's mixed kernel, 256-byte aligned
         wb = (synth.CONFIGS[name].B * synth.CONFIGS[name].weight_elems * 2 + 255) // 256 * 256
-        assert ws == wb
-        assert dc.dynconv_select_variant(d, ws) in (dc.VARIANT_FUSED, dc.VARIANT_OUTSIDE,
-                                                     dc.VARIANT_PREMIX)
+        assert dc.dynconv_workspace_size(d) == wb
     # a forced variant is reported as is
     d = dc.desc_from_config(synth.CONFIGS["resnet18_3x3"], variant=dc.VARIANT_OUTSIDE)
     assert dc.dynconv_select_variant(d) == dc.VARIANT_OUTSIDE
@@ -122,6 +135,14 @@ def test_test_hook_arguments(lib):
     assert dc.dynconv_test_hook(1, 0) == dc.OK
     assert dc.dynconv_test_hook(1, -5) == dc.ERR_INVALID_ARG
     assert dc.dynconv_test_hook(99, 0) == dc.ERR_INVALID_ARG
+    # depthwise kernel choice, persistent convolution, grouped mixing
+    for key in (8, 9, 11):
+        assert dc.dynconv_test_hook(key, 3) == dc.ERR_INVALID_ARG
+        assert dc.dynconv_test_hook(key, 0 if key == 8 else 1) == dc.OK
+    assert dc.dynconv_test_hook(10, 100) == dc.ERR_INVALID_ARG   # group bytes below 4096
+    assert dc.dynconv_test_hook(10, -1) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(10, 1 << 20) == dc.OK
+    assert dc.dynconv_test_hook(10, 1) == dc.OK
 
 
 def test_pooled_entry_points_host_side(lib):

@@ -128,6 +128,19 @@ def test_backward_dense(cfg, wg):
     _check_all(c.run(wg_variant=wg), c.reference(), cfg)
 
 
+@pytest.mark.parametrize("cfg", DENSE, ids=[c.name for c in DENSE])
+def test_backward_dense_cuda_core_mixing_gradient(cfg):
+    """The tcgen05 weight gradient with the CUDA-core mixing gradient (test
+    hook 11 = 0); the default pairs it with the tensor-core one."""
+    c = Case(cfg)
+    try:
+        assert dc.dynconv_test_hook(11, 0) == dc.OK
+        got = c.run()
+    finally:
+        dc.dynconv_test_hook(11, 1)
+    _check_all(got, c.reference(), cfg)
+
+
 @pytest.mark.parametrize("dxv", [dc.VARIANT_FUSED, dc.VARIANT_OUTSIDE, dc.VARIANT_PREMIX,
                                  dc.VARIANT_DIRECT], ids=["fused", "outside", "premix", "direct"])
 def test_backward_data_every_forward_variant(dxv):

@@ -295,3 +295,171 @@ def test_premix_cuda_core_mixer_refuses_many_experts():
         assert rc == dc.ERR_UNSUPPORTED
     finally:
         dc.dynconv_test_hook(7, 0)
+
+
+DEPTHWISE_SHAPES = [
+    # name, B, C, H, W, K, pad, n: ragged channel chunks, column bands (wide
+    # images), row bands (tall images), windows larger than the image, no
+    # padding (output smaller than the input), all three kernel sizes
+    ("dw3_small", 2, 24, 7, 9, 3, 1, 3),
+    ("dw5_ragged", 3, 40, 13, 11, 5, 2, 4),
+    ("dw7_wide", 1, 64, 9, 60, 7, 3, 2),
+    ("dw5_tall", 1, 16, 200, 8, 5, 2, 2),
+    ("dw3_many_channels", 2, 264, 6, 6, 3, 1, 2),
+    ("dw5_tiny_image", 1, 8, 3, 3, 5, 2, 1),
+    ("dw3_no_pad", 2, 32, 12, 12, 3, 0, 2),
+    ("dw7_odd", 2, 56, 10, 31, 7, 3, 5),
+]
+
+
+@pytest.mark.parametrize("kernel", [0, 1], ids=["pipelined", "per-tile"])
+@pytest.mark.parametrize("case", DEPTHWISE_SHAPES, ids=[c[0] for c in DEPTHWISE_SHAPES])
+def test_depthwise_kernels_ragged(case, kernel):
+    """Both depthwise kernels (test hook 8) against the oracle on structured
+    inputs, element by element, with and without bias."""
+    name, B, C, H, W, K, pad, n = case
+    cfg = synth.LayerConfig(name, synth.BF16, B, C, C, H, W, K, K, 1, pad, C, n, synth.SIGMOID, 1.0)
+    inp = synth.make_inputs(cfg, seed=6, structured=1.0)
+    a = alpha_f32_rounded(oracle.route(inp.x_f64, inp.Wr, inp.br, cfg.mode, cfg.tau))
+    L = Layer(inp)
+    L.alpha.copy_(torch.from_numpy(a.astype(np.float32)))
+    try:
+        assert dc.dynconv_test_hook(8, kernel) == dc.OK
+        for bias in (True, False):
+            L.y.fill_(float("nan"))
+            L.forward(dc.VARIANT_DEPTHWISE, bias="default" if bias else None)
+            assert dc.dynconv_device_status(None) == dc.OK
+            ref = oracle.forward(inp.x_f64, inp.experts_f64, a, inp.bias if bias else None,
+                                 stride=1, pad=pad, groups=C)
+            r = compare(from_device(L.y), ref, synth.BF16)
+            assert r["ok"], (name, kernel, bias, r)
+    finally:
+        dc.dynconv_test_hook(8, 0)
+
+
+def test_depthwise_full_size_per_tile_kernel():
+    """The per-tile depthwise kernel at full size (the pipelined one is the
+    default and runs in test_forward_depthwise_full_size)."""
+    try:
+        assert dc.dynconv_test_hook(8, 1) == dc.OK
+        _forward_case("effnet_dw_5x5", dc.VARIANT_DEPTHWISE)
+    finally:
+        dc.dynconv_test_hook(8, 0)
+
+
+def test_depthwise_pipelined_is_deterministic():
+    """Two calls of the pipelined depthwise kernel give identical bits (fixed
+    mixing and tap order, no atomics)."""
+    inp = layer_inputs("effnet_dw_5x5")
+    L = Layer(inp)
+    L.route()
+    outs = []
+    for _ in range(2):
+        L.forward(dc.VARIANT_DEPTHWISE)
+        outs.append(L.y.clone())
+    assert torch.equal(outs[0], outs[1])
+
+
+GROUPED = [
+    # name, B, C_in, C_out, H, W, K, pad, n, mode, tau, group bytes (test hook 10)
+    ("samples_ragged", 5, 64, 264, 9, 7, 3, 1, 12, synth.SOFTMAX, 1.0, 65536),
+    ("tiles_ragged", 5, 64, 264, 9, 7, 3, 1, 12, synth.SOFTMAX, 1.0, 1 << 20),
+    ("tiles_136", 3, 72, 136, 13, 11, 3, 1, 9, synth.SIGMOID, 1.0, 1 << 20),
+    ("samples_1x1", 7, 40, 240, 12, 12, 1, 0, 10, synth.SIGMOID, 1.0, 65536),
+    # two groups of 75 samples: more than 64 per group, the samples-as-M GEMM
+    ("samples_wide", 150, 16, 24, 5, 5, 3, 1, 9, synth.SOFTMAX, 1.0, 691200),
+]
+
+
+@pytest.mark.parametrize("case", GROUPED, ids=[c[0] for c in GROUPED])
+def test_grouped_premix_ragged(case):
+    """The grouped mixing pipeline (runs of samples, or runs of 128-channel
+    tiles, through two workspace slots and an internal stream) against the
+    oracle element by element, and bit-identical to the one-pass form."""
+    name, B, Cin, Cout, H, W, K, pad, n, mode, tau, gbytes = case
+    cfg = synth.LayerConfig(name, synth.BF16, B, Cin, Cout, H, W, K, K, 1, pad, 1, n, mode, tau)
+    inp = synth.make_inputs(cfg, seed=8, structured=1.5)
+    a32 = alpha_f32_rounded(oracle.route(inp.x_f64, inp.Wr, inp.br, mode, tau))
+    L = Layer(inp)
+    L.alpha.copy_(torch.from_numpy(a32.astype(np.float32)))
+    ws = torch.empty(dc.dynconv_workspace_size(L.desc(dc.VARIANT_PREMIX)), dtype=torch.uint8,
+                     device="cuda")
+    outs = []
+    try:
+        for hook in (gbytes, 0):
+            assert dc.dynconv_test_hook(10, hook) == dc.OK
+            for _ in range(2):
+                L.y.fill_(float("nan"))
+                L.forward(dc.VARIANT_PREMIX, workspace=ws)
+                assert dc.dynconv_device_status(None) == dc.OK
+                outs.append(L.y.clone())
+    finally:
+        dc.dynconv_test_hook(10, 1)
+    ref = oracle.forward(inp.x_f64, inp.experts_f64, a32, inp.bias, stride=1, pad=pad)
+    for o in (outs[0], outs[2]):  # grouped, one pass
+        r = compare(from_device(o), ref, synth.BF16)
+        assert r["ok"], (name, r)
+    # each form is deterministic (the grouped form may mix with the transposed
+    # GEMM, whose fp32 sums may differ from the one-pass GEMM's in the last bit)
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[2], outs[3])
+
+
+@pytest.mark.parametrize("name", ["resnet18_3x3", "effnet_expand_1x1", "deep_3x3_tau30"])
+def test_persistent_conv_bit_identical(name):
+    """The persistent PREMIX convolution (test hook 9) gives the same bits as
+    one CTA per unit: same MMA order over K, same epilogue arithmetic."""
+    inp = layer_inputs(name)
+    L = Layer(inp)
+    L.route()
+    d = L.desc(dc.VARIANT_PREMIX)
+    ws = torch.empty(dc.dynconv_workspace_size(d), dtype=torch.uint8, device="cuda")
+    outs = []
+    try:
+        for persist in (2, 0):
+            assert dc.dynconv_test_hook(9, persist) == dc.OK
+            assert dc.dynconv_test_hook(10, 0) == dc.OK
+            L.y.fill_(float("nan"))
+            dc.check(dc.dynconv_forward(d, L.x, L.experts, L.alpha, L.bias, L.y, ws, ws.numel()))
+            assert dc.dynconv_device_status(None) == dc.OK
+            outs.append(L.y.clone())
+    finally:
+        dc.dynconv_test_hook(9, 1)
+        dc.dynconv_test_hook(10, 1)
+    assert torch.equal(outs[0], outs[1])
+    assert torch.isfinite(outs[0].float()).all()
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_structured_persistent_conv(case):
+    """PREMIX with the persistent convolution forced (hook 9 = 2) on the
+    ragged small cases (by default small layers run one CTA per unit)."""
+    try:
+        assert dc.dynconv_test_hook(9, 2) == dc.OK
+        test_small_structured_all_variants(case, dc.VARIANT_PREMIX)
+    finally:
+        dc.dynconv_test_hook(9, 1)
+
+
+@pytest.mark.parametrize("name", ["deep_3x3_tau30", "large_n64"])
+def test_grouped_and_one_pass_full_size(name):
+    """At full size the grouped pipeline (default for these layers; its oracle
+    parity is test_forward_tensor_core_full_size) is deterministic and agrees
+    with the one-pass PREMIX within the bf16 tolerance everywhere."""
+    inp = layer_inputs(name)
+    L = Layer(inp)
+    L.route()
+    d = L.desc(dc.VARIANT_PREMIX)
+    ws = torch.empty(dc.dynconv_workspace_size(d), dtype=torch.uint8, device="cuda")
+    outs = []
+    try:
+        for hook in (1, 1, 0):
+            assert dc.dynconv_test_hook(10, hook) == dc.OK
+            L.y.fill_(float("nan"))
+            dc.check(dc.dynconv_forward(d, L.x, L.experts, L.alpha, L.bias, L.y, ws, ws.numel()))
+            assert dc.dynconv_device_status(None) == dc.OK
+            outs.append(L.y.clone())
+    finally:
+        dc.dynconv_test_hook(10, 1)
+    assert torch.equal(outs[0], outs[1])
+    r = compare(from_device(outs[0]), from_device(outs[2]), synth.BF16)
+    assert r["ok"], (name, r)
