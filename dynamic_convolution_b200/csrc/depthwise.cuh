@@ -264,7 +264,7 @@ struct DwpShape;
 // rounded down to 8: the K*K packed weights stay in registers for the whole
 // tile.
 template <>
-struct DwpShape<3> { static constexpr int kComp = 992; static constexpr int kRegs = 64; };
+struct DwpShape<3> { static constexpr int kComp = 736; static constexpr int kRegs = 80; };
 template <>
 struct DwpShape<5> { static constexpr int kComp = 480; static constexpr int kRegs = 128; };
 template <>
@@ -280,10 +280,10 @@ struct DwpParams {
   int RB;           // output rows per tile
   int nchunks, bands, cbands;
   int S;            // stages in flight
-  int stage_bytes;  // one stage: box | weights | misc (128-aligned)
+  int stage_bytes;  // one stage: box | misc (128-aligned)
   int box_bytes;    // (RB+K-1) * (even(CB)+K-1) * CC * 2
-  int wst_off;      // weights [K*K][CC/2] packed pairs, from the stage base
   int misc_off;     // alpha[n] | a_in[CC] | a_out[CC] | chan_add[CC], from the stage base
+  int w_off;        // two mixed-kernel buffers, each [K*K][CC] weights + [CC] biases (fp32)
   int e_off;        // resident expert slabs [n][CC][K*K] bf16
   int eb_off;       // resident bias slabs [n][CC] fp32
   int bar_off;
@@ -299,7 +299,10 @@ struct DwpParams {
   long long wait_ns;
 };
 
-template <int K>
+// CCPT: the channel pairs per chunk when known at compile time (the stride
+// between staged columns, so every window load has an immediate offset), or
+// 0 for any chunk width.
+template <int K, int CCPT>
 __global__ void __maxnreg__(DwpShape<K>::kRegs)
     depthwise_pipe_kernel(const __grid_constant__ CUtensorMap xmap, DwpParams p) {
   constexpr int KK = K * K;
@@ -309,24 +312,28 @@ __global__ void __maxnreg__(DwpShape<K>::kRegs)
   unsigned char* sm = dwp_raw + ((128u - (smem_u32(dwp_raw) & 127u)) & 127u);
   const int t = threadIdx.x;
   const int warp = t >> 5, lane = t & 31;
-  const int CCp = p.CC >> 1;
+  const int CCp = CCPT > 0 ? CCPT : (p.CC >> 1);
   const int TC = ((p.CB + 1) & ~1) + K - 1;  // staged columns: even tile width + halo
 
-  // this CTA's chunk and its share of the chunk's tiles
+  // This CTA's chunk and a contiguous run of the chunk's tiles, so that
+  // consecutive tiles are the row bands of one sample and share its kernels.
   const int chunk = blockIdx.x % p.nchunks;
   const int local = blockIdx.x / p.nchunks;
   const int sharers = (gridDim.x - chunk + p.nchunks - 1) / p.nchunks;
   const int c0 = chunk * p.CC;
   const int cc_valid = min(p.CC, p.C - c0);
   const int tiles = p.B * p.bands * p.cbands;
-  const int my_tiles = local < tiles ? (tiles - local + sharers - 1) / sharers : 0;
+  const int t_begin = static_cast<int>(static_cast<long long>(local) * tiles / sharers);
+  const int t_end = static_cast<int>(static_cast<long long>(local + 1) * tiles / sharers);
+  const int my_tiles = local < sharers ? t_end - t_begin : 0;
 
   const uint32_t bar0 = smem_u32(sm + p.bar_off);
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (kDwpMaxStages + s); };
-  auto mixed = [&](int s) { return bar0 + 8u * (2 * kDwpMaxStages + s); };
-  const uint32_t ebar = bar0 + 8u * (3 * kDwpMaxStages);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.bar_off + 8 * (3 * kDwpMaxStages + 1));
+  auto mixed = [&](int g) { return bar0 + 8u * (2 * kDwpMaxStages + g); };  // 2 buffers
+  const uint32_t ebar = bar0 + 8u * (2 * kDwpMaxStages + 2);
+  volatile int* abort_flag =
+      reinterpret_cast<volatile int*>(sm + p.bar_off + 8 * (2 * kDwpMaxStages + 3));
   const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
   const __nv_bfloat16* ebuf = reinterpret_cast<const __nv_bfloat16*>(sm + p.e_off);
   const float* ebias = reinterpret_cast<const float*>(sm + p.eb_off);
@@ -335,8 +342,9 @@ __global__ void __maxnreg__(DwpShape<K>::kRegs)
     for (int s = 0; s < kDwpMaxStages; ++s) {
       mbar_init(full(s), 33);        // producer lane 0's expect-tx arrive + 32 lane arrives
       mbar_init(empty(s), NWARP_C);  // one arrive per compute warp
-      mbar_init(mixed(s), NWARP_C);
     }
+    mbar_init(mixed(0), NWARP_C);
+    mbar_init(mixed(1), NWARP_C);
     mbar_init(ebar, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -346,7 +354,7 @@ __global__ void __maxnreg__(DwpShape<K>::kRegs)
   grid_dependency_wait();  // alpha (and x) come from earlier kernels
 
   auto tile_coords = [&](int k, int& b, int& oh0, int& ow0) {
-    int u = local + k * sharers;
+    int u = t_begin + k;
     const int cb = u % p.cbands;
     u /= p.cbands;
     const int band = u % p.bands;
@@ -409,6 +417,14 @@ __global__ void __maxnreg__(DwpShape<K>::kRegs)
   if (!wait_bounded(ebar, 0, ctl, kErrWaitDwp)) return;
   const int cpair = t / CCp, pair = t - (t / CCp) * CCp;
   const int col = 2 * cpair;  // this thread's output columns col, col + 1 in the tile
+  const int w_floats = (KK + 1) * p.CC;
+  // this thread's mixing items it = t, t + NCOMP, ...: (tap, channel) walked
+  // incrementally (tap KK = the bias)
+  const int d_tap = NCOMP / p.CC, d_c = NCOMP - (NCOMP / p.CC) * p.CC;
+  int prev_b = -1, gen = -1;
+  uint64_t w2[KK];
+  uint64_t bias2 = 0;
+  float ao0 = 1.f, ao1 = 1.f;
   for (int k = 0; k < my_tiles; ++k) {
     const int s = k % p.S;
     const uint32_t ph = static_cast<uint32_t>(k / p.S) & 1u;
@@ -418,101 +434,131 @@ __global__ void __maxnreg__(DwpShape<K>::kRegs)
     unsigned char* st = sm + static_cast<size_t>(s) * p.stage_bytes;
     const float* misc = reinterpret_cast<const float*>(st + p.misc_off);
     const float* fin = misc + p.n;
-    float* wst = reinterpret_cast<float*>(st + p.wst_off);  // [KK][CCp][2]
-    float* bst = wst + KK * p.CC;                            // [CC] mixed bias (+ term)
 
-    // ---- mix this tile's kernels: tap-major items, consecutive channels
-    for (int it = t; it < (KK + 1) * p.CC; it += NCOMP) {
-      const int tap = it / p.CC, c = it - (it / p.CC) * p.CC;
-      if (c >= cc_valid) continue;
-      float sacc = 0.f;
-      if (tap < KK) {
-        for (int j = 0; j < p.n; ++j)
-          sacc = fmaf(misc[j], __bfloat162float(ebuf[(static_cast<size_t>(j) * p.CC + c) * KK + tap]),
-                      sacc);
-        wst[tap * p.CC + c] = sacc * fin[c];  // input attention folded (depthwise: one channel)
-      } else {
-        if (p.bias)
-          for (int j = 0; j < p.n; ++j) sacc = fmaf(misc[j], ebias[j * p.CC + c], sacc);
-        bst[c] = sacc + fin[2 * p.CC + c];
+    if (b != prev_b) {
+      // ---- a new sample: mix its kernels (fp32, expert by expert) into the
+      // next of the two buffers; the previous sample's buffer may still be
+      // read by a slower warp until it has passed this sample's barrier
+      prev_b = b;
+      ++gen;
+      float* wb = reinterpret_cast<float*>(sm + p.w_off) + (gen & 1) * w_floats;  // [KK][CC] | [CC]
+      int tap = t / p.CC, c = t - (t / p.CC) * p.CC;
+      for (int it = t; it < w_floats; it += NCOMP) {
+        if (c < cc_valid) {
+          float sacc = 0.f;
+          if (tap < KK) {
+            const __nv_bfloat16* e = ebuf + c * KK + tap;
+            for (int j = 0; j < p.n; ++j, e += p.CC * KK)
+              sacc = fmaf(misc[j], __bfloat162float(*e), sacc);
+            wb[it] = sacc * fin[c];  // input attention folded (depthwise: one channel)
+          } else {
+            if (p.bias)
+              for (int j = 0; j < p.n; ++j) sacc = fmaf(misc[j], ebias[j * p.CC + c], sacc);
+            wb[it] = sacc + fin[2 * p.CC + c];
+          }
+        }
+        tap += d_tap;
+        c += d_c;
+        if (c >= p.CC) { c -= p.CC; ++tap; }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(mixed(gen & 1));
+      if (!wait_bounded(mixed(gen & 1), static_cast<uint32_t>(gen >> 1) & 1u, ctl, kErrWaitDwp))
+        return;
+      // the sample's weights stay in registers for all its tiles
+#pragma unroll
+      for (int q = 0; q < KK; ++q) w2[q] = *reinterpret_cast<const uint64_t*>(wb + q * p.CC + 2 * pair);
+      bias2 = *reinterpret_cast<const uint64_t*>(wb + KK * p.CC + 2 * pair);
+      ao0 = fin[p.CC + 2 * pair];
+      ao1 = fin[p.CC + 2 * pair + 1];
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(mixed(s));
-    if (!wait_bounded(mixed(s), ph, ctl, kErrWaitDwp)) return;
 
     const int ow = ow0 + col;
     const int c = c0 + 2 * pair;
     const bool active = col < p.CB && ow < p.Wo && c < p.C;
     if (active) {
-      uint64_t w2[KK];
-#pragma unroll
-      for (int q = 0; q < KK; ++q)
-        w2[q] = *reinterpret_cast<const uint64_t*>(wst + q * p.CC + 2 * pair);
-      const uint64_t bias2 = *reinterpret_cast<const uint64_t*>(bst + 2 * pair);
-      const float ao0 = fin[p.CC + 2 * pair], ao1 = fin[p.CC + 2 * pair + 1];
       const bool scale_out = p.a_out != nullptr;
       const bool second = col + 1 < p.CB && ow + 1 < p.Wo;  // the column pair's second column
       const uint32_t* xw = reinterpret_cast<const uint32_t*>(st) + col * CCp + pair;
       const int row_words = TC * CCp;
-      __nv_bfloat16* yb = p.y + (static_cast<size_t>(b) * p.Ho * p.Wo + ow) * p.C + c;
+      const size_t ystride = static_cast<size_t>(p.Wo) * p.C;  // one output row
+      // output row o of the tile goes to ydst0 + o * ystride (rows past Ho are skipped)
+      __nv_bfloat16* ydst0 =
+          p.y + (static_cast<size_t>(b) * p.Ho * p.Wo + static_cast<size_t>(oh0) * p.Wo + ow) * p.C + c;
+      const int rows_out = min(p.RB, p.Ho - oh0);  // rows of this band inside the image
       const int rows_in = p.RB + K - 1;
-      uint64_t acc[K][2];
-#pragma unroll
-      for (int q = 0; q < K; ++q) acc[q][0] = acc[q][1] = bias2;
+      uint64_t acc[K][2];  // open output rows, slot o % K
       auto store_row = [&](uint64_t (&a)[2], int o) {
-        const int oh = oh0 + o;
-        if (oh < p.Ho) {
-          __nv_bfloat16* dst = yb + static_cast<size_t>(oh) * p.Wo * p.C;
-#pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            float lo = __uint_as_float(static_cast<uint32_t>(a[v]));
-            float hi = __uint_as_float(static_cast<uint32_t>(a[v] >> 32));
-            if (scale_out) { lo *= ao0; hi *= ao1; }
-            if (v == 0 || second)
-              *reinterpret_cast<uint32_t*>(dst + v * p.C) = pack_bf16x2(lo, hi);
-          }
+        if (o < rows_out) {
+          __nv_bfloat16* dst = ydst0 + static_cast<size_t>(o) * ystride;
+          float l0 = __uint_as_float(static_cast<uint32_t>(a[0]));
+          float h0 = __uint_as_float(static_cast<uint32_t>(a[0] >> 32));
+          float l1 = __uint_as_float(static_cast<uint32_t>(a[1]));
+          float h1 = __uint_as_float(static_cast<uint32_t>(a[1] >> 32));
+          if (scale_out) { l0 *= ao0; h0 *= ao1; l1 *= ao0; h1 *= ao1; }
+          *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(l0, h0);
+          if (second) *reinterpret_cast<uint32_t*>(dst + p.C) = pack_bf16x2(l1, h1);
         }
       };
-      // One group of K input rows starting at ir0 (a multiple of K): for input
-      // row ir the output rows o = ir - kh; row ir - (K-1) completes. GUARDED
-      // groups test the band edges (o < 0, o >= RB, ir >= rows_in).
-      auto group = [&](int ir0, auto guarded) {
-        constexpr bool G = decltype(guarded)::value;
+      // One group of K input rows starting at ir0 (a multiple of K): input
+      // row ir feeds output rows o = ir - kh, opens row ir (kh = 0: the
+      // accumulator starts from the bias) and completes row ir - (K-1). Every
+      // loop is fully unrolled, so each accumulator slot is a fixed register.
+      // The band edges (o < 0, o >= RB, ir >= rows_in) are compile-time for
+      // the HEAD group (ir0 = 0, RB >= K) and the TAIL group (ir0 = RB, RB a
+      // multiple of K); MID groups have none; GENERIC tests them at run time.
+      enum { MID = 0, HEAD = 1, TAIL = 2, GENERIC = 3 };
+      auto group = [&](int ir0, auto kind_tag) {
+        constexpr int KIND = decltype(kind_tag)::value;
+        const uint32_t* xr = xw + ir0 * row_words;
 #pragma unroll
-        for (int j = 0; j < K; ++j) {
+        for (int j = 0; j < K; ++j, xr += row_words) {
           const int ir = ir0 + j;
-          if (G && ir >= rows_in) break;
-          const uint32_t* xr = xw + ir * row_words;
+          if (KIND == TAIL && j >= K - 1) continue;              // ir >= RB + K - 1
+          if (KIND == GENERIC && ir >= rows_in) continue;
           uint64_t xv[K + 1];
 #pragma unroll
           for (int kw = 0; kw <= K; ++kw) xv[kw] = bf16x2_to_f32x2(xr[kw * CCp]);
 #pragma unroll
           for (int kh = K - 1; kh >= 0; --kh) {
             const int o = ir - kh;
-            if (G && (o < 0 || o >= p.RB)) continue;
             const int slot = (j - kh + K) % K;  // o % K
+            bool live;
+            if (KIND == MID) live = true;
+            else if (KIND == HEAD) live = j >= kh;       // o >= 0; o < K <= RB
+            else if (KIND == TAIL) live = j < kh;        // o < RB; o >= RB - K + 1 >= 0
+            else live = o >= 0 && o < p.RB;
+            if (!live) continue;
+            uint64_t a0 = kh == 0 ? bias2 : acc[slot][0];
+            uint64_t a1 = kh == 0 ? bias2 : acc[slot][1];
 #pragma unroll
             for (int kw = 0; kw < K; ++kw) {
-              acc[slot][0] = ffma2(xv[kw], w2[kh * K + kw], acc[slot][0]);
-              acc[slot][1] = ffma2(xv[kw + 1], w2[kh * K + kw], acc[slot][1]);
+              a0 = ffma2(xv[kw], w2[kh * K + kw], a0);
+              a1 = ffma2(xv[kw + 1], w2[kh * K + kw], a1);
             }
             if (kh == K - 1) {
-              store_row(acc[slot], o);
-              acc[slot][0] = acc[slot][1] = bias2;
+              uint64_t done[2] = {a0, a1};
+              store_row(done, o);
+            } else {
+              acc[slot][0] = a0;
+              acc[slot][1] = a1;
             }
           }
         }
       };
-      // groups wholly inside the band (every o in [0, RB)): ir0 >= K and
-      // ir0 + K - 1 < RB; the others are guarded
-      const int inner_end = p.RB >= K ? (p.RB - K + 1 + K - 1) / K * K : K;  // first ir0 > RB - K
-      group(0, std::true_type{});
+      using KMid = std::integral_constant<int, MID>;
+      using KHead = std::integral_constant<int, HEAD>;
+      using KTail = std::integral_constant<int, TAIL>;
+      using KGen = std::integral_constant<int, GENERIC>;
+      if (p.RB >= K && p.RB % K == 0) {
+        group(0, KHead{});
 #pragma unroll 1
-      for (int ir0 = K; ir0 < inner_end && ir0 <= p.RB - K; ir0 += K) group(ir0, std::false_type{});
+        for (int ir0 = K; ir0 < p.RB; ir0 += K) group(ir0, KMid{});
+        group(p.RB, KTail{});
+      } else {
 #pragma unroll 1
-      for (int ir0 = (inner_end > K ? inner_end : K); ir0 < rows_in; ir0 += K)
-        group(ir0, std::true_type{});
+        for (int ir0 = 0; ir0 < rows_in; ir0 += K) group(ir0, KGen{});
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty(s));

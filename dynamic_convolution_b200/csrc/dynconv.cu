@@ -64,7 +64,8 @@ std::atomic<int> g_stream_mix{0};   // PREMIX with n <= 8: mixing streamed into 
 std::atomic<int> g_premix_mixer{0};  // 0 automatic, 1 tensor-core GEMM, 2 CUDA cores (n <= 8)
 std::atomic<int> g_dw_kernel{0};     // 0 pipelined depthwise kernel when it fits, 1 the per-tile one
 std::atomic<int> g_conv_persist{1};  // PREMIX convolution: 1 persistent kernel when it fits, 0 one CTA per unit
-std::atomic<int> g_group_mix{1};     // PREMIX, n > 8, large B*|W|: 1 grouped mixing pipeline, 0 one pass
+std::atomic<int> g_group_mix{0};     // PREMIX, n > 8, large B*|W|: 1 grouped mixing pipeline, 0 one pass
+std::atomic<int> g_premix_direct{0}; // premix epilogue: 1 stores from registers when aligned, 0 staged
 std::atomic<int> g_mixgrad_tc{1};    // backward: 1 tensor-core mixing gradient when it fits, 0 CUDA cores
 std::atomic<long long> g_group_bytes{40LL << 20};  // target bytes of one group's mixed kernels
 std::atomic<long long> g_group_min{64LL << 20};    // below this B*|W| the one-pass form is used
@@ -379,24 +380,31 @@ bool dwp_plan(const dynconv_desc* d, int sms, int max_smem, bool has_bias, dc::D
   auto a128 = [](size_t v) { return (v + 127) / 128 * 128; };
   const size_t e_bytes = a128(static_cast<size_t>(d->n) * CC * KK * 2);
   const size_t eb_bytes = has_bias ? a128(static_cast<size_t>(d->n) * CC * 4) : 0;
-  const size_t wst_bytes = a128(static_cast<size_t>(KK + 1) * CC * 4);
+  const size_t w_bytes = 2 * a128(static_cast<size_t>(KK + 1) * CC * 4);  // two buffers
   const size_t misc_bytes = a128(static_cast<size_t>(d->n + 3 * CC) * 4);
   const size_t bars = 8 * (3 * dc::kDwpMaxStages + 1) + 16;
   const int TC = ((CB + 1) & ~1) + K - 1;  // staged columns
   auto stage_of = [&](int RB) {
-    return a128(static_cast<size_t>(RB + K - 1) * TC * CC * 2) + wst_bytes + misc_bytes;
+    return a128(static_cast<size_t>(RB + K - 1) * TC * CC * 2) + misc_bytes;
   };
   int S = 0, RBmax = 0;
   for (int st : {3, 2}) {
     int rb = std::min(Ho, 256 - (K - 1));
-    while (rb > 0 && 128 + st * stage_of(rb) + e_bytes + eb_bytes + bars >
+    while (rb > 0 && 128 + st * stage_of(rb) + w_bytes + e_bytes + eb_bytes + bars >
                          static_cast<size_t>(max_smem))
       --rb;
     if (rb > 0 && (rb >= std::min(Ho, 8) || st == 2)) { S = st; RBmax = rb; break; }
   }
   if (S == 0 || RBmax == 0) return false;
-  const int bands = (Ho + RBmax - 1) / RBmax;
-  const int RB = (Ho + bands - 1) / bands;
+  int bands = (Ho + RBmax - 1) / RBmax;
+  int RB = (Ho + bands - 1) / bands;
+  // a band height that is a multiple of K lets the kernel resolve every
+  // band-edge test at compile time
+  const int RBk = (RB + K - 1) / K * K;
+  if (RBk <= RBmax) {
+    RB = RBk;
+    bands = (Ho + RB - 1) / RB;
+  }
   std::memset(p, 0, sizeof(*p));
   p->B = d->B; p->C = C; p->H = d->H; p->W = d->W; p->pad = d->pad; p->n = d->n;
   p->Ho = Ho; p->Wo = Wo; p->CC = CC; p->CB = CB; p->RB = RB;
@@ -405,10 +413,10 @@ bool dwp_plan(const dynconv_desc* d, int sms, int max_smem, bool has_bias, dc::D
   p->cbands = (Wo + CB - 1) / CB;
   p->S = S;
   p->box_bytes = (RB + K - 1) * TC * CC * 2;
-  p->wst_off = static_cast<int>(a128(static_cast<size_t>(p->box_bytes)));
-  p->misc_off = p->wst_off + static_cast<int>(wst_bytes);
+  p->misc_off = static_cast<int>(a128(static_cast<size_t>(p->box_bytes)));
   p->stage_bytes = p->misc_off + static_cast<int>(misc_bytes);
-  p->e_off = S * p->stage_bytes;
+  p->w_off = S * p->stage_bytes;
+  p->e_off = p->w_off + static_cast<int>(w_bytes);
   p->eb_off = p->e_off + static_cast<int>(e_bytes);
   p->bar_off = p->eb_off + static_cast<int>(eb_bytes);
   const long long tiles_per_chunk = 1LL * d->B * p->bands * p->cbands;
@@ -664,7 +672,10 @@ int run_grouped(const dynconv_desc* d, const GroupPlan& gp, const DeviceState* s
     if (gp.kind == 1) s.B = std::min(gp.per, d->B - g * gp.per);
     else s.C_out = std::min(gp.per, d->C_out - g * gp.per);
     subs[g] = s;
-    if (!tc_plan_persist(&s, st->sms, st->max_smem_optin, &plans[g])) return DYNCONV_ERR_UNSUPPORTED;
+    // a group's convolution gets at most half of the SMs: the next group's
+    // mixing runs on the others meanwhile
+    if (!tc_plan_persist(&s, std::max(1, st->sms / 2), st->max_smem_optin, &plans[g]))
+      return DYNCONV_ERR_UNSUPPORTED;
   }
   AuxStream* ax = nullptr;
   int rc = aux_stream(stream, &ax);
@@ -706,7 +717,7 @@ int run_grouped(const dynconv_desc* d, const GroupPlan& gp, const DeviceState* s
       dc::PremixLaunch pl;
       rc = dc::plan_premix(E + c0 * taps_cin, alpha + b0 * d->n, static_cast<__nv_bfloat16*>(wsl),
                            s.B, d->n, wg, st->err, g_wait_ns.load(), mix_sms, g_encode, &pl,
-                           static_cast<long long>(wsize));
+                           static_cast<long long>(wsize), g_premix_direct.load() != 0);
       if (rc == -2) {
         std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(grouped premix) failed");
         return DYNCONV_ERR_CUDA;
@@ -968,7 +979,7 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   rc = dc::plan_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
                        static_cast<__nv_bfloat16*>(ws), d->B, d->n,
                        static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in, st->err,
-                       g_wait_ns.load(), st->sms, g_encode, &pl);
+                       g_wait_ns.load(), st->sms, g_encode, &pl, 0, g_premix_direct.load() != 0);
   if (rc == -2) {
     std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(premix) failed");
     return DYNCONV_ERR_CUDA;
@@ -1062,6 +1073,11 @@ int dynconv_test_hook(int key, long long value) {
   if (key == 11) {
     if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
     g_mixgrad_tc.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
+  if (key == 12) {
+    if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
+    g_premix_direct.store(static_cast<int>(value));
     return DYNCONV_OK;
   }
   if (key == 10) {
@@ -1249,9 +1265,16 @@ int run_depthwise_pipe(const dynconv_desc* d, const DeviceState* st, const void*
     }
     return check_launch("depthwise_pipe_kernel");
   };
-  if (K == 3) return go(dc::depthwise_pipe_kernel<3>, dc::DwpShape<3>::kComp + 32);
-  if (K == 5) return go(dc::depthwise_pipe_kernel<5>, dc::DwpShape<5>::kComp + 32);
-  return go(dc::depthwise_pipe_kernel<7>, dc::DwpShape<7>::kComp + 32);
+  // 32 channel pairs per chunk: the window's column stride is a compile-time constant
+  const bool c32 = p.CC == 64;
+  if (K == 3)
+    return c32 ? go(dc::depthwise_pipe_kernel<3, 32>, dc::DwpShape<3>::kComp + 32)
+               : go(dc::depthwise_pipe_kernel<3, 0>, dc::DwpShape<3>::kComp + 32);
+  if (K == 5)
+    return c32 ? go(dc::depthwise_pipe_kernel<5, 32>, dc::DwpShape<5>::kComp + 32)
+               : go(dc::depthwise_pipe_kernel<5, 0>, dc::DwpShape<5>::kComp + 32);
+  return c32 ? go(dc::depthwise_pipe_kernel<7, 32>, dc::DwpShape<7>::kComp + 32)
+             : go(dc::depthwise_pipe_kernel<7, 0>, dc::DwpShape<7>::kComp + 32);
 }
 
 int resolve_variant(const dynconv_desc* desc, size_t ws_bytes, const DeviceState* st) {

@@ -346,7 +346,8 @@ struct PremixLaunch {
 template <typename EncodeFn>
 inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bfloat16* out_ws,
                        int B, int n, long long wsize, int* err, long long wait_ns, int sms,
-                       EncodeFn encode, PremixLaunch* out, long long estride = 0) {
+                       EncodeFn encode, PremixLaunch* out, long long estride = 0,
+                       bool allow_direct = true) {
   // estride: elements from one expert to the next (default wsize); a larger
   // stride mixes a contiguous slice of wsize elements of every expert
   PmParams& p = out->p;
@@ -360,7 +361,8 @@ inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bf
   p.tiles = n_tiles * p.m_tiles;
   p.a_bytes = 2 * p.m_tiles * pm_kcols(n) * 16384;
   p.stage_bytes = p.nk * 512;
-  p.direct_store = (wsize % 16 == 0 && (reinterpret_cast<uintptr_t>(out_ws) & 31u) == 0) ? 1 : 0;
+  p.direct_store =
+      (allow_direct && wsize % 16 == 0 && (reinterpret_cast<uintptr_t>(out_ws) & 31u) == 0) ? 1 : 0;
   const int staging = p.direct_store ? 0 : 4 * kPmStageBytes;
   const int budget = 200 * 1024 - p.a_bytes - staging - 4 * B * n;
   p.stages = std::min(4, budget / p.stage_bytes);

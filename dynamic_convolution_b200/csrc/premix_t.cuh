@@ -12,11 +12,13 @@
 //    two TMA boxes {64 weights, K experts} per tile in the 128-byte swizzle.
 //  * B = alpha, split into bf16 hi + lo (two MMAs per K step, ~16 bits of
 //    alpha), K-major, built once per CTA.
-//  * D (fp32) in TMEM, double-buffered (2 x N columns): the epilogue of one
-//    tile overlaps the MMAs of the next.
-//  * Epilogue: lane = weight w, 32 samples per load; neighbouring lanes swap
-//    one value (shuffle) so that each lane stores two adjacent weights of one
-//    sample (even lanes sample s, odd lanes sample s+1): every store
+//  * D (fp32) in TMEM, up to 8 accumulators of N columns: the MMAs run up to
+//    8 tiles ahead of the epilogue, so the latency of one tile's MMA
+//    completion and TMEM read overlaps the others'.
+//  * Epilogue, 8 warps (two per TMEM lane quarter, alternate 16-sample
+//    column groups): lane = weight w, 16 samples per load; neighbouring lanes
+//    swap one value (shuffle) so that each lane stores two adjacent weights
+//    of one sample (even lanes sample s, odd lanes sample s+1): every store
 //    instruction writes two 64-byte runs.
 // Persistent: one CTA per SM walks the 128-weight tiles.
 #pragma once
@@ -25,12 +27,15 @@
 
 namespace dc {
 
-constexpr int kPtThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kPtThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kPtEpiWarps = 8;
+constexpr int kPtMaxAcc = 8;     // TMEM accumulators (tiles in flight between MMA and epilogue)
 constexpr int kPtM = 128;        // weights per tile
 
 struct PtParams {
   int S, n, nk;          // samples (<= 256), experts, experts padded to 16
   int npad;              // samples padded to 32 (MMA N)
+  int nacc;              // TMEM accumulators of npad columns (<= kPtMaxAcc, nacc * npad <= 512)
   int stages;
   long long wsize;       // weights to mix per sample (this launch's slice)
   long long tiles;       // ceil(wsize / 128)
@@ -56,14 +61,15 @@ __global__ void __launch_bounds__(kPtThreads, 1)
   auto full = [&](int s) { return bar_base + 8u * s; };
   auto empty = [&](int s) { return bar_base + 8u * (S + s); };
   auto tfull = [&](int a) { return bar_base + 8u * (2 * S + a); };
-  auto tempty = [&](int a) { return bar_base + 8u * (2 * S + 2 + a); };
-  const uint32_t drain_bar = bar_base + 8u * (2 * S + 4);
-  unsigned char* misc = base_ptr + (bar_base - base) + 8u * (2 * S + 5);
+  auto tempty = [&](int a) { return bar_base + 8u * (2 * S + kPtMaxAcc + a); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * S + 2 * kPtMaxAcc);
+  unsigned char* misc = base_ptr + (bar_base - base) + 8u * (2 * S + 2 * kPtMaxAcc + 1);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
   uint32_t tcols = 32;
-  while (tcols < 2u * static_cast<uint32_t>(p.npad)) tcols <<= 1;
+  while (tcols < static_cast<uint32_t>(p.nacc * p.npad)) tcols <<= 1;
+  const int NA = p.nacc;
 
   if (warp == 0) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), tcols);
@@ -76,9 +82,9 @@ __global__ void __launch_bounds__(kPtThreads, 1)
       mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < NA; ++a) {
       mbar_init(tfull(a), 1);
-      mbar_init(tempty(a), 4);
+      mbar_init(tempty(a), kPtEpiWarps);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -144,9 +150,10 @@ __global__ void __launch_bounds__(kPtThreads, 1)
       uint32_t ph = 0;
       bool ok = true;
       for (long long j = 0; j < my_tiles; ++j) {
-        const int ab = static_cast<int>(j & 1);
+        const int ab = static_cast<int>(j % NA);
+        const uint32_t aph = static_cast<uint32_t>((j / NA) & 1);
         if (!wait_bounded(full(s), ph, ctl, kErrWaitMma)) { ok = false; break; }
-        if (!wait_bounded(tempty(ab), static_cast<uint32_t>((j >> 1) & 1) ^ 1u, ctl, kErrWaitMma)) { ok = false; break; }
+        if (!wait_bounded(tempty(ab), aph ^ 1u, ctl, kErrWaitMma)) { ok = false; break; }
         tc_fence_after();
         const uint64_t ad = a_desc0 + s * stage;
         const uint32_t d = tmem_base + ab * p.npad;
@@ -166,31 +173,33 @@ __global__ void __launch_bounds__(kPtThreads, 1)
         wait_drain(drain_bar, 0, p.wait_ns, p.err);
       }
     }
-  } else {
-    // Epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = weights of the tile
+  } else if (warp < 2 + kPtEpiWarps) {
+    // Epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = weights of the tile;
+    // the two warps of a lane quarter take alternate 16-sample column groups
     const int q = warp & 3;
-    const int nch = (p.S + 31) / 32;
+    const int half = (warp - 2) >> 2;
+    const int ngroups = (p.S + 15) / 16;
+    const bool odd = lane & 1;
     for (long long j = 0; j < my_tiles; ++j) {
       const long long t = blockIdx.x + j * gridDim.x;
-      const int ab = static_cast<int>(j & 1);
-      if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j >> 1) & 1), ctl, kErrWaitEpilogue)) break;
+      const int ab = static_cast<int>(j % NA);
+      if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j / NA) & 1), ctl, kErrWaitEpilogue)) break;
       tc_fence_after();
       const long long w = t * kPtM + 32 * q + lane;    // this lane's weight
       const long long wp = w & ~1LL;                   // the pair a lane stores
       const bool wok = wp < p.wsize;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * p.npad;
-      const bool odd = lane & 1;
-      for (int ch = 0; ch < nch; ++ch) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + ch * 32, r);
-        tmem_ld_wait(r);
+      for (int g = half; g < ngroups; g += 2) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + g * 16, r);
+        tmem_ld_wait16(r);
 #pragma unroll
-        for (int v = 0; v < 32; v += 2) {
+        for (int v = 0; v < 16; v += 2) {
           // even lanes keep sample v, odd lanes sample v+1; each sends the
           // other sample's value to its neighbour
           const float mine_v = __uint_as_float(r[v]), mine_v1 = __uint_as_float(r[v + 1]);
           const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_v : mine_v1, 1);
-          const int sidx = ch * 32 + v + (odd ? 1 : 0);
+          const int sidx = g * 16 + v + (odd ? 1 : 0);
           const uint32_t packed = odd ? pack_bf16x2(other, mine_v1) : pack_bf16x2(mine_v, other);
           if (wok && sidx < p.S)
             *reinterpret_cast<uint32_t*>(p.out + static_cast<size_t>(sidx) * p.wsize + wp) = packed;
@@ -234,6 +243,7 @@ inline int plan_premix_t(const __nv_bfloat16* experts, long long estride, const 
   p.tiles = (wsize + kPtM - 1) / kPtM;
   p.a_bytes = 2 * p.nk * 128;
   p.b_bytes = ((p.nk + 63) / 64) * p.npad * 128;
+  p.nacc = std::max(2, std::min(kPtMaxAcc, 512 / p.npad));
   const int budget = 200 * 1024 - 2 * p.b_bytes;
   p.stages = std::min(6, budget / p.a_bytes);
   if (p.stages < 2) return -3;
@@ -252,7 +262,7 @@ inline int plan_premix_t(const __nv_bfloat16* experts, long long estride, const 
   // at least 120 KB, so that two CTAs never share an SM's TMEM
   out_l->smem = std::max<size_t>(120 * 1024, 1024 + 2 * static_cast<size_t>(p.b_bytes) +
                                                  static_cast<size_t>(p.stages) * p.a_bytes +
-                                                 8 * (2 * p.stages + 5) + 16);
+                                                 8 * (2 * p.stages + 2 * kPtMaxAcc + 1) + 16);
   out_l->grid = static_cast<unsigned>(std::min<long long>(p.tiles, ctas));
   return 0;
 }

@@ -11,7 +11,7 @@
 // the sample's pixels, built around the latency chain (the whole input is a
 // few MB):
 //  * the slice is contiguous in NHWC, so one thread moves it into shared
-//    memory with a few bulk copies (cp.async.bulk, at most two in flight),
+//    memory with a few bulk copies (cp.async.bulk, up to four in flight),
 //    together with the router weights Wr when they fit: the bytes in flight
 //    are not limited by per-thread load queues;
 //  * the threads add the staged pixels in a fixed order;
@@ -36,7 +36,8 @@
 namespace dc {
 
 constexpr int kRouteThreads = 256;
-constexpr int kRoutePieceBytes = 48 * 1024;  // largest bulk piece
+constexpr int kRoutePieceBytes = 24 * 1024;  // largest bulk piece
+constexpr int kRouteRing = 4;                // bulk pieces in flight per CTA
 constexpr int kRouteWrSmemBytes = 32 * 1024;  // largest Wr staged in shared memory
 constexpr int kErrWaitRoute = 0x107;
 
@@ -75,14 +76,14 @@ __host__ __device__ inline RouteSmem route_smem(int C, int n, int VEC, int elem_
     return at;
   };
   const size_t piece = static_cast<size_t>(piece_px) * C * elem_bytes;
-  s.ring = take(bulk ? 2 * piece : 0, 128);
+  s.ring = take(bulk ? kRouteRing * piece : 0, 128);
   s.wr = take(wr_smem ? static_cast<size_t>(n) * C * 4 : 0, 128);
   s.partial = take(static_cast<size_t>(lanes_p) * C * 4, 16);
   s.g = take(static_cast<size_t>(C) * 4, 16);
   s.recv = take(static_cast<size_t>(nsplit) * (wr_smem ? n : C) * 4, 16);
   s.brs = take(static_cast<size_t>(n) * 4, 16);
   s.z = take(static_cast<size_t>(n) * 4, 16);
-  s.bars = take(3 * 8, 8);
+  s.bars = take((kRouteRing + 1) * 8, 8);
   s.flag = take(4, 4);
   s.total = off;
   return s;
@@ -135,7 +136,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
   float* z = reinterpret_cast<float*>(route_raw + L.z);              // [n]
   const uint32_t ring = smem_u32(route_raw + L.ring);
   const uint32_t bar0 = smem_u32(route_raw + L.bars);
-  const uint32_t wrbar = bar0 + 16;
+  const uint32_t wrbar = bar0 + 8u * kRouteRing;  // after the ring's barriers
   volatile int* abort_flag = reinterpret_cast<volatile int*>(route_raw + L.flag);
   const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
 
@@ -159,14 +160,14 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
     ++issued;
     const int px = min(piece_px, npx - k * piece_px);
     const uint32_t bytes = static_cast<uint32_t>(px * row_bytes);
-    mbar_arrive_expect_tx(bar0 + 8u * (k & 1), bytes);
-    bulk_load(ring + static_cast<uint32_t>((k & 1) * piece_bytes), src + k * piece_bytes, bytes,
-              bar0 + 8u * (k & 1));
+    const int slot = k % kRouteRing;
+    mbar_arrive_expect_tx(bar0 + 8u * slot, bytes);
+    bulk_load(ring + static_cast<uint32_t>(slot * piece_bytes), src + k * piece_bytes, bytes,
+              bar0 + 8u * slot);
   };
 
   if (t == 0) {
-    mbar_init(bar0, 1);
-    mbar_init(bar0 + 8, 1);
+    for (int r = 0; r < kRouteRing; ++r) mbar_init(bar0 + 8u * r, 1);
     mbar_init(wrbar, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -178,7 +179,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
       mbar_arrive_expect_tx(wrbar, wb);
       bulk_load(smem_u32(wr_s), p.Wr, wb, wrbar);
     }
-    for (int k = 0; k < npieces && k < 2; ++k) issue(k);
+    for (int k = 0; k < npieces && k < kRouteRing; ++k) issue(k);
   }
   __syncthreads();
 
@@ -191,16 +192,17 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
 #pragma unroll
     for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
     for (int k = 0; k < npieces; ++k) {
-      const bool ok = wait_bounded(bar0 + 8u * (k & 1), static_cast<uint32_t>(k >> 1) & 1u, ctl,
+      const bool ok = wait_bounded(bar0 + 8u * (k % kRouteRing),
+                                   static_cast<uint32_t>(k / kRouteRing) & 1u, ctl,
                                    kErrWaitRoute);
       if (ok && active) {
         const int pk = min(piece_px, npx - k * piece_px);
-        const unsigned char* base = route_raw + L.ring + (k & 1) * piece_bytes;
+        const unsigned char* base = route_raw + L.ring + (k % kRouteRing) * piece_bytes;
         for (int px = pl; px < pk; px += lanes_p)
           add_vec<T, VEC>(base + px * row_bytes + v * (VEC * sizeof(T)), acc);
       }
       __syncthreads();  // every reader is done with this slot
-      if (t == 0 && k + 2 < npieces && ok) issue(k + 2);
+      if (t == 0 && k + kRouteRing < npieces && ok) issue(k + kRouteRing);
     }
     if (active) {
 #pragma unroll
@@ -249,8 +251,9 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
   cluster.sync();  // remote stores visible to rank 0; with Wr staged, peers may exit after this
   if (*abort_flag && t == 0) {
     // a bounded wait gave up: let the copies still in flight land before exit
-    for (int k = (issued > 2 ? issued - 2 : 0); k < issued; ++k)
-      wait_drain(bar0 + 8u * (k & 1), static_cast<uint32_t>(k >> 1) & 1u, p.wait_ns, p.err);
+    for (int k = (issued > kRouteRing ? issued - kRouteRing : 0); k < issued; ++k)
+      wait_drain(bar0 + 8u * (k % kRouteRing), static_cast<uint32_t>(k / kRouteRing) & 1u,
+                 p.wait_ns, p.err);
     if (p.wr_smem) wait_drain(wrbar, 0, p.wait_ns, p.err);
   }
   const float inv_hw = 1.0f / static_cast<float>(p.HW);

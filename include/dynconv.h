@@ -298,15 +298,21 @@ unsigned long long dynconv_launch_count(void);
  * four K steps per unit), no pooled sums are asked for and the shape fits it;
  * 2 the persistent kernel whenever it fits; 0 always one CTA per unit.
  * key 10: PREMIX with n > 8 when every sample's mixed kernel together is much
- * larger than the L2: 1 (default) mixes and convolves one group (of samples,
- * or of 128-channel tiles) at a time through two workspace slots, the mixing
- * of the next group on an internal stream overlapping the convolution of the
- * current one; 0 mixes every sample's kernel first, then convolves; a value
+ * larger than the L2: 1 mixes and convolves one group (of samples, or of
+ * 128-channel tiles) at a time through two workspace slots, the mixing of
+ * the next group on an internal stream overlapping the convolution of the
+ * current one; 0 (default; measured faster on B200 so far) mixes every
+ * sample's kernel first, then convolves; a value
  * of 4096 or more turns the grouped form on for every size, with groups of
  * about that many bytes (for tests of ragged groups).
  * key 11: the backward's mixing gradient: 1 (default) the tensor-core kernel
  * (per-sample weight gradients as bf16 hi / lo planes, one pass for the
  * expert and attention gradients) when it applies; 0 the CUDA-core kernel.
+ * key 12: the epilogue of the tensor-core mixing GEMM: 0 (default) stages
+ * each tile through shared memory and writes whole rows; 1 stores each
+ * thread's 32 mixed weights straight from registers (two 32-byte stores) when
+ * the kernel size is a multiple of 16 and the workspace 32-byte aligned
+ * (measured slower on B200). For measurements.
  * Returns DYNCONV_OK or DYNCONV_ERR_INVALID_ARG. */
 int dynconv_test_hook(int key, long long value);
 

@@ -142,7 +142,9 @@ def test_test_hook_arguments(lib):
     assert dc.dynconv_test_hook(10, 100) == dc.ERR_INVALID_ARG   # group bytes below 4096
     assert dc.dynconv_test_hook(10, -1) == dc.ERR_INVALID_ARG
     assert dc.dynconv_test_hook(10, 1 << 20) == dc.OK
-    assert dc.dynconv_test_hook(10, 1) == dc.OK
+    assert dc.dynconv_test_hook(10, 0) == dc.OK
+    assert dc.dynconv_test_hook(12, 2) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(12, 1) == dc.OK
 
 
 def test_pooled_entry_points_host_side(lib):
