@@ -242,10 +242,11 @@ namespace dc {
 //    the sample's attentions (and channel factors) stored by its lanes;
 //  * the compute warps first mix the tile's kernels together (CC*K*K weights,
 //    CC biases, fp32, from the resident slabs) into the stage, then each thread
-//    takes TWO adjacent output columns of ONE channel pair and walks the input
-//    rows of the band: for every input row it loads K+1 packed pairs and adds
-//    them into the K output rows (x 2 columns) that use that input row
-//    (vertical accumulators, packed fp32x2 FMAs: 2*K*K per row for K+1 loads);
+//    takes NC (2 or 4) adjacent output columns of ONE channel pair and walks
+//    the input rows of the band: for every input row it loads K+NC-1 packed
+//    pairs and adds them into the K output rows (x NC columns) that use that
+//    input row (vertical accumulators, packed fp32x2 FMAs: NC*K*K per row for
+//    K+NC-1 loads);
 //    an output row is stored when its last input row is in. The rows are
 //    walked in groups of K with every accumulator slot a compile-time
 //    register; only the first and the last groups carry the band-edge tests.
@@ -256,19 +257,25 @@ namespace dc {
 // all warps leave.
 // ---------------------------------------------------------------------------
 
-template <int K>
+template <int K, int NC>
 struct DwpShape;
-// Compute threads per CTA and the register cap that fits them (plus the
+// Most compute threads per CTA and the register cap that fits them (plus the
 // producer warp) in one SM's 64 K registers -- registers are granted to warps
 // in groups of four, so the cap is 64 K / (32 * warps rounded up to 4),
-// rounded down to 8: the K*K packed weights stay in registers for the whole
-// tile.
+// rounded down to 8: the K*K packed weights and the K x NC open output rows
+// stay in registers for the whole tile. NC = output columns per thread.
 template <>
-struct DwpShape<3> { static constexpr int kComp = 736; static constexpr int kRegs = 80; };
+struct DwpShape<3, 2> { static constexpr int kComp = 736; static constexpr int kRegs = 80; };
 template <>
-struct DwpShape<5> { static constexpr int kComp = 480; static constexpr int kRegs = 128; };
+struct DwpShape<5, 2> { static constexpr int kComp = 480; static constexpr int kRegs = 128; };
 template <>
-struct DwpShape<7> { static constexpr int kComp = 352; static constexpr int kRegs = 168; };
+struct DwpShape<7, 2> { static constexpr int kComp = 352; static constexpr int kRegs = 168; };
+template <>
+struct DwpShape<3, 4> { static constexpr int kComp = 608; static constexpr int kRegs = 96; };
+template <>
+struct DwpShape<5, 4> { static constexpr int kComp = 352; static constexpr int kRegs = 168; };
+template <>
+struct DwpShape<7, 4> { static constexpr int kComp = 224; static constexpr int kRegs = 255; };
 
 constexpr int kDwpMaxStages = 4;
 constexpr int kErrWaitDwp = 0x108;
@@ -277,11 +284,13 @@ struct DwpParams {
   int B, C, H, W, pad, n, Ho, Wo;
   int CC;           // channels per chunk (multiple of 8)
   int CB;           // output columns per tile
+  int nc;           // output columns per compute thread (2 or 4)
+  int ncomp;        // compute threads (a multiple of 32; the producer warp follows)
   int RB;           // output rows per tile
   int nchunks, bands, cbands;
   int S;            // stages in flight
   int stage_bytes;  // one stage: box | misc (128-aligned)
-  int box_bytes;    // (RB+K-1) * (even(CB)+K-1) * CC * 2
+  int box_bytes;    // (RB+K-1) * (CB rounded up to nc, + K-1) * CC * 2
   int misc_off;     // alpha[n] | a_in[CC] | a_out[CC] | chan_add[CC], from the stage base
   int w_off;        // two mixed-kernel buffers, each [K*K][CC] weights + [CC] biases (fp32)
   int e_off;        // resident expert slabs [n][CC][K*K] bf16
@@ -301,19 +310,19 @@ struct DwpParams {
 
 // CCPT: the channel pairs per chunk when known at compile time (the stride
 // between staged columns, so every window load has an immediate offset), or
-// 0 for any chunk width.
-template <int K, int CCPT>
-__global__ void __maxnreg__(DwpShape<K>::kRegs)
+// 0 for any chunk width. NC: output columns per compute thread.
+template <int K, int CCPT, int NC>
+__global__ void __maxnreg__((DwpShape<K, NC>::kRegs))
     depthwise_pipe_kernel(const __grid_constant__ CUtensorMap xmap, DwpParams p) {
   constexpr int KK = K * K;
-  constexpr int NCOMP = DwpShape<K>::kComp;
-  constexpr int NWARP_C = NCOMP / 32;
+  const int NCOMP = p.ncomp;
+  const int NWARP_C = NCOMP >> 5;
   extern __shared__ __align__(128) unsigned char dwp_raw[];
   unsigned char* sm = dwp_raw + ((128u - (smem_u32(dwp_raw) & 127u)) & 127u);
   const int t = threadIdx.x;
   const int warp = t >> 5, lane = t & 31;
   const int CCp = CCPT > 0 ? CCPT : (p.CC >> 1);
-  const int TC = ((p.CB + 1) & ~1) + K - 1;  // staged columns: even tile width + halo
+  const int TC = (p.CB + NC - 1) / NC * NC + K - 1;  // staged columns: tile width + halo
 
   // This CTA's chunk and a contiguous run of the chunk's tiles, so that
   // consecutive tiles are the row bands of one sample and share its kernels.
@@ -415,8 +424,8 @@ __global__ void __maxnreg__(DwpShape<K>::kRegs)
   // ================================ compute ================================
   if (my_tiles == 0) return;
   if (!wait_bounded(ebar, 0, ctl, kErrWaitDwp)) return;
-  const int cpair = t / CCp, pair = t - (t / CCp) * CCp;
-  const int col = 2 * cpair;  // this thread's output columns col, col + 1 in the tile
+  const int cgrp = t / CCp, pair = t - (t / CCp) * CCp;
+  const int col = NC * cgrp;  // this thread's output columns col .. col + NC - 1 in the tile
   const int w_floats = (KK + 1) * p.CC;
   // this thread's mixing items it = t, t + NCOMP, ...: (tap, channel) walked
   // incrementally (tap KK = the bias)
@@ -478,7 +487,7 @@ __global__ void __maxnreg__(DwpShape<K>::kRegs)
     const bool active = col < p.CB && ow < p.Wo && c < p.C;
     if (active) {
       const bool scale_out = p.a_out != nullptr;
-      const bool second = col + 1 < p.CB && ow + 1 < p.Wo;  // the column pair's second column
+      const int ncv = min(NC, min(p.CB - col, p.Wo - ow));  // columns of this thread in the image
       const uint32_t* xw = reinterpret_cast<const uint32_t*>(st) + col * CCp + pair;
       const int row_words = TC * CCp;
       const size_t ystride = static_cast<size_t>(p.Wo) * p.C;  // one output row
@@ -487,17 +496,17 @@ __global__ void __maxnreg__(DwpShape<K>::kRegs)
           p.y + (static_cast<size_t>(b) * p.Ho * p.Wo + static_cast<size_t>(oh0) * p.Wo + ow) * p.C + c;
       const int rows_out = min(p.RB, p.Ho - oh0);  // rows of this band inside the image
       const int rows_in = p.RB + K - 1;
-      uint64_t acc[K][2];  // open output rows, slot o % K
-      auto store_row = [&](uint64_t (&a)[2], int o) {
+      uint64_t acc[K][NC];  // open output rows, slot o % K
+      auto store_row = [&](const uint64_t (&a)[NC], int o) {
         if (o < rows_out) {
           __nv_bfloat16* dst = ydst0 + static_cast<size_t>(o) * ystride;
-          float l0 = __uint_as_float(static_cast<uint32_t>(a[0]));
-          float h0 = __uint_as_float(static_cast<uint32_t>(a[0] >> 32));
-          float l1 = __uint_as_float(static_cast<uint32_t>(a[1]));
-          float h1 = __uint_as_float(static_cast<uint32_t>(a[1] >> 32));
-          if (scale_out) { l0 *= ao0; h0 *= ao1; l1 *= ao0; h1 *= ao1; }
-          *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(l0, h0);
-          if (second) *reinterpret_cast<uint32_t*>(dst + p.C) = pack_bf16x2(l1, h1);
+#pragma unroll
+          for (int q = 0; q < NC; ++q) {
+            float l = __uint_as_float(static_cast<uint32_t>(a[q]));
+            float h = __uint_as_float(static_cast<uint32_t>(a[q] >> 32));
+            if (scale_out) { l *= ao0; h *= ao1; }
+            if (q == 0 || q < ncv) *reinterpret_cast<uint32_t*>(dst + q * p.C) = pack_bf16x2(l, h);
+          }
         }
       };
       // One group of K input rows starting at ir0 (a multiple of K): input
@@ -516,9 +525,9 @@ __global__ void __maxnreg__(DwpShape<K>::kRegs)
           const int ir = ir0 + j;
           if (KIND == TAIL && j >= K - 1) continue;              // ir >= RB + K - 1
           if (KIND == GENERIC && ir >= rows_in) continue;
-          uint64_t xv[K + 1];
+          uint64_t xv[K + NC - 1];
 #pragma unroll
-          for (int kw = 0; kw <= K; ++kw) xv[kw] = bf16x2_to_f32x2(xr[kw * CCp]);
+          for (int kw = 0; kw < K + NC - 1; ++kw) xv[kw] = bf16x2_to_f32x2(xr[kw * CCp]);
 #pragma unroll
           for (int kh = K - 1; kh >= 0; --kh) {
             const int o = ir - kh;
@@ -529,19 +538,18 @@ __global__ void __maxnreg__(DwpShape<K>::kRegs)
             else if (KIND == TAIL) live = j < kh;        // o < RB; o >= RB - K + 1 >= 0
             else live = o >= 0 && o < p.RB;
             if (!live) continue;
-            uint64_t a0 = kh == 0 ? bias2 : acc[slot][0];
-            uint64_t a1 = kh == 0 ? bias2 : acc[slot][1];
+            uint64_t a[NC];
 #pragma unroll
-            for (int kw = 0; kw < K; ++kw) {
-              a0 = ffma2(xv[kw], w2[kh * K + kw], a0);
-              a1 = ffma2(xv[kw + 1], w2[kh * K + kw], a1);
-            }
+            for (int q = 0; q < NC; ++q) a[q] = kh == 0 ? bias2 : acc[slot][q];
+#pragma unroll
+            for (int kw = 0; kw < K; ++kw)
+#pragma unroll
+              for (int q = 0; q < NC; ++q) a[q] = ffma2(xv[kw + q], w2[kh * K + kw], a[q]);
             if (kh == K - 1) {
-              uint64_t done[2] = {a0, a1};
-              store_row(done, o);
+              store_row(a, o);
             } else {
-              acc[slot][0] = a0;
-              acc[slot][1] = a1;
+#pragma unroll
+              for (int q = 0; q < NC; ++q) acc[slot][q] = a[q];
             }
           }
         }

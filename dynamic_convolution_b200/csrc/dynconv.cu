@@ -61,10 +61,17 @@ std::atomic<int> g_inject_skip{0};
 std::atomic<int> g_route_split{0};  // 0: automatic
 std::atomic<int> g_use_pdl{1};      // programmatic launch edges on forward kernels
 std::atomic<int> g_stream_mix{0};   // PREMIX with n <= 8: mixing streamed into the convolution
-std::atomic<int> g_premix_mixer{0};  // 0 automatic, 1 tensor-core GEMM, 2 CUDA cores (n <= 8)
-std::atomic<int> g_dw_kernel{0};     // 0 pipelined depthwise kernel when it fits, 1 the per-tile one
+std::atomic<int> g_premix_mixer{0};  // 0 automatic, 1 tensor-core GEMM, 2 CUDA cores (n <= 8),
+                                     // 3 the transposed tensor-core GEMM (B <= 256)
+std::atomic<int> g_dw_kernel{0};     // 0 pipelined depthwise kernel when it fits, 1 the per-tile one,
+                                     // 2 / 3 the pipelined one with 2 / 4 columns per thread
+constexpr int kDwpDefaultNc = 2;     // columns per thread of the pipelined depthwise kernel
+constexpr int kTransposedMixMax = 0;   // batches up to this mix with the transposed GEMM by default
+                                     // (none: the M = samples GEMM with eight epilogue warps
+                                     // measured faster even at 32 samples)
 std::atomic<int> g_conv_persist{1};  // PREMIX convolution: 1 persistent kernel when it fits, 0 one CTA per unit
-std::atomic<int> g_group_mix{0};     // PREMIX, n > 8, large B*|W|: 1 grouped mixing pipeline, 0 one pass
+std::atomic<int> g_group_mix{0};     // PREMIX, n > 8, large B*|W|: 0 one pass, 1 grouped mixing
+                                     // pipeline (concurrent), 2 grouped in sequence
 std::atomic<int> g_premix_direct{0}; // premix epilogue: 1 stores from registers when aligned, 0 staged
 std::atomic<int> g_mixgrad_tc{1};    // backward: 1 tensor-core mixing gradient when it fits, 0 CUDA cores
 std::atomic<long long> g_group_bytes{40LL << 20};  // target bytes of one group's mixed kernels
@@ -345,69 +352,105 @@ bool depthwise_ok(const dynconv_desc* d) {
          out_size(d->W, d->KW, 1, d->pad) >= 1;
 }
 
-// Plan of the pipelined depthwise kernel (depthwise_pipe_kernel): chunk width
-// CC and tile width CB so that the CC/2 x CB compute threads fill the kernel's
-// thread count with the least waste (idle threads, channels past C, columns
-// past W_out); then the tallest row band RB for which three stages, the
-// resident expert and bias slabs and the barriers fit in shared memory (two
-// stages when three do not fit). False when the shape does not fit.
-bool dwp_plan(const dynconv_desc* d, int sms, int max_smem, bool has_bias, dc::DwpParams* p,
-              int* grid, size_t* smem_out) {
+// Plan of the pipelined depthwise kernel (depthwise_pipe_kernel) with `nc`
+// output columns per thread: chunk width CC and tile width CB so that the
+// CC/2 x ceil(CB/nc) compute threads fill the kernel's most threads with the
+// least waste (idle threads, channels past C, columns past W_out); then the
+// tallest row band RB for which three stages, the resident expert and bias
+// slabs and the barriers fit in shared memory (two stages when three do not
+// fit). False when the shape does not fit.
+bool dwp_plan(const dynconv_desc* d, int sms, int max_smem, bool has_bias, int nc,
+              dc::DwpParams* p, int* grid, size_t* smem_out) {
   const int K = d->KH, KK = K * K;
-  const int ncomp = K == 3 ? dc::DwpShape<3>::kComp : K == 5 ? dc::DwpShape<5>::kComp
-                                                            : dc::DwpShape<7>::kComp;
+  int ncomp = 0;
+  if (nc == 2)
+    ncomp = K == 3 ? dc::DwpShape<3, 2>::kComp : K == 5 ? dc::DwpShape<5, 2>::kComp
+                                                        : dc::DwpShape<7, 2>::kComp;
+  else if (nc == 4)
+    ncomp = K == 3 ? dc::DwpShape<3, 4>::kComp : K == 5 ? dc::DwpShape<5, 4>::kComp
+                                                        : dc::DwpShape<7, 4>::kComp;
+  else
+    return false;
   const int Ho = out_size(d->H, K, 1, d->pad), Wo = out_size(d->W, K, 1, d->pad);
   const int C = d->C_in;
+  auto a128 = [](size_t v) { return (v + 127) / 128 * 128; };
+  const size_t bars = 8 * (3 * dc::kDwpMaxStages + 1) + 16;
+  // Shared bytes of a chunk width: the resident slabs, the two mixed-kernel
+  // buffers, one stage's attentions; and the band plan of a (CC, CB): the
+  // tallest band for which S = 3 stages fit (S = 2 when that band would be
+  // shorter than min(Ho, 8)), balanced over the bands, then rounded up to a
+  // multiple of K when that still fits (every band-edge test of the kernel
+  // is then resolved at compile time).
+  struct Slabs { size_t e, eb, w, misc; };
+  auto slabs_of = [&](int CC) {
+    return Slabs{a128(static_cast<size_t>(d->n) * CC * KK * 2),
+                 has_bias ? a128(static_cast<size_t>(d->n) * CC * 4) : 0,
+                 2 * a128(static_cast<size_t>(KK + 1) * CC * 4),
+                 a128(static_cast<size_t>(d->n + 3 * CC) * 4)};
+  };
+  auto band_plan = [&](int CC, int CB, int* S, int* RB, int* bands) {
+    const Slabs sl = slabs_of(CC);
+    const size_t fixed = 128 + sl.w + sl.e + sl.eb + bars;
+    const size_t TC = static_cast<size_t>((CB + nc - 1) / nc * nc + K - 1);
+    if (fixed >= static_cast<size_t>(max_smem)) return false;
+    for (int st : {3, 2}) {
+      const size_t per = (static_cast<size_t>(max_smem) - fixed) / st;
+      if (per <= sl.misc) continue;
+      const long long rows = static_cast<long long>((per - sl.misc) / 128 * 128 / (TC * CC * 2));
+      const long long rb = std::min<long long>({rows - (K - 1), Ho, 256 - (K - 1)});
+      if (rb <= 0 || (rb < std::min(Ho, 8) && st == 3)) continue;
+      int nb = static_cast<int>((Ho + rb - 1) / rb);
+      int r = (Ho + nb - 1) / nb;
+      const int rk = (r + K - 1) / K * K;
+      if (rk <= rb) {
+        r = rk;
+        nb = (Ho + r - 1) / r;
+      }
+      *S = st;
+      *RB = r;
+      *bands = nb;
+      return true;
+    }
+    return false;
+  };
   double best = -1;
   int bCC = 0, bCB = 0;
   for (int CC = 8; CC <= std::min(256, (C + 7) / 8 * 8); CC += 8) {
     const int nch = (C + CC - 1) / CC;
-    for (int CB = 1; CB <= std::min(Wo, 254 - (K - 1)); ++CB) {
-      const int thr = CC / 2 * ((CB + 1) / 2);  // one thread per channel pair and column pair
+    for (int CB = 1; CB <= std::min(Wo, 256 - (K - 1) - (nc - 1)); ++CB) {
+      const int thr = CC / 2 * ((CB + nc - 1) / nc);  // one thread per channel pair and column group
       if (thr > ncomp) break;
+      int S = 0, RB = 0, bands = 0;
+      if (!band_plan(CC, CB, &S, &RB, &bands)) continue;
       const int cbands = (Wo + CB - 1) / CB;
-      // the halo columns are staged for every tile: a mild preference for wide
-      // tiles; a warp of 32 consecutive pairs of one column pair reads without
-      // bank conflicts, other chunk widths with some
-      const double eff = static_cast<double>(thr) / ncomp * C / (nch * CC) * Wo / (cbands * CB) *
-                         (1.0 - 0.25 * (K - 1) / (CB + K - 1.0)) *
-                         ((CC / 2) % 32 == 0 ? 1.0 : 0.85);
+      const int warps = (thr + 31) / 32;
+      // useful work: channels past C, columns past W_out (the tile width
+      // rounded up to nc), rows past H_out and the idle lanes of the last
+      // warp are waste; the halo columns and rows are staged for every tile
+      // (a mild preference for wide and tall tiles); a warp of 32 consecutive
+      // pairs of one column group reads without bank conflicts, other chunk
+      // widths with some; fewer than 8 compute warps hide latency less well
+      const double eff =
+          static_cast<double>(C) / (nch * CC) * Wo /
+          (static_cast<double>(cbands) * ((CB + nc - 1) / nc * nc)) * Ho /
+          (static_cast<double>(bands) * RB) * thr / (32.0 * warps) *
+          (1.0 - 0.25 * (K - 1) / (CB + K - 1.0)) * (1.0 - 0.25 * (K - 1) / (RB + K - 1.0)) *
+          ((CC / 2) % 32 == 0 ? 1.0 : 0.85) * std::min(1.0, warps / 8.0);
       if (eff > best + 1e-9) { best = eff; bCC = CC; bCB = CB; }
     }
   }
   if (bCC == 0) return false;
   const int CC = bCC, CB = bCB;
-  auto a128 = [](size_t v) { return (v + 127) / 128 * 128; };
-  const size_t e_bytes = a128(static_cast<size_t>(d->n) * CC * KK * 2);
-  const size_t eb_bytes = has_bias ? a128(static_cast<size_t>(d->n) * CC * 4) : 0;
-  const size_t w_bytes = 2 * a128(static_cast<size_t>(KK + 1) * CC * 4);  // two buffers
-  const size_t misc_bytes = a128(static_cast<size_t>(d->n + 3 * CC) * 4);
-  const size_t bars = 8 * (3 * dc::kDwpMaxStages + 1) + 16;
-  const int TC = ((CB + 1) & ~1) + K - 1;  // staged columns
-  auto stage_of = [&](int RB) {
-    return a128(static_cast<size_t>(RB + K - 1) * TC * CC * 2) + misc_bytes;
-  };
-  int S = 0, RBmax = 0;
-  for (int st : {3, 2}) {
-    int rb = std::min(Ho, 256 - (K - 1));
-    while (rb > 0 && 128 + st * stage_of(rb) + w_bytes + e_bytes + eb_bytes + bars >
-                         static_cast<size_t>(max_smem))
-      --rb;
-    if (rb > 0 && (rb >= std::min(Ho, 8) || st == 2)) { S = st; RBmax = rb; break; }
-  }
-  if (S == 0 || RBmax == 0) return false;
-  int bands = (Ho + RBmax - 1) / RBmax;
-  int RB = (Ho + bands - 1) / bands;
-  // a band height that is a multiple of K lets the kernel resolve every
-  // band-edge test at compile time
-  const int RBk = (RB + K - 1) / K * K;
-  if (RBk <= RBmax) {
-    RB = RBk;
-    bands = (Ho + RB - 1) / RB;
-  }
+  int S = 0, RB = 0, bands = 0;
+  if (!band_plan(CC, CB, &S, &RB, &bands)) return false;
+  const Slabs sl = slabs_of(CC);
+  const size_t e_bytes = sl.e, eb_bytes = sl.eb, w_bytes = sl.w, misc_bytes = sl.misc;
+  const int TC = (CB + nc - 1) / nc * nc + K - 1;  // staged columns
   std::memset(p, 0, sizeof(*p));
   p->B = d->B; p->C = C; p->H = d->H; p->W = d->W; p->pad = d->pad; p->n = d->n;
   p->Ho = Ho; p->Wo = Wo; p->CC = CC; p->CB = CB; p->RB = RB;
+  p->nc = nc;
+  p->ncomp = (CC / 2 * ((CB + nc - 1) / nc) + 31) / 32 * 32;
   p->nchunks = (C + CC - 1) / CC;
   p->bands = bands;
   p->cbands = (Wo + CB - 1) / CB;
@@ -769,6 +812,122 @@ int run_grouped(const dynconv_desc* d, const GroupPlan& gp, const DeviceState* s
   return DYNCONV_OK;
 }
 
+// The grouped PREMIX form in sequence on the caller's stream: for each group
+// the mixing kernel (all SMs) writes the group's mixed kernels into one
+// workspace slot, then the convolution (all SMs) reads them back -- from L2,
+// since the slot (tens of MB) is far smaller than the L2 and was just
+// written. No internal stream: every launch carries a programmatic edge, and
+// the convolution never signals its dependents early, so the next group's
+// mixing reads and overwrites the slot only once the convolution has
+// completed.
+int run_grouped_seq(const dynconv_desc* d, const GroupPlan& gp, const DeviceState* st,
+                    const void* x, const void* experts, const float* alpha, const float* bias,
+                    void* y, void* ws, const float* a_out, const float* chan_add,
+                    float chan_scale, cudaStream_t stream) {
+  const size_t taps_cin = static_cast<size_t>(d->KH) * d->KW * d->C_in;
+  const size_t wsize = d->C_out * taps_cin;
+  std::vector<TcPlan> plans(gp.groups);
+  std::vector<dynconv_desc> subs(gp.groups);
+  for (int g = 0; g < gp.groups; ++g) {
+    dynconv_desc s = *d;
+    if (gp.kind == 1) s.B = std::min(gp.per, d->B - g * gp.per);
+    else s.C_out = std::min(gp.per, d->C_out - g * gp.per);
+    subs[g] = s;
+    // channel groups write into y at a channel offset: only the persistent
+    // kernel takes one
+    const bool ok = gp.kind == 2 ? tc_plan_persist(&s, st->sms, st->max_smem_optin, &plans[g])
+                                 : tc_plan(&s, DYNCONV_VARIANT_PREMIX, st->sms, st->max_smem_optin,
+                                           &plans[g]);
+    if (!ok) return DYNCONV_ERR_UNSUPPORTED;
+  }
+  const __nv_bfloat16* E = static_cast<const __nv_bfloat16*>(experts);
+  int rc = DYNCONV_OK;
+  for (int g = 0; g < gp.groups; ++g) {
+    const dynconv_desc& s = subs[g];
+    const size_t b0 = gp.kind == 1 ? static_cast<size_t>(g) * gp.per : 0;
+    const size_t c0 = gp.kind == 2 ? static_cast<size_t>(g) * gp.per : 0;
+    const long long wg = static_cast<long long>(s.C_out) * static_cast<long long>(taps_cin);
+    cudaError_t e;
+    if (g_premix_mixer.load() == 3 && s.B <= 256) {
+      dc::PremixTLaunch pl;
+      rc = dc::plan_premix_t(E + c0 * taps_cin, static_cast<long long>(wsize), alpha + b0 * d->n,
+                             static_cast<__nv_bfloat16*>(ws), s.B, d->n, wg, st->err,
+                             g_wait_ns.load(), st->sms, g_encode, &pl);
+      if (rc == -2) {
+        std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(grouped premix) failed");
+        return DYNCONV_ERR_CUDA;
+      }
+      if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
+      e = ensure_smem(dc::premix_t_kernel, pl.smem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix_t)");
+      e = launch_pdl(dc::premix_t_kernel, dim3(pl.grid), dim3(dc::kPtThreads), pl.smem, stream,
+                     pl.emap, pl.p);
+      if (e != cudaSuccess) {
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return cuda_fail(e, "premix_t_kernel launch (grouped)");
+      }
+      rc = check_launch("premix_t_kernel (grouped)");
+    } else {
+      dc::PremixLaunch pl;
+      rc = dc::plan_premix(E + c0 * taps_cin, alpha + b0 * d->n, static_cast<__nv_bfloat16*>(ws),
+                           s.B, d->n, wg, st->err, g_wait_ns.load(), st->sms, g_encode, &pl,
+                           static_cast<long long>(wsize), g_premix_direct.load() != 0);
+      if (rc == -2) {
+        std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(grouped premix) failed");
+        return DYNCONV_ERR_CUDA;
+      }
+      if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
+      e = ensure_smem(dc::premix_kernel, pl.smem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
+      e = launch_pdl(dc::premix_kernel, dim3(pl.grid), dim3(dc::kPmThreads), pl.smem, stream,
+                     pl.emap, pl.p);
+      if (e != cudaSuccess) {
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return cuda_fail(e, "premix_kernel launch (grouped)");
+      }
+      rc = check_launch("premix_kernel (grouped)");
+    }
+    if (rc) return rc;
+    TcPlan& pp = plans[g];
+    const size_t xoff = b0 * d->H * d->W * d->C_in;
+    const size_t yoff = b0 * d->H * d->W * d->C_out;
+    pp.p.experts = E;
+    pp.p.alpha = alpha + b0 * d->n;
+    pp.p.bias = bias;
+    pp.p.y = static_cast<__nv_bfloat16*>(y) + yoff;
+    pp.p.err = st->err;
+    pp.p.wait_ns = g_wait_ns.load();
+    pp.p.a_out = a_out ? a_out + b0 * d->C_out : nullptr;
+    pp.p.chan_add = chan_add ? chan_add + b0 * d->C_out : nullptr;
+    pp.p.chan_scale = chan_scale;
+    CUtensorMap xmap, wmap;
+    rc = encode_x_map(&xmap, static_cast<const __nv_bfloat16*>(x) + xoff, &s, pp.p.Wp,
+                      pp.p.b_box_rows);
+    if (rc) return rc;
+    rc = encode_w_map(&wmap, ws, &s);
+    if (rc) return rc;
+    if (gp.kind == 1) {
+      rc = launch_premix_conv(&s, pp, st, static_cast<const __nv_bfloat16*>(x) + xoff, xmap, wmap,
+                              stream);
+    } else {
+      pp.p.co_base = static_cast<int>(c0);
+      pp.p.ld_c = d->C_out;
+      pp.p.x_early = g_use_pdl.load() ? 1 : 0;
+      e = ensure_smem(dc::tc_conv_persist_kernel, pp.smem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc_conv_persist)");
+      e = launch_pdl(dc::tc_conv_persist_kernel, dim3(pp.grid), dim3(dc::kTcThreads), pp.smem,
+                     stream, xmap, wmap, pp.p);
+      if (e != cudaSuccess) {
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return cuda_fail(e, "tc_conv_persist_kernel launch (grouped)");
+      }
+      rc = check_launch("tc_conv_persist_kernel (grouped)");
+    }
+    if (rc) return rc;
+  }
+  return DYNCONV_OK;
+}
+
 // State slot of the streamed mixing for (device, stream): launches on one
 // stream are ordered, so they may share a slot; every stream gets a slot of
 // its own, kept for the life of the process. When all kMcSlots slots of the
@@ -934,9 +1093,13 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   // large B*|W| with the tensor-core mixer: the grouped pipeline through L2
   if (g_group_mix.load() && ysum == nullptr && a_in == nullptr && g_premix_mixer.load() != 2) {
     const GroupPlan gp = group_plan(d);
-    if (gp.kind != 0 && ws_bytes >= 2 * gp.slot && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0) {
-      rc = run_grouped(d, gp, st, x, experts, alpha, bias, y, ws, a_out, chan_add, chan_scale,
-                       stream);
+    const bool seq = g_group_mix.load() == 2;
+    if (gp.kind != 0 && ws_bytes >= (seq ? 1 : 2) * gp.slot &&
+        (reinterpret_cast<uintptr_t>(ws) & 255u) == 0) {
+      rc = seq ? run_grouped_seq(d, gp, st, x, experts, alpha, bias, y, ws, a_out, chan_add,
+                                 chan_scale, stream)
+               : run_grouped(d, gp, st, x, experts, alpha, bias, y, ws, a_out, chan_add,
+                             chan_scale, stream);
       if (rc != DYNCONV_ERR_UNSUPPORTED) return rc;
     }
   }
@@ -975,6 +1138,33 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
     if (g_premix_mixer.load() == 2) return DYNCONV_ERR_UNSUPPORTED;
   }
   if (a_in != nullptr) return DYNCONV_ERR_UNSUPPORTED;  // the GEMM mixer does not take it
+  const long long wsize_all = static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in;
+  const int mixer = g_premix_mixer.load();
+  if ((mixer == 3 && d->B <= 256) || (mixer == 0 && d->B <= kTransposedMixMax)) {
+    // the transposed mixing GEMM (M = weights, N = samples) over the whole batch
+    dc::PremixTLaunch tl;
+    rc = dc::plan_premix_t(static_cast<const __nv_bfloat16*>(experts), wsize_all, alpha,
+                           static_cast<__nv_bfloat16*>(ws), d->B, d->n, wsize_all, st->err,
+                           g_wait_ns.load(), st->sms, g_encode, &tl);
+    if (rc == -2) {
+      std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(premix_t) failed");
+      return DYNCONV_ERR_CUDA;
+    }
+    if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
+    cudaError_t e = ensure_smem(dc::premix_t_kernel, tl.smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix_t)");
+    e = launch_pdl(dc::premix_t_kernel, dim3(tl.grid), dim3(dc::kPtThreads), tl.smem, stream,
+                   tl.emap, tl.p);
+    if (e != cudaSuccess) {
+      g_launches.fetch_add(1, std::memory_order_relaxed);
+      return cuda_fail(e, "premix_t_kernel launch");
+    }
+    rc = check_launch("premix_t_kernel");
+    if (rc) return rc;
+    rc = encode_w_map(&wmap, ws, d);
+    if (rc) return rc;
+    return launch_premix_conv(d, plan, st, x, xmap, wmap, stream);
+  }
   dc::PremixLaunch pl;
   rc = dc::plan_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
                        static_cast<__nv_bfloat16*>(ws), d->B, d->n,
@@ -1051,7 +1241,7 @@ int dynconv_test_hook(int key, long long value) {
     return DYNCONV_OK;
   }
   if (key == 7) {
-    if (value < 0 || value > 2) return DYNCONV_ERR_INVALID_ARG;
+    if (value < 0 || value > 3) return DYNCONV_ERR_INVALID_ARG;
     g_premix_mixer.store(static_cast<int>(value));
     return DYNCONV_OK;
   }
@@ -1061,7 +1251,7 @@ int dynconv_test_hook(int key, long long value) {
     return DYNCONV_OK;
   }
   if (key == 8) {
-    if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
+    if (value < 0 || value > 3) return DYNCONV_ERR_INVALID_ARG;
     g_dw_kernel.store(static_cast<int>(value));
     return DYNCONV_OK;
   }
@@ -1081,10 +1271,15 @@ int dynconv_test_hook(int key, long long value) {
     return DYNCONV_OK;
   }
   if (key == 10) {
-    if (value < 0 || (value > 1 && value < 4096)) return DYNCONV_ERR_INVALID_ARG;
-    g_group_mix.store(value != 0 ? 1 : 0);
-    g_group_bytes.store(value >= 4096 ? value : (40LL << 20));
-    g_group_min.store(value >= 4096 ? 0 : (64LL << 20));
+    // 0 off, 1 concurrent groups, 2 sequential groups; >= 4096: concurrent
+    // groups of about that many bytes at every size; a negative value <= -4096:
+    // sequential groups of about -value bytes at every size
+    if (value > 2 && value < 4096) return DYNCONV_ERR_INVALID_ARG;
+    if (value < 0 && value > -4096) return DYNCONV_ERR_INVALID_ARG;
+    const long long bytes = value >= 4096 ? value : value <= -4096 ? -value : 0;
+    g_group_mix.store(value == 0 ? 0 : (value == 2 || value <= -4096) ? 2 : 1);
+    g_group_bytes.store(bytes ? bytes : (40LL << 20));
+    g_group_min.store(bytes ? 0 : (64LL << 20));
     return DYNCONV_OK;
   }
   return DYNCONV_ERR_INVALID_ARG;
@@ -1218,7 +1413,9 @@ int run_depthwise_pipe(const dynconv_desc* d, const DeviceState* st, const void*
   dc::DwpParams p;
   int grid = 0;
   size_t smem = 0;
-  if (!dwp_plan(d, st->sms, st->max_smem_optin, bias != nullptr, &p, &grid, &smem))
+  const int hook = g_dw_kernel.load();
+  const int nc = hook == 3 ? 4 : hook == 2 ? 2 : kDwpDefaultNc;
+  if (!dwp_plan(d, st->sms, st->max_smem_optin, bias != nullptr, nc, &p, &grid, &smem))
     return DYNCONV_ERR_UNSUPPORTED;
   const int K = d->KH;
   p.experts = static_cast<const __nv_bfloat16*>(experts);
@@ -1238,7 +1435,7 @@ int run_depthwise_pipe(const dynconv_desc* d, const DeviceState* st, const void*
                                  static_cast<cuuint64_t>(d->W) * d->C_in * 2,
                                  static_cast<cuuint64_t>(d->H) * d->W * d->C_in * 2};
   const cuuint32_t box[4] = {static_cast<cuuint32_t>(p.CC),
-                             static_cast<cuuint32_t>(((p.CB + 1) & ~1) + K - 1),
+                             static_cast<cuuint32_t>((p.CB + nc - 1) / nc * nc + K - 1),
                              static_cast<cuuint32_t>(p.RB + K - 1), 1u};
   const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
   if (g_encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides,
@@ -1267,14 +1464,19 @@ int run_depthwise_pipe(const dynconv_desc* d, const DeviceState* st, const void*
   };
   // 32 channel pairs per chunk: the window's column stride is a compile-time constant
   const bool c32 = p.CC == 64;
-  if (K == 3)
-    return c32 ? go(dc::depthwise_pipe_kernel<3, 32>, dc::DwpShape<3>::kComp + 32)
-               : go(dc::depthwise_pipe_kernel<3, 0>, dc::DwpShape<3>::kComp + 32);
-  if (K == 5)
-    return c32 ? go(dc::depthwise_pipe_kernel<5, 32>, dc::DwpShape<5>::kComp + 32)
-               : go(dc::depthwise_pipe_kernel<5, 0>, dc::DwpShape<5>::kComp + 32);
-  return c32 ? go(dc::depthwise_pipe_kernel<7, 32>, dc::DwpShape<7>::kComp + 32)
-             : go(dc::depthwise_pipe_kernel<7, 0>, dc::DwpShape<7>::kComp + 32);
+  const int threads = p.ncomp + 32;
+#define DC_DWP_GO(KV, NCV) \
+  return c32 ? go(dc::depthwise_pipe_kernel<KV, 32, NCV>, threads) \
+             : go(dc::depthwise_pipe_kernel<KV, 0, NCV>, threads)
+  if (nc == 4) {
+    if (K == 3) DC_DWP_GO(3, 4);
+    if (K == 5) DC_DWP_GO(5, 4);
+    DC_DWP_GO(7, 4);
+  }
+  if (K == 3) DC_DWP_GO(3, 2);
+  if (K == 5) DC_DWP_GO(5, 2);
+  DC_DWP_GO(7, 2);
+#undef DC_DWP_GO
 }
 
 int resolve_variant(const dynconv_desc* desc, size_t ws_bytes, const DeviceState* st) {
@@ -1320,7 +1522,7 @@ int forward_impl(const dynconv_desc* desc, const void* x, const void* experts,
     case DYNCONV_VARIANT_DEPTHWISE: {
       if (!depthwise_ok(desc)) return DYNCONV_ERR_UNSUPPORTED;
       if (!aligned16(x) || !aligned16(y)) return DYNCONV_ERR_MISALIGNED;
-      if (g_dw_kernel.load() == 0 && aligned16(experts) && (bias == nullptr || aligned16(bias))) {
+      if (g_dw_kernel.load() != 1 && aligned16(experts) && (bias == nullptr || aligned16(bias))) {
         rc = run_depthwise_pipe(desc, st, x, experts, alpha, bias, y, a_in, a_out, chan_add,
                                 chan_scale, s);
         if (rc != DYNCONV_ERR_UNSUPPORTED) {

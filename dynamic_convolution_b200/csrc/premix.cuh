@@ -14,10 +14,14 @@
 //    rows per expert with the 128-byte swizzle; 64-weight atoms sit
 //    LBO = K*128 bytes apart, 8-expert groups SBO = 1024 bytes apart.
 //  * D (fp32) lives in TMEM, double-buffered (2 x 256 columns) so the
-//    epilogue of one tile overlaps the MMAs of the next; the epilogue rounds to
-//    bf16 and each thread (one sample) stores 64 contiguous bytes per chunk,
-//    straight from registers as two whole 32-byte sectors when every kernel
-//    is a multiple of 16 weights, else through an XOR-staged shared tile.
+//    epilogue of one tile overlaps the MMAs of the next. Eight epilogue warps,
+//    two per TMEM lane quarter (32 samples), each taking one 128-column half
+//    of the tile, two 32-column TMEM loads in flight: each rounds to bf16,
+//    stages its 32 x 128 block in shared memory (XOR-swizzled 16-byte
+//    chunks), and writes it back as whole 256-byte row segments (two samples
+//    per store instruction). (A second form stores each lane's 64 contiguous
+//    bytes straight from registers; measured slower, it stays for
+//    measurements.)
 // Persistent: one CTA per SM walks the (weight-tile, sample-tile) space.
 #pragma once
 
@@ -25,9 +29,11 @@
 
 namespace dc {
 
-constexpr int kPmThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kPmThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kPmEpiWarps = 8;    // two per TMEM lane quarter, one 128-column half each
 constexpr int kPmN = 256;         // weights per tile
-constexpr int kPmStageBytes = 32 * kPmN * 2;  // one warp's 32 samples x 256 bf16
+constexpr int kPmHalf = kPmN / 2; // columns of one epilogue warp
+constexpr int kPmStageBytes = 32 * kPmHalf * 2;  // one warp's 32 samples x 128 bf16
 
 __host__ __device__ inline int pm_nk(int n) { return (n + 15) / 16 * 16; }
 __host__ __device__ inline int pm_kcols(int n) { return (pm_nk(n) + 63) / 64; }
@@ -41,7 +47,7 @@ inline bool premix_shape_ok(int B, int n, int Cout, int taps, int Cin) {
   const long long stage = 1LL * pm_nk(n) * 512;
   const long long alpha_bytes = 4LL * B * n;  // alpha staged in shared memory
   return a_bytes <= 65536 && alpha_bytes <= 16384 &&
-         a_bytes + 2 * stage + 4 * kPmStageBytes + alpha_bytes <= 200 * 1024;
+         a_bytes + 2 * stage + kPmEpiWarps * kPmStageBytes + alpha_bytes <= 200 * 1024;
 }
 
 struct PmParams {
@@ -78,8 +84,8 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   const int kcols = (p.nk + 63) / 64;
   const uint32_t a_base = base;                         // [m_tile][hi/lo][kcol][128 rows x 128 B]
   const uint32_t e_base = a_base + p.a_bytes;           // [stage][4 atoms][nk rows x 128 B]
-  const uint32_t st_base = e_base + S * p.stage_bytes;  // epilogue staging: 4 warps x 16 KB
-  const uint32_t bar_base = st_base + (p.direct_store ? 0u : 4u * kPmStageBytes);
+  const uint32_t st_base = e_base + S * p.stage_bytes;  // epilogue staging: 8 warps x 8 KB
+  const uint32_t bar_base = st_base + (p.direct_store ? 0u : kPmEpiWarps * kPmStageBytes);
   auto full = [&](int s) { return bar_base + 8u * s; };
   auto empty = [&](int s) { return bar_base + 8u * (S + s); };
   auto tfull = [&](int a) { return bar_base + 8u * (2 * S + a); };
@@ -106,7 +112,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull(a), 1);
-      mbar_init(tempty(a), 4);
+      mbar_init(tempty(a), kPmEpiWarps);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -220,63 +226,12 @@ __global__ void __launch_bounds__(kPmThreads, 1)
         wait_drain(drain_bar, 0, p.wait_ns, p.err);
       }
     }
-  } else if (p.direct_store) {
-    // Epilogue, direct form (every sample's kernel a multiple of 16 weights,
-    // workspace 32-byte aligned): warp w reads TMEM lanes 32*(w%4) .. +31 (=
-    // 32 samples of the tile) 32 columns at a time, the next load in flight
-    // while the current one is rounded to bf16, and each lane writes its
-    // sample's 64 contiguous bytes as two 32-byte stores: whole sectors, no
-    // shared-memory round trip.
-    const int q = warp & 3;
-    long long ntile = ntile0;
-    int mt = mt0;
-    for (long long j = 0; j < my_tiles; ++j) {
-      const int ab = static_cast<int>(j & 1);
-      if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j >> 1) & 1), ctl, kErrWaitEpilogue)) break;
-      tc_fence_after();
-      const int row0 = mt * 128 + 32 * q;
-      if (row0 < p.B) {
-        const int b = row0 + lane;
-        const long long w0 = ntile * kPmN;
-        __nv_bfloat16* dst = p.out + static_cast<size_t>(b < p.B ? b : 0) * p.wsize + w0;
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * kPmN;
-        uint32_t ra[32], rb[32];
-        auto emit = [&](const uint32_t (&r)[32], int ch) {
-          uint32_t o[16];
-#pragma unroll
-          for (int v = 0; v < 16; ++v)
-            o[v] = pack_bf16x2(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (b < p.B && w0 + ch * 32 + h * 16 < p.wsize) st_global_v8(dst + ch * 32 + h * 16, o + 8 * h);
-          }
-        };
-        tmem_ld_32x32b_x32(taddr, ra);
-#pragma unroll 1
-        for (int ch = 0; ch < kPmN / 32; ch += 2) {
-          tmem_ld_wait(ra);
-          tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, rb);
-          emit(ra, ch);
-          tmem_ld_wait(rb);
-          if (ch + 2 < kPmN / 32) tmem_ld_32x32b_x32(taddr + (ch + 2) * 32, ra);
-          emit(rb, ch + 1);
-        }
-      }
-      // the TMEM buffer is free once every lane's loads completed
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty(ab));
-      ntile += dn;
-      mt += dm;
-      if (mt >= p.m_tiles) { mt -= p.m_tiles; ++ntile; }
-    }
-  } else {
+  } else if (warp < 2 + kPmEpiWarps) {
     // Epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 (= 32 samples of the
-    // tile), rounds to bf16 and stages its 32 x 256 block in shared memory with
-    // the 16-byte chunk index XOR-ed by the row, so that the staging writes and
-    // the read-back are both conflict-free; then each store instruction writes
-    // one sample's 512 contiguous bytes (four full lines).
+    // tile) and the columns of its half, 32 at a time with the next load in
+    // flight.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const uint32_t stg = st_base + (warp - 2) * kPmStageBytes;
     long long ntile = ntile0;
     int mt = mt0;
@@ -285,41 +240,87 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j >> 1) & 1), ctl, kErrWaitEpilogue)) break;
       tc_fence_after();
       // a warp whose 32 samples are all past the batch only releases the buffer
-      const bool live = mt * 128 + 32 * q < p.B;
-#pragma unroll 1
-      for (int ch = 0; ch < (live ? kPmN / 32 : 0); ++ch) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * kPmN + ch * 32, r);
-        tmem_ld_wait();
+      const int row0 = mt * 128 + 32 * q;
+      const bool live = row0 < p.B;
+      const long long w0 = ntile * kPmN + half * kPmHalf;
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * kPmN + half * kPmHalf;
+      if (live) {
+        uint32_t ra[32], rb[32];
+        if (p.direct_store) {
+          // each lane (one sample) writes 64 contiguous bytes per chunk as two
+          // 32-byte stores straight from registers
+          const int b = row0 + lane;
+          __nv_bfloat16* dst = p.out + static_cast<size_t>(b < p.B ? b : 0) * p.wsize + w0;
+          auto emit = [&](const uint32_t (&r)[32], int ch) {
+            uint32_t o[16];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 o;
-          o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-          o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-          o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-          o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-          const int c = ch * 4 + v;  // 16-byte chunk of this sample's 512-byte row
-          st_shared_v4(stg + lane * 512 + ((c ^ lane) << 4), o);
+            for (int v = 0; v < 16; ++v)
+              o[v] = pack_bf16x2(__uint_as_float(r[2 * v]), __uint_as_float(r[2 * v + 1]));
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              if (b < p.B && w0 + ch * 32 + h * 16 < p.wsize)
+                st_global_v8(dst + ch * 32 + h * 16, o + 8 * h);
+          };
+          tmem_ld_32x32b_x32(taddr, ra);
+#pragma unroll 1
+          for (int ch = 0; ch < kPmHalf / 32; ch += 2) {
+            tmem_ld_wait(ra);
+            tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, rb);
+            emit(ra, ch);
+            tmem_ld_wait(rb);
+            if (ch + 2 < kPmHalf / 32) tmem_ld_32x32b_x32(taddr + (ch + 2) * 32, ra);
+            emit(rb, ch + 1);
+          }
+        } else {
+          // staged: row `lane` of the 32 x 256-byte block, 16-byte chunk c at
+          // position c ^ (lane % 16): 32 lanes fill each bank group evenly
+          auto stage_chunk = [&](const uint32_t (&r)[32], int ch) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+              o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+              o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+              o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+              const int c = ch * 4 + v;  // 16-byte chunk of this sample's 256-byte segment
+              st_shared_v4(stg + lane * 256 + ((c ^ (lane & 15)) << 4), o);
+            }
+          };
+          tmem_ld_32x32b_x32(taddr, ra);
+#pragma unroll 1
+          for (int ch = 0; ch < kPmHalf / 32; ch += 2) {
+            tmem_ld_wait(ra);
+            tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, rb);
+            stage_chunk(ra, ch);
+            tmem_ld_wait(rb);
+            if (ch + 2 < kPmHalf / 32) tmem_ld_32x32b_x32(taddr + (ch + 2) * 32, ra);
+            stage_chunk(rb, ch + 1);
+          }
         }
       }
-      // TMEM buffer is free once every lane's loads completed
+      // the TMEM buffer is free once every lane's loads completed
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty(ab));
-      const long long w = ntile * kPmN + lane * 8;
-      const bool wok = w < p.wsize;
-      const int nrows = live ? min(32, p.B - (mt * 128 + 32 * q)) : 0;
+      if (live && !p.direct_store) {
+        // two samples per store instruction: lanes 0..15 row sr, 16..31 row sr+1,
+        // 16 bytes each = one 256-byte segment per row
+        const int part = lane & 15;
+        const long long w = w0 + part * 8;
+        const bool wok = w < p.wsize;
+        const int nrows = min(32, p.B - row0);
 #pragma unroll 4
-      for (int sr = 0; sr < nrows; ++sr) {
-        const int b = mt * 128 + 32 * q + sr;
-        uint4 v;
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                     : "r"(stg + sr * 512 + ((lane ^ sr) << 4)));
-        if (wok)
-          *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.wsize + w) = v;
+        for (int sr = lane >> 4; sr < 32; sr += 2) {
+          uint4 v;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(stg + sr * 256 + ((part ^ (sr & 15)) << 4)));
+          if (wok && sr < nrows)
+            *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row0 + sr) * p.wsize + w) = v;
+        }
+        __syncwarp();
       }
-      __syncwarp();
       ntile += dn;
       mt += dm;
       if (mt >= p.m_tiles) { mt -= p.m_tiles; ++ntile; }
@@ -363,7 +364,7 @@ inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bf
   p.stage_bytes = p.nk * 512;
   p.direct_store =
       (allow_direct && wsize % 16 == 0 && (reinterpret_cast<uintptr_t>(out_ws) & 31u) == 0) ? 1 : 0;
-  const int staging = p.direct_store ? 0 : 4 * kPmStageBytes;
+  const int staging = p.direct_store ? 0 : kPmEpiWarps * kPmStageBytes;
   const int budget = 200 * 1024 - p.a_bytes - staging - 4 * B * n;
   p.stages = std::min(4, budget / p.stage_bytes);
   if (p.stages < 2) return -3;

@@ -286,25 +286,29 @@ unsigned long long dynconv_launch_count(void);
  * calls on further streams run the two-kernel form.
  * key 7: which kernel mixes the per-sample kernels of the two-kernel PREMIX
  * form: 0 (default) the CUDA-core mixer when n <= 8, else the tensor-core
- * mixing GEMM; 1 always the tensor-core GEMM (and never the streamed kernel of
+ * GEMM with M = samples; 1 always that GEMM (and never the streamed kernel of
  * key 6); 2 the CUDA-core mixer only (forward returns
- * DYNCONV_ERR_UNSUPPORTED when n > 8).
+ * DYNCONV_ERR_UNSUPPORTED when n > 8); 3 the transposed GEMM (M = weights,
+ * N = samples) for batches of at most 256. The tensor-core mixers take no
+ * input attention.
  * key 8: which kernel runs DEPTHWISE: 0 (default) the pipelined kernel
  * (persistent CTAs, resident expert slabs, TMA-fed ring of input tiles) when
- * the shape fits it, else the per-tile kernel; 1 always the per-tile kernel.
+ * the shape fits it, else the per-tile kernel; 1 always the per-tile kernel;
+ * 2 / 3 the pipelined kernel with 2 / 4 output columns per thread.
  * key 9: the convolution of PREMIX: 1 (default) the persistent kernel (one
  * CTA per SM, two TMEM accumulators, the epilogue of one unit overlapping the
  * next unit's MMAs) where it pays (three or more units per CTA, or at most
  * four K steps per unit), no pooled sums are asked for and the shape fits it;
  * 2 the persistent kernel whenever it fits; 0 always one CTA per unit.
  * key 10: PREMIX with n > 8 when every sample's mixed kernel together is much
- * larger than the L2: 1 mixes and convolves one group (of samples, or of
- * 128-channel tiles) at a time through two workspace slots, the mixing of
- * the next group on an internal stream overlapping the convolution of the
- * current one; 0 (default; measured faster on B200 so far) mixes every
- * sample's kernel first, then convolves; a value
- * of 4096 or more turns the grouped form on for every size, with groups of
- * about that many bytes (for tests of ragged groups).
+ * larger than the L2: 0 (default) mixes every sample's kernel first, then
+ * convolves; 1 mixes and convolves one group (of samples, or of 128-channel
+ * tiles) at a time through two workspace slots, the mixing of the next group
+ * on an internal stream overlapping the convolution of the current one; 2
+ * does the same in sequence on the caller's stream through one slot (each
+ * group's mixed kernels read back from L2). A value of 4096 or more turns
+ * form 1 on for every size, and a value of -4096 or less form 2, with groups
+ * of about |value| bytes (for tests of ragged groups and for tuning).
  * key 11: the backward's mixing gradient: 1 (default) the tensor-core kernel
  * (per-sample weight gradients as bf16 hi / lo planes, one pass for the
  * expert and attention gradients) when it applies; 0 the CUDA-core kernel.

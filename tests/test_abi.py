@@ -137,11 +137,14 @@ def test_test_hook_arguments(lib):
     assert dc.dynconv_test_hook(99, 0) == dc.ERR_INVALID_ARG
     # depthwise kernel choice, persistent convolution, grouped mixing
     for key in (8, 9, 11):
-        assert dc.dynconv_test_hook(key, 3) == dc.ERR_INVALID_ARG
+        assert dc.dynconv_test_hook(key, 4 if key == 8 else 3) == dc.ERR_INVALID_ARG
         assert dc.dynconv_test_hook(key, 0 if key == 8 else 1) == dc.OK
     assert dc.dynconv_test_hook(10, 100) == dc.ERR_INVALID_ARG   # group bytes below 4096
     assert dc.dynconv_test_hook(10, -1) == dc.ERR_INVALID_ARG
     assert dc.dynconv_test_hook(10, 1 << 20) == dc.OK
+    assert dc.dynconv_test_hook(10, -(1 << 20)) == dc.OK     # sequential groups of 1 MB
+    assert dc.dynconv_test_hook(10, 3) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(10, 2) == dc.OK
     assert dc.dynconv_test_hook(10, 0) == dc.OK
     assert dc.dynconv_test_hook(12, 2) == dc.ERR_INVALID_ARG
     assert dc.dynconv_test_hook(12, 1) == dc.OK

@@ -284,6 +284,18 @@ def test_premix_mixers_full_size(name, mixer):
         dc.dynconv_test_hook(7, 0)
 
 
+@pytest.mark.parametrize("name", ["resnet18_3x3", "deep_3x3_tau30", "large_n64"])
+def test_premix_transposed_mixer_full_size(name):
+    """PREMIX with the transposed mixing GEMM over the whole batch (test hook
+    7 = 3: M = weights, N = samples) against the oracle on sampled whole
+    samples."""
+    try:
+        assert dc.dynconv_test_hook(7, 3) == dc.OK
+        _forward_case(name, dc.VARIANT_PREMIX, workspace=True)
+    finally:
+        dc.dynconv_test_hook(7, 0)
+
+
 def test_premix_cuda_core_mixer_refuses_many_experts():
     inp = layer_inputs("deep_3x3_tau30")
     L = Layer(inp)
@@ -312,11 +324,14 @@ DEPTHWISE_SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("kernel", [0, 1], ids=["pipelined", "per-tile"])
+@pytest.mark.parametrize("kernel", [0, 1, 2, 3],
+                         ids=["pipelined", "per-tile", "pipelined-2col", "pipelined-4col"])
 @pytest.mark.parametrize("case", DEPTHWISE_SHAPES, ids=[c[0] for c in DEPTHWISE_SHAPES])
 def test_depthwise_kernels_ragged(case, kernel):
-    """Both depthwise kernels (test hook 8) against the oracle on structured
-    inputs, element by element, with and without bias."""
+    """Every depthwise kernel form (test hook 8: the pipelined kernel with its
+    default, 2 or 4 output columns per thread, and the per-tile kernel)
+    against the oracle on structured inputs, element by element, with and
+    without bias."""
     name, B, C, H, W, K, pad, n = case
     cfg = synth.LayerConfig(name, synth.BF16, B, C, C, H, W, K, K, 1, pad, C, n, synth.SIGMOID, 1.0)
     inp = synth.make_inputs(cfg, seed=6, structured=1.0)
@@ -337,11 +352,12 @@ def test_depthwise_kernels_ragged(case, kernel):
         dc.dynconv_test_hook(8, 0)
 
 
-def test_depthwise_full_size_per_tile_kernel():
-    """The per-tile depthwise kernel at full size (the pipelined one is the
-    default and runs in test_forward_depthwise_full_size)."""
+@pytest.mark.parametrize("kernel", [1, 2, 3], ids=["per-tile", "pipelined-2col", "pipelined-4col"])
+def test_depthwise_full_size_kernel_forms(kernel):
+    """Each depthwise kernel form at full size (the default form runs in
+    test_forward_depthwise_full_size)."""
     try:
-        assert dc.dynconv_test_hook(8, 1) == dc.OK
+        assert dc.dynconv_test_hook(8, kernel) == dc.OK
         _forward_case("effnet_dw_5x5", dc.VARIANT_DEPTHWISE)
     finally:
         dc.dynconv_test_hook(8, 0)
@@ -372,11 +388,15 @@ GROUPED = [
 
 
 @pytest.mark.parametrize("case", GROUPED, ids=[c[0] for c in GROUPED])
-def test_grouped_premix_ragged(case):
+@pytest.mark.parametrize("seq", [False, True], ids=["concurrent", "sequential"])
+def test_grouped_premix_ragged(case, seq):
     """The grouped mixing pipeline (runs of samples, or runs of 128-channel
-    tiles, through two workspace slots and an internal stream) against the
-    oracle element by element, next to the one-pass form; each deterministic."""
+    tiles; concurrent: two workspace slots and an internal stream; sequential:
+    one slot on the caller's stream) against the oracle element by element,
+    next to the one-pass form; each deterministic."""
     name, B, Cin, Cout, H, W, K, pad, n, mode, tau, gbytes = case
+    if seq:
+        gbytes = -gbytes
     cfg = synth.LayerConfig(name, synth.BF16, B, Cin, Cout, H, W, K, K, 1, pad, 1, n, mode, tau)
     inp = synth.make_inputs(cfg, seed=8, structured=1.5)
     a32 = alpha_f32_rounded(oracle.route(inp.x_f64, inp.Wr, inp.br, mode, tau))
@@ -440,8 +460,9 @@ def test_small_structured_persistent_conv(case):
         dc.dynconv_test_hook(9, 1)
 
 
+@pytest.mark.parametrize("mode", [1, 2], ids=["concurrent", "sequential"])
 @pytest.mark.parametrize("name", ["deep_3x3_tau30", "large_n64"])
-def test_grouped_and_one_pass_full_size(name):
+def test_grouped_and_one_pass_full_size(name, mode):
     """At full size the grouped pipeline (test hook 10; off by default) is
     deterministic, matches the oracle on sampled whole samples and agrees
     with the one-pass PREMIX within the bf16 tolerance everywhere."""
@@ -454,7 +475,7 @@ def test_grouped_and_one_pass_full_size(name):
     ws = torch.empty(dc.dynconv_workspace_size(d), dtype=torch.uint8, device="cuda")
     outs = []
     try:
-        for hook in (1, 1, 0):
+        for hook in (mode, mode, 0):
             assert dc.dynconv_test_hook(10, hook) == dc.OK
             L.y.fill_(float("nan"))
             dc.check(dc.dynconv_forward(d, L.x, L.experts, L.alpha, L.bias, L.y, ws, ws.numel()))
