@@ -23,11 +23,14 @@
 // The weight operand A (128 x 64 bf16 per step, K-major, 128-byte swizzle)
 // depends on the variant:
 //   FUSED    A = sum_i alpha_{b,i} E_i[co-tile][tap][c-chunk], mixed by 8 warps
-//            on CUDA cores from 16-byte expert loads and rounded once to bf16:
+//            on CUDA cores from expert tiles that one thread TMA-loads into a
+//            ring in shared memory (the same swizzled layout as A, so the mix
+//            is elementwise) and rounded once to bf16:
 //            the kernel is a weighted sum of n static kernels with weights
 //            that depend on the input (KernelWarehouse, abstract), one
 //            kernel per example (CondConv, abstract);
-//   OUTSIDE  the step also runs over the experts and A = alpha_{b,i} E_i: the
+//   OUTSIDE  the step also runs over the experts and A = alpha_{b,i} E_i (one
+//            TMA-loaded expert tile per step, scaled and rounded): the
 //            sum over experts happens in the accumulator,
 //            y = sum_i alpha_i (x conv W_i) -- the same result by linearity;
 //   PREMIX   A = W_b tile, TMA-loaded from a workspace where the premix kernel
@@ -85,7 +88,19 @@ struct TcParams {
   int co_base;            // persistent kernel: channel offset of this launch in y and the biases
   int ld_c;               // persistent kernel: channel stride of y and bias rows (0: Cout)
   int x_early;            // persistent kernel: first x boxes may load before the grid wait
+  int se;                 // FUSED / OUTSIDE: expert-tile stages (16 KB each)
+  unsigned long long* stamps;  // optional [grid][8] phase stamps for measurements, or null
 };
+
+// Phase stamps of one CTA (measurement hook): slot i of this CTA's 8 holds the
+// SM cycle counter (slots 0..5), the SM id (6) and the global timer at entry
+// (7, nanoseconds, to align CTAs of different SMs).
+__device__ __forceinline__ void tc_stamp(const TcParams& p, int i) {
+  if (p.stamps != nullptr) {
+    p.stamps[static_cast<size_t>(blockIdx.x) * 8 + i] = clock64();
+    if (i == 0) p.stamps[static_cast<size_t>(blockIdx.x) * 8 + 7] = globaltimer_ns();
+  }
+}
 
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, int base_mode) {
   uint64_t d = smem_desc_sw128(saddr);
@@ -115,8 +130,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* base_ptr = tc_smem_raw + (base - raw);
   const int SA = p.sa, SB = p.sb;
+  const int SE = VARIANT == kPremix ? 0 : p.se;  // expert-tile stages (FUSED, OUTSIDE)
   const uint32_t a_base = base;
-  const uint32_t b_base = a_base + SA * kTcATileBytes;
+  const uint32_t e_base = a_base + SA * kTcATileBytes;
+  const uint32_t b_base = e_base + SE * kTcATileBytes;
   const uint32_t bar_base = b_base + SB * p.b_tile_bytes;
   auto fullA = [&](int s) { return bar_base + 8u * s; };
   auto emptyA = [&](int s) { return bar_base + 8u * (SA + s); };
@@ -124,7 +141,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto emptyB = [&](int s) { return bar_base + 8u * (2 * SA + SB + s); };
   const uint32_t accum_bar = bar_base + 8u * (2 * SA + 2 * SB);
   const uint32_t drain_bar = accum_bar + 8u;
-  unsigned char* misc = base_ptr + (bar_base - base) + 8u * (2 * SA + 2 * SB + 2);
+  auto fullE = [&](int s) { return bar_base + 8u * (2 * SA + 2 * SB + 2 + s); };
+  auto emptyE = [&](int s) { return bar_base + 8u * (2 * SA + 2 * SB + 2 + SE + s); };
+  unsigned char* misc = base_ptr + (bar_base - base) + 8u * (2 * SA + 2 * SB + 2 + 2 * SE);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   float* alpha_s = reinterpret_cast<float*>(misc + 16);
@@ -138,6 +157,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_relinquish();
   }
   if (threadIdx.x == 32) {
+    tc_stamp(p, 0);  // entry
     for (int s = 0; s < SA; ++s) {
       mbar_init(fullA(s), VARIANT == kPremix ? 1 : kTcMixThreads / 32);
       mbar_init(emptyA(s), 1);
@@ -148,14 +168,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     mbar_init(accum_bar, 1);
     mbar_init(drain_bar, 1);
+    for (int s = 0; s < SE; ++s) {
+      mbar_init(fullE(s), 1);
+      mbar_init(emptyE(s), kTcMixThreads / 32);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&xmap);
-    if (VARIANT == kPremix) tma_prefetch_desc(&wmap);
+    tma_prefetch_desc(&wmap);
   }
   __syncwarp();
   grid_dependency_wait();
   if (threadIdx.x == 32) {
+    tc_stamp(p, 1);  // past the grid wait
     // The first loads need nothing but the barriers: issue them now so their
     // latency overlaps the rest of the set-up.
     const int pre_b = p.kc < SB ? p.kc : SB;
@@ -200,7 +225,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         wait_drain(fullB(j % SB), static_cast<uint32_t>(j / SB) & 1u, p.wait_ns, p.err);
     }
   } else if (warp == 2) {
-    // ======================= weight producer (PREMIX only) =======================
+    // ============ expert-tile producer (FUSED, OUTSIDE): TMA, consumption order ============
+    if (VARIANT != kPremix && lane == 0) {
+      const int ne = VARIANT == kFused ? p.n : 1;
+      int issued = 0;
+      bool ok = true;
+      for (int k = 0; k < p.k_steps && ok; ++k) {
+        const int cc = k / p.spc, t = k % p.spc;
+        const int tap = VARIANT == kFused ? t : t % taps;
+        for (int j = 0; j < ne; ++j, ++issued) {
+          const int i = VARIANT == kFused ? j : t / taps;  // expert
+          const int s = issued % SE;
+          const uint32_t ph = static_cast<uint32_t>(issued / SE) & 1u;
+          if (!wait_bounded(emptyE(s), ph ^ 1u, ctl, kErrWaitProducer)) { ok = false; break; }
+          mbar_arrive_expect_tx(fullE(s), kTcATileBytes);
+          tma_load_3d(e_base + s * kTcATileBytes, &wmap, fullE(s), cc * 64, tap, i * p.Cout + m0);
+        }
+      }
+      for (int j = (issued > SE ? issued - SE : 0); j < issued; ++j)
+        wait_drain(fullE(j % SE), static_cast<uint32_t>(j / SE) & 1u, p.wait_ns, p.err);
+    }
+    // ======================= weight producer (PREMIX) =======================
     if (VARIANT == kPremix && lane == 0) {
       const int pre_a = p.k_steps < SA ? p.k_steps : SA;  // issued during set-up
       int issued = pre_a;
@@ -241,6 +286,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = p.k_steps > 0 && wait_bounded(fullB(0), 0, ctl, kErrWaitMma) &&
                 wait_bounded(fullA(0), 0, ctl, kErrWaitMma);
       if (ok) tc_fence_after();
+      tc_stamp(p, 2);  // first operands in shared memory
       for (int k = 0; k < p.k_steps && ok; ++k) {
         const uint64_t ad = a_desc0 + s * (kTcATileBytes >> 4);
         const uint64_t bd = b_desc0 + sbi * b_stage + tap_off;
@@ -269,8 +315,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (++s == static_cast<uint32_t>(SA)) { s = 0; ph ^= 1u; }
         // operands of the next step
+        // (with a single activation stage the next chunk's box can only land
+        // after this chunk's MMAs release the stage: wait for it after the commit)
+        const bool b_now = chunk_end && SB > 1;
         if (k + 1 < p.k_steps) {
-          if (chunk_end && !wait_bounded(fullB(sbi), phb, ctl, kErrWaitMma)) ok = false;
+          if (b_now && !wait_bounded(fullB(sbi), phb, ctl, kErrWaitMma)) ok = false;
           if (ok && !wait_bounded(fullA(s), ph, ctl, kErrWaitMma)) ok = false;
           if (ok) tc_fence_after();
         }
@@ -278,7 +327,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (two) tc_mma_f16(tmem_base + p.n_mma0, ad + 6, bd + b_n1 + 6, idesc1, 1u);
         tc_commit(emptyA(s_cur));
         if (chunk_end) tc_commit(emptyB(sbi_cur));
+        if (ok && chunk_end && SB == 1 && k + 1 < p.k_steps) {
+          if (!wait_bounded(fullB(sbi), phb, ctl, kErrWaitMma)) ok = false;
+          else tc_fence_after();
+        }
       }
+      tc_stamp(p, 3);  // last MMA issued
       if (ok) {
         tc_commit(accum_bar);
       } else {
@@ -289,81 +343,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp >= kTcMixWarp0) {
     const int mt_id = threadIdx.x - kTcMixWarp0 * 32;  // 0..255
     // ======================= mixers (FUSED / OUTSIDE) =======================
+    // The expert tiles arrive by TMA in the same 128-byte-swizzled K-major
+    // layout as the A tile, so the mix is elementwise over shared memory:
+    // thread t takes the 16-byte chunks t, t + 256, t + 512, t + 768 of every
+    // tile (conflict-free), accumulates alpha_i * E_i in fp32 in expert order
+    // (FUSED: the step's n experts; OUTSIDE: the step's one expert) and
+    // rounds once to bf16 into the A stage.
     if (VARIANT != kPremix) {
-      const size_t wsize = static_cast<size_t>(p.Cout) * taps * p.Cin;  // one expert
-      // this thread's four 16-byte chunks: rows r0 + 32u (u = 0..3), chunk j
-      const int j = mt_id & 7;
-      const int r0 = mt_id >> 3;
-      for (int k = 0; k < p.k_steps; ++k) {
+      const int ne = VARIANT == kFused ? p.n : 1;
+      int consumed = 0;
+      bool ok = true;
+      for (int k = 0; k < p.k_steps && ok; ++k) {
         const int s = k % SA;
         const uint32_t ph = static_cast<uint32_t>(k / SA) & 1u;
         if (!wait_bounded(emptyA(s), ph ^ 1u, ctl, kErrWaitMixer)) break;
-        const int cc = k / p.spc, t = k % p.spc;
-        const int tap = (VARIANT == kOutside) ? t % taps : t;
-        const uint32_t a_s = a_base + s * kTcATileBytes;
-        const int ci = cc * 64 + j * 8;
-        float acc[4][8];
+        const int t = k % p.spc;
+        uint64_t acc[4][4];
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[uu][e] = 0.f;
-        const __nv_bfloat16* src[4];
-        bool live[4];
+          for (int e = 0; e < 4; ++e) acc[uu][e] = 0ull;
+        for (int j = 0; j < ne; ++j, ++consumed) {
+          const int es = consumed % SE;
+          const uint32_t eph = static_cast<uint32_t>(consumed / SE) & 1u;
+          if (!wait_bounded(fullE(es), eph, ctl, kErrWaitMixer)) { ok = false; break; }
+          const float a = alpha_s[VARIANT == kFused ? j : t / taps];
+          const uint64_t a2 = pack_f32x2(a, a);
+          const uint32_t src = e_base + es * kTcATileBytes + mt_id * 16;
+          uint4 v[4];
 #pragma unroll
-        for (int uu = 0; uu < 4; ++uu) {
-          const int co = m0 + r0 + 32 * uu;
-          live[uu] = co < p.Cout && ci < p.Cin;
-          src[uu] = p.experts + (static_cast<size_t>(live[uu] ? co : 0) * taps + tap) * p.Cin +
-                    (live[uu] ? ci : 0);
-        }
-        if (VARIANT == kFused) {
-          // two experts x four chunks = eight 16-byte loads in flight per thread
-          for (int i = 0; i < p.n; i += 2) {
-            const bool two = i + 1 < p.n;
-            uint4 v0[4], v1[4];
-#pragma unroll
-            for (int uu = 0; uu < 4; ++uu) {
-              v0[uu] = live[uu] ? ld_nc_v4(src[uu] + i * wsize) : make_uint4(0u, 0u, 0u, 0u);
-              v1[uu] = (live[uu] && two) ? ld_nc_v4(src[uu] + (i + 1) * wsize)
-                                         : make_uint4(0u, 0u, 0u, 0u);
-            }
-            const float a0 = alpha_s[i];
-            const float a1 = two ? alpha_s[i + 1] : 0.f;
-#pragma unroll
-            for (int uu = 0; uu < 4; ++uu) {
-              const uint32_t w0[4] = {v0[uu].x, v0[uu].y, v0[uu].z, v0[uu].w};
-              const uint32_t w1[4] = {v1[uu].x, v1[uu].y, v1[uu].z, v1[uu].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                acc[uu][2 * e] = fmaf(a0, bf16lo_to_f32(w0[e]), acc[uu][2 * e]);
-                acc[uu][2 * e + 1] = fmaf(a0, bf16hi_to_f32(w0[e]), acc[uu][2 * e + 1]);
-                acc[uu][2 * e] = fmaf(a1, bf16lo_to_f32(w1[e]), acc[uu][2 * e]);
-                acc[uu][2 * e + 1] = fmaf(a1, bf16hi_to_f32(w1[e]), acc[uu][2 * e + 1]);
-              }
-            }
-          }
-        } else {  // OUTSIDE: A = alpha_i * W_i for this step's expert i
-          const int i = t / taps;
-          const float a = alpha_s[i];
+          for (int uu = 0; uu < 4; ++uu) v[uu] = ld_shared_v4(src + uu * 4096);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(emptyE(es));  // this warp is done reading the slot
 #pragma unroll
           for (int uu = 0; uu < 4; ++uu) {
-            const uint4 v = live[uu] ? ld_nc_v4(src[uu] + i * wsize) : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              acc[uu][2 * e] = a * bf16lo_to_f32(w[e]);
-              acc[uu][2 * e + 1] = a * bf16hi_to_f32(w[e]);
-            }
+            acc[uu][0] = ffma2(a2, bf16x2_to_f32x2(v[uu].x), acc[uu][0]);
+            acc[uu][1] = ffma2(a2, bf16x2_to_f32x2(v[uu].y), acc[uu][1]);
+            acc[uu][2] = ffma2(a2, bf16x2_to_f32x2(v[uu].z), acc[uu][2]);
+            acc[uu][3] = ffma2(a2, bf16x2_to_f32x2(v[uu].w), acc[uu][3]);
           }
         }
+        if (!ok) break;
+        const uint32_t dst = a_base + s * kTcATileBytes + mt_id * 16;
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu) {
-          const int r = r0 + 32 * uu;
-          const uint4 packed =
-              make_uint4(pack_bf16x2(acc[uu][0], acc[uu][1]), pack_bf16x2(acc[uu][2], acc[uu][3]),
-                         pack_bf16x2(acc[uu][4], acc[uu][5]), pack_bf16x2(acc[uu][6], acc[uu][7]));
-          // K-major, 128-byte swizzle: 16-byte chunk j of row r lands at chunk j ^ (r % 8)
-          st_shared_v4(a_s + r * 128 + ((j ^ (r & 7)) << 4), packed);
+          uint4 o;
+          o.x = pack_bf16x2(__uint_as_float(static_cast<uint32_t>(acc[uu][0])),
+                            __uint_as_float(static_cast<uint32_t>(acc[uu][0] >> 32)));
+          o.y = pack_bf16x2(__uint_as_float(static_cast<uint32_t>(acc[uu][1])),
+                            __uint_as_float(static_cast<uint32_t>(acc[uu][1] >> 32)));
+          o.z = pack_bf16x2(__uint_as_float(static_cast<uint32_t>(acc[uu][2])),
+                            __uint_as_float(static_cast<uint32_t>(acc[uu][2] >> 32)));
+          o.w = pack_bf16x2(__uint_as_float(static_cast<uint32_t>(acc[uu][3])),
+                            __uint_as_float(static_cast<uint32_t>(acc[uu][3] >> 32)));
+          st_shared_v4(dst + uu * 4096, o);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -393,6 +426,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const float so = (p.a_out != nullptr && co < p.Cout) ? p.a_out[static_cast<size_t>(b) * p.Cout + co] : 1.f;
     if (wait_bounded(accum_bar, 0, ctl, kErrWaitEpilogue)) {
       tc_fence_after();
+      if (threadIdx.x == 96) tc_stamp(p, 4);  // accumulator complete
       // Per warp: chunks of 32 pixels x 32 output channels. The next chunk's
       // TMEM load is in flight while this one is rounded, transposed through a
       // 2 KB staging tile in the (now idle) A stage buffers, and written as
@@ -487,6 +521,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // ---- teardown
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) {
+    tc_stamp(p, 5);  // epilogue done
+    if (p.stamps != nullptr) {
+      uint32_t smid;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+      p.stamps[static_cast<size_t>(blockIdx.x) * 8 + 6] = smid;
+    }
+  }
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);
@@ -570,6 +612,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_relinquish();
   }
   if (threadIdx.x == 32) {
+    tc_stamp(p, 0);  // entry
     for (int s = 0; s < SA; ++s) {
       mbar_init(fullA(s), 1);
       mbar_init(emptyA(s), 1);
@@ -608,6 +651,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
   grid_dependency_wait();
+  if (threadIdx.x == 32) tc_stamp(p, 1);  // past the grid wait
   const int taps = p.KH * p.KW;
   const uint32_t acc_cols = p.tmem_cols >> 1;
 
@@ -679,6 +723,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         tc_fence_after();
+        if (i == 0) tc_stamp(p, 2);  // first operands of the first unit
         for (int k = 0; k < p.k_steps && ok; ++k) {
           const uint64_t ad = a_desc0 + s * (kTcATileBytes >> 4);
           const uint64_t bd = b_desc0 + sbi * b_stage + tap_off;
@@ -710,6 +755,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (chunk_end) tc_commit(emptyB(sbi_cur));
         }
         if (ok) tc_commit(tfull(ab));
+        if (i == 0) tc_stamp(p, 3);       // first unit's MMAs issued
+        if (i == my_units - 1) tc_stamp(p, 4);  // last unit's MMAs issued
       }
       if (!ok) {
         tc_commit(drain_bar);
@@ -799,6 +846,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) {
+    tc_stamp(p, 5);  // every unit's epilogue done
+    if (p.stamps != nullptr) {
+      uint32_t smid;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+      p.stamps[static_cast<size_t>(blockIdx.x) * 8 + 6] = smid;
+    }
+  }
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);

@@ -75,6 +75,7 @@ std::atomic<int> g_group_mix{0};     // PREMIX, n > 8, large B*|W|: 0 one pass, 
 std::atomic<int> g_premix_direct{0}; // premix epilogue: 1 stores from registers when aligned, 0 staged
 std::atomic<int> g_mixgrad_tc{1};    // backward: 1 tensor-core mixing gradient when it fits, 0 CUDA cores
 std::atomic<long long> g_group_bytes{40LL << 20};  // target bytes of one group's mixed kernels
+std::atomic<unsigned long long> g_conv_stamps{0};  // device buffer for the convolution's phase stamps
 std::atomic<long long> g_group_min{64LL << 20};    // below this B*|W| the one-pass form is used
 thread_local char g_last_err[256] = "";
 
@@ -243,17 +244,35 @@ bool tc_plan(const dynconv_desc* d, int variant, int sms, int max_smem, TcPlan* 
     const int rows = std::max(box_rows * Wp, s_tap_max + n_pad);
     const int b_tile = (rows * 128 + 1023) / 1024 * 1024;
     const size_t fixed = 1024 /*align slack*/ + 8 * 64 /*barriers*/ + 16 + 4 * d->n + 64;
-    const int sb = kc > 1 ? 2 : 1;
-    if (fixed + sb * static_cast<size_t>(b_tile) + 2 * dc::kTcATileBytes > static_cast<size_t>(max_smem))
-      continue;
-    int sa = static_cast<int>((max_smem - fixed - sb * static_cast<size_t>(b_tile)) / dc::kTcATileBytes);
-    sa = std::min(sa, 8);
+    const size_t T = dc::kTcATileBytes;
+    int sb = kc > 1 ? 2 : 1;
+    int sa = 0, se = 0;
+    if (variant == DYNCONV_VARIANT_PREMIX) {
+      if (fixed + sb * static_cast<size_t>(b_tile) + 2 * T > static_cast<size_t>(max_smem)) continue;
+      sa = static_cast<int>((max_smem - fixed - sb * static_cast<size_t>(b_tile)) / T);
+      sa = std::min(sa, 8);
+    } else {
+      // two A stages and a ring of expert tiles (ideally two K steps' worth,
+      // at least two tiles); one activation stage when two leave too few
+      const int ne = variant == DYNCONV_VARIANT_FUSED ? d->n : 1;
+      const int want = std::min(16, std::max(4, 2 * ne));
+      for (int tsb = sb; tsb >= 1 && se < want; --tsb) {
+        const long long room = static_cast<long long>(max_smem) - static_cast<long long>(fixed) -
+                               tsb * static_cast<long long>(b_tile) - 2 * static_cast<long long>(T);
+        const int fit = room > 0 ? static_cast<int>(std::min<long long>(room / T, want)) : 0;
+        if (fit > se) { se = fit; sb = tsb; }
+      }
+      if (se < 2) continue;
+      sa = 2;
+    }
     const int tiles_h = (d->H + R - 1) / R;
     const long long units = 1LL * d->B * tiles_h * m_tiles;
     const long long waves = (units + sms - 1) / sms;
     const double mma = 2.0 * n_pad;
+    // operand bytes per K step: PREMIX one mixed-kernel tile (~20 B/clk from
+    // HBM or L2), FUSED n expert tiles and OUTSIDE one (L2-resident, TMA)
     const double a_bytes = variant == DYNCONV_VARIANT_FUSED ? 16384.0 * d->n : 16384.0;
-    const double a_cost = a_bytes / 20.0;
+    const double a_cost = a_bytes / (variant == DYNCONV_VARIANT_PREMIX ? 20.0 : 40.0);
     const double b_cost = static_cast<double>(box_rows) * Wp * 128.0 / 20.0;
     const double t_unit = k_steps * std::max(mma, a_cost) + kc * b_cost / 4.0 + 40.0 * n_pad + 3000.0;
     const double cost = waves * t_unit;
@@ -261,14 +280,14 @@ bool tc_plan(const dynconv_desc* d, int variant, int sms, int max_smem, TcPlan* 
       found = true;
       best.cost = cost;
       best.grid = static_cast<int>(units);
-      best.smem = fixed + sb * static_cast<size_t>(b_tile) + sa * static_cast<size_t>(dc::kTcATileBytes);
+      best.smem = fixed + sb * static_cast<size_t>(b_tile) + (sa + se) * T;
       dc::TcParams& p = best.p;
       std::memset(&p, 0, sizeof(p));
       p.B = d->B; p.H = d->H; p.W = d->W; p.Cin = d->C_in; p.Cout = d->C_out;
       p.KH = d->KH; p.KW = d->KW; p.pad = d->pad; p.n = d->n;
       p.R = R; p.tiles_h = tiles_h; p.m_tiles = m_tiles; p.Wp = Wp; p.n_virt = n_virt;
       p.n_mma0 = n0; p.n_mma1 = n1; p.kc = kc; p.spc = spc; p.k_steps = k_steps;
-      p.sa = sa; p.sb = sb; p.b_tile_bytes = b_tile; p.b_box_rows = box_rows;
+      p.sa = sa; p.sb = sb; p.se = se; p.b_tile_bytes = b_tile; p.b_box_rows = box_rows;
       p.desc_base_mode = g_desc_base_mode;
       uint32_t cols = 32;
       while (cols < static_cast<uint32_t>(n_pad)) cols <<= 1;
@@ -594,7 +613,7 @@ int launch_premix_conv(const dynconv_desc* d, const TcPlan& plan, const DeviceSt
     const dc::TcParams& q = plan.p;
     pp.p.experts = q.experts; pp.p.alpha = q.alpha; pp.p.bias = q.bias; pp.p.y = q.y;
     pp.p.err = q.err; pp.p.wait_ns = q.wait_ns; pp.p.a_out = q.a_out;
-    pp.p.chan_add = q.chan_add; pp.p.chan_scale = q.chan_scale;
+    pp.p.chan_add = q.chan_add; pp.p.chan_scale = q.chan_scale; pp.p.stamps = q.stamps;
     // launched right after one of this library's mixing kernels (they signal
     // dependents only past their own wait), with a programmatic edge
     pp.p.x_early = g_use_pdl.load() ? 1 : 0;
@@ -1071,12 +1090,21 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   plan.p.err = st->err;
   plan.p.wait_ns = g_wait_ns.load();
   plan.p.inject_skip = g_inject_skip.exchange(0);
+  plan.p.stamps = reinterpret_cast<unsigned long long*>(g_conv_stamps.load());
   CUtensorMap xmap, wmap;
   std::memset(&wmap, 0, sizeof(wmap));
   int rc = encode_x_map(&xmap, x, d, plan.p.Wp, plan.p.b_box_rows);
   if (rc) return rc;
-  if (variant == DYNCONV_VARIANT_FUSED) return launch_tc<dc::kFused>(plan, xmap, wmap, stream);
-  if (variant == DYNCONV_VARIANT_OUTSIDE) return launch_tc<dc::kOutside>(plan, xmap, wmap, stream);
+  if (variant == DYNCONV_VARIANT_FUSED || variant == DYNCONV_VARIANT_OUTSIDE) {
+    // the experts as n "samples" of the mixed-kernel layout: tiles {64 ci, 1 tap, 128 co}
+    if (!aligned16(experts)) return DYNCONV_ERR_MISALIGNED;
+    dynconv_desc de = *d;
+    de.B = d->n;
+    rc = encode_w_map(&wmap, experts, &de);
+    if (rc) return rc;
+    return variant == DYNCONV_VARIANT_FUSED ? launch_tc<dc::kFused>(plan, xmap, wmap, stream)
+                                            : launch_tc<dc::kOutside>(plan, xmap, wmap, stream);
+  }
   // PREMIX: mix every sample's kernel into the workspace, then convolve from it
   const size_t need = premix_workspace(d);
   if (need == 0) return DYNCONV_ERR_UNSUPPORTED;
@@ -1263,6 +1291,11 @@ int dynconv_test_hook(int key, long long value) {
   if (key == 11) {
     if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
     g_mixgrad_tc.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
+  if (key == 13) {
+    // a device buffer of at least grid * 8 64-bit words (0: off)
+    g_conv_stamps.store(static_cast<unsigned long long>(value));
     return DYNCONV_OK;
   }
   if (key == 12) {

@@ -263,6 +263,14 @@ __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) {
 }
 
 // Packed fp32 pair in one 64-bit register: `lo` in bits 0-31.
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
   return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
 }

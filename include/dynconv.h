@@ -317,6 +317,16 @@ unsigned long long dynconv_launch_count(void);
  * thread's 32 mixed weights straight from registers (two 32-byte stores) when
  * the kernel size is a multiple of 16 and the workspace 32-byte aligned
  * (measured slower on B200). For measurements.
+ * key 13: the address of a device buffer of 64-bit words (0, the default:
+ * off). While it is set, each CTA of the PREMIX, FUSED and OUTSIDE
+ * tensor-core convolutions writes 8 words at [block * 8]: its SM cycle
+ * counter at entry, past the grid wait, when the first operands are in
+ * shared memory, after the MMA issue of the (one-CTA-per-unit kernel: only;
+ * persistent kernel: first) unit, when the accumulator is complete
+ * (persistent kernel: after the last unit's MMA issue) and when every
+ * epilogue is done; its SM id; and the global timer at entry. The buffer
+ * must hold 8 words per CTA of every such launch made meanwhile. For
+ * measurements.
  * Returns DYNCONV_OK or DYNCONV_ERR_INVALID_ARG. */
 int dynconv_test_hook(int key, long long value);
 
