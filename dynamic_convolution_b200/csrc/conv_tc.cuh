@@ -36,9 +36,10 @@
 //   PREMIX   A = W_b tile, TMA-loaded from a workspace where the premix kernel
 //            stored every sample's mixed kernel.
 // One thread issues tcgen05.mma (M=128, N<=256 per instruction, K=16) and
-// commits each stage back to its "empty" barrier. The epilogue (8 warps) reads
-// TMEM lane = output channel, adds the mixed bias sum_i alpha_i bias_i, rounds
-// to bf16, transposes through shared memory and writes 16-byte NHWC segments.
+// commits each stage back to its "empty" barrier. The epilogue reads TMEM
+// lane = output channel with 16x256b loads, adds the mixed bias
+// sum_i alpha_i bias_i, rounds to bf16, transposes 8x8 blocks into shared
+// memory with stmatrix and writes 16-byte NHWC segments.
 // Every barrier wait is bounded; on expiry the CTA raises an abort flag,
 // records an error word, drains its in-flight TMA / MMA work, frees TMEM and
 // exits.
@@ -102,6 +103,52 @@ __device__ __forceinline__ void tc_stamp(const TcParams& p, int i) {
   }
 }
 
+// ---- epilogue building blocks (both kernels)
+// A warp owns one TMEM lane quarter (32 output channels) and walks its
+// 32-pixel chunks. A chunk is loaded as two 16x256b.x4 loads (lanes 0..15 and
+// 16..31 of the quarter): thread t then holds, per half h and 8-pixel group
+// j, channels 16h + t/4 (e = 0) and 16h + 8 + t/4 (e = 1) at pixels 8j + 2(t%4)
+// and +1 -- exactly the fragment of an 8x8 (channels x pixels) b16 matrix, so
+// one stmatrix.trans per four matrices writes the chunk pixel-major into the
+// warp's 2 KB staging tile: 64-byte pixel rows, 16-byte chunk c (channels
+// 8c .. 8c+7) of local pixel p at position c ^ ((p >> 1) & 3), conflict-free
+// for the matrix stores and for the 16-byte read-back.
+__device__ __forceinline__ void epi_load_chunk(uint32_t trow, int col, uint32_t (&r)[32]) {
+  tmem_ld_16x256b_x4(trow + static_cast<uint32_t>(col), r);
+  tmem_ld_16x256b_x4(trow + (16u << 16) + static_cast<uint32_t>(col), r + 16);
+}
+
+__device__ __forceinline__ uint32_t epi_slot(uint32_t stage, int pix, int chunk) {
+  return stage + pix * 64 + ((chunk ^ ((pix >> 1) & 3)) << 4);
+}
+
+// y = (accumulator + bias) * scale, rounded once to bf16, staged transposed.
+// bias[h][e] and scale[h][e] belong to channel 16h + 8e + lane/4 of the quarter.
+__device__ __forceinline__ void epi_stage_chunk(const uint32_t (&r)[32], const float (&bias)[2][2],
+                                                const float (&scale)[2][2], uint32_t stage,
+                                                int lane) {
+  const int m = lane >> 3, rr = lane & 7;  // this thread addresses row rr of matrix m
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t P[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t* v = r + 16 * h + 4 * j;
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        P[j][e] = pack_bf16x2((__uint_as_float(v[2 * e]) + bias[h][e]) * scale[h][e],
+                              (__uint_as_float(v[2 * e + 1]) + bias[h][e]) * scale[h][e]);
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      // matrices (e, j) = (0, 2s2), (1, 2s2), (0, 2s2+1), (1, 2s2+1)
+      const int pix = 8 * (2 * s2 + (m >> 1)) + rr;
+      stmatrix_x4_trans(epi_slot(stage, pix, 2 * h + (m & 1)), P[2 * s2][0], P[2 * s2][1],
+                        P[2 * s2 + 1][0], P[2 * s2 + 1][1]);
+    }
+  }
+}
+
 __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, int base_mode) {
   uint64_t d = smem_desc_sw128(saddr);
   if (base_mode) d |= static_cast<uint64_t>((saddr >> 7) & 7u) << 49;
@@ -143,10 +190,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t drain_bar = accum_bar + 8u;
   auto fullE = [&](int s) { return bar_base + 8u * (2 * SA + 2 * SB + 2 + s); };
   auto emptyE = [&](int s) { return bar_base + 8u * (2 * SA + 2 * SB + 2 + SE + s); };
-  unsigned char* misc = base_ptr + (bar_base - base) + 8u * (2 * SA + 2 * SB + 2 + 2 * SE);
+  const uint32_t bias_bar = bar_base + 8u * (2 * SA + 2 * SB + 2 + 2 * SE);
+  unsigned char* misc = base_ptr + (bar_base - base) + 8u * (2 * SA + 2 * SB + 3 + 2 * SE);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   float* alpha_s = reinterpret_cast<float*>(misc + 16);
+  // the tile's 128 mixed biases and output attentions, made by warp 3 while
+  // the MMAs run
+  float* bias_s = reinterpret_cast<float*>(misc + 16 + ((4 * p.n + 15) & ~15));
+  float* scale_s = bias_s + 128;
 
   const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
 
@@ -168,6 +220,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     mbar_init(accum_bar, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(bias_bar, 1);
     for (int s = 0; s < SE; ++s) {
       mbar_init(fullE(s), 1);
       mbar_init(emptyE(s), kTcMixThreads / 32);
@@ -406,25 +459,48 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
 
+  if (warp == 3) {
+    // ---- the tile's mixed biases sum_i alpha_i bias_i[co] (+ the per-channel
+    // term) and output attentions, one channel per lane and pass, while the
+    // MMAs run; published through bias_bar
+    const float* ab = VARIANT == kPremix ? p.alpha + static_cast<size_t>(b) * p.n : alpha_s;
+    for (int c = lane; c < 128; c += 32) {
+      const int co = m0 + c;
+      float acc = 0.f;
+      if (p.bias != nullptr && co < p.Cout)
+        for (int i = 0; i < p.n; ++i)
+          acc = fmaf(ab[i], p.bias[static_cast<size_t>(i) * p.Cout + co], acc);
+      if (p.chan_add != nullptr && co < p.Cout)
+        acc = fmaf(p.chan_add[static_cast<size_t>(b) * p.Cout + co], p.chan_scale, acc);
+      bias_s[c] = acc;
+      // output attention: y = a_out * (conv + mixed bias), channel by channel
+      scale_s[c] = (p.a_out != nullptr && co < p.Cout) ? p.a_out[static_cast<size_t>(b) * p.Cout + co]
+                                                       : 1.f;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bias_bar);
+  }
+
   // ======================= epilogue (all 12 warps) =======================
   // Warps 0..2 join once their lane 0 is done with its producer / MMA role,
-  // warp 3 has no other role. Warp w reads TMEM lane quarter w % 4 (output
-  // channels 32*(w%4) ..) and every third 32-pixel chunk from w / 4.
+  // warp 3 once the biases are made. Warp w reads TMEM lane quarter w % 4
+  // (output channels 32*(w%4) ..) and every third 32-pixel chunk from w / 4.
   __syncwarp();
   {
     const int q = warp & 3;   // TMEM lane quarter
     const int grp = warp >> 2;  // chunk phase 0..2
-    const int co = m0 + 32 * q + lane;
-    float bb = 0.f;
-    if (p.bias != nullptr && co < p.Cout) {
-      const float* ab = VARIANT == kPremix ? p.alpha + static_cast<size_t>(b) * p.n : alpha_s;
-      for (int i = 0; i < p.n; ++i) bb = fmaf(ab[i], p.bias[static_cast<size_t>(i) * p.Cout + co], bb);
-    }
-    if (p.chan_add != nullptr && co < p.Cout)
-      bb = fmaf(p.chan_add[static_cast<size_t>(b) * p.Cout + co], p.chan_scale, bb);
-    // output attention: y = a_out * (conv + mixed bias), channel by channel
-    const float so = (p.a_out != nullptr && co < p.Cout) ? p.a_out[static_cast<size_t>(b) * p.Cout + co] : 1.f;
-    if (wait_bounded(accum_bar, 0, ctl, kErrWaitEpilogue)) {
+    if (wait_bounded(accum_bar, 0, ctl, kErrWaitEpilogue) &&
+        wait_bounded(bias_bar, 0, ctl, kErrWaitEpilogue)) {
+      // the mixed bias (and output attention) of this thread's four channels
+      // 32q + 16h + 8e + lane/4 of the tile
+      float bb[2][2], so[2][2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          bb[h][e] = bias_s[32 * q + 16 * h + 8 * e + (lane >> 2)];
+          so[h][e] = scale_s[32 * q + 16 * h + 8 * e + (lane >> 2)];
+        }
       tc_fence_after();
       if (threadIdx.x == 96) tc_stamp(p, 4);  // accumulator complete
       // Per warp: chunks of 32 pixels x 32 output channels. The next chunk's
@@ -447,17 +523,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) ps[e] = 0.f;
       auto process = [&](const uint32_t (&r)[32], int ch) {
-#pragma unroll
-        for (int jj = 0; jj < 32; jj += 2) {
-          const uint32_t w = pack_bf16x2((__uint_as_float(r[jj]) + bb) * so,
-                                         (__uint_as_float(r[jj + 1]) + bb) * so);
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + jj * 64 + lane * 2),
-                       "h"(static_cast<unsigned short>(w & 0xFFFFu))
-                       : "memory");
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + (jj + 1) * 64 + lane * 2),
-                       "h"(static_cast<unsigned short>(w >> 16))
-                       : "memory");
-        }
+        epi_stage_chunk(r, bb, so, stage, lane);
         __syncwarp();
         int pix = ch * 32 + (lane >> 2);
         int rr = pix / p.Wp;
@@ -466,10 +532,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int it = 0; it < 4; ++it) {
           const int oh = h0 + rr;
           if (c_ok && pix < p.n_virt && cw < p.W && oh < p.H) {
-            uint4 v;
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                         : "r"(stage + (it * 8 + (lane >> 2)) * 64 + part * 16));
+            const uint4 v = ld_shared_v4(epi_slot(stage, it * 8 + (lane >> 2), part));
             *reinterpret_cast<uint4*>(ybase + (static_cast<size_t>(oh) * p.W + cw) * p.Cout) = v;
             if (pool) {
               const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
@@ -488,15 +551,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       };
       uint32_t ra[32], rb[32];
       int ch = grp;
-      if (ch < nchunks) tmem_ld_32x32b_x32(trow + ch * 32, ra);
+      if (ch < nchunks) epi_load_chunk(trow, ch * 32, ra);
       while (ch < nchunks) {
         tmem_ld_wait(ra);
-        if (ch + 3 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 3) * 32, rb);
+        if (ch + 3 < nchunks) epi_load_chunk(trow, (ch + 3) * 32, rb);
         process(ra, ch);
         ch += 3;
         if (ch >= nchunks) break;
         tmem_ld_wait(rb);
-        if (ch + 3 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 3) * 32, ra);
+        if (ch + 3 < nchunks) epi_load_chunk(trow, (ch + 3) * 32, ra);
         process(rb, ch);
         ch += 3;
       }
@@ -776,15 +839,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int ab = i & 1;
       int b, h0, m0, th;
       decode(i, b, h0, m0, th);
-      const int co = m0 + 32 * q + lane;  // channel of this launch; cb + co in y and the biases
-      float bb = 0.f;
-      if (p.bias != nullptr && co < p.Cout) {
-        const float* al = p.alpha + static_cast<size_t>(b) * p.n;
-        for (int e = 0; e < p.n; ++e) bb = fmaf(al[e], p.bias[static_cast<size_t>(e) * ldc + cb + co], bb);
-      }
-      if (p.chan_add != nullptr && co < p.Cout)
-        bb = fmaf(p.chan_add[static_cast<size_t>(b) * ldc + cb + co], p.chan_scale, bb);
-      const float so = (p.a_out != nullptr && co < p.Cout) ? p.a_out[static_cast<size_t>(b) * ldc + cb + co] : 1.f;
+      // the mixed bias (and output attention) of this thread's four channels
+      // 32q + 16h + 8e + lane/4 of the tile (cb + co in y and the biases)
+      float bb[2][2], so[2][2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e2 = 0; e2 < 2; ++e2) {
+          const int co = m0 + 32 * q + 16 * h + 8 * e2 + (lane >> 2);
+          float acc = 0.f;
+          if (p.bias != nullptr && co < p.Cout) {
+            const float* al = p.alpha + static_cast<size_t>(b) * p.n;
+            for (int e = 0; e < p.n; ++e)
+              acc = fmaf(al[e], p.bias[static_cast<size_t>(e) * ldc + cb + co], acc);
+          }
+          if (p.chan_add != nullptr && co < p.Cout)
+            acc = fmaf(p.chan_add[static_cast<size_t>(b) * ldc + cb + co], p.chan_scale, acc);
+          bb[h][e2] = acc;
+          so[h][e2] = (p.a_out != nullptr && co < p.Cout)
+                          ? p.a_out[static_cast<size_t>(b) * ldc + cb + co] : 1.f;
+        }
       if (!wait_bounded(tfull(ab), static_cast<uint32_t>(i >> 1) & 1u, ctl, kErrWaitEpilogue)) break;
       tc_fence_after();
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * acc_cols;
@@ -792,17 +866,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const bool c_ok = c8 < p.Cout;
       __nv_bfloat16* ybase = p.y + static_cast<size_t>(b) * p.H * p.W * ldc + cb + c8;
       auto process = [&](const uint32_t (&r)[32], int ch) {
-#pragma unroll
-        for (int jj = 0; jj < 32; jj += 2) {
-          const uint32_t w = pack_bf16x2((__uint_as_float(r[jj]) + bb) * so,
-                                         (__uint_as_float(r[jj + 1]) + bb) * so);
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + jj * 64 + lane * 2),
-                       "h"(static_cast<unsigned short>(w & 0xFFFFu))
-                       : "memory");
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stage + (jj + 1) * 64 + lane * 2),
-                       "h"(static_cast<unsigned short>(w >> 16))
-                       : "memory");
-        }
+        epi_stage_chunk(r, bb, so, stage, lane);
         __syncwarp();
         int pix = ch * 32 + (lane >> 2);
         int rr = pix / p.Wp;
@@ -811,10 +875,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int it = 0; it < 4; ++it) {
           const int oh = h0 + rr;
           if (c_ok && pix < p.n_virt && cw < p.W && oh < p.H) {
-            uint4 v;
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                         : "r"(stage + (it * 8 + (lane >> 2)) * 64 + part * 16));
+            const uint4 v = ld_shared_v4(epi_slot(stage, it * 8 + (lane >> 2), part));
             *reinterpret_cast<uint4*>(ybase + (static_cast<size_t>(oh) * p.W + cw) * ldc) = v;
           }
           pix += 8;
@@ -825,15 +886,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       };
       uint32_t ra[32], rb[32];
       int ch = grp;
-      if (ch < nchunks) tmem_ld_32x32b_x32(trow + ch * 32, ra);
+      if (ch < nchunks) epi_load_chunk(trow, ch * 32, ra);
       while (ch < nchunks) {
         tmem_ld_wait(ra);
-        if (ch + 2 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 2) * 32, rb);
+        if (ch + 2 < nchunks) epi_load_chunk(trow, (ch + 2) * 32, rb);
         process(ra, ch);
         ch += 2;
         if (ch >= nchunks) break;
         tmem_ld_wait(rb);
-        if (ch + 2 < nchunks) tmem_ld_32x32b_x32(trow + (ch + 2) * 32, ra);
+        if (ch + 2 < nchunks) epi_load_chunk(trow, (ch + 2) * 32, ra);
         process(rb, ch);
         ch += 2;
       }

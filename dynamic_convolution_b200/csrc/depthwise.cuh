@@ -528,30 +528,47 @@ __global__ void __maxnreg__((DwpShape<K, NC>::kRegs))
           uint64_t xv[K + NC - 1];
 #pragma unroll
           for (int kw = 0; kw < K + NC - 1; ++kw) xv[kw] = bf16x2_to_f32x2(xr[kw * CCp]);
+          // the K open rows this input row feeds (kh = 0 opens row ir from
+          // the bias, kh = K-1 completes row ir - K + 1); for small windows the
+          // products run kw-outer so that the K x NC accumulator chains
+          // interleave
+          bool live[K];
+          uint64_t a[K][NC];
 #pragma unroll
-          for (int kh = K - 1; kh >= 0; --kh) {
+          for (int kh = 0; kh < K; ++kh) {
             const int o = ir - kh;
-            const int slot = (j - kh + K) % K;  // o % K
-            bool live;
-            if (KIND == MID) live = true;
-            else if (KIND == HEAD) live = j >= kh;       // o >= 0; o < K <= RB
-            else if (KIND == TAIL) live = j < kh;        // o < RB; o >= RB - K + 1 >= 0
-            else live = o >= 0 && o < p.RB;
-            if (!live) continue;
-            uint64_t a[NC];
+            if (KIND == MID) live[kh] = true;
+            else if (KIND == HEAD) live[kh] = j >= kh;   // o >= 0; o < K <= RB
+            else if (KIND == TAIL) live[kh] = j < kh;    // o < RB; o >= RB - K + 1 >= 0
+            else live[kh] = o >= 0 && o < p.RB;
 #pragma unroll
-            for (int q = 0; q < NC; ++q) a[q] = kh == 0 ? bias2 : acc[slot][q];
+            for (int q = 0; q < NC; ++q) a[kh][q] = kh == 0 ? bias2 : acc[(j - kh + K) % K][q];
+          }
+          if constexpr (K * NC <= 10) {
 #pragma unroll
             for (int kw = 0; kw < K; ++kw)
 #pragma unroll
-              for (int q = 0; q < NC; ++q) a[q] = ffma2(xv[kw + q], w2[kh * K + kw], a[q]);
-            if (kh == K - 1) {
-              store_row(a, o);
-            } else {
+              for (int kh = 0; kh < K; ++kh)
+                if (live[kh])
 #pragma unroll
-              for (int q = 0; q < NC; ++q) acc[slot][q] = a[q];
-            }
+                  for (int q = 0; q < NC; ++q)
+                    a[kh][q] = ffma2(xv[kw + q], w2[kh * K + kw], a[kh][q]);
+          } else {  // larger windows: row by row (fewer live registers)
+#pragma unroll
+            for (int kh = 0; kh < K; ++kh)
+              if (live[kh])
+#pragma unroll
+                for (int kw = 0; kw < K; ++kw)
+#pragma unroll
+                  for (int q = 0; q < NC; ++q)
+                    a[kh][q] = ffma2(xv[kw + q], w2[kh * K + kw], a[kh][q]);
           }
+          if (live[K - 1]) store_row(a[K - 1], ir - (K - 1));
+#pragma unroll
+          for (int kh = 0; kh < K - 1; ++kh)
+            if (live[kh])
+#pragma unroll
+              for (int q = 0; q < NC; ++q) acc[(j - kh + K) % K][q] = a[kh][q];  // slot o % K
         }
       };
       using KMid = std::integral_constant<int, MID>;

@@ -243,7 +243,8 @@ bool tc_plan(const dynconv_desc* d, int variant, int sms, int max_smem, TcPlan* 
     if (n_pad > 256) { n0 = 256; n1 = n_pad - 256; }
     const int rows = std::max(box_rows * Wp, s_tap_max + n_pad);
     const int b_tile = (rows * 128 + 1023) / 1024 * 1024;
-    const size_t fixed = 1024 /*align slack*/ + 8 * 64 /*barriers*/ + 16 + 4 * d->n + 64;
+    const size_t fixed = 1024 /*align slack*/ + 8 * 64 /*barriers*/ + 16 + 4 * d->n + 64 +
+                         1024 /*the tile's biases and output attentions*/;
     const size_t T = dc::kTcATileBytes;
     int sb = kc > 1 ? 2 : 1;
     int sa = 0, se = 0;

@@ -181,6 +181,31 @@ __device__ __forceinline__ void tmem_ld_wait16(uint32_t (&r)[16]) {
       :
       : "memory");
 }
+// 16 TMEM lanes x 256 bits, four times along the columns (32 columns): thread
+// t receives, for column group j = 0..3, r[4j] = (lane t/4, column 8j + 2(t%4)),
+// r[4j+1] = (lane t/4, next column), r[4j+2], r[4j+3] = the same columns of
+// lane t/4 + 8.
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Four 8x8 b16 matrices stored transposed: register i is this thread's
+// fragment of matrix i (row t/4, columns 2(t%4) and +1); threads 8i .. 8i+7
+// give the shared addresses of matrix i's eight 16-byte rows.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1,
+                                                  uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};"
+               ::"r"(addr), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
