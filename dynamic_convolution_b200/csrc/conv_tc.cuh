@@ -88,7 +88,7 @@ struct TcParams {
   float chan_scale;       // bias before the single rounding of y
   int co_base;            // persistent kernel: channel offset of this launch in y and the biases
   int ld_c;               // persistent kernel: channel stride of y and bias rows (0: Cout)
-  int x_early;            // persistent kernel: first x boxes may load before the grid wait
+  int x_early;            // PREMIX: first x boxes may load before the grid wait (after a mixer)
   int se;                 // FUSED / OUTSIDE: expert-tile stages (16 KB each)
   unsigned long long* stamps;  // optional [grid][8] phase stamps for measurements, or null
 };
@@ -231,13 +231,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tma_prefetch_desc(&wmap);
   }
   __syncwarp();
+  // The first activation boxes need nothing but the barriers. After one of
+  // this library's mixing kernels (p.x_early: they signal their dependents
+  // only once every CTA is past its own wait, so whatever wrote x has
+  // completed) they are issued before this kernel's wait, overlapping the
+  // mixing kernel's tail; otherwise right after it.
+  const int pre_b = p.kc < SB ? p.kc : SB;
+  if (threadIdx.x == 32 && p.x_early) {
+    for (int cc = 0; cc < pre_b; ++cc) {
+      mbar_arrive_expect_tx(fullB(cc), 64u * 2u * p.Wp * p.b_box_rows);
+      tma_load_4d(b_base + cc * p.b_tile_bytes, &xmap, fullB(cc), cc * 64, -p.pad, h0 - p.pad, b);
+    }
+  }
   grid_dependency_wait();
   if (threadIdx.x == 32) {
     tc_stamp(p, 1);  // past the grid wait
-    // The first loads need nothing but the barriers: issue them now so their
-    // latency overlaps the rest of the set-up.
-    const int pre_b = p.kc < SB ? p.kc : SB;
-    for (int cc = 0; cc < pre_b; ++cc) {
+    for (int cc = 0; cc < (p.x_early ? 0 : pre_b); ++cc) {
       mbar_arrive_expect_tx(fullB(cc), 64u * 2u * p.Wp * p.b_box_rows);
       tma_load_4d(b_base + cc * p.b_tile_bytes, &xmap, fullB(cc), cc * 64, -p.pad, h0 - p.pad, b);
     }
@@ -279,7 +288,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp == 2) {
     // ============ expert-tile producer (FUSED, OUTSIDE): TMA, consumption order ============
-    if (VARIANT != kPremix && lane == 0) {
+    if constexpr (VARIANT != kPremix) {
+      if (lane == 0) {
       const int ne = VARIANT == kFused ? p.n : 1;
       int issued = 0;
       bool ok = true;
@@ -297,6 +307,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       for (int j = (issued > SE ? issued - SE : 0); j < issued; ++j)
         wait_drain(fullE(j % SE), static_cast<uint32_t>(j / SE) & 1u, p.wait_ns, p.err);
+      }
     }
     // ======================= weight producer (PREMIX) =======================
     if (VARIANT == kPremix && lane == 0) {
@@ -402,7 +413,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // tile (conflict-free), accumulates alpha_i * E_i in fp32 in expert order
     // (FUSED: the step's n experts; OUTSIDE: the step's one expert) and
     // rounds once to bf16 into the A stage.
-    if (VARIANT != kPremix) {
+    if constexpr (VARIANT != kPremix) {
       const int ne = VARIANT == kFused ? p.n : 1;
       int consumed = 0;
       bool ok = true;

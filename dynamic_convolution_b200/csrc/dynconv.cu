@@ -631,7 +631,9 @@ int launch_premix_conv(const dynconv_desc* d, const TcPlan& plan, const DeviceSt
     }
     return check_launch("tc_conv_persist_kernel");
   }
-  return launch_tc<dc::kPremix>(plan, xmap, wmap, stream);
+  TcPlan np = plan;
+  np.p.x_early = g_use_pdl.load() ? 1 : 0;  // right after one of this library's mixing kernels
+  return launch_tc<dc::kPremix>(np, xmap, wmap, stream);
 }
 
 // ------------------------------------------------------------ grouped PREMIX
@@ -1145,6 +1147,8 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
       ps.out = static_cast<__nv_bfloat16*>(ws);
       ps.a_in = a_in;
       ps.Cin = d->C_in;
+      ps.stamps = g_conv_stamps.load() ? reinterpret_cast<unsigned long long*>(g_conv_stamps.load()) +
+                                             4096 * 8 : nullptr;  // after the convolution's
       size_t smem = sizeof(float) * static_cast<size_t>(d->B) * d->n;
       if (a_in != nullptr) smem += sizeof(float) * static_cast<size_t>(d->B) * d->C_in;
       if (smem > static_cast<size_t>(st->max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
@@ -1380,7 +1384,8 @@ int dynconv_route(const dynconv_desc* desc, const void* x, const float* Wr, cons
   if (smem > static_cast<size_t>(st->max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
 
   dc::RouteParams p{desc->B, C, HW, desc->n, mode, tau, x, Wr, br, alpha,
-                    nsplit, piece_px, wr_smem, st->err, g_wait_ns.load()};
+                    nsplit, piece_px, wr_smem, st->err, g_wait_ns.load(),
+                    reinterpret_cast<unsigned long long*>(g_conv_stamps.load())};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nsplit, desc->B, 1);
   cfg.blockDim = dim3(dc::kRouteThreads, 1, 1);
@@ -1462,6 +1467,7 @@ int run_depthwise_pipe(const dynconv_desc* d, const DeviceState* st, const void*
   p.chan_scale = chan_scale;
   p.err = st->err;
   p.wait_ns = g_wait_ns.load();
+  p.stamps = reinterpret_cast<unsigned long long*>(g_conv_stamps.load());
   CUtensorMap xmap;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d->C_in), static_cast<cuuint64_t>(d->W),
                               static_cast<cuuint64_t>(d->H), static_cast<cuuint64_t>(d->B)};

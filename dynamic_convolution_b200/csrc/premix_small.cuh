@@ -35,6 +35,7 @@ struct PsParams {
   __nv_bfloat16* out;            // [B][wsize]
   const float* a_in;             // [B][Cin] input channel attention, or null
   int Cin;                       // input channels (with a_in: weight w has channel w % Cin)
+  unsigned long long* stamps;    // optional [grid][8] phase stamps for measurements, or null
 };
 
 // NMAX: the expert count rounded up to 2, 4 or 8 (fewer registers for fewer experts)
@@ -42,7 +43,19 @@ template <int NMAX>
 __global__ void __launch_bounds__(kPsThreads) premix_small_kernel(PsParams p) {
   extern __shared__ float ps_alpha[];  // [B][n], then [B][Cin] when a_in is given
   float* ps_ain = ps_alpha + p.B * p.n;
+  // phase stamps (measurement hook): [0] entry, [1] past the grid wait,
+  // [5] end, [6] SM id, [7] global timer at entry
+  unsigned long long* stp =
+      (p.stamps != nullptr && threadIdx.x == 0) ? p.stamps + blockIdx.x * 8 : nullptr;
+  if (stp) {
+    stp[0] = clock64();
+    stp[7] = globaltimer_ns();
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    stp[6] = smid;
+  }
   grid_dependency_wait();  // alpha comes from the routing kernel
+  if (stp) stp[1] = clock64();
   // The convolution may be scheduled once every CTA of this grid is past its
   // wait: everything launched before this kernel (the writer of x included)
   // has then completed, so the convolution may load x before its own wait.
@@ -111,6 +124,7 @@ __global__ void __launch_bounds__(kPsThreads) premix_small_kernel(PsParams p) {
       *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.wsize + ch * 8) = o;
     }
   }
+  if (stp) stp[5] = clock64();
 }
 
 // Host-side plan: as many samples per thread (up to 16) as keep at least one

@@ -54,6 +54,7 @@ struct RouteParams {
   int wr_smem;      // 1: Wr staged in shared memory, partial logits per rank
   int* err;
   long long wait_ns;
+  unsigned long long* stamps;  // optional [grid][8] phase stamps for measurements, or null
 };
 
 // Shared-memory carve-up, in bytes; the host sizes the launch with `total`.
@@ -172,7 +173,20 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // phase stamps (measurement hook): [0] entry, [1] past the grid wait, [2]
+  // slice summed, [3] past the cluster barrier, [5] end, [6] SM id, [7]
+  // global timer at entry
+  unsigned long long* stp =
+      (p.stamps != nullptr && t == 0) ? p.stamps + (static_cast<size_t>(b) * nsplit + rank) * 8 : nullptr;
+  if (stp) {
+    stp[0] = clock64();
+    stp[7] = globaltimer_ns();
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    stp[6] = smid;
+  }
   grid_dependency_wait();
+  if (stp) stp[1] = clock64();
   if (t == 0) {
     if (p.wr_smem) {
       const uint32_t wb = static_cast<uint32_t>(p.n) * C * 4u;
@@ -221,6 +235,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
       for (int j = 0; j < VEC; ++j) partial[static_cast<size_t>(pl) * C + v * VEC + j] = acc[j];
     }
   }
+  if (stp) stp[2] = clock64();
   if (rank == 0)  // read now: its latency overlaps the reductions below
     for (int i = t; i < p.n; i += kRouteThreads) brs[i] = p.br ? p.br[i] : 0.f;
   __syncthreads();
@@ -249,6 +264,10 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
     for (int c = t; c < C; c += kRouteThreads) dst[c] = g[c];
   }
   cluster.sync();  // remote stores visible to rank 0; with Wr staged, peers may exit after this
+  if (stp) {
+    stp[3] = clock64();
+    stp[5] = stp[3];
+  }
   if (*abort_flag && t == 0) {
     // a bounded wait gave up: let the copies still in flight land before exit
     for (int k = (issued > kRouteRing ? issued - kRouteRing : 0); k < issued; ++k)
@@ -309,6 +328,7 @@ __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(RouteParams p) 
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
         if (lane < p.n) out[lane] = e * (1.0f / s);
       }
+      if (stp) stp[5] = clock64();
     }
     return;
   }

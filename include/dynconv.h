@@ -318,8 +318,12 @@ unsigned long long dynconv_launch_count(void);
  * the kernel size is a multiple of 16 and the workspace 32-byte aligned
  * (measured slower on B200). For measurements.
  * key 13: the address of a device buffer of 64-bit words (0, the default:
- * off). While it is set, each CTA of the PREMIX, FUSED and OUTSIDE
- * tensor-core convolutions writes 8 words at [block * 8]: its SM cycle
+ * off). While it is set, the routing kernel (CTA rank r of sample b at
+ * [(b * ranks + r) * 8]), the pipelined depthwise kernel and the CUDA-core
+ * mixing kernel (at [(4096 + block) * 8]) record their phase times (the
+ * layouts are described at the kernels), and each CTA of
+ * the PREMIX, FUSED and OUTSIDE tensor-core convolutions writes 8 words at
+ * [block * 8]: its SM cycle
  * counter at entry, past the grid wait, when the first operands are in
  * shared memory, after the MMA issue of the (one-CTA-per-unit kernel: only;
  * persistent kernel: first) unit, when the accumulator is complete
