@@ -276,7 +276,7 @@ int run_chansum(const dynconv_desc* d, int sms, const void* v, int P, int C, flo
 // experts and kernels of a multiple of 128 weights.
 bool mixgrad_tc_ok(const dynconv_desc* d) {
   return dc_lib::mixgrad_tc_enabled() && d->dtype == DYNCONV_BF16 && d->B >= 1 && d->B <= 256 &&
-         d->n <= 32 && wsize_of(d) % dcb::kMtTile == 0;
+         d->n <= 64 && wsize_of(d) % dcb::kMtTile == 0;
 }
 
 // dexperts (complete) and one dalpha partial per CTA; returns the number of
@@ -286,7 +286,7 @@ int run_mixgrad_tc(const dynconv_desc* d, const dc_lib::DeviceInfo& di, const vo
                    int max_parts, int* nparts, cudaStream_t s) {
   const long long ws = wsize_of(d);
   dcb::MtParams p{};
-  p.B = d->B; p.n = d->n; p.nk = d->n <= 16 ? 16 : 32;
+  p.B = d->B; p.n = d->n; p.nk = d->n <= 16 ? 16 : d->n <= 32 ? 32 : 64;
   p.halves = (d->B + 127) / 128;
   p.wsize = ws;
   p.tiles = ws / dcb::kMtTile;
@@ -550,7 +550,14 @@ int dynconv_backward_data(const dynconv_desc* desc, const void* dy, const void* 
     if (rc) return rc;
     const int Cg = d->C_in / d->groups, Coutg = d->C_out / d->groups;
     const int taps_groups = d->KH * d->KW * d->groups;
-    if (Cg >= 8 && Coutg >= 8 && taps_groups <= 65535 && d->n <= 65535) {
+    if (d->dtype == DYNCONV_BF16 && Cg % 8 == 0 && Coutg % 8 == 0 && taps_groups <= 65535 &&
+        d->n <= 65535 && (reinterpret_cast<uintptr_t>(experts) & 15u) == 0) {
+      // 64 x 64 tiles moved as 16-byte chunks
+      const dim3 grid(((Cg + 63) / 64) * ((Coutg + 63) / 64), taps_groups, d->n);
+      dcb::transpose_experts_v8_kernel<<<grid, 256, 0, s>>>(
+          d->C_in, d->C_out, d->KH, d->KW, d->groups, static_cast<const __nv_bfloat16*>(experts),
+          reinterpret_cast<__nv_bfloat16*>(workspace));
+    } else if (Cg >= 8 && Coutg >= 8 && taps_groups <= 65535 && d->n <= 65535) {
       // 32 x 32 tiles of each group's [Coutg][Cg] matrix per (tap, group, expert)
       const dim3 grid(((Cg + 31) / 32) * ((Coutg + 31) / 32), taps_groups, d->n), block(32, 8);
       if (d->dtype == DYNCONV_F32)

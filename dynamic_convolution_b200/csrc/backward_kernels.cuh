@@ -663,4 +663,47 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The same flipped transposition for bf16 with both channel counts of a
+// group multiples of 8, in 64 x 64 tiles moved as 16-byte chunks: a CTA reads
+// 64 output-channel rows of 128 contiguous bytes, stages them in shared
+// memory (row pitch 66 elements, so the column gathers spread over the
+// banks) and writes 64 input-channel rows of 128 contiguous bytes. Grid
+// (tiles of the group's [Coutg][Cg] matrix, taps * groups, n); 256 threads.
+__global__ void __launch_bounds__(256)
+    transpose_experts_v8_kernel(int Cin, int Cout, int KH, int KW, int groups,
+                                const __nv_bfloat16* __restrict__ E, __nv_bfloat16* __restrict__ Et) {
+  constexpr int kPitch = 66;  // elements per staged row
+  __shared__ __align__(16) unsigned short tile[64 * kPitch];
+  const int Cg = Cin / groups, Coutg = Cout / groups;
+  const int tiles_c = (Cg + 63) / 64;
+  const int cil0 = (blockIdx.x % tiles_c) * 64, col0 = (blockIdx.x / tiles_c) * 64;
+  const int taps = KH * KW;
+  const int tap = blockIdx.y % taps, g = blockIdx.y / taps;
+  const int kh = tap / KW, kw = tap - kh * KW;
+  const int tap_src = (KH - 1 - kh) * KW + (KW - 1 - kw);
+  const size_t i = blockIdx.z;
+  for (int u = threadIdx.x; u < 512; u += 256) {
+    const int r = u >> 3, c8 = (u & 7) * 8;  // output-channel row, input-channel offset
+    const int col = col0 + r, cil = cil0 + c8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (col < Coutg && cil < Cg)
+      v = *reinterpret_cast<const uint4*>(E + ((i * Cout + g * Coutg + col) * taps + tap_src) * Cg + cil);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(tile + r * kPitch + c8);
+    dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+  }
+  __syncthreads();
+  for (int u = threadIdx.x; u < 512; u += 256) {
+    const int r = u >> 3, c8 = (u & 7) * 8;  // input-channel row, output-channel offset
+    const int cil = cil0 + r, col = col0 + c8;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w[j] = static_cast<uint32_t>(tile[(c8 + 2 * j) * kPitch + r]) |
+             (static_cast<uint32_t>(tile[(c8 + 2 * j + 1) * kPitch + r]) << 16);
+    if (col < Coutg && cil < Cg)
+      *reinterpret_cast<uint4*>(Et + ((i * Cin + g * Cg + cil) * taps + tap) * Coutg + col) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 }  // namespace dcb

@@ -32,7 +32,7 @@ constexpr int kMtThreads = 192;
 constexpr int kMtTile = 128;  // weights per tile
 
 struct MtParams {
-  int B, n, nk;       // samples (<= 256), experts (<= 32), experts padded to 16 (16 or 32)
+  int B, n, nk;       // samples (<= 256), experts (<= 64), experts padded to 16, 32 or 64
   int halves;         // ceil(B / 128)
   int stages;
   long long wsize;
@@ -72,9 +72,11 @@ __global__ void __launch_bounds__(kMtThreads, 1)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
-  // TMEM columns: dexperts accumulators (2 nk <= 64 columns) at 0 and 64,
-  // dalpha halves (nk <= 32) at 128 and 160
-  constexpr uint32_t kCols = 256;
+  // TMEM columns: two dexperts accumulators of 2 nk columns (hi | lo) at 0
+  // and 2 nk, then the dalpha halves (nk columns each) from 4 nk
+  const uint32_t dex_cols = 2u * p.nk;
+  const uint32_t da_base = 2u * dex_cols;
+  const uint32_t kCols = da_base + 2u * p.nk <= 256u ? 256u : 512u;
 
   if (warp == 0) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), kCols);
@@ -170,7 +172,7 @@ __global__ void __launch_bounds__(kMtThreads, 1)
           ok = false;
           break;
         }
-        const uint32_t d_dex = tmem_base + ab * 64;
+        const uint32_t d_dex = tmem_base + ab * dex_cols;
         for (int h = 0; h < p.halves; ++h) {
           if (!wait_bounded(full(s), ph, ctl, kErrWaitMma)) { ok = false; break; }
           tc_fence_after();
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(kMtThreads, 1)
             tc_mma_f16(d_dex, dl_mn + aoff, al + boff, idesc_dex, 1u);
           }
           // dalpha of this half: K = the tile's 128 weights, two 64-weight atoms
-          const uint32_t d_da = tmem_base + 128 + h * 32;
+          const uint32_t d_da = tmem_base + da_base + h * p.nk;
           for (int kk = 0; kk < 8; ++kk) {
             const int a = kk >> 2;
             const uint64_t koff = (kk & 3) * 2;
@@ -223,39 +225,43 @@ __global__ void __launch_bounds__(kMtThreads, 1)
         break;
       }
       tc_fence_after();
-      // columns 0..nk-1: dW * alpha_hi, nk..2nk-1: dW * alpha_lo
-      uint32_t r[32], r2[32];
-      const uint32_t ta = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * 64;
-      tmem_ld_32x32b_x32(ta, r);
-      tmem_ld_32x32b_x32(ta + 32, r2);
-      tmem_ld_wait(r);
-      tmem_ld_wait(r2);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty(ab));
+      // columns 0..nk-1: dW * alpha_hi, nk..2nk-1: dW * alpha_lo; 32 experts
+      // per pass
+      const uint32_t ta = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * dex_cols;
       float* dst = p.dexperts + t * kMtTile + 32 * q + lane;
-      if (p.nk == 16) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (i < p.n) dst[static_cast<size_t>(i) * p.wsize] = __uint_as_float(r[i]) + __uint_as_float(r[i + 16]);
-      } else {
+      for (int e0 = 0; e0 < p.nk; e0 += 32) {
+        uint32_t r[32], r2[32];
+        tmem_ld_32x32b_x32(ta + e0, r);
+        tmem_ld_32x32b_x32(ta + p.nk + e0, r2);
+        tmem_ld_wait(r);
+        tmem_ld_wait(r2);
+        if (e0 + 32 >= p.nk) {
+          // every read of this accumulator is complete: release it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty(ab));
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (i < p.n) dst[static_cast<size_t>(i) * p.wsize] = __uint_as_float(r[i]) + __uint_as_float(r2[i]);
+          if (e0 + i < p.n && i < p.nk)
+            dst[static_cast<size_t>(e0 + i) * p.wsize] = __uint_as_float(r[i]) + __uint_as_float(r2[i]);
       }
     }
     if (ok && my_tiles > 0 && wait_bounded(adone, 0, ctl, kErrWaitEpilogue)) {
       tc_fence_after();
       for (int h = 0; h < p.halves; ++h) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + 128 + h * 32, r);
-        tmem_ld_wait(r);
-        const int b = h * 128 + 32 * q + lane;
-        if (b < p.B) {
-          float* dst = p.part + (static_cast<size_t>(blockIdx.x) * p.B + b) * p.n;
+        for (int e0 = 0; e0 < p.nk; e0 += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(
+              tmem_base + (static_cast<uint32_t>(32 * q) << 16) + da_base + h * p.nk + e0, r);
+          tmem_ld_wait(r);
+          const int b = h * 128 + 32 * q + lane;
+          if (b < p.B) {
+            float* dst = p.part + (static_cast<size_t>(blockIdx.x) * p.B + b) * p.n + e0;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < p.n) dst[i] = __uint_as_float(r[i]);
+            for (int i = 0; i < 32; ++i)
+              if (e0 + i < p.n && i < p.nk) dst[i] = __uint_as_float(r[i]);
+          }
         }
       }
     } else if (my_tiles == 0) {
