@@ -34,6 +34,7 @@ constexpr int kPmEpiWarps = 8;    // two per TMEM lane quarter, one 128-column h
 constexpr int kPmN = 256;         // weights per tile
 constexpr int kPmHalf = kPmN / 2; // columns of one epilogue warp
 constexpr int kPmStageBytes = 32 * kPmHalf * 2;  // one warp's 32 samples x 128 bf16
+constexpr int kPmMaxStages = 4;   // expert stages in flight (8 measured slower on the deep 3x3 layer)
 
 __host__ __device__ inline int pm_nk(int n) { return (n + 15) / 16 * 16; }
 __host__ __device__ inline int pm_kcols(int n) { return (pm_nk(n) + 63) / 64; }
@@ -57,6 +58,9 @@ struct PmParams {
   int a_bytes;           // bytes of all A operands
   int stage_bytes;       // bytes of one expert stage
   int direct_store;      // 1: epilogue stores from registers (wsize % 16 == 0, out 32-byte aligned)
+  int stg_bytes;         // one epilogue warp's staging tile: 32 samples x (128 / rep) bf16
+  int rep;               // 1, 2 or 4: copies of the batch in the 128 A rows (B <= 128 / rep), each
+                         // copy's epilogue warps storing 256 / rep of the tile's columns
   const float* alpha;
   __nv_bfloat16* out;    // [B][wsize]
   int* err;
@@ -85,7 +89,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   const uint32_t a_base = base;                         // [m_tile][hi/lo][kcol][128 rows x 128 B]
   const uint32_t e_base = a_base + p.a_bytes;           // [stage][4 atoms][nk rows x 128 B]
   const uint32_t st_base = e_base + S * p.stage_bytes;  // epilogue staging: 8 warps x 8 KB
-  const uint32_t bar_base = st_base + (p.direct_store ? 0u : kPmEpiWarps * kPmStageBytes);
+  const uint32_t bar_base = st_base + (p.direct_store ? 0u : kPmEpiWarps * p.stg_bytes);
   auto full = [&](int s) { return bar_base + 8u * s; };
   auto empty = [&](int s) { return bar_base + 8u * (S + s); };
   auto tfull = [&](int a) { return bar_base + 8u * (2 * S + a); };
@@ -130,10 +134,12 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   for (int e = threadIdx.x; e < p.a_bytes / 16; e += kPmThreads)
     st_shared_v4(a_base + e * 16, make_uint4(0u, 0u, 0u, 0u));
   __syncthreads();
-  for (int e = threadIdx.x; e < na; e += kPmThreads) {
-    const int m = e / p.n, k = e - m * p.n;  // sample row, expert
-    const int mt = m >> 7, r = m & 127;
-    const float a = alpha_s[e];
+  const int spr = 128 / p.rep;  // A rows per copy of the batch
+  for (int e = threadIdx.x; e < na * p.rep; e += kPmThreads) {
+    const int g = e / na, e1 = e - g * na;   // copy, (sample, expert)
+    const int m = e1 / p.n, k = e1 - m * p.n;  // sample row, expert
+    const int mt = m >> 7, r = (m & 127) + g * spr;
+    const float a = alpha_s[e1];
     const __nv_bfloat16 hi = __float2bfloat16_rn(a);
     const __nv_bfloat16 lo = __float2bfloat16_rn(a - __bfloat162float(hi));
     const uint32_t off = static_cast<uint32_t>(k >> 6) * 16384u + r * 128u +
@@ -232,19 +238,25 @@ __global__ void __launch_bounds__(kPmThreads, 1)
     // flight.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
-    const uint32_t stg = st_base + (warp - 2) * kPmStageBytes;
+    const uint32_t stg = st_base + (warp - 2) * p.stg_bytes;
     long long ntile = ntile0;
     int mt = mt0;
     for (long long j = 0; j < my_tiles; ++j) {
       const int ab = static_cast<int>(j & 1);
       if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j >> 1) & 1), ctl, kErrWaitEpilogue)) break;
       tc_fence_after();
-      // a warp whose 32 samples are all past the batch only releases the buffer
-      const int row0 = mt * 128 + 32 * q;
+      // TMEM lanes 32q .. 32q+31 hold samples row0 .. row0+31 of copy g; copy
+      // g's warps store columns [g, g+1) * 256 / rep of the tile, this half
+      // of them (cw columns). A warp whose samples are all past the batch
+      // only releases the buffer.
+      const int g = (32 * q) / spr;
+      const int row0 = mt * 128 + 32 * q - g * spr;
+      const int cw = kPmHalf / p.rep;
+      const int col0 = g * (kPmN / p.rep) + half * cw;
       const bool live = row0 < p.B;
-      const long long w0 = ntile * kPmN + half * kPmHalf;
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * kPmN + half * kPmHalf;
+      const long long w0 = ntile * kPmN + (p.rep == 1 ? half * kPmHalf : col0);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * kPmN +
+                             (p.rep == 1 ? half * kPmHalf : col0);
       if (live) {
         uint32_t ra[32], rb[32];
         if (p.direct_store) {
@@ -273,8 +285,9 @@ __global__ void __launch_bounds__(kPmThreads, 1)
             emit(rb, ch + 1);
           }
         } else {
-          // staged: row `lane` of the 32 x 256-byte block, 16-byte chunk c at
-          // position c ^ (lane % 16): 32 lanes fill each bank group evenly
+          // staged: row `lane` of the 32 x (2 cw)-byte block, 16-byte chunk c
+          // at position c ^ (lane % (cw / 8)): 32 lanes fill the bank groups evenly
+          const int cpr = cw / 8;  // 16-byte chunks per row
           auto stage_chunk = [&](const uint32_t (&r)[32], int ch) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -283,18 +296,20 @@ __global__ void __launch_bounds__(kPmThreads, 1)
               o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
               o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
               o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-              const int c = ch * 4 + v;  // 16-byte chunk of this sample's 256-byte segment
-              st_shared_v4(stg + lane * 256 + ((c ^ (lane & 15)) << 4), o);
+              const int c = ch * 4 + v;  // 16-byte chunk of this sample's segment
+              st_shared_v4(stg + lane * (2 * cw) + ((c ^ (lane & (cpr - 1))) << 4), o);
             }
           };
+          const int nch = cw / 32;
           tmem_ld_32x32b_x32(taddr, ra);
 #pragma unroll 1
-          for (int ch = 0; ch < kPmHalf / 32; ch += 2) {
+          for (int ch = 0; ch < nch; ch += 2) {
             tmem_ld_wait(ra);
-            tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, rb);
+            if (ch + 1 < nch) tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, rb);
             stage_chunk(ra, ch);
+            if (ch + 1 >= nch) break;
             tmem_ld_wait(rb);
-            if (ch + 2 < kPmHalf / 32) tmem_ld_32x32b_x32(taddr + (ch + 2) * 32, ra);
+            if (ch + 2 < nch) tmem_ld_32x32b_x32(taddr + (ch + 2) * 32, ra);
             stage_chunk(rb, ch + 1);
           }
         }
@@ -304,18 +319,21 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty(ab));
       if (live && !p.direct_store) {
-        // two samples per store instruction: lanes 0..15 row sr, 16..31 row sr+1,
-        // 16 bytes each = one 256-byte segment per row
-        const int part = lane & 15;
+        // 32 / cpr samples per store instruction, cpr lanes of 16 bytes each
+        // covering one sample's 2 cw-byte segment (cw = 128: lanes 0..15 row
+        // sr, 16..31 row sr + 1)
+        const int cpr = cw / 8;
+        const int part = lane & (cpr - 1);
+        const int rstep = 32 / cpr;
         const long long w = w0 + part * 8;
         const bool wok = w < p.wsize;
         const int nrows = min(32, p.B - row0);
 #pragma unroll 4
-        for (int sr = lane >> 4; sr < 32; sr += 2) {
+        for (int sr = lane / cpr; sr < 32; sr += rstep) {
           uint4 v;
           asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                       : "r"(stg + sr * 256 + ((part ^ (sr & 15)) << 4)));
+                       : "r"(stg + sr * (2 * cw) + ((part ^ (sr & (cpr - 1))) << 4)));
           if (wok && sr < nrows)
             *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row0 + sr) * p.wsize + w) = v;
         }
@@ -364,9 +382,13 @@ inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bf
   p.stage_bytes = p.nk * 512;
   p.direct_store =
       (allow_direct && wsize % 16 == 0 && (reinterpret_cast<uintptr_t>(out_ws) & 31u) == 0) ? 1 : 0;
-  const int staging = p.direct_store ? 0 : kPmEpiWarps * kPmStageBytes;
+  // small batches: copies of the batch fill the 128 accumulator rows, so that
+  // every epilogue warp has samples to store (each copy a share of the columns)
+  p.rep = (p.direct_store || p.m_tiles != 1) ? 1 : B <= 32 ? 4 : B <= 64 ? 2 : 1;
+  p.stg_bytes = kPmStageBytes / p.rep;
+  const int staging = p.direct_store ? 0 : kPmEpiWarps * p.stg_bytes;
   const int budget = 200 * 1024 - p.a_bytes - staging - 4 * B * n;
-  p.stages = std::min(4, budget / p.stage_bytes);
+  p.stages = std::min(kPmMaxStages, budget / p.stage_bytes);
   if (p.stages < 2) return -3;
   p.alpha = alpha;
   p.out = out_ws;
