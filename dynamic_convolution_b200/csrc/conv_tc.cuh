@@ -123,7 +123,9 @@ __device__ __forceinline__ uint32_t epi_slot(uint32_t stage, int pix, int chunk)
 }
 
 // y = (accumulator + bias) * scale, rounded once to bf16, staged transposed.
-// bias[h][e] and scale[h][e] belong to channel 16h + 8e + lane/4 of the quarter.
+// bias[h][e] and scale[h][e] belong to channel 16h + 8e + lane/4 of the quarter
+// (SCALED false: no output attention, scale 1).
+template <bool SCALED>
 __device__ __forceinline__ void epi_stage_chunk(const uint32_t (&r)[32], const float (&bias)[2][2],
                                                 const float (&scale)[2][2], uint32_t stage,
                                                 int lane) {
@@ -135,9 +137,15 @@ __device__ __forceinline__ void epi_stage_chunk(const uint32_t (&r)[32], const f
     for (int j = 0; j < 4; ++j) {
       const uint32_t* v = r + 16 * h + 4 * j;
 #pragma unroll
-      for (int e = 0; e < 2; ++e)
-        P[j][e] = pack_bf16x2((__uint_as_float(v[2 * e]) + bias[h][e]) * scale[h][e],
-                              (__uint_as_float(v[2 * e + 1]) + bias[h][e]) * scale[h][e]);
+      for (int e = 0; e < 2; ++e) {
+        float a = __uint_as_float(v[2 * e]) + bias[h][e];
+        float b = __uint_as_float(v[2 * e + 1]) + bias[h][e];
+        if (SCALED) {
+          a *= scale[h][e];
+          b *= scale[h][e];
+        }
+        P[j][e] = pack_bf16x2(a, b);
+      }
     }
 #pragma unroll
     for (int s2 = 0; s2 < 2; ++s2) {
@@ -534,7 +542,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) ps[e] = 0.f;
       auto process = [&](const uint32_t (&r)[32], int ch) {
-        epi_stage_chunk(r, bb, so, stage, lane);
+        if (p.a_out != nullptr) epi_stage_chunk<true>(r, bb, so, stage, lane);
+        else epi_stage_chunk<false>(r, bb, so, stage, lane);
         __syncwarp();
         int pix = ch * 32 + (lane >> 2);
         int rr = pix / p.Wp;
@@ -877,7 +886,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const bool c_ok = c8 < p.Cout;
       __nv_bfloat16* ybase = p.y + static_cast<size_t>(b) * p.H * p.W * ldc + cb + c8;
       auto process = [&](const uint32_t (&r)[32], int ch) {
-        epi_stage_chunk(r, bb, so, stage, lane);
+        if (p.a_out != nullptr) epi_stage_chunk<true>(r, bb, so, stage, lane);
+        else epi_stage_chunk<false>(r, bb, so, stage, lane);
         __syncwarp();
         int pix = ch * 32 + (lane >> 2);
         int rr = pix / p.Wp;
