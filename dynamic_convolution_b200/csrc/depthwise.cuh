@@ -363,17 +363,15 @@ __global__ void __maxnreg__((DwpShape<K, NC>::kRegs))
   __syncthreads();
   grid_dependency_wait();  // alpha (and x) come from earlier kernels
   // phase stamps (measurement hook): [0] entry after set-up, [1] slabs in,
-  // [2] first tile in, [3] cycles thread 0 waited for tiles, [4] cycles it
-  // spent mixing, [5] end, [6] SM id, [7] global timer at entry
-  unsigned long long* stp = p.stamps != nullptr && t == 0 ? p.stamps + blockIdx.x * 8 : nullptr;
-  if (stp) {
+  // [5] end, [6] SM id, [7] global timer at entry
+  if (p.stamps != nullptr && t == 0) {
+    unsigned long long* stp = p.stamps + blockIdx.x * 8;
     stp[0] = clock64();
     stp[7] = globaltimer_ns();
     uint32_t smid;
     asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
     stp[6] = smid;
   }
-  unsigned long long wait_cyc = 0, mix_cyc = 0;
 
   auto tile_coords = [&](int k, int& b, int& oh0, int& ow0) {
     int u = t_begin + k;
@@ -437,7 +435,7 @@ __global__ void __maxnreg__((DwpShape<K, NC>::kRegs))
   // ================================ compute ================================
   if (my_tiles == 0) return;
   if (!wait_bounded(ebar, 0, ctl, kErrWaitDwp)) return;
-  if (stp) stp[1] = clock64();
+  if (p.stamps != nullptr && t == 0) p.stamps[blockIdx.x * 8 + 1] = clock64();
   const int cgrp = t / CCp, pair = t - (t / CCp) * CCp;
   const int col = NC * cgrp;  // this thread's output columns col .. col + NC - 1 in the tile
   const int w_floats = (KK + 1) * p.CC;
@@ -451,19 +449,13 @@ __global__ void __maxnreg__((DwpShape<K, NC>::kRegs))
   for (int k = 0; k < my_tiles; ++k) {
     const int s = k % p.S;
     const uint32_t ph = static_cast<uint32_t>(k / p.S) & 1u;
-    const unsigned long long w0 = stp ? clock64() : 0;
     if (!wait_bounded(full(s), ph, ctl, kErrWaitDwp)) return;
-    if (stp) {
-      wait_cyc += clock64() - w0;
-      if (k == 0) stp[2] = clock64();
-    }
     int b, oh0, ow0;
     tile_coords(k, b, oh0, ow0);
     unsigned char* st = sm + static_cast<size_t>(s) * p.stage_bytes;
     const float* misc = reinterpret_cast<const float*>(st + p.misc_off);
     const float* fin = misc + p.n;
 
-    const unsigned long long m0c = stp ? clock64() : 0;
     if (b != prev_b) {
       // ---- a new sample: mix its kernels (fp32, expert by expert) into the
       // next of the two buffers; the previous sample's buffer may still be
@@ -498,7 +490,6 @@ __global__ void __maxnreg__((DwpShape<K, NC>::kRegs))
 #pragma unroll
       for (int q = 0; q < KK; ++q) w2[q] = *reinterpret_cast<const uint64_t*>(wb + q * p.CC + 2 * pair);
       bias2 = *reinterpret_cast<const uint64_t*>(wb + KK * p.CC + 2 * pair);
-      if (stp) mix_cyc += clock64() - m0c;
       ao0 = fin[p.CC + 2 * pair];
       ao1 = fin[p.CC + 2 * pair + 1];
     }
@@ -609,11 +600,7 @@ __global__ void __maxnreg__((DwpShape<K, NC>::kRegs))
     __syncwarp();
     if (lane == 0) mbar_arrive(empty(s));
   }
-  if (stp) {
-    stp[3] = wait_cyc;
-    stp[4] = mix_cyc;
-    stp[5] = clock64();
-  }
+  if (p.stamps != nullptr && t == 0) p.stamps[blockIdx.x * 8 + 5] = clock64();
 }
 
 }  // namespace dc

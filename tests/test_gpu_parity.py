@@ -268,6 +268,42 @@ def test_streamed_mixing_equals_two_kernels(name):
     assert torch.isfinite(outs[0].float()).all()
 
 
+def test_streamed_mixing_more_streams_than_slots():
+    """The streamed mixing keeps per-stream counters in a fixed number of
+    device slots (64). With more streams than free slots, a stream without a
+    slot runs the two-kernel form instead of sharing another stream's
+    counters: every stream's output equals the two-kernel output bit for bit."""
+    cfg = synth.LayerConfig("slots", synth.BF16, 4, 64, 64, 8, 8, 3, 3, 1, 1, 1, 4,
+                            synth.SIGMOID, 1.0)
+    inp = synth.make_inputs(cfg, seed=12, structured=1.0)
+    L = Layer(inp)
+    L.route()
+    d = L.desc(dc.VARIANT_PREMIX)
+    nbytes = dc.dynconv_workspace_size(d)
+    ws0 = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    try:
+        assert dc.dynconv_test_hook(7, 2) == dc.OK  # two-kernel form, CUDA-core mixer
+        dc.check(dc.dynconv_forward(d, L.x, L.experts, L.alpha, L.bias, L.y, ws0, nbytes))
+        torch.cuda.synchronize()
+        ref = L.y.clone()
+        assert dc.dynconv_test_hook(7, 0) == dc.OK
+        assert dc.dynconv_test_hook(6, 1) == dc.OK  # streamed mixing
+        streams = [torch.cuda.Stream() for _ in range(72)]
+        outs = [torch.full_like(L.y, float("nan")) for _ in streams]
+        wss = [torch.zeros(nbytes, dtype=torch.uint8, device="cuda") for _ in streams]
+        torch.cuda.synchronize()
+        for st, y, ws in zip(streams, outs, wss):
+            dc.check(dc.dynconv_forward(d, L.x, L.experts, L.alpha, L.bias, y, ws, nbytes,
+                                        st.cuda_stream), "dynconv_forward (streamed)")
+        torch.cuda.synchronize()
+        assert dc.dynconv_device_status(None) == dc.OK
+    finally:
+        dc.dynconv_test_hook(6, 0)
+        dc.dynconv_test_hook(7, 0)
+    for y in outs:
+        assert torch.equal(y, ref)
+
+
 @pytest.mark.parametrize("name", ["resnet18_3x3", "effnet_expand_1x1"])
 @pytest.mark.parametrize("mixer", [(0, 1), (0, 2), (1, 0)], ids=["gemm", "cuda-core", "streamed"])
 def test_premix_mixers_full_size(name, mixer):
