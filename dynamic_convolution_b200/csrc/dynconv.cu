@@ -72,10 +72,12 @@ constexpr int kTransposedMixMax = 0;   // batches up to this mix with the transp
 std::atomic<int> g_conv_persist{1};  // PREMIX convolution: 1 persistent kernel when it fits, 0 one CTA per unit
 std::atomic<int> g_group_mix{0};     // PREMIX, n > 8, large B*|W|: 0 one pass, 1 grouped mixing
                                      // pipeline (concurrent), 2 grouped in sequence
-std::atomic<int> g_premix_direct{0}; // premix epilogue: 1 stores from registers when aligned, 0 staged
+std::atomic<int> g_premix_direct{0}; // premix epilogue: 0 per-lane stores of staged rows, 1 stores
+                                     // from registers when aligned, 2 TMA stores of staged boxes
 std::atomic<int> g_mixgrad_tc{1};    // backward: 1 tensor-core mixing gradient when it fits, 0 CUDA cores
 std::atomic<long long> g_group_bytes{40LL << 20};  // target bytes of one group's mixed kernels
-std::atomic<unsigned long long> g_conv_stamps{0};  // device buffer for the convolution's phase stamps
+std::atomic<unsigned long long> g_conv_stamps{0};
+std::atomic<int> g_persist_rows{0};  // persistent convolution: output rows per unit (0: planned)  // device buffer for the convolution's phase stamps
 std::atomic<long long> g_group_min{64LL << 20};    // below this B*|W| the one-pass form is used
 thread_local char g_last_err[256] = "";
 
@@ -318,10 +320,12 @@ bool tc_plan_persist(const dynconv_desc* d, int sms, int max_smem, TcPlan* out) 
   const int s_tap_max = (d->KH - 1) * Wp + (d->KW - 1);
   bool found = false;
   TcPlan best;
+  const int want_rows = g_persist_rows.load();
   for (int R = 1; R <= d->H; ++R) {
     const int n_virt = R * Wp;
     const int n_pad = (n_virt + 15) / 16 * 16;
     if (n_pad > 256) break;
+    if (want_rows > 0 && R != std::min(want_rows, d->H)) continue;
     const int box_rows = R + d->KH - 1;
     if (box_rows > 256) break;
     const int rows = std::max(box_rows * Wp, s_tap_max + n_pad);
@@ -782,7 +786,7 @@ int run_grouped(const dynconv_desc* d, const GroupPlan& gp, const DeviceState* s
       dc::PremixLaunch pl;
       rc = dc::plan_premix(E + c0 * taps_cin, alpha + b0 * d->n, static_cast<__nv_bfloat16*>(wsl),
                            s.B, d->n, wg, st->err, g_wait_ns.load(), mix_sms, g_encode, &pl,
-                           static_cast<long long>(wsize), g_premix_direct.load() != 0);
+                           static_cast<long long>(wsize), g_premix_direct.load());
       if (rc == -2) {
         std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(grouped premix) failed");
         return DYNCONV_ERR_CUDA;
@@ -790,7 +794,7 @@ int run_grouped(const dynconv_desc* d, const GroupPlan& gp, const DeviceState* s
       if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
       e = ensure_smem(dc::premix_kernel, pl.smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
-      dc::premix_kernel<<<pl.grid, dc::kPmThreads, pl.smem, ax->aux>>>(pl.emap, pl.p);
+      dc::premix_kernel<<<pl.grid, dc::kPmThreads, pl.smem, ax->aux>>>(pl.emap, pl.omap, pl.p);
       rc = check_launch("premix_kernel (grouped)");
     }
     if (rc) return rc;
@@ -893,7 +897,7 @@ int run_grouped_seq(const dynconv_desc* d, const GroupPlan& gp, const DeviceStat
       dc::PremixLaunch pl;
       rc = dc::plan_premix(E + c0 * taps_cin, alpha + b0 * d->n, static_cast<__nv_bfloat16*>(ws),
                            s.B, d->n, wg, st->err, g_wait_ns.load(), st->sms, g_encode, &pl,
-                           static_cast<long long>(wsize), g_premix_direct.load() != 0);
+                           static_cast<long long>(wsize), g_premix_direct.load());
       if (rc == -2) {
         std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(grouped premix) failed");
         return DYNCONV_ERR_CUDA;
@@ -902,7 +906,7 @@ int run_grouped_seq(const dynconv_desc* d, const GroupPlan& gp, const DeviceStat
       e = ensure_smem(dc::premix_kernel, pl.smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
       e = launch_pdl(dc::premix_kernel, dim3(pl.grid), dim3(dc::kPmThreads), pl.smem, stream,
-                     pl.emap, pl.p);
+                     pl.emap, pl.omap, pl.p);
       if (e != cudaSuccess) {
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return cuda_fail(e, "premix_kernel launch (grouped)");
@@ -1202,7 +1206,7 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   rc = dc::plan_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
                        static_cast<__nv_bfloat16*>(ws), d->B, d->n,
                        static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in, st->err,
-                       g_wait_ns.load(), st->sms, g_encode, &pl, 0, g_premix_direct.load() != 0);
+                       g_wait_ns.load(), st->sms, g_encode, &pl, 0, g_premix_direct.load());
   if (rc == -2) {
     std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(premix) failed");
     return DYNCONV_ERR_CUDA;
@@ -1212,7 +1216,7 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
     cudaError_t e = ensure_smem(dc::premix_kernel, pl.smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
     e = launch_pdl(dc::premix_kernel, dim3(pl.grid), dim3(dc::kPmThreads), pl.smem, stream,
-                   pl.emap, pl.p);
+                   pl.emap, pl.omap, pl.p);
     if (e != cudaSuccess) {
       g_launches.fetch_add(1, std::memory_order_relaxed);
       return cuda_fail(e, "premix_kernel launch");
@@ -1303,8 +1307,13 @@ int dynconv_test_hook(int key, long long value) {
     g_conv_stamps.store(static_cast<unsigned long long>(value));
     return DYNCONV_OK;
   }
+  if (key == 14) {
+    if (value < 0 || value > 256) return DYNCONV_ERR_INVALID_ARG;
+    g_persist_rows.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
   if (key == 12) {
-    if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
+    if (value < 0 || value > 2) return DYNCONV_ERR_INVALID_ARG;
     g_premix_direct.store(static_cast<int>(value));
     return DYNCONV_OK;
   }

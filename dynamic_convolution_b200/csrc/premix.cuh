@@ -18,10 +18,13 @@
 //    two per TMEM lane quarter (32 samples), each taking one 128-column half
 //    of the tile, two 32-column TMEM loads in flight: each rounds to bf16,
 //    stages its 32 x 128 block in shared memory (XOR-swizzled 16-byte
-//    chunks), and writes it back as whole 256-byte row segments (two samples
-//    per store instruction). (A second form stores each lane's 64 contiguous
-//    bytes straight from registers; measured slower, it stays for
-//    measurements.)
+//    chunks), and writes it back as whole 256-byte row segments (two
+//    samples per store instruction). (Two other forms stay for
+//    measurements, both measured slower: each lane storing its 64 contiguous
+//    bytes straight from registers, and the staged block as 64-column boxes
+//    in the 128-byte swizzle written by TMA tensor stores -- the TMA unit
+//    writes the 32 scattered sample rows of a box more slowly than the
+//    lanes do.)
 // Persistent: one CTA per SM walks the (weight-tile, sample-tile) space.
 #pragma once
 
@@ -57,7 +60,9 @@ struct PmParams {
   long long tiles;       // n_tiles * m_tiles
   int a_bytes;           // bytes of all A operands
   int stage_bytes;       // bytes of one expert stage
-  int direct_store;      // 1: epilogue stores from registers (wsize % 16 == 0, out 32-byte aligned)
+  int store_mode;        // epilogue: 0 staged rows written by per-lane 16-byte stores; 1
+                         // stores from registers (wsize % 16 == 0, out 32-byte aligned); 2
+                         // staged boxes written by TMA tensor stores
   int stg_bytes;         // one epilogue warp's staging tile: 32 samples x (128 / rep) bf16
   int rep;               // 1, 2 or 4: copies of the batch in the 128 A rows (B <= 128 / rep), each
                          // copy's epilogue warps storing 256 / rep of the tile's columns
@@ -78,7 +83,8 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t 
 }
 
 __global__ void __launch_bounds__(kPmThreads, 1)
-    premix_kernel(const __grid_constant__ CUtensorMap emap, PmParams p) {
+    premix_kernel(const __grid_constant__ CUtensorMap emap,
+                  const __grid_constant__ CUtensorMap omap, PmParams p) {
   extern __shared__ __align__(1024) unsigned char pm_smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(pm_smem_raw);
@@ -89,7 +95,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   const uint32_t a_base = base;                         // [m_tile][hi/lo][kcol][128 rows x 128 B]
   const uint32_t e_base = a_base + p.a_bytes;           // [stage][4 atoms][nk rows x 128 B]
   const uint32_t st_base = e_base + S * p.stage_bytes;  // epilogue staging: 8 warps x 8 KB
-  const uint32_t bar_base = st_base + (p.direct_store ? 0u : kPmEpiWarps * p.stg_bytes);
+  const uint32_t bar_base = st_base + (p.store_mode == 1 ? 0u : kPmEpiWarps * p.stg_bytes);
   auto full = [&](int s) { return bar_base + 8u * s; };
   auto empty = [&](int s) { return bar_base + 8u * (S + s); };
   auto tfull = [&](int a) { return bar_base + 8u * (2 * S + a); };
@@ -122,6 +128,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&emap);
+    if (p.store_mode == 2) tma_prefetch_desc(&omap);
   }
   // A operands: alpha split into bf16 hi + lo, zero outside [B) x [n).
   // Stage alpha in shared memory first (all loads in flight at once), then
@@ -239,6 +246,15 @@ __global__ void __launch_bounds__(kPmThreads, 1)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const uint32_t stg = st_base + (warp - 2) * p.stg_bytes;
+    // TMA-store staging (store_mode 2): boxes of bc columns x 32 samples,
+    // rows of 2 bc bytes in the tensor map's swizzle -- 16-byte chunk c of
+    // row r at c ^ (r % 8) for 128-byte rows, c ^ ((r / 2) % 4) for 64-byte
+    // rows, which also spreads a store instruction's 32 rows over the banks
+    const int cw = kPmHalf / p.rep;        // columns of this warp
+    const int bc = cw < 64 ? cw : 64;      // columns of one box
+    const int cpb_log = bc == 64 ? 3 : 2;  // log2 of 16-byte chunks per box row
+    const int sw_sh = 3 - cpb_log;
+    const uint32_t box_bytes = 64u * bc;   // 32 rows x 2 bc bytes
     long long ntile = ntile0;
     int mt = mt0;
     for (long long j = 0; j < my_tiles; ++j) {
@@ -251,7 +267,6 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       // only releases the buffer.
       const int g = (32 * q) / spr;
       const int row0 = mt * 128 + 32 * q - g * spr;
-      const int cw = kPmHalf / p.rep;
       const int col0 = g * (kPmN / p.rep) + half * cw;
       const bool live = row0 < p.B;
       const long long w0 = ntile * kPmN + (p.rep == 1 ? half * kPmHalf : col0);
@@ -259,7 +274,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
                              (p.rep == 1 ? half * kPmHalf : col0);
       if (live) {
         uint32_t ra[32], rb[32];
-        if (p.direct_store) {
+        if (p.store_mode == 1) {
           // each lane (one sample) writes 64 contiguous bytes per chunk as two
           // 32-byte stores straight from registers
           const int b = row0 + lane;
@@ -283,6 +298,37 @@ __global__ void __launch_bounds__(kPmThreads, 1)
             tmem_ld_wait(rb);
             if (ch + 2 < kPmHalf / 32) tmem_ld_32x32b_x32(taddr + (ch + 2) * 32, ra);
             emit(rb, ch + 1);
+          }
+        } else if (p.store_mode == 2) {
+          // the previous tile's stores have finished reading the staging tile
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+          auto stage_box = [&](const uint32_t (&r)[32], int ch) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+              o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+              o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+              o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+              const int c = ch * 4 + v;  // 16-byte chunk of this sample's cw columns
+              const int box = c >> cpb_log, cc = c & ((1 << cpb_log) - 1);
+              st_shared_v4(stg + box * box_bytes + lane * (2 * bc) +
+                               ((cc ^ ((lane >> sw_sh) & ((1 << cpb_log) - 1))) << 4),
+                           o);
+            }
+          };
+          const int nch = cw / 32;
+          tmem_ld_32x32b_x32(taddr, ra);
+#pragma unroll 1
+          for (int ch = 0; ch < nch; ch += 2) {
+            tmem_ld_wait(ra);
+            if (ch + 1 < nch) tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, rb);
+            stage_box(ra, ch);
+            if (ch + 1 >= nch) break;
+            tmem_ld_wait(rb);
+            if (ch + 2 < nch) tmem_ld_32x32b_x32(taddr + (ch + 2) * 32, ra);
+            stage_box(rb, ch + 1);
           }
         } else {
           // staged: row `lane` of the 32 x (2 cw)-byte block, 16-byte chunk c
@@ -318,7 +364,19 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty(ab));
-      if (live && !p.direct_store) {
+      if (live && p.store_mode == 2) {
+        // publish the staged boxes to the async proxy, then one lane stores
+        // them (rows past the batch and columns past the kernel are clipped)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int box = 0; box * bc < cw; ++box)
+            if (w0 + box * bc < p.wsize)
+              tma_store_2d(&omap, stg + box * box_bytes, static_cast<int>(w0 + box * bc), row0);
+          bulk_commit_group();
+        }
+      }
+      if (live && p.store_mode == 0) {
         // 32 / cpr samples per store instruction, cpr lanes of 16 bytes each
         // covering one sample's 2 cw-byte segment (cw = 128: lanes 0..15 row
         // sr, 16..31 row sr + 1)
@@ -343,6 +401,8 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       mt += dm;
       if (mt >= p.m_tiles) { mt -= p.m_tiles; ++ntile; }
     }
+    // every store of this warp has completed before the CTA exits
+    if (lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();
@@ -357,6 +417,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
 struct PremixLaunch {
   PmParams p;
   CUtensorMap emap;
+  CUtensorMap omap;  // the output [B][wsize] for the TMA stores (store_mode 2)
   unsigned grid = 0;
   size_t smem = 0;
 };
@@ -366,9 +427,11 @@ template <typename EncodeFn>
 inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bfloat16* out_ws,
                        int B, int n, long long wsize, int* err, long long wait_ns, int sms,
                        EncodeFn encode, PremixLaunch* out, long long estride = 0,
-                       bool allow_direct = true) {
+                       int store_mode = 0) {
   // estride: elements from one expert to the next (default wsize); a larger
-  // stride mixes a contiguous slice of wsize elements of every expert
+  // stride mixes a contiguous slice of wsize elements of every expert.
+  // store_mode: the epilogue form asked for (PmParams::store_mode); a form
+  // whose alignment the output does not meet falls back to 0.
   PmParams& p = out->p;
   p = PmParams{};
   p.B = B;
@@ -380,13 +443,18 @@ inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bf
   p.tiles = n_tiles * p.m_tiles;
   p.a_bytes = 2 * p.m_tiles * pm_kcols(n) * 16384;
   p.stage_bytes = p.nk * 512;
-  p.direct_store =
-      (allow_direct && wsize % 16 == 0 && (reinterpret_cast<uintptr_t>(out_ws) & 31u) == 0) ? 1 : 0;
+  const uintptr_t oaddr = reinterpret_cast<uintptr_t>(out_ws);
+  if (store_mode == 1 && wsize % 16 == 0 && (oaddr & 31u) == 0)
+    p.store_mode = 1;
+  else if (store_mode == 2 && (oaddr & 15u) == 0 && wsize < (1LL << 31))
+    p.store_mode = 2;
+  else
+    p.store_mode = 0;
   // small batches: copies of the batch fill the 128 accumulator rows, so that
   // every epilogue warp has samples to store (each copy a share of the columns)
-  p.rep = (p.direct_store || p.m_tiles != 1) ? 1 : B <= 32 ? 4 : B <= 64 ? 2 : 1;
+  p.rep = (p.store_mode == 1 || p.m_tiles != 1) ? 1 : B <= 32 ? 4 : B <= 64 ? 2 : 1;
   p.stg_bytes = kPmStageBytes / p.rep;
-  const int staging = p.direct_store ? 0 : kPmEpiWarps * p.stg_bytes;
+  const int staging = p.store_mode == 1 ? 0 : kPmEpiWarps * p.stg_bytes;
   const int budget = 200 * 1024 - p.a_bytes - staging - 4 * B * n;
   p.stages = std::min(kPmMaxStages, budget / p.stage_bytes);
   if (p.stages < 2) return -3;
@@ -402,6 +470,21 @@ inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bf
              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return -2;
+  if (p.store_mode == 2) {
+    // boxes of min(128 / rep, 64) columns x 32 samples; 128-byte rows take the
+    // 128-byte swizzle, 64-byte rows (four copies of the batch) the 64-byte one
+    const int bc = std::min(kPmHalf / p.rep, 64);
+    const cuuint64_t odims[2] = {static_cast<cuuint64_t>(wsize), static_cast<cuuint64_t>(B)};
+    const cuuint64_t ostrides[1] = {static_cast<cuuint64_t>(wsize) * 2};
+    const cuuint32_t obox[2] = {static_cast<cuuint32_t>(bc), 32u};
+    if (encode(&out->omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_ws, odims, ostrides, obox, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE,
+               bc == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return -2;
+  } else {
+    std::memset(&out->omap, 0, sizeof(out->omap));
+  }
   // at least 120 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
   out->smem = std::max<size_t>(120 * 1024, 1024 + static_cast<size_t>(p.a_bytes) +
                                                static_cast<size_t>(p.stages) * p.stage_bytes +

@@ -313,10 +313,12 @@ unsigned long long dynconv_launch_count(void);
  * (per-sample weight gradients as bf16 hi / lo planes, one pass for the
  * expert and attention gradients) when it applies; 0 the CUDA-core kernel.
  * key 12: the epilogue of the tensor-core mixing GEMM: 0 (default) stages
- * each tile through shared memory and writes whole rows; 1 stores each
- * thread's 32 mixed weights straight from registers (two 32-byte stores) when
- * the kernel size is a multiple of 16 and the workspace 32-byte aligned
- * (measured slower on B200). For measurements.
+ * each warp's block in shared memory and writes it with per-lane 16-byte
+ * stores (two samples' rows per instruction); 1 stores each thread's 32
+ * mixed weights straight from registers (two 32-byte stores) when the kernel
+ * size is a multiple of 16 and the workspace 32-byte aligned; 2 stages the
+ * block as swizzled boxes and writes them with TMA tensor stores (both
+ * measured slower on B200). For measurements.
  * key 13: the address of a device buffer of 64-bit words (0, the default:
  * off). While it is set, the routing kernel (CTA rank r of sample b at
  * [(b * ranks + r) * 8]), the pipelined depthwise kernel and the CUDA-core
@@ -331,6 +333,10 @@ unsigned long long dynconv_launch_count(void);
  * epilogue is done; its SM id; and the global timer at entry. The buffer
  * must hold 8 words per CTA of every such launch made meanwhile. For
  * measurements.
+ * key 14: output rows per unit of the persistent PREMIX convolution: 0
+ * (default) as planned; 1..256 that many (capped at the layer's height)
+ * when such a unit fits, else the convolution falls back to one CTA per
+ * unit. For measurements.
  * Returns DYNCONV_OK or DYNCONV_ERR_INVALID_ARG. */
 int dynconv_test_hook(int key, long long value);
 

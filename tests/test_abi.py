@@ -146,8 +146,16 @@ def test_test_hook_arguments(lib):
     assert dc.dynconv_test_hook(10, 3) == dc.ERR_INVALID_ARG
     assert dc.dynconv_test_hook(10, 2) == dc.OK
     assert dc.dynconv_test_hook(10, 0) == dc.OK
-    assert dc.dynconv_test_hook(12, 2) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(12, 3) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(12, -1) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(12, 2) == dc.OK
     assert dc.dynconv_test_hook(12, 1) == dc.OK
+    assert dc.dynconv_test_hook(12, 0) == dc.OK
+    assert dc.dynconv_test_hook(14, 257) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(14, -1) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(14, 7) == dc.OK
+    assert dc.dynconv_test_hook(14, 0) == dc.OK
+    assert dc.dynconv_test_hook(15, 0) == dc.ERR_INVALID_ARG   # no such key
 
 
 def test_pooled_entry_points_host_side(lib):

@@ -332,12 +332,16 @@ def test_premix_transposed_mixer_full_size(name):
         dc.dynconv_test_hook(7, 0)
 
 
-@pytest.mark.parametrize("B", [3, 40, 100], ids=["B3-four-copies", "B40-two-copies", "B100"])
-def test_premix_gemm_small_batches(B):
-    """The tensor-core mixing GEMM (test hook 7 = 1) when the batch is copied
-    into the 128 accumulator rows (B <= 32: four copies, B <= 64: two), each
-    copy's epilogue warps storing a share of the columns: against the oracle
-    element by element on a ragged kernel size."""
+@pytest.mark.parametrize("store", [0, 1, 2], ids=["lane-store", "register-store", "tma-store"])
+@pytest.mark.parametrize("B", [3, 40, 100, 250],
+                         ids=["B3-four-copies", "B40-two-copies", "B100", "B250-ragged-row-tile"])
+def test_premix_gemm_small_batches(B, store):
+    """The tensor-core mixing GEMM (test hook 7 = 1) with each epilogue form
+    (test hook 12): the batch copied into the 128 accumulator rows (B <= 32:
+    four copies, B <= 64: two), each copy's epilogue warps storing a share of
+    the columns; a ragged second row tile (B = 250); a kernel size that is not
+    a multiple of the 256-weight tile. Against the oracle element by
+    element."""
     cfg = synth.LayerConfig(f"premix_b{B}", synth.BF16, B, 24, 40, 7, 9, 3, 3, 1, 1, 1, 12,
                             synth.SOFTMAX, 2.0)
     inp = synth.make_inputs(cfg, seed=11, structured=1.0)
@@ -348,14 +352,16 @@ def test_premix_gemm_small_batches(B):
                      device="cuda")
     try:
         assert dc.dynconv_test_hook(7, 1) == dc.OK
+        assert dc.dynconv_test_hook(12, store) == dc.OK
         L.y.fill_(float("nan"))
         L.forward(dc.VARIANT_PREMIX, workspace=ws)
         assert dc.dynconv_device_status(None) == dc.OK
     finally:
         dc.dynconv_test_hook(7, 0)
+        dc.dynconv_test_hook(12, 0)
     ref = oracle.forward(inp.x_f64, inp.experts_f64, a32, inp.bias, stride=1, pad=1)
     r = compare(from_device(L.y), ref, synth.BF16)
-    assert r["ok"], (B, r)
+    assert r["ok"], (B, store, r)
 
 
 def test_premix_cuda_core_mixer_refuses_many_experts():
