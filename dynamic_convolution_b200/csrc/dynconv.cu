@@ -49,6 +49,7 @@ struct DeviceState {
   int sms = 0;
   int max_smem_optin = 0;
   int cc_major = 0, cc_minor = 0;
+  long long l2_bytes = 0;
 };
 
 std::mutex g_mu;
@@ -72,12 +73,13 @@ constexpr int kTransposedMixMax = 0;   // batches up to this mix with the transp
 std::atomic<int> g_conv_persist{1};  // PREMIX convolution: 1 persistent kernel when it fits, 0 one CTA per unit
 std::atomic<int> g_group_mix{0};     // PREMIX, n > 8, large B*|W|: 0 one pass, 1 grouped mixing
                                      // pipeline (concurrent), 2 grouped in sequence
-std::atomic<int> g_premix_direct{0}; // premix epilogue: 0 per-lane stores of staged rows, 1 stores
-                                     // from registers when aligned, 2 TMA stores of staged boxes
+std::atomic<int> g_premix_direct{0}; // premix epilogue: 1 stores from registers when aligned, 0 staged
 std::atomic<int> g_mixgrad_tc{1};    // backward: 1 tensor-core mixing gradient when it fits, 0 CUDA cores
 std::atomic<long long> g_group_bytes{40LL << 20};  // target bytes of one group's mixed kernels
 std::atomic<unsigned long long> g_conv_stamps{0};
-std::atomic<int> g_persist_rows{0};  // persistent convolution: output rows per unit (0: planned)  // device buffer for the convolution's phase stamps
+std::atomic<int> g_persist_rows{0};  // persistent convolution: output rows per unit (0: planned)
+std::atomic<int> g_premix_dyn{1};    // mixing GEMM (one pass) tiles from a counter: 1 when the
+                                     // experts exceed half the L2, 2 always, 0 never (static)  // device buffer for the convolution's phase stamps
 std::atomic<long long> g_group_min{64LL << 20};    // below this B*|W| the one-pass form is used
 thread_local char g_last_err[256] = "";
 
@@ -112,6 +114,7 @@ int device_state(DeviceState** out) {
     }
     st.sms = prop.multiProcessorCount;
     st.max_smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
+    st.l2_bytes = prop.l2CacheSize;
     st.cc_major = prop.major;
     st.cc_minor = prop.minor;
     void* addr = nullptr;
@@ -498,10 +501,12 @@ bool dwp_plan(const dynconv_desc* d, int sms, int max_smem, bool has_bias, int n
 size_t premix_wb_bytes(const dynconv_desc* d) {
   return (static_cast<size_t>(d->B) * d->C_out * d->KH * d->KW * d->C_in * 2 + 255) & ~size_t(255);
 }
+// The mixed kernels, then 256 bytes for the mixing GEMM's tile counter.
+constexpr size_t kPmCtrBytes = 256;
 size_t premix_workspace(const dynconv_desc* d) {
   if (!tc_shape_ok(d)) return 0;
   if (!dc::premix_shape_ok(d->B, d->n, d->C_out, d->KH * d->KW, d->C_in)) return 0;
-  return premix_wb_bytes(d);
+  return premix_wb_bytes(d) + kPmCtrBytes;
 }
 
 // Cost-model choice among the kernels that can run this descriptor.
@@ -786,7 +791,7 @@ int run_grouped(const dynconv_desc* d, const GroupPlan& gp, const DeviceState* s
       dc::PremixLaunch pl;
       rc = dc::plan_premix(E + c0 * taps_cin, alpha + b0 * d->n, static_cast<__nv_bfloat16*>(wsl),
                            s.B, d->n, wg, st->err, g_wait_ns.load(), mix_sms, g_encode, &pl,
-                           static_cast<long long>(wsize), g_premix_direct.load());
+                           static_cast<long long>(wsize), g_premix_direct.load() != 0);
       if (rc == -2) {
         std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(grouped premix) failed");
         return DYNCONV_ERR_CUDA;
@@ -794,7 +799,7 @@ int run_grouped(const dynconv_desc* d, const GroupPlan& gp, const DeviceState* s
       if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
       e = ensure_smem(dc::premix_kernel, pl.smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
-      dc::premix_kernel<<<pl.grid, dc::kPmThreads, pl.smem, ax->aux>>>(pl.emap, pl.omap, pl.p);
+      dc::premix_kernel<<<pl.grid, dc::kPmThreads, pl.smem, ax->aux>>>(pl.emap, pl.p);
       rc = check_launch("premix_kernel (grouped)");
     }
     if (rc) return rc;
@@ -897,7 +902,7 @@ int run_grouped_seq(const dynconv_desc* d, const GroupPlan& gp, const DeviceStat
       dc::PremixLaunch pl;
       rc = dc::plan_premix(E + c0 * taps_cin, alpha + b0 * d->n, static_cast<__nv_bfloat16*>(ws),
                            s.B, d->n, wg, st->err, g_wait_ns.load(), st->sms, g_encode, &pl,
-                           static_cast<long long>(wsize), g_premix_direct.load());
+                           static_cast<long long>(wsize), g_premix_direct.load() != 0);
       if (rc == -2) {
         std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(grouped premix) failed");
         return DYNCONV_ERR_CUDA;
@@ -906,7 +911,7 @@ int run_grouped_seq(const dynconv_desc* d, const GroupPlan& gp, const DeviceStat
       e = ensure_smem(dc::premix_kernel, pl.smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
       e = launch_pdl(dc::premix_kernel, dim3(pl.grid), dim3(dc::kPmThreads), pl.smem, stream,
-                     pl.emap, pl.omap, pl.p);
+                     pl.emap, pl.p);
       if (e != cudaSuccess) {
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return cuda_fail(e, "premix_kernel launch (grouped)");
@@ -1203,10 +1208,21 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
     return launch_premix_conv(d, plan, st, x, xmap, wmap, stream);
   }
   dc::PremixLaunch pl;
+  // tile counter after the mixed kernels, zeroed on the stream before the launch
+  // (when the expert bank streams from HBM, the CTAs' expert reads arrive at
+  // uneven rates; from L2 they do not, and the counter's memset would only
+  // cost the launch its programmatic overlap with the routing kernel)
+  const double expert_bytes = 2.0 * d->n * d->C_out * d->KH * d->KW * d->C_in;
+  const int dyn = g_premix_dyn.load();
+  unsigned int* tile_ctr =
+      (dyn == 2 || (dyn == 1 && expert_bytes > 0.5 * st->l2_bytes))
+          ? reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + premix_wb_bytes(d))
+          : nullptr;
   rc = dc::plan_premix(static_cast<const __nv_bfloat16*>(experts), alpha,
                        static_cast<__nv_bfloat16*>(ws), d->B, d->n,
                        static_cast<long long>(d->C_out) * d->KH * d->KW * d->C_in, st->err,
-                       g_wait_ns.load(), st->sms, g_encode, &pl, 0, g_premix_direct.load());
+                       g_wait_ns.load(), st->sms, g_encode, &pl, 0, g_premix_direct.load() != 0,
+                       tile_ctr);
   if (rc == -2) {
     std::snprintf(g_last_err, sizeof(g_last_err), "cuTensorMapEncodeTiled(premix) failed");
     return DYNCONV_ERR_CUDA;
@@ -1215,8 +1231,12 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   {
     cudaError_t e = ensure_smem(dc::premix_kernel, pl.smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
+    if (tile_ctr != nullptr) {
+      e = cudaMemsetAsync(tile_ctr, 0, sizeof(unsigned int), stream);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(premix tile counter)");
+    }
     e = launch_pdl(dc::premix_kernel, dim3(pl.grid), dim3(dc::kPmThreads), pl.smem, stream,
-                   pl.emap, pl.omap, pl.p);
+                   pl.emap, pl.p);
     if (e != cudaSuccess) {
       g_launches.fetch_add(1, std::memory_order_relaxed);
       return cuda_fail(e, "premix_kernel launch");
@@ -1307,13 +1327,18 @@ int dynconv_test_hook(int key, long long value) {
     g_conv_stamps.store(static_cast<unsigned long long>(value));
     return DYNCONV_OK;
   }
+  if (key == 18) {
+    if (value < 0 || value > 2) return DYNCONV_ERR_INVALID_ARG;
+    g_premix_dyn.store(static_cast<int>(value));
+    return DYNCONV_OK;
+  }
   if (key == 14) {
     if (value < 0 || value > 256) return DYNCONV_ERR_INVALID_ARG;
     g_persist_rows.store(static_cast<int>(value));
     return DYNCONV_OK;
   }
   if (key == 12) {
-    if (value < 0 || value > 2) return DYNCONV_ERR_INVALID_ARG;
+    if (value != 0 && value != 1) return DYNCONV_ERR_INVALID_ARG;
     g_premix_direct.store(static_cast<int>(value));
     return DYNCONV_OK;
   }

@@ -18,14 +18,17 @@
 //    two per TMEM lane quarter (32 samples), each taking one 128-column half
 //    of the tile, two 32-column TMEM loads in flight: each rounds to bf16,
 //    stages its 32 x 128 block in shared memory (XOR-swizzled 16-byte
-//    chunks), and writes it back as whole 256-byte row segments (two
-//    samples per store instruction). (Two other forms stay for
-//    measurements, both measured slower: each lane storing its 64 contiguous
-//    bytes straight from registers, and the staged block as 64-column boxes
-//    in the 128-byte swizzle written by TMA tensor stores -- the TMA unit
-//    writes the 32 scattered sample rows of a box more slowly than the
-//    lanes do.)
-// Persistent: one CTA per SM walks the (weight-tile, sample-tile) space.
+//    chunks), and writes it back as whole 256-byte row segments (two samples
+//    per store instruction). (A second form stores each lane's 64 contiguous
+//    bytes straight from registers; measured slower, it stays for
+//    measurements.)
+// Persistent: one CTA per SM walks the (weight-tile, sample-tile) space,
+// either statically (tile c + j * grid for CTA c, every role counting along)
+// or taking the next tile from a global counter, so that CTAs whose expert
+// reads arrive faster take more tiles; then the producer publishes each
+// tile's index in a 16-entry ring in shared memory (tagged with its sequence
+// number) for the MMA and epilogue warps, and an end entry closes the
+// sequence.
 #pragma once
 
 #include "common.cuh"
@@ -60,9 +63,7 @@ struct PmParams {
   long long tiles;       // n_tiles * m_tiles
   int a_bytes;           // bytes of all A operands
   int stage_bytes;       // bytes of one expert stage
-  int store_mode;        // epilogue: 0 staged rows written by per-lane 16-byte stores; 1
-                         // stores from registers (wsize % 16 == 0, out 32-byte aligned); 2
-                         // staged boxes written by TMA tensor stores
+  int direct_store;      // 1: epilogue stores from registers (wsize % 16 == 0, out 32-byte aligned)
   int stg_bytes;         // one epilogue warp's staging tile: 32 samples x (128 / rep) bf16
   int rep;               // 1, 2 or 4: copies of the batch in the 128 A rows (B <= 128 / rep), each
                          // copy's epilogue warps storing 256 / rep of the tile's columns
@@ -70,7 +71,10 @@ struct PmParams {
   __nv_bfloat16* out;    // [B][wsize]
   int* err;
   long long wait_ns;
+  unsigned int* tile_ctr;  // zeroed counter: tiles taken dynamically (null: statically)
 };
+
+constexpr int kPmRing = 16;  // tile-index ring entries (more than stages + 3 in flight)
 
 __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
   uint64_t d = 0;
@@ -83,8 +87,7 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t 
 }
 
 __global__ void __launch_bounds__(kPmThreads, 1)
-    premix_kernel(const __grid_constant__ CUtensorMap emap,
-                  const __grid_constant__ CUtensorMap omap, PmParams p) {
+    premix_kernel(const __grid_constant__ CUtensorMap emap, PmParams p) {
   extern __shared__ __align__(1024) unsigned char pm_smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(pm_smem_raw);
@@ -95,7 +98,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   const uint32_t a_base = base;                         // [m_tile][hi/lo][kcol][128 rows x 128 B]
   const uint32_t e_base = a_base + p.a_bytes;           // [stage][4 atoms][nk rows x 128 B]
   const uint32_t st_base = e_base + S * p.stage_bytes;  // epilogue staging: 8 warps x 8 KB
-  const uint32_t bar_base = st_base + (p.store_mode == 1 ? 0u : kPmEpiWarps * p.stg_bytes);
+  const uint32_t bar_base = st_base + (p.direct_store ? 0u : kPmEpiWarps * p.stg_bytes);
   auto full = [&](int s) { return bar_base + 8u * s; };
   auto empty = [&](int s) { return bar_base + 8u * (S + s); };
   auto tfull = [&](int a) { return bar_base + 8u * (2 * S + a); };
@@ -105,6 +108,9 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   const WaitCtl ctl{abort_flag, p.err, p.wait_ns};
+  // ring entry of sequence number j: (j << 32) | (tile + 1), 0 in the low half = end
+  volatile unsigned long long* ring = reinterpret_cast<volatile unsigned long long*>(
+      misc + 16 + ((4 * p.B * p.n + 15) & ~15));
 
   if (warp == 0) {
     tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), 512);
@@ -126,9 +132,9 @@ __global__ void __launch_bounds__(kPmThreads, 1)
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
+    for (int i = 0; i < kPmRing; ++i) ring[i] = ~0ull;  // no sequence number matches
     fence_mbar_init();
     tma_prefetch_desc(&emap);
-    if (p.store_mode == 2) tma_prefetch_desc(&omap);
   }
   // A operands: alpha split into bf16 hi + lo, zero outside [B) x [n).
   // Stage alpha in shared memory first (all loads in flight at once), then
@@ -164,26 +170,67 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Static hand-out: tile j of this CTA is t = blockIdx.x + j * gridDim.x,
+  // walked with incremental counters by every role (no END entry needed).
+  const bool dyn = p.tile_ctr != nullptr;
   const long long my_tiles =
       p.tiles > blockIdx.x ? (p.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-
-  // Tile j of this CTA is t = blockIdx.x + j * gridDim.x, i.e. (weight tile
-  // t / m_tiles, sample tile t % m_tiles); every role walks the same sequence
-  // with incremental counters (no 64-bit divisions on the issue paths).
   const long long ntile0 = blockIdx.x / p.m_tiles;
   const int mt0 = blockIdx.x % p.m_tiles;
   const long long dn = gridDim.x / p.m_tiles;
   const int dm = gridDim.x % p.m_tiles;
+  // Tile t is (weight tile t / m_tiles, sample tile t % m_tiles). The
+  // epilogue finds tile j's ring entry once the producer has written it (before
+  // that tile's loads, long before its accumulator is complete): a bounded
+  // poll on the entry's sequence tag.
+  auto ring_tile = [&](long long j, long long& t) -> bool {
+    const unsigned long long want = static_cast<unsigned long long>(j) << 32;
+    unsigned long long e = ring[j & (kPmRing - 1)];
+    if ((e & ~0xFFFFFFFFull) != want) {
+      const uint64_t t0 = globaltimer_ns();
+      while (((e = ring[j & (kPmRing - 1)]) & ~0xFFFFFFFFull) != want) {
+        if (*abort_flag) return false;
+        if (static_cast<long long>(globaltimer_ns() - t0) > p.wait_ns) {
+          *abort_flag = 1;
+          atomicCAS(p.err, 0, kErrWaitEpilogue);
+          return false;
+        }
+      }
+    }
+    t = static_cast<long long>(e & 0xFFFFFFFFull) - 1;
+    return true;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       long long issued = 0;
-      long long ntile = ntile0;
-      int mt = mt0;
       int s = 0;
       uint32_t ph = 0;
-      for (long long j = 0; j < my_tiles; ++j) {
+      bool ended = false;
+      long long ntile_s = ntile0;
+      int mt_s = mt0;
+      for (long long j = 0;; ++j) {
+        if (!dyn && j >= my_tiles) break;
         if (!wait_bounded(empty(s), ph ^ 1u, ctl, kErrWaitProducer)) break;
+        long long ntile = ntile_s;
+        if (dyn) {
+          // a tile is claimed only once a stage is free to load it
+          long long t = static_cast<long long>(atomicAdd(p.tile_ctr, 1u));
+          if (t >= p.tiles) t = -1;  // end of this CTA's sequence
+          ring[j & (kPmRing - 1)] = (static_cast<unsigned long long>(j) << 32) |
+                                    static_cast<unsigned long long>(t + 1);
+          if (t < 0) {
+            mbar_arrive(full(s));  // publishes the end entry
+            ended = true;
+            break;
+          }
+          ntile = p.m_tiles == 1 ? t : static_cast<long long>(static_cast<uint32_t>(t) /
+                                                            static_cast<uint32_t>(p.m_tiles));
+        } else {
+          ntile_s += dn;
+          mt_s += dm;
+          if (mt_s >= p.m_tiles) { mt_s -= p.m_tiles; ++ntile_s; }
+        }
         mbar_arrive_expect_tx(full(s), static_cast<uint32_t>(p.stage_bytes));
         const uint32_t dst = e_base + s * p.stage_bytes;
 #pragma unroll
@@ -191,12 +238,14 @@ __global__ void __launch_bounds__(kPmThreads, 1)
           tma_load_2d(dst + a * p.nk * 128, &emap, full(s),
                       static_cast<int>(ntile * kPmN + a * 64), 0);
         ++issued;
-        ntile += dn;
-        mt += dm;
-        if (mt >= p.m_tiles) { mt -= p.m_tiles; ++ntile; }
         if (++s == S) { s = 0; ph ^= 1u; }
       }
-      for (long long j = (issued > S ? issued - S : 0); j < issued; ++j)
+      // every load in flight lands before the CTA exits; the end entry reused
+      // the stage of load issued - S (consumed: its empty barrier had fired),
+      // and its arrive moved that barrier one phase on, so that load is not
+      // waited for again
+      for (long long j = (issued > S ? issued - S : 0) + (ended && issued >= S ? 1 : 0); j < issued;
+           ++j)
         wait_drain(full(static_cast<int>(j % S)), static_cast<uint32_t>((j / S) & 1), p.wait_ns,
                    p.err);
     }
@@ -209,14 +258,29 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       const uint64_t a_half = static_cast<uint64_t>(kcols) * (16384 >> 4);  // hi -> lo
       const uint64_t stage = static_cast<uint64_t>(p.stage_bytes) >> 4;
       const int ksteps = p.nk / 16;
-      int mt = mt0;
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (long long j = 0; j < my_tiles; ++j) {
+      int mt_s = mt0;
+      for (long long j = 0;; ++j) {
+        if (!dyn && j >= my_tiles) break;
         const int ab = static_cast<int>(j & 1);
         if (!wait_bounded(full(s), ph, ctl, kErrWaitMma)) { ok = false; break; }
+        // (dynamic: the entry was written before the arrive that completed full(s))
+        const unsigned long long e = dyn ? ring[j & (kPmRing - 1)] : 1ull;
         if (!wait_bounded(tempty(ab), static_cast<uint32_t>((j >> 1) & 1) ^ 1u, ctl, kErrWaitMma)) { ok = false; break; }
+        if ((e & 0xFFFFFFFFull) == 0) {
+          mbar_arrive(tfull(ab));  // end: the epilogue reads the end entry
+          break;
+        }
+        int mt = mt_s;
+        if (dyn) {
+          const uint32_t tt = static_cast<uint32_t>(e) - 1u;  // 32-bit tile index (tiles < 2^31)
+          mt = p.m_tiles == 1 ? 0 : static_cast<int>(tt % static_cast<uint32_t>(p.m_tiles));
+        } else {
+          mt_s += dm;
+          if (mt_s >= p.m_tiles) mt_s -= p.m_tiles;
+        }
         tc_fence_after();
         const uint64_t bd = e_desc0 + s * stage;
         const uint64_t ad = a_desc0 + static_cast<uint64_t>(mt) * 2 * a_half;
@@ -230,8 +294,6 @@ __global__ void __launch_bounds__(kPmThreads, 1)
         }
         tc_commit(empty(s));
         tc_commit(tfull(ab));
-        mt += dm;
-        if (mt >= p.m_tiles) mt -= p.m_tiles;
         if (++s == S) { s = 0; ph ^= 1u; }
       }
       if (!ok) {
@@ -246,20 +308,26 @@ __global__ void __launch_bounds__(kPmThreads, 1)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const uint32_t stg = st_base + (warp - 2) * p.stg_bytes;
-    // TMA-store staging (store_mode 2): boxes of bc columns x 32 samples,
-    // rows of 2 bc bytes in the tensor map's swizzle -- 16-byte chunk c of
-    // row r at c ^ (r % 8) for 128-byte rows, c ^ ((r / 2) % 4) for 64-byte
-    // rows, which also spreads a store instruction's 32 rows over the banks
-    const int cw = kPmHalf / p.rep;        // columns of this warp
-    const int bc = cw < 64 ? cw : 64;      // columns of one box
-    const int cpb_log = bc == 64 ? 3 : 2;  // log2 of 16-byte chunks per box row
-    const int sw_sh = 3 - cpb_log;
-    const uint32_t box_bytes = 64u * bc;   // 32 rows x 2 bc bytes
-    long long ntile = ntile0;
-    int mt = mt0;
-    for (long long j = 0; j < my_tiles; ++j) {
+    long long ntile_s = ntile0;
+    int mt_s = mt0;
+    for (long long j = 0;; ++j) {
+      if (!dyn && j >= my_tiles) break;
       const int ab = static_cast<int>(j & 1);
       if (!wait_bounded(tfull(ab), static_cast<uint32_t>((j >> 1) & 1), ctl, kErrWaitEpilogue)) break;
+      long long ntile = ntile_s;
+      int mt = mt_s;
+      if (dyn) {
+        long long t;
+        if (!ring_tile(j, t) || t < 0) break;
+        const uint32_t tt = static_cast<uint32_t>(t);
+        ntile = p.m_tiles == 1 ? static_cast<long long>(tt)
+                               : static_cast<long long>(tt / static_cast<uint32_t>(p.m_tiles));
+        mt = static_cast<int>(tt - static_cast<uint32_t>(ntile) * static_cast<uint32_t>(p.m_tiles));
+      } else {
+        ntile_s += dn;
+        mt_s += dm;
+        if (mt_s >= p.m_tiles) { mt_s -= p.m_tiles; ++ntile_s; }
+      }
       tc_fence_after();
       // TMEM lanes 32q .. 32q+31 hold samples row0 .. row0+31 of copy g; copy
       // g's warps store columns [g, g+1) * 256 / rep of the tile, this half
@@ -267,6 +335,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       // only releases the buffer.
       const int g = (32 * q) / spr;
       const int row0 = mt * 128 + 32 * q - g * spr;
+      const int cw = kPmHalf / p.rep;
       const int col0 = g * (kPmN / p.rep) + half * cw;
       const bool live = row0 < p.B;
       const long long w0 = ntile * kPmN + (p.rep == 1 ? half * kPmHalf : col0);
@@ -274,7 +343,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
                              (p.rep == 1 ? half * kPmHalf : col0);
       if (live) {
         uint32_t ra[32], rb[32];
-        if (p.store_mode == 1) {
+        if (p.direct_store) {
           // each lane (one sample) writes 64 contiguous bytes per chunk as two
           // 32-byte stores straight from registers
           const int b = row0 + lane;
@@ -298,37 +367,6 @@ __global__ void __launch_bounds__(kPmThreads, 1)
             tmem_ld_wait(rb);
             if (ch + 2 < kPmHalf / 32) tmem_ld_32x32b_x32(taddr + (ch + 2) * 32, ra);
             emit(rb, ch + 1);
-          }
-        } else if (p.store_mode == 2) {
-          // the previous tile's stores have finished reading the staging tile
-          if (lane == 0) bulk_wait_group_read<0>();
-          __syncwarp();
-          auto stage_box = [&](const uint32_t (&r)[32], int ch) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-              o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-              o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-              o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-              const int c = ch * 4 + v;  // 16-byte chunk of this sample's cw columns
-              const int box = c >> cpb_log, cc = c & ((1 << cpb_log) - 1);
-              st_shared_v4(stg + box * box_bytes + lane * (2 * bc) +
-                               ((cc ^ ((lane >> sw_sh) & ((1 << cpb_log) - 1))) << 4),
-                           o);
-            }
-          };
-          const int nch = cw / 32;
-          tmem_ld_32x32b_x32(taddr, ra);
-#pragma unroll 1
-          for (int ch = 0; ch < nch; ch += 2) {
-            tmem_ld_wait(ra);
-            if (ch + 1 < nch) tmem_ld_32x32b_x32(taddr + (ch + 1) * 32, rb);
-            stage_box(ra, ch);
-            if (ch + 1 >= nch) break;
-            tmem_ld_wait(rb);
-            if (ch + 2 < nch) tmem_ld_32x32b_x32(taddr + (ch + 2) * 32, ra);
-            stage_box(rb, ch + 1);
           }
         } else {
           // staged: row `lane` of the 32 x (2 cw)-byte block, 16-byte chunk c
@@ -364,19 +402,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty(ab));
-      if (live && p.store_mode == 2) {
-        // publish the staged boxes to the async proxy, then one lane stores
-        // them (rows past the batch and columns past the kernel are clipped)
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          for (int box = 0; box * bc < cw; ++box)
-            if (w0 + box * bc < p.wsize)
-              tma_store_2d(&omap, stg + box * box_bytes, static_cast<int>(w0 + box * bc), row0);
-          bulk_commit_group();
-        }
-      }
-      if (live && p.store_mode == 0) {
+      if (live && !p.direct_store) {
         // 32 / cpr samples per store instruction, cpr lanes of 16 bytes each
         // covering one sample's 2 cw-byte segment (cw = 128: lanes 0..15 row
         // sr, 16..31 row sr + 1)
@@ -397,12 +423,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
         }
         __syncwarp();
       }
-      ntile += dn;
-      mt += dm;
-      if (mt >= p.m_tiles) { mt -= p.m_tiles; ++ntile; }
     }
-    // every store of this warp has completed before the CTA exits
-    if (lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();
@@ -417,7 +438,6 @@ __global__ void __launch_bounds__(kPmThreads, 1)
 struct PremixLaunch {
   PmParams p;
   CUtensorMap emap;
-  CUtensorMap omap;  // the output [B][wsize] for the TMA stores (store_mode 2)
   unsigned grid = 0;
   size_t smem = 0;
 };
@@ -427,11 +447,9 @@ template <typename EncodeFn>
 inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bfloat16* out_ws,
                        int B, int n, long long wsize, int* err, long long wait_ns, int sms,
                        EncodeFn encode, PremixLaunch* out, long long estride = 0,
-                       int store_mode = 0) {
+                       bool allow_direct = true, unsigned int* tile_ctr = nullptr) {
   // estride: elements from one expert to the next (default wsize); a larger
-  // stride mixes a contiguous slice of wsize elements of every expert.
-  // store_mode: the epilogue form asked for (PmParams::store_mode); a form
-  // whose alignment the output does not meet falls back to 0.
+  // stride mixes a contiguous slice of wsize elements of every expert
   PmParams& p = out->p;
   p = PmParams{};
   p.B = B;
@@ -443,25 +461,21 @@ inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bf
   p.tiles = n_tiles * p.m_tiles;
   p.a_bytes = 2 * p.m_tiles * pm_kcols(n) * 16384;
   p.stage_bytes = p.nk * 512;
-  const uintptr_t oaddr = reinterpret_cast<uintptr_t>(out_ws);
-  if (store_mode == 1 && wsize % 16 == 0 && (oaddr & 31u) == 0)
-    p.store_mode = 1;
-  else if (store_mode == 2 && (oaddr & 15u) == 0 && wsize < (1LL << 31))
-    p.store_mode = 2;
-  else
-    p.store_mode = 0;
+  p.direct_store =
+      (allow_direct && wsize % 16 == 0 && (reinterpret_cast<uintptr_t>(out_ws) & 31u) == 0) ? 1 : 0;
   // small batches: copies of the batch fill the 128 accumulator rows, so that
   // every epilogue warp has samples to store (each copy a share of the columns)
-  p.rep = (p.store_mode == 1 || p.m_tiles != 1) ? 1 : B <= 32 ? 4 : B <= 64 ? 2 : 1;
+  p.rep = (p.direct_store || p.m_tiles != 1) ? 1 : B <= 32 ? 4 : B <= 64 ? 2 : 1;
   p.stg_bytes = kPmStageBytes / p.rep;
-  const int staging = p.store_mode == 1 ? 0 : kPmEpiWarps * p.stg_bytes;
-  const int budget = 200 * 1024 - p.a_bytes - staging - 4 * B * n;
+  const int staging = p.direct_store ? 0 : kPmEpiWarps * p.stg_bytes;
+  const int budget = 200 * 1024 - p.a_bytes - staging - 4 * B * n - 16 - 8 * kPmRing;
   p.stages = std::min(kPmMaxStages, budget / p.stage_bytes);
-  if (p.stages < 2) return -3;
+  if (p.stages < 2 || p.tiles >= (1LL << 31)) return -3;
   p.alpha = alpha;
   p.out = out_ws;
   p.err = err;
   p.wait_ns = wait_ns;
+  p.tile_ctr = tile_ctr;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(wsize), static_cast<cuuint64_t>(n)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(estride > 0 ? estride : wsize) * 2};
   const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(p.nk)};
@@ -470,26 +484,12 @@ inline int plan_premix(const __nv_bfloat16* experts, const float* alpha, __nv_bf
              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return -2;
-  if (p.store_mode == 2) {
-    // boxes of min(128 / rep, 64) columns x 32 samples; 128-byte rows take the
-    // 128-byte swizzle, 64-byte rows (four copies of the batch) the 64-byte one
-    const int bc = std::min(kPmHalf / p.rep, 64);
-    const cuuint64_t odims[2] = {static_cast<cuuint64_t>(wsize), static_cast<cuuint64_t>(B)};
-    const cuuint64_t ostrides[1] = {static_cast<cuuint64_t>(wsize) * 2};
-    const cuuint32_t obox[2] = {static_cast<cuuint32_t>(bc), 32u};
-    if (encode(&out->omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out_ws, odims, ostrides, obox, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE,
-               bc == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return -2;
-  } else {
-    std::memset(&out->omap, 0, sizeof(out->omap));
-  }
   // at least 120 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
   out->smem = std::max<size_t>(120 * 1024, 1024 + static_cast<size_t>(p.a_bytes) +
                                                static_cast<size_t>(p.stages) * p.stage_bytes +
                                                staging + 8 * (2 * p.stages + 5) + 16 +
-                                               4 * static_cast<size_t>(B) * n);
+                                               ((4 * static_cast<size_t>(B) * n + 15) & ~15) +
+                                               8 * kPmRing);
   out->grid = static_cast<unsigned>(std::min<long long>(p.tiles, sms));
   return 0;
 }

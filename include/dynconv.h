@@ -120,7 +120,10 @@ int dynconv_route(const dynconv_desc* desc, const void* x, const float* Wr, cons
  *   workspace      device scratch of workspace_bytes bytes, or NULL/0. Only the
  *                  PREMIX variant uses it; AUTO never picks PREMIX unless the
  *                  workspace is large enough. It holds every sample's mixed
- *                  kernel; its contents need not be preserved between calls.
+ *                  kernel and, after them, the mixing GEMM's tile counter
+ *                  (zeroed on the stream by each call); its contents need not
+ *                  be preserved between calls, and two calls in flight at once
+ *                  need two workspaces.
  *                  (The counters with which the streamed mixing publishes each
  *                  K slice live in library-owned device memory, one slot per
  *                  stream, zero between launches; after a bounded wait expired
@@ -313,12 +316,10 @@ unsigned long long dynconv_launch_count(void);
  * (per-sample weight gradients as bf16 hi / lo planes, one pass for the
  * expert and attention gradients) when it applies; 0 the CUDA-core kernel.
  * key 12: the epilogue of the tensor-core mixing GEMM: 0 (default) stages
- * each warp's block in shared memory and writes it with per-lane 16-byte
- * stores (two samples' rows per instruction); 1 stores each thread's 32
- * mixed weights straight from registers (two 32-byte stores) when the kernel
- * size is a multiple of 16 and the workspace 32-byte aligned; 2 stages the
- * block as swizzled boxes and writes them with TMA tensor stores (both
- * measured slower on B200). For measurements.
+ * each tile through shared memory and writes whole rows; 1 stores each
+ * thread's 32 mixed weights straight from registers (two 32-byte stores) when
+ * the kernel size is a multiple of 16 and the workspace 32-byte aligned
+ * (measured slower on B200). For measurements.
  * key 13: the address of a device buffer of 64-bit words (0, the default:
  * off). While it is set, the routing kernel (CTA rank r of sample b at
  * [(b * ranks + r) * 8]), the pipelined depthwise kernel and the CUDA-core
@@ -337,6 +338,12 @@ unsigned long long dynconv_launch_count(void);
  * (default) as planned; 1..256 that many (capped at the layer's height)
  * when such a unit fits, else the convolution falls back to one CTA per
  * unit. For measurements.
+ * key 18: how the tensor-core mixing GEMM of a one-pass PREMIX forward hands
+ * out its tiles: from a counter in the workspace (zeroed on the stream before
+ * the launch), each CTA taking the next tile, so that CTAs whose expert tiles
+ * arrive faster take more -- 1 (default) when the expert bank is larger than
+ * half the L2, 2 always, 0 never (statically: tile c + j * grid to CTA c).
+ * Same results either way.
  * Returns DYNCONV_OK or DYNCONV_ERR_INVALID_ARG. */
 int dynconv_test_hook(int key, long long value);
 

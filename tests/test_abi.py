@@ -118,7 +118,7 @@ def test_variant_selection_per_config(lib):
         d = dc.desc_from_config(synth.CONFIGS[name])
         # every sample's mixed kernel, 256-byte aligned
         wb = (synth.CONFIGS[name].B * synth.CONFIGS[name].weight_elems * 2 + 255) // 256 * 256
-        assert dc.dynconv_workspace_size(d) == wb
+        assert dc.dynconv_workspace_size(d) == wb + 256   # + the mixing GEMM's tile counter
     # a forced variant is reported as is
     d = dc.desc_from_config(synth.CONFIGS["resnet18_3x3"], variant=dc.VARIANT_OUTSIDE)
     assert dc.dynconv_select_variant(d) == dc.VARIANT_OUTSIDE
@@ -146,15 +146,18 @@ def test_test_hook_arguments(lib):
     assert dc.dynconv_test_hook(10, 3) == dc.ERR_INVALID_ARG
     assert dc.dynconv_test_hook(10, 2) == dc.OK
     assert dc.dynconv_test_hook(10, 0) == dc.OK
-    assert dc.dynconv_test_hook(12, 3) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(12, 2) == dc.ERR_INVALID_ARG
     assert dc.dynconv_test_hook(12, -1) == dc.ERR_INVALID_ARG
-    assert dc.dynconv_test_hook(12, 2) == dc.OK
     assert dc.dynconv_test_hook(12, 1) == dc.OK
     assert dc.dynconv_test_hook(12, 0) == dc.OK
     assert dc.dynconv_test_hook(14, 257) == dc.ERR_INVALID_ARG
     assert dc.dynconv_test_hook(14, -1) == dc.ERR_INVALID_ARG
     assert dc.dynconv_test_hook(14, 7) == dc.OK
     assert dc.dynconv_test_hook(14, 0) == dc.OK
+    assert dc.dynconv_test_hook(18, 3) == dc.ERR_INVALID_ARG
+    assert dc.dynconv_test_hook(18, 2) == dc.OK
+    assert dc.dynconv_test_hook(18, 0) == dc.OK
+    assert dc.dynconv_test_hook(18, 1) == dc.OK
     assert dc.dynconv_test_hook(15, 0) == dc.ERR_INVALID_ARG   # no such key
 
 

@@ -332,16 +332,17 @@ def test_premix_transposed_mixer_full_size(name):
         dc.dynconv_test_hook(7, 0)
 
 
-@pytest.mark.parametrize("store", [0, 1, 2], ids=["lane-store", "register-store", "tma-store"])
+@pytest.mark.parametrize("tiles", [2, 0], ids=["counter", "static"])
+@pytest.mark.parametrize("store", [0, 1], ids=["lane-store", "register-store"])
 @pytest.mark.parametrize("B", [3, 40, 100, 250],
                          ids=["B3-four-copies", "B40-two-copies", "B100", "B250-ragged-row-tile"])
-def test_premix_gemm_small_batches(B, store):
+def test_premix_gemm_small_batches(B, store, tiles):
     """The tensor-core mixing GEMM (test hook 7 = 1) with each epilogue form
-    (test hook 12): the batch copied into the 128 accumulator rows (B <= 32:
-    four copies, B <= 64: two), each copy's epilogue warps storing a share of
-    the columns; a ragged second row tile (B = 250); a kernel size that is not
-    a multiple of the 256-weight tile. Against the oracle element by
-    element."""
+    (test hook 12) and tile hand-out (test hook 18): the batch copied into the
+    128 accumulator rows (B <= 32: four copies, B <= 64: two), each copy's
+    epilogue warps storing a share of the columns; a ragged second row tile
+    (B = 250); a kernel size that is not a multiple of the 256-weight tile.
+    Against the oracle element by element."""
     cfg = synth.LayerConfig(f"premix_b{B}", synth.BF16, B, 24, 40, 7, 9, 3, 3, 1, 1, 1, 12,
                             synth.SOFTMAX, 2.0)
     inp = synth.make_inputs(cfg, seed=11, structured=1.0)
@@ -353,15 +354,42 @@ def test_premix_gemm_small_batches(B, store):
     try:
         assert dc.dynconv_test_hook(7, 1) == dc.OK
         assert dc.dynconv_test_hook(12, store) == dc.OK
+        assert dc.dynconv_test_hook(18, tiles) == dc.OK
         L.y.fill_(float("nan"))
         L.forward(dc.VARIANT_PREMIX, workspace=ws)
         assert dc.dynconv_device_status(None) == dc.OK
     finally:
         dc.dynconv_test_hook(7, 0)
         dc.dynconv_test_hook(12, 0)
+        dc.dynconv_test_hook(18, 1)
     ref = oracle.forward(inp.x_f64, inp.experts_f64, a32, inp.bias, stride=1, pad=1)
     r = compare(from_device(L.y), ref, synth.BF16)
-    assert r["ok"], (B, store, r)
+    assert r["ok"], (B, store, tiles, r)
+
+
+@pytest.mark.parametrize("name", ["deep_3x3_tau30", "large_n64"])
+def test_premix_gemm_tile_order_identical(name):
+    """The mixing GEMM with its tiles handed out by the workspace counter (test
+    hook 18 = 2) and statically (18 = 0) at full size: each tile's arithmetic
+    does not depend on which CTA takes it, so the outputs are bit-identical;
+    twice in a row with the counter (it is re-zeroed per call)."""
+    inp = layer_inputs(name)
+    L = Layer(inp)
+    L.route()
+    ws = torch.empty(dc.dynconv_workspace_size(L.desc(dc.VARIANT_PREMIX)), dtype=torch.uint8,
+                     device="cuda")
+    try:
+        assert dc.dynconv_test_hook(18, 0) == dc.OK
+        L.forward(dc.VARIANT_PREMIX, workspace=ws)
+        ref = L.y.clone()
+        assert dc.dynconv_test_hook(18, 2) == dc.OK
+        for _ in range(2):
+            L.y.fill_(float("nan"))
+            L.forward(dc.VARIANT_PREMIX, workspace=ws)
+            assert dc.dynconv_device_status(None) == dc.OK
+            assert torch.equal(L.y, ref)
+    finally:
+        dc.dynconv_test_hook(18, 1)
 
 
 def test_premix_cuda_core_mixer_refuses_many_experts():
