@@ -252,6 +252,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
   grid_dependency_wait();
+  // the next kernel on the stream (a routing kernel of the next layer) may
+  // be scheduled while this one runs: it waits for this grid's completion
+  // before it reads anything this grid writes
+  grid_launch_dependents();
   if (threadIdx.x == 32) {
     tc_stamp(p, 1);  // past the grid wait
     for (int cc = 0; cc < (p.x_early ? 0 : pre_b); ++cc) {
@@ -734,6 +738,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
   grid_dependency_wait();
+  // the next kernel on the stream (a routing kernel of the next layer) may
+  // be scheduled while this one runs: it waits for this grid's completion
+  // before it reads anything this grid writes
+  grid_launch_dependents();
   if (threadIdx.x == 32) tc_stamp(p, 1);  // past the grid wait
   const int taps = p.KH * p.KW;
   const uint32_t acc_cols = p.tmem_cols >> 1;

@@ -82,6 +82,10 @@ __global__ void __launch_bounds__(kDwThreads, K <= 5 ? 2 : 1)
   const WaitCtl ctl{const_cast<volatile int*>(&abort_flag), p.err, p.wait_ns};
 
   grid_dependency_wait();  // alpha (and possibly x) come from earlier kernels
+  // the next kernel on the stream (a routing kernel of the next layer) may
+  // be scheduled while this one runs: it waits for this grid's completion
+  // before it reads anything this grid writes
+  grid_launch_dependents();
   if (t == 0) {
     abort_flag = 0;
     mbar_init(bar_a, 1);
@@ -362,6 +366,10 @@ __global__ void __maxnreg__((DwpShape<K, NC>::kRegs))
   }
   __syncthreads();
   grid_dependency_wait();  // alpha (and x) come from earlier kernels
+  // the next kernel on the stream (a routing kernel of the next layer) may
+  // be scheduled while this one runs: it waits for this grid's completion
+  // before it reads anything this grid writes
+  grid_launch_dependents();
   // phase stamps (measurement hook): [0] entry after set-up, [1] slabs in,
   // [5] end, [6] SM id, [7] global timer at entry
   if (p.stamps != nullptr && t == 0) {

@@ -47,6 +47,10 @@ __global__ void __launch_bounds__(kDirectThreads) direct_conv_kernel(DirectParam
   const int wrow = taps * Cg;  // weights per output channel
 
   grid_dependency_wait();  // alpha (and possibly x) come from earlier kernels
+  // the next kernel on the stream (a routing kernel of the next layer) may
+  // be scheduled while this one runs: it waits for this grid's completion
+  // before it reads anything this grid writes
+  grid_launch_dependents();
   float* alpha_s = dsm;                     // [n]
   float* bias_s = alpha_s + p.n;            // [cob]
   float* w_s = bias_s + p.cob;              // [cob][KH][KW][Cg]
