@@ -797,9 +797,10 @@ int run_grouped(const dynconv_desc* d, const GroupPlan& gp, const DeviceState* s
         return DYNCONV_ERR_CUDA;
       }
       if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
-      e = ensure_smem(dc::premix_kernel, pl.smem);
+      const auto pk = dc::premix_kernel_for(pl.p.rep);
+      e = ensure_smem(pk, pl.smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
-      dc::premix_kernel<<<pl.grid, dc::kPmThreads, pl.smem, ax->aux>>>(pl.emap, pl.p);
+      pk<<<pl.grid, dc::kPmThreads, pl.smem, ax->aux>>>(pl.emap, pl.p);
       rc = check_launch("premix_kernel (grouped)");
     }
     if (rc) return rc;
@@ -908,9 +909,10 @@ int run_grouped_seq(const dynconv_desc* d, const GroupPlan& gp, const DeviceStat
         return DYNCONV_ERR_CUDA;
       }
       if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
-      e = ensure_smem(dc::premix_kernel, pl.smem);
+      const auto pk = dc::premix_kernel_for(pl.p.rep);
+      e = ensure_smem(pk, pl.smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
-      e = launch_pdl(dc::premix_kernel, dim3(pl.grid), dim3(dc::kPmThreads), pl.smem, stream,
+      e = launch_pdl(pk, dim3(pl.grid), dim3(dc::kPmThreads), pl.smem, stream,
                      pl.emap, pl.p);
       if (e != cudaSuccess) {
         g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -1229,13 +1231,14 @@ int run_tc(const dynconv_desc* d, int variant, const DeviceState* st, const void
   }
   if (rc != 0) return DYNCONV_ERR_UNSUPPORTED;
   {
-    cudaError_t e = ensure_smem(dc::premix_kernel, pl.smem);
+    const auto pk = dc::premix_kernel_for(pl.p.rep);
+    cudaError_t e = ensure_smem(pk, pl.smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(premix)");
     if (tile_ctr != nullptr) {
       e = cudaMemsetAsync(tile_ctr, 0, sizeof(unsigned int), stream);
       if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(premix tile counter)");
     }
-    e = launch_pdl(dc::premix_kernel, dim3(pl.grid), dim3(dc::kPmThreads), pl.smem, stream,
+    e = launch_pdl(pk, dim3(pl.grid), dim3(dc::kPmThreads), pl.smem, stream,
                    pl.emap, pl.p);
     if (e != cudaSuccess) {
       g_launches.fetch_add(1, std::memory_order_relaxed);

@@ -86,6 +86,10 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t 
   return d;
 }
 
+// REP = p.rep, a template parameter so that the epilogue's column split,
+// chunk count and store pattern are compile-time constants (the epilogue is
+// the kernel's bound when the expert bank is L2-resident).
+template <int REP>
 __global__ void __launch_bounds__(kPmThreads, 1)
     premix_kernel(const __grid_constant__ CUtensorMap emap, PmParams p) {
   extern __shared__ __align__(1024) unsigned char pm_smem_raw[];
@@ -147,8 +151,8 @@ __global__ void __launch_bounds__(kPmThreads, 1)
   for (int e = threadIdx.x; e < p.a_bytes / 16; e += kPmThreads)
     st_shared_v4(a_base + e * 16, make_uint4(0u, 0u, 0u, 0u));
   __syncthreads();
-  const int spr = 128 / p.rep;  // A rows per copy of the batch
-  for (int e = threadIdx.x; e < na * p.rep; e += kPmThreads) {
+  constexpr int spr = 128 / REP;  // A rows per copy of the batch
+  for (int e = threadIdx.x; e < na * REP; e += kPmThreads) {
     const int g = e / na, e1 = e - g * na;   // copy, (sample, expert)
     const int m = e1 / p.n, k = e1 - m * p.n;  // sample row, expert
     const int mt = m >> 7, r = (m & 127) + g * spr;
@@ -335,12 +339,12 @@ __global__ void __launch_bounds__(kPmThreads, 1)
       // only releases the buffer.
       const int g = (32 * q) / spr;
       const int row0 = mt * 128 + 32 * q - g * spr;
-      const int cw = kPmHalf / p.rep;
-      const int col0 = g * (kPmN / p.rep) + half * cw;
+      constexpr int cw = kPmHalf / REP;
+      const int col0 = g * (kPmN / REP) + half * cw;
       const bool live = row0 < p.B;
-      const long long w0 = ntile * kPmN + (p.rep == 1 ? half * kPmHalf : col0);
+      const long long w0 = ntile * kPmN + (REP == 1 ? half * kPmHalf : col0);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + ab * kPmN +
-                             (p.rep == 1 ? half * kPmHalf : col0);
+                             (REP == 1 ? half * kPmHalf : col0);
       if (live) {
         uint32_t ra[32], rb[32];
         if (p.direct_store) {
@@ -371,7 +375,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
         } else {
           // staged: row `lane` of the 32 x (2 cw)-byte block, 16-byte chunk c
           // at position c ^ (lane % (cw / 8)): 32 lanes fill the bank groups evenly
-          const int cpr = cw / 8;  // 16-byte chunks per row
+          constexpr int cpr = cw / 8;  // 16-byte chunks per row
           auto stage_chunk = [&](const uint32_t (&r)[32], int ch) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -384,7 +388,7 @@ __global__ void __launch_bounds__(kPmThreads, 1)
               st_shared_v4(stg + lane * (2 * cw) + ((c ^ (lane & (cpr - 1))) << 4), o);
             }
           };
-          const int nch = cw / 32;
+          constexpr int nch = cw / 32;
           tmem_ld_32x32b_x32(taddr, ra);
 #pragma unroll 1
           for (int ch = 0; ch < nch; ch += 2) {
@@ -406,9 +410,9 @@ __global__ void __launch_bounds__(kPmThreads, 1)
         // 32 / cpr samples per store instruction, cpr lanes of 16 bytes each
         // covering one sample's 2 cw-byte segment (cw = 128: lanes 0..15 row
         // sr, 16..31 row sr + 1)
-        const int cpr = cw / 8;
+        constexpr int cpr = cw / 8;
         const int part = lane & (cpr - 1);
-        const int rstep = 32 / cpr;
+        constexpr int rstep = 32 / cpr;
         const long long w = w0 + part * 8;
         const bool wok = w < p.wsize;
         const int nrows = min(32, p.B - row0);
@@ -432,6 +436,11 @@ __global__ void __launch_bounds__(kPmThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
+}
+
+// The kernel instantiation for a plan's copy count (PmParams::rep).
+inline void (*premix_kernel_for(int rep))(const CUtensorMap, PmParams) {
+  return rep == 4 ? premix_kernel<4> : rep == 2 ? premix_kernel<2> : premix_kernel<1>;
 }
 
 // Host-side plan of one premix launch.
