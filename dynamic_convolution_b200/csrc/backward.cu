@@ -496,7 +496,7 @@ int dynconv_route_backward(const dynconv_desc* desc, const void* x, const float*
   dc_lib::DeviceInfo di;
   rc = dc_lib::device_info(&di);
   if (rc) return rc;
-  const size_t smem_param = sizeof(float) * static_cast<size_t>(B);
+  const size_t smem_param = sizeof(float) * ((static_cast<size_t>(B) + 3) / 4 * 4 + dcb::kBwThreads);
   const size_t smem_dg = sizeof(float) * (static_cast<size_t>(n) + dcb::kBwThreads);
   if (smem_param > static_cast<size_t>(di.max_smem_optin)) return DYNCONV_ERR_UNSUPPORTED;
   // the channel sums of x go to dg first (scratch), then dg is overwritten;
@@ -516,9 +516,15 @@ int dynconv_route_backward(const dynconv_desc* desc, const void* x, const float*
     if (e != cudaSuccess) return dc_lib::cuda_error(e, "cudaFuncSetAttribute(route_bwd_param)");
   }
   const float inv_hw = 1.f / static_cast<float>(desc->H * desc->W);
-  dcb::route_bwd_param_kernel<<<dim3((C + dcb::kBwThreads - 1) / dcb::kBwThreads, n),
-                                dcb::kBwThreads, smem_param, s>>>(B, C, n, inv_hw, mode, tau,
-                                                                  alpha, dalpha, dg, dWr, dbr);
+  // the most sample slices (shorter chains) that keep the grid within one CTA per SM
+  int slices = dcb::kRbpMaxSlices;
+  while (slices > 1 &&
+         static_cast<long long>((C + dcb::kBwThreads / slices - 1) / (dcb::kBwThreads / slices)) * n >
+             sms)
+    slices >>= 1;
+  const int cpc = dcb::kBwThreads / slices;
+  dcb::route_bwd_param_kernel<<<dim3((C + cpc - 1) / cpc, n), dcb::kBwThreads, smem_param, s>>>(
+      B, C, n, slices, inv_hw, mode, tau, alpha, dalpha, dg, dWr, dbr);
   rc = dc_lib::launched("route_bwd_param_kernel");
   if (rc) return rc;
   dcb::route_bwd_dg_kernel<<<dim3((C + dcb::kBwThreads - 1) / dcb::kBwThreads, B),

@@ -481,30 +481,46 @@ __device__ __forceinline__ float dz_of(const float* a, const float* da, int n, i
 }
 
 // Router parameters: dWr[i][c] = sum_b dz[b][i] * gsum[b][c] / HW and
-// dbr[i] = sum_b dz[b][i]. Grid (ceil(C / 256), n): the CTA first takes
-// dz[b][i] for every sample into shared memory (one thread per sample).
+// dbr[i] = sum_b dz[b][i]. Grid (ceil(C / (256 / slices)), n): the CTA first
+// takes dz[b][i] for every sample into shared memory (one thread per sample);
+// then `slices` (1, 2, 4 or 8) groups of its threads each sum a contiguous
+// part of the samples for 256 / slices consecutive channels (coalesced rows
+// of gsum), and the first group adds the partial sums in group order -- a
+// fixed order, with `slices` chains per channel instead of one over the batch.
+constexpr int kRbpMaxSlices = 8;
 __global__ void __launch_bounds__(kBwThreads)
-    route_bwd_param_kernel(int B, int C, int n, float inv_hw, int mode, float tau,
+    route_bwd_param_kernel(int B, int C, int n, int slices, float inv_hw, int mode, float tau,
                            const float* __restrict__ alpha, const float* __restrict__ dalpha,
                            const float* __restrict__ gsum, float* __restrict__ dWr,
                            float* __restrict__ dbr) {
-  extern __shared__ float dz_s[];  // [B]
+  extern __shared__ float dz_s[];  // [B], then the partial sums [slices][256 / slices]
+  float* part = dz_s + ((B + 3) & ~3);
   const int i = blockIdx.y;
   for (int b = threadIdx.x; b < B; b += kBwThreads)
     dz_s[b] = dz_of(alpha + static_cast<size_t>(b) * n, dalpha + static_cast<size_t>(b) * n, n,
                     i, mode, tau);
   __syncthreads();
-  const int c = blockIdx.x * kBwThreads + threadIdx.x;
+  const int cpc = kBwThreads / slices;  // channels per CTA
+  const int lane = threadIdx.x % cpc, q = threadIdx.x / cpc;
+  const int c = blockIdx.x * cpc + lane;
+  const int per = (B + slices - 1) / slices;
+  const int b0 = q * per, b1 = min(B, b0 + per);
+  float s = 0.f;
   if (c < C) {
-    float s = 0.f;
 #pragma unroll 8
-    for (int b = 0; b < B; ++b) s = fmaf(dz_s[b], gsum[static_cast<size_t>(b) * C + c], s);
-    dWr[static_cast<size_t>(i) * C + c] = s * inv_hw;
+    for (int b = b0; b < b1; ++b) s = fmaf(dz_s[b], gsum[static_cast<size_t>(b) * C + c], s);
+  }
+  part[threadIdx.x] = s;  // = part[q * cpc + lane]
+  __syncthreads();
+  if (q == 0 && c < C) {
+    float t = 0.f;
+    for (int k = 0; k < slices; ++k) t += part[k * cpc + lane];
+    dWr[static_cast<size_t>(i) * C + c] = t * inv_hw;
   }
   if (dbr && blockIdx.x == 0 && threadIdx.x == 0) {
-    float s = 0.f;
-    for (int b = 0; b < B; ++b) s += dz_s[b];
-    dbr[i] = s;
+    float t = 0.f;
+    for (int b = 0; b < B; ++b) t += dz_s[b];
+    dbr[i] = t;
   }
 }
 
