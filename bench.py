@@ -276,10 +276,19 @@ def profile_traffic(kernel_tag: str, workload: str, src_hash: str):
     return d.get("dram_bytes_per_launch")
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and blank space: what the compiler sees
+    of it, so that an edit of a comment does not orphan the captured profiles."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(" ".join(line.split()) for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash(csrc: str | None = None) -> str:
-    """Hash of the forward translation unit's sources: dynconv.cu and every
-    csrc header it includes, directly or not (the backward and cell units
-    compile separately and cannot change the forward kernels)."""
+    """Hash of the forward translation unit's code: dynconv.cu and every csrc
+    header it includes, directly or not (the backward and cell units compile
+    separately and cannot change the forward kernels), comments and blank
+    space left out."""
     csrc = csrc or os.path.join(ROOT, "dynamic_convolution_b200", "csrc")
     seen, todo = set(), ["dynconv.cu"]
     while todo:
@@ -291,9 +300,9 @@ def kernel_source_hash(csrc: str | None = None) -> str:
             todo += re.findall(r'^#include "([^"]+)"', f.read(), flags=re.M)
     h = hashlib.sha256()
     for fn in sorted(seen):
-        with open(os.path.join(csrc, fn), "rb") as f:
+        with open(os.path.join(csrc, fn), encoding="utf-8") as f:
             h.update(fn.encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

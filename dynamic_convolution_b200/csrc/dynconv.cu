@@ -76,10 +76,10 @@ std::atomic<int> g_group_mix{0};     // PREMIX, n > 8, large B*|W|: 0 one pass, 
 std::atomic<int> g_premix_direct{0}; // premix epilogue: 1 stores from registers when aligned, 0 staged
 std::atomic<int> g_mixgrad_tc{1};    // backward: 1 tensor-core mixing gradient when it fits, 0 CUDA cores
 std::atomic<long long> g_group_bytes{40LL << 20};  // target bytes of one group's mixed kernels
-std::atomic<unsigned long long> g_conv_stamps{0};
+std::atomic<unsigned long long> g_conv_stamps{0};  // device buffer for the kernels' phase stamps
 std::atomic<int> g_persist_rows{0};  // persistent convolution: output rows per unit (0: planned)
 std::atomic<int> g_premix_dyn{1};    // mixing GEMM (one pass) tiles from a counter: 1 when the
-                                     // experts exceed half the L2, 2 always, 0 never (static)  // device buffer for the convolution's phase stamps
+                                     // experts exceed half the L2, 2 always, 0 never (static)
 std::atomic<long long> g_group_min{64LL << 20};    // below this B*|W| the one-pass form is used
 thread_local char g_last_err[256] = "";
 

@@ -23,8 +23,9 @@ def test_cpu_baseline_cells_small():
 
 
 def test_source_hash_covers_the_forward_unit_only(tmp_path):
-    """On a copy of the sources: the hash changes with a forward header and not
-    with a backward or cell source (those compile in other translation units)."""
+    """On a copy of the sources: the hash changes with the code of a forward
+    header and not with a backward or cell source (those compile in other
+    translation units), nor with a comment or blank lines anywhere."""
     src = os.path.join(bench.ROOT, "dynamic_convolution_b200", "csrc")
     dst = tmp_path / "csrc"
     shutil.copytree(src, dst)
@@ -34,8 +35,10 @@ def test_source_hash_covers_the_forward_unit_only(tmp_path):
                         ("backward_kernels.cuh", False), ("cells_kernels.cuh", False)):
         path = dst / fn
         orig = path.read_bytes()
-        path.write_bytes(orig + b"\n// probe\n")
+        path.write_bytes(orig + b"\nstatic const int hash_probe_value = 1;\n")
         assert (bench.kernel_source_hash(str(dst)) != base) == changes, fn
+        path.write_bytes(orig + b"\n// a comment\n/* and a block\n comment */\n\n")
+        assert bench.kernel_source_hash(str(dst)) == base, fn
         path.write_bytes(orig)
 
 
