@@ -244,10 +244,42 @@ int run_chansum(const dynconv_desc* d, int sms, const void* v, int P, int C, flo
   const int vec = bf ? 8 : 4;
   const bool vok = C % vec == 0 && aligned16(v);
   const size_t smem = sizeof(float) * dcb::kBwThreads * (vok ? vec : 1);
-  const int slices = scratch ? chansum_slices(d->B, P, sms) : 1;
+  int slices = scratch ? chansum_slices(d->B, P, sms) : 1;
+  // up to 8 slices: one cluster per sample adds them in shared memory (no
+  // finishing kernel, no scratch); more go through the scratch and a second pass
+  const size_t smem_cl = smem + sizeof(float) * static_cast<size_t>(C);
+  const bool cluster = slices > 1 && slices <= 16 && smem_cl <= 48 * 1024;
+  if (cluster) slices = std::min(slices, 8);
   if (slices == 1) scratch = out;  // one slice: the partial is the sum
   const int Ps = (P + slices - 1) / slices;
   const dim3 grid(slices, d->B);
+  if (cluster) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(dcb::kBwThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_cl;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = slices;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (bf)
+      e = vok ? cudaLaunchKernelEx(&cfg, dcb::chansum_kernel<__nv_bfloat16, 8, true>,
+                                   static_cast<const __nv_bfloat16*>(v), P, C, Ps, out)
+              : cudaLaunchKernelEx(&cfg, dcb::chansum_kernel<__nv_bfloat16, 1, true>,
+                                   static_cast<const __nv_bfloat16*>(v), P, C, Ps, out);
+    else
+      e = vok ? cudaLaunchKernelEx(&cfg, dcb::chansum_kernel<float, 4, true>,
+                                   static_cast<const float*>(v), P, C, Ps, out)
+              : cudaLaunchKernelEx(&cfg, dcb::chansum_kernel<float, 1, true>,
+                                   static_cast<const float*>(v), P, C, Ps, out);
+    if (e != cudaSuccess) return dc_lib::cuda_error(e, "chansum_kernel (cluster) launch");
+    return dc_lib::launched("chansum_kernel");
+  }
   if (bf) {
     if (vok)
       dcb::chansum_kernel<__nv_bfloat16, 8><<<grid, dcb::kBwThreads, smem, s>>>(

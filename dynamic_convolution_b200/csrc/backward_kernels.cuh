@@ -13,6 +13,7 @@
 // results do not depend on scheduling.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -47,10 +48,15 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // pixel lanes), four 16-byte loads in flight; the L lane sums are added in
 // lane order. chansum_finish_kernel adds the slices in order. VEC = 1 is the
 // unvectorised form (any C, any alignment).
-template <typename T, int VEC>
+// CLUSTER: the slices of a sample form one thread-block cluster (at most 8);
+// each CTA keeps its slice's sums in shared memory and, after a cluster
+// barrier, rank 0 adds the ranks' sums in rank order (the finishing pass's
+// order, so the same bits) and writes out[b][c]; no second kernel.
+template <typename T, int VEC, bool CLUSTER = false>
 __global__ void __launch_bounds__(kBwThreads) chansum_kernel(const T* __restrict__ v, int P, int C,
                                                              int Ps, float* __restrict__ part) {
-  extern __shared__ float cs_part[];  // [L][C]
+  extern __shared__ float cs_part[];  // [L][C], then (CLUSTER) this slice's sums [C]
+  float* mine = cs_part + kBwThreads * VEC;
   const int b = blockIdx.y, slice = blockIdx.x;
   const int nslices = gridDim.x;
   const int p_begin = slice * Ps, p_end = min(P, p_begin + Ps);
@@ -96,8 +102,25 @@ __global__ void __launch_bounds__(kBwThreads) chansum_kernel(const T* __restrict
     for (int e = t; e < nvec * VEC; e += kBwThreads) {
       float s = 0.f;
       for (int l = 0; l < L; ++l) s += cs_part[l * (nvec * VEC) + e];
-      part[(static_cast<size_t>(b) * nslices + slice) * C + static_cast<size_t>(v0) * VEC + e] = s;
+      if constexpr (CLUSTER)
+        mine[static_cast<size_t>(v0) * VEC + e] = s;
+      else
+        part[(static_cast<size_t>(b) * nslices + slice) * C + static_cast<size_t>(v0) * VEC + e] = s;
     }
+    if constexpr (CLUSTER) __syncthreads();  // cs_part is reused by the next chunk
+  }
+  if constexpr (CLUSTER) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();  // every slice's sums are in its shared memory
+    if (cluster.block_rank() == 0) {
+      for (int c = threadIdx.x; c < C; c += kBwThreads) {
+        float s = 0.f;
+        for (int r = 0; r < nslices; ++r) s += cluster.map_shared_rank(mine, r)[c];
+        part[static_cast<size_t>(b) * C + c] = s;
+      }
+    }
+    cluster.sync();  // no CTA leaves while rank 0 reads its shared memory
   }
 }
 
